@@ -1,0 +1,531 @@
+#!/usr/bin/env python
+"""Benchmark of the MoLE lookup path on B200.
+
+Workload (default): the 1B-activated-shaped MoLE model -- 16 layers, each with
+its own table LUT[50304, 16, 2048] bf16 (3.3 GB) and router Wr[2048, 16] --
+over a prefill batch of T = 16384 tokens with Zipf(1.1) ids.  One step is one
+pass of the lookup path of a forward pass: mole_lookup_combine for each of the
+16 layers (router GEMV + softmax + direct-addressed gather + gate-weighted
+sum), every layer with its own hidden states.  Tables are seeded N(0, 0.02)
+fills (the combine's time does not depend on the values); ids and hidden
+states are fresh per step.  A step touches 16 distinct tables of 3.3 GB, so
+inputs are far larger than the 126 MB L2.
+
+Also measured in the same run (own keys in the JSON line): the one-off table
+build (410M-shaped layer, tensor cores), the NF3-compressed table combine, and
+the other prefill cases of the 1B-shaped layer.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank runs its own batch on its own GPU (weak scaling, no
+data-path collective); rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from mixture_lookup_experts_b200 import inputs  # noqa: E402
+
+METRIC = "MoLE lookup-combine tokens/s & HBM GB/s vs 8 TB/s; LUT build TFLOP/s"
+UNIT = "tokens/s"
+KERNEL_SOURCES = ["mixture_lookup_experts_b200/csrc/combine.cu", "mixture_lookup_experts_b200/csrc/common.cuh"]
+PROFILE_SUMMARY = "profiles/combine_bf16_1b_T16384_zipf.md"
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--tokens", type=int, default=16384)
+    ap.add_argument("--ids", choices=["zipf", "uniform"], default="zipf")
+    ap.add_argument("--no-extras", action="store_true", help="skip the build / NF3 / other-case legs")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def workload_config(T: int, kind: str) -> dict:
+    s = inputs.SHAPES["1b"]
+    return {
+        "workload": f"1B-activated-shaped MoLE lookup path, {s.layers} layers x mole_lookup_combine, "
+                    f"prefill T={T}, {'Zipf(1.1)' if kind == 'zipf' else 'uniform'} ids",
+        "V": s.V, "D": s.D, "N": s.N, "layers": s.layers, "tokens_per_step": T, "ids": kind,
+        "table_dtype": "bf16", "accumulate": "f32", "out_dtype": "f32",
+        "l2": "inputs larger than L2: each step reads 16 distinct 3.3 GB layer tables",
+        "data": "synthetic seeded N(0,0.02) tables; fresh ids and hidden states per step",
+    }
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML, polled from a thread)
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int):
+        self.ok = False
+        self.samples, self.reasons = [], 0
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            # NVML may see more GPUs than CUDA does: find ours by PCI address
+            pr = torch.cuda.get_device_properties(device_index)
+            bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self._stop = threading.Event()
+
+    def _poll(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._poll, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        names = [n for b, n in self.REASONS.items() if self.reasons & b and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), d.get("bf16_tflops_sustained"), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, rel), "rb").read())
+    return h.hexdigest()
+
+
+def profiled_traffic():
+    """(bytes per launch, note) from the committed ncu summary if it was taken
+    on the current kernel source; else (None, reason)."""
+    p = os.path.join(ROOT, PROFILE_SUMMARY)
+    if not os.path.exists(p):
+        return None, "no ncu summary committed"
+    fields = {}
+    for line in open(p):
+        if ":" in line and line.strip().startswith(("traffic_bytes_per_launch", "kernel_source_sha256")):
+            k, v = line.split(":", 1)
+            fields[k.strip()] = v.strip().strip("`")
+    if fields.get("kernel_source_sha256") != kernel_source_hash():
+        return None, "kernel changed since the ncu capture"
+    try:
+        return float(fields["traffic_bytes_per_launch"]), "ncu dram__bytes_read.sum + dram__bytes_write.sum"
+    except (KeyError, ValueError):
+        return None, "summary lacks traffic"
+
+
+def combine_bytes(U: float, T: int, D: int, N: int) -> float:
+    """Algorithmic bytes of one combine launch: unique table rows + h in +
+    out (fp32) + router weights + ids."""
+    return U * N * D * 2 + T * D * 2 + T * D * 4 + D * N * 2 + 4 * T
+
+
+def nf3_bytes(U: float, T: int, D: int, N: int) -> float:
+    return U * N * D * (3 / 8 + 2 / 64) + T * D * 2 + T * D * 4 + D * N * 2 + 4 * T
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the CPU oracle, as it stands, on a bounded sample
+# ---------------------------------------------------------------------------
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    shape = inputs.SHAPES["1b"]
+    V, D, N, L = shape.V, shape.D, shape.N, shape.layers
+    sample_T = 256  # tokens per layer per step (bounded sample of the T-token batch)
+    rng = np.random.default_rng(shape.seed)
+    cores = oracle.max_threads()
+
+    def one_step(seed):
+        r = np.random.default_rng(seed)
+        t0 = time.perf_counter()
+        done = 0
+        for layer in range(L):
+            ids = inputs.draw_ids(r, sample_T, V, args.ids)
+            uniq, inv = np.unique(ids, return_inverse=True)
+            rows = inputs.normal(r, (uniq.size, N, D), 0.02, "bf16")  # the rows this sample reads
+            Wr = inputs.normal(r, (D, N), 0.02, "bf16")
+            h = inputs.normal(r, (sample_T, D), 1.0, "bf16")
+            gen = time.perf_counter()
+            oracle.combine(inv.astype(np.int32), h, Wr, rows)
+            done += time.perf_counter() - gen
+        return done
+
+    for i in range(args.warmup):
+        one_step(1000 + i)
+    times = [one_step(2000 + i) for i in range(args.steps)]
+    total = sum(times)
+    value = sample_T * args.steps / total  # tokens through all 16 layers per second
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(args.tokens, args.ids),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{sample_T} tokens per layer x {L} layers per step (input generation "
+                                   f"excluded), fp64 C oracle with OpenMP over tokens"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    from mixture_lookup_experts_b200 import mole
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=torch.device("cuda", local_rank))
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream()
+
+    shape = inputs.SHAPES["1b"]
+    V, D, N, L = shape.V, shape.D, shape.N, shape.layers
+    T = args.tokens
+    W, K = args.warmup, args.steps
+
+    # ---- layer tables and routers (seeded per rank) ----
+    g = torch.Generator(device=dev)
+    g.manual_seed(shape.seed + 7919 * rank)
+    luts = [(torch.randn((V, N, D), generator=g, device=dev) * 0.02).to(torch.bfloat16) for _ in range(L)]
+    routers = [(torch.randn((D, N), generator=g, device=dev) * 0.02).to(torch.bfloat16) for _ in range(L)]
+    # per-step batches: a pool of P distinct (ids, h) per layer slot, rotated
+    P = 4
+    rng = np.random.default_rng(shape.seed + 104729 * rank)
+    id_pool = [[torch.from_numpy(inputs.draw_ids(rng, T, V, args.ids)).to(dev) for _ in range(L)] for _ in range(P)]
+    h_pool = [[(torch.randn((T, D), generator=g, device=dev)).to(torch.bfloat16) for _ in range(L)]
+              for _ in range(P)]
+    uniq_counts = [[int(torch.unique(x).numel()) for x in pool] for pool in id_pool]
+    out = torch.empty((T, D), dtype=torch.float32, device=dev)
+
+    def step(i, events=None):
+        p = i % P
+        for layer in range(L):
+            if events is not None:
+                events[layer][0].record(stream)
+            mole.mole_lookup_combine(id_pool[p][layer], h_pool[p][layer], routers[layer], luts[layer], out=out,
+                                     stream=stream)
+            if events is not None:
+                events[layer][1].record(stream)
+
+    # ---- warm-up ----
+    for i in range(W):
+        step(i)
+    st = mole.mole_check(stream, timeout_ms=60000)
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+
+    # ---- timed region: K steps, barrier + synchronize on both sides ----
+    kern_events = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+                    for _ in range(L)] for _ in range(K)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clocks:
+        t_start.record(stream)
+        for i in range(K):
+            step(W + i, kern_events[i])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    st = mole.mole_check(stream, timeout_ms=60000)
+    if st != 0:
+        raise RuntimeError(f"device status {st} in the timed region")
+    kern_ms = [kern_events[i][l][0].elapsed_time(kern_events[i][l][1]) for i in range(K) for l in range(L)]
+    avg_kern_ms = sum(kern_ms) / len(kern_ms)
+    U_avg = sum(uniq_counts[(W + i) % P][l] for i in range(K) for l in range(L)) / (K * L)
+
+    t = torch.tensor([elapsed_ms, avg_kern_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms, max_kern_ms = float(t[0]), float(t[1])
+    value = world * T * K / (max_ms / 1e3)
+
+    # ---- end to end through the C ABI with host buffers ----
+    h_host = [torch.empty((T, D), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    ids_host = torch.empty((L, T), dtype=torch.int32).pin_memory()
+    out_host = torch.empty((T, D), dtype=torch.float32).pin_memory()
+    for s in range(2):
+        h_host[s].copy_(h_pool[0][s])
+    ids_host.copy_(torch.stack(id_pool[0]).cpu())
+    h_stage = torch.empty((T, D), dtype=torch.bfloat16, device=dev)
+    ids_stage = torch.empty((L, T), dtype=torch.int32, device=dev)
+
+    def e2e_step():
+        ids_stage.copy_(ids_host, non_blocking=True)
+        for layer in range(L):
+            h_stage.copy_(h_host[layer % 2], non_blocking=True)
+            mole.mole_lookup_combine(ids_stage[layer], h_stage, routers[layer], luts[layer], out=out, stream=stream)
+            out_host.copy_(out, non_blocking=True)
+
+    for _ in range(min(W, 3)):
+        e2e_step()
+    torch.cuda.synchronize()
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    K_e2e = max(1, min(K, 20))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e_start.record(stream)
+    for _ in range(K_e2e):
+        e2e_step()
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    e_ms = torch.tensor([e_start.elapsed_time(e_end)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+    e2e_value = world * T * K_e2e / (float(e_ms[0]) / 1e3)
+    h2d = L * T * D * 2 + L * T * 4
+    d2h = L * T * D * 4
+    del h_host, out_host, h_stage
+
+    # ---- roofline of the combine kernel ----
+    hbm_peak, bf16_peak, bf16_sust, peak_kind = measured_peaks()
+    alg_bytes = combine_bytes(U_avg, T, D, N)
+    achieved_gbs = alg_bytes / (max_kern_ms / 1e3) / 1e9
+    traffic, traffic_note = profiled_traffic()
+    roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved_gbs / hbm_peak, "traffic": traffic,
+                "kernel": "combine_kernel<bf16 router, 16 experts, bf16 table>",
+                "algorithmic_bytes_per_launch": alg_bytes, "unique_rows_per_launch": U_avg,
+                "avg_launch_us": max_kern_ms * 1e3, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
+                "frac_of_8TBs": achieved_gbs / 8000.0, "traffic_source": traffic_note}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": max_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic", "config": workload_config(T, args.ids),
+        "layer_tokens_per_s": value * L, "hbm_gbs": achieved_gbs,
+        "roofline": roofline,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": K_e2e, "note": "per step: ids + 16 hidden-state batches H2D from pinned memory, "
+                                        "16 combine calls through the C ABI, 16 outputs D2H"},
+        "gpu_launches": K * L,
+        "clocks": clocks.summary(),
+    }
+
+    # ---- extras: other prefill cases, NF3 table, table build ----
+    if not args.no_extras:
+        line["cases"] = other_cases(mole, luts, routers, rng, g, dev, stream, W, T, args.ids)
+        line["nf3"] = nf3_leg(mole, luts, routers, id_pool, h_pool, uniq_counts, dev, stream, W, K, T, P)
+        del luts
+        torch.cuda.empty_cache()
+        line["build"] = build_leg(mole, dev, stream, bf16_peak, bf16_sust, peak_kind)
+
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def time_launches(fn, n, stream):
+    import torch
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for i in range(n):
+        ev[i][0].record(stream)
+        fn(i)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def other_cases(mole, luts, routers, rng, g, dev, stream, W, T_main, kind_main):
+    import torch
+    shape = inputs.SHAPES["1b"]
+    V, D, N, L = shape.V, shape.D, shape.N, shape.layers
+    hbm_peak = measured_peaks()[0]
+    res = {}
+    for T in (4096, 16384):
+        for kind in ("zipf", "uniform"):
+            if T == T_main and kind == kind_main:
+                continue
+            ids = [torch.from_numpy(inputs.draw_ids(rng, T, V, kind)).to(dev) for _ in range(L)]
+            hs = [torch.randn((T, D), generator=g, device=dev).to(torch.bfloat16) for _ in range(L)]
+            U = sum(int(torch.unique(x).numel()) for x in ids) / L
+            out = torch.empty((T, D), dtype=torch.float32, device=dev)
+
+            def fn(i):
+                lay = i % L
+                mole.mole_lookup_combine(ids[lay], hs[lay], routers[lay], luts[lay], out=out, stream=stream)
+
+            for i in range(max(W, 3) * L):
+                fn(i)
+            ms = time_launches(fn, 4 * L, stream)
+            avg = sum(ms) / len(ms)
+            b = combine_bytes(U, T, D, N)
+            res[f"T{T}_{kind}"] = {"tokens_per_s_per_layer": T / (avg / 1e3), "avg_launch_us": avg * 1e3,
+                                   "unique_rows": U, "achieved_gbs": b / (avg / 1e3) / 1e9,
+                                   "frac_of_measured_hbm": b / (avg / 1e3) / 1e9 / hbm_peak}
+            del ids, hs, out
+    return res
+
+
+def nf3_leg(mole, luts, routers, id_pool, h_pool, uniq_counts, dev, stream, W, K, T, P):
+    import torch
+    shape = inputs.SHAPES["1b_nf3"]
+    D, N, L = shape.D, shape.N, shape.layers
+    hbm_peak = measured_peaks()[0]
+    tables = []
+    q_ms = []
+    for lay in range(L):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        tables.append(mole.mole_quantize_lut_nf3(luts[lay], stream=stream))
+        e1.record(stream)
+        q_ms.append((e0, e1))
+    torch.cuda.synchronize()
+    q_avg = sum(a.elapsed_time(b) for a, b in q_ms) / L
+    out = torch.empty((T, D), dtype=torch.float32, device=dev)
+
+    def fn(i):
+        p, lay = (i // L) % P, i % L
+        c, s = tables[lay]
+        mole.mole_lookup_combine_nf3(id_pool[p][lay], h_pool[p][lay], routers[lay], c, s, out=out, stream=stream)
+
+    for i in range(W * L):
+        fn(i)
+    n = max(1, min(K, 20)) * L
+    ms = time_launches(fn, n, stream)
+    avg = sum(ms) / len(ms)
+    U = sum(uniq_counts[(i // L) % P][i % L] for i in range(n)) / n
+    b = nf3_bytes(U, T, D, N)
+    assert mole.mole_check(stream) == 0
+    V = shape.V
+    q_bytes = V * N * D * 2 + V * N * D * 3 / 8 + V * N * (D // 64) * 2
+    del tables
+    return {"tokens_per_s": T / (avg / 1e3) / L, "tokens_per_s_per_layer": T / (avg / 1e3),
+            "avg_launch_us": avg * 1e3, "achieved_gbs": b / (avg / 1e3) / 1e9,
+            "frac_of_measured_hbm": b / (avg / 1e3) / 1e9 / hbm_peak, "algorithmic_bytes_per_launch": b,
+            "quantize_ms_per_layer": q_avg, "quantize_gbs": q_bytes / (q_avg / 1e3) / 1e9,
+            "workload": f"1B-shaped NF3 table (codes + fp16 scale per 64), T={T}, same ids/h as the main case"}
+
+
+def build_leg(mole, dev, stream, bf16_peak, bf16_sust, peak_kind):
+    import torch
+    shape = inputs.SHAPES["410m"]
+    V, D, N, Dr = shape.V, shape.D, shape.N, shape.Dr
+    g = torch.Generator(device=dev)
+    g.manual_seed(shape.seed)
+    E = (torch.randn((V, D), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+    W1 = (torch.randn((N, D, Dr), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+    W2 = (torch.randn((N, Dr, D), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+    lut = torch.empty((V, N, D), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(mole.mole_build_lut_workspace(V, D, N, Dr, torch.bfloat16, 0), dtype=torch.uint8, device=dev)
+    mole.mole_build_lut(E, W1, W2, lut=lut, workspace=ws, stream=stream)
+    ms = time_launches(lambda i: mole.mole_build_lut(E, W1, W2, lut=lut, workspace=ws, stream=stream), 3, stream)
+    assert mole.mole_check(stream) == 0
+    best = min(ms)
+    flops = 4.0 * V * D * Dr * N
+    tf = flops / (best / 1e3) / 1e12
+    return {"workload": f"410M-shaped table build V={V} D={D} N={N} Dr={Dr} GELU (2 tcgen05 GEMMs per expert group)",
+            "tflops": tf, "ms": best, "flops": flops, "frac_of_bf16_peak": tf / bf16_peak,
+            "peak": bf16_peak, "peak_source": f"{peak_kind} burst bf16 (MEASURED_PEAKS.json)",
+            "frac_of_sustained": (tf / bf16_sust) if bf16_sust else None, "frac_of_2250": tf / 2250.0}
+
+
+def cpu_baseline(args):
+    """The oracle, as it stands, on a bounded sample of the workload."""
+    import oracle
+    oracle.build()
+    shape = inputs.SHAPES["1b"]
+    V, D, N, L = shape.V, shape.D, shape.N, shape.layers
+    r = np.random.default_rng(99)
+    sample_T = 1024
+    ids = inputs.draw_ids(r, sample_T, V, args.ids)
+    uniq, inv = np.unique(ids, return_inverse=True)
+    rows = inputs.normal(r, (uniq.size, N, D), 0.02, "bf16")
+    Wr = inputs.normal(r, (D, N), 0.02, "bf16")
+    h = inputs.normal(r, (sample_T, D), 1.0, "bf16")
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.combine(inv.astype(np.int32), h, Wr, rows)
+        reps += 1
+        if time.perf_counter() - t0 > 10.0 or reps >= 50:
+            break
+    dt = time.perf_counter() - t0
+    per_layer = sample_T * reps / dt
+    return {"value": per_layer / L, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"{sample_T} tokens of one 1B-shaped layer x {reps} repetitions ({dt:.1f} s); "
+                      f"tokens/s through {L} layers = per-layer rate / {L}"}
+
+
+if __name__ == "__main__":
+    main()

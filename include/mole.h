@@ -1,0 +1,170 @@
+/*
+ * mole.h -- C ABI of libmole, the B200 (sm_100a) implementation of the
+ * Mixture-of-Lookup-Experts (MoLE) inference lookup path.
+ *
+ * Source page ("MoLE page"): "ICML 2025 Spotlight | 华为诺亚提出端侧大模型新架构MoLE，
+ * 内存搬运代价降低1000倍" (zejuncao.github.io, 2025-05-07).  The page states the
+ * method in prose only (its formulas and figures were lost); the readings this
+ * library takes are stated at each entry point.
+ *
+ * Conventions for every entry point:
+ *   - Tensor pointers are DEVICE pointers owned by the caller, row-major and
+ *     contiguous.  The library never frees or retains them.
+ *   - Work is enqueued asynchronously on `stream` (0 = legacy default stream).
+ *     Argument errors are detected on the host and returned synchronously;
+ *     nothing is launched then.
+ *   - Errors detected on the device (a token id outside [0, V), a wait that ran
+ *     out of time) set a per-device error word; `mole_check` reads and clears
+ *     it.  A token with a bad id gets a NaN output row.
+ *   - The library allocates no device memory of its own apart from static
+ *     per-device variables (the error word).  Scratch memory, where an entry
+ *     point needs it, is passed in by the caller.
+ *   - bf16 tensors are IEEE bfloat16 bit patterns; fp16 scales are IEEE binary16.
+ */
+#ifndef MOLE_H_
+#define MOLE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOLE_OK = 0,
+  MOLE_ERR_ARG = 1,          /* bad pointer, size or enum value */
+  MOLE_ERR_ALIGN = 2,        /* a pointer is not 16-byte aligned where required */
+  MOLE_ERR_UNSUPPORTED = 3,  /* valid but unsupported shape (see each call) */
+  MOLE_ERR_WORKSPACE = 4,    /* scratch buffer missing or too small */
+  MOLE_ERR_INDEX = 5,        /* (mole_check) a token id was outside [0, V) */
+  MOLE_ERR_CUDA = 6,         /* a CUDA runtime/driver call failed */
+  MOLE_ERR_TIMEOUT = 7,      /* (mole_check) host wait or device wait ran out */
+  MOLE_ERR_NO_DEVICE = 8     /* no sm_100 device current */
+} mole_status;
+
+typedef enum { MOLE_F32 = 0, MOLE_BF16 = 1 } mole_dtype;
+
+typedef enum {
+  MOLE_ACT_GELU_ERF = 0,   /* x * Phi(x) (default reading of "GELU FFN") */
+  MOLE_ACT_GELU_TANH = 1,  /* tanh approximation of GELU */
+  MOLE_ACT_RELU = 2,
+  MOLE_ACT_SILU = 3,
+  MOLE_ACT_IDENTITY = 4
+} mole_act;
+
+/* Human-readable name of a status code (static storage). */
+const char* mole_status_str(mole_status s);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int mole_version(void);
+
+/*
+ * ---- Reparameterisation: build the lookup table (MoLE page, 推理阶段) ----
+ *
+ * Feeds the embedding matrix to every routed expert:
+ *     LUT[v, j, :] = f_j(E[v, :]),   f_j(x) = act(x . W1[j]) . W2[j]
+ * (expert form and activation are this library's reading; the page prints no
+ * formula).  All routed experts are evaluated; the experts can be dropped
+ * afterwards.
+ *
+ *   embed : [V, D]       dt
+ *   W1    : [N, D, Dr]   dt
+ *   W2    : [N, Dr, D]   dt
+ *   lut   : [V, N, D]    dt  (output; token v's N rows are contiguous)
+ *   workspace: scratch for the expert hidden activations H = act(E . W1[j]);
+ *     at least mole_build_lut_workspace(...) bytes for one expert at a time,
+ *     more lets several experts run per launch (up to all N).  Contents on
+ *     return are unspecified.
+ * dt == MOLE_BF16: bf16 in, fp32 accumulate on the tcgen05 tensor cores, H
+ *   rounded to bf16, bf16 out.  Tensor-core path needs D % 64 == 0 and
+ *   Dr % 64 == 0 and 16-byte aligned pointers; other shapes use a CUDA-core path.
+ * dt == MOLE_F32: fp32 throughout on CUDA cores.
+ * Returns MOLE_ERR_WORKSPACE if ws_bytes is below the one-expert minimum.
+ */
+size_t mole_build_lut_workspace(int64_t V, int64_t D, int32_t N, int64_t Dr, mole_dtype dt,
+                                int32_t experts_per_launch);
+mole_status mole_build_lut(const void* embed, const void* W1, const void* W2, int64_t V,
+                           int64_t D, int32_t N, int64_t Dr, mole_act act, mole_dtype dt,
+                           void* lut, void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * ---- Lookup-combine (MoLE page, 训练阶段 + 推理阶段) ----
+ *
+ * For each token t (router on the hidden state, all N routed experts active,
+ * rows fetched by direct addressing on the token id):
+ *     z_j = sum_d h[t, d] Wr[d, j]          (fp32 accumulate)
+ *     g   = softmax(z)                        (max-subtracted, fp32)
+ *     out[t, :] = sum_j g_j LUT[ids[t], j, :]  (fp32 accumulate)
+ * Only the routed-expert mixture is produced; shared experts and the residual
+ * are the caller's.
+ *
+ *   ids : [T] int32 in [0, V)    h : [T, D] dt    Wr : [D, N] dt
+ *   lut : [V, N, D] dt           out : [T, D] fp32 (overwritten)
+ * dt == MOLE_BF16 needs D % 16 == 0, N <= 32 and 16-byte aligned h, lut, out.
+ * dt == MOLE_F32 needs D % 4 == 0, N <= 32 and 16-byte aligned h, lut, out.
+ * T == 0 is a no-op.  A token with ids[t] outside [0, V) gets a NaN row and
+ * sets the device error word (MOLE_ERR_INDEX from mole_check).
+ */
+mole_status mole_lookup_combine(const int32_t* ids, int64_t T, const void* h, const void* Wr,
+                                const void* lut, int64_t V, int32_t N, int64_t D,
+                                mole_dtype dt, float* out, cudaStream_t stream);
+
+/*
+ * ---- NF3 table compression (MoLE page, 实验结果: 3-bit table, e.g. NF3) ----
+ *
+ * Quantises a bf16 table [V, N, D] (D % 64 == 0) in blocks of 64 consecutive
+ * elements of one (v, j) row, in IEEE fp32:
+ *     s = fp16(min(max_e |x_e|, 65504))                 (ties to even)
+ *     c_e = #{k : x_e / s > mid_k}   (s > 0; correctly rounded division)
+ *     c_e = 3 (the level 0.0)        (s == 0)
+ * with the NormalFloat k=3 levels (QLoRA construction, rounded to fp16; see
+ * mole_nf3_levels) and mid_k the fp32 midpoints of adjacent levels.  Code e
+ * occupies bits [3e, 3e+3) of the block's 24-byte little-endian bit string.
+ *   codes  : [V, N, D/64, 24] uint8    scales : [V, N, D/64] fp16 bits
+ * lut_bf16 must be 16-byte aligned; codes 8-byte aligned.
+ */
+mole_status mole_quantize_lut_nf3(const void* lut_bf16, int64_t V, int32_t N, int64_t D,
+                                  uint8_t* codes, uint16_t* scales, cudaStream_t stream);
+
+/*
+ * mole_lookup_combine over an NF3 table: the row element for (id, j, d) is
+ * level[c] * s of its block (exact in fp32), dequantised in registers inside
+ * the gather.  Same arguments and error behaviour as mole_lookup_combine,
+ * with D % 64 == 0.
+ */
+mole_status mole_lookup_combine_nf3(const int32_t* ids, int64_t T, const void* h,
+                                    const void* Wr, const uint8_t* codes,
+                                    const uint16_t* scales, int64_t V, int32_t N, int64_t D,
+                                    mole_dtype dt, float* out, cudaStream_t stream);
+
+/* The 8 NF3 levels as fp16 bit patterns (ascending; index 3 is 0.0) and the 7
+ * fp32 decision midpoints.  Host-only; no device work. */
+void mole_nf3_levels(uint16_t levels_f16[8]);
+void mole_nf3_midpoints(float mid[7]);
+
+/*
+ * ---- Gather plan (the set of table rows a batch fetches; MoLE page, 复杂度分析) ----
+ *
+ * uniq[0..n_uniq) receives the distinct ids of the batch in ascending order,
+ * slot[t] the index of ids[t] in uniq.  uniq has capacity T; n_uniq is one
+ * device int32.  Needs V <= 524288 (the id set is kept on chip).  Ids outside
+ * [0, V) are skipped (slot = -1) and set the device error word.
+ */
+mole_status mole_gather_plan(const int32_t* ids, int64_t T, int64_t V, int32_t* uniq,
+                             int32_t* n_uniq, int32_t* slot, cudaStream_t stream);
+
+/*
+ * Waits (polling, at most timeout_ms; < 0 = no limit) for `stream` to drain,
+ * then reads and clears this device's error word.  Returns MOLE_OK,
+ * MOLE_ERR_INDEX (bad token id), MOLE_ERR_TIMEOUT (stream still busy, or a
+ * device-side wait gave up), or MOLE_ERR_CUDA (an asynchronous CUDA error).
+ */
+mole_status mole_check(cudaStream_t stream, int timeout_ms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOLE_H_ */

@@ -1,0 +1,119 @@
+// api.cu -- extern "C" entry points of libmole (declared in include/mole.h).
+// Validates arguments on the host, then enqueues the kernels on the caller's
+// stream.  No entry point allocates device memory.
+#include "common.cuh"
+
+namespace {
+
+bool valid_dtype(mole_dtype dt) { return dt == MOLE_F32 || dt == MOLE_BF16; }
+bool valid_act(mole_act a) { return a >= MOLE_ACT_GELU_ERF && a <= MOLE_ACT_IDENTITY; }
+size_t dtype_size(mole_dtype dt) { return dt == MOLE_BF16 ? 2 : 4; }
+
+mole_status check_device() {
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOLE_ERR_NO_DEVICE;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return MOLE_ERR_NO_DEVICE;
+  return major == 10 ? MOLE_OK : MOLE_ERR_NO_DEVICE;
+}
+
+// Shared checks of the two combine entry points.
+mole_status check_combine(const int32_t* ids, int64_t T, const void* h, const void* Wr, const void* table,
+                          int64_t V, int32_t N, int64_t D, float* out) {
+  if (T < 0 || V <= 0 || V > INT32_MAX || N <= 0 || D <= 0 || D > (1 << 20)) return MOLE_ERR_ARG;
+  if (T > 0 && (!ids || !h || !Wr || !table || !out)) return MOLE_ERR_ARG;
+  if (N > 32) return MOLE_ERR_UNSUPPORTED;
+  if (T > ((int64_t)1 << 40)) return MOLE_ERR_UNSUPPORTED;
+  if (!mole::aligned16(h) || !mole::aligned16(out)) return MOLE_ERR_ALIGN;
+  return MOLE_OK;
+}
+
+}  // namespace
+
+extern "C" size_t mole_build_lut_workspace(int64_t V, int64_t D, int32_t N, int64_t Dr, mole_dtype dt,
+                                           int32_t experts_per_launch) {
+  (void)D;
+  if (V <= 0 || N <= 0 || Dr <= 0 || !valid_dtype(dt)) return 0;
+  const int64_t e = (experts_per_launch <= 0 || experts_per_launch > N) ? N : experts_per_launch;
+  return (size_t)V * (size_t)Dr * dtype_size(dt) * (size_t)e;
+}
+
+extern "C" mole_status mole_build_lut(const void* embed, const void* W1, const void* W2, int64_t V, int64_t D,
+                                      int32_t N, int64_t Dr, mole_act act, mole_dtype dt, void* lut,
+                                      void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  if (!valid_dtype(dt) || !valid_act(act)) return MOLE_ERR_ARG;
+  if (V <= 0 || D <= 0 || N <= 0 || Dr <= 0) return MOLE_ERR_ARG;
+  if (!embed || !W1 || !W2 || !lut) return MOLE_ERR_ARG;
+  if (V > INT32_MAX || D > INT32_MAX || Dr > INT32_MAX) return MOLE_ERR_UNSUPPORTED;
+  if (!workspace || ws_bytes < mole_build_lut_workspace(V, D, N, Dr, dt, 1)) return MOLE_ERR_WORKSPACE;
+  mole_status st = check_device();
+  if (st != MOLE_OK) return st;
+  if (dt == MOLE_BF16 && mole::build_tc_supported(V, D, Dr, embed, W1, W2, lut, workspace))
+    return mole::build_tc(embed, W1, W2, V, D, N, Dr, (int)act, lut, workspace, ws_bytes, stream);
+  return mole::build_simt(embed, W1, W2, V, D, N, Dr, (int)act, dt == MOLE_BF16, lut, workspace, ws_bytes,
+                          stream);
+}
+
+extern "C" mole_status mole_lookup_combine(const int32_t* ids, int64_t T, const void* h, const void* Wr,
+                                           const void* lut, int64_t V, int32_t N, int64_t D, mole_dtype dt,
+                                           float* out, cudaStream_t stream) {
+  if (!valid_dtype(dt)) return MOLE_ERR_ARG;
+  mole_status st = check_combine(ids, T, h, Wr, lut, V, N, D, out);
+  if (st != MOLE_OK) return st;
+  if (dt == MOLE_BF16 && D % 16 != 0) return MOLE_ERR_UNSUPPORTED;
+  if (dt == MOLE_F32 && D % 4 != 0) return MOLE_ERR_UNSUPPORTED;
+  if (!mole::aligned16(lut)) return MOLE_ERR_ALIGN;
+  if (T == 0) return MOLE_OK;
+  st = check_device();
+  if (st != MOLE_OK) return st;
+  return mole::combine_dispatch(ids, T, h, Wr, lut, nullptr, V, N, (int)D, dt == MOLE_BF16,
+                                dt == MOLE_BF16 ? 0 : 1, out, stream);
+}
+
+extern "C" mole_status mole_quantize_lut_nf3(const void* lut_bf16, int64_t V, int32_t N, int64_t D,
+                                             uint8_t* codes, uint16_t* scales, cudaStream_t stream) {
+  if (!lut_bf16 || !codes || !scales || V <= 0 || N <= 0 || D <= 0) return MOLE_ERR_ARG;
+  if (D % 64 != 0) return MOLE_ERR_UNSUPPORTED;
+  if (!mole::aligned16(lut_bf16) || !mole::aligned8(codes) || (reinterpret_cast<uintptr_t>(scales) & 1u))
+    return MOLE_ERR_ALIGN;
+  mole_status st = check_device();
+  if (st != MOLE_OK) return st;
+  return mole::nf3_quantize_launch(lut_bf16, V, N, D, codes, scales, stream);
+}
+
+extern "C" mole_status mole_lookup_combine_nf3(const int32_t* ids, int64_t T, const void* h, const void* Wr,
+                                               const uint8_t* codes, const uint16_t* scales, int64_t V,
+                                               int32_t N, int64_t D, mole_dtype dt, float* out,
+                                               cudaStream_t stream) {
+  if (!valid_dtype(dt)) return MOLE_ERR_ARG;
+  mole_status st = check_combine(ids, T, h, Wr, codes, V, N, D, out);
+  if (st != MOLE_OK) return st;
+  if (T > 0 && !scales) return MOLE_ERR_ARG;
+  if (D % 64 != 0) return MOLE_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(codes) & 3u) || (reinterpret_cast<uintptr_t>(scales) & 1u))
+    return MOLE_ERR_ALIGN;
+  if (T == 0) return MOLE_OK;
+  st = check_device();
+  if (st != MOLE_OK) return st;
+  return mole::combine_dispatch(ids, T, h, Wr, codes, scales, V, N, (int)D, dt == MOLE_BF16, 2, out, stream);
+}
+
+extern "C" void mole_nf3_levels(uint16_t levels_f16[8]) {
+  float mid[7];
+  mole::nf3_tables(levels_f16, mid);
+}
+
+extern "C" void mole_nf3_midpoints(float mid[7]) {
+  uint16_t levels[8];
+  mole::nf3_tables(levels, mid);
+}
+
+extern "C" mole_status mole_gather_plan(const int32_t* ids, int64_t T, int64_t V, int32_t* uniq,
+                                        int32_t* n_uniq, int32_t* slot, cudaStream_t stream) {
+  if (T < 0 || V <= 0 || !n_uniq) return MOLE_ERR_ARG;
+  if (T > 0 && (!ids || !uniq || !slot)) return MOLE_ERR_ARG;
+  if (T > INT32_MAX) return MOLE_ERR_UNSUPPORTED;
+  mole_status st = check_device();
+  if (st != MOLE_OK) return st;
+  return mole::gather_plan_launch(ids, T, V, uniq, n_uniq, slot, stream);
+}

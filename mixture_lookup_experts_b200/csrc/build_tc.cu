@@ -1,0 +1,444 @@
+// build_tc.cu -- table build on the 5th-generation tensor cores (tcgen05 + TMEM,
+// operands staged by TMA).  MoLE page, 推理阶段: the embedding matrix is fed to
+// every routed expert, LUT[v, j, :] = act(E[v] . W1[j]) . W2[j].
+//
+// The build is two batched bf16 GEMMs per group of experts (fp32 accumulate):
+//   GEMM1  H[e]          = act(E . W1[e])   E [V, D] K-major, W1[e] [D, Dr] N-major
+//   GEMM2  LUT[:, e, :]  = H[e] . W2[e]     H[e] [V, Dr] K-major, W2[e] [Dr, D] N-major
+// H is rounded to bf16 (the operand type of the second contraction).
+//
+// Kernel: persistent, one CTA per SM, 6 warps with fixed roles
+//   warp 0      TMA producer (one lane): A box 64(K) x 128(M), B four boxes
+//               64(N) x 64(K), all 128-byte swizzled, into a 4-stage ring;
+//   warp 1      TMEM owner + MMA issuer (one lane): tcgen05.mma kind::f16,
+//               M=128 N=256 K=16, accumulators double-buffered in TMEM
+//               (2 x 256 fp32 columns = all 512), tcgen05.commit frees smem
+//               stages and signals a finished accumulator;
+//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 32 columns, activation,
+//               bf16 rounding, 16-byte stores (row stride ldc, so the second
+//               GEMM writes the strided LUT[:, e, :] directly).
+// Tiles (expert, m-block, n-block) are dealt round-robin to the CTAs with the
+// n-block fastest, so concurrently running CTAs share the A rows and the whole
+// B[e] panel through L2.
+//
+// Every wait is bounded (a few seconds of %globaltimer); a wait that runs out
+// sets the device error word, all roles leave their loops, outstanding copies
+// and MMAs are drained with bounded waits, and TMEM is released before exit.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+
+namespace mole {
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_STAGE = BM * BK * 2;  // 16 KB
+constexpr int B_BOX = BK * 64 * 2;    // 8 KB: 64 k-rows of 64 n
+constexpr int B_STAGE = BK * BN * 2;  // 32 KB
+constexpr int STAGE_BYTES = A_STAGE + B_STAGE;
+constexpr int ACC_COLS = BN;
+constexpr int TMEM_COLS = 2 * ACC_COLS;  // 512: two accumulators
+constexpr int kThreads = 192;
+constexpr int kSmemBytes = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES + 256 /*barriers*/;
+constexpr uint64_t kWaitLimitNs = 4000000000ull;
+
+// Instruction descriptor, kind::f16: D fp32, A bf16 K-major, B bf16 N-major
+// (bit 16), N/8 at bits 17-22, M/16 at bits 24-28.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
+                            ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+
+struct Params {
+  int M, N, K;            // per expert: C[M, N] = act(A[M, K] . B[K, N])
+  int a_batched;          // A has an expert coordinate (else shared by all experts)
+  int act;
+  uint16_t* C;            // bf16 output
+  int64_t ldc;            // elements between rows of C
+  int64_t c_estride;      // elements between experts of C
+  int m_blocks, n_blocks;
+  int64_t tiles;
+  unsigned* err;
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_test(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits for the phase with the given parity to complete.  Gives up (returns
+// false) when *abort is set by another role or after kWaitLimitNs, in which
+// case it sets *abort and the device error word.
+__device__ __noinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort, unsigned* err) {
+  if (mbar_test(b, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_test(b, parity)) return true;
+    if ((i & 63) == 0) {
+      if (*abort) return false;
+      if (globaltimer() - t0 > kWaitLimitNs) {
+        *abort = 1;
+        atomicOr(err, kErrTimeout);
+        return false;
+      }
+    }
+  }
+}
+
+// Bounded wait used while draining after an abort (ignores the abort flag).
+__device__ __noinline__ void mbar_drain(uint64_t* b, uint32_t parity) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_test(b, parity))
+    if (globaltimer() - t0 > kWaitLimitNs) return;
+}
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
+                                            int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
+      "[%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 layout version 1.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3fffu);
+  d |= (uint64_t)((lbo >> 4) & 0x3fffu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3fffu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void decode_tile(const Params& p, int64_t tile, int& e, int& mb, int& nb) {
+  const int64_t per_e = (int64_t)p.m_blocks * p.n_blocks;
+  e = (int)(tile / per_e);
+  const int64_t r = tile - (int64_t)e * per_e;
+  mb = (int)(r / p.n_blocks);
+  nb = (int)(r - (int64_t)mb * p.n_blocks);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                   const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_STAGE;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * B_STAGE);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    mbar_init(drain, 1);
+    *abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int kblocks = (p.K + BK - 1) / BK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      uint32_t it = 0;
+      bool ok = true;
+      for (int64_t tile = blockIdx.x; ok && tile < p.tiles; tile += gridDim.x) {
+        int e, mb, nb;
+        decode_tile(p, tile, e, mb, nb);
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const uint32_t s = it % STAGES, ph = (it / STAGES) & 1u;
+          if (!mbar_wait(&empty[s], ph ^ 1u, abort, p.err)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&full[s], STAGE_BYTES);
+          tma_load_3d(sA + s * A_STAGE, &map_a, &full[s], kb * BK, mb * BM, p.a_batched ? e : 0);
+#pragma unroll
+          for (int q = 0; q < BN / 64; ++q)
+            tma_load_3d(sB + s * B_STAGE + q * B_BOX, &map_b, &full[s], nb * BN + q * 64, kb * BK, e);
+        }
+      }
+      // Drain: the last (up to STAGES) issued loads must have landed before exit.
+      const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0u;
+      for (uint32_t i = first; i < it; ++i) mbar_drain(&full[i % STAGES], (i / STAGES) & 1u);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      uint32_t it = 0, tl = 0;
+      bool ok = true, issued = false;
+      for (int64_t tile = blockIdx.x; ok && tile < p.tiles; tile += gridDim.x, ++tl) {
+        const uint32_t acc = tl & 1u, aph = (tl >> 1) & 1u;
+        if (!mbar_wait(&tempty[acc], aph ^ 1u, abort, p.err)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const uint32_t s = it % STAGES, ph = (it / STAGES) & 1u;
+          if (!mbar_wait(&full[s], ph, abort, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + s * A_STAGE), b0 = smem_u32(sB + s * B_STAGE);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            // A: K-major, advance 16 elements (32 B) inside the swizzle atom.
+            // B: N-major, advance 16 k-rows (2 atoms of 8 rows x 128 B).
+            umma(d_tmem, sw128_desc(a0 + 32 * k, 16, 1024), sw128_desc(b0 + 2048 * k, B_BOX, 1024),
+                 (kb | k) != 0);
+          }
+          issued = true;
+          umma_commit(&empty[s]);
+        }
+        if (ok) umma_commit(&tfull[acc]);
+      }
+      if (!ok && issued) {
+        // Make sure no MMA still writes TMEM when it is released.
+        umma_commit(drain);
+        mbar_drain(drain, 0);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int quad = warp & 3;  // TMEM lanes this warp may access
+    uint32_t tl = 0;
+    for (int64_t tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++tl) {
+      const uint32_t acc = tl & 1u, aph = (tl >> 1) & 1u;
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(&tfull[acc], aph, abort, p.err);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      tc_fence_after();
+      int e, mb, nb;
+      decode_tile(p, tile, e, mb, nb);
+      const int m = mb * BM + quad * 32 + lane;
+      uint16_t* crow = p.C + (int64_t)e * p.c_estride + (int64_t)m * p.ldc;
+      for (int chunk = 0; chunk < BN / 32; ++chunk) {
+        const int col0 = nb * BN + chunk * 32;
+        if (col0 >= p.N) break;  // warp-uniform
+        uint32_t r[32];
+        tmem_ld32(tmem_base + ((uint32_t)(quad * 32) << 16) + acc * ACC_COLS + chunk * 32, r);
+        if (m < p.M) {
+          uint32_t packed[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float x0 = apply_act(p.act, __uint_as_float(r[2 * i]));
+            const float x1 = apply_act(p.act, __uint_as_float(r[2 * i + 1]));
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(x0, x1);
+            packed[i] = *reinterpret_cast<const uint32_t*>(&b2);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(crow + col0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 3-D bf16 tensor map {d0 (contiguous), d1, d2} with a box {64, box1, 1},
+// 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1_bytes,
+              uint64_t s2_bytes, uint32_t box1) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {s1_bytes, s2_bytes};
+  cuuint32_t box[3] = {64, box1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+mole_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, Params p, cudaStream_t stream) {
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
+        cudaSuccess)
+      return MOLE_ERR_CUDA;
+    attr_set = true;
+  }
+  const int n_sm = num_sms();
+  if (n_sm <= 0) return MOLE_ERR_NO_DEVICE;
+  const int64_t grid = std::min<int64_t>(p.tiles, n_sm);
+  gemm_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, stream>>>(ma, mb, p);
+  return cuda_status(cudaGetLastError());
+}
+
+}  // namespace
+
+bool build_tc_supported(int64_t V, int64_t D, int64_t Dr, const void* E, const void* W1, const void* W2,
+                        const void* lut, const void* ws) {
+  int dev = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (major != 10 || minor != 0) return false;
+  if (D % 64 != 0 || Dr % 64 != 0 || V < 1 || V > (1LL << 31) - 1) return false;
+  return aligned16(E) && aligned16(W1) && aligned16(W2) && aligned16(lut) && aligned16(ws) && encode_fn();
+}
+
+mole_status build_tc(const void* E, const void* W1, const void* W2, int64_t V, int64_t D, int N, int64_t Dr,
+                     int act, void* lut, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  const size_t per_expert = (size_t)V * Dr * 2;
+  const int group = (int)std::min<size_t>((size_t)N, ws_bytes / per_expert);
+  if (group < 1) return MOLE_ERR_WORKSPACE;
+  unsigned* err = error_word();
+  if (!err) return MOLE_ERR_CUDA;
+  const uint16_t* e16 = static_cast<const uint16_t*>(E);
+  const uint16_t* w1 = static_cast<const uint16_t*>(W1);
+  const uint16_t* w2 = static_cast<const uint16_t*>(W2);
+  uint16_t* H = static_cast<uint16_t*>(ws);
+  uint16_t* L = static_cast<uint16_t*>(lut);
+  for (int e0 = 0; e0 < N; e0 += group) {
+    const int g = std::min(group, N - e0);
+    // GEMM1: H[e] = act(E . W1[e0 + e])
+    CUtensorMap ma, mb;
+    if (!make_map(&ma, e16, D, V, 1, D * 2, V * D * 2, BM)) return MOLE_ERR_CUDA;
+    if (!make_map(&mb, w1 + (int64_t)e0 * D * Dr, Dr, D, g, Dr * 2, D * Dr * 2, BK)) return MOLE_ERR_CUDA;
+    Params p1{};
+    p1.M = (int)V;
+    p1.N = (int)Dr;
+    p1.K = (int)D;
+    p1.a_batched = 0;
+    p1.act = act;
+    p1.C = H;
+    p1.ldc = Dr;
+    p1.c_estride = V * Dr;
+    p1.m_blocks = (int)((V + BM - 1) / BM);
+    p1.n_blocks = (int)((Dr + BN - 1) / BN);
+    p1.tiles = (int64_t)g * p1.m_blocks * p1.n_blocks;
+    p1.err = err;
+    mole_status st = launch_gemm(ma, mb, p1, stream);
+    if (st != MOLE_OK) return st;
+    // GEMM2: LUT[:, e0 + e, :] = H[e] . W2[e0 + e]
+    if (!make_map(&ma, H, Dr, V, g, Dr * 2, V * Dr * 2, BM)) return MOLE_ERR_CUDA;
+    if (!make_map(&mb, w2 + (int64_t)e0 * Dr * D, D, Dr, g, D * 2, Dr * D * 2, BK)) return MOLE_ERR_CUDA;
+    Params p2{};
+    p2.M = (int)V;
+    p2.N = (int)D;
+    p2.K = (int)Dr;
+    p2.a_batched = 1;
+    p2.act = MOLE_ACT_IDENTITY;
+    p2.C = L + (int64_t)e0 * D;
+    p2.ldc = (int64_t)N * D;
+    p2.c_estride = D;
+    p2.m_blocks = (int)((V + BM - 1) / BM);
+    p2.n_blocks = (int)((D + BN - 1) / BN);
+    p2.tiles = (int64_t)g * p2.m_blocks * p2.n_blocks;
+    p2.err = err;
+    st = launch_gemm(ma, mb, p2, stream);
+    if (st != MOLE_OK) return st;
+  }
+  return MOLE_OK;
+}
+
+}  // namespace mole

@@ -1,0 +1,103 @@
+// common.cuh -- internal helpers shared by the libmole translation units.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+#include "mole.h"
+
+namespace mole {
+
+// Bits of the per-device error word (set by kernels with atomicOr).
+enum : unsigned {
+  kErrIndex = 1u,    // a token id outside [0, V)
+  kErrTimeout = 2u,  // a bounded device-side wait gave up
+};
+
+// Device address of this device's error word (resolved once per device).
+unsigned* error_word();
+
+// Number of SMs of the current device (cached per device).
+int num_sms();
+
+// Turns a launch / runtime error into a status.
+inline mole_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOLE_OK : MOLE_ERR_CUDA; }
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned8(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7u) == 0; }
+
+// ---- device helpers -------------------------------------------------------
+
+// bf16 pair packed in a 32-bit word -> the two fp32 values (exact).
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// 16-byte read-only load that does not allocate in L1 (streamed table rows).
+__device__ __forceinline__ uint4 ldg_stream(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ uint2 ldg_stream8(const void* p) {
+  uint2 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
+               : "=r"(r.x), "=r"(r.y)
+               : "l"(p));
+  return r;
+}
+
+// 16-byte store with an evict-first hint (outputs are written once).
+__device__ __forceinline__ void stg_stream(void* p, float4 v) {
+  asm volatile("st.global.cs.v4.f32 [%0], {%1,%2,%3,%4};" ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z),
+               "f"(v.w)
+               : "memory");
+}
+
+}  // namespace mole
+
+namespace mole {
+
+// Expert FFN activation (reading of the page's "GELU FFN": exact GELU x*Phi(x)).
+__device__ __forceinline__ float apply_act(int act, float x) {
+  switch (act) {
+    case MOLE_ACT_GELU_ERF: return x * normcdff(x);
+    case MOLE_ACT_GELU_TANH: {
+      const float u = 0.7978845608028654f * fmaf(0.044715f * x, x * x, x);  // sqrt(2/pi) (x + 0.044715 x^3)
+      return 0.5f * x * (1.f + tanhf(u));
+    }
+    case MOLE_ACT_RELU: return x > 0.f ? x : 0.f;
+    case MOLE_ACT_SILU: return x / (1.f + expf(-x));
+    default: return x;
+  }
+}
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(uint16_t b) { return __uint_as_float((uint32_t)b << 16); }
+
+// Build-path entry points (build_simt.cu / build_tc.cu).
+mole_status build_simt(const void* E, const void* W1, const void* W2, int64_t V, int64_t D, int N,
+                       int64_t Dr, int act, bool bf16, void* lut, void* ws, size_t ws_bytes,
+                       cudaStream_t stream);
+bool build_tc_supported(int64_t V, int64_t D, int64_t Dr, const void* E, const void* W1,
+                        const void* W2, const void* lut, const void* ws);
+mole_status build_tc(const void* E, const void* W1, const void* W2, int64_t V, int64_t D, int N,
+                     int64_t Dr, int act, void* lut, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+// Combine / NF3 / plan entry points (combine.cu / plan.cu).
+mole_status combine_dispatch(const int32_t* ids, int64_t T, const void* h, const void* Wr,
+                             const void* table, const uint16_t* scales, int64_t V, int N, int D,
+                             bool bf16_inputs, int table_kind, float* out, cudaStream_t stream);
+mole_status nf3_quantize_launch(const void* lut, int64_t V, int N, int64_t D, uint8_t* codes,
+                                uint16_t* scales, cudaStream_t stream);
+void nf3_tables(uint16_t levels[8], float mid[7]);
+mole_status gather_plan_launch(const int32_t* ids, int64_t T, int64_t V, int32_t* uniq,
+                               int32_t* n_uniq, int32_t* slot, cudaStream_t stream);
+
+}  // namespace mole

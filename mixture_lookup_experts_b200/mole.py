@@ -1,0 +1,193 @@
+"""ctypes binding of libmole (include/mole.h): same entry-point names, argument
+marshalling only.  Every step of the computation runs in the library's CUDA
+kernels; PyTorch supplies device memory and the current stream.
+
+Importing this module loads ``libmole.so`` from this package directory and
+raises ``ImportError`` if it is missing -- there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmole.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"libmole.so not found at {LIB_PATH}; build it with "
+        "`python -m mixture_lookup_experts_b200._build` (nvcc, sm_100a)")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+MOLE_OK = 0
+STATUS = {0: "MOLE_OK", 1: "MOLE_ERR_ARG", 2: "MOLE_ERR_ALIGN", 3: "MOLE_ERR_UNSUPPORTED",
+          4: "MOLE_ERR_WORKSPACE", 5: "MOLE_ERR_INDEX", 6: "MOLE_ERR_CUDA", 7: "MOLE_ERR_TIMEOUT",
+          8: "MOLE_ERR_NO_DEVICE"}
+F32, BF16 = 0, 1
+ACT = {"gelu": 0, "gelu_erf": 0, "gelu_tanh": 1, "relu": 2, "silu": 3, "identity": 4}
+
+# Every function include/mole.h declares, with its ctypes signature.
+_P, _I64, _I32, _I, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int, ctypes.c_size_t
+SIGNATURES = {
+    "mole_status_str": ([_I], ctypes.c_char_p),
+    "mole_version": ([], _I),
+    "mole_build_lut_workspace": ([_I64, _I64, _I32, _I64, _I, _I32], _SZ),
+    "mole_build_lut": ([_P, _P, _P, _I64, _I64, _I32, _I64, _I, _I, _P, _P, _SZ, _P], _I),
+    "mole_lookup_combine": ([_P, _I64, _P, _P, _P, _I64, _I32, _I64, _I, _P, _P], _I),
+    "mole_quantize_lut_nf3": ([_P, _I64, _I32, _I64, _P, _P, _P], _I),
+    "mole_lookup_combine_nf3": ([_P, _I64, _P, _P, _P, _P, _I64, _I32, _I64, _I, _P, _P], _I),
+    "mole_nf3_levels": ([_P], None),
+    "mole_nf3_midpoints": ([_P], None),
+    "mole_gather_plan": ([_P, _I64, _I64, _P, _P, _P, _P], _I),
+    "mole_check": ([_P, _I], _I),
+}
+for _name, (_args, _res) in SIGNATURES.items():
+    _fn = getattr(lib, _name)
+    _fn.argtypes = _args
+    _fn.restype = _res
+
+
+class MoleError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)} "
+                         f"({lib.mole_status_str(status).decode()})")
+
+
+def _ok(status: int, where: str) -> None:
+    if status != MOLE_OK:
+        raise MoleError(status, where)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _contig(*ts):
+    for t in ts:
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def mole_version() -> int:
+    return lib.mole_version()
+
+
+def mole_status_str(status: int) -> str:
+    return lib.mole_status_str(status).decode()
+
+
+def mole_build_lut_workspace(V: int, D: int, N: int, Dr: int, dtype=torch.bfloat16,
+                             experts_per_launch: int = 0) -> int:
+    dt = BF16 if dtype == torch.bfloat16 else F32
+    return int(lib.mole_build_lut_workspace(V, D, N, Dr, dt, experts_per_launch))
+
+
+def mole_build_lut(embed: torch.Tensor, W1: torch.Tensor, W2: torch.Tensor, act: str = "gelu",
+                   lut: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                   stream=None) -> torch.Tensor:
+    """LUT[v, j, :] = act(E[v] . W1[j]) . W2[j] on the device (see mole.h)."""
+    _contig(embed, W1, W2, lut, workspace)
+    V, D = embed.shape
+    N, D2, Dr = W1.shape
+    if D2 != D or tuple(W2.shape) != (N, Dr, D):
+        raise ValueError("shape mismatch: embed [V,D], W1 [N,D,Dr], W2 [N,Dr,D]")
+    dt = _dt(embed)
+    if lut is None:
+        lut = torch.empty((V, N, D), dtype=embed.dtype, device=embed.device)
+    if workspace is None:
+        nbytes = mole_build_lut_workspace(V, D, N, Dr, embed.dtype, 0)
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=embed.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _ok(lib.mole_build_lut(_ptr(embed), _ptr(W1), _ptr(W2), V, D, N, Dr, ACT[act], dt, _ptr(lut),
+                           _ptr(workspace), ws_bytes, _stream(stream)), "mole_build_lut")
+    return lut
+
+
+def mole_lookup_combine(ids: torch.Tensor, h: torch.Tensor, Wr: torch.Tensor, lut: torch.Tensor,
+                        out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """out[t] = sum_j softmax(h[t] . Wr)_j LUT[ids[t], j] (fp32 out; see mole.h)."""
+    _contig(ids, h, Wr, lut, out)
+    V, N, D = lut.shape
+    T = ids.numel()
+    if out is None:
+        out = torch.empty((T, D), dtype=torch.float32, device=h.device)
+    _ok(lib.mole_lookup_combine(_ptr(ids), T, _ptr(h), _ptr(Wr), _ptr(lut), V, N, D, _dt(h), _ptr(out),
+                                _stream(stream)), "mole_lookup_combine")
+    return out
+
+
+def mole_quantize_lut_nf3(lut: torch.Tensor, codes: torch.Tensor | None = None,
+                          scales: torch.Tensor | None = None, stream=None):
+    """NF3 codes [V, N, D/64, 24] uint8 and fp16 scales [V, N, D/64] (see mole.h)."""
+    _contig(lut, codes, scales)
+    V, N, D = lut.shape
+    if codes is None:
+        codes = torch.empty((V, N, D // 64, 24), dtype=torch.uint8, device=lut.device)
+    if scales is None:
+        scales = torch.empty((V, N, D // 64), dtype=torch.float16, device=lut.device)
+    _ok(lib.mole_quantize_lut_nf3(_ptr(lut), V, N, D, _ptr(codes), _ptr(scales), _stream(stream)),
+        "mole_quantize_lut_nf3")
+    return codes, scales
+
+
+def mole_lookup_combine_nf3(ids: torch.Tensor, h: torch.Tensor, Wr: torch.Tensor, codes: torch.Tensor,
+                            scales: torch.Tensor, out: torch.Tensor | None = None, stream=None):
+    _contig(ids, h, Wr, codes, scales, out)
+    V, N, nb, _ = codes.shape
+    D = nb * 64
+    T = ids.numel()
+    if out is None:
+        out = torch.empty((T, D), dtype=torch.float32, device=h.device)
+    _ok(lib.mole_lookup_combine_nf3(_ptr(ids), T, _ptr(h), _ptr(Wr), _ptr(codes), _ptr(scales), V, N, D,
+                                    _dt(h), _ptr(out), _stream(stream)), "mole_lookup_combine_nf3")
+    return out
+
+
+def mole_nf3_levels():
+    buf = (ctypes.c_uint16 * 8)()
+    lib.mole_nf3_levels(ctypes.cast(buf, ctypes.c_void_p))
+    return list(buf)
+
+
+def mole_nf3_midpoints():
+    buf = (ctypes.c_float * 7)()
+    lib.mole_nf3_midpoints(ctypes.cast(buf, ctypes.c_void_p))
+    return list(buf)
+
+
+def mole_gather_plan(ids: torch.Tensor, V: int, stream=None):
+    """(uniq[:n], slot) of a batch's ids (see mole.h).  Synchronises to read n."""
+    _contig(ids)
+    T = ids.numel()
+    uniq = torch.empty(max(T, 1), dtype=torch.int32, device=ids.device)
+    slot = torch.empty(max(T, 1), dtype=torch.int32, device=ids.device)
+    n = torch.zeros(1, dtype=torch.int32, device=ids.device)
+    _ok(lib.mole_gather_plan(_ptr(ids), T, V, _ptr(uniq), _ptr(n), _ptr(slot), _stream(stream)),
+        "mole_gather_plan")
+    k = int(n.item())
+    return uniq[:k], slot[:T]
+
+
+def mole_check(stream=None, timeout_ms: int = 10000) -> int:
+    """Drain the stream (bounded) and return the device error status (0 = ok)."""
+    return int(lib.mole_check(_stream(stream), timeout_ms))

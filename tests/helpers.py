@@ -1,0 +1,67 @@
+"""Shared test helpers: host/device marshalling and the tolerance metrics."""
+import numpy as np
+import torch
+
+from mixture_lookup_experts_b200 import inputs
+
+# Combine tolerance: per token, ||out_gpu - out_ref||_2 / ||out_ref||_2 <= 1e-5
+# (fp32 accumulation over bf16 table values).
+COMBINE_RTOL = 1e-5
+# Table build tolerance: 2 bf16 ulps of the fp64 reference, the ulp taken at
+# max(|ref|, 2^-8 * rms of that (v, j) row).
+BUILD_MAX_ULPS = 2.0
+
+
+def dev(a: np.ndarray, device="cuda") -> torch.Tensor:
+    """numpy -> device tensor; uint16 arrays are bf16 bit patterns."""
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16).copy()).view(torch.bfloat16).to(device)
+    return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+
+def host_bits(t: torch.Tensor) -> np.ndarray:
+    """device bf16 tensor -> uint16 bit patterns; fp32 -> float32."""
+    t = t.detach().cpu().contiguous()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16)
+    if t.dtype == torch.float16:
+        return t.view(torch.int16).numpy().view(np.uint16)
+    return t.numpy()
+
+
+def as_f64(a: np.ndarray) -> np.ndarray:
+    return (inputs.bf16_bits_to_f32(a) if a.dtype == np.uint16 else a).astype(np.float64)
+
+
+def rel_l2_rows(got: np.ndarray, ref: np.ndarray) -> np.ndarray:
+    got = got.astype(np.float64)
+    num = np.linalg.norm(got - ref, axis=-1)
+    den = np.linalg.norm(ref, axis=-1)
+    return np.where(den > 0, num / np.where(den > 0, den, 1), np.where(num <= 1e-30, 0.0, np.inf))
+
+
+def assert_combine_close(got: np.ndarray, ref: np.ndarray, rtol=COMBINE_RTOL):
+    err = rel_l2_rows(got, ref)
+    worst = int(np.argmax(err)) if err.size else 0
+    assert err.size == 0 or err.max() <= rtol, f"max rel L2 {err.max():.3e} at token {worst}"
+    return float(err.max()) if err.size else 0.0
+
+
+def bf16_ulp(x: np.ndarray) -> np.ndarray:
+    """One bf16 unit in the last place at magnitude |x| (normal range)."""
+    ax = np.maximum(np.abs(x), 2.0 ** -126)
+    return 2.0 ** (np.floor(np.log2(ax)) - 7)
+
+
+def build_ulps(got: np.ndarray, ref: np.ndarray) -> np.ndarray:
+    """|got - ref| in bf16 ulps at max(|ref|, 2^-8 rms(row)); rows are the last axis."""
+    g = as_f64(got) if got.dtype == np.uint16 else got.astype(np.float64)
+    rms = np.sqrt(np.mean(ref ** 2, axis=-1, keepdims=True))
+    scale = np.maximum(np.abs(ref), 2.0 ** -8 * rms)
+    return np.abs(g - ref) / bf16_ulp(scale)
+
+
+def compact_rows(lut_host_rows: np.ndarray, ids: np.ndarray):
+    """Remap ids onto a compact table holding only the rows the batch uses."""
+    uniq, inv = np.unique(ids, return_inverse=True)
+    return uniq, inv.astype(np.int32).ravel()

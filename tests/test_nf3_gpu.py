@@ -1,0 +1,111 @@
+"""Parity of the NF3 path (CUDA, through the C ABI) against the oracle: codes
+and scales bit-exact, the fused dequant-gather-combine within 1e-5 per token.
+
+MoLE page ("ICML 2025 Spotlight | 华为诺亚提出端侧大模型新架构MoLE...", zejuncao.github.io),
+实验结果: the table keeps its quality when stored at 3 bits (e.g. NF3).
+"""
+import numpy as np
+import pytest
+import torch
+
+from helpers import assert_combine_close, dev, host_bits
+from mixture_lookup_experts_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def _special_blocks(lut):
+    """Overwrite a few blocks with edge cases: zeros, tiny values, values past
+    the fp16 range (scale saturates), exact level multiples, one huge outlier."""
+    f = inputs.bf16_bits_to_f32(lut).copy()
+    V, N, D = f.shape
+    f[0, 0, 0:64] = 0.0
+    f[0, 0, 64:128] = np.float32(1e-30)
+    if D >= 192:
+        f[0, 0, 128:192] = np.linspace(-7e4, 7e4, 64, dtype=np.float32)
+    f[1, 0, :64] = np.float32(3.0) * np.array([-1, -0.535, -0.247, 0, 0.1833, 0.382, 0.623, 1.0] * 8, np.float32)
+    if N >= 2:
+        f[1, 1, :64] = np.float32(1e-3)
+        f[1, 1, 5] = np.float32(5.0)
+    return inputs.f32_to_bf16_bits(f)
+
+
+@pytest.mark.parametrize("V,N,D", [(64, 16, 256), (33, 5, 128), (7, 1, 64), (300, 16, 2048)])
+def test_quantize_bit_exact(mole, oracle_mod, V, N, D):
+    rng = np.random.default_rng(V * N + D)
+    lut = _special_blocks(inputs.normal(rng, (V, N, D), 0.02, "bf16"))
+    codes, scales = mole.mole_quantize_lut_nf3(dev(lut))
+    ref_codes, ref_scales = oracle_mod.quantize_nf3(lut)
+    np.testing.assert_array_equal(codes.cpu().numpy(), ref_codes)
+    np.testing.assert_array_equal(host_bits(scales), ref_scales)
+
+
+@pytest.mark.parametrize("V,N,D,T,dtype", [
+    (300, 16, 2048, 300, "bf16"), (100, 16, 128, 77, "bf16"), (50, 5, 64, 19, "bf16"),
+    (64, 24, 256, 40, "bf16"), (80, 8, 192, 33, "f32"),
+])
+def test_combine_nf3_matches_oracle(mole, oracle_mod, V, N, D, T, dtype):
+    rng = np.random.default_rng(T + D)
+    lut = inputs.normal(rng, (V, N, D), 0.02, "bf16")
+    Wr = inputs.normal(rng, (D, N), 0.02, dtype)
+    h = inputs.normal(rng, (T, D), 1.0, dtype)
+    ids = inputs.zipf_ids(rng, T, V)
+    ids[0], ids[-1] = 0, V - 1
+    codes, scales = oracle_mod.quantize_nf3(lut)  # the oracle's codes are the input here
+    out = mole.mole_lookup_combine_nf3(dev(ids), dev(h), dev(Wr), dev(codes),
+                                       dev(scales).view(torch.float16))
+    assert mole.mole_check() == 0
+    ref, _ = oracle_mod.combine_nf3(ids, h, Wr, codes, scales)
+    assert_combine_close(out.cpu().numpy(), ref)
+
+
+def test_combine_nf3_bad_ids(mole, oracle_mod):
+    V, N, D, T = 40, 16, 128, 20
+    rng = np.random.default_rng(3)
+    lut = inputs.normal(rng, (V, N, D), 0.02, "bf16")
+    Wr = inputs.normal(rng, (D, N), 0.02, "bf16")
+    h = inputs.normal(rng, (T, D), 1.0, "bf16")
+    ids = rng.integers(0, V, T).astype(np.int32)
+    ids[[2, 9]] = [-5, V]
+    codes, scales = oracle_mod.quantize_nf3(lut)
+    out = mole.mole_lookup_combine_nf3(dev(ids), dev(h), dev(Wr), dev(codes), dev(scales).view(torch.float16))
+    assert mole.mole_check() == 5
+    got = out.cpu().numpy()
+    assert np.isnan(got[[2, 9]]).all()
+    ref, nbad = oracle_mod.combine_nf3(ids, h, Wr, codes, scales)
+    ok = np.ones(T, bool)
+    ok[[2, 9]] = False
+    assert_combine_close(got[ok], ref[ok])
+
+
+@pytest.mark.parametrize("T,kind", [(1, "zipf"), (64, "zipf"), (4096, "zipf"), (16384, "zipf"), (16384, "uniform")])
+def test_nf3_full_size_sampled(mole, oracle_mod, T, kind):
+    """1B-shaped layer: quantise the full [50304, 16, 2048] table on the GPU,
+    check sampled code blocks bit-exactly and sampled tokens of the fused
+    combine against the oracle on the same codes."""
+    shape = inputs.SHAPES["1b_nf3"]
+    V, D, N = shape.V, shape.D, shape.N
+    g = torch.Generator(device="cuda")
+    g.manual_seed(shape.seed)
+    lut = (torch.randn((V, N, D), generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+    codes, scales = mole.mole_quantize_lut_nf3(lut)
+    rng = np.random.default_rng(shape.seed + T)
+    Wr = inputs.normal(rng, (D, N), 0.02, "bf16")
+    ids = inputs.draw_ids(rng, T, V, kind)
+    ids[0], ids[-1] = 0, V - 1
+    h = inputs.normal(rng, (T, D), 1.0, "bf16")
+    out = mole.mole_lookup_combine_nf3(dev(ids), dev(h), dev(Wr), codes, scales)
+    assert mole.mole_check() == 0
+    sample = np.unique(np.concatenate([[0, T - 1], rng.integers(0, T, 46)]))
+    uniq, inv = np.unique(ids[sample], return_inverse=True)
+    sel = torch.from_numpy(uniq.astype(np.int64)).cuda()
+    rows = host_bits(lut[sel])
+    # codes of the sampled rows are bit-exact
+    ref_codes, ref_scales = oracle_mod.quantize_nf3(rows)
+    np.testing.assert_array_equal(codes[sel].cpu().numpy(), ref_codes)
+    np.testing.assert_array_equal(host_bits(scales[sel]), ref_scales)
+    ref, _ = oracle_mod.combine_nf3(inv.astype(np.int32), h[sample], Wr, ref_codes, ref_scales)
+    got = out[torch.from_numpy(sample).cuda()].cpu().numpy()
+    assert_combine_close(got, ref)
+    del lut, codes, scales, out
+    torch.cuda.empty_cache()
