@@ -166,6 +166,28 @@ def profiled_traffic():
         return None, "summary lacks traffic"
 
 
+def rank_seeds(base: int, rank: int):
+    """(device generator seed, host rng seed) of a rank: each rank draws its own
+    tables and batches (weak scaling: per-rank work is fixed as ranks grow)."""
+    return base + 7919 * rank, base + 104729 * rank
+
+
+def max_over_ranks(values, device):
+    """Element-wise maximum of per-rank timings (the job takes as long as its
+    slowest rank); a no-op on a single process."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def whole_job_tokens_per_s(world: int, tokens_per_step: int, steps: int, max_ms: float) -> float:
+    """Tokens processed by all ranks divided by the slowest rank's time."""
+    return world * tokens_per_step * steps / (max_ms / 1e3)
+
+
 def combine_bytes(U: float, T: int, D: int, N: int) -> float:
     """Algorithmic bytes of one combine launch: unique table rows + h in +
     out (fp32) + router weights + ids."""
@@ -257,12 +279,13 @@ def main():
 
     # ---- layer tables and routers (seeded per rank) ----
     g = torch.Generator(device=dev)
-    g.manual_seed(shape.seed + 7919 * rank)
+    dev_seed, host_seed = rank_seeds(shape.seed, rank)
+    g.manual_seed(dev_seed)
     luts = [(torch.randn((V, N, D), generator=g, device=dev) * 0.02).to(torch.bfloat16) for _ in range(L)]
     routers = [(torch.randn((D, N), generator=g, device=dev) * 0.02).to(torch.bfloat16) for _ in range(L)]
     # per-step batches: a pool of P distinct (ids, h) per layer slot, rotated
     P = 4
-    rng = np.random.default_rng(shape.seed + 104729 * rank)
+    rng = np.random.default_rng(host_seed)
     id_pool = [[torch.from_numpy(inputs.draw_ids(rng, T, V, args.ids)).to(dev) for _ in range(L)] for _ in range(P)]
     h_pool = [[(torch.randn((T, D), generator=g, device=dev)).to(torch.bfloat16) for _ in range(L)]
               for _ in range(P)]
@@ -309,11 +332,8 @@ def main():
     avg_kern_ms = sum(kern_ms) / len(kern_ms)
     U_avg = sum(uniq_counts[(W + i) % P][l] for i in range(K) for l in range(L)) / (K * L)
 
-    t = torch.tensor([elapsed_ms, avg_kern_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms, max_kern_ms = float(t[0]), float(t[1])
-    value = world * T * K / (max_ms / 1e3)
+    max_ms, max_kern_ms = max_over_ranks([elapsed_ms, avg_kern_ms], dev)
+    value = whole_job_tokens_per_s(world, T, K, max_ms)
 
     # ---- end to end through the C ABI with host buffers ----
     h_host = [torch.empty((T, D), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
@@ -345,10 +365,8 @@ def main():
         e2e_step()
     e_end.record(stream)
     torch.cuda.synchronize()
-    e_ms = torch.tensor([e_start.elapsed_time(e_end)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
-    e2e_value = world * T * K_e2e / (float(e_ms[0]) / 1e3)
+    (e_ms,) = max_over_ranks([e_start.elapsed_time(e_end)], dev)
+    e2e_value = whole_job_tokens_per_s(world, T, K_e2e, e_ms)
     h2d = L * T * D * 2 + L * T * 4
     d2h = L * T * D * 4
     del h_host, out_host, h_stage

@@ -7,14 +7,15 @@
 //   GEMM2  LUT[:, e, :]  = H[e] . W2[e]     H[e] [V, Dr] K-major, W2[e] [Dr, D] N-major
 // H is rounded to bf16 (the operand type of the second contraction).
 //
-// Kernel: persistent, one CTA per SM, 6 warps with fixed roles
+// Kernel: persistent, one CTA per SM, 10 warps with fixed roles
 //   warp 0      TMA producer (one lane): A box 64(K) x 128(M), B four boxes
 //               64(N) x 64(K), all 128-byte swizzled, into a 4-stage ring;
 //   warp 1      TMEM owner + MMA issuer (one lane): tcgen05.mma kind::f16,
 //               M=128 N=256 K=16, accumulators double-buffered in TMEM
 //               (2 x 256 fp32 columns = all 512), tcgen05.commit frees smem
 //               stages and signals a finished accumulator;
-//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 32 columns, activation,
+//   warps 2..9  epilogue, two warps per TMEM lane quadrant (each takes half of
+//               the 256 columns): tcgen05.ld 32 lanes x 32 columns, activation,
 //               bf16 rounding, 16-byte stores (row stride ldc, so the second
 //               GEMM writes the strided LUT[:, e, :] directly).
 // Tiles (expert, m-block, n-block) are dealt round-robin to the CTAs with the
@@ -39,7 +40,8 @@ constexpr int B_STAGE = BK * BN * 2;  // 32 KB
 constexpr int STAGE_BYTES = A_STAGE + B_STAGE;
 constexpr int ACC_COLS = BN;
 constexpr int TMEM_COLS = 2 * ACC_COLS;  // 512: two accumulators
-constexpr int kThreads = 192;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kSmemBytes = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES + 256 /*barriers*/;
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 
@@ -201,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4);
+      mbar_init(&tempty[a], kEpiWarps);
     }
     mbar_init(drain, 1);
     *abort = 0;
@@ -283,8 +285,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else {
-    // ---------------- epilogue (warps 2..5) ----------------
-    const int quad = warp & 3;  // TMEM lanes this warp may access
+    // ---------------- epilogue (warps 2..9) ----------------
+    const int quad = warp & 3;                 // TMEM lanes this warp may access
+    const int chunk0 = ((warp - 2) >> 2) * (BN / 64);  // first of its BN/64 column chunks
     uint32_t tl = 0;
     for (int64_t tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, ++tl) {
       const uint32_t acc = tl & 1u, aph = (tl >> 1) & 1u;
@@ -297,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       decode_tile(p, tile, e, mb, nb);
       const int m = mb * BM + quad * 32 + lane;
       uint16_t* crow = p.C + (int64_t)e * p.c_estride + (int64_t)m * p.ldc;
-      for (int chunk = 0; chunk < BN / 32; ++chunk) {
+      for (int chunk = chunk0; chunk < chunk0 + BN / 64; ++chunk) {
         const int col0 = nb * BN + chunk * 32;
         if (col0 >= p.N) break;  // warp-uniform
         uint32_t r[32];

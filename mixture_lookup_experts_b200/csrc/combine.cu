@@ -104,6 +104,7 @@ __device__ __forceinline__ void router_tile(const Smem& s, const int32_t* __rest
   constexpr int NP = 8 * NT;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (kBf16Router) {
+    constexpr int KB = 8;  // k-steps whose A fragments are fetched before their MMAs
     const uint16_t* h = static_cast<const uint16_t*>(h_);
     const int g = lane >> 2, c = lane & 3, ldw = D + 8;
     float acc[NT][4];
@@ -114,14 +115,25 @@ __device__ __forceinline__ void router_tile(const Smem& s, const int32_t* __rest
     const uint16_t* h1 = h + (t0 + (ok1 ? g + 8 : 0)) * (int64_t)D + 4 * c;
     const uint16_t* w = s.wrt + g * ldw + 4 * c;
     const int ksteps = D >> 4;
-    for (int ks = warp; ks < ksteps; ks += kWarps) {
-      const int d = ks << 4;
-      uint2 a0 = ok0 ? __ldg(reinterpret_cast<const uint2*>(h0 + d)) : make_uint2(0u, 0u);
-      uint2 a1 = ok1 ? __ldg(reinterpret_cast<const uint2*>(h1 + d)) : make_uint2(0u, 0u);
+    for (int kb = warp; kb < ksteps; kb += kWarps * KB) {
+      uint2 a0[KB], a1[KB];
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const uint2 b = *reinterpret_cast<const uint2*>(w + nt * 8 * ldw + d);
-        mma_16816(acc[nt], a0.x, a1.x, a0.y, a1.y, b.x, b.y);
+      for (int i = 0; i < KB; ++i) {
+        const int ks = kb + i * kWarps;
+        const bool in = ks < ksteps;
+        a0[i] = (in && ok0) ? __ldg(reinterpret_cast<const uint2*>(h0 + (ks << 4))) : make_uint2(0u, 0u);
+        a1[i] = (in && ok1) ? __ldg(reinterpret_cast<const uint2*>(h1 + (ks << 4))) : make_uint2(0u, 0u);
+      }
+#pragma unroll
+      for (int i = 0; i < KB; ++i) {
+        const int ks = kb + i * kWarps;
+        if (ks < ksteps) {
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            const uint2 b = *reinterpret_cast<const uint2*>(w + nt * 8 * ldw + (ks << 4));
+            mma_16816(acc[nt], a0[i].x, a1[i].x, a0[i].y, a1[i].y, b.x, b.y);
+          }
+        }
       }
     }
     float* pw = s.part + warp * kTileMax * NP;
@@ -195,91 +207,132 @@ __device__ __forceinline__ void router_tile(const Smem& s, const int32_t* __rest
   __syncthreads();
 }
 
+// Which (token row, unit) pairs of a tile this thread handles, for `per_tok`
+// units per token: with fewer units per token than threads, several tokens
+// are covered per pass; computed once per thread, so the gather loop does no
+// division.
+struct UnitMap {
+  int r0, rstep, v0, vstep;
+  __device__ __forceinline__ UnitMap(int per_tok) {
+    const int tid = threadIdx.x;
+    if (per_tok >= kThreads) {
+      r0 = 0;
+      rstep = 1;
+      v0 = tid;
+      vstep = kThreads;
+    } else {
+      const int rp = kThreads / per_tok;
+      v0 = tid % per_tok;
+      r0 = tid / per_tok;
+      rstep = rp;
+      vstep = per_tok;
+      if (r0 >= rp) r0 = kTileMax;  // spare threads: no unit
+    }
+  }
+};
+
 __device__ __forceinline__ void store_nan(float* o, int n) {
-  for (int i = 0; i < n; i += 4) stg_stream(o + i, make_float4(NAN, NAN, NAN, NAN));
+  for (int i = 0; i < n; i += 4) __stcs(reinterpret_cast<float4*>(o + i), make_float4(NAN, NAN, NAN, NAN));
 }
 
-// Gather + combine of one tile from a bf16 table: unit = (token, 8-wide vector).
-template <int NT>
-__device__ __forceinline__ void combine_tile_bf16(const Smem& s, const uint16_t* __restrict__ lut,
-                                                  int64_t V, int N, int D, int64_t t0, int rows,
-                                                  float* __restrict__ out, unsigned* err) {
+__device__ __forceinline__ void load_gates(const float* gr, float* g, int n) {
+  for (int i = 0; i < n; i += 4) {
+    const float4 v = *reinterpret_cast<const float4*>(gr + i);
+    g[i] = v.x;
+    g[i + 1] = v.y;
+    g[i + 2] = v.z;
+    g[i + 3] = v.w;
+  }
+}
+
+// Gather + combine of one tile from a bf16 table: unit = (token, 8-wide
+// vector).  All N row loads of a unit are issued before its first FMA; with
+// an exact expert count there is no predication at all.
+template <int NT, bool kExactN>
+__device__ __forceinline__ void combine_tile_bf16(const Smem& s, const UnitMap& um,
+                                                  const uint16_t* __restrict__ lut, int64_t V, int N,
+                                                  int D, int64_t t0, int rows, float* __restrict__ out,
+                                                  unsigned* err) {
   constexpr int NP = 8 * NT;
-  constexpr int CH = NP < 16 ? NP : 16;  // rows loaded per batch (bounds registers)
+  constexpr int CH = NP < 16 ? NP : 16;  // rows in flight per batch (64 registers)
   const int DV = D >> 3;
-  const int units = rows * DV;
-  for (int u = threadIdx.x; u < units; u += kThreads) {
-    const int r = u / DV, v = u - r * DV;
+  for (int r = um.r0; r < rows; r += um.rstep) {
     const int id = s.tok_id[r];
-    float* o = out + (t0 + r) * (int64_t)D + v * 8;
-    if (id < 0 || (int64_t)id >= V) {
-      if (v == 0) atomicOr(err, kErrIndex);
-      store_nan(o, 8);
-      continue;
-    }
-    const uint16_t* src = lut + (int64_t)id * N * D + v * 8;
-    const float* gr = s.gates + r * NP;
-    float a[8];
+    float g[NP];
+    load_gates(s.gates + r * NP, g, NP);
+    for (int v = um.v0; v < DV; v += um.vstep) {
+      float* o = out + (t0 + r) * (int64_t)D + v * 8;
+      if (id < 0 || (int64_t)id >= V) {
+        if (v == 0) atomicOr(err, kErrIndex);
+        store_nan(o, 8);
+        continue;
+      }
+      const uint4* src = reinterpret_cast<const uint4*>(lut + (int64_t)id * N * D) + v;
+      float a[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) a[i] = 0.f;
+      for (int i = 0; i < 8; ++i) a[i] = 0.f;
 #pragma unroll
-    for (int j0 = 0; j0 < NP; j0 += CH) {
-      uint4 x[CH];
+      for (int j0 = 0; j0 < NP; j0 += CH) {
+        uint4 x[CH];
 #pragma unroll
-      for (int j = 0; j < CH; ++j)
-        if (j0 + j < N) x[j] = ldg_stream(src + (int64_t)(j0 + j) * D);
+        for (int j = 0; j < CH; ++j) {
+          const int jj = kExactN ? j0 + j : min(j0 + j, N - 1);  // padded experts re-read a valid row
+          x[j] = __ldg(src + (int64_t)jj * DV);
+        }
 #pragma unroll
-      for (int j = 0; j < CH; ++j) {
-        if (j0 + j < N) {
-          const float gj = gr[j0 + j];
-          a[0] = fmaf(gj, bf16_lo(x[j].x), a[0]);
-          a[1] = fmaf(gj, bf16_hi(x[j].x), a[1]);
-          a[2] = fmaf(gj, bf16_lo(x[j].y), a[2]);
-          a[3] = fmaf(gj, bf16_hi(x[j].y), a[3]);
-          a[4] = fmaf(gj, bf16_lo(x[j].z), a[4]);
-          a[5] = fmaf(gj, bf16_hi(x[j].z), a[5]);
-          a[6] = fmaf(gj, bf16_lo(x[j].w), a[6]);
-          a[7] = fmaf(gj, bf16_hi(x[j].w), a[7]);
+        for (int j = 0; j < CH; ++j) {
+          if (kExactN || j0 + j < N) {
+            const float gj = g[j0 + j];
+            a[0] = fmaf(gj, bf16_lo(x[j].x), a[0]);
+            a[1] = fmaf(gj, bf16_hi(x[j].x), a[1]);
+            a[2] = fmaf(gj, bf16_lo(x[j].y), a[2]);
+            a[3] = fmaf(gj, bf16_hi(x[j].y), a[3]);
+            a[4] = fmaf(gj, bf16_lo(x[j].z), a[4]);
+            a[5] = fmaf(gj, bf16_hi(x[j].z), a[5]);
+            a[6] = fmaf(gj, bf16_lo(x[j].w), a[6]);
+            a[7] = fmaf(gj, bf16_hi(x[j].w), a[7]);
+          }
         }
       }
+      __stcs(reinterpret_cast<float4*>(o), make_float4(a[0], a[1], a[2], a[3]));
+      __stcs(reinterpret_cast<float4*>(o + 4), make_float4(a[4], a[5], a[6], a[7]));
     }
-    stg_stream(o, make_float4(a[0], a[1], a[2], a[3]));
-    stg_stream(o + 4, make_float4(a[4], a[5], a[6], a[7]));
   }
 }
 
 // Gather + combine of one tile from an fp32 table: unit = (token, 4-wide vector).
-template <int NT>
-__device__ __forceinline__ void combine_tile_f32(const Smem& s, const float* __restrict__ lut,
-                                                 int64_t V, int N, int D, int64_t t0, int rows,
-                                                 float* __restrict__ out, unsigned* err) {
+template <int NT, bool kExactN>
+__device__ __forceinline__ void combine_tile_f32(const Smem& s, const UnitMap& um,
+                                                 const float* __restrict__ lut, int64_t V, int N, int D,
+                                                 int64_t t0, int rows, float* __restrict__ out,
+                                                 unsigned* err) {
   constexpr int NP = 8 * NT;
   const int DV = D >> 2;
-  const int units = rows * DV;
-  for (int u = threadIdx.x; u < units; u += kThreads) {
-    const int r = u / DV, v = u - r * DV;
+  for (int r = um.r0; r < rows; r += um.rstep) {
     const int id = s.tok_id[r];
-    float* o = out + (t0 + r) * (int64_t)D + v * 4;
-    if (id < 0 || (int64_t)id >= V) {
-      if (v == 0) atomicOr(err, kErrIndex);
-      store_nan(o, 4);
-      continue;
-    }
-    const float* src = lut + (int64_t)id * N * D + v * 4;
-    const float* gr = s.gates + r * NP;
-    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int j = 0; j < NP; ++j) {
-      if (j < N) {
-        const float4 x = __ldg(reinterpret_cast<const float4*>(src + (int64_t)j * D));
-        const float gj = gr[j];
-        a.x = fmaf(gj, x.x, a.x);
-        a.y = fmaf(gj, x.y, a.y);
-        a.z = fmaf(gj, x.z, a.z);
-        a.w = fmaf(gj, x.w, a.w);
+    float g[NP];
+    load_gates(s.gates + r * NP, g, NP);
+    for (int v = um.v0; v < DV; v += um.vstep) {
+      float* o = out + (t0 + r) * (int64_t)D + v * 4;
+      if (id < 0 || (int64_t)id >= V) {
+        if (v == 0) atomicOr(err, kErrIndex);
+        store_nan(o, 4);
+        continue;
       }
+      const float4* src = reinterpret_cast<const float4*>(lut + (int64_t)id * N * D) + v;
+      float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int j = 0; j < NP; ++j) {
+        if (kExactN || j < N) {
+          const float4 x = __ldg(src + (int64_t)j * DV);
+          a.x = fmaf(g[j], x.x, a.x);
+          a.y = fmaf(g[j], x.y, a.y);
+          a.z = fmaf(g[j], x.z, a.z);
+          a.w = fmaf(g[j], x.w, a.w);
+        }
+      }
+      __stcs(reinterpret_cast<float4*>(o), a);
     }
-    stg_stream(o, a);
   }
 }
 
@@ -309,72 +362,74 @@ __device__ __forceinline__ void nf3_fma4(uint32_t sel, float a, float* acc) {
 
 // Gather + combine of one tile from an NF3 table: unit = (token, 32-element
 // half block); the half block's codes are 12 bytes (3 words) per expert row.
-template <int NT>
-__device__ __forceinline__ void combine_tile_nf3(const Smem& s, const uint8_t* __restrict__ codes,
-                                                 const uint16_t* __restrict__ scales, int64_t V,
-                                                 int N, int D, int64_t t0, int rows,
-                                                 float* __restrict__ out, unsigned* err) {
+template <int NT, bool kExactN>
+__device__ __forceinline__ void combine_tile_nf3(const Smem& s, const UnitMap& um,
+                                                 const uint8_t* __restrict__ codes,
+                                                 const uint16_t* __restrict__ scales, int64_t V, int N,
+                                                 int D, int64_t t0, int rows, float* __restrict__ out,
+                                                 unsigned* err) {
   constexpr int NP = 8 * NT;
   constexpr int CH = NP < 8 ? NP : 8;
-  const int NB = D >> 6;       // 64-element blocks per row
-  const int HB = D >> 5;       // half blocks per row
-  const int units = rows * HB;
-  for (int u = threadIdx.x; u < units; u += kThreads) {
-    const int r = u / HB, hb = u - r * HB;
+  const int NB = D >> 6;  // 64-element blocks per row
+  const int HB = D >> 5;  // half blocks per row
+  for (int r = um.r0; r < rows; r += um.rstep) {
     const int id = s.tok_id[r];
-    float* o = out + (t0 + r) * (int64_t)D + hb * 32;
-    if (id < 0 || (int64_t)id >= V) {
-      if (hb == 0) atomicOr(err, kErrIndex);
-      store_nan(o, 32);
-      continue;
-    }
-    const int b = hb >> 1, half = hb & 1;
-    const int64_t blk0 = (int64_t)id * N * NB + b;  // block of expert 0
-    const float* gr = s.gates + r * NP;
-    float acc[32];
+    float g[NP];
+    load_gates(s.gates + r * NP, g, NP);
+    for (int hb = um.v0; hb < HB; hb += um.vstep) {
+      float* o = out + (t0 + r) * (int64_t)D + hb * 32;
+      if (id < 0 || (int64_t)id >= V) {
+        if (hb == 0) atomicOr(err, kErrIndex);
+        store_nan(o, 32);
+        continue;
+      }
+      const int b = hb >> 1, half = hb & 1;
+      const int64_t blk0 = (int64_t)id * N * NB + b;  // block of expert 0
+      float acc[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+      for (int i = 0; i < 32; ++i) acc[i] = 0.f;
 #pragma unroll
-    for (int j0 = 0; j0 < NP; j0 += CH) {
-      uint32_t w[CH][3];
-      float sc[CH];
+      for (int j0 = 0; j0 < NP; j0 += CH) {
+        uint32_t w[CH][3];
+        float sc[CH];
 #pragma unroll
-      for (int j = 0; j < CH; ++j) {
-        if (j0 + j < N) {
-          const int64_t blk = blk0 + (int64_t)(j0 + j) * NB;
+        for (int j = 0; j < CH; ++j) {
+          const int jj = kExactN ? j0 + j : min(j0 + j, N - 1);
+          const int64_t blk = blk0 + (int64_t)jj * NB;
           const uint32_t* cw = reinterpret_cast<const uint32_t*>(codes + blk * 24 + half * 12);
           w[j][0] = __ldg(cw);
           w[j][1] = __ldg(cw + 1);
           w[j][2] = __ldg(cw + 2);
           sc[j] = __half2float(__ushort_as_half(__ldg(scales + blk)));
         }
-      }
 #pragma unroll
-      for (int j = 0; j < CH; ++j) {
-        if (j0 + j < N) {
-          const float a = gr[j0 + j] * sc[j];
-          const uint32_t x0 = w[j][0];
-          const uint32_t x1 = __funnelshift_r(w[j][0], w[j][1], 24);
-          const uint32_t x2 = __funnelshift_r(w[j][1], w[j][2], 16);
-          const uint32_t x3 = w[j][2] >> 8;
-          uint32_t sl, sh;
-          nf3_selectors(x0, sl, sh);
-          nf3_fma4(sl, a, acc + 0);
-          nf3_fma4(sh, a, acc + 4);
-          nf3_selectors(x1, sl, sh);
-          nf3_fma4(sl, a, acc + 8);
-          nf3_fma4(sh, a, acc + 12);
-          nf3_selectors(x2, sl, sh);
-          nf3_fma4(sl, a, acc + 16);
-          nf3_fma4(sh, a, acc + 20);
-          nf3_selectors(x3, sl, sh);
-          nf3_fma4(sl, a, acc + 24);
-          nf3_fma4(sh, a, acc + 28);
+        for (int j = 0; j < CH; ++j) {
+          if (kExactN || j0 + j < N) {
+            const float a = g[j0 + j] * sc[j];
+            const uint32_t x0 = w[j][0];
+            const uint32_t x1 = __funnelshift_r(w[j][0], w[j][1], 24);
+            const uint32_t x2 = __funnelshift_r(w[j][1], w[j][2], 16);
+            const uint32_t x3 = w[j][2] >> 8;
+            uint32_t sl, sh;
+            nf3_selectors(x0, sl, sh);
+            nf3_fma4(sl, a, acc + 0);
+            nf3_fma4(sh, a, acc + 4);
+            nf3_selectors(x1, sl, sh);
+            nf3_fma4(sl, a, acc + 8);
+            nf3_fma4(sh, a, acc + 12);
+            nf3_selectors(x2, sl, sh);
+            nf3_fma4(sl, a, acc + 16);
+            nf3_fma4(sh, a, acc + 20);
+            nf3_selectors(x3, sl, sh);
+            nf3_fma4(sl, a, acc + 24);
+            nf3_fma4(sh, a, acc + 28);
+          }
         }
       }
-    }
 #pragma unroll
-    for (int i = 0; i < 32; i += 4) stg_stream(o + i, make_float4(acc[i], acc[i + 1], acc[i + 2], acc[i + 3]));
+      for (int i = 0; i < 32; i += 4)
+        __stcs(reinterpret_cast<float4*>(o + i), make_float4(acc[i], acc[i + 1], acc[i + 2], acc[i + 3]));
+    }
   }
 }
 
@@ -392,7 +447,7 @@ struct CombineArgs {
   unsigned* err;
 };
 
-template <bool kBf16Router, int NT, int kTable>
+template <bool kBf16Router, int NT, int kTable, bool kExactN>
 __global__ void __launch_bounds__(kThreads, 2) combine_kernel(const CombineArgs p) {
   constexpr int NP = 8 * NT;
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -407,17 +462,21 @@ __global__ void __launch_bounds__(kThreads, 2) combine_kernel(const CombineArgs 
     }
     __syncthreads();
   }
+  const int per_tok = kTable == kTableBf16 ? (p.D >> 3) : kTable == kTableF32 ? (p.D >> 2) : (p.D >> 5);
+  const UnitMap um(per_tok);
   for (int64_t tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x) {
     const int64_t t0 = tile * p.TT;
     const int rows = (int)(p.T - t0 < p.TT ? p.T - t0 : p.TT);
     router_tile<kBf16Router, NT>(s, p.ids, p.h, p.Wr, t0, rows, p.N, p.D);
     if (kTable == kTableBf16)
-      combine_tile_bf16<NT>(s, static_cast<const uint16_t*>(p.table), p.V, p.N, p.D, t0, rows, p.out, p.err);
+      combine_tile_bf16<NT, kExactN>(s, um, static_cast<const uint16_t*>(p.table), p.V, p.N, p.D, t0, rows,
+                                     p.out, p.err);
     else if (kTable == kTableF32)
-      combine_tile_f32<NT>(s, static_cast<const float*>(p.table), p.V, p.N, p.D, t0, rows, p.out, p.err);
+      combine_tile_f32<NT, kExactN>(s, um, static_cast<const float*>(p.table), p.V, p.N, p.D, t0, rows,
+                                    p.out, p.err);
     else
-      combine_tile_nf3<NT>(s, static_cast<const uint8_t*>(p.table), p.scales, p.V, p.N, p.D, t0, rows,
-                           p.out, p.err);
+      combine_tile_nf3<NT, kExactN>(s, um, static_cast<const uint8_t*>(p.table), p.scales, p.V, p.N, p.D,
+                                    t0, rows, p.out, p.err);
     // the next tile's router writes part/gates/tok_id only after its own
     // __syncthreads, which every thread reaches after finishing this tile
   }
@@ -439,12 +498,12 @@ int choose_tile(int64_t T, int n_sm) {
   return best;
 }
 
-template <bool kBf16Router, int NT, int kTable>
+template <bool kBf16Router, int NT, int kTable, bool kExactN>
 mole_status launch_one(CombineArgs p, cudaStream_t stream) {
   constexpr int NP = 8 * NT;
   const size_t smem = smem_bytes_for<kBf16Router, NP>(p.D);
   if (smem > 227 * 1024) return MOLE_ERR_UNSUPPORTED;
-  auto kern = combine_kernel<kBf16Router, NT, kTable>;
+  auto kern = combine_kernel<kBf16Router, NT, kTable, kExactN>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return MOLE_ERR_CUDA;
   const int n_sm = num_sms();
@@ -461,9 +520,12 @@ mole_status launch_one(CombineArgs p, cudaStream_t stream) {
 
 template <bool kBf16Router, int kTable>
 mole_status launch_combine(const CombineArgs& p, cudaStream_t stream) {
-  if (p.N <= 8) return launch_one<kBf16Router, 1, kTable>(p, stream);
-  if (p.N <= 16) return launch_one<kBf16Router, 2, kTable>(p, stream);
-  return launch_one<kBf16Router, 4, kTable>(p, stream);
+  if (p.N == 16) return launch_one<kBf16Router, 2, kTable, true>(p, stream);
+  if (p.N == 8) return launch_one<kBf16Router, 1, kTable, true>(p, stream);
+  if (p.N <= 8) return launch_one<kBf16Router, 1, kTable, false>(p, stream);
+  if (p.N <= 16) return launch_one<kBf16Router, 2, kTable, false>(p, stream);
+  if (p.N == 32) return launch_one<kBf16Router, 4, kTable, true>(p, stream);
+  return launch_one<kBf16Router, 4, kTable, false>(p, stream);
 }
 
 }  // namespace

@@ -8,8 +8,15 @@ from mixture_lookup_experts_b200 import inputs
 # (fp32 accumulation over bf16 table values).
 COMBINE_RTOL = 1e-5
 # Table build tolerance: 2 bf16 ulps of the fp64 reference, the ulp taken at
-# max(|ref|, 2^-8 * rms of that (v, j) row).
+# max(|ref|, rms of that (v, j) row / 8).  Below the floor an element is the
+# result of cancellation: there a legitimate 1-ulp difference in the bf16
+# rounding of one hidden activation H_k (the GPU rounds its fp32 sum, the
+# oracle its fp64 sum) moves the output by ~2^-8 |H_k W2_kd|, i.e. about
+# 8c/sqrt(Dr) floored ulps with c = |H_k W2_kd| / (rms(H) rms(W2)).
 BUILD_MAX_ULPS = 2.0
+BUILD_FLOOR = 1.0 / 8
+# and per (v, j) row, relative L2 error at most the bf16 rounding level
+BUILD_ROW_RTOL = 2.0 ** -8
 
 
 def dev(a: np.ndarray, device="cuda") -> torch.Tensor:
@@ -53,12 +60,23 @@ def bf16_ulp(x: np.ndarray) -> np.ndarray:
     return 2.0 ** (np.floor(np.log2(ax)) - 7)
 
 
-def build_ulps(got: np.ndarray, ref: np.ndarray) -> np.ndarray:
-    """|got - ref| in bf16 ulps at max(|ref|, 2^-8 rms(row)); rows are the last axis."""
+def build_ulps(got: np.ndarray, ref: np.ndarray, floor: float = BUILD_FLOOR) -> np.ndarray:
+    """|got - ref| in bf16 ulps at max(|ref|, floor * rms(row)); rows are the last axis."""
     g = as_f64(got) if got.dtype == np.uint16 else got.astype(np.float64)
     rms = np.sqrt(np.mean(ref ** 2, axis=-1, keepdims=True))
-    scale = np.maximum(np.abs(ref), 2.0 ** -8 * rms)
+    scale = np.maximum(np.abs(ref), floor * rms)
     return np.abs(g - ref) / bf16_ulp(scale)
+
+
+def assert_build_close(got: np.ndarray, ref: np.ndarray):
+    """Element-wise <= 2 floored bf16 ulps and per-row relative L2 <= 2^-8."""
+    g = as_f64(got) if got.dtype == np.uint16 else got.astype(np.float64)
+    ulps = build_ulps(got, ref)
+    rel = rel_l2_rows(g, ref)
+    msg = (f"max {ulps.max():.2f} floored bf16 ulps (mean {ulps.mean():.3f}, "
+           f"{(ulps > 1).mean() * 100:.3f}% > 1); max row rel L2 {rel.max():.2e}")
+    assert ulps.max() <= BUILD_MAX_ULPS and rel.max() <= BUILD_ROW_RTOL, msg
+    return ulps
 
 
 def compact_rows(lut_host_rows: np.ndarray, ids: np.ndarray):
