@@ -54,6 +54,9 @@ def _L():
         P, I64, I32, I = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_int
         lib.oracle_build_lut.argtypes = [P, P, P, I64, I64, I32, I64, I, I, I, P, I64, P, I]
         lib.oracle_build_lut.restype = I
+        lib.oracle_build_lut_ex.argtypes = [P, P, P, I64, I64, I32, I64, I, I, I, P, I64, P, P, P, I]
+        lib.oracle_build_lut_ex.restype = I
+        lib.oracle_round_bf16_array.argtypes = [P, P, I64]
         lib.oracle_combine.argtypes = [P, I64, P, I, P, I, P, I, I64, I32, I64, P, P, I]
         lib.oracle_combine.restype = I64
         lib.oracle_gather_plan.argtypes = [P, I64, I64, P, P, P]
@@ -114,13 +117,17 @@ def round_f16(x: float) -> float:
 
 
 def build_lut(E, W1, W2, act_name: str = "gelu", round_h: bool = True, rows=None,
-              nthreads: int = 0) -> np.ndarray:
+              nthreads: int = 0, with_allowance: bool = False):
     """LUT[v, j, :] = act(E[v] . W1[j]) . W2[j] for the requested rows (fp64).
 
     MoLE page, 推理阶段: the embedding matrix is fed to every routed expert.
     E [V, D], W1 [N, D, Dr], W2 [N, Dr, D]; all fp32 or all bf16 bits.
-    Returns [len(rows), N, D] (or [V, N, D] when rows is None).
+    Returns [len(rows), N, D] (or [V, N, D] when rows is None); with
+    with_allowance (needs round_h) also the per-element allowance for
+    ambiguous bf16 roundings of the hidden activation and their count.
     """
+    if with_allowance:
+        return _build_lut_ex(E, W1, W2, act_name, round_h, rows, nthreads)
     E, W1, W2 = _c(E), _c(W1), _c(W2)
     dt = _dtype_code(E)
     assert _dtype_code(W1) == dt and _dtype_code(W2) == dt
@@ -138,6 +145,34 @@ def build_lut(E, W1, W2, act_name: str = "gelu", round_h: bool = True, rows=None
     if rc != 0:
         raise ValueError("oracle_build_lut: bad argument")
     return out
+
+
+def _build_lut_ex(E, W1, W2, act_name, round_h, rows, nthreads):
+    E, W1, W2 = _c(E), _c(W1), _c(W2)
+    dt = _dtype_code(E)
+    V, D = E.shape
+    N, _, Dr = W1.shape
+    if rows is None:
+        n_rows, rows_p = V, None
+    else:
+        rows_arr = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        n_rows, rows_p = rows_arr.size, _p(rows_arr)
+    out = np.empty((n_rows, N, D), dtype=np.float64)
+    allow = np.empty((n_rows, N, D), dtype=np.float64)
+    n_amb = np.zeros(1, dtype=np.int64)
+    rc = _L().oracle_build_lut_ex(_p(E), _p(W1), _p(W2), V, D, N, Dr, ACT[act_name], dt, 1 if round_h else 0,
+                                  rows_p, n_rows, _p(out), _p(allow), _p(n_amb), nthreads)
+    if rc != 0:
+        raise ValueError("oracle_build_lut_ex: bad argument")
+    return out, allow, int(n_amb[0])
+
+
+def round_bf16_array(x: np.ndarray) -> np.ndarray:
+    """Element-wise bf16 rounding (ties to even) of float64 values."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    y = np.empty_like(x)
+    _L().oracle_round_bf16_array(_p(x), _p(y), x.size)
+    return y
 
 
 def combine(ids, h, Wr, lut, V: int | None = None, nthreads: int = 0, return_gates=False):

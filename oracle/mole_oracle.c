@@ -157,10 +157,48 @@ int oracle_max_threads(void) {
  * bf16 (ties to even) before the second product.
  * Returns 0, or -1 on a bad argument / row index.
  */
+/* One unit in the last place of the bf16 value b (normal range; the larger of
+ * the two ulps at a power of two). */
+static double bf16_ulp_of(double b) {
+  double a = fabs(b);
+  if (a < 0x1p-126) return 0x1p-133;
+  int e;
+  frexp(a, &e); /* a = m 2^e, m in [0.5, 1): a lies in [2^(e-1), 2^e) */
+  return ldexp(1.0, e - 1 - 7);
+}
+
+/*
+ * As oracle_build_lut, plus (when allow != NULL, bf16 rounding only) an error
+ * allowance per output element for hidden activations whose bf16 rounding is
+ * ambiguous.  A device computes u = x . W1 in fp32 and the activation in
+ * fp32, so its pre-rounding value may sit on the other side of a bf16
+ * rounding boundary than the exact one when the exact value is closer to that
+ * boundary than
+ *     beta_k = 1.2 * 2^-19 * M_k + 2^-21 |a_k|,
+ * with M_k the largest magnitude of the running sum of u_k taken in order of
+ * d (1.2 bounds the activation's slope, 2^-19 M_k the fp32 accumulation error
+ * over K/16 steps of 16 products with margin, 2^-21 |a_k| the activation's
+ * own error).  For such k either rounding is legitimate, so
+ *     allow[r, j, e] = sum_{ambiguous k} ulp(a_k) |W2[j, k, e]|.
+ * n_ambiguous (nullable) receives the number of ambiguous hidden values.
+ */
+int oracle_build_lut_ex(const void* E, const void* W1, const void* W2, int64_t V,
+                        int64_t D, int32_t N, int64_t Dr, int act, int dtype,
+                        int round_h, const int64_t* rows, int64_t n_rows,
+                        double* out, double* allow, int64_t* n_ambiguous, int nthreads);
+
 int oracle_build_lut(const void* E, const void* W1, const void* W2, int64_t V,
                      int64_t D, int32_t N, int64_t Dr, int act, int dtype,
                      int round_h, const int64_t* rows, int64_t n_rows,
                      double* out, int nthreads) {
+  return oracle_build_lut_ex(E, W1, W2, V, D, N, Dr, act, dtype, round_h, rows, n_rows, out, NULL,
+                             NULL, nthreads);
+}
+
+int oracle_build_lut_ex(const void* E, const void* W1, const void* W2, int64_t V,
+                        int64_t D, int32_t N, int64_t Dr, int act, int dtype,
+                        int round_h, const int64_t* rows, int64_t n_rows,
+                        double* out, double* allow, int64_t* n_ambiguous, int nthreads) {
   if (V <= 0 || D <= 0 || N <= 0 || Dr <= 0 || n_rows < 0) return -1;
   if (rows == NULL && n_rows != V) return -1;
   for (int64_t r = 0; r < n_rows; ++r) {
@@ -169,37 +207,67 @@ int oracle_build_lut(const void* E, const void* W1, const void* W2, int64_t V,
   }
   set_threads(nthreads);
   int bad = 0;
-#pragma omp parallel for schedule(dynamic) reduction(| : bad)
+  int64_t n_amb = 0;
+#pragma omp parallel for schedule(dynamic) reduction(| : bad) reduction(+ : n_amb)
   for (int64_t r = 0; r < n_rows; ++r) {
     int64_t v = rows ? rows[r] : r;
     double* x = (double*)malloc(sizeof(double) * (size_t)D);
     double* u = (double*)malloc(sizeof(double) * (size_t)Dr);
-    if (!x || !u) { bad = 1; free(x); free(u); continue; }
+    double* mag = (double*)malloc(sizeof(double) * (size_t)Dr);
+    double* amb = (double*)malloc(sizeof(double) * (size_t)Dr);
+    if (!x || !u || !mag || !amb) { bad = 1; free(x); free(u); free(mag); free(amb); continue; }
     for (int64_t d = 0; d < D; ++d) x[d] = load_elem(E, dtype, v * D + d);
     for (int32_t j = 0; j < N; ++j) {
-      /* u = x . W1[j] */
-      for (int64_t k = 0; k < Dr; ++k) u[k] = 0.0;
+      /* u = x . W1[j], tracking the largest running magnitude of each sum */
+      for (int64_t k = 0; k < Dr; ++k) { u[k] = 0.0; mag[k] = 0.0; }
       for (int64_t d = 0; d < D; ++d) {
         const int64_t base = ((int64_t)j * D + d) * Dr;
-        for (int64_t k = 0; k < Dr; ++k) u[k] += x[d] * load_elem(W1, dtype, base + k);
+        for (int64_t k = 0; k < Dr; ++k) {
+          u[k] += x[d] * load_elem(W1, dtype, base + k);
+          if (fabs(u[k]) > mag[k]) mag[k] = fabs(u[k]);
+        }
       }
-      /* a = act(u), optionally rounded to bf16 */
+      /* a = act(u), optionally rounded to bf16; amb[k] = ulp if ambiguous */
       for (int64_t k = 0; k < Dr; ++k) {
         double a = act_fn(act, u[k]);
-        u[k] = round_h ? round_bf16(a) : a;
+        amb[k] = 0.0;
+        if (round_h) {
+          double ar = round_bf16(a);
+          if (allow) {
+            double ulp = bf16_ulp_of(ar);
+            double to_boundary = 0.5 * ulp - fabs(a - ar);
+            double beta = 1.2 * 0x1p-19 * mag[k] + 0x1p-21 * fabs(a);
+            if (to_boundary <= beta) { amb[k] = ulp; n_amb += 1; }
+          }
+          a = ar;
+        }
+        u[k] = a;
       }
       /* out = a . W2[j] */
       double* o = out + (r * N + j) * D;
-      for (int64_t e = 0; e < D; ++e) o[e] = 0.0;
+      double* al = allow ? allow + (r * N + j) * D : NULL;
+      for (int64_t e = 0; e < D; ++e) { o[e] = 0.0; if (al) al[e] = 0.0; }
       for (int64_t k = 0; k < Dr; ++k) {
         const int64_t base = ((int64_t)j * Dr + k) * D;
-        for (int64_t e = 0; e < D; ++e) o[e] += u[k] * load_elem(W2, dtype, base + e);
+        for (int64_t e = 0; e < D; ++e) {
+          double w = load_elem(W2, dtype, base + e);
+          o[e] += u[k] * w;
+          if (al && amb[k] != 0.0) al[e] += amb[k] * fabs(w);
+        }
       }
     }
     free(x);
     free(u);
+    free(mag);
+    free(amb);
   }
+  if (n_ambiguous) *n_ambiguous = n_amb;
   return bad ? -1 : 0;
+}
+
+/* Element-wise bf16 rounding (ties to even) of n doubles. */
+void oracle_round_bf16_array(const double* x, double* y, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) y[i] = round_bf16(x[i]);
 }
 
 /* ------------------------------------------------------------------------- */

@@ -68,13 +68,21 @@ def build_ulps(got: np.ndarray, ref: np.ndarray, floor: float = BUILD_FLOOR) -> 
     return np.abs(g - ref) / bf16_ulp(scale)
 
 
-def assert_build_close(got: np.ndarray, ref: np.ndarray):
-    """Element-wise <= 2 floored bf16 ulps and per-row relative L2 <= 2^-8."""
+def assert_build_close(got: np.ndarray, ref: np.ndarray, allow: np.ndarray | None = None):
+    """|got - ref| <= 2 bf16 ulps at max(|ref|, rms(row)/8) + allow, element-wise,
+    and per-row relative L2 <= 2^-8.  `allow` is the oracle's allowance for hidden
+    activations whose bf16 rounding is ambiguous (either rounding is legitimate)."""
     g = as_f64(got) if got.dtype == np.uint16 else got.astype(np.float64)
-    ulps = build_ulps(got, ref)
+    rms = np.sqrt(np.mean(ref ** 2, axis=-1, keepdims=True))
+    ulp = bf16_ulp(np.maximum(np.abs(ref), BUILD_FLOOR * rms))
+    err = np.abs(g - ref)
+    if allow is None:
+        allow = np.zeros_like(ref)
+    ulps = np.maximum(err - allow, 0.0) / ulp
     rel = rel_l2_rows(g, ref)
-    msg = (f"max {ulps.max():.2f} floored bf16 ulps (mean {ulps.mean():.3f}, "
-           f"{(ulps > 1).mean() * 100:.3f}% > 1); max row rel L2 {rel.max():.2e}")
+    used = (err > BUILD_MAX_ULPS * ulp).mean() * 100
+    msg = (f"max {ulps.max():.2f} floored bf16 ulps beyond the allowance (mean {ulps.mean():.3f}; "
+           f"{used:.4f}% of elements need the allowance); max row rel L2 {rel.max():.2e}")
     assert ulps.max() <= BUILD_MAX_ULPS and rel.max() <= BUILD_ROW_RTOL, msg
     return ulps
 

@@ -5,8 +5,9 @@ MoLE page ("ICML 2025 Spotlight | 华为诺亚提出端侧大模型新架构MoLE
   - bit-exact on dyadic data where every sum is exact in fp32 (identity / ReLU),
     so any mismatch is an indexing or pipeline fault, not rounding;
   - on N(0, 0.02) data with GELU-type activations: 2 bf16 ulps of the fp64
-    reference, the ulp taken at max(|ref|, rms(row)/8), and row relative L2
-    <= 2^-8 (see helpers.py for why the floor sits at rms/8).
+    reference, the ulp taken at max(|ref|, rms(row)/8), plus the oracle's
+    allowance for hidden activations whose bf16 rounding is ambiguous, and row
+    relative L2 <= 2^-8 (see helpers.py).
 The oracle rounds the hidden activation to bf16 where the bf16 build does.
 """
 import numpy as np
@@ -24,8 +25,8 @@ def _weights(V, D, N, Dr, dtype, seed):
     return inputs.expert_weights(shape)
 
 
-def _check(lut_gpu, ref):
-    return assert_build_close(host_bits(lut_gpu), ref)
+def _check(lut_gpu, ref, allow=None):
+    return assert_build_close(host_bits(lut_gpu), ref, allow)
 
 
 def _dyadic(rng, shape):
@@ -53,7 +54,8 @@ def test_build_tensor_core_bit_exact_on_dyadic_data(mole, oracle_mod, V, D, N, D
     W2 = inputs.f32_to_bf16_bits(_dyadic(rng, (N, Dr, D)))
     lut = mole.mole_build_lut(dev(E), dev(W1), dev(W2), act=act)
     assert mole.mole_check() == 0
-    ref = oracle_mod.build_lut(E, W1, W2, act_name=act, round_h=True)
+    # the bf16 table is the exact value rounded to bf16 (ties to even)
+    ref = oracle_mod.round_bf16_array(oracle_mod.build_lut(E, W1, W2, act_name=act, round_h=True))
     got = as_f64(host_bits(lut))
     bad = np.argwhere(got != ref)
     assert bad.size == 0, f"{len(bad)} of {got.size} elements differ, first at {bad[:5].tolist()}"
@@ -69,8 +71,8 @@ def test_build_bf16_tensor_core_matches_oracle(mole, oracle_mod, V, D, N, Dr, ac
     _, E, W1, W2 = _weights(V, D, N, Dr, "bf16", V + D + Dr)
     lut = mole.mole_build_lut(dev(E), dev(W1), dev(W2), act=act)
     assert mole.mole_check() == 0
-    ref = oracle_mod.build_lut(E, W1, W2, act_name=act, round_h=True)
-    _check(lut, ref)
+    ref, allow, _ = oracle_mod.build_lut(E, W1, W2, act_name=act, round_h=True, with_allowance=True)
+    _check(lut, ref, allow)
 
 
 def test_build_workspace_groups_give_the_same_table(mole):
@@ -108,8 +110,8 @@ def test_build_bf16_cuda_core_path(mole, oracle_mod):
     V, D, N, Dr = 97, 48, 3, 1040
     _, E, W1, W2 = _weights(V, D, N, Dr, "bf16", 21)
     lut = mole.mole_build_lut(dev(E), dev(W1), dev(W2))
-    ref = oracle_mod.build_lut(E, W1, W2, act_name="gelu", round_h=True)
-    _check(lut, ref)
+    ref, allow, _ = oracle_mod.build_lut(E, W1, W2, act_name="gelu", round_h=True, with_allowance=True)
+    _check(lut, ref, allow)
 
 
 def test_reparameterisation_invariant_on_gpu(mole, oracle_mod):
@@ -145,7 +147,8 @@ def test_build_full_size_sampled_rows(mole, oracle_mod, shape_name, n_rows):
     edges = [0, 1, 127, 128, 129, 255, 256, V - 129, V - 128, V - 2, V - 1]
     rows = np.unique(np.concatenate([edges, rng.integers(0, V, max(0, n_rows - len(edges)))]))
     E_rows = host_bits(E[torch.from_numpy(rows).cuda()])
-    ref = oracle_mod.build_lut(E_rows, host_bits(W1), host_bits(W2), act_name="gelu", round_h=True)
-    _check(lut[torch.from_numpy(rows).cuda()], ref)
+    ref, allow, _ = oracle_mod.build_lut(E_rows, host_bits(W1), host_bits(W2), act_name="gelu", round_h=True,
+                                         with_allowance=True)
+    _check(lut[torch.from_numpy(rows).cuda()], ref, allow)
     del E, W1, W2, lut
     torch.cuda.empty_cache()

@@ -396,3 +396,26 @@ def test_nf3_combine_is_combine_of_dequantized(oracle_mod):
     g = scipy.special.softmax(_f(h) @ _f(Wr), axis=1)
     np.testing.assert_allclose(out, np.einsum("tj,tjd->td", g, deq[ids]), rtol=1e-12, atol=1e-16)
     assert nb == 0
+
+
+def test_build_allowance_flags_only_values_at_a_rounding_boundary(oracle_mod):
+    # u_0 = 1 + 2^-8 lies exactly between the bf16 neighbours 1 and 1 + 2^-7
+    # (ambiguous); u_1 = 1 + 2^-9 is a quarter ulp from 1 (not ambiguous).
+    E = np.array([[1.0]], np.float32)
+    W1 = np.array([[[1 + 2 ** -8, 1 + 2 ** -9]]], np.float32)
+    W2 = np.array([[[2.0], [3.0]]], np.float32)
+    out, allow, n_amb = oracle_mod.build_lut(E, W1, W2, act_name="identity", round_h=True, with_allowance=True)
+    assert n_amb == 1
+    assert out[0, 0, 0] == 1.0 * 2 + 1.0 * 3  # both round to 1 (ties to even)
+    assert allow[0, 0, 0] == 2 ** -7 * 2.0    # one ulp of the ambiguous value times |W2|
+    # the allowance path computes the same table as the plain one
+    _, _, E2, W12, W22 = _tiny(16, dtype="bf16")
+    a = oracle_mod.build_lut(E2, W12, W22, act_name="gelu", round_h=True)
+    b, al, _ = oracle_mod.build_lut(E2, W12, W22, act_name="gelu", round_h=True, with_allowance=True)
+    np.testing.assert_array_equal(a, b)
+    assert (al >= 0).all()
+
+
+def test_round_bf16_array_matches_scalar(oracle_mod):
+    x = np.random.default_rng(8).standard_normal(500) * 10
+    np.testing.assert_array_equal(oracle_mod.round_bf16_array(x), [oracle_mod.round_bf16(v) for v in x])
