@@ -55,17 +55,23 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--tokens", type=int, default=16384)
     ap.add_argument("--ids", choices=["zipf", "uniform"], default="zipf")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="layer tables to allocate (default: the model's 16); fewer only for profiling runs")
     ap.add_argument("--no-extras", action="store_true", help="skip the build / NF3 / other-case legs")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--build-only", action="store_true",
+                    help="run only the table-build leg (for profiling the tensor-core kernels)")
     return ap.parse_args()
 
 
-def workload_config(T: int, kind: str) -> dict:
+def workload_config(T: int, kind: str, layers: int | None = None) -> dict:
     s = inputs.SHAPES["1b"]
+    layers = s.layers if layers is None else layers
     return {
-        "workload": f"1B-activated-shaped MoLE lookup path, {s.layers} layers x mole_lookup_combine, "
+        "workload": f"1B-activated-shaped MoLE lookup path, {layers} layers x mole_lookup_combine, "
                     f"prefill T={T}, {'Zipf(1.1)' if kind == 'zipf' else 'uniform'} ids",
-        "V": s.V, "D": s.D, "N": s.N, "layers": s.layers, "tokens_per_step": T, "ids": kind,
+        "V": s.V, "D": s.D, "N": s.N, "layers": layers, "tokens_per_step": T, "ids": kind,
         "table_dtype": "bf16", "accumulate": "f32", "out_dtype": "f32",
         "l2": "inputs larger than L2: each step reads 16 distinct 3.3 GB layer tables",
         "data": "synthetic seeded N(0,0.02) tables; fresh ids and hidden states per step",
@@ -272,8 +278,19 @@ def main():
     dev = torch.device("cuda", local_rank)
     stream = torch.cuda.current_stream()
 
+    if args.build_only:
+        hbm_peak, bf16_peak, bf16_sust, peak_kind = measured_peaks()
+        res = build_leg(mole, dev, stream, bf16_peak, bf16_sust, peak_kind, reps=max(1, args.steps),
+                        warmup=max(1, args.warmup))
+        if rank == 0:
+            print(json.dumps({"build": res}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
     shape = inputs.SHAPES["1b"]
-    V, D, N, L = shape.V, shape.D, shape.N, shape.layers
+    V, D, N = shape.V, shape.D, shape.N
+    L = shape.layers if args.layers is None else max(1, args.layers)
     T = args.tokens
     W, K = args.warmup, args.steps
 
@@ -336,10 +353,58 @@ def main():
     value = whole_job_tokens_per_s(world, T, K, max_ms)
 
     # ---- end to end through the C ABI with host buffers ----
+    e2e = None if args.no_e2e else e2e_leg(mole, id_pool, h_pool, routers, luts, out, dev, stream, world, W, K, T, L)
+
+    # ---- roofline of the combine kernel ----    hbm_peak, bf16_peak, bf16_sust, peak_kind = measured_peaks()
+    alg_bytes = combine_bytes(U_avg, T, D, N)
+    achieved_gbs = alg_bytes / (max_kern_ms / 1e3) / 1e9
+    traffic, traffic_note = profiled_traffic()
+    roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
+                "frac": achieved_gbs / hbm_peak, "traffic": traffic,
+                "kernel": "combine_kernel<bf16 router, 16 experts, bf16 table>",
+                "algorithmic_bytes_per_launch": alg_bytes, "unique_rows_per_launch": U_avg,
+                "avg_launch_us": max_kern_ms * 1e3, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
+                "frac_of_8TBs": achieved_gbs / 8000.0, "traffic_source": traffic_note}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": max_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic", "config": workload_config(T, args.ids, L),
+        "layer_tokens_per_s": value * L, "hbm_gbs": achieved_gbs,
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": K * L,
+        "clocks": clocks.summary(),
+    }
+
+    # ---- extras: other prefill cases, NF3 table, table build ----
+    if not args.no_extras:
+        line["cases"] = other_cases(mole, luts, routers, rng, g, dev, stream, W, T, args.ids, L)
+        line["nf3"] = nf3_leg(mole, luts, routers, id_pool, h_pool, uniq_counts, dev, stream, W, K, T, P, L)
+        del luts
+        torch.cuda.empty_cache()
+        line["build"] = build_leg(mole, dev, stream, bf16_peak, bf16_sust, peak_kind)
+
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def e2e_leg(mole, id_pool, h_pool, routers, luts, out, dev, stream, world, W, K, T, L):
+    """The same metric through the C ABI with host buffers: per step the ids
+    and the L hidden-state batches are copied host -> device from pinned
+    memory, the L combine calls run, and the L outputs are copied back."""
+    import torch
+    import torch.distributed as dist
+    D = out.shape[1]
     h_host = [torch.empty((T, D), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
     ids_host = torch.empty((L, T), dtype=torch.int32).pin_memory()
     out_host = torch.empty((T, D), dtype=torch.float32).pin_memory()
-    for s in range(2):
+    for s in range(min(2, L)):
         h_host[s].copy_(h_pool[0][s])
     ids_host.copy_(torch.stack(id_pool[0]).cpu())
     h_stage = torch.empty((T, D), dtype=torch.bfloat16, device=dev)
@@ -366,51 +431,10 @@ def main():
     e_end.record(stream)
     torch.cuda.synchronize()
     (e_ms,) = max_over_ranks([e_start.elapsed_time(e_end)], dev)
-    e2e_value = whole_job_tokens_per_s(world, T, K_e2e, e_ms)
-    h2d = L * T * D * 2 + L * T * 4
-    d2h = L * T * D * 4
-    del h_host, out_host, h_stage
-
-    # ---- roofline of the combine kernel ----
-    hbm_peak, bf16_peak, bf16_sust, peak_kind = measured_peaks()
-    alg_bytes = combine_bytes(U_avg, T, D, N)
-    achieved_gbs = alg_bytes / (max_kern_ms / 1e3) / 1e9
-    traffic, traffic_note = profiled_traffic()
-    roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved_gbs / hbm_peak, "traffic": traffic,
-                "kernel": "combine_kernel<bf16 router, 16 experts, bf16 table>",
-                "algorithmic_bytes_per_launch": alg_bytes, "unique_rows_per_launch": U_avg,
-                "avg_launch_us": max_kern_ms * 1e3, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
-                "frac_of_8TBs": achieved_gbs / 8000.0, "traffic_source": traffic_note}
-
-    line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
-        "ms_per_step": max_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic", "config": workload_config(T, args.ids),
-        "layer_tokens_per_s": value * L, "hbm_gbs": achieved_gbs,
-        "roofline": roofline,
-        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "steps": K_e2e, "note": "per step: ids + 16 hidden-state batches H2D from pinned memory, "
-                                        "16 combine calls through the C ABI, 16 outputs D2H"},
-        "gpu_launches": K * L,
-        "clocks": clocks.summary(),
-    }
-
-    # ---- extras: other prefill cases, NF3 table, table build ----
-    if not args.no_extras:
-        line["cases"] = other_cases(mole, luts, routers, rng, g, dev, stream, W, T, args.ids)
-        line["nf3"] = nf3_leg(mole, luts, routers, id_pool, h_pool, uniq_counts, dev, stream, W, K, T, P)
-        del luts
-        torch.cuda.empty_cache()
-        line["build"] = build_leg(mole, dev, stream, bf16_peak, bf16_sust, peak_kind)
-
-    if rank == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(args)
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    return {"value": whole_job_tokens_per_s(world, T, K_e2e, e_ms), "unit": UNIT,
+            "h2d_bytes_per_step": L * T * D * 2 + L * T * 4, "d2h_bytes_per_step": L * T * D * 4,
+            "steps": K_e2e, "note": f"per step: ids + {L} hidden-state batches H2D from pinned memory, "
+                                    f"{L} combine calls through the C ABI, {L} outputs D2H"}
 
 
 def time_launches(fn, n, stream):
@@ -424,10 +448,10 @@ def time_launches(fn, n, stream):
     return [a.elapsed_time(b) for a, b in ev]
 
 
-def other_cases(mole, luts, routers, rng, g, dev, stream, W, T_main, kind_main):
+def other_cases(mole, luts, routers, rng, g, dev, stream, W, T_main, kind_main, L):
     import torch
     shape = inputs.SHAPES["1b"]
-    V, D, N, L = shape.V, shape.D, shape.N, shape.layers
+    V, D, N = shape.V, shape.D, shape.N
     hbm_peak = measured_peaks()[0]
     res = {}
     for T in (4096, 16384):
@@ -455,10 +479,10 @@ def other_cases(mole, luts, routers, rng, g, dev, stream, W, T_main, kind_main):
     return res
 
 
-def nf3_leg(mole, luts, routers, id_pool, h_pool, uniq_counts, dev, stream, W, K, T, P):
+def nf3_leg(mole, luts, routers, id_pool, h_pool, uniq_counts, dev, stream, W, K, T, P, L):
     import torch
     shape = inputs.SHAPES["1b_nf3"]
-    D, N, L = shape.D, shape.N, shape.layers
+    D, N = shape.D, shape.N
     hbm_peak = measured_peaks()[0]
     tables = []
     q_ms = []
@@ -495,7 +519,7 @@ def nf3_leg(mole, luts, routers, id_pool, h_pool, uniq_counts, dev, stream, W, K
             "workload": f"1B-shaped NF3 table (codes + fp16 scale per 64), T={T}, same ids/h as the main case"}
 
 
-def build_leg(mole, dev, stream, bf16_peak, bf16_sust, peak_kind):
+def build_leg(mole, dev, stream, bf16_peak, bf16_sust, peak_kind, reps=3, warmup=1):
     import torch
     shape = inputs.SHAPES["410m"]
     V, D, N, Dr = shape.V, shape.D, shape.N, shape.Dr
@@ -506,8 +530,9 @@ def build_leg(mole, dev, stream, bf16_peak, bf16_sust, peak_kind):
     W2 = (torch.randn((N, Dr, D), generator=g, device=dev) * 0.02).to(torch.bfloat16)
     lut = torch.empty((V, N, D), dtype=torch.bfloat16, device=dev)
     ws = torch.empty(mole.mole_build_lut_workspace(V, D, N, Dr, torch.bfloat16, 0), dtype=torch.uint8, device=dev)
-    mole.mole_build_lut(E, W1, W2, lut=lut, workspace=ws, stream=stream)
-    ms = time_launches(lambda i: mole.mole_build_lut(E, W1, W2, lut=lut, workspace=ws, stream=stream), 3, stream)
+    for _ in range(warmup):
+        mole.mole_build_lut(E, W1, W2, lut=lut, workspace=ws, stream=stream)
+    ms = time_launches(lambda i: mole.mole_build_lut(E, W1, W2, lut=lut, workspace=ws, stream=stream), reps, stream)
     assert mole.mole_check(stream) == 0
     best = min(ms)
     flops = 4.0 * V * D * Dr * N

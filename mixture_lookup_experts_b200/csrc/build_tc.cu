@@ -43,7 +43,6 @@ constexpr int TMEM_COLS = 2 * ACC_COLS;  // 512: two accumulators
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kSmemBytes = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES + 256 /*barriers*/;
-constexpr uint64_t kWaitLimitNs = 4000000000ull;
 
 // Instruction descriptor, kind::f16: D fp32, A bf16 K-major, B bf16 N-major
 // (bit 16), N/8 at bits 17-22, M/16 at bits 24-28.
@@ -61,67 +60,6 @@ struct Params {
   int64_t tiles;
   unsigned* err;
 };
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ uint64_t globaltimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_test(uint64_t* b, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(b)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Waits for the phase with the given parity to complete.  Gives up (returns
-// false) when *abort is set by another role or after kWaitLimitNs, in which
-// case it sets *abort and the device error word.
-__device__ __noinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort, unsigned* err) {
-  if (mbar_test(b, parity)) return true;
-  const uint64_t t0 = globaltimer();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_test(b, parity)) return true;
-    if ((i & 63) == 0) {
-      if (*abort) return false;
-      if (globaltimer() - t0 > kWaitLimitNs) {
-        *abort = 1;
-        atomicOr(err, kErrTimeout);
-        return false;
-      }
-    }
-  }
-}
-
-// Bounded wait used while draining after an abort (ignores the abort flag).
-__device__ __noinline__ void mbar_drain(uint64_t* b, uint32_t parity) {
-  const uint64_t t0 = globaltimer();
-  while (!mbar_test(b, parity))
-    if (globaltimer() - t0 > kWaitLimitNs) return;
-}
 
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
                                             int c2) {
@@ -170,6 +108,34 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Activation, bf16 rounding and 16-byte stores of one 32-column chunk of a
+// row held in registers (the activation is a template argument so the
+// per-element loop has no branch).
+template <int ACT>
+__device__ __forceinline__ void store_chunk(const uint32_t (&r)[32], uint16_t* dst_row) {
+  uint32_t packed[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float x0 = act_t<ACT>(__uint_as_float(r[2 * i]));
+    const float x1 = act_t<ACT>(__uint_as_float(r[2 * i + 1]));
+    const __nv_bfloat162 b2 = __floats2bfloat162_rn(x0, x1);
+    packed[i] = *reinterpret_cast<const uint32_t*>(&b2);
+  }
+  uint4* dst = reinterpret_cast<uint4*>(dst_row);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+}
+
+__device__ __forceinline__ void store_chunk_act(int act, const uint32_t (&r)[32], uint16_t* dst_row) {
+  switch (act) {
+    case MOLE_ACT_GELU_ERF: store_chunk<MOLE_ACT_GELU_ERF>(r, dst_row); break;
+    case MOLE_ACT_GELU_TANH: store_chunk<MOLE_ACT_GELU_TANH>(r, dst_row); break;
+    case MOLE_ACT_RELU: store_chunk<MOLE_ACT_RELU>(r, dst_row); break;
+    case MOLE_ACT_SILU: store_chunk<MOLE_ACT_SILU>(r, dst_row); break;
+    default: store_chunk<MOLE_ACT_IDENTITY>(r, dst_row); break;
+  }
 }
 
 __device__ __forceinline__ void decode_tile(const Params& p, int64_t tile, int& e, int& mb, int& nb) {
@@ -305,20 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (col0 >= p.N) break;  // warp-uniform
         uint32_t r[32];
         tmem_ld32(tmem_base + ((uint32_t)(quad * 32) << 16) + acc * ACC_COLS + chunk * 32, r);
-        if (m < p.M) {
-          uint32_t packed[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float x0 = apply_act(p.act, __uint_as_float(r[2 * i]));
-            const float x1 = apply_act(p.act, __uint_as_float(r[2 * i + 1]));
-            const __nv_bfloat162 b2 = __floats2bfloat162_rn(x0, x1);
-            packed[i] = *reinterpret_cast<const uint32_t*>(&b2);
-          }
-          uint4* dst = reinterpret_cast<uint4*>(crow + col0);
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
-        }
+        if (m < p.M) store_chunk_act(p.act, r, crow + col0);
       }
       tc_fence_before();
       __syncwarp();
@@ -330,6 +283,238 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
+// CTA-pair variant (tcgen05 cta_group::2): a cluster of 2 CTAs computes a
+// 256 x 256 tile.  Each CTA TMA-loads its own 128 rows of A and its own 128
+// columns of B (no multicast); the even CTA issues M=256 N=256 K=16 MMAs that
+// read both CTAs' shared memory and write each CTA's 128 x 256 fp32
+// accumulator into its own TMEM.  Per SM this halves the B bytes per flop, so
+// a 6-stage ring of 32 KB per CTA buffers 1.5x more MMA work than the 1-CTA
+// ring.  Barriers: full[s] lives in the even CTA (both CTAs' copies complete
+// on it); empty[s] and tfull[a] exist in both CTAs and are signalled by one
+// multicast tcgen05.commit; tempty[a] lives in the even CTA and counts the
+// epilogue warps of both CTAs.
+// ---------------------------------------------------------------------------
+constexpr int STAGES2 = 6;
+constexpr int A_STAGE2 = BM * BK * 2;        // this CTA's 128 rows, 16 KB
+constexpr int B_STAGE2 = BK * (BN / 2) * 2;  // this CTA's 128 columns, 16 KB
+constexpr int STAGE2_BYTES = A_STAGE2 + B_STAGE2;
+constexpr int kSmemBytes2 = 1024 + STAGES2 * STAGE2_BYTES + 256;
+constexpr uint32_t kIdesc2 = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((uint32_t)(BN >> 3) << 17) |
+                             ((uint32_t)(2 * BM >> 4) << 24);
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Address of the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* map, uint32_t bar_cluster, int c0,
+                                                 int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+      "%4, %5}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(kIdesc2), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive on the barrier at this offset in the CTAs of `mask` when all prior
+// MMAs of this thread are complete.
+__device__ __forceinline__ void umma_commit_pair(uint64_t* bar, uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(mask)
+      : "memory");
+}
+
+__device__ __noinline__ void spin_ns(uint64_t ns) {
+  const uint64_t t0 = globaltimer();
+  while (globaltimer() - t0 < ns) {
+  }
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    gemm_tc2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                    const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES2 * A_STAGE2;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES2 * B_STAGE2);
+  uint64_t* empty = full + STAGES2;
+  uint64_t* tfull = empty + STAGES2;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES2; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 2 * kEpiWarps);
+    }
+    mbar_init(drain, 1);
+    *abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int kblocks = (p.K + BK - 1) / BK;
+  const int64_t pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+  bool aborted = false;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer (both CTAs) ----------------
+      uint32_t it = 0;
+      bool ok = true;
+      for (int64_t tile = pair; ok && tile < p.tiles; tile += n_pairs) {
+        int e, mb, nb;
+        decode_tile(p, tile, e, mb, nb);
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const uint32_t s = it % STAGES2, ph = (it / STAGES2) & 1u;
+          if (!mbar_wait(&empty[s], ph ^ 1u, abort, p.err)) {
+            ok = false;
+            break;
+          }
+          if (leader) mbar_expect_tx(&full[s], 2 * STAGE2_BYTES);
+          const uint32_t bar = mapa(smem_u32(&full[s]), 0);
+          tma_load_3d_pair(sA + s * A_STAGE2, &map_a, bar, kb * BK, mb * 2 * BM + (int)rank * BM,
+                           p.a_batched ? e : 0);
+#pragma unroll
+          for (int q = 0; q < BN / 128; ++q)
+            tma_load_3d_pair(sB + s * B_STAGE2 + q * B_BOX, &map_b, bar, nb * BN + (int)rank * (BN / 2) + q * 64,
+                             kb * BK, e);
+        }
+      }
+      if (leader) {
+        const uint32_t first = it > (uint32_t)STAGES2 ? it - STAGES2 : 0u;
+        for (uint32_t i = first; i < it; ++i) mbar_drain(&full[i % STAGES2], (i / STAGES2) & 1u);
+      }
+      aborted = !ok;
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ---------------- MMA issuer (even CTA) ----------------
+      uint32_t it = 0, tl = 0;
+      bool ok = true, issued = false;
+      for (int64_t tile = pair; ok && tile < p.tiles; tile += n_pairs, ++tl) {
+        const uint32_t acc = tl & 1u, aph = (tl >> 1) & 1u;
+        if (!mbar_wait(&tempty[acc], aph ^ 1u, abort, p.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const uint32_t s = it % STAGES2, ph = (it / STAGES2) & 1u;
+          if (!mbar_wait(&full[s], ph, abort, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + s * A_STAGE2), b0 = smem_u32(sB + s * B_STAGE2);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            umma_pair(d_tmem, sw128_desc(a0 + 32 * k, 16, 1024), sw128_desc(b0 + 2048 * k, B_BOX, 1024),
+                      (kb | k) != 0);
+          issued = true;
+          umma_commit_pair(&empty[s], 0x3);
+        }
+        if (ok) umma_commit_pair(&tfull[acc], 0x3);
+      }
+      if (!ok && issued) {
+        umma_commit_pair(drain, 0x1);
+        mbar_drain(drain, 0);
+      }
+      aborted = !ok;
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue (warps 2..9 of both CTAs) ----------------
+    const int quad = warp & 3;
+    const int chunk0 = ((warp - 2) >> 2) * (BN / 64);
+    uint32_t tl = 0;
+    for (int64_t tile = pair; tile < p.tiles; tile += n_pairs, ++tl) {
+      const uint32_t acc = tl & 1u, aph = (tl >> 1) & 1u;
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(&tfull[acc], aph, abort, p.err);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) {
+        aborted = true;
+        break;
+      }
+      tc_fence_after();
+      int e, mb, nb;
+      decode_tile(p, tile, e, mb, nb);
+      const int m = mb * 2 * BM + (int)rank * BM + quad * 32 + lane;
+      uint16_t* crow = p.C + (int64_t)e * p.c_estride + (int64_t)m * p.ldc;
+      for (int chunk = chunk0; chunk < chunk0 + BN / 64; ++chunk) {
+        const int col0 = nb * BN + chunk * 32;
+        if (col0 >= p.N) break;  // warp-uniform
+        uint32_t r[32];
+        tmem_ld32(tmem_base + ((uint32_t)(quad * 32) << 16) + acc * ACC_COLS + chunk * 32, r);
+        if (m < p.M) store_chunk_act(p.act, r, crow + col0);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa(smem_u32(&tempty[acc]), 0));
+    }
+  }
+
+  // A CTA that gave up leaves its peer's copies time to land before the pair
+  // passes the final cluster barrier (the even CTA drains its own barriers).
+  if (__syncthreads_or(aborted ? 1 : 0) && !leader) spin_ns(10000000ull);
+  tc_fence_before();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
                  : "memory");
   }
 }
@@ -361,18 +546,27 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-mole_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, Params p, cudaStream_t stream) {
-  static bool attr_set = false;
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) !=
-        cudaSuccess)
-      return MOLE_ERR_CUDA;
-    attr_set = true;
+mole_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, Params p, bool pair_tiles,
+                        cudaStream_t stream) {
+  static bool attr_set[64][2] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOLE_ERR_CUDA;
+  if (!attr_set[dev][pair_tiles]) {
+    const cudaError_t e =
+        pair_tiles ? cudaFuncSetAttribute(gemm_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes2)
+                   : cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return MOLE_ERR_CUDA;
+    attr_set[dev][pair_tiles] = true;
   }
   const int n_sm = num_sms();
   if (n_sm <= 0) return MOLE_ERR_NO_DEVICE;
-  const int64_t grid = std::min<int64_t>(p.tiles, n_sm);
-  gemm_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, stream>>>(ma, mb, p);
+  if (pair_tiles) {
+    const int64_t pairs = std::min<int64_t>(p.tiles, n_sm / 2);
+    gemm_tc2_kernel<<<(unsigned)(2 * pairs), kThreads, kSmemBytes2, stream>>>(ma, mb, p);
+  } else {
+    const int64_t grid = std::min<int64_t>(p.tiles, n_sm);
+    gemm_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, stream>>>(ma, mb, p);
+  }
   return cuda_status(cudaGetLastError());
 }
 
@@ -401,6 +595,9 @@ mole_status build_tc(const void* E, const void* W1, const void* W2, int64_t V, i
   const uint16_t* w2 = static_cast<const uint16_t*>(W2);
   uint16_t* H = static_cast<uint16_t*>(ws);
   uint16_t* L = static_cast<uint16_t*>(lut);
+  // CTA pairs (256-row tiles) once there are at least two 128-row blocks
+  const bool pair_tiles = V >= 2 * BM;
+  const int mtile = pair_tiles ? 2 * BM : BM;
   for (int e0 = 0; e0 < N; e0 += group) {
     const int g = std::min(group, N - e0);
     // GEMM1: H[e] = act(E . W1[e0 + e])
@@ -416,11 +613,11 @@ mole_status build_tc(const void* E, const void* W1, const void* W2, int64_t V, i
     p1.C = H;
     p1.ldc = Dr;
     p1.c_estride = V * Dr;
-    p1.m_blocks = (int)((V + BM - 1) / BM);
+    p1.m_blocks = (int)((V + mtile - 1) / mtile);
     p1.n_blocks = (int)((Dr + BN - 1) / BN);
     p1.tiles = (int64_t)g * p1.m_blocks * p1.n_blocks;
     p1.err = err;
-    mole_status st = launch_gemm(ma, mb, p1, stream);
+    mole_status st = launch_gemm(ma, mb, p1, pair_tiles, stream);
     if (st != MOLE_OK) return st;
     // GEMM2: LUT[:, e0 + e, :] = H[e] . W2[e0 + e]
     if (!make_map(&ma, H, Dr, V, g, Dr * 2, V * Dr * 2, BM)) return MOLE_ERR_CUDA;
@@ -434,11 +631,11 @@ mole_status build_tc(const void* E, const void* W1, const void* W2, int64_t V, i
     p2.C = L + (int64_t)e0 * D;
     p2.ldc = (int64_t)N * D;
     p2.c_estride = D;
-    p2.m_blocks = (int)((V + BM - 1) / BM);
+    p2.m_blocks = (int)((V + mtile - 1) / mtile);
     p2.n_blocks = (int)((D + BN - 1) / BN);
     p2.tiles = (int64_t)g * p2.m_blocks * p2.n_blocks;
     p2.err = err;
-    st = launch_gemm(ma, mb, p2, stream);
+    st = launch_gemm(ma, mb, p2, pair_tiles, stream);
     if (st != MOLE_OK) return st;
   }
   return MOLE_OK;

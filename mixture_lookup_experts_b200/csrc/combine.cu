@@ -447,6 +447,322 @@ struct CombineArgs {
   unsigned* err;
 };
 
+// ---------------------------------------------------------------------------
+// TMA-staged gather for bf16 tables.  Three roles per persistent CTA (one per
+// SM), pipelined through shared memory:
+//   producer warp   one thread copies each token's whole row block
+//                   LUT[id, 0..N-1, :] (N*D*2 contiguous bytes) into a ring of
+//                   slots with cp.async.bulk (completion on the slot's mbarrier),
+//                   running ahead of the consumers by the ring depth; ids come
+//                   from a per-tile prefetch held in the warp's registers;
+//   router warps    (4) compute the next tile's logits on the tensor cores
+//                   (mma.sync, D split over the 4 warps) and its softmax, into
+//                   one of two gate buffers;
+//   consumer warps  (8) combine each token from its slot (16-byte shared-memory
+//                   reads, fp32 FMAs) and store fp32 outputs.
+// The bulk copies keep up to ring-depth x 64 KB in flight per SM without
+// occupying load registers or per-thread request slots, and the router's
+// latency overlaps the previous tile's combine.
+// ---------------------------------------------------------------------------
+constexpr int kCons = 8;                                  // consumer warps
+constexpr int kRout = 4;                                  // router warps
+constexpr int kTmaThreads = (kCons + kRout + 1) * 32;     // + producer warp
+constexpr int kProducerWarp = kCons + kRout;
+constexpr int kRingBudget = 160 * 1024;                   // bytes of row slots
+
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void named_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Barrier over `threads` threads that also returns the AND of `pred`.
+__device__ __forceinline__ bool named_sync_and(int id, int threads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(pred ? 1u : 0u), "r"(id), "r"(threads)
+      : "memory");
+  return r != 0;
+}
+
+struct TmaSmem {
+  uint16_t* wrt;    // [NP][D + 8] bf16 Wr^T
+  float* part;      // [kRout][kTileMax][NP]
+  float* gates;     // [2][kTileMax][NP]
+  int* tok;         // [2][kTileMax]
+  uint8_t* ring;    // [n_slots][slot_bytes]
+  uint64_t* full;   // [n_slots]
+  uint64_t* empty;  // [n_slots]
+  uint64_t* gfull;  // [2]
+  uint64_t* gempty; // [2]
+  int* abort;
+};
+
+template <int NP>
+__host__ __device__ constexpr size_t tma_fixed_bytes(int D) {
+  return (size_t)NP * (D + 8) * 2 + (size_t)kRout * kTileMax * NP * 4 + 2 * (size_t)kTileMax * NP * 4 +
+         2 * (size_t)kTileMax * 4;
+}
+
+template <int NP>
+__host__ __device__ constexpr size_t tma_smem_bytes(int D, int n_slots, int slot_bytes) {
+  return ((tma_fixed_bytes<NP>(D) + 127) / 128) * 128 + (size_t)n_slots * slot_bytes + (2 * (size_t)n_slots + 4) * 8 +
+         16;
+}
+
+template <int NP>
+__device__ __forceinline__ TmaSmem tma_carve(uint8_t* base, int D, int n_slots, int slot_bytes) {
+  TmaSmem s;
+  size_t off = 0;
+  s.wrt = reinterpret_cast<uint16_t*>(base);
+  off += (size_t)NP * (D + 8) * 2;
+  s.part = reinterpret_cast<float*>(base + off);
+  off += (size_t)kRout * kTileMax * NP * 4;
+  s.gates = reinterpret_cast<float*>(base + off);
+  off += 2 * (size_t)kTileMax * NP * 4;
+  s.tok = reinterpret_cast<int*>(base + off);
+  off += 2 * (size_t)kTileMax * 4;
+  off = (off + 127) / 128 * 128;
+  s.ring = base + off;
+  off += (size_t)n_slots * slot_bytes;
+  s.full = reinterpret_cast<uint64_t*>(base + off);
+  s.empty = s.full + n_slots;
+  s.gfull = s.empty + n_slots;
+  s.gempty = s.gfull + 2;
+  s.abort = reinterpret_cast<int*>(s.gempty + 2);
+  return s;
+}
+
+// Router of one tile by the kRout router warps (named barrier 2): logits on
+// the tensor cores, D split over the warps, then softmax into gates[b].
+template <int NT>
+__device__ __forceinline__ void router_tile_rw(const TmaSmem& s, int b, const int32_t* __restrict__ ids,
+                                               const uint16_t* __restrict__ h, int64_t t0, int rows, int N,
+                                               int D) {
+  constexpr int NP = 8 * NT;
+  constexpr int KB = 8;
+  const int rw = (threadIdx.x >> 5) - kCons;  // router warp index 0..kRout-1
+  const int lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3, ldw = D + 8;
+  float acc[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+  const bool ok0 = g < rows, ok1 = g + 8 < rows;
+  const uint16_t* h0 = h + (t0 + (ok0 ? g : 0)) * (int64_t)D + 4 * c;
+  const uint16_t* h1 = h + (t0 + (ok1 ? g + 8 : 0)) * (int64_t)D + 4 * c;
+  const uint16_t* w = s.wrt + g * ldw + 4 * c;
+  const int ksteps = D >> 4;
+  for (int kb = rw; kb < ksteps; kb += kRout * KB) {
+    uint2 a0[KB], a1[KB];
+#pragma unroll
+    for (int i = 0; i < KB; ++i) {
+      const int ks = kb + i * kRout;
+      const bool in = ks < ksteps;
+      a0[i] = (in && ok0) ? __ldg(reinterpret_cast<const uint2*>(h0 + (ks << 4))) : make_uint2(0u, 0u);
+      a1[i] = (in && ok1) ? __ldg(reinterpret_cast<const uint2*>(h1 + (ks << 4))) : make_uint2(0u, 0u);
+    }
+#pragma unroll
+    for (int i = 0; i < KB; ++i) {
+      const int ks = kb + i * kRout;
+      if (ks < ksteps) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const uint2 bb = *reinterpret_cast<const uint2*>(w + nt * 8 * ldw + (ks << 4));
+          mma_16816(acc[nt], a0[i].x, a1[i].x, a0[i].y, a1[i].y, bb.x, bb.y);
+        }
+      }
+    }
+  }
+  float* pw = s.part + rw * kTileMax * NP;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    pw[g * NP + nt * 8 + 2 * c] = acc[nt][0];
+    pw[g * NP + nt * 8 + 2 * c + 1] = acc[nt][1];
+    pw[(g + 8) * NP + nt * 8 + 2 * c] = acc[nt][2];
+    pw[(g + 8) * NP + nt * 8 + 2 * c + 1] = acc[nt][3];
+  }
+  named_sync(2, kRout * 32);
+  float* gb = s.gates + b * kTileMax * NP;
+  const int rtid = rw * 32 + lane;
+  if (rtid < rows) s.tok[b * kTileMax + rtid] = __ldg(ids + t0 + rtid);
+  constexpr int RPW = 32 / NP;
+  const int sub = lane / NP, jl = lane % NP;
+  for (int rb = rw * RPW; rb < rows; rb += kRout * RPW) {
+    const int r = rb + sub;
+    const bool act = r < rows;
+    float z = 0.f;
+    if (act) {
+#pragma unroll
+      for (int q = 0; q < kRout; ++q) z += s.part[(q * kTileMax + r) * NP + jl];
+    }
+    const bool valid = act && jl < N;
+    float m = valid ? z : -INFINITY;
+#pragma unroll
+    for (int off = NP / 2; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    const float e = valid ? expf(z - m) : 0.f;
+    float sum = e;
+#pragma unroll
+    for (int off = NP / 2; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    if (act) gb[r * NP + jl] = valid ? e / sum : 0.f;
+  }
+  named_sync(2, kRout * 32);  // gates, tok written; part free for the next tile
+}
+
+template <int NT, bool kExactN>
+__global__ void __launch_bounds__(kTmaThreads, 1)
+    combine_tma_kernel(const CombineArgs p, int n_slots, int slot_bytes) {
+  constexpr int NP = 8 * NT;
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  const TmaSmem s = tma_carve<NP>(smem_raw, p.D, n_slots, slot_bytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint16_t* wr = static_cast<const uint16_t*>(p.Wr);
+  const int ldw = p.D + 8;
+  for (int i = threadIdx.x; i < p.D * NP; i += kTmaThreads) {
+    const int d = i / NP, j = i - d * NP;
+    s.wrt[j * ldw + d] = j < p.N ? wr[(int64_t)d * p.N + j] : (uint16_t)0;
+  }
+  if (threadIdx.x == 0) {
+    for (int q = 0; q < n_slots; ++q) {
+      mbar_init(&s.full[q], 1);
+      mbar_init(&s.empty[q], kCons);
+    }
+    for (int q = 0; q < 2; ++q) {
+      mbar_init(&s.gfull[q], 1);
+      mbar_init(&s.gempty[q], kCons);
+    }
+    *s.abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  volatile int* abort = s.abort;
+  const uint16_t* lut = static_cast<const uint16_t*>(p.table);
+  const uint32_t row_bytes = (uint32_t)p.N * (uint32_t)p.D * 2u;
+
+  if (warp == kProducerWarp) {
+    // ---------------- producer: bulk copies of row blocks ----------------
+    uint32_t it = 0;
+    bool ok = true;
+    int64_t tile = blockIdx.x;
+    int next_id = (tile < p.n_tiles && lane < p.TT && tile * p.TT + lane < p.T) ? __ldg(p.ids + tile * p.TT + lane) : -1;
+    for (; ok && tile < p.n_tiles; tile += gridDim.x) {
+      const int64_t t0 = tile * p.TT;
+      const int rows = (int)(p.T - t0 < p.TT ? p.T - t0 : p.TT);
+      const int my_id = next_id;
+      const int64_t nt0 = (tile + gridDim.x) * p.TT;  // prefetch the next tile's ids
+      next_id = (tile + gridDim.x < p.n_tiles && lane < p.TT && nt0 + lane < p.T) ? __ldg(p.ids + nt0 + lane) : -1;
+      for (int r = 0; r < rows; ++r, ++it) {
+        const int id = __shfl_sync(0xffffffffu, my_id, r);
+        if (lane == 0) {
+          const uint32_t q = it % n_slots, ph = (it / n_slots) & 1u;
+          if (!mbar_wait(&s.empty[q], ph ^ 1u, abort, p.err)) {
+            ok = false;
+          } else if (id >= 0 && (int64_t)id < p.V) {
+            mbar_expect_tx(&s.full[q], row_bytes);
+            bulk_g2s(s.ring + (size_t)q * slot_bytes, lut + (int64_t)id * p.N * p.D, row_bytes, &s.full[q]);
+          } else {
+            mbar_arrive(&s.full[q]);  // nothing to copy: the consumers write a NaN row
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+      }
+    }
+    if (lane == 0) {  // the last copies must have landed before the CTA exits
+      const uint32_t first = it > (uint32_t)n_slots ? it - n_slots : 0u;
+      for (uint32_t i = first; i < it; ++i) mbar_drain(&s.full[i % n_slots], (i / n_slots) & 1u);
+    }
+    __syncwarp();
+  } else if (warp >= kCons) {
+    // ---------------- router warps ----------------
+    uint32_t tl = 0;
+    for (int64_t tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++tl) {
+      const int b = tl & 1;
+      const uint32_t ph = (tl >> 1) & 1u;
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(&s.gempty[b], ph ^ 1u, abort, p.err);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      // all router warps agree (a barrier among them only) before going on
+      if (!named_sync_and(3, kRout * 32, ok)) break;
+      const int64_t t0 = tile * p.TT;
+      const int rows = (int)(p.T - t0 < p.TT ? p.T - t0 : p.TT);
+      router_tile_rw<NT>(s, b, p.ids, static_cast<const uint16_t*>(p.h), t0, rows, p.N, p.D);
+      if (warp == kCons && lane == 0) mbar_arrive(&s.gfull[b]);
+    }
+  } else {
+    // ---------------- consumer warps ----------------
+    const int DV = p.D >> 3;
+    uint32_t it = 0, tl = 0;
+    bool ok = true;
+    for (int64_t tile = blockIdx.x; ok && tile < p.n_tiles; tile += gridDim.x, ++tl) {
+      const int b = tl & 1;
+      const uint32_t gph = (tl >> 1) & 1u;
+      if (lane == 0) ok = mbar_wait(&s.gfull[b], gph, abort, p.err);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      const int64_t t0 = tile * p.TT;
+      const int rows = (int)(p.T - t0 < p.TT ? p.T - t0 : p.TT);
+      const float* gbuf = s.gates + b * kTileMax * NP;
+      for (int r = 0; r < rows; ++r, ++it) {
+        const uint32_t q = it % n_slots, ph = (it / n_slots) & 1u;
+        if (lane == 0) ok = mbar_wait(&s.full[q], ph, abort, p.err);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+        const int id = s.tok[b * kTileMax + r];
+        const bool valid = id >= 0 && (int64_t)id < p.V;
+        float g[NP];
+        load_gates(gbuf + r * NP, g, NP);
+        const uint8_t* slot = s.ring + (size_t)q * slot_bytes;
+        for (int v = threadIdx.x; v < DV; v += kCons * 32) {
+          float* o = p.out + (t0 + r) * (int64_t)p.D + v * 8;
+          if (!valid) {
+            if (v == 0) atomicOr(p.err, kErrIndex);
+            store_nan(o, 8);
+            continue;
+          }
+          const uint4* src = reinterpret_cast<const uint4*>(slot) + v;
+          float a[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) a[i] = 0.f;
+#pragma unroll
+          for (int j = 0; j < NP; ++j) {
+            if (kExactN || j < p.N) {
+              const uint4 x = src[(int64_t)j * DV];
+              const float gj = g[j];
+              a[0] = fmaf(gj, bf16_lo(x.x), a[0]);
+              a[1] = fmaf(gj, bf16_hi(x.x), a[1]);
+              a[2] = fmaf(gj, bf16_lo(x.y), a[2]);
+              a[3] = fmaf(gj, bf16_hi(x.y), a[3]);
+              a[4] = fmaf(gj, bf16_lo(x.z), a[4]);
+              a[5] = fmaf(gj, bf16_hi(x.z), a[5]);
+              a[6] = fmaf(gj, bf16_lo(x.w), a[6]);
+              a[7] = fmaf(gj, bf16_hi(x.w), a[7]);
+            }
+          }
+          __stcs(reinterpret_cast<float4*>(o), make_float4(a[0], a[1], a[2], a[3]));
+          __stcs(reinterpret_cast<float4*>(o + 4), make_float4(a[4], a[5], a[6], a[7]));
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.empty[q]);
+      }
+      __syncwarp();
+      if (ok && lane == 0) mbar_arrive(&s.gempty[b]);
+    }
+  }
+  __syncthreads();
+}
+
+
 template <bool kBf16Router, int NT, int kTable, bool kExactN>
 __global__ void __launch_bounds__(kThreads, 2) combine_kernel(const CombineArgs p) {
   constexpr int NP = 8 * NT;
@@ -518,6 +834,40 @@ mole_status launch_one(CombineArgs p, cudaStream_t stream) {
   return cuda_status(cudaGetLastError());
 }
 
+template <int NT, bool kExactN>
+mole_status launch_tma(CombineArgs p, cudaStream_t stream) {
+  constexpr int NP = 8 * NT;
+  const int64_t row_bytes = (int64_t)p.N * p.D * 2;
+  const int slot_bytes = (int)((row_bytes + 127) / 128 * 128);
+  int n_slots = (int)std::min<int64_t>(8, kRingBudget / slot_bytes);
+  size_t smem = 0;
+  while (n_slots >= 2 && (smem = tma_smem_bytes<NP>(p.D, n_slots, slot_bytes)) > 227 * 1024) --n_slots;
+  if (n_slots < 2) return MOLE_ERR_UNSUPPORTED;
+  auto kern = combine_tma_kernel<NT, kExactN>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return MOLE_ERR_CUDA;
+  const int n_sm = num_sms();
+  if (n_sm <= 0) return MOLE_ERR_NO_DEVICE;
+  p.TT = choose_tile(p.T, n_sm);
+  p.n_tiles = (p.T + p.TT - 1) / p.TT;
+  const int64_t grid = std::min<int64_t>(p.n_tiles, n_sm);
+  kern<<<(unsigned)grid, kTmaThreads, smem, stream>>>(p, n_slots, slot_bytes);
+  return cuda_status(cudaGetLastError());
+}
+
+// bf16 table: the TMA-staged kernel when a ring of >= 2 row blocks fits in
+// shared memory, else the register-gather kernel.
+mole_status launch_bf16_table(const CombineArgs& p, cudaStream_t stream) {
+  mole_status st = MOLE_ERR_UNSUPPORTED;
+  if (p.N == 16) st = launch_tma<2, true>(p, stream);
+  else if (p.N == 8) st = launch_tma<1, true>(p, stream);
+  else if (p.N < 8) st = launch_tma<1, false>(p, stream);
+  else if (p.N < 16) st = launch_tma<2, false>(p, stream);
+  else if (p.N == 32) st = launch_tma<4, true>(p, stream);
+  else st = launch_tma<4, false>(p, stream);
+  return st;
+}
+
 template <bool kBf16Router, int kTable>
 mole_status launch_combine(const CombineArgs& p, cudaStream_t stream) {
   if (p.N == 16) return launch_one<kBf16Router, 2, kTable, true>(p, stream);
@@ -550,7 +900,11 @@ mole_status combine_dispatch(const int32_t* ids, int64_t T, const void* h, const
   if (!p.err) return MOLE_ERR_CUDA;
   if (table_kind == kTableNf3)
     return bf16_inputs ? launch_combine<true, kTableNf3>(p, stream) : launch_combine<false, kTableNf3>(p, stream);
-  if (table_kind == kTableBf16) return launch_combine<true, kTableBf16>(p, stream);
+  if (table_kind == kTableBf16) {
+    const mole_status st = launch_bf16_table(p, stream);
+    if (st != MOLE_ERR_UNSUPPORTED) return st;
+    return launch_combine<true, kTableBf16>(p, stream);
+  }
   return launch_combine<false, kTableF32>(p, stream);
 }
 

@@ -81,6 +81,24 @@ __device__ __forceinline__ float gelu_as7126(float u) {
   return u * (u >= 0.f ? 1.0f - half_erfc : half_erfc);
 }
 
+// Expert FFN activation with the kind fixed at compile time (no branch in
+// per-element loops).
+template <int ACT>
+__device__ __forceinline__ float act_t(float x) {
+  if constexpr (ACT == MOLE_ACT_GELU_ERF) {
+    return gelu_as7126(x);
+  } else if constexpr (ACT == MOLE_ACT_GELU_TANH) {
+    const float u = 0.7978845608028654f * fmaf(0.044715f * x, x * x, x);
+    return 0.5f * x * (1.f + tanhf(u));
+  } else if constexpr (ACT == MOLE_ACT_RELU) {
+    return x > 0.f ? x : 0.f;
+  } else if constexpr (ACT == MOLE_ACT_SILU) {
+    return __fdividef(x, 1.f + __expf(-x));
+  } else {
+    return x;
+  }
+}
+
 // Expert FFN activation (reading of the page's "GELU FFN": exact GELU x*Phi(x)).
 __device__ __forceinline__ float apply_act(int act, float x) {
   switch (act) {
@@ -116,5 +134,73 @@ mole_status nf3_quantize_launch(const void* lut, int64_t V, int N, int64_t D, ui
 void nf3_tables(uint16_t levels[8], float mid[7]);
 mole_status gather_plan_launch(const int32_t* ids, int64_t T, int64_t V, int32_t* uniq,
                                int32_t* n_uniq, int32_t* slot, cudaStream_t stream);
+
+}  // namespace mole
+
+namespace mole {
+
+// ---- mbarrier helpers with bounded waits (shared by the TMA pipelines) ----
+constexpr uint64_t kWaitLimitNs = 4000000000ull;  // a wait gives up after 4 s
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_test(uint64_t* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits for the phase with the given parity to complete.  Gives up (returns
+// false) when *abort is set by another role or after kWaitLimitNs, in which
+// case it sets *abort and the device error word.
+static __device__ __noinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort, unsigned* err) {
+  if (mbar_test(b, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_test(b, parity)) return true;
+    if ((i & 63) == 0) {
+      if (*abort) return false;
+      if (globaltimer() - t0 > kWaitLimitNs) {
+        *abort = 1;
+        atomicOr(err, kErrTimeout);
+        return false;
+      }
+    }
+  }
+}
+
+// Bounded wait used while draining after an abort (ignores the abort flag).
+static __device__ __noinline__ void mbar_drain(uint64_t* b, uint32_t parity) {
+  const uint64_t t0 = globaltimer();
+  while (!mbar_test(b, parity))
+    if (globaltimer() - t0 > kWaitLimitNs) return;
+}
 
 }  // namespace mole

@@ -40,6 +40,8 @@ def _run(mole, ids, h, Wr, lut):
     (256, 96, 24, 40, "uniform"),
     (128, 48, 32, 33, "uniform"),
     (50304, 2048, 16, 300, "zipf"),
+    (64, 2048, 32, 40, "uniform"),   # row block of 128 KB: register-gather kernel
+    (96, 1024, 24, 77, "zipf"),      # 48 KB row blocks, padded expert count
 ])
 def test_combine_bf16_matches_oracle(mole, oracle_mod, V, D, N, T, kind):
     ids, h, Wr, lut = _layer(100 + D + N + T, V, D, N, T, ids_kind=kind)
