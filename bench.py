@@ -62,6 +62,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--build-only", action="store_true",
                     help="run only the table-build leg (for profiling the tensor-core kernels)")
+    ap.add_argument("--build-experts", type=int, default=None,
+                    help="experts in the build leg (default: the model's 16); fewer only for profiling runs")
     return ap.parse_args()
 
 
@@ -281,7 +283,7 @@ def main():
     if args.build_only:
         hbm_peak, bf16_peak, bf16_sust, peak_kind = measured_peaks()
         res = build_leg(mole, dev, stream, bf16_peak, bf16_sust, peak_kind, reps=max(1, args.steps),
-                        warmup=max(1, args.warmup))
+                        warmup=max(1, args.warmup), experts=args.build_experts)
         if rank == 0:
             print(json.dumps({"build": res}), flush=True)
         if world > 1:
@@ -519,10 +521,10 @@ def nf3_leg(mole, luts, routers, id_pool, h_pool, uniq_counts, dev, stream, W, K
             "workload": f"1B-shaped NF3 table (codes + fp16 scale per 64), T={T}, same ids/h as the main case"}
 
 
-def build_leg(mole, dev, stream, bf16_peak, bf16_sust, peak_kind, reps=3, warmup=1):
+def build_leg(mole, dev, stream, bf16_peak, bf16_sust, peak_kind, reps=3, warmup=1, experts=None):
     import torch
     shape = inputs.SHAPES["410m"]
-    V, D, N, Dr = shape.V, shape.D, shape.N, shape.Dr
+    V, D, N, Dr = shape.V, shape.D, shape.N if experts is None else max(1, experts), shape.Dr
     g = torch.Generator(device=dev)
     g.manual_seed(shape.seed)
     E = (torch.randn((V, D), generator=g, device=dev) * 0.02).to(torch.bfloat16)
