@@ -357,13 +357,14 @@ def main():
     # ---- end to end through the C ABI with host buffers ----
     e2e = None if args.no_e2e else e2e_leg(mole, id_pool, h_pool, routers, luts, out, dev, stream, world, W, K, T, L)
 
-    # ---- roofline of the combine kernel ----    hbm_peak, bf16_peak, bf16_sust, peak_kind = measured_peaks()
+    # ---- roofline of the combine kernel ----
+    hbm_peak, bf16_peak, bf16_sust, peak_kind = measured_peaks()
     alg_bytes = combine_bytes(U_avg, T, D, N)
     achieved_gbs = alg_bytes / (max_kern_ms / 1e3) / 1e9
     traffic, traffic_note = profiled_traffic()
     roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved_gbs / hbm_peak, "traffic": traffic,
-                "kernel": "combine_kernel<bf16 router, 16 experts, bf16 table>",
+                "kernel": "combine_tma_kernel<16 experts> (bulk-copy ring, router warps, consumer warps)",
                 "algorithmic_bytes_per_launch": alg_bytes, "unique_rows_per_launch": U_avg,
                 "avg_launch_us": max_kern_ms * 1e3, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
                 "frac_of_8TBs": achieved_gbs / 8000.0, "traffic_source": traffic_note}
