@@ -17,8 +17,9 @@
  *     out of time) set a per-device error word; `mole_check` reads and clears
  *     it.  A token with a bad id gets a NaN output row.
  *   - The library allocates no device memory of its own apart from static
- *     per-device variables (the error word).  Scratch memory, where an entry
- *     point needs it, is passed in by the caller.
+ *     per-device variables (the error word, and the fixed scratch array of
+ *     mole_build_lut_noalloc).  Scratch memory, where the other entry points
+ *     need it, is passed in by the caller.
  *   - bf16 tensors are IEEE bfloat16 bit patterns; fp16 scales are IEEE binary16.
  */
 #ifndef MOLE_H_
@@ -88,6 +89,30 @@ size_t mole_build_lut_workspace(int64_t V, int64_t D, int32_t N, int64_t Dr, mol
 mole_status mole_build_lut(const void* embed, const void* W1, const void* W2, int64_t V,
                            int64_t D, int32_t N, int64_t Dr, mole_act act, mole_dtype dt,
                            void* lut, void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * mole_build_lut without caller-provided scratch, for callers that cannot
+ * allocate device memory when they build a table: code running while a stream
+ * is captured into a CUDA graph (an allocation there breaks the capture),
+ * serving loops that allow no device allocation after start-up, and plugin
+ * hosts that give plugins no allocator.  The MoLE page has no counterpart; it
+ * is an interface convenience.
+ *
+ * Same arguments, layouts and results as mole_build_lut, minus the workspace:
+ * the hidden activations of each group of experts live in a fixed 16 MiB array
+ * in this library's device memory (held by every GPU that loads the library
+ * until the process exits).  One expert's activations, V * Dr * (2 bytes for
+ * bf16, 4 for fp32), must fit in it, else MOLE_ERR_WORKSPACE and nothing is
+ * launched.  The first call on each device looks the array's device address
+ * up (cudaGetSymbolAddress); make that first call before any stream capture.
+ * Every call uses the same array: calls that overlap on the GPU (other
+ * streams, other threads) race on it; the array needs no clearing between
+ * calls (each expert's activations are written before they are read).  No
+ * device memory is allocated or freed.
+ */
+mole_status mole_build_lut_noalloc(const void* embed, const void* W1, const void* W2, int64_t V,
+                                   int64_t D, int32_t N, int64_t Dr, mole_act act, mole_dtype dt,
+                                   void* lut, cudaStream_t stream);
 
 /*
  * ---- Lookup-combine (MoLE page, 训练阶段 + 推理阶段) ----

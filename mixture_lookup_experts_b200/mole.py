@@ -36,6 +36,7 @@ SIGNATURES = {
     "mole_version": ([], _I),
     "mole_build_lut_workspace": ([_I64, _I64, _I32, _I64, _I, _I32], _SZ),
     "mole_build_lut": ([_P, _P, _P, _I64, _I64, _I32, _I64, _I, _I, _P, _P, _SZ, _P], _I),
+    "mole_build_lut_noalloc": ([_P, _P, _P, _I64, _I64, _I32, _I64, _I, _I, _P, _P], _I),
     "mole_lookup_combine": ([_P, _I64, _P, _P, _P, _I64, _I32, _I64, _I, _P, _P], _I),
     "mole_quantize_lut_nf3": ([_P, _I64, _I32, _I64, _P, _P, _P], _I),
     "mole_lookup_combine_nf3": ([_P, _I64, _P, _P, _P, _P, _I64, _I32, _I64, _I, _P, _P], _I),
@@ -120,6 +121,22 @@ def mole_build_lut(embed: torch.Tensor, W1: torch.Tensor, W2: torch.Tensor, act:
     ws_bytes = workspace.numel() * workspace.element_size()
     _ok(lib.mole_build_lut(_ptr(embed), _ptr(W1), _ptr(W2), V, D, N, Dr, ACT[act], dt, _ptr(lut),
                            _ptr(workspace), ws_bytes, _stream(stream)), "mole_build_lut")
+    return lut
+
+
+def mole_build_lut_noalloc(embed: torch.Tensor, W1: torch.Tensor, W2: torch.Tensor, act: str = "gelu",
+                           lut: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """mole_build_lut with the scratch in the library's fixed device array
+    (no allocation inside the call; see mole.h for the size limit)."""
+    _contig(embed, W1, W2, lut)
+    V, D = embed.shape
+    N, D2, Dr = W1.shape
+    if D2 != D or tuple(W2.shape) != (N, Dr, D):
+        raise ValueError("shape mismatch: embed [V,D], W1 [N,D,Dr], W2 [N,Dr,D]")
+    if lut is None:
+        lut = torch.empty((V, N, D), dtype=embed.dtype, device=embed.device)
+    _ok(lib.mole_build_lut_noalloc(_ptr(embed), _ptr(W1), _ptr(W2), V, D, N, Dr, ACT[act], _dt(embed), _ptr(lut),
+                                   _stream(stream)), "mole_build_lut_noalloc")
     return lut
 
 
