@@ -95,6 +95,58 @@ __device__ __forceinline__ Smem carve(uint8_t* base, int D) {
   return s;
 }
 
+// Stage Wr^T in shared memory: wrt[j][d] = Wr[d][j] (bf16), zero rows j >= N.
+// Loads are issued in batches of 8 per thread before their stores so their
+// latencies overlap (a dependent load per element would serialise them).
+template <int NP, int kNThreads>
+__device__ __forceinline__ void stage_wrt(uint16_t* wrt, const uint16_t* __restrict__ wr, int N, int D) {
+  const int ldw = D + 8;
+  if (N == NP && (reinterpret_cast<uintptr_t>(wr) & 15u) == 0) {
+    // 16-byte loads of 8 experts of one row d, 16 per thread in flight
+    const int total8 = D * NP / 8;
+    for (int base = threadIdx.x; base < total8; base += kNThreads * 16) {
+      uint4 v[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int i = base + u * kNThreads;
+        if (i < total8) v[u] = __ldg(reinterpret_cast<const uint4*>(wr) + i);
+      }
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int i = base + u * kNThreads;
+        if (i < total8) {
+          const int d = (i * 8) / NP, j0 = (i * 8) % NP;
+          const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            wrt[(j0 + 2 * e) * ldw + d] = (uint16_t)(w[e] & 0xffffu);
+            wrt[(j0 + 2 * e + 1) * ldw + d] = (uint16_t)(w[e] >> 16);
+          }
+        }
+      }
+    }
+    return;
+  }
+  const int total = D * NP;
+  for (int base = threadIdx.x; base < total; base += kNThreads * 8) {
+    uint16_t v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = base + u * kNThreads;
+      const int d = i / NP, j = i - d * NP;
+      v[u] = (i < total && j < N) ? __ldg(wr + (int64_t)d * N + j) : (uint16_t)0;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = base + u * kNThreads;
+      if (i < total) {
+        const int d = i / NP, j = i - d * NP;
+        wrt[j * ldw + d] = v[u];
+      }
+    }
+  }
+}
+
 // Router + softmax for one tile of `rows` tokens starting at t0.  On return
 // (after a __syncthreads) s.gates[r][j] and s.tok_id[r] are valid for r < rows.
 template <bool kBf16Router, int NT>
@@ -104,7 +156,7 @@ __device__ __forceinline__ void router_tile(const Smem& s, const int32_t* __rest
   constexpr int NP = 8 * NT;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (kBf16Router) {
-    constexpr int KB = 8;  // k-steps whose A fragments are fetched before their MMAs
+    constexpr int KB = 16;  // k-steps whose A fragments are fetched before their MMAs
     const uint16_t* h = static_cast<const uint16_t*>(h_);
     const int g = lane >> 2, c = lane & 3, ldw = D + 8;
     float acc[NT][4];
@@ -448,27 +500,25 @@ struct CombineArgs {
 };
 
 // ---------------------------------------------------------------------------
-// TMA-staged gather for bf16 tables.  Three roles per persistent CTA (one per
-// SM), pipelined through shared memory:
-//   producer warp   one thread copies each token's whole row block
-//                   LUT[id, 0..N-1, :] (N*D*2 contiguous bytes) into a ring of
-//                   slots with cp.async.bulk (completion on the slot's mbarrier),
-//                   running ahead of the consumers by the ring depth; ids come
-//                   from a per-tile prefetch held in the warp's registers;
-//   router warps    (4) compute the next tile's logits on the tensor cores
-//                   (mma.sync, D split over the 4 warps) and its softmax, into
-//                   one of two gate buffers;
-//   consumer warps  (8) combine each token from its slot (16-byte shared-memory
-//                   reads, fp32 FMAs) and store fp32 outputs.
-// The bulk copies keep up to ring-depth x 64 KB in flight per SM without
-// occupying load registers or per-thread request slots, and the router's
-// latency overlaps the previous tile's combine.
+// Two-kernel path for prefill-sized batches (bf16 inputs; bf16 or NF3 table).
+//
+// 1. router_gates_kernel: persistent CTAs (Wr^T staged once in shared memory)
+//    compute the gates of 16-token tiles on the tensor cores (router_tile) and
+//    write each token's N gates into the first N floats of that token's own
+//    output row -- memory the caller provides and the second kernel overwrites.
+// 2. gather_kernel: per CTA one producer thread streams each token's whole row
+//    block (N*D*2 contiguous bytes; for NF3 the code block and the scale
+//    block) and its gate vector into a ring of shared-memory slots with
+//    cp.async.bulk, completion counted on the slot's mbarrier; consumer warps
+//    combine from shared memory (16-byte reads, fp32 FMAs) and store fp32
+//    outputs.  Bulk copies keep ring-depth x 64 KB in flight per SM without
+//    registers or per-thread request slots, so the gather streams at the DRAM
+//    rate, and the router's latency no longer sits inside the gather.
 // ---------------------------------------------------------------------------
-constexpr int kCons = 8;                                  // consumer warps
-constexpr int kRout = 4;                                  // router warps
-constexpr int kTmaThreads = (kCons + kRout + 1) * 32;     // + producer warp
-constexpr int kProducerWarp = kCons + kRout;
-constexpr int kRingBudget = 160 * 1024;                   // bytes of row slots
+constexpr int kGatherCons = 16;                           // consumer warps
+constexpr int kGatherThreads = (kGatherCons + 1) * 32;    // + producer warp
+constexpr int kGatherProducer = kGatherCons;
+constexpr int kRingBudget = 200 * 1024;                   // bytes of row slots
 
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(
@@ -478,304 +528,304 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
-__device__ __forceinline__ void named_sync(int id, int threads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
-}
-
-// Barrier over `threads` threads that also returns the AND of `pred`.
-__device__ __forceinline__ bool named_sync_and(int id, int threads, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, %2, %3, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"(pred ? 1u : 0u), "r"(id), "r"(threads)
-      : "memory");
-  return r != 0;
-}
-
-struct TmaSmem {
-  uint16_t* wrt;    // [NP][D + 8] bf16 Wr^T
-  float* part;      // [kRout][kTileMax][NP]
-  float* gates;     // [2][kTileMax][NP]
-  int* tok;         // [2][kTileMax]
-  uint8_t* ring;    // [n_slots][slot_bytes]
-  uint64_t* full;   // [n_slots]
-  uint64_t* empty;  // [n_slots]
-  uint64_t* gfull;  // [2]
-  uint64_t* gempty; // [2]
-  int* abort;
-};
-
-template <int NP>
-__host__ __device__ constexpr size_t tma_fixed_bytes(int D) {
-  return (size_t)NP * (D + 8) * 2 + (size_t)kRout * kTileMax * NP * 4 + 2 * (size_t)kTileMax * NP * 4 +
-         2 * (size_t)kTileMax * 4;
-}
-
-template <int NP>
-__host__ __device__ constexpr size_t tma_smem_bytes(int D, int n_slots, int slot_bytes) {
-  return ((tma_fixed_bytes<NP>(D) + 127) / 128) * 128 + (size_t)n_slots * slot_bytes + (2 * (size_t)n_slots + 4) * 8 +
-         16;
-}
-
-template <int NP>
-__device__ __forceinline__ TmaSmem tma_carve(uint8_t* base, int D, int n_slots, int slot_bytes) {
-  TmaSmem s;
-  size_t off = 0;
-  s.wrt = reinterpret_cast<uint16_t*>(base);
-  off += (size_t)NP * (D + 8) * 2;
-  s.part = reinterpret_cast<float*>(base + off);
-  off += (size_t)kRout * kTileMax * NP * 4;
-  s.gates = reinterpret_cast<float*>(base + off);
-  off += 2 * (size_t)kTileMax * NP * 4;
-  s.tok = reinterpret_cast<int*>(base + off);
-  off += 2 * (size_t)kTileMax * 4;
-  off = (off + 127) / 128 * 128;
-  s.ring = base + off;
-  off += (size_t)n_slots * slot_bytes;
-  s.full = reinterpret_cast<uint64_t*>(base + off);
-  s.empty = s.full + n_slots;
-  s.gfull = s.empty + n_slots;
-  s.gempty = s.gfull + 2;
-  s.abort = reinterpret_cast<int*>(s.gempty + 2);
-  return s;
-}
-
-// Router of one tile by the kRout router warps (named barrier 2): logits on
-// the tensor cores, D split over the warps, then softmax into gates[b].
-template <int NT>
-__device__ __forceinline__ void router_tile_rw(const TmaSmem& s, int b, const int32_t* __restrict__ ids,
-                                               const uint16_t* __restrict__ h, int64_t t0, int rows, int N,
-                                               int D) {
-  constexpr int NP = 8 * NT;
-  constexpr int KB = 8;
-  const int rw = (threadIdx.x >> 5) - kCons;  // router warp index 0..kRout-1
-  const int lane = threadIdx.x & 31;
-  const int g = lane >> 2, c = lane & 3, ldw = D + 8;
-  float acc[NT][4];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-  const bool ok0 = g < rows, ok1 = g + 8 < rows;
-  const uint16_t* h0 = h + (t0 + (ok0 ? g : 0)) * (int64_t)D + 4 * c;
-  const uint16_t* h1 = h + (t0 + (ok1 ? g + 8 : 0)) * (int64_t)D + 4 * c;
-  const uint16_t* w = s.wrt + g * ldw + 4 * c;
-  const int ksteps = D >> 4;
-  for (int kb = rw; kb < ksteps; kb += kRout * KB) {
-    uint2 a0[KB], a1[KB];
-#pragma unroll
-    for (int i = 0; i < KB; ++i) {
-      const int ks = kb + i * kRout;
-      const bool in = ks < ksteps;
-      a0[i] = (in && ok0) ? __ldg(reinterpret_cast<const uint2*>(h0 + (ks << 4))) : make_uint2(0u, 0u);
-      a1[i] = (in && ok1) ? __ldg(reinterpret_cast<const uint2*>(h1 + (ks << 4))) : make_uint2(0u, 0u);
-    }
-#pragma unroll
-    for (int i = 0; i < KB; ++i) {
-      const int ks = kb + i * kRout;
-      if (ks < ksteps) {
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          const uint2 bb = *reinterpret_cast<const uint2*>(w + nt * 8 * ldw + (ks << 4));
-          mma_16816(acc[nt], a0[i].x, a1[i].x, a0[i].y, a1[i].y, bb.x, bb.y);
+// Lane 0 of the warp waits (bounded); the result is broadcast to the warp.
+__device__ __forceinline__ bool warp_wait(uint64_t* b, uint32_t parity, volatile int* abort, unsigned* err) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0) {
+    if (!mbar_test(b, parity)) {
+      const uint64_t t0 = globaltimer();
+      for (;;) {
+        if (mbar_test(b, parity)) break;
+        if (*abort) { ok = false; break; }
+        if (globaltimer() - t0 > kWaitLimitNs) {
+          *abort = 1;
+          atomicOr(err, kErrTimeout);
+          ok = false;
+          break;
         }
       }
     }
   }
-  float* pw = s.part + rw * kTileMax * NP;
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    pw[g * NP + nt * 8 + 2 * c] = acc[nt][0];
-    pw[g * NP + nt * 8 + 2 * c + 1] = acc[nt][1];
-    pw[(g + 8) * NP + nt * 8 + 2 * c] = acc[nt][2];
-    pw[(g + 8) * NP + nt * 8 + 2 * c + 1] = acc[nt][3];
-  }
-  named_sync(2, kRout * 32);
-  float* gb = s.gates + b * kTileMax * NP;
-  const int rtid = rw * 32 + lane;
-  if (rtid < rows) s.tok[b * kTileMax + rtid] = __ldg(ids + t0 + rtid);
-  constexpr int RPW = 32 / NP;
-  const int sub = lane / NP, jl = lane % NP;
-  for (int rb = rw * RPW; rb < rows; rb += kRout * RPW) {
-    const int r = rb + sub;
-    const bool act = r < rows;
-    float z = 0.f;
-    if (act) {
-#pragma unroll
-      for (int q = 0; q < kRout; ++q) z += s.part[(q * kTileMax + r) * NP + jl];
-    }
-    const bool valid = act && jl < N;
-    float m = valid ? z : -INFINITY;
-#pragma unroll
-    for (int off = NP / 2; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-    const float e = valid ? expf(z - m) : 0.f;
-    float sum = e;
-#pragma unroll
-    for (int off = NP / 2; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-    if (act) gb[r * NP + jl] = valid ? e / sum : 0.f;
-  }
-  named_sync(2, kRout * 32);  // gates, tok written; part free for the next tile
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
-template <int NT, bool kExactN>
-__global__ void __launch_bounds__(kTmaThreads, 1)
-    combine_tma_kernel(const CombineArgs p, int n_slots, int slot_bytes) {
+// Slot layout: [0, row_bytes) table row block, [scales_off, +scale_bytes)
+// NF3 scales, [gates_off, +NP*4) the token's gates.
+struct GatherLayout {
+  int n_slots, slot_bytes, scales_off, gates_off;
+};
+
+template <int NT>
+__global__ void __launch_bounds__(kThreads, 2) router_gates_kernel(const CombineArgs p) {
   constexpr int NP = 8 * NT;
   extern __shared__ __align__(128) uint8_t smem_raw[];
-  const TmaSmem s = tma_carve<NP>(smem_raw, p.D, n_slots, slot_bytes);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint16_t* wr = static_cast<const uint16_t*>(p.Wr);
-  const int ldw = p.D + 8;
-  for (int i = threadIdx.x; i < p.D * NP; i += kTmaThreads) {
-    const int d = i / NP, j = i - d * NP;
-    s.wrt[j * ldw + d] = j < p.N ? wr[(int64_t)d * p.N + j] : (uint16_t)0;
+  const Smem s = carve<true, NP>(smem_raw, p.D);
+  stage_wrt<NP, kThreads>(s.wrt, static_cast<const uint16_t*>(p.Wr), p.N, p.D);
+  __syncthreads();
+  for (int64_t tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x) {
+    const int64_t t0 = tile * p.TT;
+    const int rows = (int)(p.T - t0 < p.TT ? p.T - t0 : p.TT);
+    router_tile<true, NT>(s, p.ids, p.h, p.Wr, t0, rows, p.N, p.D);
+    for (int i = threadIdx.x; i < rows * NP; i += kThreads) {
+      const int r = i / NP, j = i - r * NP;
+      p.out[(t0 + r) * (int64_t)p.D + j] = s.gates[i];
+    }
+    // s.gates is rewritten only after the next tile's first barrier
   }
+}
+
+template <int NT, bool kExactN, int kTable, int kChunks>
+__global__ void __launch_bounds__(kGatherThreads, 1) gather_kernel(const CombineArgs p, const GatherLayout L) {
+  constexpr int NP = 8 * NT;
+  constexpr int JC = NP / kChunks;  // expert rows per chunk (kChunks > 1 only with N == NP)
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  uint8_t* ring = smem_raw;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw + (size_t)L.n_slots * L.slot_bytes);
+  uint64_t* empty = full + L.n_slots;
+  int* slot_id = reinterpret_cast<int*>(empty + L.n_slots);
+  int* abort_flag = slot_id + L.n_slots;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int q = 0; q < n_slots; ++q) {
-      mbar_init(&s.full[q], 1);
-      mbar_init(&s.empty[q], kCons);
+    for (int q = 0; q < L.n_slots; ++q) {
+      mbar_init(&full[q], 1);
+      mbar_init(&empty[q], kGatherCons);
     }
-    for (int q = 0; q < 2; ++q) {
-      mbar_init(&s.gfull[q], 1);
-      mbar_init(&s.gempty[q], kCons);
-    }
-    *s.abort = 0;
+    *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
-  volatile int* abort = s.abort;
-  const uint16_t* lut = static_cast<const uint16_t*>(p.table);
-  const uint32_t row_bytes = (uint32_t)p.N * (uint32_t)p.D * 2u;
+  volatile int* abort = abort_flag;
+  const int NB = p.D >> 6;
+  // bytes of one chunk of a token's row block (bf16: JC rows of D; NF3: all
+  // code rows, then the scale rows at scales_off)
+  const uint32_t chunk_bytes = kTable == kTableBf16 ? (uint32_t)JC * (uint32_t)p.D * 2u
+                                                    : (uint32_t)p.N * (uint32_t)NB * 24u;
+  const uint32_t scale_bytes = kTable == kTableBf16 ? 0u : (uint32_t)p.N * (uint32_t)NB * 2u;
+  const uint32_t gate_bytes = NP * 4u;
+  // this CTA's tokens: t = blockIdx.x + k * gridDim.x, k = 0, 1, ...
+  const int64_t n_mine = p.T > blockIdx.x ? (p.T - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
 
-  if (warp == kProducerWarp) {
-    // ---------------- producer: bulk copies of row blocks ----------------
-    uint32_t it = 0;
+  if (warp == kGatherProducer) {
+    // ---------------- producer ----------------
+    int64_t k0 = 0;
+    int my_id = lane < n_mine ? __ldg(p.ids + blockIdx.x + (int64_t)lane * gridDim.x) : -1;
+    int next_id = 32 + lane < n_mine ? __ldg(p.ids + blockIdx.x + (int64_t)(32 + lane) * gridDim.x) : -1;
+    uint32_t q = 0, ph = 0, issued = 0;
     bool ok = true;
-    int64_t tile = blockIdx.x;
-    int next_id = (tile < p.n_tiles && lane < p.TT && tile * p.TT + lane < p.T) ? __ldg(p.ids + tile * p.TT + lane) : -1;
-    for (; ok && tile < p.n_tiles; tile += gridDim.x) {
-      const int64_t t0 = tile * p.TT;
-      const int rows = (int)(p.T - t0 < p.TT ? p.T - t0 : p.TT);
-      const int my_id = next_id;
-      const int64_t nt0 = (tile + gridDim.x) * p.TT;  // prefetch the next tile's ids
-      next_id = (tile + gridDim.x < p.n_tiles && lane < p.TT && nt0 + lane < p.T) ? __ldg(p.ids + nt0 + lane) : -1;
-      for (int r = 0; r < rows; ++r, ++it) {
-        const int id = __shfl_sync(0xffffffffu, my_id, r);
+    for (int64_t k = 0; ok && k < n_mine; ++k) {
+      if (k - k0 == 32) {  // next batch of 32 ids; prefetch the one after
+        k0 = k;
+        my_id = next_id;
+        const int64_t kn = k0 + 32 + lane;
+        next_id = kn < n_mine ? __ldg(p.ids + blockIdx.x + kn * gridDim.x) : -1;
+      }
+      const int id = __shfl_sync(0xffffffffu, my_id, (int)(k - k0));
+      const bool valid = id >= 0 && (int64_t)id < p.V;
+      const int64_t t = blockIdx.x + k * gridDim.x;
+#pragma unroll
+      for (int c = 0; c < kChunks; ++c) {
+        ok = warp_wait(&empty[q], ph ^ 1u, abort, p.err);
+        if (!ok) break;
         if (lane == 0) {
-          const uint32_t q = it % n_slots, ph = (it / n_slots) & 1u;
-          if (!mbar_wait(&s.empty[q], ph ^ 1u, abort, p.err)) {
-            ok = false;
-          } else if (id >= 0 && (int64_t)id < p.V) {
-            mbar_expect_tx(&s.full[q], row_bytes);
-            bulk_g2s(s.ring + (size_t)q * slot_bytes, lut + (int64_t)id * p.N * p.D, row_bytes, &s.full[q]);
+          uint8_t* slot = ring + (size_t)q * L.slot_bytes;
+          slot_id[q] = id;
+          if (valid) {
+            const uint32_t bytes = chunk_bytes + (c == 0 ? gate_bytes : 0u) + scale_bytes;
+            mbar_expect_tx(&full[q], bytes);
+            if (kTable == kTableBf16) {
+              bulk_g2s(slot, static_cast<const uint16_t*>(p.table) + ((int64_t)id * p.N + c * JC) * p.D, chunk_bytes,
+                       &full[q]);
+            } else {
+              bulk_g2s(slot, static_cast<const uint8_t*>(p.table) + (int64_t)id * chunk_bytes, chunk_bytes, &full[q]);
+              bulk_g2s(slot + L.scales_off, p.scales + (int64_t)id * p.N * NB, scale_bytes, &full[q]);
+            }
+            if (c == 0) bulk_g2s(slot + L.gates_off, p.out + t * p.D, gate_bytes, &full[q]);
           } else {
-            mbar_arrive(&s.full[q]);  // nothing to copy: the consumers write a NaN row
+            mbar_arrive(&full[q]);  // nothing to copy: the consumers write a NaN row
           }
         }
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        if (!ok) break;
+        ++issued;
+        if (++q == (uint32_t)L.n_slots) {
+          q = 0;
+          ph ^= 1u;
+        }
       }
     }
     if (lane == 0) {  // the last copies must have landed before the CTA exits
-      const uint32_t first = it > (uint32_t)n_slots ? it - n_slots : 0u;
-      for (uint32_t i = first; i < it; ++i) mbar_drain(&s.full[i % n_slots], (i / n_slots) & 1u);
+      for (uint32_t i = 0; i < issued && i < (uint32_t)L.n_slots; ++i) {
+        q = q == 0 ? L.n_slots - 1 : q - 1;
+        if (q == (uint32_t)L.n_slots - 1) ph ^= 1u;
+        mbar_drain(&full[q], ph);
+      }
     }
     __syncwarp();
-  } else if (warp >= kCons) {
-    // ---------------- router warps ----------------
-    uint32_t tl = 0;
-    for (int64_t tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++tl) {
-      const int b = tl & 1;
-      const uint32_t ph = (tl >> 1) & 1u;
-      bool ok = true;
-      if (lane == 0) ok = mbar_wait(&s.gempty[b], ph ^ 1u, abort, p.err);
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-      // all router warps agree (a barrier among them only) before going on
-      if (!named_sync_and(3, kRout * 32, ok)) break;
-      const int64_t t0 = tile * p.TT;
-      const int rows = (int)(p.T - t0 < p.TT ? p.T - t0 : p.TT);
-      router_tile_rw<NT>(s, b, p.ids, static_cast<const uint16_t*>(p.h), t0, rows, p.N, p.D);
-      if (warp == kCons && lane == 0) mbar_arrive(&s.gfull[b]);
-    }
   } else {
-    // ---------------- consumer warps ----------------
-    const int DV = p.D >> 3;
-    uint32_t it = 0, tl = 0;
+    // ---------------- consumers ----------------
+    // Tokens are dealt to G groups of gw warps (a token has per_tok units:
+    // 4-element (8-byte) vectors of a bf16 row, or 32-element NF3 half
+    // blocks).  Every warp waits on every slot and releases it, so slot phases
+    // stay in step; only the owning group computes.
+    const int per_tok = kTable == kTableBf16 ? (p.D >> 2) : (p.D >> 5);
+    const int wpt = (per_tok + 31) >> 5;
+    const int G = wpt >= kGatherCons ? 1 : kGatherCons / wpt;
+    const int gw = kGatherCons / G;
+    const int grp = warp / gw;
+    const int lt = threadIdx.x - grp * gw * 32;
+    const bool one_unit = kTable == kTableBf16 && per_tok <= gw * 32;
+    int gsel = 0;  // == token index % G
+    uint32_t q = 0, ph = 0;
     bool ok = true;
-    for (int64_t tile = blockIdx.x; ok && tile < p.n_tiles; tile += gridDim.x, ++tl) {
-      const int b = tl & 1;
-      const uint32_t gph = (tl >> 1) & 1u;
-      if (lane == 0) ok = mbar_wait(&s.gfull[b], gph, abort, p.err);
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-      if (!ok) break;
-      const int64_t t0 = tile * p.TT;
-      const int rows = (int)(p.T - t0 < p.TT ? p.T - t0 : p.TT);
-      const float* gbuf = s.gates + b * kTileMax * NP;
-      for (int r = 0; r < rows; ++r, ++it) {
-        const uint32_t q = it % n_slots, ph = (it / n_slots) & 1u;
-        if (lane == 0) ok = mbar_wait(&s.full[q], ph, abort, p.err);
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        if (!ok) break;
-        const int id = s.tok[b * kTileMax + r];
-        const bool valid = id >= 0 && (int64_t)id < p.V;
+    for (int64_t k = 0; ok && k < n_mine; ++k) {
+      const bool mine = gsel == grp;
+      const int64_t t = blockIdx.x + k * gridDim.x;
+      float* orow = p.out + t * p.D;
+      if (kTable == kTableBf16 && one_unit) {
+        // one 4-wide vector per thread, accumulated across the chunks
         float g[NP];
-        load_gates(gbuf + r * NP, g, NP);
-        const uint8_t* slot = s.ring + (size_t)q * slot_bytes;
-        for (int v = threadIdx.x; v < DV; v += kCons * 32) {
-          float* o = p.out + (t0 + r) * (int64_t)p.D + v * 8;
-          if (!valid) {
-            if (v == 0) atomicOr(p.err, kErrIndex);
-            store_nan(o, 8);
-            continue;
+        float a[4] = {0.f, 0.f, 0.f, 0.f};
+        bool valid = false;
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) {
+          ok = warp_wait(&full[q], ph, abort, p.err);
+          if (!ok) break;
+          const uint8_t* slot = ring + (size_t)q * L.slot_bytes;
+          if (c == 0) {
+            const int id = slot_id[q];
+            valid = id >= 0 && (int64_t)id < p.V;
+            if (mine && valid) load_gates(reinterpret_cast<const float*>(slot + L.gates_off), g, NP);
           }
-          const uint4* src = reinterpret_cast<const uint4*>(slot) + v;
-          float a[8];
+          if (mine && valid && lt < per_tok) {
+            const uint2* src = reinterpret_cast<const uint2*>(slot) + lt;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) a[i] = 0.f;
-#pragma unroll
-          for (int j = 0; j < NP; ++j) {
-            if (kExactN || j < p.N) {
-              const uint4 x = src[(int64_t)j * DV];
-              const float gj = g[j];
-              a[0] = fmaf(gj, bf16_lo(x.x), a[0]);
-              a[1] = fmaf(gj, bf16_hi(x.x), a[1]);
-              a[2] = fmaf(gj, bf16_lo(x.y), a[2]);
-              a[3] = fmaf(gj, bf16_hi(x.y), a[3]);
-              a[4] = fmaf(gj, bf16_lo(x.z), a[4]);
-              a[5] = fmaf(gj, bf16_hi(x.z), a[5]);
-              a[6] = fmaf(gj, bf16_lo(x.w), a[6]);
-              a[7] = fmaf(gj, bf16_hi(x.w), a[7]);
+            for (int jj = 0; jj < JC; ++jj) {
+              const int j = c * JC + jj;
+              if (kExactN || j < p.N) {
+                const uint2 x = src[jj * per_tok];
+                const float gj = g[j];
+                a[0] = fmaf(gj, bf16_lo(x.x), a[0]);
+                a[1] = fmaf(gj, bf16_hi(x.x), a[1]);
+                a[2] = fmaf(gj, bf16_lo(x.y), a[2]);
+                a[3] = fmaf(gj, bf16_hi(x.y), a[3]);
+              }
             }
           }
-          __stcs(reinterpret_cast<float4*>(o), make_float4(a[0], a[1], a[2], a[3]));
-          __stcs(reinterpret_cast<float4*>(o + 4), make_float4(a[4], a[5], a[6], a[7]));
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[q]);
+          if (++q == (uint32_t)L.n_slots) {
+            q = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!ok) break;
+        if (mine && lt < per_tok) {
+          float* o = orow + lt * 4;
+          if (valid) {
+            __stcs(reinterpret_cast<float4*>(o), make_float4(a[0], a[1], a[2], a[3]));
+          } else {
+            if (lt == 0) atomicOr(p.err, kErrIndex);
+            store_nan(o, 4);
+          }
+        }
+      } else {
+        // several units per thread: the whole token is in one slot (kChunks == 1)
+        ok = warp_wait(&full[q], ph, abort, p.err);
+        if (!ok) break;
+        if (mine) {
+          const int id = slot_id[q];
+          const bool valid = id >= 0 && (int64_t)id < p.V;
+          const uint8_t* slot = ring + (size_t)q * L.slot_bytes;
+          float g[NP];
+          if (valid) load_gates(reinterpret_cast<const float*>(slot + L.gates_off), g, NP);
+          const int units = kTable == kTableBf16 ? (p.D >> 3) : per_tok;  // 8-wide vectors here
+          for (int v = lt; v < units; v += gw * 32) {
+            if (kTable == kTableBf16) {
+              float* o = orow + v * 8;
+              if (!valid) {
+                if (v == 0) atomicOr(p.err, kErrIndex);
+                store_nan(o, 8);
+                continue;
+              }
+              const uint4* src = reinterpret_cast<const uint4*>(slot) + v;
+              float a[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) a[i] = 0.f;
+#pragma unroll
+              for (int j = 0; j < NP; ++j) {
+                if (kExactN || j < p.N) {
+                  const uint4 x = src[(int64_t)j * units];
+                  const float gj = g[j];
+                  a[0] = fmaf(gj, bf16_lo(x.x), a[0]);
+                  a[1] = fmaf(gj, bf16_hi(x.x), a[1]);
+                  a[2] = fmaf(gj, bf16_lo(x.y), a[2]);
+                  a[3] = fmaf(gj, bf16_hi(x.y), a[3]);
+                  a[4] = fmaf(gj, bf16_lo(x.z), a[4]);
+                  a[5] = fmaf(gj, bf16_hi(x.z), a[5]);
+                  a[6] = fmaf(gj, bf16_lo(x.w), a[6]);
+                  a[7] = fmaf(gj, bf16_hi(x.w), a[7]);
+                }
+              }
+              __stcs(reinterpret_cast<float4*>(o), make_float4(a[0], a[1], a[2], a[3]));
+              __stcs(reinterpret_cast<float4*>(o + 4), make_float4(a[4], a[5], a[6], a[7]));
+            } else {
+              float* o = orow + v * 32;
+              if (!valid) {
+                if (v == 0) atomicOr(p.err, kErrIndex);
+                store_nan(o, 32);
+                continue;
+              }
+              const int blk_in_row = v >> 1, half = v & 1;
+              const uint16_t* sc_row = reinterpret_cast<const uint16_t*>(slot + L.scales_off);
+              float acc[32];
+#pragma unroll
+              for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+#pragma unroll
+              for (int j = 0; j < NP; ++j) {
+                if (kExactN || j < p.N) {
+                  const int blk = j * NB + blk_in_row;
+                  const uint32_t* cw = reinterpret_cast<const uint32_t*>(slot + blk * 24 + half * 12);
+                  const uint32_t w0 = cw[0], w1 = cw[1], w2 = cw[2];
+                  const float a = g[j] * __half2float(__ushort_as_half(sc_row[blk]));
+                  uint32_t sl, sh;
+                  nf3_selectors(w0, sl, sh);
+                  nf3_fma4(sl, a, acc + 0);
+                  nf3_fma4(sh, a, acc + 4);
+                  nf3_selectors(__funnelshift_r(w0, w1, 24), sl, sh);
+                  nf3_fma4(sl, a, acc + 8);
+                  nf3_fma4(sh, a, acc + 12);
+                  nf3_selectors(__funnelshift_r(w1, w2, 16), sl, sh);
+                  nf3_fma4(sl, a, acc + 16);
+                  nf3_fma4(sh, a, acc + 20);
+                  nf3_selectors(w2 >> 8, sl, sh);
+                  nf3_fma4(sl, a, acc + 24);
+                  nf3_fma4(sh, a, acc + 28);
+                }
+              }
+#pragma unroll
+              for (int i = 0; i < 32; i += 4)
+                __stcs(reinterpret_cast<float4*>(o + i), make_float4(acc[i], acc[i + 1], acc[i + 2], acc[i + 3]));
+            }
+          }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&s.empty[q]);
+        if (lane == 0) mbar_arrive(&empty[q]);
+        if (++q == (uint32_t)L.n_slots) {
+          q = 0;
+          ph ^= 1u;
+        }
       }
-      __syncwarp();
-      if (ok && lane == 0) mbar_arrive(&s.gempty[b]);
+      if (++gsel == G) gsel = 0;
     }
   }
   __syncthreads();
 }
-
 
 template <bool kBf16Router, int NT, int kTable, bool kExactN>
 __global__ void __launch_bounds__(kThreads, 2) combine_kernel(const CombineArgs p) {
   constexpr int NP = 8 * NT;
-  extern __shared__ __align__(16) uint8_t smem_raw[];
+  extern __shared__ __align__(128) uint8_t smem_raw[];
   const Smem s = carve<kBf16Router, NP>(smem_raw, p.D);
   if (kBf16Router) {
-    // Stage Wr^T once per CTA: wrt[j][d] = Wr[d][j], zero rows j >= N.
-    const uint16_t* wr = static_cast<const uint16_t*>(p.Wr);
-    const int ldw = p.D + 8;
-    for (int i = threadIdx.x; i < p.D * NP; i += kThreads) {
-      const int d = i / NP, j = i - d * NP;
-      s.wrt[j * ldw + d] = j < p.N ? wr[(int64_t)d * p.N + j] : (uint16_t)0;
-    }
+    stage_wrt<NP, kThreads>(s.wrt, static_cast<const uint16_t*>(p.Wr), p.N, p.D);
     __syncthreads();
   }
   const int per_tok = kTable == kTableBf16 ? (p.D >> 3) : kTable == kTableF32 ? (p.D >> 2) : (p.D >> 5);
@@ -834,38 +884,64 @@ mole_status launch_one(CombineArgs p, cudaStream_t stream) {
   return cuda_status(cudaGetLastError());
 }
 
-template <int NT, bool kExactN>
-mole_status launch_tma(CombineArgs p, cudaStream_t stream) {
+template <int NT, bool kExactN, int kTable, int kChunks>
+mole_status launch_two_kernel(CombineArgs p, cudaStream_t stream) {
   constexpr int NP = 8 * NT;
-  const int64_t row_bytes = (int64_t)p.N * p.D * 2;
-  const int slot_bytes = (int)((row_bytes + 127) / 128 * 128);
-  int n_slots = (int)std::min<int64_t>(8, kRingBudget / slot_bytes);
-  size_t smem = 0;
-  while (n_slots >= 2 && (smem = tma_smem_bytes<NP>(p.D, n_slots, slot_bytes)) > 227 * 1024) --n_slots;
-  if (n_slots < 2) return MOLE_ERR_UNSUPPORTED;
-  auto kern = combine_tma_kernel<NT, kExactN>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+  if (p.D < NP) return MOLE_ERR_UNSUPPORTED;  // gates are parked in the output row
+  const int64_t NB = p.D / 64;
+  GatherLayout L{};
+  int64_t off;
+  if (kTable == kTableBf16) {
+    off = (int64_t)(NP / kChunks) * p.D * 2;
+  } else {
+    // both bulk copies need 16-byte aligned sources and sizes
+    if (((int64_t)p.N * NB) % 8 != 0) return MOLE_ERR_UNSUPPORTED;
+    const int64_t code_bytes = (int64_t)p.N * NB * 24;
+    L.scales_off = (int)((code_bytes + 127) / 128 * 128);
+    off = L.scales_off + (int64_t)p.N * NB * 2;
+  }
+  L.gates_off = (int)((off + 15) / 16 * 16);
+  L.slot_bytes = (int)((L.gates_off + NP * 4 + 127) / 128 * 128);
+  L.n_slots = (int)std::min<int64_t>(16, kRingBudget / L.slot_bytes);
+  if (L.n_slots < 2 * kChunks) return MOLE_ERR_UNSUPPORTED;
+  const size_t gsmem = (size_t)L.n_slots * L.slot_bytes + (size_t)L.n_slots * 20 + 16;
+  const size_t rsmem = smem_bytes_for<true, NP>(p.D);
+  if (gsmem > 227 * 1024 || rsmem > 227 * 1024) return MOLE_ERR_UNSUPPORTED;
+  auto rkern = router_gates_kernel<NT>;
+  auto gkern = gather_kernel<NT, kExactN, kTable, kChunks>;
+  if (cudaFuncSetAttribute(rkern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem) != cudaSuccess ||
+      cudaFuncSetAttribute(gkern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gsmem) != cudaSuccess)
     return MOLE_ERR_CUDA;
   const int n_sm = num_sms();
   if (n_sm <= 0) return MOLE_ERR_NO_DEVICE;
-  p.TT = choose_tile(p.T, n_sm);
+  p.TT = kTileMax;
   p.n_tiles = (p.T + p.TT - 1) / p.TT;
-  const int64_t grid = std::min<int64_t>(p.n_tiles, n_sm);
-  kern<<<(unsigned)grid, kTmaThreads, smem, stream>>>(p, n_slots, slot_bytes);
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, rkern, kThreads, rsmem) != cudaSuccess || occ < 1)
+    return MOLE_ERR_UNSUPPORTED;
+  rkern<<<(unsigned)std::min<int64_t>(p.n_tiles, (int64_t)occ * n_sm), kThreads, rsmem, stream>>>(p);
+  gkern<<<(unsigned)std::min<int64_t>(p.T, n_sm), kGatherThreads, gsmem, stream>>>(p, L);
   return cuda_status(cudaGetLastError());
 }
 
-// bf16 table: the TMA-staged kernel when a ring of >= 2 row blocks fits in
-// shared memory, else the register-gather kernel.
-mole_status launch_bf16_table(const CombineArgs& p, cudaStream_t stream) {
-  mole_status st = MOLE_ERR_UNSUPPORTED;
-  if (p.N == 16) st = launch_tma<2, true>(p, stream);
-  else if (p.N == 8) st = launch_tma<1, true>(p, stream);
-  else if (p.N < 8) st = launch_tma<1, false>(p, stream);
-  else if (p.N < 16) st = launch_tma<2, false>(p, stream);
-  else if (p.N == 32) st = launch_tma<4, true>(p, stream);
-  else st = launch_tma<4, false>(p, stream);
-  return st;
+// Batches of at least kTwoKernelMinT tokens (bf16 inputs, bf16 or NF3 table)
+// take the router + gather kernel pair; smaller batches and shapes it does not
+// cover take the single fused kernel (MOLE_ERR_UNSUPPORTED tells the caller).
+constexpr int64_t kTwoKernelMinT = 1024;
+
+template <int kTable>
+mole_status launch_staged(const CombineArgs& p, cudaStream_t stream) {
+  if (p.T < kTwoKernelMinT) return MOLE_ERR_UNSUPPORTED;
+  // bf16 rows above 40 KB per token (e.g. 16 x 2048) travel as two 8-expert
+  // halves, so the ring holds twice as many slots in flight
+  if (kTable == kTableBf16 && p.N == 16 && (int64_t)p.N * p.D * 2 > 40 * 1024 && p.D / 4 <= kGatherCons * 32)
+    return launch_two_kernel<2, true, kTable, 2>(p, stream);
+  if (p.N == 16) return launch_two_kernel<2, true, kTable, 1>(p, stream);
+  if (p.N == 8) return launch_two_kernel<1, true, kTable, 1>(p, stream);
+  if (p.N < 8) return launch_two_kernel<1, false, kTable, 1>(p, stream);
+  if (p.N < 16) return launch_two_kernel<2, false, kTable, 1>(p, stream);
+  if (p.N == 32) return launch_two_kernel<4, true, kTable, 1>(p, stream);
+  return launch_two_kernel<4, false, kTable, 1>(p, stream);
 }
 
 template <bool kBf16Router, int kTable>
@@ -898,10 +974,14 @@ mole_status combine_dispatch(const int32_t* ids, int64_t T, const void* h, const
   p.out = out;
   p.err = error_word();
   if (!p.err) return MOLE_ERR_CUDA;
-  if (table_kind == kTableNf3)
-    return bf16_inputs ? launch_combine<true, kTableNf3>(p, stream) : launch_combine<false, kTableNf3>(p, stream);
+  if (table_kind == kTableNf3) {
+    if (!bf16_inputs) return launch_combine<false, kTableNf3>(p, stream);
+    const mole_status st = launch_staged<kTableNf3>(p, stream);
+    if (st != MOLE_ERR_UNSUPPORTED) return st;
+    return launch_combine<true, kTableNf3>(p, stream);
+  }
   if (table_kind == kTableBf16) {
-    const mole_status st = launch_bf16_table(p, stream);
+    const mole_status st = launch_staged<kTableBf16>(p, stream);
     if (st != MOLE_ERR_UNSUPPORTED) return st;
     return launch_combine<true, kTableBf16>(p, stream);
   }

@@ -42,6 +42,12 @@ def _run(mole, ids, h, Wr, lut):
     (50304, 2048, 16, 300, "zipf"),
     (64, 2048, 32, 40, "uniform"),   # row block of 128 KB: register-gather kernel
     (96, 1024, 24, 77, "zipf"),      # 48 KB row blocks, padded expert count
+    # >= 1024 tokens: router kernel + bulk-copy gather kernel
+    (3000, 768, 16, 2000, "zipf"),   # two token groups per CTA
+    (500, 256, 16, 1500, "uniform"),
+    (300, 64, 8, 1100, "uniform"),
+    (200, 128, 13, 1024, "zipf"),    # padded expert count
+    (64, 2048, 32, 1030, "uniform"), # 128 KB row blocks: no ring fits, fused kernel
 ])
 def test_combine_bf16_matches_oracle(mole, oracle_mod, V, D, N, T, kind):
     ids, h, Wr, lut = _layer(100 + D + N + T, V, D, N, T, ids_kind=kind)
@@ -86,16 +92,17 @@ def test_combine_edges(mole, oracle_mod):
     assert mole.mole_check() == 0
 
 
-def test_combine_bad_ids_give_nan_rows_and_index_error(mole, oracle_mod):
+@pytest.mark.parametrize("T", [40, 1500])
+def test_combine_bad_ids_give_nan_rows_and_index_error(mole, oracle_mod, T):
     V, D, N = 300, 128, 16
-    ids, h, Wr, lut = _layer(32, V, D, N, 40)
+    ids, h, Wr, lut = _layer(32, V, D, N, T)
     ids[[3, 17, 39]] = [-1, V, 2 ** 31 - 1]
     got, st = _run(mole, ids, h, Wr, lut)
     assert st == 5  # MOLE_ERR_INDEX
     assert mole.mole_check() == 0  # the error word was cleared
     ref, nbad = oracle_mod.combine(ids, h, Wr, lut)
     assert nbad == 3
-    bad = np.zeros(40, bool)
+    bad = np.zeros(T, bool)
     bad[[3, 17, 39]] = True
     assert np.isnan(got[bad]).all()
     assert_combine_close(got[~bad], ref[~bad])

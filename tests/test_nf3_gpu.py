@@ -43,6 +43,8 @@ def test_quantize_bit_exact(mole, oracle_mod, V, N, D):
 @pytest.mark.parametrize("V,N,D,T,dtype", [
     (300, 16, 2048, 300, "bf16"), (100, 16, 128, 77, "bf16"), (50, 5, 64, 19, "bf16"),
     (64, 24, 256, 40, "bf16"), (80, 8, 192, 33, "f32"),
+    (200, 16, 256, 1500, "bf16"), (300, 8, 2048, 1100, "bf16"),  # router + gather kernels
+    (100, 5, 128, 1200, "bf16"),  # N*D/64 not a multiple of 8: fused kernel
 ])
 def test_combine_nf3_matches_oracle(mole, oracle_mod, V, N, D, T, dtype):
     rng = np.random.default_rng(T + D)
@@ -59,8 +61,9 @@ def test_combine_nf3_matches_oracle(mole, oracle_mod, V, N, D, T, dtype):
     assert_combine_close(out.cpu().numpy(), ref)
 
 
-def test_combine_nf3_bad_ids(mole, oracle_mod):
-    V, N, D, T = 40, 16, 128, 20
+@pytest.mark.parametrize("T", [20, 1200])
+def test_combine_nf3_bad_ids(mole, oracle_mod, T):
+    V, N, D = 40, 16, 128
     rng = np.random.default_rng(3)
     lut = inputs.normal(rng, (V, N, D), 0.02, "bf16")
     Wr = inputs.normal(rng, (D, N), 0.02, "bf16")
