@@ -4,12 +4,14 @@
 Workload (default): the 1B-activated-shaped MoLE model -- 16 layers, each with
 its own table LUT[50304, 16, 2048] bf16 (3.3 GB) and router Wr[2048, 16] --
 over a prefill batch of T = 16384 tokens with Zipf(1.1) ids.  One step is one
-pass of the lookup path of a forward pass: mole_lookup_combine for each of the
-16 layers (router GEMV + softmax + direct-addressed gather + gate-weighted
-sum), every layer with its own hidden states.  Tables are seeded N(0, 0.02)
-fills (the combine's time does not depend on the values); ids and hidden
-states are fresh per step.  A step touches 16 distinct tables of 3.3 GB, so
-inputs are far larger than the 126 MB L2.
+pass of the lookup path of a forward pass: the batch's token grouping
+(mole_token_groups_build, once: every layer indexes its table with the same
+token ids) and a combine for each of the 16 layers (router GEMV + softmax +
+direct-addressed gather + gate-weighted sum), every layer with its own hidden
+states.  Tables are seeded N(0, 0.02) fills (the combine's time does not
+depend on the values); ids and hidden states rotate over a pool of 4 batches.
+A step touches 16 distinct tables of 3.3 GB, so inputs are far larger than
+the 126 MB L2.  --path plain runs mole_lookup_combine per layer instead.
 
 Also measured in the same run (own keys in the JSON line): the one-off table
 build (410M-shaped layer, tensor cores), the NF3-compressed table combine, and
@@ -43,8 +45,17 @@ from mixture_lookup_experts_b200 import inputs  # noqa: E402
 
 METRIC = "MoLE lookup-combine tokens/s & HBM GB/s vs 8 TB/s; LUT build TFLOP/s"
 UNIT = "tokens/s"
-KERNEL_SOURCES = ["mixture_lookup_experts_b200/csrc/combine.cu", "mixture_lookup_experts_b200/csrc/common.cuh"]
-PROFILE_SUMMARY = "profiles/combine_bf16_1b_T16384_zipf.md"
+KERNEL_SOURCES = ["mixture_lookup_experts_b200/csrc/combine.cu", "mixture_lookup_experts_b200/csrc/grouped.cu",
+                  "mixture_lookup_experts_b200/csrc/combine_common.cuh", "mixture_lookup_experts_b200/csrc/common.cuh"]
+PROFILE_SUMMARY = {"grouped": "profiles/combine_grouped_bf16_1b_T16384_zipf.md",
+                   "plain": "profiles/combine_bf16_1b_T16384_zipf.md"}
+KERNELS = {
+    "grouped": "mole_lookup_combine_groups = router_group_kernel (tensor-core router, gates to the tokens' list "
+               "positions) + grouped_gather_kernel (one bulk copy per distinct row block, all of its tokens combined "
+               "from shared memory); duration = the call (the per-step grouping is timed apart)",
+    "plain": "mole_lookup_combine = router_gates_kernel (tensor-core router, gates parked in the output rows) + "
+             "gather_kernel (bulk-copy ring of row blocks, consumer warps); duration = the call",
+}
 
 
 def parse_args():
@@ -55,6 +66,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--tokens", type=int, default=16384)
     ap.add_argument("--ids", choices=["zipf", "uniform"], default="zipf")
+    ap.add_argument("--path", choices=["grouped", "plain"], default="grouped",
+                    help="grouped: mole_lookup_combine_grouped (default); plain: mole_lookup_combine")
     ap.add_argument("--layers", type=int, default=None,
                     help="layer tables to allocate (default: the model's 16); fewer only for profiling runs")
     ap.add_argument("--no-extras", action="store_true", help="skip the build / NF3 / other-case legs")
@@ -67,16 +80,42 @@ def parse_args():
     return ap.parse_args()
 
 
-def workload_config(T: int, kind: str, layers: int | None = None) -> dict:
+class Combiner:
+    """The combine call of the chosen path.  grouped: the batch's token
+    grouping is built once per step (prepare) and serves every layer's
+    mole_lookup_combine_groups; plain: mole_lookup_combine per layer."""
+
+    def __init__(self, mole, path: str, T: int, V: int, N: int, dev):
+        import torch
+        self.mole, self.path, self.V, self.N = mole, path, V, N
+        self.groups = None
+        if path == "grouped":
+            self.groups = torch.empty(mole.mole_token_groups_workspace(T, N), dtype=torch.uint8, device=dev)
+
+    def prepare(self, ids, stream):
+        if self.path == "grouped":
+            self.mole.mole_token_groups_build(ids, self.V, self.N, groups=self.groups, stream=stream)
+
+    def __call__(self, ids, h, Wr, lut, out, stream):
+        if self.path == "grouped":
+            self.mole.mole_lookup_combine_groups(ids, self.groups, h, Wr, lut, out=out, stream=stream)
+        else:
+            self.mole.mole_lookup_combine(ids, h, Wr, lut, out=out, stream=stream)
+
+
+def workload_config(T: int, kind: str, layers: int | None = None, path: str = "grouped") -> dict:
     s = inputs.SHAPES["1b"]
     layers = s.layers if layers is None else layers
+    call = "mole_lookup_combine_groups" if path == "grouped" else "mole_lookup_combine"
     return {
-        "workload": f"1B-activated-shaped MoLE lookup path, {layers} layers x mole_lookup_combine, "
-                    f"prefill T={T}, {'Zipf(1.1)' if kind == 'zipf' else 'uniform'} ids",
+        "workload": f"1B-activated-shaped MoLE lookup path, {layers} layers x {call}"
+                    f"{' (one token grouping per step)' if path == 'grouped' else ''}, "
+                    f"prefill T={T}, {'Zipf(1.1)' if kind == 'zipf' else 'uniform'} ids shared by the layers",
         "V": s.V, "D": s.D, "N": s.N, "layers": layers, "tokens_per_step": T, "ids": kind,
         "table_dtype": "bf16", "accumulate": "f32", "out_dtype": "f32",
         "l2": "inputs larger than L2: each step reads 16 distinct 3.3 GB layer tables",
-        "data": "synthetic seeded N(0,0.02) tables; fresh ids and hidden states per step",
+        "data": "synthetic seeded N(0,0.02) tables; per step one id batch (shared by the layers) and per-layer "
+                "hidden states, rotating over a pool of 4",
     }
 
 
@@ -155,10 +194,10 @@ def kernel_source_hash() -> str:
     return h.hexdigest()
 
 
-def profiled_traffic():
+def profiled_traffic(path: str):
     """(bytes per launch, note) from the committed ncu summary if it was taken
     on the current kernel source; else (None, reason)."""
-    p = os.path.join(ROOT, PROFILE_SUMMARY)
+    p = os.path.join(ROOT, PROFILE_SUMMARY[path])
     if not os.path.exists(p):
         return None, "no ncu summary committed"
     fields = {}
@@ -224,11 +263,10 @@ def run_reference(args):
 
     def one_step(seed):
         r = np.random.default_rng(seed)
-        t0 = time.perf_counter()
         done = 0
+        ids = inputs.draw_ids(r, sample_T, V, args.ids)  # the batch's ids, shared by the layers
+        uniq, inv = np.unique(ids, return_inverse=True)
         for layer in range(L):
-            ids = inputs.draw_ids(r, sample_T, V, args.ids)
-            uniq, inv = np.unique(ids, return_inverse=True)
             rows = inputs.normal(r, (uniq.size, N, D), 0.02, "bf16")  # the rows this sample reads
             Wr = inputs.normal(r, (D, N), 0.02, "bf16")
             h = inputs.normal(r, (sample_T, D), 1.0, "bf16")
@@ -305,19 +343,29 @@ def main():
     # per-step batches: a pool of P distinct (ids, h) per layer slot, rotated
     P = 4
     rng = np.random.default_rng(host_seed)
-    id_pool = [[torch.from_numpy(inputs.draw_ids(rng, T, V, args.ids)).to(dev) for _ in range(L)] for _ in range(P)]
+    # every layer of a step indexes its table with the same token ids (the
+    # batch's), with its own hidden states
+    id_pool = [[torch.from_numpy(inputs.draw_ids(rng, T, V, args.ids)).to(dev)] * L for _ in range(P)]
     h_pool = [[(torch.randn((T, D), generator=g, device=dev)).to(torch.bfloat16) for _ in range(L)]
               for _ in range(P)]
     uniq_counts = [[int(torch.unique(x).numel()) for x in pool] for pool in id_pool]
     out = torch.empty((T, D), dtype=torch.float32, device=dev)
+    combine = Combiner(mole, args.path, T, V, N, dev)
+    prep_events = []
 
     def step(i, events=None):
         p = i % P
+        if events is not None:
+            e = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            e[0].record(stream)
+        combine.prepare(id_pool[p][0], stream)
+        if events is not None:
+            e[1].record(stream)
+            prep_events.append(e)
         for layer in range(L):
             if events is not None:
                 events[layer][0].record(stream)
-            mole.mole_lookup_combine(id_pool[p][layer], h_pool[p][layer], routers[layer], luts[layer], out=out,
-                                     stream=stream)
+            combine(id_pool[p][layer], h_pool[p][layer], routers[layer], luts[layer], out, stream)
             if events is not None:
                 events[layer][1].record(stream)
 
@@ -351,22 +399,23 @@ def main():
     avg_kern_ms = sum(kern_ms) / len(kern_ms)
     U_avg = sum(uniq_counts[(W + i) % P][l] for i in range(K) for l in range(L)) / (K * L)
 
-    max_ms, max_kern_ms = max_over_ranks([elapsed_ms, avg_kern_ms], dev)
+    prep_ms = [a.elapsed_time(b) for a, b in prep_events[-K:]] if prep_events else [0.0]
+    avg_prep_ms = sum(prep_ms) / len(prep_ms)
+    max_ms, max_kern_ms, max_prep_ms = max_over_ranks([elapsed_ms, avg_kern_ms, avg_prep_ms], dev)
     value = whole_job_tokens_per_s(world, T, K, max_ms)
 
     # ---- end to end through the C ABI with host buffers ----
-    e2e = None if args.no_e2e else e2e_leg(mole, id_pool, h_pool, routers, luts, out, dev, stream, world, W, K, T, L)
+    e2e = None if args.no_e2e else e2e_leg(combine, id_pool, h_pool, routers, luts, out, dev, stream, world, W, K,
+                                           T, L)
 
     # ---- roofline of the combine kernel ----
     hbm_peak, bf16_peak, bf16_sust, peak_kind = measured_peaks()
     alg_bytes = combine_bytes(U_avg, T, D, N)
     achieved_gbs = alg_bytes / (max_kern_ms / 1e3) / 1e9
-    traffic, traffic_note = profiled_traffic()
+    traffic, traffic_note = profiled_traffic(args.path)
     roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
                 "frac": achieved_gbs / hbm_peak, "traffic": traffic,
-                "kernel": "mole_lookup_combine = router_gates_kernel (tensor-core router, gates parked in the "
-                          "output rows) + gather_kernel (bulk-copy ring of row blocks, consumer warps); "
-                          "duration = the call, both kernels",
+                "kernel": KERNELS[args.path],
                 "algorithmic_bytes_per_launch": alg_bytes, "unique_rows_per_launch": U_avg,
                 "avg_launch_us": max_kern_ms * 1e3, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
                 "frac_of_8TBs": achieved_gbs / 8000.0, "traffic_source": traffic_note}
@@ -374,17 +423,19 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": max_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic", "config": workload_config(T, args.ids, L),
+        "dtype": "bf16", "data": "synthetic", "config": workload_config(T, args.ids, L, args.path),
         "layer_tokens_per_s": value * L, "hbm_gbs": achieved_gbs,
         "roofline": roofline,
         "e2e": e2e,
-        "gpu_launches": K * L,
+        # per layer: router kernel + gather kernel (T >= 1024); per step: the grouping kernel (grouped path)
+        "gpu_launches": K * L * (2 if T >= 1024 else 1) + (K if args.path == "grouped" else 0),
+        "token_groups_build_us_per_step": max_prep_ms * 1e3 if args.path == "grouped" else None,
         "clocks": clocks.summary(),
     }
 
     # ---- extras: other prefill cases, NF3 table, table build ----
     if not args.no_extras:
-        line["cases"] = other_cases(mole, luts, routers, rng, g, dev, stream, W, T, args.ids, L)
+        line["cases"] = other_cases(mole, luts, routers, rng, g, dev, stream, W, T, args.ids, args.path, L)
         line["nf3"] = nf3_leg(mole, luts, routers, id_pool, h_pool, uniq_counts, dev, stream, W, K, T, P, L)
         del luts
         torch.cuda.empty_cache()
@@ -399,7 +450,7 @@ def main():
         dist.destroy_process_group()
 
 
-def e2e_leg(mole, id_pool, h_pool, routers, luts, out, dev, stream, world, W, K, T, L):
+def e2e_leg(combine, id_pool, h_pool, routers, luts, out, dev, stream, world, W, K, T, L):
     """The same metric through the C ABI with host buffers: per step the ids
     and the L hidden-state batches are copied host -> device from pinned
     memory, the L combine calls run, and the L outputs are copied back."""
@@ -407,19 +458,20 @@ def e2e_leg(mole, id_pool, h_pool, routers, luts, out, dev, stream, world, W, K,
     import torch.distributed as dist
     D = out.shape[1]
     h_host = [torch.empty((T, D), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    ids_host = torch.empty((L, T), dtype=torch.int32).pin_memory()
+    ids_host = torch.empty((T,), dtype=torch.int32).pin_memory()
     out_host = torch.empty((T, D), dtype=torch.float32).pin_memory()
     for s in range(min(2, L)):
         h_host[s].copy_(h_pool[0][s])
-    ids_host.copy_(torch.stack(id_pool[0]).cpu())
+    ids_host.copy_(id_pool[0][0].cpu())
     h_stage = torch.empty((T, D), dtype=torch.bfloat16, device=dev)
-    ids_stage = torch.empty((L, T), dtype=torch.int32, device=dev)
+    ids_stage = torch.empty((T,), dtype=torch.int32, device=dev)
 
     def e2e_step():
         ids_stage.copy_(ids_host, non_blocking=True)
+        combine.prepare(ids_stage, stream)
         for layer in range(L):
             h_stage.copy_(h_host[layer % 2], non_blocking=True)
-            mole.mole_lookup_combine(ids_stage[layer], h_stage, routers[layer], luts[layer], out=out, stream=stream)
+            combine(ids_stage, h_stage, routers[layer], luts[layer], out, stream)
             out_host.copy_(out, non_blocking=True)
 
     for _ in range(min(W, 3)):
@@ -437,9 +489,9 @@ def e2e_leg(mole, id_pool, h_pool, routers, luts, out, dev, stream, world, W, K,
     torch.cuda.synchronize()
     (e_ms,) = max_over_ranks([e_start.elapsed_time(e_end)], dev)
     return {"value": whole_job_tokens_per_s(world, T, K_e2e, e_ms), "unit": UNIT,
-            "h2d_bytes_per_step": L * T * D * 2 + L * T * 4, "d2h_bytes_per_step": L * T * D * 4,
-            "steps": K_e2e, "note": f"per step: ids + {L} hidden-state batches H2D from pinned memory, "
-                                    f"{L} combine calls through the C ABI, {L} outputs D2H"}
+            "h2d_bytes_per_step": L * T * D * 2 + T * 4, "d2h_bytes_per_step": L * T * D * 4,
+            "steps": K_e2e, "note": f"per step: the batch's ids + {L} hidden-state batches H2D from pinned memory, "
+                                    f"the token grouping and {L} combine calls through the C ABI, {L} outputs D2H"}
 
 
 def time_launches(fn, n, stream):
@@ -453,7 +505,10 @@ def time_launches(fn, n, stream):
     return [a.elapsed_time(b) for a, b in ev]
 
 
-def other_cases(mole, luts, routers, rng, g, dev, stream, W, T_main, kind_main, L):
+def other_cases(mole, luts, routers, rng, g, dev, stream, W, T_main, kind_main, path_main, L):
+    """The other prefill cases of the 1B-shaped layer, on both combine paths:
+    one id batch shared by the L layers, the grouping built once (its time
+    reported apart), per-layer combine calls timed."""
     import torch
     shape = inputs.SHAPES["1b"]
     V, D, N = shape.V, shape.D, shape.N
@@ -461,25 +516,32 @@ def other_cases(mole, luts, routers, rng, g, dev, stream, W, T_main, kind_main, 
     res = {}
     for T in (4096, 16384):
         for kind in ("zipf", "uniform"):
-            if T == T_main and kind == kind_main:
-                continue
-            ids = [torch.from_numpy(inputs.draw_ids(rng, T, V, kind)).to(dev) for _ in range(L)]
+            ids = torch.from_numpy(inputs.draw_ids(rng, T, V, kind)).to(dev)
             hs = [torch.randn((T, D), generator=g, device=dev).to(torch.bfloat16) for _ in range(L)]
-            U = sum(int(torch.unique(x).numel()) for x in ids) / L
+            U = int(torch.unique(ids).numel())
             out = torch.empty((T, D), dtype=torch.float32, device=dev)
+            for path in ("grouped", "plain"):
+                if T == T_main and kind == kind_main and path == path_main:
+                    continue
+                combine = Combiner(mole, path, T, V, N, dev)
+                combine.prepare(ids, stream)
 
-            def fn(i):
-                lay = i % L
-                mole.mole_lookup_combine(ids[lay], hs[lay], routers[lay], luts[lay], out=out, stream=stream)
+                def fn(i):
+                    lay = i % L
+                    combine(ids, hs[lay], routers[lay], luts[lay], out, stream)
 
-            for i in range(max(W, 3) * L):
-                fn(i)
-            ms = time_launches(fn, 4 * L, stream)
-            avg = sum(ms) / len(ms)
-            b = combine_bytes(U, T, D, N)
-            res[f"T{T}_{kind}"] = {"tokens_per_s_per_layer": T / (avg / 1e3), "avg_launch_us": avg * 1e3,
-                                   "unique_rows": U, "achieved_gbs": b / (avg / 1e3) / 1e9,
-                                   "frac_of_measured_hbm": b / (avg / 1e3) / 1e9 / hbm_peak}
+                for i in range(max(W, 3) * L):
+                    fn(i)
+                ms = time_launches(fn, 4 * L, stream)
+                avg = sum(ms) / len(ms)
+                prep = time_launches(lambda i: combine.prepare(ids, stream), 5, stream)
+                b = combine_bytes(U, T, D, N)
+                res[f"T{T}_{kind}_{path}"] = {"tokens_per_s_per_layer": T / (avg / 1e3), "avg_launch_us": avg * 1e3,
+                                              "unique_rows": U, "achieved_gbs": b / (avg / 1e3) / 1e9,
+                                              "frac_of_measured_hbm": b / (avg / 1e3) / 1e9 / hbm_peak,
+                                              "token_groups_build_us": (sum(prep) / len(prep) * 1e3
+                                                                        if path == "grouped" else None)}
+                del combine
             del ids, hs, out
     return res
 

@@ -137,6 +137,46 @@ mole_status mole_lookup_combine(const int32_t* ids, int64_t T, const void* h, co
                                 mole_dtype dt, float* out, cudaStream_t stream);
 
 /*
+ * ---- Token groups: the combine with each distinct row block read once ----
+ * (MoLE page, 复杂度分析: a token's traffic is its N expert-output rows; a batch
+ * that repeats an id needs that id's rows only once.  推理阶段: every MoLE
+ * layer indexes its table with the same input token ids, so one grouping of
+ * the batch serves all layers.)
+ *
+ * mole_token_groups_build groups the batch's tokens by id into `groups`, a
+ * caller-owned device buffer of at least mole_token_groups_workspace(T, N)
+ * bytes, 16-byte aligned (N = the experts of the layers it will serve).  Its
+ * contents are opaque; the grouping stays valid until the buffer is rebuilt.
+ * Ids outside [0, V) are left out of every group and set the device error
+ * word (MOLE_ERR_INDEX).  One cooperative kernel launch (all of its CTAs
+ * resident at once).
+ *
+ * mole_lookup_combine_groups is mole_lookup_combine (same arguments, layouts,
+ * results bit for bit, and error behaviour) for a batch whose grouping was
+ * built from the same ids, T and N: each distinct id's row block is read once
+ * and applied to all of that id's tokens.  The call also writes one layer's
+ * gates into `groups`, so calls that share a groups buffer must not overlap
+ * on the GPU.  The grouped kernels serve bf16 inputs with T >= 1024; other
+ * calls run the mole_lookup_combine kernels (the grouping is then unused).
+ *
+ * mole_lookup_combine_grouped builds the grouping in `workspace` and runs
+ * mole_lookup_combine_groups, for a single layer;
+ * mole_lookup_combine_grouped_workspace equals mole_token_groups_workspace.
+ * All three return MOLE_ERR_WORKSPACE if the buffer is NULL or too small
+ * (T > 0) and MOLE_ERR_ALIGN if it is not 16-byte aligned.
+ */
+size_t mole_token_groups_workspace(int64_t T, int32_t N);
+mole_status mole_token_groups_build(const int32_t* ids, int64_t T, int64_t V, int32_t N, void* groups,
+                                    size_t bytes, cudaStream_t stream);
+mole_status mole_lookup_combine_groups(const int32_t* ids, int64_t T, const void* groups, size_t bytes,
+                                       const void* h, const void* Wr, const void* lut, int64_t V, int32_t N,
+                                       int64_t D, mole_dtype dt, float* out, cudaStream_t stream);
+size_t mole_lookup_combine_grouped_workspace(int64_t T, int32_t N);
+mole_status mole_lookup_combine_grouped(const int32_t* ids, int64_t T, const void* h, const void* Wr,
+                                        const void* lut, int64_t V, int32_t N, int64_t D, mole_dtype dt,
+                                        float* out, void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/*
  * ---- NF3 table compression (MoLE page, 实验结果: 3-bit table, e.g. NF3) ----
  *
  * Quantises a bf16 table [V, N, D] (D % 64 == 0) in blocks of 64 consecutive

@@ -70,6 +70,76 @@ extern "C" mole_status mole_lookup_combine(const int32_t* ids, int64_t T, const 
                                 dt == MOLE_BF16 ? 0 : 1, out, stream);
 }
 
+extern "C" size_t mole_token_groups_workspace(int64_t T, int32_t N) { return mole::token_groups_bytes(T, N); }
+
+extern "C" size_t mole_lookup_combine_grouped_workspace(int64_t T, int32_t N) {
+  return mole::token_groups_bytes(T, N);
+}
+
+namespace {
+mole_status check_groups(int64_t T, int32_t N, const void* groups, size_t bytes) {
+  if (T == 0) return MOLE_OK;
+  if (!groups || bytes < mole::token_groups_bytes(T, N)) return MOLE_ERR_WORKSPACE;
+  if (!mole::aligned16(groups)) return MOLE_ERR_ALIGN;
+  return MOLE_OK;
+}
+
+mole_status check_combine_bf16(const int32_t* ids, int64_t T, const void* h, const void* Wr, const void* lut,
+                               int64_t V, int32_t N, int64_t D, mole_dtype dt, float* out) {
+  if (!valid_dtype(dt)) return MOLE_ERR_ARG;
+  mole_status st = check_combine(ids, T, h, Wr, lut, V, N, D, out);
+  if (st != MOLE_OK) return st;
+  if (dt == MOLE_BF16 && D % 16 != 0) return MOLE_ERR_UNSUPPORTED;
+  if (dt == MOLE_F32 && D % 4 != 0) return MOLE_ERR_UNSUPPORTED;
+  if (!mole::aligned16(lut)) return MOLE_ERR_ALIGN;
+  return MOLE_OK;
+}
+}  // namespace
+
+extern "C" mole_status mole_token_groups_build(const int32_t* ids, int64_t T, int64_t V, int32_t N, void* groups,
+                                               size_t bytes, cudaStream_t stream) {
+  if (T < 0 || V <= 0 || V > INT32_MAX || N <= 0) return MOLE_ERR_ARG;
+  if (T > 0 && !ids) return MOLE_ERR_ARG;
+  if (N > 32) return MOLE_ERR_UNSUPPORTED;
+  mole_status st = check_groups(T, N, groups, bytes);
+  if (st != MOLE_OK || T == 0) return st;
+  st = check_device();
+  if (st != MOLE_OK) return st;
+  return mole::token_groups_build(ids, T, V, N, groups, bytes, stream);
+}
+
+extern "C" mole_status mole_lookup_combine_groups(const int32_t* ids, int64_t T, const void* groups, size_t bytes,
+                                                  const void* h, const void* Wr, const void* lut, int64_t V,
+                                                  int32_t N, int64_t D, mole_dtype dt, float* out,
+                                                  cudaStream_t stream) {
+  mole_status st = check_combine_bf16(ids, T, h, Wr, lut, V, N, D, dt, out);
+  if (st != MOLE_OK) return st;
+  st = check_groups(T, N, groups, bytes);
+  if (st != MOLE_OK || T == 0) return st;
+  st = check_device();
+  if (st != MOLE_OK) return st;
+  if (dt == MOLE_BF16 && mole::aligned16(Wr)) {
+    st = mole::combine_groups(groups, bytes, T, h, Wr, lut, N, (int)D, out, stream);
+    if (st != MOLE_ERR_UNSUPPORTED) return st;
+  }
+  return mole::combine_dispatch(ids, T, h, Wr, lut, nullptr, V, N, (int)D, dt == MOLE_BF16, dt == MOLE_BF16 ? 0 : 1,
+                                out, stream);
+}
+
+extern "C" mole_status mole_lookup_combine_grouped(const int32_t* ids, int64_t T, const void* h, const void* Wr,
+                                                   const void* lut, int64_t V, int32_t N, int64_t D,
+                                                   mole_dtype dt, float* out, void* workspace, size_t ws_bytes,
+                                                   cudaStream_t stream) {
+  mole_status st = check_combine_bf16(ids, T, h, Wr, lut, V, N, D, dt, out);
+  if (st != MOLE_OK) return st;
+  st = check_groups(T, N, workspace, ws_bytes);
+  if (st != MOLE_OK || T == 0) return st;
+  st = check_device();
+  if (st != MOLE_OK) return st;
+  return mole::combine_grouped_dispatch(ids, T, h, Wr, lut, nullptr, V, N, (int)D, dt == MOLE_BF16,
+                                        dt == MOLE_BF16 ? 0 : 1, out, workspace, ws_bytes, stream);
+}
+
 extern "C" mole_status mole_quantize_lut_nf3(const void* lut_bf16, int64_t V, int32_t N, int64_t D,
                                              uint8_t* codes, uint16_t* scales, cudaStream_t stream) {
   if (!lut_bf16 || !codes || !scales || V <= 0 || N <= 0 || D <= 0) return MOLE_ERR_ARG;

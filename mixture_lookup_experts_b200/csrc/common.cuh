@@ -131,6 +131,19 @@ mole_status combine_dispatch(const int32_t* ids, int64_t T, const void* h, const
                              bool bf16_inputs, int table_kind, float* out, cudaStream_t stream);
 mole_status nf3_quantize_launch(const void* lut, int64_t V, int N, int64_t D, uint8_t* codes,
                                 uint16_t* scales, cudaStream_t stream);
+// Id-grouped combine (grouped.cu): the grouping of a batch's tokens by id
+// (built once per batch), one layer's combine with it, and both in one call;
+// the combines fall back to combine_dispatch where the grouped kernels do not
+// apply.
+size_t token_groups_bytes(int64_t T, int N);
+mole_status token_groups_build(const int32_t* ids, int64_t T, int64_t V, int N, void* buf, size_t bytes,
+                               cudaStream_t stream);
+mole_status combine_groups(const void* buf, size_t bytes, int64_t T, const void* h, const void* Wr,
+                           const void* table, int N, int D, float* out, cudaStream_t stream);
+mole_status combine_grouped_dispatch(const int32_t* ids, int64_t T, const void* h, const void* Wr,
+                                     const void* table, const uint16_t* scales, int64_t V, int N, int D,
+                                     bool bf16_inputs, int table_kind, float* out, void* ws, size_t ws_bytes,
+                                     cudaStream_t stream);
 void nf3_tables(uint16_t levels[8], float mid[7]);
 mole_status gather_plan_launch(const int32_t* ids, int64_t T, int64_t V, int32_t* uniq,
                                int32_t* n_uniq, int32_t* slot, cudaStream_t stream);
@@ -176,6 +189,22 @@ __device__ __forceinline__ bool mbar_test(uint64_t* b, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+
+// try_wait with a suspend-time hint: a thread whose phase is not complete
+// sleeps in the barrier unit (issuing nothing) until the phase completes or
+// about hint_ns have passed, instead of spinning on the scheduler.
+__device__ __forceinline__ bool mbar_test_sleep(uint64_t* b, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(b)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+constexpr uint32_t kSuspendHintNs = 20000;
 
 // Waits for the phase with the given parity to complete.  Gives up (returns
 // false) when *abort is set by another role or after kWaitLimitNs, in which

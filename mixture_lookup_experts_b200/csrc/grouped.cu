@@ -1,0 +1,736 @@
+// grouped.cu -- lookup-combine with the batch's tokens grouped by token id
+// (MoLE page, 推理阶段 and 复杂度分析: what moves per token is its block of N
+// expert-output rows, addressed by the token id).  A prefill batch of text
+// repeats ids -- with Zipf-distributed ids, 16384 tokens over a 50K
+// vocabulary hold about 4K distinct ids -- and every token with the same id
+// reads the same row block.  This path fetches each distinct row block once
+// per batch and combines all of that id's tokens from one shared-memory copy.
+// Every MoLE layer indexes its table with the same input token ids, so the
+// grouping is built once per batch and serves all layers.
+//
+//  1. group_plan_kernel (cooperative launch; once per batch):
+//       step 0  every token's id goes into an open-addressing hash table
+//               (one atomicCAS per distinct id of a warp), and the token
+//               takes a rank inside its id's group (one atomicAdd per
+//               distinct slot of a warp, __match_any_sync);
+//       step 1  per CTA, the token and work-item totals (by item size) of a
+//               range of table slots (an item = up to kItemTokens tokens of
+//               one id), added atomically to grid totals: the running total
+//               a CTA sees is its base inside each region;
+//       step 2  per id the offset of its token range in the list and its
+//               item records, laid out by item size, largest first;
+//       step 3  every token's list position: list[pos] = t, tok_pos[t] = pos.
+//     Steps 1-3 each start after a grid-wide barrier (bounded wait).
+//  2. router_group_kernel (per layer; persistent, 2 CTAs per SM): the
+//     tensor-core router + softmax of combine_common.cuh; each token's gates
+//     go to its list position, so an item's gates are contiguous.
+//  3. grouped_gather_kernel (per layer; one CTA per SM, 9 warps): a producer
+//     warp copies each work item's row block and its tokens' gates (two
+//     cp.async.bulk) into a ring of shared-memory slots; 8 consumer warps
+//     convert each 4-element vector of the N rows to fp32 once and apply it
+//     to every token of the item.
+//
+// Per token the arithmetic is that of the ungrouped kernels (the same router
+// code, then out = sum over j = 0..N-1, in order, of g_j * x_j with fp32
+// FMAs), so both paths give bit-identical outputs; only the order in which
+// tokens are processed differs.
+#include "combine_common.cuh"
+
+namespace mole {
+namespace {
+
+constexpr int kItemTokens = 16;     // tokens per work item
+constexpr int kPlanThreads = 256;
+constexpr int kPlanMaxGrid = 1024;
+constexpr int64_t kGroupedMinT = 1024;
+constexpr int64_t kGroupedMaxT = int64_t(1) << 30;
+
+// Per-CTA totals of step 1: [0] tokens, [n] work items of n tokens (n = 1..kItemTokens).
+constexpr int kAgg = kItemTokens + 1;
+
+// Control words (set to 0xFFFFFFFF when a grouping is built): work items,
+// the three grid-barrier counters, the abort word, and the running totals of
+// step 1 (value + 1 = the sum so far).
+enum : int { kCtlItems = 1, kCtlBar = 2, kCtlAbort = 5, kCtlTot = 8, kCtlWords = kCtlTot + kAgg };
+
+// The grouping of one batch (the caller's buffer, carved by carve_ws).
+struct GroupWs {
+  int* key;       // [hcap] id in the slot, -1 = empty
+  int* cnt;       // [hcap] tokens in the slot minus one
+  unsigned* ctl;  // [kCtlWords]
+  int* off;       // [hcap] first list position of the slot's tokens
+  int* tok_slot;  // [T] slot of token t (-1 for a bad id)
+  int* tok_rank;  // [T] rank of token t in its id's group
+  int* tok_pos;   // [T] list position of token t (-1 for a bad id)
+  int* list;      // [T] tokens grouped by id
+  int4* items;    // [T + T / kItemTokens + 1] {id, first list position, tokens, 0}
+  float* gates;   // [T][NP] one layer's gates by list position
+  int hcap_log2;
+  size_t clear_bytes;  // key .. ctl, one contiguous range
+};
+
+int padded_experts(int N) { return N <= 8 ? 8 : N <= 16 ? 16 : 32; }
+
+// Carves the buffer at `base` (nullptr: size query); returns its size.
+size_t carve_ws(void* base, int64_t T, int NP, GroupWs* w) {
+  int lg = 10;
+  while ((int64_t(1) << lg) < 2 * T) ++lg;
+  const int64_t hcap = int64_t(1) << lg;
+  size_t off = 0;
+  auto take = [&off](size_t bytes) {
+    const size_t o = off;
+    off += (bytes + 255) / 256 * 256;
+    return o;
+  };
+  const size_t clear = 8 * (size_t)hcap + 4 * kCtlWords;
+  const size_t o_clear = take(clear);
+  const size_t o_off = take(4 * (size_t)hcap);
+  const size_t o_tslot = take(4 * (size_t)T);
+  const size_t o_trank = take(4 * (size_t)T);
+  const size_t o_tpos = take(4 * (size_t)T);
+  const size_t o_list = take(4 * (size_t)T);
+  const size_t o_items = take(16 * (size_t)(T + T / kItemTokens + 1));
+  const size_t o_gates = take(4 * (size_t)T * NP);
+  if (w != nullptr && base != nullptr) {
+    uint8_t* b = static_cast<uint8_t*>(base);
+    w->key = reinterpret_cast<int*>(b + o_clear);
+    w->cnt = w->key + hcap;
+    w->ctl = reinterpret_cast<unsigned*>(w->cnt + hcap);
+    w->off = reinterpret_cast<int*>(b + o_off);
+    w->tok_slot = reinterpret_cast<int*>(b + o_tslot);
+    w->tok_rank = reinterpret_cast<int*>(b + o_trank);
+    w->tok_pos = reinterpret_cast<int*>(b + o_tpos);
+    w->list = reinterpret_cast<int*>(b + o_list);
+    w->items = reinterpret_cast<int4*>(b + o_items);
+    w->gates = reinterpret_cast<float*>(b + o_gates);
+    w->hcap_log2 = lg;
+    w->clear_bytes = clear;
+  }
+  return off;
+}
+
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ unsigned ld_relaxed_u32(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+
+// Grid-wide barrier of a cooperative launch, split in two so that work can
+// run between the arrival and the wait; `counter` starts at 0xFFFFFFFF and
+// serves one barrier per call.  grid_arrive publishes this CTA's earlier
+// writes and counts it in.
+__device__ __forceinline__ void grid_arrive(unsigned* counter) {
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) atomicAdd(counter, 1u);
+}
+
+// Waits until every CTA has arrived.  Bounded: after kWaitLimitNs, or when
+// another CTA has given up, it returns false (the giving-up CTA sets the
+// abort word and the timeout bit).
+__device__ bool grid_wait(unsigned* counter, unsigned* abort_word, unsigned* err, int* flag) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    const unsigned target = gridDim.x - 1u;
+    if (ld_acquire(counter) != target) {
+      const uint64_t t0 = globaltimer();
+      while (ld_acquire(counter) != target) {
+        if (ld_acquire(abort_word) != 0xFFFFFFFFu) {
+          ok = 0;
+          break;
+        }
+        if (globaltimer() - t0 > kWaitLimitNs) {
+          atomicExch(abort_word, 1u);
+          atomicOr(err, kErrTimeout);
+          ok = 0;
+          break;
+        }
+      }
+    }
+    __threadfence();
+    *flag = ok;
+  }
+  __syncthreads();
+  return *flag != 0;
+}
+
+// Exclusive scan of (a, b) over the CTA in thread order; totals in (ta, tb).
+// `red` holds 2 * kWarps ints.
+__device__ __forceinline__ void block_scan2(int& a, int& b, int& ta, int& tb, int* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int ia = a, ib = b;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int x = __shfl_up_sync(0xffffffffu, ia, o), y = __shfl_up_sync(0xffffffffu, ib, o);
+    if (lane >= o) {
+      ia += x;
+      ib += y;
+    }
+  }
+  if (lane == 31) {
+    red[2 * warp] = ia;
+    red[2 * warp + 1] = ib;
+  }
+  __syncthreads();
+  int wa = 0, wb = 0, sa = 0, sb = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    const int x = red[2 * w], y = red[2 * w + 1];
+    if (w < warp) {
+      wa += x;
+      wb += y;
+    }
+    sa += x;
+    sb += y;
+  }
+  __syncthreads();
+  a = wa + ia - a;
+  b = wb + ib - b;
+  ta = sa;
+  tb = sb;
+}
+
+// Slot of `id` in the hash table (linear probing), inserting it if new.
+__device__ __forceinline__ int plan_insert(const GroupWs& w, int id) {
+  const unsigned mask = (1u << w.hcap_log2) - 1u;
+  unsigned hh = ((unsigned)id * 2654435761u) >> (32 - w.hcap_log2);
+  for (unsigned probe = 0; probe <= mask; ++probe) {
+    const int k = atomicCAS(&w.key[hh], -1, id);
+    if (k == -1 || k == id) return (int)hh;
+    hh = (hh + 1u) & mask;
+  }
+  return -1;  // not reached: the table has at least 2T slots
+}
+
+// This CTA's range [s0, s1) of hash-table slots.
+__device__ __forceinline__ void slot_range(const GroupWs& w, int64_t& s0, int64_t& s1) {
+  const int64_t hcap = int64_t(1) << w.hcap_log2;
+  s0 = (int64_t)blockIdx.x * hcap / gridDim.x;
+  s1 = ((int64_t)blockIdx.x + 1) * hcap / gridDim.x;
+}
+
+__device__ __forceinline__ int warp_sum(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Step 1: token and per-size item totals of this CTA's slot range, added to
+// the grid totals; the values the totals had before (in whatever order the
+// CTAs arrive) become this CTA's bases within each region.  `cls` and
+// `cbase` are kAgg ints of shared memory.
+__device__ void plan_count(const GroupWs& w, int* cls, int* cbase) {
+  int64_t s0, s1;
+  slot_range(w, s0, s1);
+  if (threadIdx.x < kAgg) cls[threadIdx.x] = 0;
+  __syncthreads();
+  int sc = 0;
+  for (int64_t h = s0 + threadIdx.x; h < s1; h += kThreads) {
+    if (w.key[h] == -1) continue;
+    const int c = w.cnt[h] + 1;
+    sc += c;
+    if (c >= kItemTokens) atomicAdd(&cls[kItemTokens], c / kItemTokens);
+    if (c % kItemTokens) atomicAdd(&cls[c % kItemTokens], 1);
+  }
+  sc = warp_sum(sc);
+  if ((threadIdx.x & 31) == 0 && sc) atomicAdd(&cls[0], sc);
+  __syncthreads();
+  if (threadIdx.x < kAgg) {
+    const int v = cls[threadIdx.x];
+    cbase[threadIdx.x] = v ? (int)(atomicAdd(&w.ctl[kCtlTot + threadIdx.x], (unsigned)v) + 1u) : 0;
+  }
+}
+
+// Step 2: list offsets and item records of this CTA's slot range.  Items are
+// laid out by size, largest first (all full items, then 15-token items, ...),
+// so dealing them round-robin to the gather CTAs spreads the tokens evenly.
+// `cur` is kAgg ints of shared memory, `red` 2 * kWarps.
+__device__ void plan_offsets(const GroupWs& w, const int* cbase, int* cur, int* red) {
+  int64_t s0, s1;
+  slot_range(w, s0, s1);
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int n = kItemTokens; n >= 1; --n) {
+      cur[n] = acc + cbase[n];
+      acc += (int)(ld_relaxed_u32(&w.ctl[kCtlTot + n]) + 1u);  // ordered by the grid barrier
+    }
+    if (blockIdx.x == 0) w.ctl[kCtlItems] = (unsigned)acc;
+  }
+  __syncthreads();
+  int bt = cbase[0];
+  for (int64_t base = s0; base < s1; base += kThreads) {
+    const int64_t h = base + threadIdx.x;
+    const int id = h < s1 ? w.key[h] : -1;
+    const int c = id != -1 ? w.cnt[h] + 1 : 0;
+    int pc = c, unused = 0, sc, su;
+    block_scan2(pc, unused, sc, su, red);
+    if (id != -1) {
+      const int o = bt + pc;
+      w.off[h] = o;
+      const int nf = c / kItemTokens, r = c % kItemTokens;
+      if (nf) {
+        const int p0 = atomicAdd(&cur[kItemTokens], nf);
+        for (int k = 0; k < nf; ++k) w.items[p0 + k] = make_int4(id, o + k * kItemTokens, kItemTokens, 0);
+      }
+      if (r) w.items[atomicAdd(&cur[r], 1)] = make_int4(id, o + nf * kItemTokens, r, 0);
+    }
+    bt += sc;
+  }
+}
+
+// This CTA's contiguous range [t0, t1) of the batch's tokens.
+__device__ __forceinline__ void token_range(int64_t T, int64_t& t0, int64_t& t1) {
+  t0 = (int64_t)blockIdx.x * T / gridDim.x;
+  t1 = ((int64_t)blockIdx.x + 1) * T / gridDim.x;
+}
+
+// Step 0: insert this CTA's tokens and rank them inside their id's group.
+__device__ void plan_insert_tokens(const int32_t* __restrict__ ids, int64_t T, int64_t V, const GroupWs& w,
+                                   unsigned* err) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int64_t t0, t1;
+  token_range(T, t0, t1);
+  for (int64_t base = t0 + (int64_t)warp * 32; base < t1; base += kPlanThreads) {
+    const int64_t t = base + lane;
+    const bool act = t < t1;
+    const int id = act ? __ldg(ids + t) : -1;
+    const bool good = act && id >= 0 && (int64_t)id < V;
+    if (act && !good) atomicOr(err, kErrIndex);
+    // one insert per distinct id of the warp (the leader's), shared by shuffle
+    const unsigned same = __match_any_sync(0xffffffffu, good ? id : -1);
+    const int lead = __ffs(same) - 1;
+    int slot = (good && lane == lead) ? plan_insert(w, id) : -1;
+    slot = __shfl_sync(0xffffffffu, slot, lead);
+    if (!good) slot = -1;
+    // one atomicAdd per distinct slot of the warp; ranks by lane order
+    const unsigned peers = __match_any_sync(0xffffffffu, slot);
+    const int leader = __ffs(peers) - 1;
+    int first = 0;
+    if (slot >= 0 && lane == leader) first = atomicAdd(&w.cnt[slot], __popc(peers)) + 1;
+    first = __shfl_sync(0xffffffffu, first, leader);
+    if (act) {
+      w.tok_slot[t] = slot;
+      w.tok_rank[t] = first + __popc(peers & ((1u << lane) - 1u));
+    }
+  }
+}
+
+// Step 3: every token of this CTA to its list position.
+__device__ void plan_scatter(const GroupWs& w, int64_t T) {
+  int64_t t0, t1;
+  token_range(T, t0, t1);
+  for (int64_t t = t0 + threadIdx.x; t < t1; t += kPlanThreads) {
+    const int slot = w.tok_slot[t];
+    const int pos = slot >= 0 ? w.off[slot] + w.tok_rank[t] : -1;
+    w.tok_pos[t] = pos;
+    if (pos >= 0) w.list[pos] = (int)t;
+  }
+}
+
+__global__ void __launch_bounds__(kPlanThreads) group_plan_kernel(const int32_t* __restrict__ ids, int64_t T,
+                                                                   int64_t V, const GroupWs w, unsigned* err) {
+  __shared__ int red[2 * kWarps];
+  __shared__ int cls[kAgg], cbase[kAgg];
+  __shared__ int flag;
+  plan_insert_tokens(ids, T, V, w, err);
+  grid_arrive(&w.ctl[kCtlBar + 0]);
+  bool ok = grid_wait(&w.ctl[kCtlBar + 0], &w.ctl[kCtlAbort], err, &flag);
+  if (ok) plan_count(w, cls, cbase);
+  grid_arrive(&w.ctl[kCtlBar + 1]);
+  if (ok) ok = grid_wait(&w.ctl[kCtlBar + 1], &w.ctl[kCtlAbort], err, &flag);
+  if (ok) plan_offsets(w, cbase, cls, red);
+  grid_arrive(&w.ctl[kCtlBar + 2]);
+  if (ok) ok = grid_wait(&w.ctl[kCtlBar + 2], &w.ctl[kCtlAbort], err, &flag);
+  if (ok) plan_scatter(w, T);
+}
+
+struct GArgs {
+  int64_t T;
+  const uint16_t* h;
+  const uint16_t* Wr;
+  const uint16_t* table;
+  int N, D;
+  float* out;
+  unsigned* err;
+};
+
+// One layer's router: gates to the tokens' list positions; a token with a
+// bad id gets a NaN output row (and the index bit of the error word).
+template <int NT>
+__global__ void __launch_bounds__(kThreads, 2) router_group_kernel(const GArgs p, const GroupWs w) {
+  constexpr int NP = 8 * NT;
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  const Smem s = carve<true, NP>(smem_raw, p.D);
+  // list positions of the tile's tokens, loaded one tile ahead (thread r < 16)
+  int pos_next = -1;
+  {
+    const int64_t t = (int64_t)blockIdx.x * kTileMax + threadIdx.x;
+    if (threadIdx.x < kTileMax && t < p.T) pos_next = w.tok_pos[t];
+  }
+  router_tiles<NT>(s, p.h, p.Wr, p.T, p.N, p.D, [&](int64_t t0, int rows) {
+    if (threadIdx.x < kTileMax) {
+      s.tok_id[threadIdx.x] = pos_next;
+      const int64_t tn = t0 + (int64_t)gridDim.x * kTileMax + threadIdx.x;
+      pos_next = tn < p.T ? w.tok_pos[tn] : -1;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < rows * NP; i += kThreads) {
+      const int r = i / NP, j = i - r * NP;
+      const int pos = s.tok_id[r];
+      if (pos >= 0) w.gates[(int64_t)pos * NP + j] = s.gates[i];
+    }
+    for (int r = 0; r < rows; ++r) {
+      if (s.tok_id[r] >= 0) continue;
+      if (threadIdx.x == 0) atomicOr(p.err, kErrIndex);
+      float* o = p.out + (t0 + r) * p.D;
+      for (int d = 4 * threadIdx.x; d < p.D; d += 4 * kThreads)
+        __stcs(reinterpret_cast<float4*>(o + d), make_float4(NAN, NAN, NAN, NAN));
+    }
+  });
+}
+
+// Slot layout: [0, gates_off) the id's row block (N rows of D bf16),
+// [gates_off, + kItemTokens * NP * 4) the gates of the item's tokens.
+struct GroupLayout {
+  int n_slots, slot_bytes, gates_off;
+};
+
+// 8 consumer warps + 1 producer warp: 3 warps per scheduler, so a thread may
+// hold 168 registers -- the N rows of its 4-element vector stay in registers
+// in fp32 (up to 16 experts) while it serves every token of the item.
+constexpr int kGroupCons = 8;
+constexpr bool kPairTokens = true;
+
+// bf16 -> fp32 through opaque instructions: the compiler keeps the converted
+// values in registers across the item's tokens instead of converting again
+// per token (which it otherwise prefers, to save registers).
+__device__ __forceinline__ float bf16_lo_held(uint32_t x) {
+  uint32_t u;
+  asm volatile("shl.b32 %0, %1, 16;" : "=r"(u) : "r"(x));
+  return __uint_as_float(u);
+}
+__device__ __forceinline__ float bf16_hi_held(uint32_t x) {
+  uint32_t u;
+  asm volatile("and.b32 %0, %1, 0xffff0000;" : "=r"(u) : "r"(x));
+  return __uint_as_float(u);
+}
+constexpr int kGroupThreads = (kGroupCons + 1) * 32;
+constexpr int kGroupProducer = kGroupCons;
+
+// out[t, 4v .. 4v+3] for one token from the N rows of the unit (x, fp32 or
+// packed bf16 pairs) and the token's gates g (NP floats in shared memory).
+template <int NP, bool kExactN, bool kPacked>
+__device__ __forceinline__ float4 combine_unit(const float (&xf)[kPacked ? 1 : NP][4], const uint2 (&xp)[kPacked ? NP : 1],
+                                               const float* g, int N) {
+  const float4* g4 = reinterpret_cast<const float4*>(g);
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+  for (int jq = 0; jq < NP / 4; ++jq) {
+    const float4 gv = g4[jq];
+    const float gg[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int j = 4 * jq + e;
+      if (kExactN || j < N) {
+        float x0, x1, x2, x3;
+        if (kPacked) {
+          const uint2 r = xp[kPacked ? j : 0];
+          x0 = bf16_lo(r.x);
+          x1 = bf16_hi(r.x);
+          x2 = bf16_lo(r.y);
+          x3 = bf16_hi(r.y);
+        } else {
+          x0 = xf[kPacked ? 0 : j][0];
+          x1 = xf[kPacked ? 0 : j][1];
+          x2 = xf[kPacked ? 0 : j][2];
+          x3 = xf[kPacked ? 0 : j][3];
+        }
+        a0 = fmaf(gg[e], x0, a0);
+        a1 = fmaf(gg[e], x1, a1);
+        a2 = fmaf(gg[e], x2, a2);
+        a3 = fmaf(gg[e], x3, a3);
+      }
+    }
+  }
+  return make_float4(a0, a1, a2, a3);
+}
+
+template <int NT, bool kExactN>
+__global__ void __launch_bounds__(kGroupThreads, 1) grouped_gather_kernel(const GArgs p, const GroupWs w,
+                                                                          const GroupLayout L) {
+  constexpr int NP = 8 * NT;
+  constexpr int C = kItemTokens;
+  constexpr bool kPacked = NP > 16;  // 32 experts: keep rows as bf16 pairs, convert per token
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  uint8_t* ring = smem_raw;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw + (size_t)L.n_slots * L.slot_bytes);
+  uint64_t* empty = full + L.n_slots;
+  int* slot_n = reinterpret_cast<int*>(empty + L.n_slots);
+  int* slot_tok = slot_n + L.n_slots;  // [n_slots][C]
+  int* abort_flag = slot_tok + L.n_slots * C;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int q = 0; q < L.n_slots; ++q) {
+      mbar_init(&full[q], 2);  // the copies' arrive.expect_tx + the token list's arrive
+      mbar_init(&empty[q], kGroupCons);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (ld_relaxed_u32(&w.ctl[kCtlAbort]) != 0xFFFFFFFFu) return;  // plan abandoned (error word set)
+  volatile int* abort = abort_flag;
+  const int n_items = (int)ld_relaxed_u32(&w.ctl[kCtlItems]);
+  const int my_n = n_items > (int)blockIdx.x ? (n_items - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
+  const uint32_t row_bytes = (uint32_t)p.N * (uint32_t)p.D * 2u;
+
+  if (warp == kGroupProducer) {
+    // ---------------- producer ----------------
+    // item records 32 at a time (one per lane); each item's tokens are
+    // loaded one item ahead
+    // The CTA's items are items[blockIdx.x + m * gridDim.x], m = 0 .. my_n-1,
+    // largest first.  Step k takes them alternately from the front and the
+    // back (large, small, large, ...), so the copies of small items proceed
+    // while the consumers work through large ones.
+    auto record = [&](int kk) {
+      const int m = (kk & 1) ? my_n - 1 - (kk >> 1) : (kk >> 1);
+      return kk < my_n ? w.items[blockIdx.x + (size_t)m * gridDim.x] : make_int4(0, 0, 0, 0);
+    };
+    // records of steps k0 + lane (my_item) and k0 + 32 + lane (nx_item)
+    int k0 = 0;
+    int4 my_item = record(lane);
+    int4 nx_item = record(32 + lane);
+    int next_tok = -1;
+    if (my_n > 0) {
+      const int pos = __shfl_sync(0xffffffffu, my_item.y, 0), n = __shfl_sync(0xffffffffu, my_item.z, 0);
+      next_tok = lane < n ? w.list[pos + lane] : -1;
+    }
+    uint32_t q = 0, ph = 0, issued = 0;
+    bool ok = true;
+    for (int k = 0; ok && k < my_n; ++k) {
+      const int id = __shfl_sync(0xffffffffu, my_item.x, k - k0);
+      const int pos = __shfl_sync(0xffffffffu, my_item.y, k - k0);
+      const int n = __shfl_sync(0xffffffffu, my_item.z, k - k0);
+      const int tok = next_tok;
+      if (k + 1 < my_n) {  // prefetch the next item's record batch and tokens
+        if (k + 1 - k0 == 32) {
+          k0 = k + 1;
+          my_item = nx_item;
+          nx_item = record(k0 + 32 + lane);
+        }
+        const int pos1 = __shfl_sync(0xffffffffu, my_item.y, k + 1 - k0);
+        const int n1 = __shfl_sync(0xffffffffu, my_item.z, k + 1 - k0);
+        next_tok = lane < n1 ? w.list[pos1 + lane] : -1;
+      }
+      ok = warp_wait(&empty[q], ph ^ 1u, abort, p.err);
+      if (!ok) break;
+      uint8_t* slot = ring + (size_t)q * L.slot_bytes;
+      // the copies first; the token list (loaded one item ahead) after them
+      if (lane == 0) {
+        const uint32_t gate_bytes = (uint32_t)n * NP * 4u;
+        mbar_expect_tx(&full[q], row_bytes + gate_bytes);
+        bulk_g2s(slot, p.table + (int64_t)id * p.N * p.D, row_bytes, &full[q]);
+        bulk_g2s(slot + L.gates_off, w.gates + (int64_t)pos * NP, gate_bytes, &full[q]);
+      }
+      if (lane < n) slot_tok[q * C + lane] = tok;
+      if (lane == 0) slot_n[q] = n;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&full[q]);
+      ++issued;
+      if (++q == (uint32_t)L.n_slots) {
+        q = 0;
+        ph ^= 1u;
+      }
+    }
+    if (lane == 0) {  // the last copies must have landed before the CTA exits
+      for (uint32_t i = 0; i < issued && i < (uint32_t)L.n_slots; ++i) {
+        q = q == 0 ? L.n_slots - 1 : q - 1;
+        if (q == (uint32_t)L.n_slots - 1) ph ^= 1u;
+        mbar_drain(&full[q], ph);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------- consumers ----------------
+    // unit = 4 consecutive elements of D; with fewer units than consumer
+    // threads, Gt thread groups split the item's tokens
+    const int lt = threadIdx.x;
+    const int units = p.D >> 2;
+    constexpr int kCT = kGroupCons * 32;
+    const int Gt = units >= kCT ? 1 : kCT / units;
+    const int grp = units >= kCT ? 0 : lt / units;
+    const int v0 = units >= kCT ? lt : lt - grp * units;
+    const int vstep = units >= kCT ? kCT : units;
+    const bool active = grp < Gt;
+    uint32_t q = 0, ph = 0;
+    for (int k = 0; k < my_n; ++k) {
+      if (!warp_wait(&full[q], ph, abort, p.err)) break;
+      if (active) {
+        const int n = slot_n[q];
+        const uint8_t* slot = ring + (size_t)q * L.slot_bytes;
+        const float* gs = reinterpret_cast<const float*>(slot + L.gates_off);
+        for (int v = v0; v < units; v += vstep) {
+          float xf[kPacked ? 1 : NP][4];
+          uint2 xp[kPacked ? NP : 1];
+#pragma unroll
+          for (int j = 0; j < NP; ++j) {
+            uint2 r = make_uint2(0u, 0u);
+            if (kExactN || j < p.N) r = *reinterpret_cast<const uint2*>(slot + ((size_t)j * p.D + 4 * v) * 2);
+            if (kPacked) {
+              xp[kPacked ? j : 0] = r;
+            } else {
+              xf[kPacked ? 0 : j][0] = bf16_lo_held(r.x);
+              xf[kPacked ? 0 : j][1] = bf16_hi_held(r.x);
+              xf[kPacked ? 0 : j][2] = bf16_lo_held(r.y);
+              xf[kPacked ? 0 : j][3] = bf16_hi_held(r.y);
+            }
+          }
+          int i = grp;
+          // two tokens at a time (8 independent FMA chains); one at a time with
+          // packed rows, where a pair would convert every row twice at once
+          for (; kPairTokens && !kPacked && i + Gt < n; i += 2 * Gt) {
+            const float4 o0 = combine_unit<NP, kExactN, kPacked>(xf, xp, gs + i * NP, p.N);
+            const float4 o1 = combine_unit<NP, kExactN, kPacked>(xf, xp, gs + (i + Gt) * NP, p.N);
+            __stcs(reinterpret_cast<float4*>(p.out + (int64_t)slot_tok[q * C + i] * p.D + 4 * v), o0);
+            __stcs(reinterpret_cast<float4*>(p.out + (int64_t)slot_tok[q * C + i + Gt] * p.D + 4 * v), o1);
+          }
+          for (; i < n; i += Gt) {
+            const float4 o0 = combine_unit<NP, kExactN, kPacked>(xf, xp, gs + i * NP, p.N);
+            __stcs(reinterpret_cast<float4*>(p.out + (int64_t)slot_tok[q * C + i] * p.D + 4 * v), o0);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[q]);
+      if (++q == (uint32_t)L.n_slots) {
+        q = 0;
+        ph ^= 1u;
+      }
+    }
+  }
+  __syncthreads();
+}
+
+template <int NT, bool kExactN>
+mole_status launch_layer(const GArgs& p, const GroupWs& w, cudaStream_t stream) {
+  constexpr int NP = 8 * NT;
+  constexpr int C = kItemTokens;
+  GroupLayout L{};
+  const int64_t row_bytes = (int64_t)p.N * p.D * 2;
+  L.gates_off = (int)((row_bytes + 127) / 128 * 128);
+  L.slot_bytes = (int)((L.gates_off + (int64_t)C * NP * 4 + 127) / 128 * 128);
+  L.n_slots = (int)std::min<int64_t>(16, kRingBudget / L.slot_bytes);
+  if (L.n_slots < 2) return MOLE_ERR_UNSUPPORTED;
+  const size_t gsmem = (size_t)L.n_slots * L.slot_bytes + (size_t)L.n_slots * (16 + 4 + 4 * C) + 16;
+  const size_t rsmem = smem_bytes_for<true, NP>(p.D);
+  if (gsmem > 227 * 1024 || rsmem > 227 * 1024) return MOLE_ERR_UNSUPPORTED;
+  auto rkern = router_group_kernel<NT>;
+  auto gkern = grouped_gather_kernel<NT, kExactN>;
+  if (cudaFuncSetAttribute(rkern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem) != cudaSuccess ||
+      cudaFuncSetAttribute(gkern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gsmem) != cudaSuccess)
+    return MOLE_ERR_CUDA;
+  const int n_sm = num_sms();
+  if (n_sm <= 0) return MOLE_ERR_NO_DEVICE;
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, rkern, kThreads, rsmem) != cudaSuccess || occ < 1)
+    return MOLE_ERR_UNSUPPORTED;
+  const int64_t n_tiles = (p.T + kTileMax - 1) / kTileMax;
+  rkern<<<(unsigned)std::min<int64_t>(n_tiles, (int64_t)occ * n_sm), kThreads, rsmem, stream>>>(p, w);
+  gkern<<<(unsigned)n_sm, kGroupThreads, gsmem, stream>>>(p, w, L);
+  return cuda_status(cudaGetLastError());
+}
+
+mole_status layer_dispatch(const GArgs& p, const GroupWs& w, cudaStream_t stream) {
+  if (p.N == 16) return launch_layer<2, true>(p, w, stream);
+  if (p.N == 8) return launch_layer<1, true>(p, w, stream);
+  if (p.N < 8) return launch_layer<1, false>(p, w, stream);
+  if (p.N < 16) return launch_layer<2, false>(p, w, stream);
+  if (p.N == 32) return launch_layer<4, true>(p, w, stream);
+  return launch_layer<4, false>(p, w, stream);
+}
+
+// Whether the grouped kernels take a call of this shape (else the
+// mole_lookup_combine kernels do, and the grouping is not used).
+bool grouped_applies(int64_t T, int N, int D) {
+  if (T < kGroupedMinT || T > kGroupedMaxT || N < 1 || N > 32) return false;
+  const int64_t slot = ((int64_t)N * D * 2 + 127) / 128 * 128 + (int64_t)kItemTokens * padded_experts(N) * 4;
+  return kRingBudget / slot >= 2 && smem_bytes_for<true, 32>(D) <= 227 * 1024;
+}
+
+}  // namespace
+
+size_t token_groups_bytes(int64_t T, int N) {
+  if (T <= 0 || N <= 0 || N > 32) return 0;
+  return carve_ws(nullptr, T, padded_experts(N), nullptr);
+}
+
+mole_status token_groups_build(const int32_t* ids, int64_t T, int64_t V, int N, void* buf, size_t bytes,
+                               cudaStream_t stream) {
+  if (T > kGroupedMaxT) return MOLE_ERR_UNSUPPORTED;
+  GroupWs w{};
+  if (carve_ws(buf, T, padded_experts(N), &w) > bytes) return MOLE_ERR_WORKSPACE;
+  unsigned* err = error_word();
+  if (!err) return MOLE_ERR_CUDA;
+  const int n_sm = num_sms();
+  if (n_sm <= 0) return MOLE_ERR_NO_DEVICE;
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, group_plan_kernel, kPlanThreads, 0) != cudaSuccess ||
+      occ < 1)
+    return MOLE_ERR_UNSUPPORTED;
+  const int64_t grid =
+      std::min<int64_t>(std::min<int64_t>((T + kPlanThreads - 1) / kPlanThreads, (int64_t)occ * n_sm), kPlanMaxGrid);
+  if (cudaMemsetAsync(w.key, 0xFF, w.clear_bytes, stream) != cudaSuccess) return MOLE_ERR_CUDA;
+  // cooperative launch: the grid barriers need every CTA resident
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)std::max<int64_t>(grid, 1));
+  cfg.blockDim = dim3(kPlanThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, group_plan_kernel, ids, T, V, w, err) != cudaSuccess) return MOLE_ERR_CUDA;
+  return MOLE_OK;
+}
+
+mole_status combine_groups(const void* buf, size_t bytes, int64_t T, const void* h, const void* Wr,
+                           const void* table, int N, int D, float* out, cudaStream_t stream) {
+  GroupWs w{};
+  if (carve_ws(const_cast<void*>(buf), T, padded_experts(N), &w) > bytes) return MOLE_ERR_WORKSPACE;
+  if (!grouped_applies(T, N, D)) return MOLE_ERR_UNSUPPORTED;
+  GArgs p{};
+  p.T = T;
+  p.h = static_cast<const uint16_t*>(h);
+  p.Wr = static_cast<const uint16_t*>(Wr);
+  p.table = static_cast<const uint16_t*>(table);
+  p.N = N;
+  p.D = D;
+  p.out = out;
+  p.err = error_word();
+  if (!p.err) return MOLE_ERR_CUDA;
+  return layer_dispatch(p, w, stream);
+}
+
+mole_status combine_grouped_dispatch(const int32_t* ids, int64_t T, const void* h, const void* Wr,
+                                     const void* table, const uint16_t* scales, int64_t V, int N, int D,
+                                     bool bf16_inputs, int table_kind, float* out, void* ws, size_t ws_bytes,
+                                     cudaStream_t stream) {
+  if (bf16_inputs && table_kind == 0 && grouped_applies(T, N, D) && aligned16(Wr) && aligned16(table)) {
+    mole_status st = token_groups_build(ids, T, V, N, ws, ws_bytes, stream);
+    if (st != MOLE_OK) return st;
+    return combine_groups(ws, ws_bytes, T, h, Wr, table, N, D, out, stream);
+  }
+  return combine_dispatch(ids, T, h, Wr, table, scales, V, N, D, bf16_inputs, table_kind, out, stream);
+}
+
+}  // namespace mole

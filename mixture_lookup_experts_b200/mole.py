@@ -38,6 +38,11 @@ SIGNATURES = {
     "mole_build_lut": ([_P, _P, _P, _I64, _I64, _I32, _I64, _I, _I, _P, _P, _SZ, _P], _I),
     "mole_build_lut_noalloc": ([_P, _P, _P, _I64, _I64, _I32, _I64, _I, _I, _P, _P], _I),
     "mole_lookup_combine": ([_P, _I64, _P, _P, _P, _I64, _I32, _I64, _I, _P, _P], _I),
+    "mole_token_groups_workspace": ([_I64, _I32], _SZ),
+    "mole_token_groups_build": ([_P, _I64, _I64, _I32, _P, _SZ, _P], _I),
+    "mole_lookup_combine_groups": ([_P, _I64, _P, _SZ, _P, _P, _P, _I64, _I32, _I64, _I, _P, _P], _I),
+    "mole_lookup_combine_grouped_workspace": ([_I64, _I32], _SZ),
+    "mole_lookup_combine_grouped": ([_P, _I64, _P, _P, _P, _I64, _I32, _I64, _I, _P, _P, _SZ, _P], _I),
     "mole_quantize_lut_nf3": ([_P, _I64, _I32, _I64, _P, _P, _P], _I),
     "mole_lookup_combine_nf3": ([_P, _I64, _P, _P, _P, _P, _I64, _I32, _I64, _I, _P, _P], _I),
     "mole_nf3_levels": ([_P], None),
@@ -150,6 +155,62 @@ def mole_lookup_combine(ids: torch.Tensor, h: torch.Tensor, Wr: torch.Tensor, lu
         out = torch.empty((T, D), dtype=torch.float32, device=h.device)
     _ok(lib.mole_lookup_combine(_ptr(ids), T, _ptr(h), _ptr(Wr), _ptr(lut), V, N, D, _dt(h), _ptr(out),
                                 _stream(stream)), "mole_lookup_combine")
+    return out
+
+
+def mole_token_groups_workspace(T: int, N: int) -> int:
+    return int(lib.mole_token_groups_workspace(T, N))
+
+
+def mole_token_groups_build(ids: torch.Tensor, V: int, N: int, groups: torch.Tensor | None = None,
+                            stream=None) -> torch.Tensor:
+    """Groups the batch's tokens by id (once per batch; serves every layer
+    with N experts).  Returns the groups buffer (see mole.h)."""
+    _contig(ids, groups)
+    T = ids.numel()
+    if groups is None:
+        groups = torch.empty(max(1, mole_token_groups_workspace(T, N)), dtype=torch.uint8, device=ids.device)
+    nbytes = groups.numel() * groups.element_size()
+    _ok(lib.mole_token_groups_build(_ptr(ids), T, V, N, _ptr(groups), nbytes, _stream(stream)),
+        "mole_token_groups_build")
+    return groups
+
+
+def mole_lookup_combine_groups(ids: torch.Tensor, groups: torch.Tensor, h: torch.Tensor, Wr: torch.Tensor,
+                               lut: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """mole_lookup_combine over a grouping built from the same ids (each
+    distinct row block read once); same result bit for bit (see mole.h)."""
+    _contig(ids, groups, h, Wr, lut, out)
+    V, N, D = lut.shape
+    T = ids.numel()
+    if out is None:
+        out = torch.empty((T, D), dtype=torch.float32, device=h.device)
+    nbytes = groups.numel() * groups.element_size()
+    _ok(lib.mole_lookup_combine_groups(_ptr(ids), T, _ptr(groups), nbytes, _ptr(h), _ptr(Wr), _ptr(lut), V, N, D,
+                                       _dt(h), _ptr(out), _stream(stream)), "mole_lookup_combine_groups")
+    return out
+
+
+def mole_lookup_combine_grouped_workspace(T: int, N: int) -> int:
+    return int(lib.mole_lookup_combine_grouped_workspace(T, N))
+
+
+def mole_lookup_combine_grouped(ids: torch.Tensor, h: torch.Tensor, Wr: torch.Tensor, lut: torch.Tensor,
+                                out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                                stream=None) -> torch.Tensor:
+    """mole_lookup_combine with tokens grouped by id (each distinct row block
+    fetched once per batch); same result bit for bit (see mole.h)."""
+    _contig(ids, h, Wr, lut, out, workspace)
+    V, N, D = lut.shape
+    T = ids.numel()
+    if out is None:
+        out = torch.empty((T, D), dtype=torch.float32, device=h.device)
+    if workspace is None:
+        workspace = torch.empty(max(1, mole_lookup_combine_grouped_workspace(T, N)), dtype=torch.uint8,
+                                device=h.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _ok(lib.mole_lookup_combine_grouped(_ptr(ids), T, _ptr(h), _ptr(Wr), _ptr(lut), V, N, D, _dt(h), _ptr(out),
+                                        _ptr(workspace), ws_bytes, _stream(stream)), "mole_lookup_combine_grouped")
     return out
 
 

@@ -79,3 +79,40 @@ def test_valid_arguments_reach_the_device_check(mole):
     P = 0x100000
     # all checks pass, then there is no sm_100 device here
     assert mole.lib.mole_lookup_combine(P, 5, P, P, P, 10, 4, 64, 1, P, None) == 8
+
+
+def test_grouped_workspace_size_and_checks(mole):
+    size = mole.mole_lookup_combine_grouped_workspace
+    assert size(0, 16) == 0 and size(100, 0) == 0 and size(100, 33) == 0
+    s1, s2 = size(16384, 16), size(32768, 16)
+    # hash table (2T slots, 12 B each), 4 per-token int arrays, items, gates
+    assert s1 >= 16384 * (4 * 4 + 16 + 16 * 4) + 2 * 16384 * 12
+    assert s2 > s1 and size(16384, 32) > s1
+    lib = mole.lib
+    P = 0x100000
+    ws = size(5, 4)
+    assert lib.mole_lookup_combine_grouped(P, 5, P, P, P, 10, 4, 64, 1, P, None, ws, None) == 4      # no workspace
+    assert lib.mole_lookup_combine_grouped(P, 5, P, P, P, 10, 4, 64, 1, P, P, ws - 1, None) == 4     # too small
+    assert lib.mole_lookup_combine_grouped(P, 5, P, P, P, 10, 4, 64, 1, P, P + 8, ws, None) == 2     # misaligned
+    assert lib.mole_lookup_combine_grouped(P, 5, P, P, P, 10, 4, 24, 1, P, P, ws, None) == 3         # D % 16
+    assert lib.mole_lookup_combine_grouped(P, 0, P, P, P, 10, 4, 64, 1, P, None, 0, None) == 0       # T == 0
+    import torch
+    if not torch.cuda.is_available():
+        assert lib.mole_lookup_combine_grouped(P, 5, P, P, P, 10, 4, 64, 1, P, P, ws, None) == 8     # no device
+
+
+def test_token_groups_checks(mole):
+    lib = mole.lib
+    P = 0x100000
+    assert mole.mole_token_groups_workspace(16384, 16) == mole.mole_lookup_combine_grouped_workspace(16384, 16)
+    assert mole.mole_token_groups_workspace(16384, 8) < mole.mole_token_groups_workspace(16384, 16)
+    ws = mole.mole_token_groups_workspace(5, 4)
+    assert lib.mole_token_groups_build(P, 5, 10, 4, None, ws, None) == 4
+    assert lib.mole_token_groups_build(P, 5, 10, 4, P, ws - 1, None) == 4
+    assert lib.mole_token_groups_build(P, 5, 10, 4, P + 4, ws, None) == 2
+    assert lib.mole_token_groups_build(P, 5, 10, 40, P, ws, None) == 3
+    assert lib.mole_token_groups_build(None, 5, 10, 4, P, ws, None) == 1
+    assert lib.mole_token_groups_build(P, 0, 10, 4, None, 0, None) == 0
+    assert lib.mole_lookup_combine_groups(P, 5, None, ws, P, P, P, 10, 4, 64, 1, P, None) == 4
+    assert lib.mole_lookup_combine_groups(P, 5, P, ws, P, P, P, 10, 4, 24, 1, P, None) == 3
+    assert lib.mole_lookup_combine_groups(P, 0, None, 0, P, P, P, 10, 4, 64, 1, P, None) == 0
