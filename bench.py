@@ -46,14 +46,15 @@ from mixture_lookup_experts_b200 import inputs  # noqa: E402
 METRIC = "MoLE lookup-combine tokens/s & HBM GB/s vs 8 TB/s; LUT build TFLOP/s"
 UNIT = "tokens/s"
 KERNEL_SOURCES = ["mixture_lookup_experts_b200/csrc/combine.cu", "mixture_lookup_experts_b200/csrc/grouped.cu",
-                  "mixture_lookup_experts_b200/csrc/combine_common.cuh", "mixture_lookup_experts_b200/csrc/common.cuh"]
+                  "mixture_lookup_experts_b200/csrc/router_tc.cu", "mixture_lookup_experts_b200/csrc/combine_common.cuh",
+                  "mixture_lookup_experts_b200/csrc/common.cuh"]
 PROFILE_SUMMARY = {"grouped": "profiles/combine_grouped_bf16_1b_T16384_zipf.md",
                    "plain": "profiles/combine_bf16_1b_T16384_zipf.md"}
 KERNELS = {
-    "grouped": "mole_lookup_combine_groups = router_group_kernel (tensor-core router, gates to the tokens' list "
-               "positions) + grouped_gather_kernel (one bulk copy per distinct row block, all of its tokens combined "
-               "from shared memory); duration = the call (the per-step grouping is timed apart)",
-    "plain": "mole_lookup_combine = router_gates_kernel (tensor-core router, gates parked in the output rows) + "
+    "grouped": "mole_lookup_combine_groups = router_tc_kernel (tcgen05 router, TMA-streamed h, gates to the tokens' "
+               "list positions) + grouped_gather_kernel (one bulk copy per distinct row block, all of its tokens "
+               "combined from shared memory); duration = the call (the per-step grouping is timed apart)",
+    "plain": "mole_lookup_combine = router_tc_kernel (tcgen05 router, gates parked in the output rows) + "
              "gather_kernel (bulk-copy ring of row blocks, consumer warps); duration = the call",
 }
 

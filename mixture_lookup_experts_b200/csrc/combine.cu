@@ -280,6 +280,8 @@ __global__ void __launch_bounds__(kGatherThreads, 1) gather_kernel(const Combine
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
+  pdl_trigger();
+  pdl_wait();  // the router's gates are complete
   volatile int* abort = abort_flag;
   const int NB = p.D >> 6;
   // bytes of one chunk of a token's row block (bf16: JC rows of D; NF3: all
@@ -513,7 +515,8 @@ __global__ void __launch_bounds__(kThreads, 2) combine_kernel(const CombineArgs 
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const Smem s = carve<kBf16Router, NP>(smem_raw, p.D);
   if (kBf16Router) {
-    stage_wrt<NP, kThreads>(s.wrt, static_cast<const uint16_t*>(p.Wr), p.N, p.D);
+    // (the element-wise staging: the fused kernel's registers are spoken for)
+    stage_wrt<NP, kThreads, false>(s.wrt, static_cast<const uint16_t*>(p.Wr), p.N, p.D);
     __syncthreads();
   }
   const int per_tok = kTable == kTableBf16 ? (p.D >> 3) : kTable == kTableF32 ? (p.D >> 2) : (p.D >> 5);
@@ -607,9 +610,16 @@ mole_status launch_two_kernel(CombineArgs p, cudaStream_t stream) {
   int occ = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, rkern, kThreads, rsmem) != cudaSuccess || occ < 1)
     return MOLE_ERR_UNSUPPORTED;
-  rkern<<<(unsigned)std::min<int64_t>(p.n_tiles, (int64_t)occ * n_sm), kThreads, rsmem, stream>>>(p);
-  gkern<<<(unsigned)std::min<int64_t>(p.T, n_sm), kGatherThreads, gsmem, stream>>>(p, L);
-  return cuda_status(cudaGetLastError());
+  if (router_tc_supported(p.T, p.N, p.D, p.h, p.Wr)) {
+    const mole_status st = router_tc_launch(p.h, p.Wr, p.T, p.D, false, p.out, nullptr, nullptr, stream);
+    if (st != MOLE_OK) return st;
+  } else if (launch_pdl(rkern, (unsigned)std::min<int64_t>(p.n_tiles, (int64_t)occ * n_sm), kThreads, rsmem, stream,
+                        p) != cudaSuccess) {
+    return MOLE_ERR_CUDA;
+  }
+  if (launch_pdl(gkern, (unsigned)std::min<int64_t>(p.T, n_sm), kGatherThreads, gsmem, stream, p, L) != cudaSuccess)
+    return MOLE_ERR_CUDA;
+  return MOLE_OK;
 }
 
 // Batches of at least kTwoKernelMinT tokens (bf16 inputs, bf16 or NF3 table)

@@ -79,31 +79,44 @@ __device__ __forceinline__ Smem carve(uint8_t* base, int D) {
 }
 
 // Stage Wr^T in shared memory: wrt[j][d] = Wr[d][j] (bf16), zero rows j >= N.
-// Loads are issued in batches of 8 per thread before their stores so their
-// latencies overlap (a dependent load per element would serialise them).
-template <int NP, int kNThreads, int kDepth = 16>
+// Fast path (N == NP, 16-byte aligned Wr, D % 8 == 0): each thread takes 8
+// consecutive rows d0..d0+7 and, per 8-expert slice and 4 rows at a time,
+// loads their 16-byte pieces, transposes the 4 x 8 bf16 block in registers
+// (byte permutes) and writes 8-byte pieces of 8 rows of wrt.
+// Otherwise element by element, loads issued in batches before their stores
+// so their latencies overlap.
+template <int NP, int kNThreads, bool kFast = true>
 __device__ __forceinline__ void stage_wrt(uint16_t* wrt, const uint16_t* __restrict__ wr, int N, int D) {
   const int ldw = D + 8;
-  if (N == NP && (reinterpret_cast<uintptr_t>(wr) & 15u) == 0) {
-    // 16-byte loads of 8 experts of one row d, kDepth per thread in flight
-    const int total8 = D * NP / 8;
-    for (int base = threadIdx.x; base < total8; base += kNThreads * kDepth) {
-      uint4 v[kDepth];
+  if (kFast && N == NP && (reinterpret_cast<uintptr_t>(wr) & 15u) == 0 && (D & 7) == 0) {
+    constexpr int Q = NP / 8;  // 16-byte pieces of a Wr row
+    // every CTA reads all of Wr at about the same moment: each starts at a
+    // different row so the requests spread over the L2 slices
+    const int n_tasks = D >> 3;
+    const int rot = (int)((blockIdx.x * 97u) % (unsigned)n_tasks);
+    for (int k = threadIdx.x; k < n_tasks; k += kNThreads) {
+      const int task = k + rot < n_tasks ? k + rot : k + rot - n_tasks;
+      const int d0 = task * 8;
+      const uint4* src = reinterpret_cast<const uint4*>(wr) + (size_t)d0 * Q;
 #pragma unroll
-      for (int u = 0; u < kDepth; ++u) {
-        const int i = base + u * kNThreads;
-        if (i < total8) v[u] = __ldg(reinterpret_cast<const uint4*>(wr) + i);
-      }
+      for (int q = 0; q < Q; ++q) {    // experts 8q .. 8q+7
 #pragma unroll
-      for (int u = 0; u < kDepth; ++u) {
-        const int i = base + u * kNThreads;
-        if (i < total8) {
-          const int d = (i * 8) / NP, j0 = (i * 8) % NP;
-          const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+        for (int hf = 0; hf < 2; ++hf) {  // rows d0 + 4hf .. d0 + 4hf + 3
+          uint32_t r[4][4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            wrt[(j0 + 2 * e) * ldw + d] = (uint16_t)(w[e] & 0xffffu);
-            wrt[(j0 + 2 * e + 1) * ldw + d] = (uint16_t)(w[e] >> 16);
+          for (int i = 0; i < 4; ++i) {
+            const uint4 v = __ldg(src + (4 * hf + i) * Q + q);
+            r[i][0] = v.x;
+            r[i][1] = v.y;
+            r[i][2] = v.z;
+            r[i][3] = v.w;
+          }
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {  // expert pair (8q + 2m, 8q + 2m + 1)
+            const uint2 lo = make_uint2(__byte_perm(r[0][m], r[1][m], 0x5410), __byte_perm(r[2][m], r[3][m], 0x5410));
+            const uint2 hi = make_uint2(__byte_perm(r[0][m], r[1][m], 0x7632), __byte_perm(r[2][m], r[3][m], 0x7632));
+            *reinterpret_cast<uint2*>(wrt + (size_t)(8 * q + 2 * m) * ldw + d0 + 4 * hf) = lo;
+            *reinterpret_cast<uint2*>(wrt + (size_t)(8 * q + 2 * m + 1) * ldw + d0 + 4 * hf) = hi;
           }
         }
       }
@@ -275,8 +288,8 @@ __device__ __forceinline__ void router_softmax(const Smem& s, int rows, int N, c
 }
 
 // Persistent router loop over this CTA's 16-token tiles (blockIdx.x,
-// blockIdx.x + gridDim.x, ...) for bf16 inputs: Wr^T is staged once, the
-// first batch of A fragments of the next tile is loaded right after the
+// blockIdx.x + gridDim.x, ...) for bf16 inputs: Wr^T is staged once, then
+// the first batch of A fragments of the next tile is loaded right after the
 // current tile's MMAs (into the registers those MMAs just consumed), so the
 // loads are in flight during the partial-sum exchange, the softmax and the
 // gate stores.  After each tile, sink(t0, rows) reads s.gates.
@@ -292,10 +305,15 @@ __device__ __forceinline__ void router_tiles(const Smem& s, const uint16_t* __re
     const int64_t t0 = tile * kTileMax;
     return (int)(T - t0 < kTileMax ? T - t0 : kTileMax);
   };
+  // under a programmatic dependent launch: let the next kernel get scheduled,
+  // then wait for the previous one (it may have produced h, Wr or whatever
+  // the sink overwrites)
+  pdl_trigger();
+  pdl_wait();
+  stage_wrt<NP, kThreads>(s.wrt, Wr, N, D);  // before the A registers are live
   RouterA<KB> A;
   int64_t tile = blockIdx.x;
   if (tile < n_tiles) router_load_a<KB>(A, h, tile * kTileMax, rows_of(tile), D, warp);
-  stage_wrt<NP, kThreads, 8>(s.wrt, Wr, N, D);  // 32 registers beside A
   __syncthreads();
   for (; tile < n_tiles; tile += gridDim.x) {
     const int64_t t0 = tile * kTileMax;

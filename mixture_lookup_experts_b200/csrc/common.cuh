@@ -4,6 +4,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
+#include <utility>
 #include <stdint.h>
 
 #include <algorithm>
@@ -26,6 +27,25 @@ int num_sms();
 
 // Turns a launch / runtime error into a status.
 inline mole_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOLE_OK : MOLE_ERR_CUDA; }
+
+// Launches `kernel` with programmatic stream serialization: it may begin
+// while the previous kernel in the stream finishes (the kernel waits with
+// griddepcontrol.wait before touching that kernel's results).
+template <class... KArgs, class... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool aligned8(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7u) == 0; }
@@ -131,6 +151,11 @@ mole_status combine_dispatch(const int32_t* ids, int64_t T, const void* h, const
                              bool bf16_inputs, int table_kind, float* out, cudaStream_t stream);
 mole_status nf3_quantize_launch(const void* lut, int64_t V, int N, int64_t D, uint8_t* codes,
                                 uint16_t* scales, cudaStream_t stream);
+// Router of a prefill batch on the tensor cores (router_tc.cu; N == 16):
+// gates into the tokens' output rows, or (grouped) at their list positions.
+bool router_tc_supported(int64_t T, int N, int64_t D, const void* h, const void* Wr);
+mole_status router_tc_launch(const void* h, const void* Wr, int64_t T, int64_t D, bool grouped, float* out,
+                             const int* tok_pos, float* gates, cudaStream_t stream);
 // Id-grouped combine (grouped.cu): the grouping of a batch's tokens by id
 // (built once per batch), one layer's combine with it, and both in one call;
 // the combines fall back to combine_dispatch where the grouped kernels do not
@@ -189,6 +214,14 @@ __device__ __forceinline__ bool mbar_test(uint64_t* b, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+
+// Programmatic dependent launch (kernels launched with the programmatic
+// stream serialization attribute may start while the previous kernel in the
+// stream is still running): pdl_trigger lets the next kernel start early;
+// pdl_wait blocks until the previous kernel has completed and its memory is
+// visible.  Both are no-ops for kernels launched without the attribute.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // try_wait with a suspend-time hint: a thread whose phase is not complete
 // sleeps in the barrier unit (issuing nothing) until the phase completes or

@@ -21,9 +21,10 @@
 //               item records, laid out by item size, largest first;
 //       step 3  every token's list position: list[pos] = t, tok_pos[t] = pos.
 //     Steps 1-3 each start after a grid-wide barrier (bounded wait).
-//  2. router_group_kernel (per layer; persistent, 2 CTAs per SM): the
-//     tensor-core router + softmax of combine_common.cuh; each token's gates
-//     go to its list position, so an item's gates are contiguous.
+//  2. the router (per layer): router_tc.cu's tcgen05 kernel for 16 experts,
+//     else router_group_kernel (persistent, 2 CTAs per SM, the mma.sync
+//     router of combine_common.cuh); each token's gates go to its list
+//     position, so an item's gates are contiguous.
 //  3. grouped_gather_kernel (per layer; one CTA per SM, 9 warps): a producer
 //     warp copies each work item's row block and its tokens' gates (two
 //     cp.async.bulk) into a ring of shared-memory slots; 8 consumer warps
@@ -369,18 +370,19 @@ __global__ void __launch_bounds__(kThreads, 2) router_group_kernel(const GArgs p
   constexpr int NP = 8 * NT;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const Smem s = carve<true, NP>(smem_raw, p.D);
-  // list positions of the tile's tokens, loaded one tile ahead (thread r < 16)
+  // list positions of the tile's tokens, loaded one tile ahead (thread r <
+  // 16); the first tile's inside the first sink, after router_tiles has
+  // waited for the previous kernel (it may be the one building the grouping)
   int pos_next = -1;
-  {
-    const int64_t t = (int64_t)blockIdx.x * kTileMax + threadIdx.x;
-    if (threadIdx.x < kTileMax && t < p.T) pos_next = w.tok_pos[t];
-  }
+  bool first = true;
   router_tiles<NT>(s, p.h, p.Wr, p.T, p.N, p.D, [&](int64_t t0, int rows) {
     if (threadIdx.x < kTileMax) {
+      if (first && t0 + threadIdx.x < p.T) pos_next = w.tok_pos[t0 + threadIdx.x];
       s.tok_id[threadIdx.x] = pos_next;
       const int64_t tn = t0 + (int64_t)gridDim.x * kTileMax + threadIdx.x;
       pos_next = tn < p.T ? w.tok_pos[tn] : -1;
     }
+    first = false;
     __syncthreads();
     for (int i = threadIdx.x; i < rows * NP; i += kThreads) {
       const int r = i / NP, j = i - r * NP;
@@ -407,7 +409,6 @@ struct GroupLayout {
 // hold 168 registers -- the N rows of its 4-element vector stay in registers
 // in fp32 (up to 16 experts) while it serves every token of the item.
 constexpr int kGroupCons = 8;
-constexpr bool kPairTokens = true;
 
 // bf16 -> fp32 through opaque instructions: the compiler keeps the converted
 // values in registers across the item's tokens instead of converting again
@@ -463,6 +464,35 @@ __device__ __forceinline__ float4 combine_unit(const float (&xf)[kPacked ? 1 : N
   return make_float4(a0, a1, a2, a3);
 }
 
+// out for 4 tokens at once (gates at g + k * gstride floats, k = 0..3):
+// 16 independent FMA chains over the N rows held in fp32.
+template <int NP, bool kExactN>
+__device__ __forceinline__ void combine_quad(const float (&xf)[NP][4], const float* g, int gstride, int N,
+                                             float (&o)[4][4]) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) o[k][0] = o[k][1] = o[k][2] = o[k][3] = 0.f;
+#pragma unroll
+  for (int jq = 0; jq < NP / 4; ++jq) {
+    float4 gv[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) gv[k] = reinterpret_cast<const float4*>(g + k * gstride)[jq];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int j = 4 * jq + e;
+      if (kExactN || j < N) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float gk = e == 0 ? gv[k].x : e == 1 ? gv[k].y : e == 2 ? gv[k].z : gv[k].w;
+          o[k][0] = fmaf(gk, xf[j][0], o[k][0]);
+          o[k][1] = fmaf(gk, xf[j][1], o[k][1]);
+          o[k][2] = fmaf(gk, xf[j][2], o[k][2]);
+          o[k][3] = fmaf(gk, xf[j][3], o[k][3]);
+        }
+      }
+    }
+  }
+}
+
 template <int NT, bool kExactN>
 __global__ void __launch_bounds__(kGroupThreads, 1) grouped_gather_kernel(const GArgs p, const GroupWs w,
                                                                           const GroupLayout L) {
@@ -486,6 +516,8 @@ __global__ void __launch_bounds__(kGroupThreads, 1) grouped_gather_kernel(const 
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
+  pdl_trigger();
+  pdl_wait();  // the router's gates (and, before it, the grouping) are complete
   if (ld_relaxed_u32(&w.ctl[kCtlAbort]) != 0xFFFFFFFFu) return;  // plan abandoned (error word set)
   volatile int* abort = abort_flag;
   const int n_items = (int)ld_relaxed_u32(&w.ctl[kCtlItems]);
@@ -594,13 +626,16 @@ __global__ void __launch_bounds__(kGroupThreads, 1) grouped_gather_kernel(const 
             }
           }
           int i = grp;
-          // two tokens at a time (8 independent FMA chains); one at a time with
-          // packed rows, where a pair would convert every row twice at once
-          for (; kPairTokens && !kPacked && i + Gt < n; i += 2 * Gt) {
-            const float4 o0 = combine_unit<NP, kExactN, kPacked>(xf, xp, gs + i * NP, p.N);
-            const float4 o1 = combine_unit<NP, kExactN, kPacked>(xf, xp, gs + (i + Gt) * NP, p.N);
-            __stcs(reinterpret_cast<float4*>(p.out + (int64_t)slot_tok[q * C + i] * p.D + 4 * v), o0);
-            __stcs(reinterpret_cast<float4*>(p.out + (int64_t)slot_tok[q * C + i + Gt] * p.D + 4 * v), o1);
+          if constexpr (!kPacked) {
+            // four tokens at a time (16 independent FMA chains)
+            for (; i + 3 * Gt < n; i += 4 * Gt) {
+              float o[4][4];
+              combine_quad<NP, kExactN>(xf, gs + i * NP, Gt * NP, p.N, o);
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                __stcs(reinterpret_cast<float4*>(p.out + (int64_t)slot_tok[q * C + i + k * Gt] * p.D + 4 * v),
+                       make_float4(o[k][0], o[k][1], o[k][2], o[k][3]));
+            }
           }
           for (; i < n; i += Gt) {
             const float4 o0 = combine_unit<NP, kExactN, kPacked>(xf, xp, gs + i * NP, p.N);
@@ -643,9 +678,15 @@ mole_status launch_layer(const GArgs& p, const GroupWs& w, cudaStream_t stream) 
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, rkern, kThreads, rsmem) != cudaSuccess || occ < 1)
     return MOLE_ERR_UNSUPPORTED;
   const int64_t n_tiles = (p.T + kTileMax - 1) / kTileMax;
-  rkern<<<(unsigned)std::min<int64_t>(n_tiles, (int64_t)occ * n_sm), kThreads, rsmem, stream>>>(p, w);
-  gkern<<<(unsigned)n_sm, kGroupThreads, gsmem, stream>>>(p, w, L);
-  return cuda_status(cudaGetLastError());
+  if (router_tc_supported(p.T, p.N, p.D, p.h, p.Wr)) {
+    const mole_status st = router_tc_launch(p.h, p.Wr, p.T, p.D, true, p.out, w.tok_pos, w.gates, stream);
+    if (st != MOLE_OK) return st;
+  } else if (launch_pdl(rkern, (unsigned)std::min<int64_t>(n_tiles, (int64_t)occ * n_sm), kThreads, rsmem, stream,
+                        p, w) != cudaSuccess) {
+    return MOLE_ERR_CUDA;
+  }
+  if (launch_pdl(gkern, (unsigned)n_sm, kGroupThreads, gsmem, stream, p, w, L) != cudaSuccess) return MOLE_ERR_CUDA;
+  return MOLE_OK;
 }
 
 mole_status layer_dispatch(const GArgs& p, const GroupWs& w, cudaStream_t stream) {
