@@ -352,23 +352,21 @@ def main():
     uniq_counts = [[int(torch.unique(x).numel()) for x in pool] for pool in id_pool]
     out = torch.empty((T, D), dtype=torch.float32, device=dev)
     combine = Combiner(mole, args.path, T, V, N, dev)
-    prep_events = []
 
     def step(i, events=None):
+        """One step; with `events` (start, grouped, end) recorded around the
+        grouping and the layer calls -- none between layers, so consecutive
+        layer kernels overlap their launches (programmatic dependent launch)."""
         p = i % P
         if events is not None:
-            e = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            e[0].record(stream)
+            events[0].record(stream)
         combine.prepare(id_pool[p][0], stream)
         if events is not None:
-            e[1].record(stream)
-            prep_events.append(e)
+            events[1].record(stream)
         for layer in range(L):
-            if events is not None:
-                events[layer][0].record(stream)
             combine(id_pool[p][layer], h_pool[p][layer], routers[layer], luts[layer], out, stream)
-            if events is not None:
-                events[layer][1].record(stream)
+        if events is not None:
+            events[2].record(stream)
 
     # ---- warm-up ----
     for i in range(W):
@@ -378,8 +376,7 @@ def main():
         raise RuntimeError(f"device status {st} after warm-up")
 
     # ---- timed region: K steps, barrier + synchronize on both sides ----
-    kern_events = [[[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
-                    for _ in range(L)] for _ in range(K)]
+    kern_events = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
@@ -396,11 +393,12 @@ def main():
     st = mole.mole_check(stream, timeout_ms=60000)
     if st != 0:
         raise RuntimeError(f"device status {st} in the timed region")
-    kern_ms = [kern_events[i][l][0].elapsed_time(kern_events[i][l][1]) for i in range(K) for l in range(L)]
-    avg_kern_ms = sum(kern_ms) / len(kern_ms)
+    # per layer call: the step's layer span / L (mean over the timed steps)
+    layers_ms = [kern_events[i][1].elapsed_time(kern_events[i][2]) for i in range(K)]
+    avg_kern_ms = sum(layers_ms) / (K * L)
     U_avg = sum(uniq_counts[(W + i) % P][l] for i in range(K) for l in range(L)) / (K * L)
 
-    prep_ms = [a.elapsed_time(b) for a, b in prep_events[-K:]] if prep_events else [0.0]
+    prep_ms = [kern_events[i][0].elapsed_time(kern_events[i][1]) for i in range(K)]
     avg_prep_ms = sum(prep_ms) / len(prep_ms)
     max_ms, max_kern_ms, max_prep_ms = max_over_ranks([elapsed_ms, avg_kern_ms, avg_prep_ms], dev)
     value = whole_job_tokens_per_s(world, T, K, max_ms)
@@ -418,7 +416,8 @@ def main():
                 "frac": achieved_gbs / hbm_peak, "traffic": traffic,
                 "kernel": KERNELS[args.path],
                 "algorithmic_bytes_per_launch": alg_bytes, "unique_rows_per_launch": U_avg,
-                "avg_launch_us": max_kern_ms * 1e3, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
+                "avg_launch_us": max_kern_ms * 1e3, "launch_timing": "per layer call = (step - grouping) / layers, "
+                "CUDA events per step on the launching stream", "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
                 "frac_of_8TBs": achieved_gbs / 8000.0, "traffic_source": traffic_note}
 
     line = {
@@ -495,6 +494,18 @@ def e2e_leg(combine, id_pool, h_pool, routers, luts, out, dev, stream, world, W,
                                     f"the token grouping and {L} combine calls through the C ABI, {L} outputs D2H"}
 
 
+def time_block(fn, n, stream):
+    """ms for n back-to-back calls between two CUDA events."""
+    import torch
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(n):
+        fn(i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b)
+
+
 def time_launches(fn, n, stream):
     import torch
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
@@ -533,8 +544,7 @@ def other_cases(mole, luts, routers, rng, g, dev, stream, W, T_main, kind_main, 
 
                 for i in range(max(W, 3) * L):
                     fn(i)
-                ms = time_launches(fn, 4 * L, stream)
-                avg = sum(ms) / len(ms)
+                avg = time_block(fn, 4 * L, stream) / (4 * L)  # no events between calls
                 prep = time_launches(lambda i: combine.prepare(ids, stream), 5, stream)
                 b = combine_bytes(U, T, D, N)
                 res[f"T{T}_{kind}_{path}"] = {"tokens_per_s_per_layer": T / (avg / 1e3), "avg_launch_us": avg * 1e3,
