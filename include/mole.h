@@ -204,6 +204,21 @@ mole_status mole_lookup_combine_nf3(const int32_t* ids, int64_t T, const void* h
                                     const uint16_t* scales, int64_t V, int32_t N, int64_t D,
                                     mole_dtype dt, float* out, cudaStream_t stream);
 
+/*
+ * mole_lookup_combine_nf3 for a batch whose token grouping was built from the
+ * same ids, T and N (see mole_token_groups_build): each distinct id's code and
+ * scale blocks are read and decoded once and applied to all of that id's
+ * tokens.  Same arguments, results (bit for bit) and error behaviour as
+ * mole_lookup_combine_nf3, plus the groups buffer (as for
+ * mole_lookup_combine_groups).  The grouped kernels serve bf16 inputs,
+ * T >= 1024, N <= 16 with N * D/64 a multiple of 8, and 16-byte aligned codes
+ * and scales; other calls run the mole_lookup_combine_nf3 kernels.
+ */
+mole_status mole_lookup_combine_nf3_groups(const int32_t* ids, int64_t T, const void* groups, size_t bytes,
+                                           const void* h, const void* Wr, const uint8_t* codes,
+                                           const uint16_t* scales, int64_t V, int32_t N, int64_t D, mole_dtype dt,
+                                           float* out, cudaStream_t stream);
+
 /* The 8 NF3 levels as fp16 bit patterns (ascending; index 3 is 0.0) and the 7
  * fp32 decision midpoints.  Host-only; no device work. */
 void mole_nf3_levels(uint16_t levels_f16[8]);

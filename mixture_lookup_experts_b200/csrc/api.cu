@@ -119,11 +119,33 @@ extern "C" mole_status mole_lookup_combine_groups(const int32_t* ids, int64_t T,
   st = check_device();
   if (st != MOLE_OK) return st;
   if (dt == MOLE_BF16 && mole::aligned16(Wr)) {
-    st = mole::combine_groups(groups, bytes, T, h, Wr, lut, N, (int)D, out, stream);
+    st = mole::combine_groups(groups, bytes, T, h, Wr, lut, nullptr, false, N, (int)D, out, stream);
     if (st != MOLE_ERR_UNSUPPORTED) return st;
   }
   return mole::combine_dispatch(ids, T, h, Wr, lut, nullptr, V, N, (int)D, dt == MOLE_BF16, dt == MOLE_BF16 ? 0 : 1,
                                 out, stream);
+}
+
+extern "C" mole_status mole_lookup_combine_nf3_groups(const int32_t* ids, int64_t T, const void* groups,
+                                                      size_t bytes, const void* h, const void* Wr,
+                                                      const uint8_t* codes, const uint16_t* scales, int64_t V,
+                                                      int32_t N, int64_t D, mole_dtype dt, float* out,
+                                                      cudaStream_t stream) {
+  if (!valid_dtype(dt)) return MOLE_ERR_ARG;
+  mole_status st = check_combine(ids, T, h, Wr, codes, V, N, D, out);
+  if (st != MOLE_OK) return st;
+  if (T > 0 && !scales) return MOLE_ERR_ARG;
+  if (D % 64 != 0) return MOLE_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(codes) & 3u) || (reinterpret_cast<uintptr_t>(scales) & 1u)) return MOLE_ERR_ALIGN;
+  st = check_groups(T, N, groups, bytes);
+  if (st != MOLE_OK || T == 0) return st;
+  st = check_device();
+  if (st != MOLE_OK) return st;
+  if (dt == MOLE_BF16 && mole::aligned16(Wr) && mole::aligned16(codes) && mole::aligned16(scales)) {
+    st = mole::combine_groups(groups, bytes, T, h, Wr, codes, scales, true, N, (int)D, out, stream);
+    if (st != MOLE_ERR_UNSUPPORTED) return st;
+  }
+  return mole::combine_dispatch(ids, T, h, Wr, codes, scales, V, N, (int)D, dt == MOLE_BF16, 2, out, stream);
 }
 
 extern "C" mole_status mole_lookup_combine_grouped(const int32_t* ids, int64_t T, const void* h, const void* Wr,

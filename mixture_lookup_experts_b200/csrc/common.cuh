@@ -164,7 +164,8 @@ size_t token_groups_bytes(int64_t T, int N);
 mole_status token_groups_build(const int32_t* ids, int64_t T, int64_t V, int N, void* buf, size_t bytes,
                                cudaStream_t stream);
 mole_status combine_groups(const void* buf, size_t bytes, int64_t T, const void* h, const void* Wr,
-                           const void* table, int N, int D, float* out, cudaStream_t stream);
+                           const void* table, const uint16_t* scales, bool nf3, int N, int D, float* out,
+                           cudaStream_t stream);
 mole_status combine_grouped_dispatch(const int32_t* ids, int64_t T, const void* h, const void* Wr,
                                      const void* table, const uint16_t* scales, int64_t V, int N, int D,
                                      bool bf16_inputs, int table_kind, float* out, void* ws, size_t ws_bytes,

@@ -357,7 +357,9 @@ struct GArgs {
   int64_t T;
   const uint16_t* h;
   const uint16_t* Wr;
-  const uint16_t* table;
+  const uint16_t* table;    // bf16 table
+  const uint8_t* codes;     // NF3 table: codes and fp16 scales
+  const uint16_t* scales;
   int N, D;
   float* out;
   unsigned* err;
@@ -402,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 2) router_group_kernel(const GArgs p
 // Slot layout: [0, gates_off) the id's row block (N rows of D bf16),
 // [gates_off, + kItemTokens * NP * 4) the gates of the item's tokens.
 struct GroupLayout {
-  int n_slots, slot_bytes, gates_off;
+  int n_slots, slot_bytes, gates_off, scales_off;  // scales_off: NF3 table only
 };
 
 // 8 consumer warps + 1 producer warp: 3 warps per scheduler, so a thread may
@@ -493,12 +495,82 @@ __device__ __forceinline__ void combine_quad(const float (&xf)[NP][4], const flo
   }
 }
 
-template <int NT, bool kExactN>
+// The NF3 table's counterparts: row j's 4 elements hold the levels, sc[j] the
+// block scale; per token the gate and the scale are multiplied first and the
+// product scales the levels, as the ungrouped kernels do.
+template <int NP, bool kExactN>
+__device__ __forceinline__ void combine_quad_nf3(const float (&xf)[NP][4], const float (&sc)[NP], const float* g,
+                                                 int gstride, int N, float (&o)[4][4]) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) o[k][0] = o[k][1] = o[k][2] = o[k][3] = 0.f;
+#pragma unroll
+  for (int jq = 0; jq < NP / 4; ++jq) {
+    float4 gv[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) gv[k] = reinterpret_cast<const float4*>(g + k * gstride)[jq];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int j = 4 * jq + e;
+      if (kExactN || j < N) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float a = (e == 0 ? gv[k].x : e == 1 ? gv[k].y : e == 2 ? gv[k].z : gv[k].w) * sc[j];
+          o[k][0] = fmaf(a, xf[j][0], o[k][0]);
+          o[k][1] = fmaf(a, xf[j][1], o[k][1]);
+          o[k][2] = fmaf(a, xf[j][2], o[k][2]);
+          o[k][3] = fmaf(a, xf[j][3], o[k][3]);
+        }
+      }
+    }
+  }
+}
+
+template <int NP, bool kExactN>
+__device__ __forceinline__ float4 combine_unit_nf3(const float (&xf)[NP][4], const float (&sc)[NP], const float* g,
+                                                   int N) {
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+  for (int j = 0; j < NP; ++j) {
+    if (kExactN || j < N) {
+      const float a = g[j] * sc[j];
+      a0 = fmaf(a, xf[j][0], a0);
+      a1 = fmaf(a, xf[j][1], a1);
+      a2 = fmaf(a, xf[j][2], a2);
+      a3 = fmaf(a, xf[j][3], a3);
+    }
+  }
+  return make_float4(a0, a1, a2, a3);
+}
+
+__device__ __forceinline__ float held(float x) {
+  uint32_t u;
+  asm volatile("mov.b32 %0, %1;" : "=r"(u) : "r"(__float_as_uint(x)));
+  return __uint_as_float(u);
+}
+
+// Levels of the 4 NF3 codes in the low 12 bits of x.
+__device__ __forceinline__ void nf3_levels4(uint32_t x, float (&f)[4]) {
+  uint32_t sl, sh;
+  nf3_selectors(x, sl, sh);
+  const uint32_t lo = prmt(kLoBytes0, kLoBytes1, sl);
+  const uint32_t hi = prmt(kHiBytes0, kHiBytes1, sl);
+  const uint32_t h01 = prmt(lo, hi, 0x5140u);
+  const uint32_t h23 = prmt(lo, hi, 0x7362u);
+  const float2 f01 = __half22float2(*reinterpret_cast<const __half2*>(&h01));
+  const float2 f23 = __half22float2(*reinterpret_cast<const __half2*>(&h23));
+  f[0] = f01.x;
+  f[1] = f01.y;
+  f[2] = f23.x;
+  f[3] = f23.y;
+}
+
+template <int NT, bool kExactN, bool kNf3>
 __global__ void __launch_bounds__(kGroupThreads, 1) grouped_gather_kernel(const GArgs p, const GroupWs w,
                                                                           const GroupLayout L) {
   constexpr int NP = 8 * NT;
   constexpr int C = kItemTokens;
-  constexpr bool kPacked = NP > 16;  // 32 experts: keep rows as bf16 pairs, convert per token
+  constexpr bool kPacked = !kNf3 && NP > 16;  // 32 experts: keep rows as bf16 pairs, convert per token
+  static_assert(!kNf3 || NP <= 16, "the NF3 consumer holds 16 rows");
   extern __shared__ __align__(128) uint8_t smem_raw[];
   uint8_t* ring = smem_raw;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw + (size_t)L.n_slots * L.slot_bytes);
@@ -523,6 +595,8 @@ __global__ void __launch_bounds__(kGroupThreads, 1) grouped_gather_kernel(const 
   const int n_items = (int)ld_relaxed_u32(&w.ctl[kCtlItems]);
   const int my_n = n_items > (int)blockIdx.x ? (n_items - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
   const uint32_t row_bytes = (uint32_t)p.N * (uint32_t)p.D * 2u;
+  const int NB = p.D >> 6;  // NF3 blocks per row
+  const uint32_t code_bytes = (uint32_t)p.N * (uint32_t)NB * 24u, scale_bytes = (uint32_t)p.N * (uint32_t)NB * 2u;
 
   if (warp == kGroupProducer) {
     // ---------------- producer ----------------
@@ -568,8 +642,14 @@ __global__ void __launch_bounds__(kGroupThreads, 1) grouped_gather_kernel(const 
       // the copies first; the token list (loaded one item ahead) after them
       if (lane == 0) {
         const uint32_t gate_bytes = (uint32_t)n * NP * 4u;
-        mbar_expect_tx(&full[q], row_bytes + gate_bytes);
-        bulk_g2s(slot, p.table + (int64_t)id * p.N * p.D, row_bytes, &full[q]);
+        if (kNf3) {
+          mbar_expect_tx(&full[q], code_bytes + scale_bytes + gate_bytes);
+          bulk_g2s(slot, p.codes + (int64_t)id * code_bytes, code_bytes, &full[q]);
+          bulk_g2s(slot + L.scales_off, p.scales + (int64_t)id * p.N * NB, scale_bytes, &full[q]);
+        } else {
+          mbar_expect_tx(&full[q], row_bytes + gate_bytes);
+          bulk_g2s(slot, p.table + (int64_t)id * p.N * p.D, row_bytes, &full[q]);
+        }
         bulk_g2s(slot + L.gates_off, w.gates + (int64_t)pos * NP, gate_bytes, &full[q]);
       }
       if (lane < n) slot_tok[q * C + lane] = tok;
@@ -612,6 +692,27 @@ __global__ void __launch_bounds__(kGroupThreads, 1) grouped_gather_kernel(const 
         for (int v = v0; v < units; v += vstep) {
           float xf[kPacked ? 1 : NP][4];
           uint2 xp[kPacked ? NP : 1];
+          float sc[NP];
+          if constexpr (kNf3) {
+            // 4 codes at bits [12u, 12u + 12) of the row's block v / 16
+            const int b = v >> 4, bit = 12 * (v & 15), wi = bit >> 5, sh = bit & 31;
+            const uint16_t* ss = reinterpret_cast<const uint16_t*>(slot + L.scales_off);
+#pragma unroll
+            for (int j = 0; j < NP; ++j) {
+              float f[4] = {0.f, 0.f, 0.f, 0.f};
+              sc[j] = 0.f;
+              if (kExactN || j < p.N) {
+                const uint32_t* cw = reinterpret_cast<const uint32_t*>(slot + (size_t)(j * NB + b) * 24);
+                const uint32_t x = __funnelshift_r(cw[wi], wi < 5 ? cw[wi + 1] : 0u, sh) & 0xfffu;
+                nf3_levels4(x, f);
+                sc[j] = held(__half2float(__ushort_as_half(ss[j * NB + b])));
+              }
+              xf[j][0] = held(f[0]);
+              xf[j][1] = held(f[1]);
+              xf[j][2] = held(f[2]);
+              xf[j][3] = held(f[3]);
+            }
+          } else {
 #pragma unroll
           for (int j = 0; j < NP; ++j) {
             uint2 r = make_uint2(0u, 0u);
@@ -625,12 +726,16 @@ __global__ void __launch_bounds__(kGroupThreads, 1) grouped_gather_kernel(const 
               xf[kPacked ? 0 : j][3] = bf16_hi_held(r.y);
             }
           }
+          }
           int i = grp;
           if constexpr (!kPacked) {
             // four tokens at a time (16 independent FMA chains)
             for (; i + 3 * Gt < n; i += 4 * Gt) {
               float o[4][4];
-              combine_quad<NP, kExactN>(xf, gs + i * NP, Gt * NP, p.N, o);
+              if constexpr (kNf3)
+                combine_quad_nf3<NP, kExactN>(xf, sc, gs + i * NP, Gt * NP, p.N, o);
+              else
+                combine_quad<NP, kExactN>(xf, gs + i * NP, Gt * NP, p.N, o);
 #pragma unroll
               for (int k = 0; k < 4; ++k)
                 __stcs(reinterpret_cast<float4*>(p.out + (int64_t)slot_tok[q * C + i + k * Gt] * p.D + 4 * v),
@@ -638,7 +743,11 @@ __global__ void __launch_bounds__(kGroupThreads, 1) grouped_gather_kernel(const 
             }
           }
           for (; i < n; i += Gt) {
-            const float4 o0 = combine_unit<NP, kExactN, kPacked>(xf, xp, gs + i * NP, p.N);
+            float4 o0;
+            if constexpr (kNf3)
+              o0 = combine_unit_nf3<NP, kExactN>(xf, sc, gs + i * NP, p.N);
+            else
+              o0 = combine_unit<NP, kExactN, kPacked>(xf, xp, gs + i * NP, p.N);
             __stcs(reinterpret_cast<float4*>(p.out + (int64_t)slot_tok[q * C + i] * p.D + 4 * v), o0);
           }
         }
@@ -654,21 +763,38 @@ __global__ void __launch_bounds__(kGroupThreads, 1) grouped_gather_kernel(const 
   __syncthreads();
 }
 
-template <int NT, bool kExactN>
+// Ring slot of a work item: the id's row block (bf16 table: N rows of D;
+// NF3 table: N x D/64 24-byte code blocks, then the fp16 scales at
+// scales_off), then the gates of up to kItemTokens tokens at gates_off.
+template <int NT>
+GroupLayout group_layout(int N, int D, bool nf3) {
+  constexpr int NP = 8 * NT;
+  GroupLayout L{};
+  int64_t off;
+  if (nf3) {
+    const int64_t NB = D / 64;
+    L.scales_off = (int)((N * NB * 24 + 127) / 128 * 128);
+    off = L.scales_off + N * NB * 2;
+  } else {
+    off = (int64_t)N * D * 2;
+  }
+  L.gates_off = (int)((off + 127) / 128 * 128);
+  L.slot_bytes = (int)((L.gates_off + (int64_t)kItemTokens * NP * 4 + 127) / 128 * 128);
+  L.n_slots = (int)std::min<int64_t>(16, kRingBudget / L.slot_bytes);
+  return L;
+}
+
+template <int NT, bool kExactN, bool kNf3>
 mole_status launch_layer(const GArgs& p, const GroupWs& w, cudaStream_t stream) {
   constexpr int NP = 8 * NT;
   constexpr int C = kItemTokens;
-  GroupLayout L{};
-  const int64_t row_bytes = (int64_t)p.N * p.D * 2;
-  L.gates_off = (int)((row_bytes + 127) / 128 * 128);
-  L.slot_bytes = (int)((L.gates_off + (int64_t)C * NP * 4 + 127) / 128 * 128);
-  L.n_slots = (int)std::min<int64_t>(16, kRingBudget / L.slot_bytes);
+  const GroupLayout L = group_layout<NT>(p.N, p.D, kNf3);
   if (L.n_slots < 2) return MOLE_ERR_UNSUPPORTED;
   const size_t gsmem = (size_t)L.n_slots * L.slot_bytes + (size_t)L.n_slots * (16 + 4 + 4 * C) + 16;
   const size_t rsmem = smem_bytes_for<true, NP>(p.D);
   if (gsmem > 227 * 1024 || rsmem > 227 * 1024) return MOLE_ERR_UNSUPPORTED;
   auto rkern = router_group_kernel<NT>;
-  auto gkern = grouped_gather_kernel<NT, kExactN>;
+  auto gkern = grouped_gather_kernel<NT, kExactN, kNf3>;
   if (cudaFuncSetAttribute(rkern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rsmem) != cudaSuccess ||
       cudaFuncSetAttribute(gkern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gsmem) != cudaSuccess)
     return MOLE_ERR_CUDA;
@@ -689,21 +815,25 @@ mole_status launch_layer(const GArgs& p, const GroupWs& w, cudaStream_t stream) 
   return MOLE_OK;
 }
 
+template <bool kNf3>
 mole_status layer_dispatch(const GArgs& p, const GroupWs& w, cudaStream_t stream) {
-  if (p.N == 16) return launch_layer<2, true>(p, w, stream);
-  if (p.N == 8) return launch_layer<1, true>(p, w, stream);
-  if (p.N < 8) return launch_layer<1, false>(p, w, stream);
-  if (p.N < 16) return launch_layer<2, false>(p, w, stream);
-  if (p.N == 32) return launch_layer<4, true>(p, w, stream);
-  return launch_layer<4, false>(p, w, stream);
+  if (p.N == 16) return launch_layer<2, true, kNf3>(p, w, stream);
+  if (p.N == 8) return launch_layer<1, true, kNf3>(p, w, stream);
+  if (p.N < 8) return launch_layer<1, false, kNf3>(p, w, stream);
+  if (p.N < 16) return launch_layer<2, false, kNf3>(p, w, stream);
+  if (kNf3) return MOLE_ERR_UNSUPPORTED;  // the NF3 consumer holds at most 16 rows
+  if (p.N == 32) return launch_layer<4, true, false>(p, w, stream);
+  return launch_layer<4, false, false>(p, w, stream);
 }
 
 // Whether the grouped kernels take a call of this shape (else the
 // mole_lookup_combine kernels do, and the grouping is not used).
-bool grouped_applies(int64_t T, int N, int D) {
-  if (T < kGroupedMinT || T > kGroupedMaxT || N < 1 || N > 32) return false;
-  const int64_t slot = ((int64_t)N * D * 2 + 127) / 128 * 128 + (int64_t)kItemTokens * padded_experts(N) * 4;
-  return kRingBudget / slot >= 2 && smem_bytes_for<true, 32>(D) <= 227 * 1024;
+bool grouped_applies(int64_t T, int N, int D, bool nf3) {
+  if (T < kGroupedMinT || T > kGroupedMaxT || N < 1 || N > (nf3 ? 16 : 32)) return false;
+  // NF3: both bulk copies need 16-byte multiples (N * D/64 a multiple of 8)
+  if (nf3 && (D % 64 != 0 || ((int64_t)N * (D / 64)) % 8 != 0)) return false;
+  const GroupLayout L = group_layout<4>(N, D, nf3);  // the widest gate area
+  return L.n_slots >= 2 && smem_bytes_for<true, 32>(D) <= 227 * 1024;
 }
 
 }  // namespace
@@ -745,31 +875,34 @@ mole_status token_groups_build(const int32_t* ids, int64_t T, int64_t V, int N, 
 }
 
 mole_status combine_groups(const void* buf, size_t bytes, int64_t T, const void* h, const void* Wr,
-                           const void* table, int N, int D, float* out, cudaStream_t stream) {
+                           const void* table, const uint16_t* scales, bool nf3, int N, int D, float* out,
+                           cudaStream_t stream) {
   GroupWs w{};
   if (carve_ws(const_cast<void*>(buf), T, padded_experts(N), &w) > bytes) return MOLE_ERR_WORKSPACE;
-  if (!grouped_applies(T, N, D)) return MOLE_ERR_UNSUPPORTED;
+  if (!grouped_applies(T, N, D, nf3)) return MOLE_ERR_UNSUPPORTED;
   GArgs p{};
   p.T = T;
   p.h = static_cast<const uint16_t*>(h);
   p.Wr = static_cast<const uint16_t*>(Wr);
   p.table = static_cast<const uint16_t*>(table);
+  p.codes = static_cast<const uint8_t*>(table);
+  p.scales = scales;
   p.N = N;
   p.D = D;
   p.out = out;
   p.err = error_word();
   if (!p.err) return MOLE_ERR_CUDA;
-  return layer_dispatch(p, w, stream);
+  return nf3 ? layer_dispatch<true>(p, w, stream) : layer_dispatch<false>(p, w, stream);
 }
 
 mole_status combine_grouped_dispatch(const int32_t* ids, int64_t T, const void* h, const void* Wr,
                                      const void* table, const uint16_t* scales, int64_t V, int N, int D,
                                      bool bf16_inputs, int table_kind, float* out, void* ws, size_t ws_bytes,
                                      cudaStream_t stream) {
-  if (bf16_inputs && table_kind == 0 && grouped_applies(T, N, D) && aligned16(Wr) && aligned16(table)) {
+  if (bf16_inputs && table_kind == 0 && grouped_applies(T, N, D, false) && aligned16(Wr) && aligned16(table)) {
     mole_status st = token_groups_build(ids, T, V, N, ws, ws_bytes, stream);
     if (st != MOLE_OK) return st;
-    return combine_groups(ws, ws_bytes, T, h, Wr, table, N, D, out, stream);
+    return combine_groups(ws, ws_bytes, T, h, Wr, table, nullptr, false, N, D, out, stream);
   }
   return combine_dispatch(ids, T, h, Wr, table, scales, V, N, D, bf16_inputs, table_kind, out, stream);
 }

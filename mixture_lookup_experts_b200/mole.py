@@ -45,6 +45,7 @@ SIGNATURES = {
     "mole_lookup_combine_grouped": ([_P, _I64, _P, _P, _P, _I64, _I32, _I64, _I, _P, _P, _SZ, _P], _I),
     "mole_quantize_lut_nf3": ([_P, _I64, _I32, _I64, _P, _P, _P], _I),
     "mole_lookup_combine_nf3": ([_P, _I64, _P, _P, _P, _P, _I64, _I32, _I64, _I, _P, _P], _I),
+    "mole_lookup_combine_nf3_groups": ([_P, _I64, _P, _SZ, _P, _P, _P, _P, _I64, _I32, _I64, _I, _P, _P], _I),
     "mole_nf3_levels": ([_P], None),
     "mole_nf3_midpoints": ([_P], None),
     "mole_gather_plan": ([_P, _I64, _I64, _P, _P, _P, _P], _I),
@@ -238,6 +239,24 @@ def mole_lookup_combine_nf3(ids: torch.Tensor, h: torch.Tensor, Wr: torch.Tensor
         out = torch.empty((T, D), dtype=torch.float32, device=h.device)
     _ok(lib.mole_lookup_combine_nf3(_ptr(ids), T, _ptr(h), _ptr(Wr), _ptr(codes), _ptr(scales), V, N, D,
                                     _dt(h), _ptr(out), _stream(stream)), "mole_lookup_combine_nf3")
+    return out
+
+
+def mole_lookup_combine_nf3_groups(ids: torch.Tensor, groups: torch.Tensor, h: torch.Tensor, Wr: torch.Tensor,
+                                   codes: torch.Tensor, scales: torch.Tensor, out: torch.Tensor | None = None,
+                                   stream=None):
+    """mole_lookup_combine_nf3 over a grouping built from the same ids (each
+    distinct code block read and decoded once); same result bit for bit."""
+    _contig(ids, groups, h, Wr, codes, scales, out)
+    V, N, nb, _ = codes.shape
+    D = nb * 64
+    T = ids.numel()
+    if out is None:
+        out = torch.empty((T, D), dtype=torch.float32, device=h.device)
+    nbytes = groups.numel() * groups.element_size()
+    _ok(lib.mole_lookup_combine_nf3_groups(_ptr(ids), T, _ptr(groups), nbytes, _ptr(h), _ptr(Wr), _ptr(codes),
+                                           _ptr(scales), V, N, D, _dt(h), _ptr(out), _stream(stream)),
+        "mole_lookup_combine_nf3_groups")
     return out
 
 

@@ -112,3 +112,77 @@ def test_nf3_full_size_sampled(mole, oracle_mod, T, kind):
     assert_combine_close(got, ref)
     del lut, codes, scales, out
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("V,N,D,T,kind", [
+    (200, 16, 256, 1500, "zipf"), (300, 8, 2048, 1100, "uniform"), (50, 16, 128, 3000, "zipf"),
+    (100, 13, 512, 1200, "zipf"),   # padded expert count (13 * 8 blocks = 104, a multiple of 8)
+    (100, 5, 128, 1200, "zipf"),    # N * D/64 not a multiple of 8: ungrouped kernels
+    (64, 16, 256, 300, "zipf"),     # below the grouping threshold: ungrouped kernels
+])
+def test_combine_nf3_groups_matches_oracle_and_ungrouped(mole, oracle_mod, V, N, D, T, kind):
+    rng = np.random.default_rng(T + D + N)
+    lut = inputs.normal(rng, (V, N, D), 0.02, "bf16")
+    Wr = inputs.normal(rng, (D, N), 0.02, "bf16")
+    h = inputs.normal(rng, (T, D), 1.0, "bf16")
+    ids = inputs.draw_ids(rng, T, V, kind)
+    ids[0], ids[-1] = 0, V - 1
+    codes, scales = oracle_mod.quantize_nf3(lut)
+    c, s = dev(codes), dev(scales).view(torch.float16)
+    groups = mole.mole_token_groups_build(dev(ids), V, N)
+    got = mole.mole_lookup_combine_nf3_groups(dev(ids), groups, dev(h), dev(Wr), c, s)
+    assert mole.mole_check() == 0
+    plain = mole.mole_lookup_combine_nf3(dev(ids), dev(h), dev(Wr), c, s)
+    assert mole.mole_check() == 0
+    assert torch.equal(got, plain)
+    ref, _ = oracle_mod.combine_nf3(ids, h, Wr, codes, scales)
+    assert_combine_close(got.cpu().numpy(), ref)
+
+
+def test_combine_nf3_groups_bad_ids(mole, oracle_mod):
+    V, N, D, T = 40, 16, 128, 1500
+    rng = np.random.default_rng(4)
+    lut = inputs.normal(rng, (V, N, D), 0.02, "bf16")
+    Wr = inputs.normal(rng, (D, N), 0.02, "bf16")
+    h = inputs.normal(rng, (T, D), 1.0, "bf16")
+    ids = rng.integers(0, V, T).astype(np.int32)
+    ids[[2, 900]] = [-5, V]
+    codes, scales = oracle_mod.quantize_nf3(lut)
+    groups = mole.mole_token_groups_build(dev(ids), V, N)
+    out = mole.mole_lookup_combine_nf3_groups(dev(ids), groups, dev(h), dev(Wr), dev(codes),
+                                              dev(scales).view(torch.float16))
+    assert mole.mole_check() == 5
+    got = out.cpu().numpy()
+    assert np.isnan(got[[2, 900]]).all()
+    ref, _ = oracle_mod.combine_nf3(ids, h, Wr, codes, scales)
+    ok = np.ones(T, bool)
+    ok[[2, 900]] = False
+    assert_combine_close(got[ok], ref[ok])
+
+
+@pytest.mark.parametrize("kind", ["zipf", "uniform"])
+def test_nf3_groups_full_size(mole, oracle_mod, kind):
+    shape = inputs.SHAPES["1b_nf3"]
+    V, D, N, T = shape.V, shape.D, shape.N, 16384
+    g = torch.Generator(device="cuda")
+    g.manual_seed(shape.seed + 7)
+    lut = (torch.randn((V, N, D), generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+    codes, scales = mole.mole_quantize_lut_nf3(lut)
+    rng = np.random.default_rng(shape.seed + 11)
+    Wr = inputs.normal(rng, (D, N), 0.02, "bf16")
+    ids = inputs.draw_ids(rng, T, V, kind)
+    h = inputs.normal(rng, (T, D), 1.0, "bf16")
+    groups = mole.mole_token_groups_build(dev(ids), V, N)
+    got = mole.mole_lookup_combine_nf3_groups(dev(ids), groups, dev(h), dev(Wr), codes, scales)
+    assert mole.mole_check() == 0
+    plain = mole.mole_lookup_combine_nf3(dev(ids), dev(h), dev(Wr), codes, scales)
+    assert mole.mole_check() == 0
+    assert torch.equal(got, plain)
+    sample = np.unique(np.concatenate([[0, T - 1], rng.integers(0, T, 30)]))
+    uniq, inv = np.unique(ids[sample], return_inverse=True)
+    sel = torch.from_numpy(uniq.astype(np.int64)).cuda()
+    ref, _ = oracle_mod.combine_nf3(inv.astype(np.int32), h[sample], Wr, codes[sel].cpu().numpy(),
+                                    host_bits(scales[sel]))
+    assert_combine_close(got[torch.from_numpy(sample).cuda()].cpu().numpy(), ref)
+    del lut, codes, scales, got, plain
+    torch.cuda.empty_cache()
