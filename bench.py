@@ -14,8 +14,9 @@ A step touches 16 distinct tables of 3.3 GB, so inputs are far larger than
 the 126 MB L2.  --path plain runs mole_lookup_combine per layer instead.
 
 Also measured in the same run (own keys in the JSON line): the one-off table
-build (410M-shaped layer, tensor cores), the NF3-compressed table combine, and
-the other prefill cases of the 1B-shaped layer.
+build (410M-shaped layer, tensor cores), the NF3-compressed table combine, the
+other prefill cases of the 1B-shaped layer, and the offloaded table (a layer
+table in pinned host memory, distinct rows staged over the host link).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -72,6 +73,7 @@ def parse_args():
     ap.add_argument("--layers", type=int, default=None,
                     help="layer tables to allocate (default: the model's 16); fewer only for profiling runs")
     ap.add_argument("--no-extras", action="store_true", help="skip the build / NF3 / other-case legs")
+    ap.add_argument("--no-offload", action="store_true", help="skip the host-resident (offloaded) table leg")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--build-only", action="store_true",
@@ -437,6 +439,8 @@ def main():
     if not args.no_extras:
         line["cases"] = other_cases(mole, luts, routers, rng, g, dev, stream, W, T, args.ids, args.path, L)
         line["nf3"] = nf3_leg(mole, luts, routers, id_pool, h_pool, uniq_counts, dev, stream, W, K, T, P, L)
+        if not args.no_offload:
+            line["offload"] = offload_leg(mole, luts, routers, rng, g, dev, stream, W, L)
         del luts
         torch.cuda.empty_cache()
         line["build"] = build_leg(mole, dev, stream, bf16_peak, bf16_sust, peak_kind)
@@ -601,6 +605,143 @@ def nf3_leg(mole, luts, routers, id_pool, h_pool, uniq_counts, dev, stream, W, K
             "quantize_ms_per_layer": q_avg, "quantize_gbs": q_bytes / (q_avg / 1e3) / 1e9,
             "workload": f"1B-shaped NF3 table (codes + fp16 scale per 64), T={T}, same ids/h as the main case, "
                         f"mole_lookup_combine_nf3_groups (grouping built once per id batch, not timed here)"}
+
+
+def offload_leg(mole, luts, routers, rng, g, dev, stream, W, L):
+    """The page's deployment scenario: the 1B-shaped layer table (3.3 GB bf16;
+    also its NF3 form) in pinned host memory.  Per batch each distinct id's
+    row block crosses the host link once (mole_offload_stage) and the combine
+    reads the staging buffer (mole_lookup_combine_offload).  Reported per
+    batch size: link bytes per token, staging time and link GB/s (against a
+    copy-engine copy of a contiguous pinned block), the combine, and a
+    decode step over L layers with the next layer's rows staged on a second
+    stream while this layer combines (two staging buffers)."""
+    import torch
+    shape = inputs.SHAPES["1b"]
+    V, D, N, Dr = shape.V, shape.D, shape.N, shape.Dr
+    row = N * D * 2
+    host = torch.empty((V, N, D), dtype=torch.bfloat16, pin_memory=True)
+    host.copy_(luts[0])
+    codes = torch.empty((V, N, D // 64, 24), dtype=torch.uint8, device=dev)
+    scales = torch.empty((V, N, D // 64), dtype=torch.float16, device=dev)
+    mole.mole_quantize_lut_nf3(luts[0], codes, scales, stream=stream)
+    hc = torch.empty(codes.shape, dtype=torch.uint8, pin_memory=True)
+    hs = torch.empty(scales.shape, dtype=torch.float16, pin_memory=True)
+    hc.copy_(codes)
+    hs.copy_(scales)
+    del codes, scales
+    torch.cuda.synchronize()
+    # the link's copy-engine rate: one contiguous 256 MiB pinned block to the device
+    blk = 256 << 20
+    src = host.view(-1).view(torch.uint8)[:blk]
+    dst = torch.empty(blk, dtype=torch.uint8, device=dev)
+    for _ in range(2):
+        dst.copy_(src, non_blocking=True)
+    ce_ms = min(time_launches(lambda i: dst.copy_(src, non_blocking=True), 5, stream))
+    ce_gbs = blk / (ce_ms / 1e3) / 1e9
+    del dst
+    moe_expert_bytes = 2 * D * Dr * 2  # one D x Dr and one Dr x D bf16 matrix
+    res = {"workload": "1B-shaped layer table [50304, 16, 2048] bf16 (3.3 GB) and its NF3 form (0.68 GB) in pinned "
+                       "host memory; Zipf(1.1) ids; grouping built once per batch (timed apart)",
+           "h2d_copy_engine_gbs": ce_gbs,
+           "moe_byte_model": {"expert_bytes": moe_expert_bytes,
+                              "note": "an offloaded MoE moves the weights of each expert a batch activates "
+                                      "(2 x D x Dr bf16 each; the routed experts of this layer before the table "
+                                      "replaced them); MoLE moves only the batch's distinct N x D row blocks"},
+           "cases": {}}
+    for nf3 in (False, True):
+        for T in ((1, 8, 64, 256, 4096, 16384) if not nf3 else (1, 64, 16384)):
+            ids_np = inputs.draw_ids(rng, T, V, "zipf")
+            U = int(np.unique(ids_np).size)
+            ids = torch.from_numpy(ids_np).to(dev)
+            groups = mole.mole_token_groups_build(ids, V, N, stream=stream)
+            staging = torch.empty(mole.mole_offload_staging_bytes(T, V, N, D, nf3=nf3), dtype=torch.uint8,
+                                  device=dev)
+            h = torch.randn((T, D), generator=g, device=dev).to(torch.bfloat16)
+            out = torch.empty((T, D), dtype=torch.float32, device=dev)
+            tab, sc = (hc, hs) if nf3 else (host, None)
+
+            def stage(i):
+                mole.mole_offload_stage(T, groups, tab, sc, staging=staging, stream=stream)
+
+            def comb(i):
+                mole.mole_lookup_combine_offload(groups, h, routers[0], staging, V, nf3=nf3, out=out, stream=stream)
+
+            def both(i):
+                stage(i)
+                comb(i)
+
+            n = 20 if T <= 4096 else 6
+            for i in range(max(W, 3)):
+                both(i)
+            st_ms = time_block(stage, n, stream) / n
+            cb_ms = time_block(comb, n, stream) / n
+            lay_ms = time_block(both, n, stream) / n
+            grp_ms = time_block(lambda i: mole.mole_token_groups_build(ids, V, N, groups=groups, stream=stream), n,
+                                stream) / n
+            assert mole.mole_check(stream) == 0
+            link = U * (N * (D // 64) * 26 if nf3 else row)
+            res["cases"][f"T{T}{'_nf3' if nf3 else ''}"] = {
+                "unique_rows": U, "link_bytes_per_layer": link, "link_bytes_per_token": link / T,
+                "stage_us": st_ms * 1e3, "stage_link_gbs": link / (st_ms / 1e3) / 1e9,
+                "stage_frac_of_copy_engine": link / (st_ms / 1e3) / 1e9 / ce_gbs,
+                "combine_us": cb_ms * 1e3, "layer_us": lay_ms * 1e3, "token_groups_build_us": grp_ms * 1e3,
+                "tokens_per_s_per_layer": T / (lay_ms / 1e3),
+                "moe_bytes_per_layer_all_experts": N * moe_expert_bytes,
+                "moe_over_mole_bytes_top1_per_token": moe_expert_bytes / (link / T)}
+            del groups, staging, h, out, ids
+    # decode step over L layers (one host table serves as every layer's: the link
+    # traffic per layer is the same), sequential vs the next layer's staging
+    # overlapped with this layer's combine
+    side = torch.cuda.Stream(device=dev)
+    for T in (1, 64):
+        ids = torch.from_numpy(inputs.draw_ids(rng, T, V, "zipf")).to(dev)
+        groups = torch.empty(mole.mole_token_groups_workspace(T, N), dtype=torch.uint8, device=dev)
+        nbytes = mole.mole_offload_staging_bytes(T, V, N, D)
+        stg = [torch.empty(nbytes, dtype=torch.uint8, device=dev) for _ in range(2)]
+        hs_l = [torch.randn((T, D), generator=g, device=dev).to(torch.bfloat16) for _ in range(L)]
+        out = torch.empty((T, D), dtype=torch.float32, device=dev)
+        e_st = [torch.cuda.Event() for _ in range(L)]
+        e_used = [torch.cuda.Event() for _ in range(2)]
+
+        def seq_step(i):
+            mole.mole_token_groups_build(ids, V, N, groups=groups, stream=stream)
+            for lay in range(L):
+                mole.mole_offload_stage(T, groups, host, staging=stg[0], stream=stream)
+                mole.mole_lookup_combine_offload(groups, hs_l[lay], routers[lay], stg[0], V, out=out, stream=stream)
+
+        def pipe_step(i):
+            mole.mole_token_groups_build(ids, V, N, groups=groups, stream=stream)
+            side.wait_stream(stream)
+            mole.mole_offload_stage(T, groups, host, staging=stg[0], stream=side)
+            e_st[0].record(side)
+            for lay in range(L):
+                if lay + 1 < L:
+                    b = (lay + 1) % 2
+                    if lay + 1 >= 2:
+                        side.wait_event(e_used[b])
+                    mole.mole_offload_stage(T, groups, host, staging=stg[b], stream=side)
+                    e_st[lay + 1].record(side)
+                stream.wait_event(e_st[lay])
+                mole.mole_lookup_combine_offload(groups, hs_l[lay], routers[lay], stg[lay % 2], V, out=out,
+                                                 stream=stream)
+                e_used[lay % 2].record(stream)
+
+        for i in range(3):
+            seq_step(i)
+            pipe_step(i)
+        n = 20
+        seq_ms = time_block(seq_step, n, stream) / n
+        pipe_ms = time_block(pipe_step, n, stream) / n
+        assert mole.mole_check(stream) == 0
+        res["cases"][f"decode_T{T}_{L}layers"] = {
+            "sequential_us_per_step": seq_ms * 1e3, "overlapped_us_per_step": pipe_ms * 1e3,
+            "tokens_per_s": T / (pipe_ms / 1e3),
+            "note": "per step: the grouping, then per layer the staging of its rows from host memory and its "
+                    "combine; overlapped = the next layer staged on a second stream into the other staging buffer"}
+        del ids, groups, stg, hs_l, out
+    del host, hc, hs
+    return res
 
 
 def build_leg(mole, dev, stream, bf16_peak, bf16_sust, peak_kind, reps=3, warmup=1, experts=None):

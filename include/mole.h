@@ -219,6 +219,56 @@ mole_status mole_lookup_combine_nf3_groups(const int32_t* ids, int64_t T, const 
                                            const uint16_t* scales, int64_t V, int32_t N, int64_t D, mole_dtype dt,
                                            float* out, cudaStream_t stream);
 
+/*
+ * ---- Offloaded table (MoLE page, 推理阶段 and 复杂度分析) ----
+ *
+ * The page's deployment: the table lives in slower, larger memory (CPU memory
+ * or storage) and per token only its N expert-output rows move to the
+ * accelerator.  Here the table (or its NF3 codes and scales) stays in host
+ * memory that is pinned and mapped into the device's address space
+ * (cudaHostAlloc, or cudaHostRegister with cudaHostRegisterMapped; memory of
+ * the current device is accepted too).  Per batch each distinct id's row
+ * block crosses the link once, into a device staging buffer, and the combine
+ * reads the staging buffer.  Both calls take a grouping of the batch built by
+ * mole_token_groups_build (same T, V and N): it numbers the batch's distinct
+ * ids 0..U-1, and the staging buffer holds the row block of distinct id u at
+ * index u.
+ *
+ * mole_offload_staging_bytes: size of the staging buffer for a batch of T
+ *   tokens over a table of V ids (room for min(T, V) row blocks).  nf3 = 0:
+ *   the table has dtype dt, [V, N, D]; nf3 = 1: NF3 codes [V, N, D/64, 24]
+ *   and fp16 scales [V, N, D/64] (D % 64 == 0).  0 for invalid arguments.
+ *
+ * mole_offload_stage copies the batch's distinct row blocks from `table`
+ *   (and, NF3, `scales`) into `staging` (device, 16-byte aligned, at least
+ *   mole_offload_staging_bytes bytes).  table must be 16-byte aligned (NF3
+ *   codes 8-byte, scales 2-byte).  If n_rows is not NULL it receives U (one
+ *   device int32).  Pageable (unregistered) host memory gives MOLE_ERR_ARG.
+ *   One kernel launch; the host table must stay unchanged until it has run.
+ *
+ * mole_lookup_combine_offload is mole_lookup_combine (or, nf3 = 1,
+ *   mole_lookup_combine_nf3) over the staged rows: the same results, bit for
+ *   bit, as those calls on the table itself, and the same error behaviour
+ *   (a token whose id is outside [0, V) gets a NaN row).  No ids argument:
+ *   the grouping holds each token's dense index.  Calls that share a groups
+ *   buffer must not overlap on the GPU (the call writes the layer's gates
+ *   into it); a staging buffer may be refilled for the next layer once the
+ *   combine that reads it has run, so two staging buffers let the next
+ *   layer's copy overlap this layer's combine.
+ *
+ * Both return MOLE_ERR_WORKSPACE for a missing or too small groups or staging
+ * buffer; T == 0 is a no-op.
+ */
+size_t mole_offload_staging_bytes(int64_t T, int64_t V, int32_t N, int64_t D, mole_dtype dt, int32_t nf3);
+mole_status mole_offload_stage(int64_t T, const void* groups, size_t bytes, const void* table,
+                               const uint16_t* scales, int64_t V, int32_t N, int64_t D, mole_dtype dt,
+                               int32_t nf3, void* staging, size_t staging_bytes, int32_t* n_rows,
+                               cudaStream_t stream);
+mole_status mole_lookup_combine_offload(int64_t T, const void* groups, size_t bytes, const void* h,
+                                        const void* Wr, const void* staging, size_t staging_bytes, int64_t V,
+                                        int32_t N, int64_t D, mole_dtype dt, int32_t nf3, float* out,
+                                        cudaStream_t stream);
+
 /* The 8 NF3 levels as fp16 bit patterns (ascending; index 3 is 0.0) and the 7
  * fp32 decision midpoints.  Host-only; no device work. */
 void mole_nf3_levels(uint16_t levels_f16[8]);

@@ -209,3 +209,57 @@ extern "C" mole_status mole_gather_plan(const int32_t* ids, int64_t T, int64_t V
   if (st != MOLE_OK) return st;
   return mole::gather_plan_launch(ids, T, V, uniq, n_uniq, slot, stream);
 }
+
+namespace {
+// Shared checks of the offloaded-table entry points.
+mole_status check_offload(int64_t T, const void* groups, size_t bytes, int64_t V, int32_t N, int64_t D,
+                          mole_dtype dt, int32_t nf3, const void* staging, size_t staging_bytes) {
+  if (!valid_dtype(dt) || (nf3 != 0 && nf3 != 1)) return MOLE_ERR_ARG;
+  if (T < 0 || V <= 0 || V > INT32_MAX || N <= 0 || D <= 0 || D > (1 << 20)) return MOLE_ERR_ARG;
+  if (N > 32 || T > mole::kMaxOffloadT) return MOLE_ERR_UNSUPPORTED;
+  if (nf3 ? D % 64 != 0 : (dt == MOLE_BF16 ? D % 16 != 0 : D % 4 != 0)) return MOLE_ERR_UNSUPPORTED;
+  mole_status st = check_groups(T, N, groups, bytes);
+  if (st != MOLE_OK || T == 0) return st;
+  if (!staging || staging_bytes < mole::offload_staging_bytes(T, V, N, (int)D, (int)dtype_size(dt), nf3 != 0))
+    return MOLE_ERR_WORKSPACE;
+  if (!mole::aligned16(staging)) return MOLE_ERR_ALIGN;
+  return MOLE_OK;
+}
+}  // namespace
+
+extern "C" size_t mole_offload_staging_bytes(int64_t T, int64_t V, int32_t N, int64_t D, mole_dtype dt,
+                                             int32_t nf3) {
+  if (T <= 0 || V <= 0 || N <= 0 || N > 32 || D <= 0 || !valid_dtype(dt) || (nf3 != 0 && nf3 != 1)) return 0;
+  if (nf3 && D % 64 != 0) return 0;
+  return mole::offload_staging_bytes(T, V, N, (int)D, (int)dtype_size(dt), nf3 != 0);
+}
+
+extern "C" mole_status mole_offload_stage(int64_t T, const void* groups, size_t bytes, const void* table,
+                                          const uint16_t* scales, int64_t V, int32_t N, int64_t D, mole_dtype dt,
+                                          int32_t nf3, void* staging, size_t staging_bytes, int32_t* n_rows,
+                                          cudaStream_t stream) {
+  mole_status st = check_offload(T, groups, bytes, V, N, D, dt, nf3, staging, staging_bytes);
+  if (st != MOLE_OK || T == 0) return st;
+  if (!table || (nf3 && !scales)) return MOLE_ERR_ARG;
+  if (reinterpret_cast<uintptr_t>(n_rows) & 3u) return MOLE_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(table) & (nf3 ? 7u : 15u)) || (nf3 && (reinterpret_cast<uintptr_t>(scales) & 1u)))
+    return MOLE_ERR_ALIGN;
+  st = check_device();
+  if (st != MOLE_OK) return st;
+  return mole::offload_stage(groups, bytes, T, table, scales, V, N, (int)D, (int)dtype_size(dt), nf3 != 0, staging,
+                             staging_bytes, n_rows, stream);
+}
+
+extern "C" mole_status mole_lookup_combine_offload(int64_t T, const void* groups, size_t bytes, const void* h,
+                                                   const void* Wr, const void* staging, size_t staging_bytes,
+                                                   int64_t V, int32_t N, int64_t D, mole_dtype dt, int32_t nf3,
+                                                   float* out, cudaStream_t stream) {
+  mole_status st = check_offload(T, groups, bytes, V, N, D, dt, nf3, staging, staging_bytes);
+  if (st != MOLE_OK || T == 0) return st;
+  if (!h || !Wr || !out) return MOLE_ERR_ARG;
+  if (!mole::aligned16(h) || !mole::aligned16(out)) return MOLE_ERR_ALIGN;
+  st = check_device();
+  if (st != MOLE_OK) return st;
+  return mole::combine_offload(groups, bytes, T, h, Wr, staging, staging_bytes, V, N, (int)D, dt == MOLE_BF16,
+                               nf3 != 0, out, stream);
+}

@@ -170,6 +170,18 @@ mole_status combine_grouped_dispatch(const int32_t* ids, int64_t T, const void* 
                                      const void* table, const uint16_t* scales, int64_t V, int N, int D,
                                      bool bf16_inputs, int table_kind, float* out, void* ws, size_t ws_bytes,
                                      cudaStream_t stream);
+// Offloaded table (grouped.cu): the batch's distinct row blocks staged from a
+// table the device reads in place (pinned host memory), and the combine that
+// reads the staging buffer.
+// Largest batch a token grouping (and so an offloaded-table call) takes.
+constexpr int64_t kMaxOffloadT = int64_t(1) << 30;
+size_t offload_staging_bytes(int64_t T, int64_t V, int N, int D, int elem_bytes, bool nf3);
+mole_status offload_stage(const void* buf, size_t bytes, int64_t T, const void* table, const void* scales,
+                          int64_t V, int N, int D, int elem_bytes, bool nf3, void* staging, size_t staging_bytes,
+                          int* n_rows, cudaStream_t stream);
+mole_status combine_offload(const void* buf, size_t bytes, int64_t T, const void* h, const void* Wr,
+                            const void* staging, size_t staging_bytes, int64_t V, int N, int D, bool bf16_inputs,
+                            bool nf3, float* out, cudaStream_t stream);
 void nf3_tables(uint16_t levels[8], float mid[7]);
 mole_status gather_plan_launch(const int32_t* ids, int64_t T, int64_t V, int32_t* uniq,
                                int32_t* n_uniq, int32_t* slot, cudaStream_t stream);

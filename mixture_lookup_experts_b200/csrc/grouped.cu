@@ -44,15 +44,16 @@ constexpr int kItemTokens = 16;     // tokens per work item
 constexpr int kPlanThreads = 256;
 constexpr int kPlanMaxGrid = 1024;
 constexpr int64_t kGroupedMinT = 1024;
-constexpr int64_t kGroupedMaxT = int64_t(1) << 30;
+constexpr int64_t kGroupedMaxT = kMaxOffloadT;
 
-// Per-CTA totals of step 1: [0] tokens, [n] work items of n tokens (n = 1..kItemTokens).
+// Per-CTA totals of step 1: [0] tokens, [n] work items of n tokens (n =
+// 1..kItemTokens), [kAgg] distinct ids.
 constexpr int kAgg = kItemTokens + 1;
 
 // Control words (set to 0xFFFFFFFF when a grouping is built): work items,
 // the three grid-barrier counters, the abort word, and the running totals of
 // step 1 (value + 1 = the sum so far).
-enum : int { kCtlItems = 1, kCtlBar = 2, kCtlAbort = 5, kCtlTot = 8, kCtlWords = kCtlTot + kAgg };
+enum : int { kCtlItems = 1, kCtlBar = 2, kCtlAbort = 5, kCtlTot = 8, kCtlWords = kCtlTot + kAgg + 1 };
 
 // The grouping of one batch (the caller's buffer, carved by carve_ws).
 struct GroupWs {
@@ -64,7 +65,10 @@ struct GroupWs {
   int* tok_rank;  // [T] rank of token t in its id's group
   int* tok_pos;   // [T] list position of token t (-1 for a bad id)
   int* list;      // [T] tokens grouped by id
-  int4* items;    // [T + T / kItemTokens + 1] {id, first list position, tokens, 0}
+  int4* items;    // [T + T / kItemTokens + 1] {id, first list position, tokens, dense index of the id}
+  int* uid_id;    // [T] the id of each dense index (distinct ids numbered 0..U-1)
+  int* slot_uid;  // [hcap] dense index of the slot's id
+  int* tok_uid;   // [T] dense index of token t's id (-1 for a bad id)
   float* gates;   // [T][NP] one layer's gates by list position
   int hcap_log2;
   size_t clear_bytes;  // key .. ctl, one contiguous range
@@ -91,6 +95,9 @@ size_t carve_ws(void* base, int64_t T, int NP, GroupWs* w) {
   const size_t o_tpos = take(4 * (size_t)T);
   const size_t o_list = take(4 * (size_t)T);
   const size_t o_items = take(16 * (size_t)(T + T / kItemTokens + 1));
+  const size_t o_uid = take(4 * (size_t)T);
+  const size_t o_suid = take(4 * (size_t)hcap);
+  const size_t o_tuid = take(4 * (size_t)T);
   const size_t o_gates = take(4 * (size_t)T * NP);
   if (w != nullptr && base != nullptr) {
     uint8_t* b = static_cast<uint8_t*>(base);
@@ -103,6 +110,9 @@ size_t carve_ws(void* base, int64_t T, int NP, GroupWs* w) {
     w->tok_pos = reinterpret_cast<int*>(b + o_tpos);
     w->list = reinterpret_cast<int*>(b + o_list);
     w->items = reinterpret_cast<int4*>(b + o_items);
+    w->uid_id = reinterpret_cast<int*>(b + o_uid);
+    w->slot_uid = reinterpret_cast<int*>(b + o_suid);
+    w->tok_uid = reinterpret_cast<int*>(b + o_tuid);
     w->gates = reinterpret_cast<float*>(b + o_gates);
     w->hcap_log2 = lg;
     w->clear_bytes = clear;
@@ -224,27 +234,30 @@ __device__ __forceinline__ int warp_sum(int v) {
   return v;
 }
 
-// Step 1: token and per-size item totals of this CTA's slot range, added to
-// the grid totals; the values the totals had before (in whatever order the
-// CTAs arrive) become this CTA's bases within each region.  `cls` and
-// `cbase` are kAgg ints of shared memory.
+// Step 1: token, per-size item and distinct-id totals of this CTA's slot
+// range, added to the grid totals; the values the totals had before (in
+// whatever order the CTAs arrive) become this CTA's bases within each region.
+// `cls` and `cbase` are kAgg + 1 ints of shared memory.
 __device__ void plan_count(const GroupWs& w, int* cls, int* cbase) {
   int64_t s0, s1;
   slot_range(w, s0, s1);
-  if (threadIdx.x < kAgg) cls[threadIdx.x] = 0;
+  if (threadIdx.x <= kAgg) cls[threadIdx.x] = 0;
   __syncthreads();
-  int sc = 0;
+  int sc = 0, su = 0;
   for (int64_t h = s0 + threadIdx.x; h < s1; h += kThreads) {
     if (w.key[h] == -1) continue;
     const int c = w.cnt[h] + 1;
     sc += c;
+    ++su;
     if (c >= kItemTokens) atomicAdd(&cls[kItemTokens], c / kItemTokens);
     if (c % kItemTokens) atomicAdd(&cls[c % kItemTokens], 1);
   }
   sc = warp_sum(sc);
+  su = warp_sum(su);
   if ((threadIdx.x & 31) == 0 && sc) atomicAdd(&cls[0], sc);
+  if ((threadIdx.x & 31) == 0 && su) atomicAdd(&cls[kAgg], su);
   __syncthreads();
-  if (threadIdx.x < kAgg) {
+  if (threadIdx.x <= kAgg) {
     const int v = cls[threadIdx.x];
     cbase[threadIdx.x] = v ? (int)(atomicAdd(&w.ctl[kCtlTot + threadIdx.x], (unsigned)v) + 1u) : 0;
   }
@@ -266,24 +279,27 @@ __device__ void plan_offsets(const GroupWs& w, const int* cbase, int* cur, int* 
     if (blockIdx.x == 0) w.ctl[kCtlItems] = (unsigned)acc;
   }
   __syncthreads();
-  int bt = cbase[0];
+  int bt = cbase[0], bu = cbase[kAgg];
   for (int64_t base = s0; base < s1; base += kThreads) {
     const int64_t h = base + threadIdx.x;
     const int id = h < s1 ? w.key[h] : -1;
     const int c = id != -1 ? w.cnt[h] + 1 : 0;
-    int pc = c, unused = 0, sc, su;
-    block_scan2(pc, unused, sc, su, red);
+    int pc = c, pu = id != -1 ? 1 : 0, sc, su;
+    block_scan2(pc, pu, sc, su, red);
     if (id != -1) {
-      const int o = bt + pc;
+      const int o = bt + pc, uid = bu + pu;
       w.off[h] = o;
+      w.slot_uid[h] = uid;
+      w.uid_id[uid] = id;
       const int nf = c / kItemTokens, r = c % kItemTokens;
       if (nf) {
         const int p0 = atomicAdd(&cur[kItemTokens], nf);
-        for (int k = 0; k < nf; ++k) w.items[p0 + k] = make_int4(id, o + k * kItemTokens, kItemTokens, 0);
+        for (int k = 0; k < nf; ++k) w.items[p0 + k] = make_int4(id, o + k * kItemTokens, kItemTokens, uid);
       }
-      if (r) w.items[atomicAdd(&cur[r], 1)] = make_int4(id, o + nf * kItemTokens, r, 0);
+      if (r) w.items[atomicAdd(&cur[r], 1)] = make_int4(id, o + nf * kItemTokens, r, uid);
     }
     bt += sc;
+    bu += su;
   }
 }
 
@@ -324,7 +340,8 @@ __device__ void plan_insert_tokens(const int32_t* __restrict__ ids, int64_t T, i
   }
 }
 
-// Step 3: every token of this CTA to its list position.
+// Step 3: every token of this CTA to its list position (and its id's dense
+// index).
 __device__ void plan_scatter(const GroupWs& w, int64_t T) {
   int64_t t0, t1;
   token_range(T, t0, t1);
@@ -332,6 +349,7 @@ __device__ void plan_scatter(const GroupWs& w, int64_t T) {
     const int slot = w.tok_slot[t];
     const int pos = slot >= 0 ? w.off[slot] + w.tok_rank[t] : -1;
     w.tok_pos[t] = pos;
+    w.tok_uid[t] = slot >= 0 ? w.slot_uid[slot] : -1;
     if (pos >= 0) w.list[pos] = (int)t;
   }
 }
@@ -339,7 +357,7 @@ __device__ void plan_scatter(const GroupWs& w, int64_t T) {
 __global__ void __launch_bounds__(kPlanThreads) group_plan_kernel(const int32_t* __restrict__ ids, int64_t T,
                                                                    int64_t V, const GroupWs w, unsigned* err) {
   __shared__ int red[2 * kWarps];
-  __shared__ int cls[kAgg], cbase[kAgg];
+  __shared__ int cls[kAgg + 1], cbase[kAgg + 1];
   __shared__ int flag;
   plan_insert_tokens(ids, T, V, w, err);
   grid_arrive(&w.ctl[kCtlBar + 0]);
@@ -363,6 +381,10 @@ struct GArgs {
   int N, D;
   float* out;
   unsigned* err;
+  // by_uid: the table holds the batch's distinct ids' row blocks by dense
+  // index (a staging buffer of `rows` blocks), not the whole vocabulary
+  int by_uid;
+  int64_t rows;
 };
 
 // One layer's router: gates to the tokens' list positions; a token with a
@@ -622,7 +644,7 @@ __global__ void __launch_bounds__(kGroupThreads, 1) grouped_gather_kernel(const 
     uint32_t q = 0, ph = 0, issued = 0;
     bool ok = true;
     for (int k = 0; ok && k < my_n; ++k) {
-      const int id = __shfl_sync(0xffffffffu, my_item.x, k - k0);
+      const int id = __shfl_sync(0xffffffffu, p.by_uid ? my_item.w : my_item.x, k - k0);
       const int pos = __shfl_sync(0xffffffffu, my_item.y, k - k0);
       const int n = __shfl_sync(0xffffffffu, my_item.z, k - k0);
       const int tok = next_tok;
@@ -635,6 +657,11 @@ __global__ void __launch_bounds__(kGroupThreads, 1) grouped_gather_kernel(const 
         const int pos1 = __shfl_sync(0xffffffffu, my_item.y, k + 1 - k0);
         const int n1 = __shfl_sync(0xffffffffu, my_item.z, k + 1 - k0);
         next_tok = lane < n1 ? w.list[pos1 + lane] : -1;
+      }
+      if (p.by_uid && (int64_t)id >= p.rows) {  // staging buffer smaller than the batch's distinct ids
+        if (lane == 0) atomicOr(p.err, kErrIndex);
+        *abort = 1;
+        break;
       }
       ok = warp_wait(&empty[q], ph ^ 1u, abort, p.err);
       if (!ok) break;
@@ -836,7 +863,195 @@ bool grouped_applies(int64_t T, int N, int D, bool nf3) {
   return L.n_slots >= 2 && smem_bytes_for<true, 32>(D) <= 227 * 1024;
 }
 
+// ---- Offloaded table: the batch's distinct row blocks into a staging buffer ----
+// The table stays in host memory (pinned and mapped into the device's address
+// space) or anywhere else the device can read.  Per batch, each distinct id's
+// row block crosses the link once, read by the SMs with 16-byte loads (many in
+// flight per thread: the link's latency is microseconds), and lands in a
+// device staging buffer at the id's dense index; the combine then reads the
+// staging buffer instead of the table.
+
+constexpr int kStageThreads = 256;
+constexpr int kStageUnroll = 4;    // accesses in flight per thread
+constexpr int kStageCtasPerSm = 8;
+
+// One array of per-id row blocks (the bf16/fp32 table, or the NF3 codes or
+// scales): row block of id v at src + v * row_bytes, staged to dst + u * row_bytes.
+struct StagePlane {
+  const uint8_t* src;
+  uint8_t* dst;
+  int64_t row_bytes;
+  int vec;  // bytes per access (16, 8, 4 or 2), dividing row_bytes and both bases
+};
+
+// Staging buffer layout for `rows` row blocks: the table's (or the NF3
+// codes') blocks, then (NF3) the scale blocks from scales_off.
+struct StageLayout {
+  int64_t rows, row_bytes, scale_row_bytes, scales_off, total;
+};
+
+StageLayout stage_layout(int64_t rows, int N, int D, int elem_bytes, bool nf3) {
+  StageLayout L{};
+  L.rows = rows;
+  if (nf3) {
+    const int64_t nb = (int64_t)N * (D / 64);
+    L.row_bytes = nb * 24;
+    L.scale_row_bytes = nb * 2;
+    L.scales_off = (rows * L.row_bytes + 255) / 256 * 256;
+    L.total = L.scales_off + rows * L.scale_row_bytes;
+  } else {
+    L.row_bytes = (int64_t)N * D * elem_bytes;
+    L.total = rows * L.row_bytes;
+  }
+  return L;
+}
+
+template <typename Vec>
+__device__ __forceinline__ void stage_plane(const StagePlane& pl, const int* __restrict__ uid_id, int64_t U,
+                                            int64_t V, unsigned* err) {
+  const int64_t per_row = pl.row_bytes / (int64_t)sizeof(Vec);
+  const int64_t cpr = (per_row + kStageThreads - 1) / kStageThreads;  // chunks of a row block
+  const int64_t tasks = U * cpr;
+  // a CTA takes kStageUnroll consecutive chunks at a time: all loads first
+  for (int64_t t0 = (int64_t)blockIdx.x * kStageUnroll; t0 < tasks; t0 += (int64_t)gridDim.x * kStageUnroll) {
+    Vec v[kStageUnroll];
+    int64_t at[kStageUnroll];
+#pragma unroll
+    for (int k = 0; k < kStageUnroll; ++k) {
+      at[k] = -1;
+      const int64_t task = t0 + k;
+      if (task < tasks) {
+        const int64_t u = task / cpr;
+        const int64_t e = (task - u * cpr) * kStageThreads + threadIdx.x;
+        const int id = uid_id[u];
+        if (id < 0 || (int64_t)id >= V) {  // a grouping built with a larger vocabulary
+          if (e == 0) atomicOr(err, kErrIndex);
+        } else if (e < per_row) {
+          v[k] = reinterpret_cast<const Vec*>(pl.src + (int64_t)id * pl.row_bytes)[e];
+          at[k] = u * per_row + e;
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kStageUnroll; ++k)
+      if (at[k] >= 0) reinterpret_cast<Vec*>(pl.dst)[at[k]] = v[k];
+  }
+}
+
+__device__ __forceinline__ void stage_any(const StagePlane& pl, const int* uid_id, int64_t U, int64_t V,
+                                          unsigned* err) {
+  switch (pl.vec) {
+    case 16: stage_plane<uint4>(pl, uid_id, U, V, err); break;
+    case 8: stage_plane<uint2>(pl, uid_id, U, V, err); break;
+    case 4: stage_plane<uint32_t>(pl, uid_id, U, V, err); break;
+    default: stage_plane<uint16_t>(pl, uid_id, U, V, err); break;
+  }
+}
+
+__global__ void __launch_bounds__(kStageThreads) stage_rows_kernel(const GroupWs w, const StagePlane a,
+                                                                   const StagePlane b, int n_planes, int64_t V,
+                                                                   int64_t cap, int* n_rows, unsigned* err) {
+  int64_t U = 0;
+  if (ld_relaxed_u32(&w.ctl[kCtlAbort]) == 0xFFFFFFFFu) U = (int64_t)(ld_relaxed_u32(&w.ctl[kCtlTot + kAgg]) + 1u);
+  if (U > cap) {  // more distinct ids than the staging buffer holds: the grouping is not this table's
+    if (blockIdx.x == 0 && threadIdx.x == 0) atomicOr(err, kErrIndex);
+    U = cap;
+  }
+  if (n_rows != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *n_rows = (int)U;
+  stage_any(a, w.uid_id, U, V, err);
+  if (n_planes > 1) stage_any(b, w.uid_id, U, V, err);
+}
+
+// The device's address of `p` (pinned host memory mapped into the device's
+// address space, or memory of the current device), or nullptr.
+const void* device_view(const void* p) {
+  cudaPointerAttributes a{};
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  if (a.type == cudaMemoryTypeHost || a.type == cudaMemoryTypeManaged) return a.devicePointer;
+  if (a.type == cudaMemoryTypeDevice) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || a.device != dev) return nullptr;
+    return a.devicePointer;
+  }
+  return nullptr;  // pageable host memory: not readable by the device
+}
+
+int access_bytes(int64_t row_bytes, const void* src, const void* dst) {
+  const uintptr_t m = reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst) | (uintptr_t)row_bytes;
+  return (m & 15u) == 0 ? 16 : (m & 7u) == 0 ? 8 : (m & 3u) == 0 ? 4 : 2;
+}
+
 }  // namespace
+
+size_t offload_staging_bytes(int64_t T, int64_t V, int N, int D, int elem_bytes, bool nf3) {
+  return (size_t)stage_layout(std::min(T, V), N, D, elem_bytes, nf3).total;
+}
+
+mole_status offload_stage(const void* buf, size_t bytes, int64_t T, const void* table, const void* scales,
+                          int64_t V, int N, int D, int elem_bytes, bool nf3, void* staging, size_t staging_bytes,
+                          int* n_rows, cudaStream_t stream) {
+  GroupWs w{};
+  if (carve_ws(const_cast<void*>(buf), T, padded_experts(N), &w) > bytes) return MOLE_ERR_WORKSPACE;
+  const StageLayout L = stage_layout(std::min(T, V), N, D, elem_bytes, nf3);
+  if ((size_t)L.total > staging_bytes) return MOLE_ERR_WORKSPACE;
+  const void* src = device_view(table);
+  const void* ssrc = nf3 ? device_view(scales) : nullptr;
+  if (src == nullptr || (nf3 && ssrc == nullptr)) return MOLE_ERR_ARG;
+  uint8_t* dst = static_cast<uint8_t*>(staging);
+  StagePlane a{static_cast<const uint8_t*>(src), dst, L.row_bytes, 0};
+  a.vec = access_bytes(a.row_bytes, a.src, a.dst);
+  StagePlane b = a;
+  if (nf3) {
+    b = StagePlane{static_cast<const uint8_t*>(ssrc), dst + L.scales_off, L.scale_row_bytes, 0};
+    b.vec = access_bytes(b.row_bytes, b.src, b.dst);
+  }
+  unsigned* err = error_word();
+  if (!err) return MOLE_ERR_CUDA;
+  const int n_sm = num_sms();
+  if (n_sm <= 0) return MOLE_ERR_NO_DEVICE;
+  // enough CTAs for every chunk of the largest possible batch, at most 8 per SM
+  const int64_t cpr = (L.row_bytes / a.vec + kStageThreads - 1) / kStageThreads;
+  const int64_t want = (L.rows * cpr + kStageUnroll - 1) / kStageUnroll;
+  const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)kStageCtasPerSm * n_sm));
+  stage_rows_kernel<<<grid, kStageThreads, 0, stream>>>(w, a, b, nf3 ? 2 : 1, V, L.rows, n_rows, err);
+  return cudaGetLastError() == cudaSuccess ? MOLE_OK : MOLE_ERR_CUDA;
+}
+
+mole_status combine_offload(const void* buf, size_t bytes, int64_t T, const void* h, const void* Wr,
+                            const void* staging, size_t staging_bytes, int64_t V, int N, int D, bool bf16_inputs,
+                            bool nf3, float* out, cudaStream_t stream) {
+  GroupWs w{};
+  if (carve_ws(const_cast<void*>(buf), T, padded_experts(N), &w) > bytes) return MOLE_ERR_WORKSPACE;
+  const int elem = bf16_inputs ? 2 : 4;
+  const StageLayout L = stage_layout(std::min(T, V), N, D, elem, nf3);
+  if ((size_t)L.total > staging_bytes) return MOLE_ERR_WORKSPACE;
+  const uint8_t* st = static_cast<const uint8_t*>(staging);
+  const uint16_t* sc = nf3 ? reinterpret_cast<const uint16_t*>(st + L.scales_off) : nullptr;
+  if (bf16_inputs && grouped_applies(T, N, D, nf3) && aligned16(Wr) && aligned16(st)) {
+    GArgs p{};
+    p.T = T;
+    p.h = static_cast<const uint16_t*>(h);
+    p.Wr = static_cast<const uint16_t*>(Wr);
+    p.table = reinterpret_cast<const uint16_t*>(st);
+    p.codes = st;
+    p.scales = sc;
+    p.N = N;
+    p.D = D;
+    p.out = out;
+    p.err = error_word();
+    p.by_uid = 1;
+    p.rows = L.rows;
+    if (!p.err) return MOLE_ERR_CUDA;
+    const mole_status s = nf3 ? layer_dispatch<true>(p, w, stream) : layer_dispatch<false>(p, w, stream);
+    if (s != MOLE_ERR_UNSUPPORTED) return s;
+  }
+  // the ungrouped kernels, addressing the staging buffer by each token's dense index
+  return combine_dispatch(w.tok_uid, T, h, Wr, st, sc, L.rows, N, D, bf16_inputs, nf3 ? 2 : (bf16_inputs ? 0 : 1),
+                          out, stream);
+}
 
 size_t token_groups_bytes(int64_t T, int N) {
   if (T <= 0 || N <= 0 || N > 32) return 0;

@@ -46,6 +46,9 @@ SIGNATURES = {
     "mole_quantize_lut_nf3": ([_P, _I64, _I32, _I64, _P, _P, _P], _I),
     "mole_lookup_combine_nf3": ([_P, _I64, _P, _P, _P, _P, _I64, _I32, _I64, _I, _P, _P], _I),
     "mole_lookup_combine_nf3_groups": ([_P, _I64, _P, _SZ, _P, _P, _P, _P, _I64, _I32, _I64, _I, _P, _P], _I),
+    "mole_offload_staging_bytes": ([_I64, _I64, _I32, _I64, _I, _I32], _SZ),
+    "mole_offload_stage": ([_I64, _P, _SZ, _P, _P, _I64, _I32, _I64, _I, _I32, _P, _SZ, _P, _P], _I),
+    "mole_lookup_combine_offload": ([_I64, _P, _SZ, _P, _P, _P, _SZ, _I64, _I32, _I64, _I, _I32, _P, _P], _I),
     "mole_nf3_levels": ([_P], None),
     "mole_nf3_midpoints": ([_P], None),
     "mole_gather_plan": ([_P, _I64, _I64, _P, _P, _P, _P], _I),
@@ -257,6 +260,54 @@ def mole_lookup_combine_nf3_groups(ids: torch.Tensor, groups: torch.Tensor, h: t
     _ok(lib.mole_lookup_combine_nf3_groups(_ptr(ids), T, _ptr(groups), nbytes, _ptr(h), _ptr(Wr), _ptr(codes),
                                            _ptr(scales), V, N, D, _dt(h), _ptr(out), _stream(stream)),
         "mole_lookup_combine_nf3_groups")
+    return out
+
+
+def mole_offload_staging_bytes(T: int, V: int, N: int, D: int, dtype=torch.bfloat16, nf3: bool = False) -> int:
+    dt = BF16 if dtype == torch.bfloat16 else F32
+    return int(lib.mole_offload_staging_bytes(T, V, N, D, dt, int(nf3)))
+
+
+def _table_shape(table: torch.Tensor, scales: torch.Tensor | None):
+    """(V, N, D, nf3) of a [V, N, D] table or NF3 codes [V, N, D/64, 24]."""
+    if scales is None:
+        V, N, D = table.shape
+        return V, N, D, False
+    V, N, nb, _ = table.shape
+    return V, N, nb * 64, True
+
+
+def mole_offload_stage(T: int, groups: torch.Tensor, table: torch.Tensor, scales: torch.Tensor | None = None,
+                       staging: torch.Tensor | None = None, n_rows: torch.Tensor | None = None,
+                       device=None, stream=None) -> torch.Tensor:
+    """Copies the batch's distinct row blocks of `table` (pinned host memory;
+    with `scales`, NF3 codes and scales) into a device staging buffer, by
+    the dense index the grouping gave each id (see mole.h)."""
+    _contig(groups, table, scales, staging, n_rows)
+    V, N, D, nf3 = _table_shape(table, scales)
+    dtype = torch.bfloat16 if nf3 else table.dtype
+    if staging is None:
+        nbytes = max(1, mole_offload_staging_bytes(T, V, N, D, dtype, nf3))
+        staging = torch.empty(nbytes, dtype=torch.uint8, device=device if device is not None else groups.device)
+    _ok(lib.mole_offload_stage(T, _ptr(groups), groups.numel(), _ptr(table), _ptr(scales), V, N, D,
+                               BF16 if dtype == torch.bfloat16 else F32, int(nf3), _ptr(staging), staging.numel(),
+                               _ptr(n_rows), _stream(stream)), "mole_offload_stage")
+    return staging
+
+
+def mole_lookup_combine_offload(groups: torch.Tensor, h: torch.Tensor, Wr: torch.Tensor, staging: torch.Tensor,
+                                V: int, nf3: bool = False, out: torch.Tensor | None = None,
+                                stream=None) -> torch.Tensor:
+    """mole_lookup_combine (nf3: mole_lookup_combine_nf3) over the rows that
+    mole_offload_stage put into `staging`; same result bit for bit."""
+    _contig(groups, h, Wr, staging, out)
+    T, D = h.shape
+    N = Wr.shape[1]
+    if out is None:
+        out = torch.empty((T, D), dtype=torch.float32, device=h.device)
+    _ok(lib.mole_lookup_combine_offload(T, _ptr(groups), groups.numel(), _ptr(h), _ptr(Wr), _ptr(staging),
+                                        staging.numel(), V, N, D, _dt(h), int(nf3), _ptr(out), _stream(stream)),
+        "mole_lookup_combine_offload")
     return out
 
 

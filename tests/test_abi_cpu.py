@@ -116,3 +116,38 @@ def test_token_groups_checks(mole):
     assert lib.mole_lookup_combine_groups(P, 5, None, ws, P, P, P, 10, 4, 64, 1, P, None) == 4
     assert lib.mole_lookup_combine_groups(P, 5, P, ws, P, P, P, 10, 4, 24, 1, P, None) == 3
     assert lib.mole_lookup_combine_groups(P, 0, None, 0, P, P, P, 10, 4, 64, 1, P, None) == 0
+
+
+def test_offload_staging_size_and_checks(mole):
+    import torch
+    size = mole.mole_offload_staging_bytes
+    # room for min(T, V) row blocks
+    assert size(16384, 50304, 16, 2048) == 16384 * 16 * 2048 * 2
+    assert size(100, 40, 16, 2048) == 40 * 16 * 2048 * 2
+    assert size(100, 40, 8, 64, torch.float32) == 40 * 8 * 64 * 4
+    nb = 16 * 2048 // 64
+    assert size(1000, 50304, 16, 2048, nf3=True) == (1000 * nb * 24 + 255) // 256 * 256 + 1000 * nb * 2
+    assert size(0, 10, 4, 64) == 0 and size(5, 10, 33, 64) == 0 and size(5, 10, 4, 96, nf3=True) == 0
+    lib = mole.lib
+    P = 0x100000
+    gws = mole.mole_token_groups_workspace(5, 4)
+    sws = size(5, 10, 4, 64)
+    stage = lib.mole_offload_stage
+    assert stage(5, None, gws, P, None, 10, 4, 64, 1, 0, P, sws, None, None) == 4          # no groups
+    assert stage(5, P, gws, P, None, 10, 4, 64, 1, 0, P, sws - 1, None, None) == 4         # staging too small
+    assert stage(5, P, gws, P, None, 10, 4, 64, 1, 0, P + 8, sws, None, None) == 2         # staging misaligned
+    assert stage(5, P, gws, None, None, 10, 4, 64, 1, 0, P, sws, None, None) == 1          # no table
+    assert stage(5, P, gws, P + 8, None, 10, 4, 64, 1, 0, P, sws, None, None) == 2         # table misaligned
+    assert stage(5, P, gws, P, None, 10, 4, 64, 1, 1, P, size(5, 10, 4, 64, nf3=True), None, None) == 1  # no scales
+    assert stage(5, P, gws, P, None, 10, 4, 64, 1, 2, P, sws, None, None) == 1             # bad table kind
+    assert stage(5, P, gws, P, None, 10, 4, 24, 1, 0, P, sws, None, None) == 3             # D % 16
+    assert stage(5, P, gws, P, None, 10, 4, 64, 1, 0, P, sws, P + 2, None) == 2            # n_rows misaligned
+    assert stage(0, None, 0, None, None, 10, 4, 64, 1, 0, None, 0, None, None) == 0         # T == 0
+    comb = lib.mole_lookup_combine_offload
+    assert comb(5, P, gws, P, P, P, sws - 1, 10, 4, 64, 1, 0, P, None) == 4
+    assert comb(5, P, gws, None, P, P, sws, 10, 4, 64, 1, 0, P, None) == 1
+    assert comb(5, P, gws, P + 4, P, P, sws, 10, 4, 64, 1, 0, P, None) == 2
+    assert comb(0, None, 0, None, None, None, 0, 10, 4, 64, 1, 0, None, None) == 0
+    if not torch.cuda.is_available():
+        assert stage(5, P, gws, P, None, 10, 4, 64, 1, 0, P, sws, None, None) == 8
+        assert comb(5, P, gws, P, P, P, sws, 10, 4, 64, 1, 0, P, None) == 8
