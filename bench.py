@@ -74,6 +74,8 @@ def parse_args():
                     help="layer tables to allocate (default: the model's 16); fewer only for profiling runs")
     ap.add_argument("--no-extras", action="store_true", help="skip the build / NF3 / other-case legs")
     ap.add_argument("--no-offload", action="store_true", help="skip the host-resident (offloaded) table leg")
+    ap.add_argument("--no-decode", action="store_true", help="skip the small-batch (decode) sweeps")
+    ap.add_argument("--decode-only", action="store_true", help="run only the small-batch (decode) sweeps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--build-only", action="store_true",
@@ -321,6 +323,14 @@ def main():
     dev = torch.device("cuda", local_rank)
     stream = torch.cuda.current_stream()
 
+    if args.decode_only:
+        res = decode_leg(mole, dev, stream)
+        if rank == 0:
+            print(json.dumps({"decode": res}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
     if args.build_only:
         hbm_peak, bf16_peak, bf16_sust, peak_kind = measured_peaks()
         res = build_leg(mole, dev, stream, bf16_peak, bf16_sust, peak_kind, reps=max(1, args.steps),
@@ -443,6 +453,8 @@ def main():
             line["offload"] = offload_leg(mole, luts, routers, rng, g, dev, stream, W, L)
         del luts
         torch.cuda.empty_cache()
+        if not args.no_decode:
+            line["decode"] = decode_leg(mole, dev, stream)
         line["build"] = build_leg(mole, dev, stream, bf16_peak, bf16_sust, peak_kind)
 
     if rank == 0 and not args.no_cpu_baseline:
@@ -741,6 +753,111 @@ def offload_leg(mole, luts, routers, rng, g, dev, stream, W, L):
                     "combine; overlapped = the next layer staged on a second stream into the other staging buffer"}
         del ids, groups, stg, hs_l, out
     del host, hc, hs
+    return res
+
+
+def graph_pass_us(passes, stream, dev, replays=60):
+    """Median device time (us) of one replay of a CUDA graph captured from
+    each of `passes` (one graph per pooled batch, replayed in rotation), and
+    the same passes run eagerly (host-launched) for comparison.  Returns
+    (graph_us or None, eager_us, note)."""
+    import torch
+    P = len(passes)
+    for p in range(P):
+        passes[p]()
+    eager = time_block(lambda i: passes[i % P](), 4 * P, stream) / (4 * P) * 1e3
+    try:
+        graphs = []
+        side = torch.cuda.Stream(device=dev)
+        for p in range(P):
+            gr = torch.cuda.CUDAGraph()
+            side.wait_stream(stream)
+            with torch.cuda.graph(gr, stream=side, capture_error_mode="thread_local"):
+                passes[p]()
+            stream.wait_stream(side)
+            graphs.append(gr)
+    except Exception as e:  # capture not possible: report the eager time only
+        torch.cuda.synchronize()
+        return None, eager, f"graph capture failed: {type(e).__name__}: {str(e)[:120]}"
+    for i in range(3 * P):
+        graphs[i % P].replay()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(replays)]
+    for i in range(replays):
+        ev[i][0].record(stream)
+        graphs[i % P].replay()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    us = statistics.median(a.elapsed_time(b) for a, b in ev) * 1e3
+    del graphs
+    return us, eager, "median of CUDA-graph replays (one graph per pooled batch, rotated)"
+
+
+def decode_leg(mole, dev, stream):
+    """Small batches on the 160M- and 410M-shaped models (decode, T <= 256,
+    bf16 tables) and the NF3 1B-shaped sweep (T = 1 .. 16384).  One pass =
+    the combine of every layer (own table, router, hidden states; the batch's
+    ids shared), captured as a CUDA graph per pooled batch (4 batches,
+    rotated, so consecutive replays read other ids), timed as the median of
+    60 replays; the eager (host-launched) pass is reported beside it."""
+    import torch
+    hbm_peak = measured_peaks()[0]
+    res = {}
+    P = 4
+    sweeps = [("160m", (1, 8, 64), False), ("410m", (1, 2, 4, 8, 16, 32, 64, 128, 256), False),
+              ("1b_nf3", (1, 8, 64, 256, 1024, 4096, 16384), True)]
+    for name, Ts, nf3 in sweeps:
+        shape = inputs.SHAPES[name]
+        V, D, N, L = shape.V, shape.D, shape.N, shape.layers
+        g = torch.Generator(device=dev)
+        g.manual_seed(shape.seed)
+        tables = []
+        for _ in range(L):
+            lut = (torch.randn((V, N, D), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+            if nf3:
+                tables.append(mole.mole_quantize_lut_nf3(lut, stream=stream))
+                del lut
+            else:
+                tables.append(lut)
+        routers = [(torch.randn((D, N), generator=g, device=dev) * 0.02).to(torch.bfloat16) for _ in range(L)]
+        rng = np.random.default_rng(shape.seed)
+        for T in Ts:
+            ids = [torch.from_numpy(inputs.draw_ids(rng, T, V, "zipf")).to(dev) for _ in range(P)]
+            U = sum(int(torch.unique(x).numel()) for x in ids) / P
+            hs = [[torch.randn((T, D), generator=g, device=dev).to(torch.bfloat16) for _ in range(L)] for _ in range(P)]
+            outs = [torch.empty((T, D), dtype=torch.float32, device=dev) for _ in range(L)]
+            groups = [mole.mole_token_groups_build(x, V, N, stream=stream) for x in ids] if T >= 1024 else None
+
+            def make_pass(p):
+                def run():
+                    for lay in range(L):
+                        if nf3 and groups is not None:
+                            mole.mole_lookup_combine_nf3_groups(ids[p], groups[p], hs[p][lay], routers[lay],
+                                                                *tables[lay], out=outs[lay])
+                        elif nf3:
+                            mole.mole_lookup_combine_nf3(ids[p], hs[p][lay], routers[lay], *tables[lay],
+                                                         out=outs[lay])
+                        else:
+                            mole.mole_lookup_combine(ids[p], hs[p][lay], routers[lay], tables[lay], out=outs[lay])
+                return run
+
+            graph_us, eager_us, note = graph_pass_us([make_pass(p) for p in range(P)], stream, dev)
+            st = mole.mole_check(stream)
+            if st != 0:
+                raise RuntimeError(f"device status {st} in the {name} T={T} sweep")
+            pass_us = graph_us if graph_us is not None else eager_us
+            b = (nf3_bytes if nf3 else combine_bytes)(U, T, D, N)
+            res[f"{name}_T{T}"] = {
+                "us_per_layer_call": pass_us / L, "us_per_pass": pass_us, "eager_us_per_pass": eager_us,
+                "tokens_per_s": T / (pass_us / 1e6), "layer_tokens_per_s": T * L / (pass_us / 1e6),
+                "unique_rows": U, "achieved_gbs": b / (pass_us / L / 1e6) / 1e9,
+                "frac_of_measured_hbm": b / (pass_us / L / 1e6) / 1e9 / hbm_peak, "layers": L,
+                "call": ("mole_lookup_combine_nf3_groups (grouping built once per batch, outside the pass)"
+                         if nf3 and groups is not None else
+                         "mole_lookup_combine_nf3" if nf3 else "mole_lookup_combine"),
+                "timing": note}
+            del ids, hs, outs, groups
+        del tables, routers
+        torch.cuda.empty_cache()
     return res
 
 

@@ -514,6 +514,10 @@ __global__ void __launch_bounds__(kThreads, 2) combine_kernel(const CombineArgs 
   constexpr int NP = 8 * NT;
   extern __shared__ __align__(128) uint8_t smem_raw[];
   const Smem s = carve<kBf16Router, NP>(smem_raw, p.D);
+  // launched with programmatic stream serialization: the launch overlaps the
+  // previous kernel's tail; every input is read after it has completed
+  pdl_trigger();
+  pdl_wait();
   if (kBf16Router) {
     // (the element-wise staging: the fused kernel's registers are spoken for)
     stage_wrt<NP, kThreads, false>(s.wrt, static_cast<const uint16_t*>(p.Wr), p.N, p.D);
@@ -571,8 +575,7 @@ mole_status launch_one(CombineArgs p, cudaStream_t stream) {
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, smem) != cudaSuccess || occ < 1)
     return MOLE_ERR_UNSUPPORTED;
   const int64_t grid = std::min<int64_t>(p.n_tiles, (int64_t)occ * n_sm);
-  kern<<<(unsigned)grid, kThreads, smem, stream>>>(p);
-  return cuda_status(cudaGetLastError());
+  return cuda_status(launch_pdl(kern, (unsigned)grid, kThreads, smem, stream, p));
 }
 
 template <int NT, bool kExactN, int kTable, int kChunks>
