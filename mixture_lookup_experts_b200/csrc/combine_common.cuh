@@ -248,18 +248,29 @@ __device__ __forceinline__ void router_f32_partials(const Smem& s, const float* 
   }
 }
 
+// The whole CTA's barrier (the router's default).
+struct CtaSync {
+  __device__ __forceinline__ void operator()() const { __syncthreads(); }
+};
+
 // Barrier, sum of the partial logits, max-subtracted softmax over the N
 // experts (NP lanes per token row; padded experts get gate 0), barrier.  If
 // `ids` is given, s.tok_id[r] = ids[t0 + r] is loaded between the barriers
 // (before the first one, threads may still be reading the previous tile's
-// ids).  On return s.gates[r][j] is valid for r < rows.
-template <bool kBf16Router, int NT>
+// ids); with kOwnId, thread r stores its argument own_id there instead.  On
+// return s.gates[r][j] is valid for r < rows.  The barriers are Sync's (the
+// kThreads threads that run the router).
+template <bool kBf16Router, int NT, class Sync = CtaSync, bool kOwnId = false>
 __device__ __forceinline__ void router_softmax(const Smem& s, int rows, int N, const int32_t* __restrict__ ids,
-                                               int64_t t0) {
+                                               int64_t t0, int own_id = 0) {
   constexpr int NP = 8 * NT;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  __syncthreads();
-  if (ids != nullptr && tid < rows) s.tok_id[tid] = __ldg(ids + t0 + tid);
+  Sync{}();
+  if (kOwnId) {
+    if (tid < rows) s.tok_id[tid] = own_id;
+  } else if (ids != nullptr && tid < rows) {
+    s.tok_id[tid] = __ldg(ids + t0 + tid);
+  }
   constexpr int RPW = 32 / NP;
   const int sub = lane / NP, jl = lane % NP;
   for (int rb = warp * RPW; rb < rows; rb += kWarps * RPW) {
@@ -284,7 +295,7 @@ __device__ __forceinline__ void router_softmax(const Smem& s, int rows, int N, c
     for (int off = NP / 2; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
     if (act) s.gates[r * NP + jl] = valid ? e / sum : 0.f;
   }
-  __syncthreads();
+  Sync{}();
 }
 
 // Persistent router loop over this CTA's 16-token tiles (blockIdx.x,

@@ -51,9 +51,17 @@ constexpr int64_t kGroupedMaxT = kMaxOffloadT;
 constexpr int kAgg = kItemTokens + 1;
 
 // Control words (set to 0xFFFFFFFF when a grouping is built): work items,
-// the three grid-barrier counters, the abort word, and the running totals of
-// step 1 (value + 1 = the sum so far).
-enum : int { kCtlItems = 1, kCtlBar = 2, kCtlAbort = 5, kCtlTot = 8, kCtlWords = kCtlTot + kAgg + 1 };
+// the three grid-barrier counters, the abort word, the running totals of
+// step 1 (value + 1 = the sum so far), and the fused layer kernel's launch
+// counter.
+enum : int {
+  kCtlItems = 1,
+  kCtlBar = 2,
+  kCtlAbort = 5,
+  kCtlTot = 8,
+  kCtlLaunches = kCtlTot + kAgg + 1,  // 64-bit launch counter of the fused layer kernel (8-byte aligned)
+  kCtlWords = kCtlLaunches + 2
+};
 
 // The grouping of one batch (the caller's buffer, carved by carve_ws).
 struct GroupWs {
@@ -70,8 +78,9 @@ struct GroupWs {
   int* slot_uid;  // [hcap] dense index of the slot's id
   int* tok_uid;   // [T] dense index of token t's id (-1 for a bad id)
   float* gates;   // [T][NP] one layer's gates by list position
+  unsigned* tile_flag;  // [ceil(T / 16)] the fused layer kernel's router-tile flags
   int hcap_log2;
-  size_t clear_bytes;  // key .. ctl, one contiguous range
+  size_t clear_bytes;  // key .. ctl .. tile_flag, one contiguous range
 };
 
 int padded_experts(int N) { return N <= 8 ? 8 : N <= 16 ? 16 : 32; }
@@ -87,7 +96,8 @@ size_t carve_ws(void* base, int64_t T, int NP, GroupWs* w) {
     off += (bytes + 255) / 256 * 256;
     return o;
   };
-  const size_t clear = 8 * (size_t)hcap + 4 * kCtlWords;
+  const size_t n_flags = (size_t)((T + 15) / 16);
+  const size_t clear = 8 * (size_t)hcap + 4 * kCtlWords + 4 * n_flags;
   const size_t o_clear = take(clear);
   const size_t o_off = take(4 * (size_t)hcap);
   const size_t o_tslot = take(4 * (size_t)T);
@@ -104,6 +114,7 @@ size_t carve_ws(void* base, int64_t T, int NP, GroupWs* w) {
     w->key = reinterpret_cast<int*>(b + o_clear);
     w->cnt = w->key + hcap;
     w->ctl = reinterpret_cast<unsigned*>(w->cnt + hcap);
+    w->tile_flag = w->ctl + kCtlWords;
     w->off = reinterpret_cast<int*>(b + o_off);
     w->tok_slot = reinterpret_cast<int*>(b + o_tslot);
     w->tok_rank = reinterpret_cast<int*>(b + o_trank);
@@ -586,206 +597,802 @@ __device__ __forceinline__ void nf3_levels4(uint32_t x, float (&f)[4]) {
   f[3] = f23.y;
 }
 
+// The ring of work items in shared memory: n_slots slots of slot_bytes, then
+// per slot a `full` barrier (three arrivals: the row block's copies, the
+// gates' copy, the token list -- each copy arrival with its byte count), an
+// `empty` barrier (one arrival per consumer warp), the item's token count and
+// token list; then the CTA's abort flag.
+struct Ring {
+  uint8_t* slots;
+  uint64_t* full;
+  uint64_t* empty;
+  int* slot_n;
+  int* slot_tok;  // [n_slots][kItemTokens]
+  int* abort;
+  int q0;         // the slot of the CTA's first work item
+};
+
+__host__ __device__ constexpr size_t ring_bytes(int n_slots, int slot_bytes) {
+  return (size_t)n_slots * slot_bytes + (size_t)n_slots * (16 + 4 + 4 * kItemTokens) + 16;
+}
+
+__device__ __forceinline__ Ring carve_ring(uint8_t* base, const GroupLayout& L) {
+  Ring r;
+  r.slots = base;
+  r.full = reinterpret_cast<uint64_t*>(base + (size_t)L.n_slots * L.slot_bytes);
+  r.empty = r.full + L.n_slots;
+  r.slot_n = reinterpret_cast<int*>(r.empty + L.n_slots);
+  r.slot_tok = r.slot_n + L.n_slots;
+  r.abort = r.slot_tok + L.n_slots * kItemTokens;
+  r.q0 = 0;
+  return r;
+}
+
+// Thread 0: barriers initialised, abort flag cleared.
+__device__ __forceinline__ void ring_init(const Ring& r, const GroupLayout& L) {
+  for (int q = 0; q < L.n_slots; ++q) {
+    mbar_init(&r.full[q], 3);
+    mbar_init(&r.empty[q], kGroupCons);
+  }
+  *r.abort = 0;
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+__device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Router-tile readiness in the fused kernel: flag[i] = `want` once the gates
+// of tokens [16 i, 16 i + 16) are stored.  want = epoch + 1, where epoch
+// numbers the fused launches on a grouping: every CTA takes an arrival index
+// from a 64-bit counter when it starts, and the CTAs of one launch take
+// consecutive indices (a launch's CTAs start after the previous launch has
+// completed), so index / gridDim is the same for all of them.  A grouping
+// build resets the counter (all ones = no arrivals) and the flags.
+struct TileFlags {
+  unsigned* flag;
+  unsigned long long* arrivals;
+  unsigned* abort_word;  // the grouping's abort word
+};
+
+// Shared-memory staging for the fused kernel's router phase.  Wr arrives by
+// one bulk copy in the ring's last slot W (wr_full) and is released back to
+// the ring once every consumer warp has its fragments in registers
+// (wr_free).  With staged hidden states, the CTA's router tiles (at most
+// kMaxStagedTiles) arrive in slots 0, 1, ... one bulk copy per token row
+// into a padded layout (h_full[j]) and are released after their MMAs
+// (h_empty[j]).  `epoch` completes when want_s holds the launch's flag value.
+constexpr int kMaxStagedTiles = 4;
+
+struct FusedSync {
+  uint64_t* wr_full;
+  uint64_t* wr_free;
+  uint64_t* epoch;
+  uint64_t* h_full;   // [kMaxStagedTiles]
+  uint64_t* h_empty;  // [kMaxStagedTiles]
+  const unsigned* want_s;
+  TileFlags tf;
+  int n_staged;       // router tiles of this CTA staged in slots 0 .. n_staged-1 (0: A from global)
+  int h_pitch;        // bytes between staged token rows (2 D + 32)
+};
+
+// Ring position of the CTA's k-th work item: the ring starts at slot q0 and
+// visits the slots in order; the k-th item is in lap k / n_slots.
+__device__ __forceinline__ uint32_t ring_slot(const Ring& r, const GroupLayout& L, int k) {
+  return (uint32_t)((r.q0 + k) % L.n_slots);
+}
+__device__ __forceinline__ uint32_t ring_parity(const GroupLayout& L, int k) {
+  return (uint32_t)((k / L.n_slots) & 1);
+}
+
+// Producer warp of the gather.  The CTA's work items are
+// items[blockIdx.x + m * gridDim.x], m = 0 .. my_n-1, largest first; step k
+// takes them alternately from the front and the back (large, small, large,
+// ...), so the copies of small items proceed while the consumers work through
+// large ones.  Item records are read 32 at a time (one per lane) and each
+// item's token list one item ahead.  With `fs` (fused kernel) the producer
+// first copies the router phase's inputs (Wr; with staged hidden states also
+// the CTA's router tiles), then requests the row blocks of the first items
+// (one per slot) as their slots come free, and requests an item's gates only
+// when the router tiles of all of its tokens have flagged them stored (flags
+// read one item ahead with the token list).
+template <int NP, bool kNf3>
+__device__ void ring_producer(const GArgs& p, const GroupWs& w, const GroupLayout& L, const Ring& r, int my_n,
+                              const FusedSync* fs) {
+  constexpr int C = kItemTokens;
+  const int lane = threadIdx.x & 31;
+  volatile int* abort = r.abort;
+  const uint32_t row_bytes = (uint32_t)p.N * (uint32_t)p.D * 2u;
+  const int NB = p.D >> 6;  // NF3 blocks per row
+  const uint32_t code_bytes = (uint32_t)p.N * (uint32_t)NB * 24u, scale_bytes = (uint32_t)p.N * (uint32_t)NB * 2u;
+  const uint32_t W = (uint32_t)L.n_slots - 1u;  // Wr's slot (fused kernel)
+  // fused kernel: the small items first (they depend on few router tiles)
+  const int from_back = fs != nullptr ? 0 : 1;
+  auto record = [&](int kk) {
+    const int m = ((kk & 1) == from_back) ? my_n - 1 - (kk >> 1) : (kk >> 1);
+    return kk < my_n ? w.items[blockIdx.x + (size_t)m * gridDim.x] : make_int4(0, 0, 0, 0);
+  };
+  // the row block's copies into slot q, on its full barrier (lane 0)
+  auto issue_rows = [&](uint32_t q, int row) {
+    uint8_t* slot = r.slots + (size_t)q * L.slot_bytes;
+    if (lane == 0) {
+      if (kNf3) {
+        mbar_expect_tx(&r.full[q], code_bytes + scale_bytes);
+        bulk_g2s(slot, p.codes + (int64_t)row * code_bytes, code_bytes, &r.full[q]);
+        bulk_g2s(slot + L.scales_off, p.scales + (int64_t)row * p.N * NB, scale_bytes, &r.full[q]);
+      } else {
+        mbar_expect_tx(&r.full[q], row_bytes);
+        bulk_g2s(slot, p.table + (int64_t)row * p.N * p.D, row_bytes, &r.full[q]);
+      }
+    }
+  };
+  auto bad_row = [&](int row) {  // staging buffer smaller than the batch's distinct ids
+    if (!p.by_uid || (int64_t)row < p.rows) return false;
+    if (lane == 0) atomicOr(p.err, kErrIndex);
+    *abort = 1;
+    return true;
+  };
+  // items 0 .. issued-1 went out in full
+  int issued = 0;
+  // abandon the layer with items k .. last-1 holding row copies but no
+  // gates or token list: the flag first (consumers check it when a slot's
+  // phase completes), then their missing arrivals, so their phases complete
+  // when the copies land and the drain below waits for them
+  auto abandon = [&](int k, int last) {
+    *abort = 1;
+    __syncwarp();
+    if (lane == 0)
+      for (int kk = k; kk < last; ++kk) {
+        mbar_arrive(&r.full[ring_slot(r, L, kk)]);
+        mbar_arrive(&r.full[ring_slot(r, L, kk)]);
+      }
+    issued = last;
+  };
+  // records of steps k0 + lane (my_item) and k0 + 32 + lane (nx_item)
+  int k0 = 0;
+  int4 my_item = record(lane);
+  int4 nx_item = record(32 + lane);
+  bool ok = true;
+  int pre = 0;  // items whose row blocks went out ahead of the main loop
+  unsigned want = 0;
+  if (fs != nullptr) {
+    // the router phase's inputs: Wr into slot W, staged router tiles into
+    // slots 0 .. n_staged-1 (token row rr by lane rr)
+    if (lane == 0) {
+      const uint32_t wr_bytes = (uint32_t)p.N * (uint32_t)p.D * 2u;
+      mbar_expect_tx(fs->wr_full, wr_bytes);
+      bulk_g2s(r.slots + (size_t)W * L.slot_bytes, p.Wr, wr_bytes, fs->wr_full);
+    }
+    for (int j = 0; j < fs->n_staged; ++j) {
+      const int64_t t0 = ((int64_t)blockIdx.x + (int64_t)j * gridDim.x) * kTileMax;
+      const int rows = (int)(p.T - t0 < kTileMax ? p.T - t0 : kTileMax);
+      if (lane == 0) mbar_expect_tx(&fs->h_full[j], (uint32_t)rows * (uint32_t)p.D * 2u);
+      __syncwarp();
+      if (lane < rows)
+        bulk_g2s(r.slots + (size_t)j * L.slot_bytes + (size_t)lane * fs->h_pitch, p.h + (t0 + lane) * p.D,
+                 (uint32_t)p.D * 2u, &fs->h_full[j]);
+    }
+    // the row blocks of the first items, as their slots come free: W once
+    // the Wr fragments are in registers, a staged tile's slot once its MMAs
+    // are done, any other slot once Wr has landed (the router's inputs go
+    // first)
+    const int first = my_n < L.n_slots ? my_n : L.n_slots;  // n_slots <= 16 < 32: all in my_item
+    for (int k = 0; ok && k < first; ++k) {
+      const int row = __shfl_sync(0xffffffffu, p.by_uid ? my_item.w : my_item.x, k);
+      if (bad_row(row)) {
+        ok = false;
+        break;
+      }
+      const uint32_t q = ring_slot(r, L, k);
+      if (q == W)
+        ok = warp_wait(fs->wr_free, 0u, abort, p.err);
+      else if ((int)q < fs->n_staged)
+        ok = warp_wait(&fs->h_empty[q], 0u, abort, p.err);
+      else
+        ok = warp_wait(fs->wr_full, 0u, abort, p.err);
+      if (!ok) break;
+      issue_rows(q, row);
+      pre = k + 1;
+    }
+    if (ok && my_n > 0) {
+      ok = warp_wait(fs->epoch, 0u, abort, p.err);
+      want = *fs->want_s;
+    }
+    if (!ok) abandon(0, pre);
+  }
+  // whether the router tile of this lane's token has stored its gates
+  auto tile_ready = [&](int tok) {
+    return tok < 0 || fs == nullptr || ld_acquire(&fs->tf.flag[tok / kTileMax]) == want;
+  };
+  int next_tok = -1;
+  bool next_ready = true;
+  if (my_n > 0 && ok) {
+    const int pos = __shfl_sync(0xffffffffu, my_item.y, 0), n = __shfl_sync(0xffffffffu, my_item.z, 0);
+    next_tok = lane < n ? w.list[pos + lane] : -1;
+    next_ready = tile_ready(next_tok);
+  }
+  for (int k = 0; ok && k < my_n; ++k) {
+    const int row = __shfl_sync(0xffffffffu, p.by_uid ? my_item.w : my_item.x, k - k0);
+    const int pos = __shfl_sync(0xffffffffu, my_item.y, k - k0);
+    const int n = __shfl_sync(0xffffffffu, my_item.z, k - k0);
+    const int tok = next_tok;
+    bool ready = next_ready;
+    if (k + 1 < my_n) {  // prefetch the next item's record batch, tokens and their flags
+      if (k + 1 - k0 == 32) {
+        k0 = k + 1;
+        my_item = nx_item;
+        nx_item = record(k0 + 32 + lane);
+      }
+      const int pos1 = __shfl_sync(0xffffffffu, my_item.y, k + 1 - k0);
+      const int n1 = __shfl_sync(0xffffffffu, my_item.z, k + 1 - k0);
+      next_tok = lane < n1 ? w.list[pos1 + lane] : -1;
+      next_ready = tile_ready(next_tok);
+    }
+    const uint32_t q = ring_slot(r, L, k);
+    if (k >= pre) {
+      if (bad_row(row)) break;
+      ok = warp_wait(&r.empty[q], ring_parity(L, k) ^ 1u, abort, p.err);
+      if (!ok) break;
+      issue_rows(q, row);
+    }
+    if (fs != nullptr) {
+      // the item's gates exist once every token's router tile has flagged
+      // (bounded wait; a CTA that gives up abandons the layer)
+      if (!__all_sync(0xffffffffu, ready)) {
+        const uint64_t t0 = globaltimer();
+        int fail = 0;
+        while (!__all_sync(0xffffffffu, ready = tile_ready(tok))) {
+          if (lane == 0) {
+            if (*abort || ld_acquire(fs->tf.abort_word) != 0xFFFFFFFFu) {
+              fail = 1;
+            } else if (globaltimer() - t0 > kWaitLimitNs) {
+              atomicExch(fs->tf.abort_word, 1u);
+              atomicOr(p.err, kErrTimeout);
+              fail = 1;
+            }
+          }
+          if (__shfl_sync(0xffffffffu, fail, 0)) break;
+        }
+        if (__shfl_sync(0xffffffffu, fail, 0)) {
+          // this item's rows and those prefetched for the items after it are out
+          abandon(k, k + 1 > pre ? k + 1 : pre);
+          ok = false;
+          break;
+        }
+      }
+      __syncwarp();
+      if (lane == 0) fence_proxy_async_global();  // gates stored by other CTAs, read by a bulk copy
+    }
+    uint8_t* slot = r.slots + (size_t)q * L.slot_bytes;
+    if (lane == 0) {
+      const uint32_t gate_bytes = (uint32_t)n * NP * 4u;
+      mbar_expect_tx(&r.full[q], gate_bytes);
+      bulk_g2s(slot + L.gates_off, w.gates + (int64_t)pos * NP, gate_bytes, &r.full[q]);
+    }
+    // the token list (loaded one item ahead) after the copies
+    if (lane < n) r.slot_tok[q * C + lane] = tok;
+    if (lane == 0) r.slot_n[q] = n;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&r.full[q]);
+    issued = k + 1;
+  }
+  if (lane == 0) {  // the last copies must have landed before the CTA exits
+    if (fs != nullptr) {
+      mbar_drain(fs->wr_full, 0u);
+      for (int j = 0; j < fs->n_staged; ++j) mbar_drain(&fs->h_full[j], 0u);
+    }
+    for (int kk = issued - 1; kk >= 0 && kk >= issued - L.n_slots; --kk)
+      mbar_drain(&r.full[ring_slot(r, L, kk)], ring_parity(L, kk));
+  }
+  __syncwarp();
+}
+
+// Consumer warps of the gather.  unit = 4 consecutive elements of D; with
+// fewer units than consumer threads, Gt thread groups split the item's tokens.
 template <int NT, bool kExactN, bool kNf3>
-__global__ void __launch_bounds__(kGroupThreads, 1) grouped_gather_kernel(const GArgs p, const GroupWs w,
-                                                                          const GroupLayout L) {
+__device__ void ring_consumers(const GArgs& p, const GroupLayout& L, const Ring& r, int my_n) {
   constexpr int NP = 8 * NT;
   constexpr int C = kItemTokens;
   constexpr bool kPacked = !kNf3 && NP > 16;  // 32 experts: keep rows as bf16 pairs, convert per token
   static_assert(!kNf3 || NP <= 16, "the NF3 consumer holds 16 rows");
-  extern __shared__ __align__(128) uint8_t smem_raw[];
-  uint8_t* ring = smem_raw;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem_raw + (size_t)L.n_slots * L.slot_bytes);
-  uint64_t* empty = full + L.n_slots;
-  int* slot_n = reinterpret_cast<int*>(empty + L.n_slots);
-  int* slot_tok = slot_n + L.n_slots;  // [n_slots][C]
-  int* abort_flag = slot_tok + L.n_slots * C;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) {
-    for (int q = 0; q < L.n_slots; ++q) {
-      mbar_init(&full[q], 2);  // the copies' arrive.expect_tx + the token list's arrive
-      mbar_init(&empty[q], kGroupCons);
+  const int lane = threadIdx.x & 31;
+  volatile int* abort = r.abort;
+  const int NB = p.D >> 6;
+  const int lt = threadIdx.x;
+  const int units = p.D >> 2;
+  constexpr int kCT = kGroupCons * 32;
+  const int Gt = units >= kCT ? 1 : kCT / units;
+  const int grp = units >= kCT ? 0 : lt / units;
+  const int v0 = units >= kCT ? lt : lt - grp * units;
+  const int vstep = units >= kCT ? kCT : units;
+  const bool active = grp < Gt;
+  for (int k = 0; k < my_n; ++k) {
+    const uint32_t q = ring_slot(r, L, k);
+    if (!warp_wait(&r.full[q], ring_parity(L, k), abort, p.err)) break;
+    if (*abort) break;  // a phase completed without its item (the producer gave up)
+    if (active) {
+      const int n = r.slot_n[q];
+      const uint8_t* slot = r.slots + (size_t)q * L.slot_bytes;
+      const float* gs = reinterpret_cast<const float*>(slot + L.gates_off);
+      for (int v = v0; v < units; v += vstep) {
+        float xf[kPacked ? 1 : NP][4];
+        uint2 xp[kPacked ? NP : 1];
+        float sc[NP];
+        if constexpr (kNf3) {
+          // 4 codes at bits [12u, 12u + 12) of the row's block v / 16
+          const int b = v >> 4, bit = 12 * (v & 15), wi = bit >> 5, sh = bit & 31;
+          const uint16_t* ss = reinterpret_cast<const uint16_t*>(slot + L.scales_off);
+#pragma unroll
+          for (int j = 0; j < NP; ++j) {
+            float f[4] = {0.f, 0.f, 0.f, 0.f};
+            sc[j] = 0.f;
+            if (kExactN || j < p.N) {
+              const uint32_t* cw = reinterpret_cast<const uint32_t*>(slot + (size_t)(j * NB + b) * 24);
+              const uint32_t x = __funnelshift_r(cw[wi], wi < 5 ? cw[wi + 1] : 0u, sh) & 0xfffu;
+              nf3_levels4(x, f);
+              sc[j] = held(__half2float(__ushort_as_half(ss[j * NB + b])));
+            }
+            xf[j][0] = held(f[0]);
+            xf[j][1] = held(f[1]);
+            xf[j][2] = held(f[2]);
+            xf[j][3] = held(f[3]);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < NP; ++j) {
+            uint2 rw = make_uint2(0u, 0u);
+            if (kExactN || j < p.N) rw = *reinterpret_cast<const uint2*>(slot + ((size_t)j * p.D + 4 * v) * 2);
+            if (kPacked) {
+              xp[kPacked ? j : 0] = rw;
+            } else {
+              xf[kPacked ? 0 : j][0] = bf16_lo_held(rw.x);
+              xf[kPacked ? 0 : j][1] = bf16_hi_held(rw.x);
+              xf[kPacked ? 0 : j][2] = bf16_lo_held(rw.y);
+              xf[kPacked ? 0 : j][3] = bf16_hi_held(rw.y);
+            }
+          }
+        }
+        int i = grp;
+        if constexpr (!kPacked) {
+          // four tokens at a time (16 independent FMA chains)
+          for (; i + 3 * Gt < n; i += 4 * Gt) {
+            float o[4][4];
+            if constexpr (kNf3)
+              combine_quad_nf3<NP, kExactN>(xf, sc, gs + i * NP, Gt * NP, p.N, o);
+            else
+              combine_quad<NP, kExactN>(xf, gs + i * NP, Gt * NP, p.N, o);
+#pragma unroll
+            for (int k2 = 0; k2 < 4; ++k2)
+              __stcs(reinterpret_cast<float4*>(p.out + (int64_t)r.slot_tok[q * C + i + k2 * Gt] * p.D + 4 * v),
+                     make_float4(o[k2][0], o[k2][1], o[k2][2], o[k2][3]));
+          }
+        }
+        for (; i < n; i += Gt) {
+          float4 o0;
+          if constexpr (kNf3)
+            o0 = combine_unit_nf3<NP, kExactN>(xf, sc, gs + i * NP, p.N);
+          else
+            o0 = combine_unit<NP, kExactN, kPacked>(xf, xp, gs + i * NP, p.N);
+          __stcs(reinterpret_cast<float4*>(p.out + (int64_t)r.slot_tok[q * C + i] * p.D + 4 * v), o0);
+        }
+      }
     }
-    *abort_flag = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&r.empty[q]);
   }
+}
+
+__device__ __forceinline__ int items_of_cta(const GroupWs& w) {
+  const int n_items = (int)ld_relaxed_u32(&w.ctl[kCtlItems]);
+  return n_items > (int)blockIdx.x ? (n_items - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
+}
+
+template <int NT, bool kExactN, bool kNf3>
+__global__ void __launch_bounds__(kGroupThreads, 1) grouped_gather_kernel(const GArgs p, const GroupWs w,
+                                                                          const GroupLayout L) {
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  const Ring r = carve_ring(smem_raw, L);
+  if (threadIdx.x == 0) ring_init(r, L);
   __syncthreads();
   pdl_trigger();
   pdl_wait();  // the router's gates (and, before it, the grouping) are complete
   if (ld_relaxed_u32(&w.ctl[kCtlAbort]) != 0xFFFFFFFFu) return;  // plan abandoned (error word set)
-  volatile int* abort = abort_flag;
-  const int n_items = (int)ld_relaxed_u32(&w.ctl[kCtlItems]);
-  const int my_n = n_items > (int)blockIdx.x ? (n_items - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
-  const uint32_t row_bytes = (uint32_t)p.N * (uint32_t)p.D * 2u;
-  const int NB = p.D >> 6;  // NF3 blocks per row
-  const uint32_t code_bytes = (uint32_t)p.N * (uint32_t)NB * 24u, scale_bytes = (uint32_t)p.N * (uint32_t)NB * 2u;
+  const int my_n = items_of_cta(w);
+  if ((threadIdx.x >> 5) == kGroupProducer)
+    ring_producer<8 * NT, kNf3>(p, w, L, r, my_n, nullptr);
+  else
+    ring_consumers<NT, kExactN, kNf3>(p, L, r, my_n);
+  __syncthreads();
+}
 
-  if (warp == kGroupProducer) {
-    // ---------------- producer ----------------
-    // item records 32 at a time (one per lane); each item's tokens are
-    // loaded one item ahead
-    // The CTA's items are items[blockIdx.x + m * gridDim.x], m = 0 .. my_n-1,
-    // largest first.  Step k takes them alternately from the front and the
-    // back (large, small, large, ...), so the copies of small items proceed
-    // while the consumers work through large ones.
-    auto record = [&](int kk) {
-      const int m = (kk & 1) ? my_n - 1 - (kk >> 1) : (kk >> 1);
-      return kk < my_n ? w.items[blockIdx.x + (size_t)m * gridDim.x] : make_int4(0, 0, 0, 0);
-    };
-    // records of steps k0 + lane (my_item) and k0 + 32 + lane (nx_item)
-    int k0 = 0;
-    int4 my_item = record(lane);
-    int4 nx_item = record(32 + lane);
-    int next_tok = -1;
-    if (my_n > 0) {
-      const int pos = __shfl_sync(0xffffffffu, my_item.y, 0), n = __shfl_sync(0xffffffffu, my_item.z, 0);
-      next_tok = lane < n ? w.list[pos + lane] : -1;
-    }
-    uint32_t q = 0, ph = 0, issued = 0;
-    bool ok = true;
-    for (int k = 0; ok && k < my_n; ++k) {
-      const int id = __shfl_sync(0xffffffffu, p.by_uid ? my_item.w : my_item.x, k - k0);
-      const int pos = __shfl_sync(0xffffffffu, my_item.y, k - k0);
-      const int n = __shfl_sync(0xffffffffu, my_item.z, k - k0);
-      const int tok = next_tok;
-      if (k + 1 < my_n) {  // prefetch the next item's record batch and tokens
-        if (k + 1 - k0 == 32) {
-          k0 = k + 1;
-          my_item = nx_item;
-          nx_item = record(k0 + 32 + lane);
-        }
-        const int pos1 = __shfl_sync(0xffffffffu, my_item.y, k + 1 - k0);
-        const int n1 = __shfl_sync(0xffffffffu, my_item.z, k + 1 - k0);
-        next_tok = lane < n1 ? w.list[pos1 + lane] : -1;
-      }
-      if (p.by_uid && (int64_t)id >= p.rows) {  // staging buffer smaller than the batch's distinct ids
-        if (lane == 0) atomicOr(p.err, kErrIndex);
-        *abort = 1;
-        break;
-      }
-      ok = warp_wait(&empty[q], ph ^ 1u, abort, p.err);
-      if (!ok) break;
-      uint8_t* slot = ring + (size_t)q * L.slot_bytes;
-      // the copies first; the token list (loaded one item ahead) after them
-      if (lane == 0) {
-        const uint32_t gate_bytes = (uint32_t)n * NP * 4u;
-        if (kNf3) {
-          mbar_expect_tx(&full[q], code_bytes + scale_bytes + gate_bytes);
-          bulk_g2s(slot, p.codes + (int64_t)id * code_bytes, code_bytes, &full[q]);
-          bulk_g2s(slot + L.scales_off, p.scales + (int64_t)id * p.N * NB, scale_bytes, &full[q]);
-        } else {
-          mbar_expect_tx(&full[q], row_bytes + gate_bytes);
-          bulk_g2s(slot, p.table + (int64_t)id * p.N * p.D, row_bytes, &full[q]);
-        }
-        bulk_g2s(slot + L.gates_off, w.gates + (int64_t)pos * NP, gate_bytes, &full[q]);
-      }
-      if (lane < n) slot_tok[q * C + lane] = tok;
-      if (lane == 0) slot_n[q] = n;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&full[q]);
-      ++issued;
-      if (++q == (uint32_t)L.n_slots) {
-        q = 0;
-        ph ^= 1u;
-      }
-    }
-    if (lane == 0) {  // the last copies must have landed before the CTA exits
-      for (uint32_t i = 0; i < issued && i < (uint32_t)L.n_slots; ++i) {
-        q = q == 0 ? L.n_slots - 1 : q - 1;
-        if (q == (uint32_t)L.n_slots - 1) ph ^= 1u;
-        mbar_drain(&full[q], ph);
-      }
-    }
-    __syncwarp();
+// ---- fused layer kernel: router phase and gather in one launch ----
+//
+// One CTA per SM.  The 8 consumer warps first compute the gates of 16-token
+// tiles (blockIdx.x, blockIdx.x + gridDim.x, ...) with mma.sync -- the same
+// k-step split, k-slot order, partial-sum order and softmax as the router
+// kernels, so the gates are bit-identical to theirs -- store them at the
+// tokens' list positions and flag each tile done.  Wr is brought into the
+// ring's last slot by one bulk copy, its fragments go to registers
+// (ldmatrix.trans) for the whole phase, and the slot returns to the ring.
+// Meanwhile the producer warp requests the row blocks of the CTA's first
+// items; it requests an item's gates once the tiles of all of the item's
+// tokens are flagged, so the gather starts while other CTAs are still
+// routing.  Then the consumers combine as in grouped_gather_kernel.  The
+// flag waits need every CTA resident: one CTA per SM, started when the
+// previous kernel lets it (all of that kernel's CTAs are running by then),
+// and each wait is bounded.  Batches large enough for the tensor-core router
+// kernel take that kernel and grouped_gather_kernel instead.
+
+constexpr int kFusedKB = 16;  // k-steps per warp (D <= 2048)
+
+// Barrier over the 8 consumer warps only (the producer warp runs apart).
+struct ConsumerSync {
+  __device__ __forceinline__ void operator()() const {
+    asm volatile("bar.sync 1, %0;" ::"n"(kGroupCons * 32) : "memory");
+  }
+};
+
+// B fragments of k-step ks for both 8-expert halves from Wr as copied
+// ([D][N] bf16, N = 8 NT): one ldmatrix.trans of 2 NT 8x8 blocks, each
+// lane giving the address of one row, in the router kernels' k-slot order
+// (slots 2c, 2c+1 <- d = 4c, 4c+1; slots 2c+8, 2c+9 <- d = 4c+2, 4c+3).
+template <int NT>
+__device__ __forceinline__ void wr_fragments(uint2 (&b)[NT], const uint16_t* wr_s, int ks) {
+  const int lane = threadIdx.x & 31;
+  const int m = lane >> 3, rr = lane & 7;  // matrix m = (slot half m & 1, expert half m >> 1); its row rr
+  const int slot = rr + 8 * (m & 1);
+  const int dl = slot < 8 ? 4 * (slot >> 1) + (slot & 1) : 4 * ((slot - 8) >> 1) + 2 + (slot & 1);
+  const uint32_t addr = smem_u32(wr_s + (ks * 16 + dl) * (8 * NT) + 8 * ((m >> 1) & (NT - 1)));
+  if constexpr (NT == 2) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(b[0].x), "=r"(b[0].y), "=r"(b[1].x), "=r"(b[1].y)
+                 : "r"(addr));
   } else {
-    // ---------------- consumers ----------------
-    // unit = 4 consecutive elements of D; with fewer units than consumer
-    // threads, Gt thread groups split the item's tokens
-    const int lt = threadIdx.x;
-    const int units = p.D >> 2;
-    constexpr int kCT = kGroupCons * 32;
-    const int Gt = units >= kCT ? 1 : kCT / units;
-    const int grp = units >= kCT ? 0 : lt / units;
-    const int v0 = units >= kCT ? lt : lt - grp * units;
-    const int vstep = units >= kCT ? kCT : units;
-    const bool active = grp < Gt;
-    uint32_t q = 0, ph = 0;
-    for (int k = 0; k < my_n; ++k) {
-      if (!warp_wait(&full[q], ph, abort, p.err)) break;
-      if (active) {
-        const int n = slot_n[q];
-        const uint8_t* slot = ring + (size_t)q * L.slot_bytes;
-        const float* gs = reinterpret_cast<const float*>(slot + L.gates_off);
-        for (int v = v0; v < units; v += vstep) {
-          float xf[kPacked ? 1 : NP][4];
-          uint2 xp[kPacked ? NP : 1];
-          float sc[NP];
-          if constexpr (kNf3) {
-            // 4 codes at bits [12u, 12u + 12) of the row's block v / 16
-            const int b = v >> 4, bit = 12 * (v & 15), wi = bit >> 5, sh = bit & 31;
-            const uint16_t* ss = reinterpret_cast<const uint16_t*>(slot + L.scales_off);
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
+                 : "=r"(b[0].x), "=r"(b[0].y)
+                 : "r"(addr));
+  }
+}
+
+// B fragments of k-step ks (both 8-expert halves) from Wr as copied, for
+// any N <= NP: element loads, zero past N.
+template <int NT>
+__device__ __forceinline__ void wr_fragments_any(uint2 (&b)[NT], const uint16_t* wr_s, int ks, int N) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
 #pragma unroll
-            for (int j = 0; j < NP; ++j) {
-              float f[4] = {0.f, 0.f, 0.f, 0.f};
-              sc[j] = 0.f;
-              if (kExactN || j < p.N) {
-                const uint32_t* cw = reinterpret_cast<const uint32_t*>(slot + (size_t)(j * NB + b) * 24);
-                const uint32_t x = __funnelshift_r(cw[wi], wi < 5 ? cw[wi + 1] : 0u, sh) & 0xfffu;
-                nf3_levels4(x, f);
-                sc[j] = held(__half2float(__ushort_as_half(ss[j * NB + b])));
-              }
-              xf[j][0] = held(f[0]);
-              xf[j][1] = held(f[1]);
-              xf[j][2] = held(f[2]);
-              xf[j][3] = held(f[3]);
-            }
-          } else {
+  for (int nt = 0; nt < NT; ++nt) {
+    const int j = nt * 8 + g;
+    uint32_t e[4] = {0u, 0u, 0u, 0u};
+    if (j < N) {
+      const uint16_t* src = wr_s + (ks * 16 + 4 * c) * N + j;
 #pragma unroll
-          for (int j = 0; j < NP; ++j) {
-            uint2 r = make_uint2(0u, 0u);
-            if (kExactN || j < p.N) r = *reinterpret_cast<const uint2*>(slot + ((size_t)j * p.D + 4 * v) * 2);
-            if (kPacked) {
-              xp[kPacked ? j : 0] = r;
-            } else {
-              xf[kPacked ? 0 : j][0] = bf16_lo_held(r.x);
-              xf[kPacked ? 0 : j][1] = bf16_hi_held(r.x);
-              xf[kPacked ? 0 : j][2] = bf16_lo_held(r.y);
-              xf[kPacked ? 0 : j][3] = bf16_hi_held(r.y);
-            }
-          }
-          }
-          int i = grp;
-          if constexpr (!kPacked) {
-            // four tokens at a time (16 independent FMA chains)
-            for (; i + 3 * Gt < n; i += 4 * Gt) {
-              float o[4][4];
-              if constexpr (kNf3)
-                combine_quad_nf3<NP, kExactN>(xf, sc, gs + i * NP, Gt * NP, p.N, o);
-              else
-                combine_quad<NP, kExactN>(xf, gs + i * NP, Gt * NP, p.N, o);
+      for (int u = 0; u < 4; ++u) e[u] = src[u * N];
+    }
+    b[nt] = make_uint2(e[0] | (e[1] << 16), e[2] | (e[3] << 16));
+  }
+}
+
+// Softmax of one tile, its gates to the tokens' list positions (NaN output
+// rows for bad ids), then its flag.
+template <int NT>
+__device__ __forceinline__ void fused_tile_finish(const GArgs& p, const GroupWs& w, const Smem& s,
+                                                  const float (&acc)[NT][4], int64_t tile, int rows, unsigned* flag,
+                                                  unsigned want, int my_pos) {
+  constexpr int NP = 8 * NT;
+  const int64_t t0 = tile * kTileMax;
+  router_store_partials<NT>(s, acc);
+  // s.tok_id[r] = the list position of token t0 + r (thread r's my_pos)
+  router_softmax<true, NT, ConsumerSync, true>(s, rows, p.N, nullptr, t0, my_pos);
+  for (int i = threadIdx.x; i < rows * NP; i += kGroupCons * 32) {
+    const int r = i / NP, j = i - r * NP;
+    const int pos = s.tok_id[r];
+    if (pos >= 0) w.gates[(int64_t)pos * NP + j] = s.gates[i];
+  }
+  if ((int)threadIdx.x < rows && my_pos < 0) {  // a bad id: its thread writes the NaN output row
+    atomicOr(p.err, kErrIndex);
+    float* o = p.out + (t0 + threadIdx.x) * p.D;
+    for (int d = 0; d < p.D; d += 4) __stcs(reinterpret_cast<float4*>(o + d), make_float4(NAN, NAN, NAN, NAN));
+  }
+  // the flag is a release by thread 0 after the barrier: every consumer's
+  // gate stores precede it (the reader acquires the flag, then fences the
+  // async proxy before its bulk copy); s.gates and s.tok_id are rewritten
+  // only after the next tile's first barrier
+  ConsumerSync{}();
+  if (threadIdx.x == 0) st_release(&flag[tile], want);
+}
+
+// A fragments of a staged router tile (token rows at h_pitch bytes in
+// shared memory), in the same k-slot order as router_load_a: lane (g, c)
+// takes 8 bytes at d = 16 ks + 4c of rows g and g + 8 (zero past `rows`).
+// With h_pitch = 2 D + 32 the 32 lanes of one load hit every bank pair once.
+template <int KB>
+__device__ __forceinline__ void router_load_a_smem(RouterA<KB>& A, const uint8_t* tile_s, int h_pitch, int rows,
+                                                   int D) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+  const bool ok0 = g < rows, ok1 = g + 8 < rows;
+  const uint8_t* r0 = tile_s + (size_t)g * h_pitch + 8 * c;
+  const uint8_t* r1 = tile_s + (size_t)(g + 8) * h_pitch + 8 * c;
+  const int ksteps = D >> 4;
 #pragma unroll
-              for (int k = 0; k < 4; ++k)
-                __stcs(reinterpret_cast<float4*>(p.out + (int64_t)slot_tok[q * C + i + k * Gt] * p.D + 4 * v),
-                       make_float4(o[k][0], o[k][1], o[k][2], o[k][3]));
-            }
-          }
-          for (; i < n; i += Gt) {
-            float4 o0;
-            if constexpr (kNf3)
-              o0 = combine_unit_nf3<NP, kExactN>(xf, sc, gs + i * NP, p.N);
-            else
-              o0 = combine_unit<NP, kExactN, kPacked>(xf, xp, gs + i * NP, p.N);
-            __stcs(reinterpret_cast<float4*>(p.out + (int64_t)slot_tok[q * C + i] * p.D + 4 * v), o0);
+  for (int i = 0; i < KB; ++i) {
+    const int ks = warp + i * kWarps;
+    const bool in = ks < ksteps;
+    A.a0[i] = (in && ok0) ? *reinterpret_cast<const uint2*>(r0 + ks * 32) : make_uint2(0u, 0u);
+    A.a1[i] = (in && ok1) ? *reinterpret_cast<const uint2*>(r1 + ks * 32) : make_uint2(0u, 0u);
+  }
+}
+
+// Waits of the consumer warps on a barrier of the router phase, with one
+// verdict for all of them (the tile loop holds barriers, so every warp must
+// take the same path): a warp whose wait failed says so before the barrier
+// and all read the verdict after it.
+__device__ __forceinline__ bool consumers_wait(uint64_t* b, uint32_t parity, volatile int* abort, unsigned* err,
+                                               volatile int* fail) {
+  if (!warp_wait(b, parity, abort, err) && (threadIdx.x & 31) == 0) *fail = 1;
+  ConsumerSync{}();
+  return *fail == 0;
+}
+
+// Router scratch of the staged path: two tiles finished together.
+constexpr int kPairRows = 2 * kTileMax;
+
+template <int NP>
+__host__ __device__ constexpr size_t pair_scratch_bytes() {
+  return (size_t)kWarps * kPairRows * NP * 4 + (size_t)kPairRows * NP * 4 + (size_t)kPairRows * 4;
+}
+
+struct PairScratch {
+  float* part;   // [kWarps][kPairRows][NP] partial logits
+  float* gates;  // [kPairRows][NP]
+  int* tok;      // [kPairRows] list positions
+};
+
+// This warp's partial logits of one tile -> rows row0 .. row0+15.
+template <int NT>
+__device__ __forceinline__ void pair_store_partials(const PairScratch& ps, const float (&acc)[NT][4], int row0) {
+  constexpr int NP = 8 * NT;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+  float* pw = ps.part + warp * kPairRows * NP;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    pw[(row0 + g) * NP + nt * 8 + 2 * c] = acc[nt][0];
+    pw[(row0 + g) * NP + nt * 8 + 2 * c + 1] = acc[nt][1];
+    pw[(row0 + g + 8) * NP + nt * 8 + 2 * c] = acc[nt][2];
+    pw[(row0 + g + 8) * NP + nt * 8 + 2 * c + 1] = acc[nt][3];
+  }
+}
+
+// Sum of the partial logits (warps in order), max-subtracted softmax over
+// the N experts: the arithmetic of router_softmax, row for row.
+template <int NT>
+__device__ __forceinline__ void pair_softmax(const PairScratch& ps, int rows, int N) {
+  constexpr int NP = 8 * NT;
+  constexpr int RPW = 32 / NP;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sub = lane / NP, jl = lane % NP;
+  for (int rb = warp * RPW; rb < rows; rb += kWarps * RPW) {
+    const int r = rb + sub;
+    const bool act = r < rows;
+    float z = 0.f;
+    if (act) {
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) z += ps.part[(w * kPairRows + r) * NP + jl];
+    }
+    const bool valid = act && jl < N;
+    float m = valid ? z : -INFINITY;
+#pragma unroll
+    for (int off = NP / 2; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    const float e = valid ? expf(z - m) : 0.f;
+    float sum = e;
+#pragma unroll
+    for (int off = NP / 2; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    if (act) ps.gates[r * NP + jl] = valid ? e / sum : 0.f;
+  }
+}
+
+// The gates of `rows` tokens (rows 0..15: tile ta; 16..: tile tb) to their
+// list positions (NaN output rows for bad ids), then the tiles' flags.
+// Thread r holds the list position of row r in my_pos.
+template <int NT>
+__device__ __forceinline__ void pair_finish(const GArgs& p, const GroupWs& w, const PairScratch& ps, int rows,
+                                            int64_t ta, int64_t tb, int my_pos, unsigned* flag, unsigned want) {
+  constexpr int NP = 8 * NT;
+  if (threadIdx.x < rows) ps.tok[threadIdx.x] = my_pos;  // (last read before the previous pair's final barrier)
+  ConsumerSync{}();
+  pair_softmax<NT>(ps, rows, p.N);
+  ConsumerSync{}();
+  for (int i = threadIdx.x; i < rows * NP; i += kGroupCons * 32) {
+    const int r = i / NP, j = i - r * NP;
+    const int pos = ps.tok[r];
+    if (pos >= 0) w.gates[(int64_t)pos * NP + j] = ps.gates[i];
+  }
+  if ((int)threadIdx.x < rows && my_pos < 0) {  // a bad id: its thread writes the NaN output row
+    atomicOr(p.err, kErrIndex);
+    const int r = threadIdx.x;
+    const int64_t t = (r < kTileMax ? ta * kTileMax + r : tb * kTileMax + r - kTileMax);
+    float* o = p.out + t * p.D;
+    for (int d = 0; d < p.D; d += 4) __stcs(reinterpret_cast<float4*>(o + d), make_float4(NAN, NAN, NAN, NAN));
+  }
+  // the flags are releases by thread 0 after the barrier: every consumer's
+  // gate stores precede them
+  ConsumerSync{}();
+  if (threadIdx.x == 0) {
+    st_release(&flag[ta], want);
+    if (rows > kTileMax) st_release(&flag[tb], want);
+  }
+}
+
+// Router phase of the fused kernel (consumer warps).  Wr's fragments for
+// this warp's k-steps go to registers once (the Wr slot then returns to the
+// ring).  A fragments: with staged tiles (kStaged) from shared memory, each
+// tile's slot released after its MMAs; otherwise from global memory, a
+// tile's requested right after the previous tile's MMAs.  The tokens' list
+// positions are loaded a tile ahead.  A failed wait abandons the layer (the
+// remaining tiles are not flagged; the other CTAs' waits give up on the
+// abort word, and the error word is set).
+template <int NT, bool kExactN, bool kStaged>
+__device__ void fused_router_phase(const GArgs& p, const GroupWs& w, const Smem& s, const PairScratch& ps,
+                                   const Ring& r, const GroupLayout& L, const FusedSync& fs, unsigned want,
+                                   volatile int* fail) {
+  constexpr int KB = kFusedKB;
+  const int warp = threadIdx.x >> 5;
+  const int ksteps = p.D >> 4;
+  const int64_t n_tiles = (p.T + kTileMax - 1) / kTileMax;
+  const int64_t G = gridDim.x;
+  volatile int* abort = r.abort;
+  const uint16_t* wr_s = reinterpret_cast<const uint16_t*>(r.slots + (size_t)(L.n_slots - 1) * L.slot_bytes);
+  auto rows_of = [&](int64_t tile) {
+    const int64_t t0 = tile * kTileMax;
+    return (int)(p.T - t0 < kTileMax ? p.T - t0 : kTileMax);
+  };
+  auto load_pos_row = [&](int64_t t, int rr) {  // the list position of token 16 t + rr
+    return (t < n_tiles && rr < rows_of(t)) ? __ldg(w.tok_pos + t * kTileMax + rr) : -1;
+  };
+  auto load_pos = [&](int64_t t) { return load_pos_row(t, (int)threadIdx.x); };
+  RouterA<KB> A;
+  int64_t tile = blockIdx.x;
+  // staged: thread r < 32 holds the list position of row r of the pair
+  // (tiles tile, tile + G); otherwise thread r < 16 that of row r of the tile
+  auto load_pair_pos = [&](int64_t t) {
+    return kStaged && threadIdx.x >= kTileMax ? load_pos_row(t + G, threadIdx.x - kTileMax) : load_pos(t);
+  };
+  int my_pos = load_pair_pos(tile);
+  if (!kStaged && tile < n_tiles) router_load_a<KB>(A, p.h, tile * kTileMax, rows_of(tile), p.D, warp);
+  // B fragments of k-steps warp + 8i: {Wr[d][j] | Wr[d+1][j] << 16, Wr[d+2][j] | Wr[d+3][j] << 16},
+  // d = 16 ks + 4c, j = 8 nt + g (the router kernels' k-slot order)
+  bool ok = consumers_wait(fs.wr_full, 0u, abort, p.err, fail);
+  uint2 bw[KB][NT];
+#pragma unroll
+  for (int i = 0; i < KB; ++i) {
+    const int ks = warp + i * kWarps;
+    if (ok && ks < ksteps) {
+      if (kExactN && p.N == 8 * NT)
+        wr_fragments<NT>(bw[i], wr_s, ks);
+      else
+        wr_fragments_any<NT>(bw[i], wr_s, ks, p.N);
+    } else {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) bw[i][nt] = make_uint2(0u, 0u);
+    }
+  }
+  ConsumerSync{}();
+  if (threadIdx.x == 0) mbar_arrive(fs.wr_free);  // the Wr slot goes back to the ring
+  if constexpr (kStaged) {
+    // the CTA's tiles two at a time: both tiles' MMAs, then one finish
+    for (int j = 0; ok && tile < n_tiles; tile += 2 * G, j += 2) {
+      const bool two = tile + G < n_tiles;
+      ok = consumers_wait(&fs.h_full[j], 0u, abort, p.err, fail);
+      if (ok && two) ok = consumers_wait(&fs.h_full[j + 1], 0u, abort, p.err, fail);
+      if (!ok) break;
+      float acc0[NT][4], acc1[NT][4];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        float (&acc)[NT][4] = u == 0 ? acc0 : acc1;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+        if (u == 1 && !two) continue;
+        router_load_a_smem<KB>(A, r.slots + (size_t)(j + u) * L.slot_bytes, fs.h_pitch, rows_of(tile + u * G), p.D);
+#pragma unroll
+        for (int i = 0; i < KB; ++i) {
+          if (warp + i * kWarps < ksteps) {
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+              mma_16816(acc[nt], A.a0[i].x, A.a1[i].x, A.a0[i].y, A.a1[i].y, bw[i][nt].x, bw[i][nt].y);
           }
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[q]);
-      if (++q == (uint32_t)L.n_slots) {
-        q = 0;
-        ph ^= 1u;
+      ConsumerSync{}();  // the tiles' slots go back to the ring
+      if (threadIdx.x == 0) {
+        mbar_arrive(&fs.h_empty[j]);
+        if (two) mbar_arrive(&fs.h_empty[j + 1]);
+      }
+      pair_store_partials<NT>(ps, acc0, 0);
+      if (two) pair_store_partials<NT>(ps, acc1, kTileMax);
+      const int rows = two ? kTileMax + rows_of(tile + G) : rows_of(tile);
+      const int pos = my_pos;
+      my_pos = load_pair_pos(tile + 2 * G);
+      pair_finish<NT>(p, w, ps, rows, tile, tile + G, pos, fs.tf.flag, want);
+    }
+  }
+  for (; !kStaged && ok && tile < n_tiles; tile += G) {
+    float acc[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll
+    for (int i = 0; i < KB; ++i) {
+      if (warp + i * kWarps < ksteps) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+          mma_16816(acc[nt], A.a0[i].x, A.a1[i].x, A.a0[i].y, A.a1[i].y, bw[i][nt].x, bw[i][nt].y);
       }
     }
+    const int pos = my_pos;
+    my_pos = load_pos(tile + G);
+    if (tile + G < n_tiles) router_load_a<KB>(A, p.h, (tile + G) * kTileMax, rows_of(tile + G), p.D, warp);
+    fused_tile_finish<NT>(p, w, s, acc, tile, rows_of(tile), fs.tf.flag, want, pos);
+  }
+  if (!ok && threadIdx.x == 0) {  // the producer stops too (it may wait for a staged tile's slot)
+    *abort = 1;
+    atomicExch(fs.tf.abort_word, 1u);
+  }
+}
+
+template <int NT, bool kExactN, bool kStaged>
+__global__ void __launch_bounds__(kGroupThreads, 1) grouped_fused_kernel(const GArgs p, const GroupWs w,
+                                                                         const GroupLayout L) {
+  constexpr int NP = 8 * NT;
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  Ring r = carve_ring(smem_raw, L);
+  r.q0 = L.n_slots - 1;  // the first item goes into Wr's slot
+  // router scratch after the ring: partial sums, gates and list positions of
+  // a tile (or, staged, of a pair of tiles)
+  uint8_t* scratch = smem_raw + (ring_bytes(L.n_slots, L.slot_bytes) + 127) / 128 * 128;
+  const Smem s = carve<false, NP>(scratch, p.D);
+  const PairScratch ps{reinterpret_cast<float*>(scratch),
+                       reinterpret_cast<float*>(scratch + (size_t)kWarps * kPairRows * NP * 4),
+                       reinterpret_cast<int*>(scratch + (size_t)(kWarps + 1) * kPairRows * NP * 4)};
+  __shared__ unsigned want_s;
+  __shared__ int skip_s, fail_s;
+  __shared__ __align__(8) uint64_t bars[3 + 2 * kMaxStagedTiles];
+  const int64_t n_tiles = (p.T + kTileMax - 1) / kTileMax;
+  const int my_tiles = n_tiles > blockIdx.x ? (int)((n_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x) : 0;
+  const FusedSync fs{&bars[0], &bars[1], &bars[2], &bars[3], &bars[3 + kMaxStagedTiles], &want_s,
+                     TileFlags{w.tile_flag, reinterpret_cast<unsigned long long*>(&w.ctl[kCtlLaunches]),
+                               &w.ctl[kCtlAbort]},
+                     kStaged ? my_tiles : 0, 2 * p.D + 32};
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 3; ++i) mbar_init(&bars[i], 1);
+    for (int j = 0; j < kMaxStagedTiles; ++j) {
+      mbar_init(&fs.h_full[j], 1);
+      mbar_init(&fs.h_empty[j], 1);
+    }
+    ring_init(r, L);  // (its fence covers all of them)
+  }
+  pdl_trigger();
+  pdl_wait();  // the grouping and every earlier kernel are complete
+  if (threadIdx.x == 0) {
+    skip_s = ld_relaxed_u32(fs.tf.abort_word) != 0xFFFFFFFFu;  // plan abandoned
+    fail_s = 0;
+  }
+  __syncthreads();
+  if (skip_s) return;
+  const int my_n = items_of_cta(w);
+  if ((threadIdx.x >> 5) == kGroupProducer) {
+    ring_producer<NP, false>(p, w, L, r, my_n, &fs);
+  } else {
+    unsigned want = 0;
+    if (threadIdx.x == 0) {  // this launch's flag value (see TileFlags)
+      const unsigned long long before = atomicAdd(fs.tf.arrivals, 1ull) + 1ull;
+      want = (unsigned)(before / gridDim.x) + 1u;
+      want_s = want;
+      mbar_arrive(fs.epoch);
+    }
+    fused_router_phase<NT, kExactN, kStaged>(p, w, s, ps, r, L, fs, want, &fail_s);
+    ring_consumers<NT, kExactN, false>(p, L, r, my_n);
   }
   __syncthreads();
 }
@@ -811,13 +1418,55 @@ GroupLayout group_layout(int N, int D, bool nf3) {
   return L;
 }
 
+
+// The fused layer kernel (bf16 table, N <= 16, D <= 2048: a warp's k-steps
+// fit the kFusedKB fragments held in registers).
+template <int NT, bool kExactN, bool kStaged>
+mole_status launch_fused_as(const GArgs& p, const GroupWs& w, const GroupLayout& L, size_t smem, int n_sm,
+                            cudaStream_t stream) {
+  auto kern = grouped_fused_kernel<NT, kExactN, kStaged>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return MOLE_ERR_CUDA;
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kGroupThreads, smem) != cudaSuccess || occ < 1)
+    return MOLE_ERR_UNSUPPORTED;
+  // one CTA per SM: all resident once the previous kernel's CTAs have left
+  return cuda_status(launch_pdl(kern, (unsigned)n_sm, kGroupThreads, smem, stream, p, w, L));
+}
+
+template <int NT, bool kExactN>
+mole_status launch_fused(const GArgs& p, const GroupWs& w, cudaStream_t stream) {
+  constexpr int NP = 8 * NT;
+  static_assert(NT <= 2, "Wr fragments of 32 experts do not fit the registers");
+  if (p.D > 16 * kWarps * kFusedKB || !aligned16(p.Wr)) return MOLE_ERR_UNSUPPORTED;
+  const GroupLayout L = group_layout<NT>(p.N, p.D, false);
+  if (L.n_slots < 2 || (int64_t)p.N * p.D * 2 > L.slot_bytes) return MOLE_ERR_UNSUPPORTED;
+  const size_t ring = (ring_bytes(L.n_slots, L.slot_bytes) + 127) / 128 * 128;
+  const size_t smem = ring + smem_bytes_for<false, NP>(p.D), smem_staged = ring + pair_scratch_bytes<NP>();
+  if (smem > 227 * 1024) return MOLE_ERR_UNSUPPORTED;
+  const int n_sm = num_sms();
+  if (n_sm <= 0) return MOLE_ERR_NO_DEVICE;
+  // staged router tiles: every CTA's tiles fit the slots other than Wr's
+  const int64_t per_cta = ((p.T + kTileMax - 1) / kTileMax + n_sm - 1) / n_sm;
+  const bool staged = per_cta <= std::min<int64_t>(kMaxStagedTiles, L.n_slots - 1) &&
+                      (int64_t)kTileMax * (2 * p.D + 32) <= L.slot_bytes && aligned16(p.h) &&
+                      smem_staged <= 227 * 1024;
+  return staged ? launch_fused_as<NT, kExactN, true>(p, w, L, smem_staged, n_sm, stream)
+                : launch_fused_as<NT, kExactN, false>(p, w, L, smem, n_sm, stream);
+}
+
 template <int NT, bool kExactN, bool kNf3>
 mole_status launch_layer(const GArgs& p, const GroupWs& w, cudaStream_t stream) {
   constexpr int NP = 8 * NT;
-  constexpr int C = kItemTokens;
+  if constexpr (!kNf3 && NT <= 2) {
+    if (!router_tc_supported(p.T, p.N, p.D, p.h, p.Wr)) {
+      const mole_status st = launch_fused<NT, kExactN>(p, w, stream);
+      if (st != MOLE_ERR_UNSUPPORTED) return st;
+    }
+  }
   const GroupLayout L = group_layout<NT>(p.N, p.D, kNf3);
   if (L.n_slots < 2) return MOLE_ERR_UNSUPPORTED;
-  const size_t gsmem = (size_t)L.n_slots * L.slot_bytes + (size_t)L.n_slots * (16 + 4 + 4 * C) + 16;
+  const size_t gsmem = ring_bytes(L.n_slots, L.slot_bytes);
   const size_t rsmem = smem_bytes_for<true, NP>(p.D);
   if (gsmem > 227 * 1024 || rsmem > 227 * 1024) return MOLE_ERR_UNSUPPORTED;
   auto rkern = router_group_kernel<NT>;
