@@ -903,7 +903,7 @@ def cpu_baseline(args):
     while True:
         oracle.combine(inv.astype(np.int32), h, Wr, rows)
         reps += 1
-        if time.perf_counter() - t0 > 10.0 or reps >= 50:
+        if time.perf_counter() - t0 > 10.0 or reps >= 5000:
             break
     dt = time.perf_counter() - t0
     per_layer = sample_T * reps / dt
