@@ -276,7 +276,7 @@ __device__ void plan_count(const GroupWs& w, int* cls, int* cbase) {
 
 // Step 2: list offsets and item records of this CTA's slot range.  Items are
 // laid out by size, largest first (all full items, then 15-token items, ...),
-// so dealing them round-robin to the gather CTAs spreads the tokens evenly.
+// so dealing them to the gather CTAs in alternating rounds spreads the tokens evenly.
 // `cur` is kAgg ints of shared memory, `red` 2 * kWarps.
 __device__ void plan_offsets(const GroupWs& w, const int* cbase, int* cur, int* red) {
   int64_t s0, s1;
@@ -689,8 +689,23 @@ __device__ __forceinline__ uint32_t ring_parity(const GroupLayout& L, int k) {
   return (uint32_t)((k / L.n_slots) & 1);
 }
 
+// The work items (largest first) are dealt to the CTAs in rounds of
+// gridDim.x, alternating direction (round m: CTA b takes the item at
+// position b of the round if m is even, gridDim.x - 1 - b if odd), so that no
+// CTA takes the largest item of every round.
+__device__ __forceinline__ int item_of_cta(int m) {
+  const int pos = (m & 1) ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x;
+  return m * (int)gridDim.x + pos;
+}
+
+__device__ __forceinline__ int items_of_cta(const GroupWs& w) {
+  const int n_items = (int)ld_relaxed_u32(&w.ctl[kCtlItems]);
+  const int full = n_items / (int)gridDim.x;  // complete rounds
+  return full + (item_of_cta(full) < n_items ? 1 : 0);
+}
+
 // Producer warp of the gather.  The CTA's work items are
-// items[blockIdx.x + m * gridDim.x], m = 0 .. my_n-1, largest first; step k
+// items[item_of_cta(m)], m = 0 .. my_n-1, largest first; step k
 // takes them alternately from the front and the back (large, small, large,
 // ...), so the copies of small items proceed while the consumers work through
 // large ones.  Item records are read 32 at a time (one per lane) and each
@@ -714,7 +729,7 @@ __device__ void ring_producer(const GArgs& p, const GroupWs& w, const GroupLayou
   const int from_back = fs != nullptr ? 0 : 1;
   auto record = [&](int kk) {
     const int m = ((kk & 1) == from_back) ? my_n - 1 - (kk >> 1) : (kk >> 1);
-    return kk < my_n ? w.items[blockIdx.x + (size_t)m * gridDim.x] : make_int4(0, 0, 0, 0);
+    return kk < my_n ? w.items[item_of_cta(m)] : make_int4(0, 0, 0, 0);
   };
   // the row block's copies into slot q, on its full barrier (lane 0)
   auto issue_rows = [&](uint32_t q, int row) {
@@ -986,10 +1001,6 @@ __device__ void ring_consumers(const GArgs& p, const GroupLayout& L, const Ring&
   }
 }
 
-__device__ __forceinline__ int items_of_cta(const GroupWs& w) {
-  const int n_items = (int)ld_relaxed_u32(&w.ctl[kCtlItems]);
-  return n_items > (int)blockIdx.x ? (n_items - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x : 0;
-}
 
 template <int NT, bool kExactN, bool kNf3>
 __global__ void __launch_bounds__(kGroupThreads, 1) grouped_gather_kernel(const GArgs p, const GroupWs w,
