@@ -75,6 +75,8 @@ def parse_args():
     ap.add_argument("--no-extras", action="store_true", help="skip the build / NF3 / other-case legs")
     ap.add_argument("--no-offload", action="store_true", help="skip the host-resident (offloaded) table leg")
     ap.add_argument("--no-decode", action="store_true", help="skip the small-batch (decode) sweeps")
+    ap.add_argument("--no-ffn", action="store_true", help="skip the FFN-block leg")
+    ap.add_argument("--ffn-only", action="store_true", help="run only the FFN-block leg")
     ap.add_argument("--decode-only", action="store_true", help="run only the small-batch (decode) sweeps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
@@ -331,6 +333,22 @@ def main():
             dist.destroy_process_group()
         return
 
+    if args.ffn_only:
+        shape = inputs.SHAPES["1b"]
+        g = torch.Generator(device=dev)
+        g.manual_seed(shape.seed)
+        luts = [(torch.randn((shape.V, shape.N, shape.D), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+                for _ in range(2)]
+        routers = [(torch.randn((shape.D, shape.N), generator=g, device=dev) * 0.02).to(torch.bfloat16)]
+        _, bf16_peak, bf16_sust, _ = measured_peaks()
+        res = ffn_leg(mole, luts, routers, np.random.default_rng(shape.seed), g, dev, stream, max(3, args.warmup),
+                      (bf16_peak, bf16_sust))
+        if rank == 0:
+            print(json.dumps({"ffn_block": res}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
     if args.build_only:
         hbm_peak, bf16_peak, bf16_sust, peak_kind = measured_peaks()
         res = build_leg(mole, dev, stream, bf16_peak, bf16_sust, peak_kind, reps=max(1, args.steps),
@@ -451,6 +469,8 @@ def main():
         line["nf3"] = nf3_leg(mole, luts, routers, id_pool, h_pool, uniq_counts, dev, stream, W, K, T, P, L)
         if not args.no_offload:
             line["offload"] = offload_leg(mole, luts, routers, rng, g, dev, stream, W, L)
+        if not args.no_ffn:
+            line["ffn_block"] = ffn_leg(mole, luts, routers, rng, g, dev, stream, W, (bf16_peak, bf16_sust))
         del luts
         torch.cuda.empty_cache()
         if not args.no_decode:
@@ -754,6 +774,61 @@ def offload_leg(mole, luts, routers, rng, g, dev, stream, W, L):
         del ids, groups, stg, hs_l, out
     del host, hc, hs
     return res
+
+
+def ffn_leg(mole, luts, routers, rng, g, dev, stream, W, peaks):
+    """The MoLE FFN block of a 1B-shaped layer (§8(f) rank 1): one shared expert
+    (D x 8192 GELU FFN, as wide as a routed expert), the routed mixture from the
+    table, and the residual, for T = 16384 Zipf tokens.  mole_ffn_block = the
+    grouped combine into a workspace, then the shared expert's two tcgen05
+    GEMMs, the second adding the mixture and the residual in its epilogue."""
+    import torch
+    shape = inputs.SHAPES["1b"]
+    V, D, N, Ds, T = shape.V, shape.D, shape.N, shape.Dr, 16384
+    bf16_peak, bf16_sust = peaks
+    W1s = (torch.randn((D, Ds), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+    W2s = (torch.randn((Ds, D), generator=g, device=dev) * 0.02).to(torch.bfloat16)
+    ids = torch.from_numpy(inputs.draw_ids(rng, T, V, "zipf")).to(dev)
+    h = torch.randn((T, D), generator=g, device=dev).to(torch.bfloat16)
+    res = torch.randn((T, D), generator=g, device=dev)
+    out = torch.empty((T, D), dtype=torch.float32, device=dev)
+    mix = torch.empty((T, D), dtype=torch.float32, device=dev)
+    groups = mole.mole_token_groups_build(ids, V, N, stream=stream)
+    ws = torch.empty(mole.mole_ffn_block_workspace(T, D, Ds), dtype=torch.uint8, device=dev)
+    flops = 4.0 * T * D * Ds
+
+    def block(i):
+        mole.mole_ffn_block(ids, groups, h, routers[0], luts[i % len(luts)], W1s, W2s, "gelu", residual=res, out=out,
+                            workspace=ws, stream=stream)
+
+    def shared(i):
+        mole.mole_shared_ffn(h, W1s, W2s, "gelu", out=out, workspace=ws, stream=stream)
+
+    def unfused(i):  # the three terms apart: combine, shared expert, then two element-wise adds
+        mole.mole_lookup_combine_groups(ids, groups, h, routers[0], luts[i % len(luts)], out=mix, stream=stream)
+        mole.mole_shared_ffn(h, W1s, W2s, "gelu", out=out, workspace=ws, stream=stream)
+        out.add_(mix).add_(res)
+
+    res_line = {}
+    for name, fn in (("ffn_block", block), ("shared_expert", shared), ("unfused", unfused)):
+        for i in range(max(W, 3)):
+            fn(i)
+        n = 10
+        ms = time_block(fn, n, stream) / n
+        res_line[f"{name}_us"] = ms * 1e3
+    assert mole.mole_check(stream) == 0
+    sh = res_line["shared_expert_us"] / 1e6
+    res_line.update({
+        "workload": f"1B-shaped FFN block: T={T} Zipf tokens, shared expert {D}x{Ds} GELU FFN (bf16, fp32 "
+                    f"accumulate), table [{V}, {N}, {D}] bf16, residual fp32",
+        "tokens_per_s": T / (res_line["ffn_block_us"] / 1e6),
+        "shared_expert_tflops": flops / sh / 1e12,
+        "shared_expert_frac_of_bf16_peak": flops / sh / 1e12 / bf16_peak,
+        "shared_expert_frac_of_sustained": (flops / sh / 1e12 / bf16_sust) if bf16_sust else None,
+        "combine_share_us": res_line["ffn_block_us"] - res_line["shared_expert_us"],
+    })
+    del W1s, W2s, h, res, out, mix, ws, groups
+    return res_line
 
 
 def graph_pass_us(passes, stream, dev, replays=60):

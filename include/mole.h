@@ -269,6 +269,42 @@ mole_status mole_lookup_combine_offload(int64_t T, const void* groups, size_t by
                                         int32_t N, int64_t D, mole_dtype dt, int32_t nf3, float* out,
                                         cudaStream_t stream);
 
+/*
+ * ---- FFN block: shared expert + routed-expert mixture + residual ----
+ * (MoLE page, 训练阶段 and 推理阶段: the shared experts stay dense FFNs on the
+ * previous layer's output at inference; only the routed experts become the
+ * table.  The page gives no formula; this library's reading: one shared
+ * expert of the routed experts' form, act(h . W1s) . W2s, and the block's
+ * output is residual + shared expert + routed mixture.)
+ *
+ * mole_shared_ffn: out = act(h . W1s) . W2s + add + residual  (fp32)
+ *   h : [T, D] bf16   W1s : [D, Ds] bf16   W2s : [Ds, D] bf16
+ *   add, residual : [T, D] fp32 or NULL   out : [T, D] fp32 (may be add or
+ *   residual: each element is read before it is written)
+ *   Two tcgen05 GEMMs (fp32 accumulate); the hidden activation is rounded to
+ *   bf16 in `workspace` (at least mole_shared_ffn_workspace(T, Ds) bytes);
+ *   the additions happen in the second GEMM's epilogue.  Needs D % 64 == 0,
+ *   Ds % 64 == 0 and 16-byte aligned pointers (else MOLE_ERR_UNSUPPORTED /
+ *   MOLE_ERR_ALIGN).
+ *
+ * mole_ffn_block: out = residual + act(h . W1s) . W2s + sum_j g_j LUT[ids[t], j]
+ *   The routed mixture is mole_lookup_combine_groups over `groups` (built from
+ *   the same ids, T and N), written into the workspace and added in the
+ *   shared expert's second GEMM epilogue.  bf16 inputs, D % 64 == 0,
+ *   Ds % 64 == 0; workspace of mole_ffn_block_workspace(T, D, Ds) bytes; out
+ *   may be residual.  Bad ids: NaN rows and MOLE_ERR_INDEX from mole_check,
+ *   as for the combine.
+ */
+size_t mole_shared_ffn_workspace(int64_t T, int64_t Ds);
+mole_status mole_shared_ffn(const void* h, const void* W1s, const void* W2s, int64_t T, int64_t D, int64_t Ds,
+                            mole_act act, const float* add, const float* residual, float* out, void* workspace,
+                            size_t ws_bytes, cudaStream_t stream);
+size_t mole_ffn_block_workspace(int64_t T, int64_t D, int64_t Ds);
+mole_status mole_ffn_block(const int32_t* ids, int64_t T, const void* groups, size_t groups_bytes, const void* h,
+                           const void* Wr, const void* lut, int64_t V, int32_t N, const void* W1s, const void* W2s,
+                           int64_t D, int64_t Ds, mole_act act, const float* residual, float* out,
+                           void* workspace, size_t ws_bytes, cudaStream_t stream);
+
 /* The 8 NF3 levels as fp16 bit patterns (ascending; index 3 is 0.0) and the 7
  * fp32 decision midpoints.  Host-only; no device work. */
 void mole_nf3_levels(uint16_t levels_f16[8]);

@@ -263,3 +263,60 @@ extern "C" mole_status mole_lookup_combine_offload(int64_t T, const void* groups
   return mole::combine_offload(groups, bytes, T, h, Wr, staging, staging_bytes, V, N, (int)D, dt == MOLE_BF16,
                                nf3 != 0, out, stream);
 }
+
+extern "C" size_t mole_shared_ffn_workspace(int64_t T, int64_t Ds) {
+  if (T <= 0 || Ds <= 0) return 0;
+  return (size_t)T * (size_t)Ds * 2;
+}
+
+extern "C" mole_status mole_shared_ffn(const void* h, const void* W1s, const void* W2s, int64_t T, int64_t D,
+                                       int64_t Ds, mole_act act, const float* add, const float* residual, float* out,
+                                       void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  if (!valid_act(act) || T < 0 || D <= 0 || Ds <= 0) return MOLE_ERR_ARG;
+  if (T == 0) return MOLE_OK;
+  if (!h || !W1s || !W2s || !out) return MOLE_ERR_ARG;
+  if (D % 64 != 0 || Ds % 64 != 0 || T > INT32_MAX || D > INT32_MAX || Ds > INT32_MAX) return MOLE_ERR_UNSUPPORTED;
+  if (!workspace || ws_bytes < mole_shared_ffn_workspace(T, Ds)) return MOLE_ERR_WORKSPACE;
+  if (!mole::aligned16(h) || !mole::aligned16(W1s) || !mole::aligned16(W2s) || !mole::aligned16(add) ||
+      !mole::aligned16(residual) || !mole::aligned16(out) || !mole::aligned16(workspace))
+    return MOLE_ERR_ALIGN;
+  mole_status st = check_device();
+  if (st != MOLE_OK) return st;
+  if (!mole::shared_ffn_tc_supported(T, D, Ds, h, W1s, W2s, add, residual, out, workspace))
+    return MOLE_ERR_UNSUPPORTED;
+  return mole::shared_ffn_tc(h, W1s, W2s, T, D, Ds, (int)act, add, residual, out, workspace, ws_bytes, stream);
+}
+
+extern "C" size_t mole_ffn_block_workspace(int64_t T, int64_t D, int64_t Ds) {
+  if (T <= 0 || D <= 0 || Ds <= 0) return 0;
+  const size_t h_bytes = ((size_t)T * (size_t)Ds * 2 + 255) / 256 * 256;
+  return h_bytes + (size_t)T * (size_t)D * 4;
+}
+
+extern "C" mole_status mole_ffn_block(const int32_t* ids, int64_t T, const void* groups, size_t groups_bytes,
+                                      const void* h, const void* Wr, const void* lut, int64_t V, int32_t N,
+                                      const void* W1s, const void* W2s, int64_t D, int64_t Ds, mole_act act,
+                                      const float* residual, float* out, void* workspace, size_t ws_bytes,
+                                      cudaStream_t stream) {
+  if (!valid_act(act)) return MOLE_ERR_ARG;
+  mole_status st = check_combine_bf16(ids, T, h, Wr, lut, V, N, D, MOLE_BF16, out);
+  if (st != MOLE_OK) return st;
+  st = check_groups(T, N, groups, groups_bytes);
+  if (st != MOLE_OK || T == 0) return st;
+  if (!W1s || !W2s || Ds <= 0) return MOLE_ERR_ARG;
+  if (D % 64 != 0 || Ds % 64 != 0 || T > INT32_MAX || Ds > INT32_MAX) return MOLE_ERR_UNSUPPORTED;
+  if (!workspace || ws_bytes < mole_ffn_block_workspace(T, D, Ds)) return MOLE_ERR_WORKSPACE;
+  if (!mole::aligned16(W1s) || !mole::aligned16(W2s) || !mole::aligned16(residual) || !mole::aligned16(workspace))
+    return MOLE_ERR_ALIGN;
+  st = check_device();
+  if (st != MOLE_OK) return st;
+  // the routed-expert mixture into the workspace (fp32 [T, D]), then the
+  // shared expert with the mixture and the residual added in its epilogue
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t h_bytes = ((size_t)T * (size_t)Ds * 2 + 255) / 256 * 256;
+  float* mix = reinterpret_cast<float*>(ws + h_bytes);
+  if (!mole::shared_ffn_tc_supported(T, D, Ds, h, W1s, W2s, mix, residual, out, ws)) return MOLE_ERR_UNSUPPORTED;
+  st = mole_lookup_combine_groups(ids, T, groups, groups_bytes, h, Wr, lut, V, N, D, MOLE_BF16, mix, stream);
+  if (st != MOLE_OK) return st;
+  return mole::shared_ffn_tc(h, W1s, W2s, T, D, Ds, (int)act, mix, residual, out, ws, h_bytes, stream);
+}

@@ -59,6 +59,12 @@ struct Params {
   int m_blocks, n_blocks;
   int64_t tiles;
   unsigned* err;
+  // fp32 output instead (one expert): Cf[m, n] = acc + add0[m, n] + add1[m, n]
+  // (either term may be absent), all three [M, N] row-major with stride ldc;
+  // Cf may be add0 or add1 (each element is read, then written, by one thread)
+  float* Cf;
+  const float* add0;
+  const float* add1;
 };
 
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
@@ -136,6 +142,38 @@ __device__ __forceinline__ void store_chunk_act(int act, const uint32_t (&r)[32]
     case MOLE_ACT_SILU: store_chunk<MOLE_ACT_SILU>(r, dst_row); break;
     default: store_chunk<MOLE_ACT_IDENTITY>(r, dst_row); break;
   }
+}
+
+// The fp32 epilogue: 32 columns of one row, plus up to two fp32 terms.
+__device__ __forceinline__ void store_chunk_f32(const uint32_t (&r)[32], const Params& p, int64_t off) {
+  float v[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+  if (p.add0 != nullptr) {
+    const float4* a = reinterpret_cast<const float4*>(p.add0 + off);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float4 t = a[q];
+      v[4 * q] += t.x;
+      v[4 * q + 1] += t.y;
+      v[4 * q + 2] += t.z;
+      v[4 * q + 3] += t.w;
+    }
+  }
+  if (p.add1 != nullptr) {
+    const float4* a = reinterpret_cast<const float4*>(p.add1 + off);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float4 t = a[q];
+      v[4 * q] += t.x;
+      v[4 * q + 1] += t.y;
+      v[4 * q + 2] += t.z;
+      v[4 * q + 3] += t.w;
+    }
+  }
+  float4* o = reinterpret_cast<float4*>(p.Cf + off);
+#pragma unroll
+  for (int q = 0; q < 8; ++q) o[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
 }
 
 __device__ __forceinline__ void decode_tile(const Params& p, int64_t tile, int& e, int& mb, int& nb) {
@@ -271,7 +309,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (col0 >= p.N) break;  // warp-uniform
         uint32_t r[32];
         tmem_ld32(tmem_base + ((uint32_t)(quad * 32) << 16) + acc * ACC_COLS + chunk * 32, r);
-        if (m < p.M) store_chunk_act(p.act, r, crow + col0);
+        if (m < p.M) {
+          if (p.Cf != nullptr)
+            store_chunk_f32(r, p, (int64_t)m * p.ldc + col0);
+          else
+            store_chunk_act(p.act, r, crow + col0);
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -499,7 +542,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (col0 >= p.N) break;  // warp-uniform
         uint32_t r[32];
         tmem_ld32(tmem_base + ((uint32_t)(quad * 32) << 16) + acc * ACC_COLS + chunk * 32, r);
-        if (m < p.M) store_chunk_act(p.act, r, crow + col0);
+        if (m < p.M) {
+          if (p.Cf != nullptr)
+            store_chunk_f32(r, p, (int64_t)m * p.ldc + col0);
+          else
+            store_chunk_act(p.act, r, crow + col0);
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -571,6 +619,67 @@ mole_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, Params p, 
 }
 
 }  // namespace
+
+bool shared_ffn_tc_supported(int64_t T, int64_t D, int64_t Ds, const void* h, const void* W1s, const void* W2s,
+                             const void* add0, const void* add1, const void* out, const void* ws) {
+  int dev = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return false;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (major != 10 || minor != 0) return false;
+  if (D % 64 != 0 || Ds % 64 != 0 || T < 1 || T > (1LL << 31) - 1 || D > (1LL << 31) - 1 || Ds > (1LL << 31) - 1)
+    return false;
+  return aligned16(h) && aligned16(W1s) && aligned16(W2s) && aligned16(add0) && aligned16(add1) && aligned16(out) &&
+         aligned16(ws) && encode_fn();
+}
+
+mole_status shared_ffn_tc(const void* h, const void* W1s, const void* W2s, int64_t T, int64_t D, int64_t Ds, int act,
+                          const float* add0, const float* add1, float* out, void* ws, size_t ws_bytes,
+                          cudaStream_t stream) {
+  if (ws_bytes < (size_t)T * Ds * 2) return MOLE_ERR_WORKSPACE;
+  unsigned* err = error_word();
+  if (!err) return MOLE_ERR_CUDA;
+  uint16_t* H = static_cast<uint16_t*>(ws);
+  const bool pair_tiles = T >= 2 * BM;
+  const int mtile = pair_tiles ? 2 * BM : BM;
+  // GEMM1: H = act(h . W1s), bf16
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, h, D, T, 1, D * 2, T * D * 2, BM)) return MOLE_ERR_CUDA;
+  if (!make_map(&mb, W1s, Ds, D, 1, Ds * 2, D * Ds * 2, BK)) return MOLE_ERR_CUDA;
+  Params p1{};
+  p1.M = (int)T;
+  p1.N = (int)Ds;
+  p1.K = (int)D;
+  p1.a_batched = 0;
+  p1.act = act;
+  p1.C = H;
+  p1.ldc = Ds;
+  p1.c_estride = T * Ds;
+  p1.m_blocks = (int)((T + mtile - 1) / mtile);
+  p1.n_blocks = (int)((Ds + BN - 1) / BN);
+  p1.tiles = (int64_t)p1.m_blocks * p1.n_blocks;
+  p1.err = err;
+  mole_status st = launch_gemm(ma, mb, p1, pair_tiles, stream);
+  if (st != MOLE_OK) return st;
+  // GEMM2: out = H . W2s + add0 + add1, fp32
+  if (!make_map(&ma, H, Ds, T, 1, Ds * 2, T * Ds * 2, BM)) return MOLE_ERR_CUDA;
+  if (!make_map(&mb, W2s, D, Ds, 1, D * 2, Ds * D * 2, BK)) return MOLE_ERR_CUDA;
+  Params p2{};
+  p2.M = (int)T;
+  p2.N = (int)D;
+  p2.K = (int)Ds;
+  p2.a_batched = 1;
+  p2.act = MOLE_ACT_IDENTITY;
+  p2.ldc = D;
+  p2.m_blocks = (int)((T + mtile - 1) / mtile);
+  p2.n_blocks = (int)((D + BN - 1) / BN);
+  p2.tiles = (int64_t)p2.m_blocks * p2.n_blocks;
+  p2.err = err;
+  p2.Cf = out;
+  p2.add0 = add0;
+  p2.add1 = add1;
+  return launch_gemm(ma, mb, p2, pair_tiles, stream);
+}
 
 bool build_tc_supported(int64_t V, int64_t D, int64_t Dr, const void* E, const void* W1, const void* W2,
                         const void* lut, const void* ws) {

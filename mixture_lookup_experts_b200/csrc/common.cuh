@@ -145,6 +145,13 @@ bool build_tc_supported(int64_t V, int64_t D, int64_t Dr, const void* E, const v
 mole_status build_tc(const void* E, const void* W1, const void* W2, int64_t V, int64_t D, int N,
                      int64_t Dr, int act, void* lut, void* ws, size_t ws_bytes, cudaStream_t stream);
 
+// Shared-expert FFN on the tensor cores (build_tc.cu): out = act(h . W1s) . W2s
+// + add0 + add1 (fp32), the hidden activation rounded to bf16 in `ws`.
+bool shared_ffn_tc_supported(int64_t T, int64_t D, int64_t Ds, const void* h, const void* W1s, const void* W2s,
+                             const void* add0, const void* add1, const void* out, const void* ws);
+mole_status shared_ffn_tc(const void* h, const void* W1s, const void* W2s, int64_t T, int64_t D, int64_t Ds, int act,
+                          const float* add0, const float* add1, float* out, void* ws, size_t ws_bytes,
+                          cudaStream_t stream);
 // Combine / NF3 / plan entry points (combine.cu / plan.cu).
 mole_status combine_dispatch(const int32_t* ids, int64_t T, const void* h, const void* Wr,
                              const void* table, const uint16_t* scales, int64_t V, int N, int D,

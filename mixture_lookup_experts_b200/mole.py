@@ -49,6 +49,10 @@ SIGNATURES = {
     "mole_offload_staging_bytes": ([_I64, _I64, _I32, _I64, _I, _I32], _SZ),
     "mole_offload_stage": ([_I64, _P, _SZ, _P, _P, _I64, _I32, _I64, _I, _I32, _P, _SZ, _P, _P], _I),
     "mole_lookup_combine_offload": ([_I64, _P, _SZ, _P, _P, _P, _SZ, _I64, _I32, _I64, _I, _I32, _P, _P], _I),
+    "mole_shared_ffn_workspace": ([_I64, _I64], _SZ),
+    "mole_shared_ffn": ([_P, _P, _P, _I64, _I64, _I64, _I, _P, _P, _P, _P, _SZ, _P], _I),
+    "mole_ffn_block_workspace": ([_I64, _I64, _I64], _SZ),
+    "mole_ffn_block": ([_P, _I64, _P, _SZ, _P, _P, _P, _I64, _I32, _P, _P, _I64, _I64, _I, _P, _P, _P, _SZ, _P], _I),
     "mole_nf3_levels": ([_P], None),
     "mole_nf3_midpoints": ([_P], None),
     "mole_gather_plan": ([_P, _I64, _I64, _P, _P, _P, _P], _I),
@@ -308,6 +312,48 @@ def mole_lookup_combine_offload(groups: torch.Tensor, h: torch.Tensor, Wr: torch
     _ok(lib.mole_lookup_combine_offload(T, _ptr(groups), groups.numel(), _ptr(h), _ptr(Wr), _ptr(staging),
                                         staging.numel(), V, N, D, _dt(h), int(nf3), _ptr(out), _stream(stream)),
         "mole_lookup_combine_offload")
+    return out
+
+
+def mole_shared_ffn_workspace(T: int, Ds: int) -> int:
+    return int(lib.mole_shared_ffn_workspace(T, Ds))
+
+
+def mole_shared_ffn(h: torch.Tensor, W1s: torch.Tensor, W2s: torch.Tensor, act: str = "gelu",
+                    add: torch.Tensor | None = None, residual: torch.Tensor | None = None,
+                    out: torch.Tensor | None = None, workspace: torch.Tensor | None = None, stream=None):
+    """out = act(h . W1s) . W2s + add + residual (fp32; see mole.h)."""
+    _contig(h, W1s, W2s, add, residual, out, workspace)
+    T, D = h.shape
+    Ds = W1s.shape[1]
+    if out is None:
+        out = torch.empty((T, D), dtype=torch.float32, device=h.device)
+    if workspace is None:
+        workspace = torch.empty(max(1, mole_shared_ffn_workspace(T, Ds)), dtype=torch.uint8, device=h.device)
+    _ok(lib.mole_shared_ffn(_ptr(h), _ptr(W1s), _ptr(W2s), T, D, Ds, ACT[act], _ptr(add), _ptr(residual), _ptr(out),
+                            _ptr(workspace), workspace.numel(), _stream(stream)), "mole_shared_ffn")
+    return out
+
+
+def mole_ffn_block_workspace(T: int, D: int, Ds: int) -> int:
+    return int(lib.mole_ffn_block_workspace(T, D, Ds))
+
+
+def mole_ffn_block(ids: torch.Tensor, groups: torch.Tensor, h: torch.Tensor, Wr: torch.Tensor, lut: torch.Tensor,
+                   W1s: torch.Tensor, W2s: torch.Tensor, act: str = "gelu", residual: torch.Tensor | None = None,
+                   out: torch.Tensor | None = None, workspace: torch.Tensor | None = None, stream=None):
+    """out = residual + act(h . W1s) . W2s + the routed-expert mixture (see mole.h)."""
+    _contig(ids, groups, h, Wr, lut, W1s, W2s, residual, out, workspace)
+    V, N, D = lut.shape
+    T = ids.numel()
+    Ds = W1s.shape[1]
+    if out is None:
+        out = torch.empty((T, D), dtype=torch.float32, device=h.device)
+    if workspace is None:
+        workspace = torch.empty(max(1, mole_ffn_block_workspace(T, D, Ds)), dtype=torch.uint8, device=h.device)
+    _ok(lib.mole_ffn_block(_ptr(ids), T, _ptr(groups), groups.numel(), _ptr(h), _ptr(Wr), _ptr(lut), V, N, _ptr(W1s),
+                           _ptr(W2s), D, Ds, ACT[act], _ptr(residual), _ptr(out), _ptr(workspace), workspace.numel(),
+                           _stream(stream)), "mole_ffn_block")
     return out
 
 

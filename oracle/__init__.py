@@ -167,6 +167,28 @@ def _build_lut_ex(E, W1, W2, act_name, round_h, rows, nthreads):
     return out, allow, int(n_amb[0])
 
 
+def ffn_block(ids, h, Wr, lut, W1s, W2s, act_name: str = "gelu", residual=None, nthreads: int = 0):
+    """out[t] = residual[t] + act(h[t] . W1s) . W2s + sum_j g_j LUT[ids[t], j] in fp64.
+
+    MoLE page, 训练阶段 / 推理阶段: at inference the shared experts remain dense
+    FFNs on the previous layer's output h, and only the routed experts become
+    the table; the layer output adds the residual (reading: one shared expert
+    of the routed experts' form).  The shared expert is build_lut's expert
+    evaluated on the rows of h (the hidden activation rounded to bf16 at the
+    same point), the mixture is combine().  Returns (out [T, D], allowance of
+    the shared expert's ambiguous bf16 roundings [T, D], n_bad).
+    """
+    T, D = h.shape
+    Ds = W1s.shape[1]
+    shared, allow, _ = build_lut(h, W1s.reshape(1, D, Ds), W2s.reshape(1, Ds, D), act_name, True, None, nthreads,
+                                 with_allowance=True)
+    mix, n_bad = combine(ids, h, Wr, lut, nthreads=nthreads)
+    out = shared[:, 0, :] + mix
+    if residual is not None:
+        out = out + np.asarray(residual, dtype=np.float64)
+    return out, allow[:, 0, :], n_bad
+
+
 def round_bf16_array(x: np.ndarray) -> np.ndarray:
     """Element-wise bf16 rounding (ties to even) of float64 values."""
     x = np.ascontiguousarray(x, dtype=np.float64)

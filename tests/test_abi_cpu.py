@@ -151,3 +151,28 @@ def test_offload_staging_size_and_checks(mole):
     if not torch.cuda.is_available():
         assert stage(5, P, gws, P, None, 10, 4, 64, 1, 0, P, sws, None, None) == 8
         assert comb(5, P, gws, P, P, P, sws, 10, 4, 64, 1, 0, P, None) == 8
+
+
+def test_ffn_checks(mole):
+    import torch
+    lib = mole.lib
+    P = 0x100000
+    assert mole.mole_shared_ffn_workspace(100, 512) == 100 * 512 * 2
+    assert mole.mole_ffn_block_workspace(100, 128, 512) >= 100 * 512 * 2 + 100 * 128 * 4
+    ws = mole.mole_shared_ffn_workspace(5, 64)
+    assert lib.mole_shared_ffn(P, P, P, 5, 64, 64, 9, None, None, P, P, ws, None) == 1       # bad act
+    assert lib.mole_shared_ffn(P, P, P, 5, 96, 64, 0, None, None, P, P, ws, None) == 3       # D % 64
+    assert lib.mole_shared_ffn(P, P, P, 5, 64, 64, 0, None, None, P, P, ws - 1, None) == 4   # workspace
+    assert lib.mole_shared_ffn(P, P, P, 5, 64, 64, 0, P + 4, None, P, P, ws, None) == 2     # misaligned add
+    assert lib.mole_shared_ffn(None, P, P, 5, 64, 64, 0, None, None, P, P, ws, None) == 1    # no h
+    assert lib.mole_shared_ffn(None, None, None, 0, 64, 64, 0, None, None, None, None, 0, None) == 0  # T == 0
+    gws = mole.mole_token_groups_workspace(5, 4)
+    fws = mole.mole_ffn_block_workspace(5, 64, 64)
+    blk = lib.mole_ffn_block
+    assert blk(P, 5, P, gws, P, P, P, 10, 4, P, P, 64, 64, 0, None, P, P, fws - 1, None) == 4
+    assert blk(P, 5, P, gws, P, P, P, 10, 4, None, P, 64, 64, 0, None, P, P, fws, None) == 1
+    assert blk(P, 5, P, gws, P, P, P, 10, 4, P, P, 64, 96, 0, None, P, P, fws, None) == 3
+    assert blk(P, 5, None, gws, P, P, P, 10, 4, P, P, 64, 64, 0, None, P, P, fws, None) == 4
+    if not torch.cuda.is_available():
+        assert lib.mole_shared_ffn(P, P, P, 5, 64, 64, 0, None, None, P, P, ws, None) == 8
+        assert blk(P, 5, P, gws, P, P, P, 10, 4, P, P, 64, 64, 0, None, P, P, fws, None) == 8

@@ -419,3 +419,59 @@ def test_build_allowance_flags_only_values_at_a_rounding_boundary(oracle_mod):
 def test_round_bf16_array_matches_scalar(oracle_mod):
     x = np.random.default_rng(8).standard_normal(500) * 10
     np.testing.assert_array_equal(oracle_mod.round_bf16_array(x), [oracle_mod.round_bf16(v) for v in x])
+
+
+# --------------------------------------------------------------------------
+# FFN block: residual + shared expert + routed mixture
+# --------------------------------------------------------------------------
+
+def _ffn_inputs(seed, T=9, D=8, N=3, Ds=16, V=6):
+    rng = np.random.default_rng(seed)
+    h = inputs.normal(rng, (T, D), 1.0, "bf16")
+    Wr = inputs.normal(rng, (D, N), 0.5, "bf16")
+    lut = inputs.normal(rng, (V, N, D), 0.5, "bf16")
+    W1s = inputs.normal(rng, (D, Ds), 0.3, "bf16")
+    W2s = inputs.normal(rng, (Ds, D), 0.3, "bf16")
+    ids = rng.integers(0, V, T).astype(np.int32)
+    res = rng.standard_normal((T, D)).astype(np.float32)
+    return ids, h, Wr, lut, W1s, W2s, res
+
+
+def test_ffn_block_without_shared_expert_is_residual_plus_mixture(oracle_mod):
+    ids, h, Wr, lut, W1s, W2s, res = _ffn_inputs(71)
+    zero = np.zeros_like(W2s)
+    out, allow, nbad = oracle_mod.ffn_block(ids, h, Wr, lut, W1s, zero, "gelu", res)
+    mix, _ = oracle_mod.combine(ids, h, Wr, lut)
+    assert nbad == 0
+    np.testing.assert_allclose(out, res.astype(np.float64) + mix, rtol=0, atol=0)
+    assert np.all(allow == 0)
+
+
+def test_ffn_block_shared_expert_selection_is_matrix_product(oracle_mod):
+    # act = identity and W1s selecting columns of h (one 1.0 per column): the
+    # hidden activation is h's columns (exact in bf16), so the shared expert is
+    # h[:, sel] @ W2s, a numpy product; a zero table leaves only it
+    ids, h, Wr, lut, _, W2s, _ = _ffn_inputs(72, D=8, Ds=16)
+    D, Ds = 8, 16
+    sel = np.random.default_rng(3).integers(0, D, Ds)
+    W1 = np.zeros((D, Ds), np.float32)
+    W1[sel, np.arange(Ds)] = 1.0
+    W1s = inputs.f32_to_bf16_bits(W1)
+    zlut = np.zeros_like(lut)
+    out, allow, _ = oracle_mod.ffn_block(ids, h, Wr, zlut, W1s, W2s, "identity")
+    ref = _f(h)[:, sel] @ _f(W2s)
+    np.testing.assert_allclose(out, ref, rtol=1e-12, atol=1e-15)
+    assert np.all(allow == 0)
+
+
+def test_ffn_block_terms_add(oracle_mod):
+    # the three terms are computed apart and summed: out(res) - out(0) = res,
+    # and the shared expert equals build_lut's expert on h's rows
+    ids, h, Wr, lut, W1s, W2s, res = _ffn_inputs(73)
+    a, _, _ = oracle_mod.ffn_block(ids, h, Wr, lut, W1s, W2s, "gelu", res)
+    b, _, _ = oracle_mod.ffn_block(ids, h, Wr, lut, W1s, W2s, "gelu", None)
+    np.testing.assert_allclose(a - b, res.astype(np.float64), rtol=0, atol=1e-12)
+    D, Ds = W1s.shape
+    shared = oracle_mod.build_lut(h, W1s.reshape(1, D, Ds), W2s.reshape(1, Ds, D), "gelu")[:, 0, :]
+    mix, _ = oracle_mod.combine(ids, h, Wr, lut)
+    np.testing.assert_allclose(b, shared + mix, rtol=0, atol=1e-14)
