@@ -48,7 +48,7 @@ METRIC = "MoLE lookup-combine tokens/s & HBM GB/s vs 8 TB/s; LUT build TFLOP/s"
 UNIT = "tokens/s"
 KERNEL_SOURCES = ["mixture_lookup_experts_b200/csrc/combine.cu", "mixture_lookup_experts_b200/csrc/grouped.cu",
                   "mixture_lookup_experts_b200/csrc/router_tc.cu", "mixture_lookup_experts_b200/csrc/combine_common.cuh",
-                  "mixture_lookup_experts_b200/csrc/common.cuh"]
+                  "mixture_lookup_experts_b200/csrc/common.cuh", "mixture_lookup_experts_b200/csrc/nf3.cuh"]
 PROFILE_SUMMARY = {"grouped": "profiles/combine_grouped_bf16_1b_T16384_zipf.md",
                    "plain": "profiles/combine_bf16_1b_T16384_zipf.md"}
 KERNELS = {
@@ -954,10 +954,22 @@ def build_leg(mole, dev, stream, bf16_peak, bf16_sust, peak_kind, reps=3, warmup
     best = min(ms)
     flops = 4.0 * V * D * Dr * N
     tf = flops / (best / 1e3) / 1e12
+    # the NF3 table straight from the build (quantising epilogue) vs build + quantiser
+    codes = torch.empty((V, N, D // 64, 24), dtype=torch.uint8, device=dev)
+    scales = torch.empty((V, N, D // 64), dtype=torch.float16, device=dev)
+    mole.mole_build_lut_nf3(E, W1, W2, codes=codes, scales=scales, workspace=ws, stream=stream)
+    nf3_ms = min(time_launches(lambda i: mole.mole_build_lut_nf3(E, W1, W2, codes=codes, scales=scales, workspace=ws,
+                                                                 stream=stream), reps, stream))
+    q_ms = min(time_launches(lambda i: mole.mole_quantize_lut_nf3(lut, codes, scales, stream=stream), reps, stream))
+    assert mole.mole_check(stream) == 0
+    del codes, scales
     return {"workload": f"410M-shaped table build V={V} D={D} N={N} Dr={Dr} GELU (2 tcgen05 GEMMs per expert group)",
             "tflops": tf, "ms": best, "flops": flops, "frac_of_bf16_peak": tf / bf16_peak,
             "peak": bf16_peak, "peak_source": f"{peak_kind} burst bf16 (MEASURED_PEAKS.json)",
-            "frac_of_sustained": (tf / bf16_sust) if bf16_sust else None, "frac_of_2250": tf / 2250.0}
+            "frac_of_sustained": (tf / bf16_sust) if bf16_sust else None, "frac_of_2250": tf / 2250.0,
+            "nf3_build_ms": nf3_ms, "build_then_quantize_ms": best + q_ms,
+            "nf3_build_note": "mole_build_lut_nf3 (NF3 quantiser in the second GEMM's epilogue, no bf16 table) vs "
+                              "mole_build_lut + mole_quantize_lut_nf3"}
 
 
 def cpu_baseline(args):

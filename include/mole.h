@@ -194,6 +194,20 @@ mole_status mole_quantize_lut_nf3(const void* lut_bf16, int64_t V, int32_t N, in
                                   uint8_t* codes, uint16_t* scales, cudaStream_t stream);
 
 /*
+ * mole_build_lut and mole_quantize_lut_nf3 in one pass: the bf16 table is
+ * never written.  The second tensor-core GEMM's epilogue rounds each output
+ * to bf16 (the value mole_build_lut would store), quantises every 64-element
+ * block of a (v, j) row in registers and writes the codes and the fp16 scale;
+ * the results equal mole_build_lut followed by mole_quantize_lut_nf3, bit for
+ * bit.  bf16 only, on the tensor-core path (D % 64 == 0, Dr % 64 == 0,
+ * 16-byte aligned embed, W1, W2 and workspace; else MOLE_ERR_UNSUPPORTED);
+ * codes 8-byte aligned.  Workspace as for mole_build_lut (dt = MOLE_BF16).
+ */
+mole_status mole_build_lut_nf3(const void* embed, const void* W1, const void* W2, int64_t V, int64_t D,
+                               int32_t N, int64_t Dr, mole_act act, uint8_t* codes, uint16_t* scales,
+                               void* workspace, size_t ws_bytes, cudaStream_t stream);
+
+/*
  * mole_lookup_combine over an NF3 table: the row element for (id, j, d) is
  * level[c] * s of its block (exact in fp32), dequantised in registers inside
  * the gather.  Same arguments and error behaviour as mole_lookup_combine,

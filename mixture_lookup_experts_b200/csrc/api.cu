@@ -320,3 +320,18 @@ extern "C" mole_status mole_ffn_block(const int32_t* ids, int64_t T, const void*
   if (st != MOLE_OK) return st;
   return mole::shared_ffn_tc(h, W1s, W2s, T, D, Ds, (int)act, mix, residual, out, ws, h_bytes, stream);
 }
+
+extern "C" mole_status mole_build_lut_nf3(const void* embed, const void* W1, const void* W2, int64_t V, int64_t D,
+                                          int32_t N, int64_t Dr, mole_act act, uint8_t* codes, uint16_t* scales,
+                                          void* workspace, size_t ws_bytes, cudaStream_t stream) {
+  if (!valid_act(act)) return MOLE_ERR_ARG;
+  if (V <= 0 || D <= 0 || N <= 0 || Dr <= 0) return MOLE_ERR_ARG;
+  if (!embed || !W1 || !W2 || !codes || !scales) return MOLE_ERR_ARG;
+  if (V > INT32_MAX || D > INT32_MAX || Dr > INT32_MAX || D % 64 != 0 || Dr % 64 != 0) return MOLE_ERR_UNSUPPORTED;
+  if (!workspace || ws_bytes < mole_build_lut_workspace(V, D, N, Dr, MOLE_BF16, 1)) return MOLE_ERR_WORKSPACE;
+  if (!mole::aligned8(codes) || (reinterpret_cast<uintptr_t>(scales) & 1u)) return MOLE_ERR_ALIGN;
+  mole_status st = check_device();
+  if (st != MOLE_OK) return st;
+  if (!mole::build_tc_supported(V, D, Dr, embed, W1, W2, workspace, workspace)) return MOLE_ERR_UNSUPPORTED;
+  return mole::build_tc_nf3(embed, W1, W2, V, D, N, Dr, (int)act, codes, scales, workspace, ws_bytes, stream);
+}

@@ -29,6 +29,7 @@
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
+#include "nf3.cuh"
 
 namespace mole {
 namespace {
@@ -65,6 +66,12 @@ struct Params {
   float* Cf;
   const float* add0;
   const float* add1;
+  // NF3 table instead (second build GEMM): the bf16-rounded outputs of each
+  // 64-column block quantised in registers; block (m, e, b) at
+  // codes + (m * q_row + e * q_e + b) * 24 and scales + the same index
+  uint8_t* codes;
+  uint16_t* scales;
+  int64_t q_row, q_e;
 };
 
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
@@ -174,6 +181,56 @@ __device__ __forceinline__ void store_chunk_f32(const uint32_t (&r)[32], const P
   float4* o = reinterpret_cast<float4*>(p.Cf + off);
 #pragma unroll
   for (int q = 0; q < 8; ++q) o[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+
+// The NF3 epilogue: two 32-column chunks (one 64-element block) of one row,
+// rounded to bf16 as the table would hold them, quantised, codes and scale
+// stored.
+__device__ __forceinline__ void store_block_nf3(const uint32_t (&r0)[32], const uint32_t (&r1)[32], const Params& p,
+                                                int64_t blk) {
+  uint32_t xw[32];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const __nv_bfloat162 a = __floats2bfloat162_rn(__uint_as_float(r0[2 * i]), __uint_as_float(r0[2 * i + 1]));
+    const __nv_bfloat162 b = __floats2bfloat162_rn(__uint_as_float(r1[2 * i]), __uint_as_float(r1[2 * i + 1]));
+    xw[i] = *reinterpret_cast<const uint32_t*>(&a);
+    xw[16 + i] = *reinterpret_cast<const uint32_t*>(&b);
+  }
+  uint32_t packed[6];
+  const uint16_t s16 = nf3_quantize_block(xw, packed);
+  uint2* dst = reinterpret_cast<uint2*>(p.codes + blk * 24);
+  dst[0] = make_uint2(packed[0], packed[1]);
+  dst[1] = make_uint2(packed[2], packed[3]);
+  dst[2] = make_uint2(packed[4], packed[5]);
+  p.scales[blk] = s16;
+}
+
+// One epilogue warp's columns of one tile: BN/64 chunks of 32 from chunk0.
+__device__ __forceinline__ void epilogue_tile(const Params& p, uint32_t taddr, int e, int m, int nb, int chunk0,
+                                              uint16_t* crow) {
+  if (p.codes != nullptr) {
+    for (int chunk = chunk0; chunk < chunk0 + BN / 64; chunk += 2) {
+      const int col0 = nb * BN + chunk * 32;
+      if (col0 >= p.N) break;  // warp-uniform; p.N % 64 == 0
+      uint32_t r0[32], r1[32];
+      tmem_ld32(taddr + chunk * 32, r0);
+      tmem_ld32(taddr + (chunk + 1) * 32, r1);
+      if (m < p.M) store_block_nf3(r0, r1, p, (int64_t)m * p.q_row + (int64_t)e * p.q_e + col0 / 64);
+    }
+    return;
+  }
+  for (int chunk = chunk0; chunk < chunk0 + BN / 64; ++chunk) {
+    const int col0 = nb * BN + chunk * 32;
+    if (col0 >= p.N) break;  // warp-uniform
+    uint32_t r[32];
+    tmem_ld32(taddr + chunk * 32, r);
+    if (m < p.M) {
+      if (p.Cf != nullptr)
+        store_chunk_f32(r, p, (int64_t)m * p.ldc + col0);
+      else
+        store_chunk_act(p.act, r, crow + col0);
+    }
+  }
 }
 
 __device__ __forceinline__ void decode_tile(const Params& p, int64_t tile, int& e, int& mb, int& nb) {
@@ -304,18 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       decode_tile(p, tile, e, mb, nb);
       const int m = mb * BM + quad * 32 + lane;
       uint16_t* crow = p.C + (int64_t)e * p.c_estride + (int64_t)m * p.ldc;
-      for (int chunk = chunk0; chunk < chunk0 + BN / 64; ++chunk) {
-        const int col0 = nb * BN + chunk * 32;
-        if (col0 >= p.N) break;  // warp-uniform
-        uint32_t r[32];
-        tmem_ld32(tmem_base + ((uint32_t)(quad * 32) << 16) + acc * ACC_COLS + chunk * 32, r);
-        if (m < p.M) {
-          if (p.Cf != nullptr)
-            store_chunk_f32(r, p, (int64_t)m * p.ldc + col0);
-          else
-            store_chunk_act(p.act, r, crow + col0);
-        }
-      }
+      epilogue_tile(p, tmem_base + ((uint32_t)(quad * 32) << 16) + acc * ACC_COLS, e, m, nb, chunk0, crow);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -537,18 +583,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       decode_tile(p, tile, e, mb, nb);
       const int m = mb * 2 * BM + (int)rank * BM + quad * 32 + lane;
       uint16_t* crow = p.C + (int64_t)e * p.c_estride + (int64_t)m * p.ldc;
-      for (int chunk = chunk0; chunk < chunk0 + BN / 64; ++chunk) {
-        const int col0 = nb * BN + chunk * 32;
-        if (col0 >= p.N) break;  // warp-uniform
-        uint32_t r[32];
-        tmem_ld32(tmem_base + ((uint32_t)(quad * 32) << 16) + acc * ACC_COLS + chunk * 32, r);
-        if (m < p.M) {
-          if (p.Cf != nullptr)
-            store_chunk_f32(r, p, (int64_t)m * p.ldc + col0);
-          else
-            store_chunk_act(p.act, r, crow + col0);
-        }
-      }
+      epilogue_tile(p, tmem_base + ((uint32_t)(quad * 32) << 16) + acc * ACC_COLS, e, m, nb, chunk0, crow);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa(smem_u32(&tempty[acc]), 0));
@@ -619,6 +654,10 @@ mole_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, Params p, 
 }
 
 }  // namespace
+
+mole_status build_tc_any(const void* E, const void* W1, const void* W2, int64_t V, int64_t D, int N, int64_t Dr,
+                         int act, void* lut, uint8_t* codes, uint16_t* scales, void* ws, size_t ws_bytes,
+                         cudaStream_t stream);
 
 bool shared_ffn_tc_supported(int64_t T, int64_t D, int64_t Ds, const void* h, const void* W1s, const void* W2s,
                              const void* add0, const void* add1, const void* out, const void* ws) {
@@ -694,6 +733,19 @@ bool build_tc_supported(int64_t V, int64_t D, int64_t Dr, const void* E, const v
 
 mole_status build_tc(const void* E, const void* W1, const void* W2, int64_t V, int64_t D, int N, int64_t Dr,
                      int act, void* lut, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  return build_tc_any(E, W1, W2, V, D, N, Dr, act, lut, nullptr, nullptr, ws, ws_bytes, stream);
+}
+
+mole_status build_tc_nf3(const void* E, const void* W1, const void* W2, int64_t V, int64_t D, int N, int64_t Dr,
+                         int act, uint8_t* codes, uint16_t* scales, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  return build_tc_any(E, W1, W2, V, D, N, Dr, act, nullptr, codes, scales, ws, ws_bytes, stream);
+}
+
+// The build's two GEMMs per group of experts; the second writes either the
+// bf16 table (lut) or, quantising in its epilogue, the NF3 codes and scales.
+mole_status build_tc_any(const void* E, const void* W1, const void* W2, int64_t V, int64_t D, int N, int64_t Dr,
+                         int act, void* lut, uint8_t* codes, uint16_t* scales, void* ws, size_t ws_bytes,
+                         cudaStream_t stream) {
   const size_t per_expert = (size_t)V * Dr * 2;
   const int group = (int)std::min<size_t>((size_t)N, ws_bytes / per_expert);
   if (group < 1) return MOLE_ERR_WORKSPACE;
@@ -737,9 +789,17 @@ mole_status build_tc(const void* E, const void* W1, const void* W2, int64_t V, i
     p2.K = (int)Dr;
     p2.a_batched = 1;
     p2.act = MOLE_ACT_IDENTITY;
-    p2.C = L + (int64_t)e0 * D;
-    p2.ldc = (int64_t)N * D;
-    p2.c_estride = D;
+    if (codes != nullptr) {
+      const int64_t nb = D / 64;  // NF3 blocks per row
+      p2.codes = codes + (int64_t)e0 * nb * 24;
+      p2.scales = scales + (int64_t)e0 * nb;
+      p2.q_row = (int64_t)N * nb;
+      p2.q_e = nb;
+    } else {
+      p2.C = L + (int64_t)e0 * D;
+      p2.ldc = (int64_t)N * D;
+      p2.c_estride = D;
+    }
     p2.m_blocks = (int)((V + mtile - 1) / mtile);
     p2.n_blocks = (int)((D + BN - 1) / BN);
     p2.tiles = (int64_t)g * p2.m_blocks * p2.n_blocks;

@@ -713,34 +713,13 @@ __global__ void __launch_bounds__(256) nf3_quantize_kernel(const uint16_t* __res
     xw[4 * i + 2] = v.z;
     xw[4 * i + 3] = v.w;
   }
-  float amax = 0.f;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(xw[i])), fabsf(bf16_hi(xw[i]))));
-  const __half s16 = __float2half_rn(fminf(amax, 65504.f));
-  const float sc = __half2float(s16);
-  const float mid[7] = {MOLE_NF3_MIDPOINTS};
-  uint32_t packed[6] = {0u, 0u, 0u, 0u, 0u, 0u};
-#pragma unroll
-  for (int e = 0; e < 64; ++e) {
-    const float x = (e & 1) ? bf16_hi(xw[e >> 1]) : bf16_lo(xw[e >> 1]);
-    uint32_t c;
-    if (sc == 0.f) {
-      c = kNf3ZeroCode;
-    } else {
-      const float y = __fdiv_rn(x, sc);
-      c = 0;
-#pragma unroll
-      for (int k = 0; k < 7; ++k) c += (y > mid[k]) ? 1u : 0u;
-    }
-    const int bit = 3 * e;
-    packed[bit >> 5] |= c << (bit & 31);
-    if ((bit & 31) > 29) packed[(bit >> 5) + 1] |= c >> (32 - (bit & 31));
-  }
+  uint32_t packed[6];
+  const uint16_t s16 = nf3_quantize_block(xw, packed);
   uint2* dst = reinterpret_cast<uint2*>(codes + blk * 24);
   dst[0] = make_uint2(packed[0], packed[1]);
   dst[1] = make_uint2(packed[2], packed[3]);
   dst[2] = make_uint2(packed[4], packed[5]);
-  scales[blk] = __half_as_ushort(s16);
+  scales[blk] = s16;
 }
 
 mole_status nf3_quantize_launch(const void* lut, int64_t V, int N, int64_t D, uint8_t* codes,

@@ -7,6 +7,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "nf3.cuh"
 
 namespace mole {
 namespace {
@@ -17,12 +18,6 @@ constexpr int kTileMax = 16;  // rows of the m16n8k16 router MMA
 
 enum TableKind { kTableBf16 = 0, kTableF32 = 1, kTableNf3 = 2 };
 
-// ---- NF3 level table (NormalFloat k=3 levels, QLoRA construction, rounded to
-// fp16; ascending, index 3 is 0.0) and the fp32 midpoints of adjacent levels.
-constexpr uint16_t kNf3Levels[8] = {0xbc00, 0xb848, 0xb3e7, 0x0000, 0x31de, 0x361d, 0x38fc, 0x3c00};
-#define MOLE_NF3_MIDPOINTS -0x1.89p-1f, -0x1.907p-2f, -0x1.f9cp-4f, 0x1.778p-4f, 0x1.218p-2f, 0x1.015p-1f, 0x1.9f8p-1f
-constexpr float kNf3Mid[7] = {MOLE_NF3_MIDPOINTS};
-constexpr int kNf3ZeroCode = 3;
 
 // Byte planes of the fp16 levels, for prmt lookups: plane[k] holds byte k of
 // level k (low bytes in kLoBytes*, high bytes in kHiBytes*).

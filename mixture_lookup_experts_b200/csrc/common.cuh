@@ -144,6 +144,9 @@ bool build_tc_supported(int64_t V, int64_t D, int64_t Dr, const void* E, const v
                         const void* W2, const void* lut, const void* ws);
 mole_status build_tc(const void* E, const void* W1, const void* W2, int64_t V, int64_t D, int N,
                      int64_t Dr, int act, void* lut, void* ws, size_t ws_bytes, cudaStream_t stream);
+// The build with the NF3 quantiser in the second GEMM's epilogue (no bf16 table).
+mole_status build_tc_nf3(const void* E, const void* W1, const void* W2, int64_t V, int64_t D, int N, int64_t Dr,
+                         int act, uint8_t* codes, uint16_t* scales, void* ws, size_t ws_bytes, cudaStream_t stream);
 
 // Shared-expert FFN on the tensor cores (build_tc.cu): out = act(h . W1s) . W2s
 // + add0 + add1 (fp32), the hidden activation rounded to bf16 in `ws`.

@@ -53,6 +53,7 @@ SIGNATURES = {
     "mole_shared_ffn": ([_P, _P, _P, _I64, _I64, _I64, _I, _P, _P, _P, _P, _SZ, _P], _I),
     "mole_ffn_block_workspace": ([_I64, _I64, _I64], _SZ),
     "mole_ffn_block": ([_P, _I64, _P, _SZ, _P, _P, _P, _I64, _I32, _P, _P, _I64, _I64, _I, _P, _P, _P, _SZ, _P], _I),
+    "mole_build_lut_nf3": ([_P, _P, _P, _I64, _I64, _I32, _I64, _I, _P, _P, _P, _SZ, _P], _I),
     "mole_nf3_levels": ([_P], None),
     "mole_nf3_midpoints": ([_P], None),
     "mole_gather_plan": ([_P, _I64, _I64, _P, _P, _P, _P], _I),
@@ -233,6 +234,26 @@ def mole_quantize_lut_nf3(lut: torch.Tensor, codes: torch.Tensor | None = None,
         scales = torch.empty((V, N, D // 64), dtype=torch.float16, device=lut.device)
     _ok(lib.mole_quantize_lut_nf3(_ptr(lut), V, N, D, _ptr(codes), _ptr(scales), _stream(stream)),
         "mole_quantize_lut_nf3")
+    return codes, scales
+
+
+def mole_build_lut_nf3(embed: torch.Tensor, W1: torch.Tensor, W2: torch.Tensor, act: str = "gelu",
+                       codes: torch.Tensor | None = None, scales: torch.Tensor | None = None,
+                       workspace: torch.Tensor | None = None, stream=None):
+    """The table build with the NF3 quantiser in its epilogue: codes
+    [V, N, D/64, 24] uint8 and fp16 scales [V, N, D/64] (see mole.h)."""
+    _contig(embed, W1, W2, codes, scales, workspace)
+    V, D = embed.shape
+    N, _, Dr = W1.shape
+    if codes is None:
+        codes = torch.empty((V, N, D // 64, 24), dtype=torch.uint8, device=embed.device)
+    if scales is None:
+        scales = torch.empty((V, N, D // 64), dtype=torch.float16, device=embed.device)
+    if workspace is None:
+        workspace = torch.empty(mole_build_lut_workspace(V, D, N, Dr, torch.bfloat16, 0), dtype=torch.uint8,
+                                device=embed.device)
+    _ok(lib.mole_build_lut_nf3(_ptr(embed), _ptr(W1), _ptr(W2), V, D, N, Dr, ACT[act], _ptr(codes), _ptr(scales),
+                               _ptr(workspace), workspace.numel(), _stream(stream)), "mole_build_lut_nf3")
     return codes, scales
 
 

@@ -176,3 +176,18 @@ def test_ffn_checks(mole):
     if not torch.cuda.is_available():
         assert lib.mole_shared_ffn(P, P, P, 5, 64, 64, 0, None, None, P, P, ws, None) == 8
         assert blk(P, 5, P, gws, P, P, P, 10, 4, P, P, 64, 64, 0, None, P, P, fws, None) == 8
+
+
+def test_build_nf3_checks(mole):
+    import torch
+    lib = mole.lib
+    P = 0x100000
+    ws = mole.mole_build_lut_workspace(10, 64, 2, 64, torch.bfloat16, 1)
+    f = lib.mole_build_lut_nf3
+    assert f(P, P, P, 10, 64, 2, 64, 9, P, P, P, ws, None) == 1       # bad act
+    assert f(P, P, P, 10, 96, 2, 64, 0, P, P, P, ws, None) == 3       # D % 64
+    assert f(P, P, P, 10, 64, 2, 64, 0, P, P, P, ws - 1, None) == 4   # workspace
+    assert f(P, P, P, 10, 64, 2, 64, 0, P + 4, P, P, ws, None) == 2   # codes misaligned
+    assert f(P, P, P, 10, 64, 2, 64, 0, None, P, P, ws, None) == 1    # no codes
+    if not torch.cuda.is_available():
+        assert f(P, P, P, 10, 64, 2, 64, 0, P, P, P, ws, None) == 8

@@ -152,3 +152,51 @@ def test_build_full_size_sampled_rows(mole, oracle_mod, shape_name, n_rows):
     _check(lut[torch.from_numpy(rows).cuda()], ref, allow)
     del E, W1, W2, lut
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("V,D,N,Dr,act,per_launch", [
+    (300, 128, 3, 256, "gelu", 0),     # ragged M; 2 blocks per row
+    (1000, 256, 2, 512, "gelu", 1),    # one expert per launch
+    (129, 64, 4, 192, "relu", 0),      # one block per row, partial N tile in GEMM1
+    (513, 448, 3, 320, "gelu", 2),     # N tails; 7 blocks per row
+    (256, 512, 2, 128, "silu", 0),
+])
+def test_build_nf3_equals_build_then_quantize(mole, oracle_mod, V, D, N, Dr, act, per_launch):
+    """The quantising epilogue gives the codes and scales of mole_build_lut
+    followed by mole_quantize_lut_nf3, bit for bit; the table it stands for
+    still meets the build tolerance against the oracle once dequantised."""
+    _, E, W1, W2 = _weights(V, D, N, Dr, "bf16", 40 + V)
+    ws = torch.empty(mole.mole_build_lut_workspace(V, D, N, Dr, torch.bfloat16, per_launch), dtype=torch.uint8,
+                     device="cuda")
+    codes, scales = mole.mole_build_lut_nf3(dev(E), dev(W1), dev(W2), act, workspace=ws)
+    assert mole.mole_check() == 0
+    lut = mole.mole_build_lut(dev(E), dev(W1), dev(W2), act)
+    c2, s2 = mole.mole_quantize_lut_nf3(lut)
+    assert mole.mole_check() == 0
+    assert torch.equal(codes, c2)
+    assert torch.equal(scales.view(torch.int16), s2.view(torch.int16))
+    # the codes are also the oracle quantiser's of that table
+    ref_codes, ref_scales = oracle_mod.quantize_nf3(host_bits(lut))
+    np.testing.assert_array_equal(codes.cpu().numpy(), ref_codes)
+    np.testing.assert_array_equal(host_bits(scales), ref_scales)
+
+
+def test_build_nf3_full_size_rows(mole, oracle_mod):
+    """410M-shaped layer (V = 50304, D = 1024, N = 16, Dr = 4096): the fused
+    NF3 build equals build + quantise on sampled rows, bit for bit."""
+    shape = inputs.SHAPES["410m"]
+    V, D, N, Dr = shape.V, shape.D, shape.N, shape.Dr
+    g = torch.Generator(device="cuda")
+    g.manual_seed(shape.seed + 3)
+    E = (torch.randn((V, D), generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+    W1 = (torch.randn((N, D, Dr), generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+    W2 = (torch.randn((N, Dr, D), generator=g, device="cuda") * 0.02).to(torch.bfloat16)
+    codes, scales = mole.mole_build_lut_nf3(E, W1, W2)
+    assert mole.mole_check() == 0
+    rows = torch.tensor([0, 1, 255, 256, 257, 12345, V - 2, V - 1], device="cuda")
+    lut = mole.mole_build_lut(E, W1, W2)
+    c2, s2 = mole.mole_quantize_lut_nf3(lut[rows].contiguous())
+    assert torch.equal(codes[rows], c2)
+    assert torch.equal(scales[rows].view(torch.int16), s2.view(torch.int16))
+    del E, W1, W2, codes, scales, lut
+    torch.cuda.empty_cache()
