@@ -48,7 +48,8 @@ METRIC = "MoLE lookup-combine tokens/s & HBM GB/s vs 8 TB/s; LUT build TFLOP/s"
 UNIT = "tokens/s"
 KERNEL_SOURCES = ["mixture_lookup_experts_b200/csrc/combine.cu", "mixture_lookup_experts_b200/csrc/grouped.cu",
                   "mixture_lookup_experts_b200/csrc/router_tc.cu", "mixture_lookup_experts_b200/csrc/combine_common.cuh",
-                  "mixture_lookup_experts_b200/csrc/common.cuh", "mixture_lookup_experts_b200/csrc/nf3.cuh"]
+                  "mixture_lookup_experts_b200/csrc/common.cuh", "mixture_lookup_experts_b200/csrc/nf3.cuh",
+                  "mixture_lookup_experts_b200/csrc/groups.cuh"]
 PROFILE_SUMMARY = {"grouped": "profiles/combine_grouped_bf16_1b_T16384_zipf.md",
                    "plain": "profiles/combine_bf16_1b_T16384_zipf.md"}
 KERNELS = {
@@ -76,6 +77,8 @@ def parse_args():
     ap.add_argument("--no-offload", action="store_true", help="skip the host-resident (offloaded) table leg")
     ap.add_argument("--no-decode", action="store_true", help="skip the small-batch (decode) sweeps")
     ap.add_argument("--no-ffn", action="store_true", help="skip the FFN-block leg")
+    ap.add_argument("--no-train", action="store_true", help="skip the training-step leg")
+    ap.add_argument("--train-only", action="store_true", help="run only the training-step leg")
     ap.add_argument("--ffn-only", action="store_true", help="run only the FFN-block leg")
     ap.add_argument("--decode-only", action="store_true", help="run only the small-batch (decode) sweeps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -333,6 +336,17 @@ def main():
             dist.destroy_process_group()
         return
 
+    if args.train_only:
+        _, bf16_peak, bf16_sust, _ = measured_peaks()
+        g = torch.Generator(device=dev)
+        g.manual_seed(inputs.SHAPES["1b"].seed)
+        res = train_leg(mole, np.random.default_rng(7), g, dev, stream, max(3, args.warmup), (bf16_peak, bf16_sust))
+        if rank == 0:
+            print(json.dumps({"train": res}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return
+
     if args.ffn_only:
         shape = inputs.SHAPES["1b"]
         g = torch.Generator(device=dev)
@@ -475,6 +489,8 @@ def main():
         torch.cuda.empty_cache()
         if not args.no_decode:
             line["decode"] = decode_leg(mole, dev, stream)
+        if not args.no_train:
+            line["train"] = train_leg(mole, rng, g, dev, stream, W, (bf16_peak, bf16_sust))
         line["build"] = build_leg(mole, dev, stream, bf16_peak, bf16_sust, peak_kind)
 
     if rank == 0 and not args.no_cpu_baseline:
@@ -829,6 +845,56 @@ def ffn_leg(mole, luts, routers, rng, g, dev, stream, W, peaks):
     })
     del W1s, W2s, h, res, out, mix, ws, groups
     return res_line
+
+
+def train_leg(mole, rng, g, dev, stream, W, peaks):
+    """One MoLE layer's training step at the 1B shape, T = 4096 Zipf tokens
+    (§8(f) rank 4): the forward evaluates the routed experts on the batch's
+    distinct ids only (tcgen05 build GEMMs), then the combine; the backward
+    (gate / router gradients, per-id dL/dY, cuBLAS GEMMs for the experts)."""
+    import torch
+    shape = inputs.SHAPES["1b"]
+    V, D, N, Dr, T = shape.V, shape.D, shape.N, shape.Dr, 4096
+    bf16_peak, _ = peaks
+    rnd = lambda *sz, sd=0.02: (torch.randn(sz, generator=g, device=dev) * sd).to(torch.bfloat16)
+    E, W1, W2, Wr, h = rnd(V, D), rnd(N, D, Dr), rnd(N, Dr, D), rnd(D, N), rnd(T, D, sd=1.0)
+    ids = torch.from_numpy(inputs.draw_ids(rng, T, V, "zipf")).to(dev)
+    groups = mole.mole_token_groups_build(ids, V, N, stream=stream)
+    out = torch.empty((T, D), dtype=torch.float32, device=dev)
+    cache = torch.empty(mole.mole_train_cache_bytes(T, V, N, D, Dr), dtype=torch.uint8, device=dev)
+    dout = torch.randn((T, D), generator=g, device=dev)
+    z = lambda *sz: torch.zeros(sz, dtype=torch.float32, device=dev)
+    grads = dict(dh=z(T, D), dWr=z(D, N), dE=z(V, D), dW1=z(N, D, Dr), dW2=z(N, Dr, D))
+    U = [0]
+
+    def fwd(i):
+        _, _, U[0] = mole.mole_train_forward(ids, groups, h, Wr, E, W1, W2, out=out, cache=cache, stream=stream)
+
+    def bwd(i):
+        mole.mole_train_backward(ids, groups, h, Wr, E, W1, W2, dout, cache, U[0], stream=stream, **grads)
+
+    for i in range(max(W, 3)):
+        fwd(i)
+        bwd(i)
+    n = 5
+    f_ms = time_block(fwd, n, stream) / n
+    b_ms = time_block(bwd, n, stream) / n
+    assert mole.mole_check(stream) == 0
+    flops_f = 4.0 * U[0] * D * Dr * N
+    flops_b = 8.0 * U[0] * D * Dr * N
+    res = {"workload": f"1B-shaped MoLE layer training step: T={T} Zipf tokens, {U[0]} distinct ids, N={N} experts "
+                       f"{D}x{Dr} GELU FFN, bf16 weights, fp32 gradients",
+           "distinct_ids": U[0], "forward_ms": f_ms, "backward_ms": b_ms,
+           "tokens_per_s": T / ((f_ms + b_ms) / 1e3),
+           "forward_expert_tflops": flops_f / (f_ms / 1e3) / 1e12,
+           "backward_expert_tflops": flops_b / (b_ms / 1e3) / 1e12,
+           "forward_frac_of_bf16_peak": flops_f / (f_ms / 1e3) / 1e12 / bf16_peak,
+           "expert_flops_saved_vs_per_token": T / max(U[0], 1),
+           "note": "forward: the table build restricted to the batch's distinct embedding rows (tcgen05) + the "
+                   "grouped combine; the forward reads the distinct-id count back to the host (one sync); "
+                   "backward GEMMs in cuBLAS"}
+    del E, W1, W2, cache, grads
+    return res
 
 
 def graph_pass_us(passes, stream, dev, replays=60):

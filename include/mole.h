@@ -319,6 +319,50 @@ mole_status mole_ffn_block(const int32_t* ids, int64_t T, const void* groups, si
                            int64_t D, int64_t Ds, mole_act act, const float* residual, float* out,
                            void* workspace, size_t ws_bytes, cudaStream_t stream);
 
+/*
+ * ---- Training: one MoLE layer forward and backward (MoLE page, 训练阶段) ----
+ *
+ * In training the routed experts take the token's embedding row as input and
+ * all N are active, mixed by the router on the previous layer's output h:
+ *     out[t] = sum_j softmax(h[t] . Wr)_j f_j(E[ids[t]]),
+ *     f_j(x) = act(x . W1[j]) . W2[j]   (hidden activation rounded to bf16)
+ * A routed expert's output depends only on the token id, so the forward
+ * evaluates the experts on the batch's distinct ids only (the table build on
+ * those embedding rows, tcgen05 GEMMs) and mixes them with the combine
+ * kernels: `out` equals mole_lookup_combine over a table built by
+ * mole_build_lut, bit for bit.  The grouping (`groups`, from
+ * mole_token_groups_build with the same ids, T, V and N) supplies the distinct
+ * ids.  The forward reads their count back to the host (one stream
+ * synchronisation) and returns it in *n_distinct; the backward takes it back.
+ *
+ * mole_train_backward adds (+=, fp32) the gradients of L = sum(out * dout)
+ * (dout [T, D] fp32) to dh [T, D], dWr [D, N], dE [V, D] (the batch's rows
+ * only), dW1 [N, D, Dr] and dW2 [N, Dr, D]; any of them may be NULL.  The
+ * backward GEMMs (bf16 operands, fp32 accumulation) run in cuBLAS, whose
+ * handle (created on a device's first backward call) holds cuBLAS's own device
+ * memory; its operands dL/dY and dL/dpre are rounded to bf16 from fp32.  The
+ * bf16 rounding of the hidden activation counts as identity in the backward.
+ * Tokens with an id outside [0, V) get NaN outputs (MOLE_ERR_INDEX from
+ * mole_check) and contribute no gradient.
+ *
+ *   h [T, D] bf16, Wr [D, N] bf16, E [V, D] bf16, W1 [N, D, Dr] bf16,
+ *   W2 [N, Dr, D] bf16; out [T, D] fp32.  D % 64 == 0, Dr % 64 == 0, N <= 32,
+ *   16-byte aligned pointers.  `cache` (device, 16-byte aligned) carries the
+ *   forward's intermediates to the backward: at least
+ *   mole_train_cache_bytes(T, V, N, D, Dr) bytes (room for min(T, V) distinct
+ *   ids), not to be reused between a step's forward and backward.
+ */
+size_t mole_train_cache_bytes(int64_t T, int64_t V, int32_t N, int64_t D, int64_t Dr);
+mole_status mole_train_forward(const int32_t* ids, int64_t T, const void* groups, size_t groups_bytes,
+                               const void* h, const void* Wr, const void* E, const void* W1, const void* W2,
+                               int64_t V, int32_t N, int64_t D, int64_t Dr, mole_act act, float* out, void* cache,
+                               size_t cache_bytes, int32_t* n_distinct, cudaStream_t stream);
+mole_status mole_train_backward(const int32_t* ids, int64_t T, const void* groups, size_t groups_bytes,
+                                const void* h, const void* Wr, const void* E, const void* W1, const void* W2,
+                                int64_t V, int32_t N, int64_t D, int64_t Dr, mole_act act, const float* dout,
+                                void* cache, size_t cache_bytes, int32_t n_distinct, float* dh, float* dWr,
+                                float* dE, float* dW1, float* dW2, cudaStream_t stream);
+
 /* The 8 NF3 levels as fp16 bit patterns (ascending; index 3 is 0.0) and the 7
  * fp32 decision midpoints.  Host-only; no device work. */
 void mole_nf3_levels(uint16_t levels_f16[8]);

@@ -335,3 +335,62 @@ extern "C" mole_status mole_build_lut_nf3(const void* embed, const void* W1, con
   if (!mole::build_tc_supported(V, D, Dr, embed, W1, W2, workspace, workspace)) return MOLE_ERR_UNSUPPORTED;
   return mole::build_tc_nf3(embed, W1, W2, V, D, N, Dr, (int)act, codes, scales, workspace, ws_bytes, stream);
 }
+
+extern "C" size_t mole_train_cache_bytes(int64_t T, int64_t V, int32_t N, int64_t D, int64_t Dr) {
+  if (T <= 0 || V <= 0 || N <= 0 || N > 32 || D <= 0 || Dr <= 0) return 0;
+  return mole::train_cache_bytes(T, V, N, D, Dr);
+}
+
+namespace {
+mole_status check_train(int64_t T, const void* groups, size_t gbytes, const void* h, const void* Wr, const void* W1,
+                        const void* W2, int64_t V, int32_t N, int64_t D, int64_t Dr, mole_act act, const void* cache,
+                        size_t cbytes) {
+  if (!valid_act(act) || T < 0 || V <= 0 || V > INT32_MAX || N <= 0 || D <= 0 || Dr <= 0) return MOLE_ERR_ARG;
+  if (T > 0 && (!h || !Wr || !W1 || !W2)) return MOLE_ERR_ARG;
+  if (N > 32 || D % 64 != 0 || Dr % 64 != 0 || T > INT32_MAX || D > INT32_MAX || Dr > INT32_MAX)
+    return MOLE_ERR_UNSUPPORTED;
+  mole_status st = check_groups(T, N, groups, gbytes);
+  if (st != MOLE_OK || T == 0) return st;
+  if (!cache || cbytes < mole::train_cache_bytes(T, V, N, D, Dr)) return MOLE_ERR_WORKSPACE;
+  if (!mole::aligned16(h) || !mole::aligned16(Wr) || !mole::aligned16(W1) || !mole::aligned16(W2) ||
+      !mole::aligned16(cache))
+    return MOLE_ERR_ALIGN;
+  return MOLE_OK;
+}
+}  // namespace
+
+extern "C" mole_status mole_train_forward(const int32_t* ids, int64_t T, const void* groups, size_t groups_bytes,
+                                          const void* h, const void* Wr, const void* E, const void* W1,
+                                          const void* W2, int64_t V, int32_t N, int64_t D, int64_t Dr, mole_act act,
+                                          float* out, void* cache, size_t cache_bytes, int32_t* n_distinct,
+                                          cudaStream_t stream) {
+  mole_status st = check_train(T, groups, groups_bytes, h, Wr, W1, W2, V, N, D, Dr, act, cache, cache_bytes);
+  if (st != MOLE_OK) return st;
+  if (n_distinct) *n_distinct = 0;
+  if (T == 0) return MOLE_OK;
+  if (!ids || !E || !out || !n_distinct) return MOLE_ERR_ARG;
+  if (!mole::aligned16(E) || !mole::aligned16(out)) return MOLE_ERR_ALIGN;
+  st = check_device();
+  if (st != MOLE_OK) return st;
+  if (!mole::build_tc_supported(std::min(T, V), D, Dr, E, W1, W2, cache, cache)) return MOLE_ERR_UNSUPPORTED;
+  return mole::train_forward(groups, groups_bytes, T, h, Wr, E, W1, W2, V, N, D, Dr, (int)act, out, cache,
+                             cache_bytes, n_distinct, stream);
+}
+
+extern "C" mole_status mole_train_backward(const int32_t* ids, int64_t T, const void* groups, size_t groups_bytes,
+                                           const void* h, const void* Wr, const void* E, const void* W1,
+                                           const void* W2, int64_t V, int32_t N, int64_t D, int64_t Dr, mole_act act,
+                                           const float* dout, void* cache, size_t cache_bytes, int32_t n_distinct,
+                                           float* dh, float* dWr, float* dE, float* dW1, float* dW2,
+                                           cudaStream_t stream) {
+  (void)ids;
+  (void)E;
+  mole_status st = check_train(T, groups, groups_bytes, h, Wr, W1, W2, V, N, D, Dr, act, cache, cache_bytes);
+  if (st != MOLE_OK || T == 0) return st;
+  if (!dout) return MOLE_ERR_ARG;
+  if (n_distinct < 0 || n_distinct > std::min(T, V)) return MOLE_ERR_ARG;
+  st = check_device();
+  if (st != MOLE_OK) return st;
+  return mole::train_backward(groups, groups_bytes, T, h, Wr, W1, W2, V, N, D, Dr, (int)act, dout, cache, cache_bytes,
+                              n_distinct, dh, dWr, dE, dW1, dW2, stream);
+}

@@ -72,6 +72,10 @@ struct Params {
   uint8_t* codes;
   uint16_t* scales;
   int64_t q_row, q_e;
+  // also the fp32 pre-activation of the bf16 output (training): element
+  // (e, m, n) at pre + e * pre_estride + m * ldc + n
+  float* pre;
+  int64_t pre_estride;
 };
 
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
@@ -225,10 +229,18 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, uint32_t taddr, i
     uint32_t r[32];
     tmem_ld32(taddr + chunk * 32, r);
     if (m < p.M) {
-      if (p.Cf != nullptr)
+      if (p.Cf != nullptr) {
         store_chunk_f32(r, p, (int64_t)m * p.ldc + col0);
-      else
+      } else {
+        if (p.pre != nullptr) {
+          float4* dst = reinterpret_cast<float4*>(p.pre + (int64_t)e * p.pre_estride + (int64_t)m * p.ldc + col0);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            dst[q] = make_float4(__uint_as_float(r[4 * q]), __uint_as_float(r[4 * q + 1]),
+                                 __uint_as_float(r[4 * q + 2]), __uint_as_float(r[4 * q + 3]));
+        }
         store_chunk_act(p.act, r, crow + col0);
+      }
     }
   }
 }
@@ -734,6 +746,54 @@ bool build_tc_supported(int64_t V, int64_t D, int64_t Dr, const void* E, const v
 mole_status build_tc(const void* E, const void* W1, const void* W2, int64_t V, int64_t D, int N, int64_t Dr,
                      int act, void* lut, void* ws, size_t ws_bytes, cudaStream_t stream) {
   return build_tc_any(E, W1, W2, V, D, N, Dr, act, lut, nullptr, nullptr, ws, ws_bytes, stream);
+}
+
+// Training forward of the routed experts on the rows of Eu [M, D]: for every
+// expert e, pre[e] = Eu . W1[e] (fp32), H[e] = act(pre[e]) (bf16), and
+// Y[:, e, :] = H[e] . W2[e] (bf16, rows of N * D).  H and pre are [N, ld_rows,
+// Dr]: expert e's matrix starts ld_rows * Dr elements after expert e-1's.
+mole_status train_experts_tc(const void* Eu, const void* W1, const void* W2, int64_t M, int64_t ld_rows, int64_t D,
+                             int N, int64_t Dr, int act, uint16_t* H, float* pre, uint16_t* Y, cudaStream_t stream) {
+  unsigned* err = error_word();
+  if (!err) return MOLE_ERR_CUDA;
+  const bool pair_tiles = M >= 2 * BM;
+  const int mtile = pair_tiles ? 2 * BM : BM;
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, Eu, D, M, 1, D * 2, M * D * 2, BM)) return MOLE_ERR_CUDA;
+  if (!make_map(&mb, W1, Dr, D, N, Dr * 2, D * Dr * 2, BK)) return MOLE_ERR_CUDA;
+  Params p1{};
+  p1.M = (int)M;
+  p1.N = (int)Dr;
+  p1.K = (int)D;
+  p1.a_batched = 0;
+  p1.act = act;
+  p1.C = H;
+  p1.ldc = Dr;
+  p1.c_estride = ld_rows * Dr;
+  p1.pre = pre;
+  p1.pre_estride = ld_rows * Dr;
+  p1.m_blocks = (int)((M + mtile - 1) / mtile);
+  p1.n_blocks = (int)((Dr + BN - 1) / BN);
+  p1.tiles = (int64_t)N * p1.m_blocks * p1.n_blocks;
+  p1.err = err;
+  mole_status st = launch_gemm(ma, mb, p1, pair_tiles, stream);
+  if (st != MOLE_OK) return st;
+  if (!make_map(&ma, H, Dr, M, N, Dr * 2, ld_rows * Dr * 2, BM)) return MOLE_ERR_CUDA;
+  if (!make_map(&mb, W2, D, Dr, N, D * 2, Dr * D * 2, BK)) return MOLE_ERR_CUDA;
+  Params p2{};
+  p2.M = (int)M;
+  p2.N = (int)D;
+  p2.K = (int)Dr;
+  p2.a_batched = 1;
+  p2.act = MOLE_ACT_IDENTITY;
+  p2.C = Y;
+  p2.ldc = (int64_t)N * D;
+  p2.c_estride = D;
+  p2.m_blocks = (int)((M + mtile - 1) / mtile);
+  p2.n_blocks = (int)((D + BN - 1) / BN);
+  p2.tiles = (int64_t)N * p2.m_blocks * p2.n_blocks;
+  p2.err = err;
+  return launch_gemm(ma, mb, p2, pair_tiles, stream);
 }
 
 mole_status build_tc_nf3(const void* E, const void* W1, const void* W2, int64_t V, int64_t D, int N, int64_t Dr,

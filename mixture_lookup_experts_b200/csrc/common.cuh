@@ -144,6 +144,9 @@ bool build_tc_supported(int64_t V, int64_t D, int64_t Dr, const void* E, const v
                         const void* W2, const void* lut, const void* ws);
 mole_status build_tc(const void* E, const void* W1, const void* W2, int64_t V, int64_t D, int N,
                      int64_t Dr, int act, void* lut, void* ws, size_t ws_bytes, cudaStream_t stream);
+// The routed experts of a training step on the rows of Eu (build_tc.cu).
+mole_status train_experts_tc(const void* Eu, const void* W1, const void* W2, int64_t M, int64_t ld_rows, int64_t D,
+                             int N, int64_t Dr, int act, uint16_t* H, float* pre, uint16_t* Y, cudaStream_t stream);
 // The build with the NF3 quantiser in the second GEMM's epilogue (no bf16 table).
 mole_status build_tc_nf3(const void* E, const void* W1, const void* W2, int64_t V, int64_t D, int N, int64_t Dr,
                          int act, uint8_t* codes, uint16_t* scales, void* ws, size_t ws_bytes, cudaStream_t stream);
@@ -192,6 +195,21 @@ mole_status offload_stage(const void* buf, size_t bytes, int64_t T, const void* 
 mole_status combine_offload(const void* buf, size_t bytes, int64_t T, const void* h, const void* Wr,
                             const void* staging, size_t staging_bytes, int64_t V, int N, int D, bool bf16_inputs,
                             bool nf3, float* out, cudaStream_t stream);
+// The batch's distinct-id count (device int) and the rows of a table for its
+// distinct ids by dense index (grouped.cu; training).
+mole_status token_groups_count(const void* buf, size_t bytes, int64_t T, int N, int* dst, cudaStream_t stream);
+mole_status gather_rows_by_uid(const void* buf, size_t bytes, int64_t T, int N, const void* table, int64_t row_bytes,
+                               int64_t V, void* dst, int64_t cap, cudaStream_t stream);
+// Training (train.cu): the cache size, the forward (experts on the batch's
+// distinct ids, then the combine) and the backward.
+size_t train_cache_bytes(int64_t T, int64_t V, int N, int64_t D, int64_t Dr);
+mole_status train_forward(const void* groups, size_t gbytes, int64_t T, const void* h, const void* Wr, const void* E,
+                          const void* W1, const void* W2, int64_t V, int N, int64_t D, int64_t Dr, int act,
+                          float* out, void* cache, size_t cbytes, int32_t* n_distinct, cudaStream_t stream);
+mole_status train_backward(const void* groups, size_t gbytes, int64_t T, const void* h, const void* Wr,
+                           const void* W1, const void* W2, int64_t V, int N, int64_t D, int64_t Dr, int act,
+                           const float* dout, void* cache, size_t cbytes, int32_t U, float* dh, float* dWr, float* dE,
+                           float* dW1, float* dW2, cudaStream_t stream);
 void nf3_tables(uint16_t levels[8], float mid[7]);
 mole_status gather_plan_launch(const int32_t* ids, int64_t T, int64_t V, int32_t* uniq,
                                int32_t* n_uniq, int32_t* slot, cudaStream_t stream);

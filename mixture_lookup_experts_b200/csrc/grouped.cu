@@ -35,114 +35,15 @@
 // code, then out = sum over j = 0..N-1, in order, of g_j * x_j with fp32
 // FMAs), so both paths give bit-identical outputs; only the order in which
 // tokens are processed differs.
-#include "combine_common.cuh"
+#include "groups.cuh"
 
 namespace mole {
 namespace {
 
-constexpr int kItemTokens = 16;     // tokens per work item
 constexpr int kPlanThreads = 256;
 constexpr int kPlanMaxGrid = 1024;
 constexpr int64_t kGroupedMinT = 1024;
 constexpr int64_t kGroupedMaxT = kMaxOffloadT;
-
-// Per-CTA totals of step 1: [0] tokens, [n] work items of n tokens (n =
-// 1..kItemTokens), [kAgg] distinct ids.
-constexpr int kAgg = kItemTokens + 1;
-
-// Control words (set to 0xFFFFFFFF when a grouping is built): work items,
-// the three grid-barrier counters, the abort word, the running totals of
-// step 1 (value + 1 = the sum so far), and the fused layer kernel's launch
-// counter.
-enum : int {
-  kCtlItems = 1,
-  kCtlBar = 2,
-  kCtlAbort = 5,
-  kCtlTot = 8,
-  kCtlLaunches = kCtlTot + kAgg + 1,  // 64-bit launch counter of the fused layer kernel (8-byte aligned)
-  kCtlWords = kCtlLaunches + 2
-};
-
-// The grouping of one batch (the caller's buffer, carved by carve_ws).
-struct GroupWs {
-  int* key;       // [hcap] id in the slot, -1 = empty
-  int* cnt;       // [hcap] tokens in the slot minus one
-  unsigned* ctl;  // [kCtlWords]
-  int* off;       // [hcap] first list position of the slot's tokens
-  int* tok_slot;  // [T] slot of token t (-1 for a bad id)
-  int* tok_rank;  // [T] rank of token t in its id's group
-  int* tok_pos;   // [T] list position of token t (-1 for a bad id)
-  int* list;      // [T] tokens grouped by id
-  int4* items;    // [T + T / kItemTokens + 1] {id, first list position, tokens, dense index of the id}
-  int* uid_id;    // [T] the id of each dense index (distinct ids numbered 0..U-1)
-  int* slot_uid;  // [hcap] dense index of the slot's id
-  int* tok_uid;   // [T] dense index of token t's id (-1 for a bad id)
-  float* gates;   // [T][NP] one layer's gates by list position
-  unsigned* tile_flag;  // [ceil(T / 16)] the fused layer kernel's router-tile flags
-  int hcap_log2;
-  size_t clear_bytes;  // key .. ctl .. tile_flag, one contiguous range
-};
-
-int padded_experts(int N) { return N <= 8 ? 8 : N <= 16 ? 16 : 32; }
-
-// Carves the buffer at `base` (nullptr: size query); returns its size.
-size_t carve_ws(void* base, int64_t T, int NP, GroupWs* w) {
-  int lg = 10;
-  while ((int64_t(1) << lg) < 2 * T) ++lg;
-  const int64_t hcap = int64_t(1) << lg;
-  size_t off = 0;
-  auto take = [&off](size_t bytes) {
-    const size_t o = off;
-    off += (bytes + 255) / 256 * 256;
-    return o;
-  };
-  const size_t n_flags = (size_t)((T + 15) / 16);
-  const size_t clear = 8 * (size_t)hcap + 4 * kCtlWords + 4 * n_flags;
-  const size_t o_clear = take(clear);
-  const size_t o_off = take(4 * (size_t)hcap);
-  const size_t o_tslot = take(4 * (size_t)T);
-  const size_t o_trank = take(4 * (size_t)T);
-  const size_t o_tpos = take(4 * (size_t)T);
-  const size_t o_list = take(4 * (size_t)T);
-  const size_t o_items = take(16 * (size_t)(T + T / kItemTokens + 1));
-  const size_t o_uid = take(4 * (size_t)T);
-  const size_t o_suid = take(4 * (size_t)hcap);
-  const size_t o_tuid = take(4 * (size_t)T);
-  const size_t o_gates = take(4 * (size_t)T * NP);
-  if (w != nullptr && base != nullptr) {
-    uint8_t* b = static_cast<uint8_t*>(base);
-    w->key = reinterpret_cast<int*>(b + o_clear);
-    w->cnt = w->key + hcap;
-    w->ctl = reinterpret_cast<unsigned*>(w->cnt + hcap);
-    w->tile_flag = w->ctl + kCtlWords;
-    w->off = reinterpret_cast<int*>(b + o_off);
-    w->tok_slot = reinterpret_cast<int*>(b + o_tslot);
-    w->tok_rank = reinterpret_cast<int*>(b + o_trank);
-    w->tok_pos = reinterpret_cast<int*>(b + o_tpos);
-    w->list = reinterpret_cast<int*>(b + o_list);
-    w->items = reinterpret_cast<int4*>(b + o_items);
-    w->uid_id = reinterpret_cast<int*>(b + o_uid);
-    w->slot_uid = reinterpret_cast<int*>(b + o_suid);
-    w->tok_uid = reinterpret_cast<int*>(b + o_tuid);
-    w->gates = reinterpret_cast<float*>(b + o_gates);
-    w->hcap_log2 = lg;
-    w->clear_bytes = clear;
-  }
-  return off;
-}
-
-__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
-  unsigned v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-__device__ __forceinline__ unsigned ld_relaxed_u32(const unsigned* p) {
-  unsigned v;
-  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
 
 // Grid-wide barrier of a cooperative launch, split in two so that work can
 // run between the arrival and the wait; `counter` starts at 0xFFFFFFFF and
@@ -1678,6 +1579,40 @@ mole_status offload_stage(const void* buf, size_t bytes, int64_t T, const void* 
   const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)kStageCtasPerSm * n_sm));
   stage_rows_kernel<<<grid, kStageThreads, 0, stream>>>(w, a, b, nf3 ? 2 : 1, V, L.rows, n_rows, err);
   return cudaGetLastError() == cudaSuccess ? MOLE_OK : MOLE_ERR_CUDA;
+}
+
+// The batch's distinct-id count into *dst (one device int32; 0 if the
+// grouping was abandoned).
+__global__ void distinct_count_kernel(const GroupWs w, int* dst) {
+  unsigned U = 0;
+  if (ld_relaxed_u32(&w.ctl[kCtlAbort]) == 0xFFFFFFFFu) U = ld_relaxed_u32(&w.ctl[kCtlTot + kAgg]) + 1u;
+  *dst = (int)U;
+}
+
+mole_status token_groups_count(const void* buf, size_t bytes, int64_t T, int N, int* dst, cudaStream_t stream) {
+  GroupWs w{};
+  if (carve_ws(const_cast<void*>(buf), T, padded_experts(N), &w) > bytes) return MOLE_ERR_WORKSPACE;
+  distinct_count_kernel<<<1, 1, 0, stream>>>(w, dst);
+  return cuda_status(cudaGetLastError());
+}
+
+// Row blocks of `table` (row_bytes each, V rows) of the batch's distinct ids
+// into dst at their dense indices (at most cap rows).
+mole_status gather_rows_by_uid(const void* buf, size_t bytes, int64_t T, int N, const void* table, int64_t row_bytes,
+                               int64_t V, void* dst, int64_t cap, cudaStream_t stream) {
+  GroupWs w{};
+  if (carve_ws(const_cast<void*>(buf), T, padded_experts(N), &w) > bytes) return MOLE_ERR_WORKSPACE;
+  StagePlane a{static_cast<const uint8_t*>(table), static_cast<uint8_t*>(dst), row_bytes, 0};
+  a.vec = access_bytes(a.row_bytes, a.src, a.dst);
+  unsigned* err = error_word();
+  if (!err) return MOLE_ERR_CUDA;
+  const int n_sm = num_sms();
+  if (n_sm <= 0) return MOLE_ERR_NO_DEVICE;
+  const int64_t cpr = (row_bytes / a.vec + kStageThreads - 1) / kStageThreads;
+  const int64_t want = (cap * cpr + kStageUnroll - 1) / kStageUnroll;
+  const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(want, (int64_t)kStageCtasPerSm * n_sm));
+  stage_rows_kernel<<<grid, kStageThreads, 0, stream>>>(w, a, a, 1, V, cap, nullptr, err);
+  return cuda_status(cudaGetLastError());
 }
 
 mole_status combine_offload(const void* buf, size_t bytes, int64_t T, const void* h, const void* Wr,

@@ -1,0 +1,408 @@
+// train.cu -- one MoLE layer in training, forward and backward.  MoLE page,
+// 训练阶段: during training the routed experts take the token's embedding row
+// as input (not the previous layer's output), all N routed experts are
+// active, and the router on the previous layer's output mixes them; the loss
+// is the language-model loss alone.  Because a routed expert's input depends
+// only on the token id, a batch needs the experts evaluated only on its
+// distinct ids (a reading that follows from the page's setup; the page does
+// not state it): the forward is the table build restricted to the batch's
+// distinct embedding rows, then the inference combine over those rows.
+//
+// Forward (cache = what the backward needs; U = the batch's distinct ids):
+//   Eu = E[distinct ids]                                  (row gather)
+//   pre_j = Eu . W1_j, H_j = act(pre_j) (bf16), Y[:, j] = H_j . W2_j
+//                                                         (the build's tcgen05 GEMMs)
+//   out[t] = sum_j g_j(h[t]) Y[u(t), j]                   (the combine kernels)
+// Backward of L with dL/dout = dout (all gradients accumulated, fp32):
+//   g, dg_j = <dout[t], Y[u(t), j]>, dz = g (dg - <g, dg>)
+//   dh[t] += dz[t] . Wr^T,  dWr += h^T dz                 (gate_grad_kernel, dwr_kernel)
+//   dY[u, j] = sum_{t: u(t) = u} g_j[t] dout[t]           (dy_kernel over the grouping's items)
+//   dpre_j = (dY_j . W2_j^T) * act'(pre_j)                (cuBLAS + act_grad_kernel)
+//   dW2_j += H_j^T dY_j,  dW1_j += Eu^T dpre_j,  dE[ids] += sum_j dpre_j . W1_j^T
+//                                                         (cuBLAS, scatter_rows_kernel)
+// The backward GEMMs are plain transposed bf16 GEMMs with fp32 accumulation
+// and run in cuBLAS; their bf16 operands dY and dpre are rounded from fp32.
+#include <cublas_v2.h>
+
+#include "groups.cuh"
+
+namespace mole {
+namespace {
+
+constexpr int kGradThreads = 256;
+constexpr int64_t kCublasWorkspace = int64_t(32) << 20;
+
+// The caller's cache buffer (cap = min(T, V) row capacity).
+struct TrainCache {
+  uint16_t* Eu;   // [cap, D] bf16
+  uint16_t* Y;    // [cap, N, D] bf16
+  uint16_t* H;    // [N, cap, Dr] bf16
+  float* pre;     // [N, cap, Dr] fp32
+  float* g;       // [T, N] gates
+  float* dz;      // [T, N] logit gradients
+  float* dY;      // [cap, N, D] fp32
+  uint16_t* dYb;  // [cap, N, D] bf16
+  uint16_t* dP;   // [N, cap, Dr] bf16: dL/dpre (first dL/dH)
+  float* dEu;     // [cap, D] fp32
+  void* blas_ws;  // cuBLAS workspace
+  int* U;         // one device int
+  size_t total;
+};
+
+size_t carve_cache(void* base, int64_t T, int64_t V, int N, int64_t D, int64_t Dr, TrainCache* c) {
+  const int64_t cap = std::min(T, V);
+  size_t off = 0;
+  auto take = [&off](size_t bytes) {
+    const size_t o = off;
+    off += (bytes + 255) / 256 * 256;
+    return o;
+  };
+  const size_t o_eu = take(2 * (size_t)cap * D);
+  const size_t o_y = take(2 * (size_t)cap * N * D);
+  const size_t o_h = take(2 * (size_t)N * cap * Dr);
+  const size_t o_pre = take(4 * (size_t)N * cap * Dr);
+  const size_t o_g = take(4 * (size_t)T * N);
+  const size_t o_dz = take(4 * (size_t)T * N);
+  const size_t o_dy = take(4 * (size_t)cap * N * D);
+  const size_t o_dyb = take(2 * (size_t)cap * N * D);
+  const size_t o_dp = take(2 * (size_t)N * cap * Dr);
+  const size_t o_deu = take(4 * (size_t)cap * D);
+  const size_t o_ws = take((size_t)kCublasWorkspace);
+  const size_t o_u = take(16);
+  if (c != nullptr && base != nullptr) {
+    uint8_t* b = static_cast<uint8_t*>(base);
+    c->Eu = reinterpret_cast<uint16_t*>(b + o_eu);
+    c->Y = reinterpret_cast<uint16_t*>(b + o_y);
+    c->H = reinterpret_cast<uint16_t*>(b + o_h);
+    c->pre = reinterpret_cast<float*>(b + o_pre);
+    c->g = reinterpret_cast<float*>(b + o_g);
+    c->dz = reinterpret_cast<float*>(b + o_dz);
+    c->dY = reinterpret_cast<float*>(b + o_dy);
+    c->dYb = reinterpret_cast<uint16_t*>(b + o_dyb);
+    c->dP = reinterpret_cast<uint16_t*>(b + o_dp);
+    c->dEu = reinterpret_cast<float*>(b + o_deu);
+    c->blas_ws = b + o_ws;
+    c->U = reinterpret_cast<int*>(b + o_u);
+    c->total = off;
+  }
+  return off;
+}
+
+__device__ __forceinline__ float ld_bf16(const uint16_t* p) { return __uint_as_float((uint32_t)*p << 16); }
+
+// Derivative of the expert activation at the pre-activation u.
+__device__ __forceinline__ float act_grad(int act, float u) {
+  switch (act) {
+    case MOLE_ACT_GELU_ERF: {  // Phi(u) + u phi(u)
+      const float Phi = 0.5f * erfcf(-u * 0.70710678118654752f);
+      const float phi = 0.39894228040143268f * expf(-0.5f * u * u);
+      return Phi + u * phi;
+    }
+    case MOLE_ACT_GELU_TANH: {  // d/du 0.5 u (1 + tanh(c (u + 0.044715 u^3)))
+      const float c = 0.79788456080286536f;
+      const float k = c * (u + 0.044715f * u * u * u);
+      const float th = tanhf(k);
+      return 0.5f * (1.f + th) + 0.5f * u * (1.f - th * th) * c * (1.f + 3.f * 0.044715f * u * u);
+    }
+    case MOLE_ACT_RELU:
+      return u > 0.f ? 1.f : 0.f;
+    case MOLE_ACT_SILU: {
+      const float s = 1.f / (1.f + expf(-u));
+      return s * (1.f + u * (1.f - s));
+    }
+    default:
+      return 1.f;
+  }
+}
+
+// One warp per token: the gates (router logits h[t] . Wr in fp32, softmax),
+// dg_j = <dout[t], Y[u(t), j]>, dz = g (dg - <g, dg>), and dh[t] += dz . Wr^T.
+// Tokens with a bad id (dense index -1) get no gradient.
+template <int NP>
+__global__ void __launch_bounds__(kGradThreads) gate_grad_kernel(const GroupWs w, const uint16_t* __restrict__ h,
+                                                                 const uint16_t* __restrict__ Wr,
+                                                                 const uint16_t* __restrict__ Y,
+                                                                 const float* __restrict__ dout, int64_t T, int N,
+                                                                 int D, float* g_out, float* dz_out, float* dh) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warps = (int64_t)gridDim.x * (kGradThreads / 32);
+  for (int64_t t = (int64_t)blockIdx.x * (kGradThreads / 32) + (threadIdx.x >> 5); t < T; t += warps) {
+    const int u = w.tok_uid[t];
+    if (u < 0) continue;
+    float z[NP], dg[NP];
+#pragma unroll
+    for (int j = 0; j < NP; ++j) z[j] = dg[j] = 0.f;
+    const uint16_t* hr = h + t * D;
+    const float* dr = dout + t * D;
+    const uint16_t* yr = Y + (int64_t)u * N * D;
+    for (int d = lane; d < D; d += 32) {
+      const float hv = ld_bf16(hr + d), dv = dr[d];
+#pragma unroll
+      for (int j = 0; j < NP; ++j)
+        if (j < N) {
+          z[j] = fmaf(hv, ld_bf16(Wr + (int64_t)d * N + j), z[j]);
+          dg[j] = fmaf(dv, ld_bf16(yr + (int64_t)j * D + d), dg[j]);
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < NP; ++j)
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        z[j] += __shfl_xor_sync(0xffffffffu, z[j], o);
+        dg[j] += __shfl_xor_sync(0xffffffffu, dg[j], o);
+      }
+    float m = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < NP; ++j)
+      if (j < N) m = fmaxf(m, z[j]);
+    float sum = 0.f;
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+      z[j] = j < N ? expf(z[j] - m) : 0.f;
+      sum += z[j];
+    }
+    float gdg = 0.f;
+#pragma unroll
+    for (int j = 0; j < NP; ++j) {
+      z[j] /= sum;  // the gate
+      gdg = fmaf(z[j], dg[j], gdg);
+    }
+    float dz[NP];
+#pragma unroll
+    for (int j = 0; j < NP; ++j) dz[j] = z[j] * (dg[j] - gdg);
+    if (lane < N) {
+#pragma unroll
+      for (int j = 0; j < NP; ++j)
+        if (j == lane) {
+          g_out[t * N + j] = z[j];
+          dz_out[t * N + j] = dz[j];
+        }
+    }
+    if (dh != nullptr) {
+      float* o = dh + t * D;
+      for (int d = lane; d < D; d += 32) {
+        float acc = 0.f;
+#pragma unroll
+        for (int j = 0; j < NP; ++j)
+          if (j < N) acc = fmaf(dz[j], ld_bf16(Wr + (int64_t)d * N + j), acc);
+        o[d] += acc;
+      }
+    }
+  }
+}
+
+// dWr[d, j] += sum_t h[t, d] dz[t, j]: a thread per d of its block's 256,
+// over its block's range of tokens; one atomic add per (d, j) per block.
+constexpr int kDwrTokens = 256;
+
+template <int NP>
+__global__ void __launch_bounds__(kGradThreads) dwr_kernel(const GroupWs w, const uint16_t* __restrict__ h,
+                                                           const float* __restrict__ dz, int64_t T, int N, int D,
+                                                           float* dWr) {
+  __shared__ float dzs[kDwrTokens][NP];
+  const int d = blockIdx.x * kGradThreads + threadIdx.x;
+  const int64_t t0 = (int64_t)blockIdx.y * kDwrTokens;
+  const int nt = (int)std::min<int64_t>(kDwrTokens, T - t0);
+  for (int i = threadIdx.x; i < nt * NP; i += kGradThreads) {
+    const int r = i / NP, j = i - r * NP;
+    dzs[r][j] = (j < N && w.tok_uid[t0 + r] >= 0) ? dz[(t0 + r) * N + j] : 0.f;
+  }
+  __syncthreads();
+  if (d >= D) return;
+  float acc[NP];
+#pragma unroll
+  for (int j = 0; j < NP; ++j) acc[j] = 0.f;
+  for (int r = 0; r < nt; ++r) {
+    const float hv = ld_bf16(h + (t0 + r) * D + d);
+#pragma unroll
+    for (int j = 0; j < NP; ++j) acc[j] = fmaf(hv, dzs[r][j], acc[j]);
+  }
+#pragma unroll
+  for (int j = 0; j < NP; ++j)
+    if (j < N) atomicAdd(dWr + (int64_t)d * N + j, acc[j]);
+}
+
+// dY[u, j, :] += sum over the item's tokens of g[t, j] dout[t, :]: one CTA per
+// work item (up to 16 tokens of one id); items of the same id add atomically.
+__global__ void __launch_bounds__(kGradThreads) dy_kernel(const GroupWs w, const float* __restrict__ g,
+                                                          const float* __restrict__ dout, int N, int D, float* dY) {
+  __shared__ int toks[kItemTokens];
+  __shared__ float gs[kItemTokens][32];
+  const int n_items = (int)ld_relaxed_u32(&w.ctl[kCtlItems]);
+  for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+    const int4 rec = w.items[it];  // {id, first list position, tokens, dense index}
+    __syncthreads();
+    if (threadIdx.x < rec.z) toks[threadIdx.x] = w.list[rec.y + threadIdx.x];
+    __syncthreads();
+    for (int i = threadIdx.x; i < rec.z * N; i += kGradThreads) {
+      const int k = i / N, j = i - k * N;
+      gs[k][j] = g[(int64_t)toks[k] * N + j];
+    }
+    __syncthreads();
+    float* dst = dY + (int64_t)rec.w * N * D;
+    for (int e = threadIdx.x; e < N * D; e += kGradThreads) {
+      const int j = e / D, d = e - j * D;
+      float acc = 0.f;
+      for (int k = 0; k < rec.z; ++k) acc = fmaf(gs[k][j], dout[(int64_t)toks[k] * D + d], acc);
+      atomicAdd(dst + e, acc);
+    }
+  }
+}
+
+__global__ void to_bf16_kernel(const float* __restrict__ x, uint16_t* __restrict__ y, int64_t n) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    y[i] = __bfloat16_as_ushort(__float2bfloat16_rn(x[i]));
+}
+
+// dP = bf16(dH * act'(pre)) over the first U rows of each expert's [cap, Dr] block.
+__global__ void act_grad_kernel(uint16_t* dP, const float* __restrict__ pre, int64_t U, int64_t cap, int64_t Dr,
+                                int N, int act) {
+  const int64_t per = U * Dr, n = per * N;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t j = i / per, r = i - j * per;
+    const int64_t k = j * cap * Dr + r;
+    const float dh = ld_bf16(dP + k);
+    dP[k] = __bfloat16_as_ushort(__float2bfloat16_rn(dh * act_grad(act, pre[k])));
+  }
+}
+
+// dE[id(u), :] += dEu[u, :] (each distinct id once).
+__global__ void scatter_rows_kernel(const GroupWs w, const float* __restrict__ dEu, int64_t U, int D, float* dE) {
+  const int64_t n = U * D;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t u = i / D, d = i - u * D;
+    dE[(int64_t)w.uid_id[u] * D + d] += dEu[i];
+  }
+}
+
+unsigned grid_for(int64_t n, int per_block) {
+  const int n_sm = num_sms();
+  return (unsigned)std::max<int64_t>(1, std::min<int64_t>((n + per_block - 1) / per_block, (int64_t)n_sm * 16));
+}
+
+// ---- cuBLAS: one handle per device, bound to the caller's stream and to a
+// workspace in the cache at each call ----
+cublasHandle_t blas_handle() {
+  static cublasHandle_t handles[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (handles[dev] == nullptr && cublasCreate(&handles[dev]) != CUBLAS_STATUS_SUCCESS) handles[dev] = nullptr;
+  return handles[dev];
+}
+
+// Row-major C[M, N] (ldc, stride sC) = alpha op(A)[M, K] op(B)[K, N] + beta C,
+// `batch` times: A, B bf16 (row-major, lda / ldb, strides sA / sB); C fp32 or
+// bf16.  (cuBLAS is column-major: it computes C^T = op(B)^T op(A)^T.)
+bool rm_gemm(cublasHandle_t hb, bool ta, bool tb, int64_t M, int64_t N, int64_t K, const void* A, int64_t lda,
+             int64_t sA, const void* B, int64_t ldb, int64_t sB, float beta, void* C, bool c_f32, int64_t ldc, int64_t sC,
+             int batch) {
+  const float alpha = 1.f;
+  return cublasGemmStridedBatchedEx(hb, tb ? CUBLAS_OP_T : CUBLAS_OP_N, ta ? CUBLAS_OP_T : CUBLAS_OP_N, (int)N,
+                                    (int)M, (int)K, &alpha, B, CUDA_R_16BF, (int)ldb, sB, A, CUDA_R_16BF, (int)lda,
+                                    sA, &beta, C, c_f32 ? CUDA_R_32F : CUDA_R_16BF, (int)ldc, sC, batch,
+                                    CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT) == CUBLAS_STATUS_SUCCESS;
+}
+
+}  // namespace
+
+size_t train_cache_bytes(int64_t T, int64_t V, int N, int64_t D, int64_t Dr) {
+  return carve_cache(nullptr, T, V, N, D, Dr, nullptr);
+}
+
+mole_status train_forward(const void* groups, size_t gbytes, int64_t T, const void* h, const void* Wr, const void* E,
+                          const void* W1, const void* W2, int64_t V, int N, int64_t D, int64_t Dr, int act,
+                          float* out, void* cache, size_t cbytes, int32_t* n_distinct, cudaStream_t stream) {
+  TrainCache c{};
+  if (carve_cache(cache, T, V, N, D, Dr, &c) > cbytes) return MOLE_ERR_WORKSPACE;
+  const int64_t cap = std::min(T, V);
+  // the batch's distinct ids (one synchronisation: the GEMM sizes follow U)
+  mole_status st = token_groups_count(groups, gbytes, T, N, c.U, stream);
+  if (st != MOLE_OK) return st;
+  int U = 0;
+  if (cudaMemcpyAsync(&U, c.U, sizeof(int), cudaMemcpyDeviceToHost, stream) != cudaSuccess ||
+      cudaStreamSynchronize(stream) != cudaSuccess)
+    return MOLE_ERR_CUDA;
+  if (U < 0 || U > cap) return MOLE_ERR_CUDA;
+  *n_distinct = U;
+  if (U > 0) {
+    st = gather_rows_by_uid(groups, gbytes, T, N, E, D * 2, V, c.Eu, cap, stream);
+    if (st != MOLE_OK) return st;
+    st = train_experts_tc(c.Eu, W1, W2, U, cap, D, N, Dr, act, c.H, c.pre, c.Y, stream);
+    if (st != MOLE_OK) return st;
+  }
+  // the combine over the batch's expert rows, addressed by dense index
+  return combine_offload(groups, gbytes, T, h, Wr, c.Y, (size_t)cap * N * D * 2, V, N, (int)D, true, false, out,
+                         stream);
+}
+
+mole_status train_backward(const void* groups, size_t gbytes, int64_t T, const void* h, const void* Wr,
+                           const void* W1, const void* W2, int64_t V, int N, int64_t D, int64_t Dr, int act,
+                           const float* dout, void* cache, size_t cbytes, int32_t U, float* dh, float* dWr, float* dE,
+                           float* dW1, float* dW2, cudaStream_t stream) {
+  TrainCache c{};
+  if (carve_cache(cache, T, V, N, D, Dr, &c) > cbytes) return MOLE_ERR_WORKSPACE;
+  GroupWs w{};
+  if (carve_ws(const_cast<void*>(groups), T, padded_experts(N), &w) > gbytes) return MOLE_ERR_WORKSPACE;
+  const int64_t cap = std::min(T, V);
+  if (U < 0 || U > cap) return MOLE_ERR_ARG;
+  const uint16_t* h16 = static_cast<const uint16_t*>(h);
+  const uint16_t* wr16 = static_cast<const uint16_t*>(Wr);
+  const int n_sm = num_sms();
+  if (n_sm <= 0) return MOLE_ERR_NO_DEVICE;
+  // gates, logit gradients, dh
+  const unsigned gg = (unsigned)std::min<int64_t>((T + 7) / 8, (int64_t)n_sm * 8);
+  if (N <= 8)
+    gate_grad_kernel<8><<<gg, kGradThreads, 0, stream>>>(w, h16, wr16, c.Y, dout, T, N, (int)D, c.g, c.dz, dh);
+  else if (N <= 16)
+    gate_grad_kernel<16><<<gg, kGradThreads, 0, stream>>>(w, h16, wr16, c.Y, dout, T, N, (int)D, c.g, c.dz, dh);
+  else
+    gate_grad_kernel<32><<<gg, kGradThreads, 0, stream>>>(w, h16, wr16, c.Y, dout, T, N, (int)D, c.g, c.dz, dh);
+  if (cudaGetLastError() != cudaSuccess) return MOLE_ERR_CUDA;
+  if (dWr != nullptr) {
+    const dim3 gw((unsigned)((D + kGradThreads - 1) / kGradThreads), (unsigned)((T + kDwrTokens - 1) / kDwrTokens));
+    if (N <= 8)
+      dwr_kernel<8><<<gw, kGradThreads, 0, stream>>>(w, h16, c.dz, T, N, (int)D, dWr);
+    else if (N <= 16)
+      dwr_kernel<16><<<gw, kGradThreads, 0, stream>>>(w, h16, c.dz, T, N, (int)D, dWr);
+    else
+      dwr_kernel<32><<<gw, kGradThreads, 0, stream>>>(w, h16, c.dz, T, N, (int)D, dWr);
+    if (cudaGetLastError() != cudaSuccess) return MOLE_ERR_CUDA;
+  }
+  if (U == 0 || (dE == nullptr && dW1 == nullptr && dW2 == nullptr)) return MOLE_OK;
+  // dY by the grouping's items, then its bf16 copy for the GEMMs
+  const int64_t ny = (int64_t)U * N * D;
+  if (cudaMemsetAsync(c.dY, 0, ny * 4, stream) != cudaSuccess) return MOLE_ERR_CUDA;
+  dy_kernel<<<(unsigned)n_sm * 4, kGradThreads, 0, stream>>>(w, c.g, dout, N, (int)D, c.dY);
+  to_bf16_kernel<<<grid_for(ny, 256), 256, 0, stream>>>(c.dY, c.dYb, ny);
+  if (cudaGetLastError() != cudaSuccess) return MOLE_ERR_CUDA;
+  cublasHandle_t hb = blas_handle();
+  if (hb == nullptr || cublasSetStream(hb, stream) != CUBLAS_STATUS_SUCCESS ||
+      cublasSetWorkspace(hb, c.blas_ws, (size_t)kCublasWorkspace) != CUBLAS_STATUS_SUCCESS)
+    return MOLE_ERR_CUDA;
+  // dH_j = dY_j . W2_j^T -> dP (bf16), then dP = dH * act'(pre)
+  if (!rm_gemm(hb, false, true, U, Dr, D, c.dYb, (int64_t)N * D, D, W2, D, Dr * D, 0.f, c.dP, false, Dr, cap * Dr, N))
+    return MOLE_ERR_CUDA;
+  act_grad_kernel<<<grid_for((int64_t)N * U * Dr, 256), 256, 0, stream>>>(c.dP, c.pre, U, cap, Dr, N, act);
+  if (cudaGetLastError() != cudaSuccess) return MOLE_ERR_CUDA;
+  // dW2_j += H_j^T dY_j
+  if (dW2 != nullptr &&
+      !rm_gemm(hb, true, false, Dr, D, U, c.H, Dr, cap * Dr, c.dYb, (int64_t)N * D, D, 1.f, dW2, true, D, Dr * D, N))
+    return MOLE_ERR_CUDA;
+  // dW1_j += Eu^T dP_j
+  if (dW1 != nullptr &&
+      !rm_gemm(hb, true, false, D, Dr, U, c.Eu, D, 0, c.dP, Dr, cap * Dr, 1.f, dW1, true, Dr, D * Dr, N))
+    return MOLE_ERR_CUDA;
+  // dEu = sum_j dP_j . W1_j^T, then dE[ids] += dEu
+  if (dE != nullptr) {
+    for (int j = 0; j < N; ++j)
+      if (!rm_gemm(hb, false, true, U, D, Dr, c.dP + (int64_t)j * cap * Dr, Dr, 0,
+                   static_cast<const uint16_t*>(W1) + (int64_t)j * D * Dr, Dr, 0, j == 0 ? 0.f : 1.f, c.dEu, true, D,
+                   0, 1))
+        return MOLE_ERR_CUDA;
+    scatter_rows_kernel<<<grid_for((int64_t)U * D, 256), 256, 0, stream>>>(w, c.dEu, U, (int)D, dE);
+    if (cudaGetLastError() != cudaSuccess) return MOLE_ERR_CUDA;
+  }
+  return MOLE_OK;
+}
+
+}  // namespace mole

@@ -54,6 +54,11 @@ SIGNATURES = {
     "mole_ffn_block_workspace": ([_I64, _I64, _I64], _SZ),
     "mole_ffn_block": ([_P, _I64, _P, _SZ, _P, _P, _P, _I64, _I32, _P, _P, _I64, _I64, _I, _P, _P, _P, _SZ, _P], _I),
     "mole_build_lut_nf3": ([_P, _P, _P, _I64, _I64, _I32, _I64, _I, _P, _P, _P, _SZ, _P], _I),
+    "mole_train_cache_bytes": ([_I64, _I64, _I32, _I64, _I64], _SZ),
+    "mole_train_forward": ([_P, _I64, _P, _SZ, _P, _P, _P, _P, _P, _I64, _I32, _I64, _I64, _I, _P, _P, _SZ, _P, _P],
+                           _I),
+    "mole_train_backward": ([_P, _I64, _P, _SZ, _P, _P, _P, _P, _P, _I64, _I32, _I64, _I64, _I, _P, _P, _SZ, _I32,
+                             _P, _P, _P, _P, _P, _P], _I),
     "mole_nf3_levels": ([_P], None),
     "mole_nf3_midpoints": ([_P], None),
     "mole_gather_plan": ([_P, _I64, _I64, _P, _P, _P, _P], _I),
@@ -376,6 +381,45 @@ def mole_ffn_block(ids: torch.Tensor, groups: torch.Tensor, h: torch.Tensor, Wr:
                            _ptr(W2s), D, Ds, ACT[act], _ptr(residual), _ptr(out), _ptr(workspace), workspace.numel(),
                            _stream(stream)), "mole_ffn_block")
     return out
+
+
+def mole_train_cache_bytes(T: int, V: int, N: int, D: int, Dr: int) -> int:
+    return int(lib.mole_train_cache_bytes(T, V, N, D, Dr))
+
+
+def mole_train_forward(ids: torch.Tensor, groups: torch.Tensor, h: torch.Tensor, Wr: torch.Tensor, E: torch.Tensor,
+                       W1: torch.Tensor, W2: torch.Tensor, act: str = "gelu", out: torch.Tensor | None = None,
+                       cache: torch.Tensor | None = None, stream=None):
+    """(out, cache, n_distinct): one MoLE layer's training forward (see mole.h)."""
+    _contig(ids, groups, h, Wr, E, W1, W2, out, cache)
+    V, D = E.shape
+    N, _, Dr = W1.shape
+    T = ids.numel()
+    if out is None:
+        out = torch.empty((T, D), dtype=torch.float32, device=h.device)
+    if cache is None:
+        cache = torch.empty(max(1, mole_train_cache_bytes(T, V, N, D, Dr)), dtype=torch.uint8, device=h.device)
+    n = ctypes.c_int32(0)
+    _ok(lib.mole_train_forward(_ptr(ids), T, _ptr(groups), groups.numel(), _ptr(h), _ptr(Wr), _ptr(E), _ptr(W1),
+                               _ptr(W2), V, N, D, Dr, ACT[act], _ptr(out), _ptr(cache), cache.numel(),
+                               ctypes.addressof(n), _stream(stream)), "mole_train_forward")
+    return out, cache, int(n.value)
+
+
+def mole_train_backward(ids: torch.Tensor, groups: torch.Tensor, h: torch.Tensor, Wr: torch.Tensor, E: torch.Tensor,
+                        W1: torch.Tensor, W2: torch.Tensor, dout: torch.Tensor, cache: torch.Tensor, n_distinct: int,
+                        act: str = "gelu", dh=None, dWr=None, dE=None, dW1=None, dW2=None, stream=None):
+    """Adds this layer's gradients of sum(out * dout) into the fp32 buffers
+    given (see mole.h); returns them."""
+    _contig(ids, groups, h, Wr, E, W1, W2, dout, cache, dh, dWr, dE, dW1, dW2)
+    V, D = E.shape
+    N, _, Dr = W1.shape
+    T = ids.numel()
+    _ok(lib.mole_train_backward(_ptr(ids), T, _ptr(groups), groups.numel(), _ptr(h), _ptr(Wr), _ptr(E), _ptr(W1),
+                                _ptr(W2), V, N, D, Dr, ACT[act], _ptr(dout), _ptr(cache), cache.numel(), n_distinct,
+                                _ptr(dh), _ptr(dWr), _ptr(dE), _ptr(dW1), _ptr(dW2), _stream(stream)),
+        "mole_train_backward")
+    return dh, dWr, dE, dW1, dW2
 
 
 def mole_nf3_levels():

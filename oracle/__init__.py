@@ -189,6 +189,87 @@ def ffn_block(ids, h, Wr, lut, W1s, W2s, act_name: str = "gelu", residual=None, 
     return out, allow[:, 0, :], n_bad
 
 
+def _bits_f64(a):
+    a = np.asarray(a)
+    if a.dtype == np.uint16:
+        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return a.astype(np.float64)
+
+
+def _act64(name, u):
+    """Expert activation on fp64 arrays (the forms of mole_oracle.c)."""
+    from scipy.special import erfc
+    if name in ("gelu", "gelu_erf"):
+        return u * 0.5 * erfc(-u / np.sqrt(2.0))
+    if name == "gelu_tanh":
+        return 0.5 * u * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (u + 0.044715 * u ** 3)))
+    if name == "relu":
+        return np.maximum(u, 0.0)
+    if name == "silu":
+        return u / (1.0 + np.exp(-u))
+    return u
+
+
+def _act64_grad(name, u):
+    """Derivative of _act64 (the chain rule written out per activation)."""
+    from scipy.special import erfc
+    if name in ("gelu", "gelu_erf"):
+        return 0.5 * erfc(-u / np.sqrt(2.0)) + u * np.exp(-0.5 * u * u) / np.sqrt(2.0 * np.pi)
+    if name == "gelu_tanh":
+        c = np.sqrt(2.0 / np.pi)
+        th = np.tanh(c * (u + 0.044715 * u ** 3))
+        return 0.5 * (1.0 + th) + 0.5 * u * (1.0 - th * th) * c * (1.0 + 3.0 * 0.044715 * u * u)
+    if name == "relu":
+        return (u > 0).astype(np.float64)
+    if name == "silu":
+        sg = 1.0 / (1.0 + np.exp(-u))
+        return sg * (1.0 + u * (1.0 - sg))
+    return np.ones_like(u)
+
+
+def train_step(ids, h, Wr, E, W1, W2, act_name: str = "gelu", dout=None, round_h: bool = True):
+    """One MoLE layer in training, forward and backward, in fp64 (numpy).
+
+    MoLE page, 训练阶段: the routed experts take the token's embedding row,
+    all N are active, and the router on the previous layer's output h mixes
+    them:  out[t] = sum_j g_j(h[t]) f_j(E[ids[t]]),  g = softmax(h Wr),
+    f_j(x) = act(x W1[j]) W2[j] with the hidden activation rounded to bf16
+    when round_h (the bf16 build's precision point; the backward treats the
+    rounding as identity).  Returns (out, grads) where grads holds the
+    gradients of L = sum(out * dout): dh, dWr, dE, dW1, dW2 (all fp64).
+    Every id must lie in [0, V).
+    """
+    ids = np.asarray(ids, dtype=np.int64)
+    hf, Wrf, Ef, W1f, W2f = (_bits_f64(x) for x in (h, Wr, E, W1, W2))
+    uniq, inv = np.unique(ids, return_inverse=True)
+    inv = inv.ravel()
+    Eu = Ef[uniq]                                      # [U, D]
+    pre = np.einsum("ud,jdr->jur", Eu, W1f)            # [N, U, Dr]
+    a = _act64(act_name, pre)
+    if round_h:
+        a = round_bf16_array(a)
+    Y = np.einsum("jur,jrd->ujd", a, W2f)              # [U, N, D]
+    z = hf @ Wrf
+    z = z - z.max(axis=1, keepdims=True)
+    g = np.exp(z)
+    g /= g.sum(axis=1, keepdims=True)
+    out = np.einsum("tj,tjd->td", g, Y[inv])
+    grads = None
+    if dout is not None:
+        do = np.asarray(dout, dtype=np.float64)
+        dg = np.einsum("td,tjd->tj", do, Y[inv])
+        dz = g * (dg - (g * dg).sum(axis=1, keepdims=True))
+        dY = np.zeros_like(Y)
+        np.add.at(dY, inv, g[:, :, None] * do[:, None, :])
+        dA = np.einsum("ujd,jrd->jur", dY, W2f)
+        dpre = dA * _act64_grad(act_name, pre)
+        dE = np.zeros_like(Ef)
+        dE[uniq] = np.einsum("jur,jdr->ud", dpre, W1f)
+        grads = {"dh": dz @ Wrf.T, "dWr": hf.T @ dz, "dE": dE,
+                 "dW1": np.einsum("ud,jur->jdr", Eu, dpre), "dW2": np.einsum("jur,ujd->jrd", a, dY)}
+    return out, grads
+
+
 def round_bf16_array(x: np.ndarray) -> np.ndarray:
     """Element-wise bf16 rounding (ties to even) of float64 values."""
     x = np.ascontiguousarray(x, dtype=np.float64)
