@@ -647,9 +647,19 @@ def nf3_leg(mole, luts, routers, id_pool, h_pool, uniq_counts, dev, stream, W, K
     assert mole.mole_check(stream) == 0
     q_bytes = V * N * D * 2 + V * N * D * 3 / 8 + V * N * (D // 64) * 2
     del tables, groups
+    # ALU roofline (plain lane arithmetic): a gate-weighted FMA per (token,
+    # expert, element) plus ~4 integer / conversion operations to decode each
+    # element of each distinct row block (bit extract, two byte-permute
+    # lookups, fp16 -> fp32), against 148 SMs x 128 lanes x the max SM clock
+    lane_ops = T * N * D + 4.0 * U * N * D
+    alu_peak = 148 * 128 * 1.965e9
+    alu_us = lane_ops / alu_peak * 1e6
     return {"tokens_per_s": T / (avg / 1e3) / L, "tokens_per_s_per_layer": T / (avg / 1e3),
             "avg_launch_us": avg * 1e3, "achieved_gbs": b / (avg / 1e3) / 1e9,
             "frac_of_measured_hbm": b / (avg / 1e3) / 1e9 / hbm_peak, "algorithmic_bytes_per_launch": b,
+            "alu": {"bound": "alu", "lane_ops_per_launch": lane_ops, "peak_lane_ops_per_s": alu_peak,
+                    "roofline_us": alu_us, "frac": alu_us / (avg * 1e3),
+                    "model": "T*N*D FMAs + 4*U*N*D decode ops; 148 SMs x 128 lanes x 1.965 GHz"},
             "quantize_ms_per_layer": q_avg, "quantize_gbs": q_bytes / (q_avg / 1e3) / 1e9,
             "workload": f"1B-shaped NF3 table (codes + fp16 scale per 64), T={T}, same ids/h as the main case, "
                         f"mole_lookup_combine_nf3_groups (grouping built once per id batch, not timed here)"}
