@@ -19,7 +19,8 @@
 //   dY[u, j] = sum_{t: u(t) = u} g_j[t] dout[t]           (dy_kernel over the grouping's items)
 //   dpre_j = (dY_j . W2_j^T) * act'(pre_j)                (cuBLAS + act_grad_kernel)
 //   dW2_j += H_j^T dY_j,  dW1_j += Eu^T dpre_j,  dE[ids] += sum_j dpre_j . W1_j^T
-//                                                         (cuBLAS, scatter_rows_kernel)
+//                                                         (cuBLAS batched over the experts,
+//                                                          scatter_rows_kernel sums the experts)
 // The backward GEMMs are plain transposed bf16 GEMMs with fp32 accumulation
 // and run in cuBLAS; their bf16 operands dY and dpre are rounded from fp32.
 #include <cublas_v2.h>
@@ -43,7 +44,7 @@ struct TrainCache {
   float* dY;      // [cap, N, D] fp32
   uint16_t* dYb;  // [cap, N, D] bf16
   uint16_t* dP;   // [N, cap, Dr] bf16: dL/dpre (first dL/dH)
-  float* dEu;     // [cap, D] fp32
+  float* dEu;     // [N, cap, D] fp32: each expert's share of dL/dEu
   void* blas_ws;  // cuBLAS workspace
   int* U;         // one device int
   size_t total;
@@ -66,7 +67,7 @@ size_t carve_cache(void* base, int64_t T, int64_t V, int N, int64_t D, int64_t D
   const size_t o_dy = take(4 * (size_t)cap * N * D);
   const size_t o_dyb = take(2 * (size_t)cap * N * D);
   const size_t o_dp = take(2 * (size_t)N * cap * Dr);
-  const size_t o_deu = take(4 * (size_t)cap * D);
+  const size_t o_deu = take(4 * (size_t)N * cap * D);
   const size_t o_ws = take((size_t)kCublasWorkspace);
   const size_t o_u = take(16);
   if (c != nullptr && base != nullptr) {
@@ -266,12 +267,16 @@ __global__ void act_grad_kernel(uint16_t* dP, const float* __restrict__ pre, int
   }
 }
 
-// dE[id(u), :] += dEu[u, :] (each distinct id once).
-__global__ void scatter_rows_kernel(const GroupWs w, const float* __restrict__ dEu, int64_t U, int D, float* dE) {
+// dE[id(u), :] += sum_j dEu[j, u, :] (each distinct id once; experts summed
+// in order).
+__global__ void scatter_rows_kernel(const GroupWs w, const float* __restrict__ dEu, int64_t U, int64_t cap, int D,
+                                    int N, float* dE) {
   const int64_t n = U * D;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t u = i / D, d = i - u * D;
-    dE[(int64_t)w.uid_id[u] * D + d] += dEu[i];
+    float acc = 0.f;
+    for (int j = 0; j < N; ++j) acc += dEu[(int64_t)j * cap * D + i];
+    dE[(int64_t)w.uid_id[u] * D + d] += acc;
   }
 }
 
@@ -392,14 +397,12 @@ mole_status train_backward(const void* groups, size_t gbytes, int64_t T, const v
   if (dW1 != nullptr &&
       !rm_gemm(hb, true, false, D, Dr, U, c.Eu, D, 0, c.dP, Dr, cap * Dr, 1.f, dW1, true, Dr, D * Dr, N))
     return MOLE_ERR_CUDA;
-  // dEu = sum_j dP_j . W1_j^T, then dE[ids] += dEu
+  // dEu_j = dP_j . W1_j^T for all experts in one batched GEMM, then
+  // dE[ids] += sum_j dEu_j
   if (dE != nullptr) {
-    for (int j = 0; j < N; ++j)
-      if (!rm_gemm(hb, false, true, U, D, Dr, c.dP + (int64_t)j * cap * Dr, Dr, 0,
-                   static_cast<const uint16_t*>(W1) + (int64_t)j * D * Dr, Dr, 0, j == 0 ? 0.f : 1.f, c.dEu, true, D,
-                   0, 1))
-        return MOLE_ERR_CUDA;
-    scatter_rows_kernel<<<grid_for((int64_t)U * D, 256), 256, 0, stream>>>(w, c.dEu, U, (int)D, dE);
+    if (!rm_gemm(hb, false, true, U, D, Dr, c.dP, Dr, cap * Dr, W1, Dr, D * Dr, 0.f, c.dEu, true, D, cap * D, N))
+      return MOLE_ERR_CUDA;
+    scatter_rows_kernel<<<grid_for((int64_t)U * D, 256), 256, 0, stream>>>(w, c.dEu, U, cap, (int)D, N, dE);
     if (cudaGetLastError() != cudaSuccess) return MOLE_ERR_CUDA;
   }
   return MOLE_OK;
