@@ -383,7 +383,9 @@ mole_status mole_gather_plan(const int32_t* ids, int64_t T, int64_t V, int32_t* 
  * Waits (polling, at most timeout_ms; < 0 = no limit) for `stream` to drain,
  * then reads and clears this device's error word.  Returns MOLE_OK,
  * MOLE_ERR_INDEX (bad token id), MOLE_ERR_TIMEOUT (stream still busy, or a
- * device-side wait gave up), or MOLE_ERR_CUDA (an asynchronous CUDA error).
+ * device-side wait gave up), MOLE_ERR_ARG (a grouping was used on a device
+ * with another SM count than the one it was built on; the layer's output was
+ * not written), or MOLE_ERR_CUDA (an asynchronous CUDA error).
  */
 mole_status mole_check(cudaStream_t stream, int timeout_ms);
 

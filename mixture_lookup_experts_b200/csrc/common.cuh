@@ -17,6 +17,7 @@ namespace mole {
 enum : unsigned {
   kErrIndex = 1u,    // a token id outside [0, V)
   kErrTimeout = 2u,  // a bounded device-side wait gave up
+  kErrGrouping = 4u, // a grouping used on a device other than the one it was built for
 };
 
 // Device address of this device's error word (resolved once per device).

@@ -21,12 +21,21 @@
 //               item records, laid out by item size, largest first;
 //       step 3  every token's list position: list[pos] = t, tok_pos[t] = pos.
 //     Steps 1-3 each start after a grid-wide barrier (bounded wait).
-//  2. the router (per layer): router_tc.cu's tcgen05 kernel for 16 experts,
-//     else router_group_kernel (persistent, 2 CTAs per SM, the mma.sync
-//     router of combine_common.cuh); each token's gates go to its list
-//     position, so an item's gates are contiguous.
-//  3. grouped_gather_kernel (per layer; one CTA per SM, 9 warps): a producer
-//     warp copies each work item's row block and its tokens' gates (two
+//     Then group_share_kernel (once per batch) lists, for each CTA of a
+//     one-CTA-per-SM layer kernel, its work items in processing order and
+//     their tokens (its share).
+//  Per layer, batches too small for the tensor-core router (fewer 128-token
+//  tiles than about 3/4 of the SMs):
+//  2. grouped_local_kernel (one CTA per SM, 9 warps): each CTA computes the
+//     gates of its own share's tokens (mma.sync router, gates kept in shared
+//     memory), then gathers and combines its work items as in 3.
+//  Per layer, otherwise:
+//  2. the router: router_tc.cu's tcgen05 kernel for 16 experts, else
+//     router_group_kernel (persistent, 2 CTAs per SM, the mma.sync router of
+//     combine_common.cuh); each token's gates go to its list position, so an
+//     item's gates are contiguous.
+//  3. grouped_gather_kernel (one CTA per SM, 9 warps): a producer warp
+//     copies each work item's row block and its tokens' gates (two
 //     cp.async.bulk) into a ring of shared-memory slots; 8 consumer warps
 //     convert each 4-element vector of the N rows to fp32 once and apply it
 //     to every token of the item.
@@ -510,7 +519,6 @@ struct Ring {
   int* slot_n;
   int* slot_tok;  // [n_slots][kItemTokens]
   int* abort;
-  int q0;         // the slot of the CTA's first work item
 };
 
 __host__ __device__ constexpr size_t ring_bytes(int n_slots, int slot_bytes) {
@@ -525,112 +533,82 @@ __device__ __forceinline__ Ring carve_ring(uint8_t* base, const GroupLayout& L) 
   r.slot_n = reinterpret_cast<int*>(r.empty + L.n_slots);
   r.slot_tok = r.slot_n + L.n_slots;
   r.abort = r.slot_tok + L.n_slots * kItemTokens;
-  r.q0 = 0;
   return r;
 }
 
-// Thread 0: barriers initialised, abort flag cleared.
-__device__ __forceinline__ void ring_init(const Ring& r, const GroupLayout& L) {
+// Thread 0: barriers initialised (`full_arrivals` per full phase), abort
+// flag cleared.
+__device__ __forceinline__ void ring_init(const Ring& r, const GroupLayout& L, int full_arrivals = 3) {
   for (int q = 0; q < L.n_slots; ++q) {
-    mbar_init(&r.full[q], 3);
+    mbar_init(&r.full[q], full_arrivals);
     mbar_init(&r.empty[q], kGroupCons);
   }
   *r.abort = 0;
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
-__device__ __forceinline__ void fence_proxy_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
-__device__ __forceinline__ void st_release(unsigned* p, unsigned v) {
-  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
-// Router-tile readiness in the fused kernel: flag[i] = `want` once the gates
-// of tokens [16 i, 16 i + 16) are stored.  want = epoch + 1, where epoch
-// numbers the fused launches on a grouping: every CTA takes an arrival index
-// from a 64-bit counter when it starts, and the CTAs of one launch take
-// consecutive indices (a launch's CTAs start after the previous launch has
-// completed), so index / gridDim is the same for all of them.  A grouping
-// build resets the counter (all ones = no arrivals) and the flags.
-struct TileFlags {
-  unsigned* flag;
-  unsigned long long* arrivals;
-  unsigned* abort_word;  // the grouping's abort word
-};
-
-// Shared-memory staging for the fused kernel's router phase.  Wr arrives by
-// one bulk copy in the ring's last slot W (wr_full) and is released back to
-// the ring once every consumer warp has its fragments in registers
-// (wr_free).  With staged hidden states, the CTA's router tiles (at most
-// kMaxStagedTiles) arrive in slots 0, 1, ... one bulk copy per token row
-// into a padded layout (h_full[j]) and are released after their MMAs
-// (h_empty[j]).  `epoch` completes when want_s holds the launch's flag value.
-constexpr int kMaxStagedTiles = 4;
-
-struct FusedSync {
+// The CTA-local layer kernel's router input Wr arrives by bulk copies in the
+// ring's last slot W (wr_full) and goes back to the ring once every consumer
+// warp holds its B fragments in registers (wr_free).  The CTA's work item
+// records come from its share, in processing order.
+struct LocalSync {
   uint64_t* wr_full;
   uint64_t* wr_free;
-  uint64_t* epoch;
-  uint64_t* h_full;   // [kMaxStagedTiles]
-  uint64_t* h_empty;  // [kMaxStagedTiles]
-  const unsigned* want_s;
-  TileFlags tf;
-  int n_staged;       // router tiles of this CTA staged in slots 0 .. n_staged-1 (0: A from global)
-  int h_pitch;        // bytes between staged token rows (2 D + 32)
+  const int4* recs;  // [my_n]
 };
 
-// Ring position of the CTA's k-th work item: the ring starts at slot q0 and
-// visits the slots in order; the k-th item is in lap k / n_slots.
-__device__ __forceinline__ uint32_t ring_slot(const Ring& r, const GroupLayout& L, int k) {
-  return (uint32_t)((r.q0 + k) % L.n_slots);
+// Ring position of the CTA's k-th work item: slot k mod n_slots, in lap
+// k / n_slots.
+__device__ __forceinline__ uint32_t ring_slot(const Ring&, const GroupLayout& L, int k) {
+  return (uint32_t)(k % L.n_slots);
 }
 __device__ __forceinline__ uint32_t ring_parity(const GroupLayout& L, int k) {
   return (uint32_t)((k / L.n_slots) & 1);
 }
 
-// The work items (largest first) are dealt to the CTAs in rounds of
-// gridDim.x, alternating direction (round m: CTA b takes the item at
-// position b of the round if m is even, gridDim.x - 1 - b if odd), so that no
-// CTA takes the largest item of every round.
-__device__ __forceinline__ int item_of_cta(int m) {
-  const int pos = (m & 1) ? (int)gridDim.x - 1 - (int)blockIdx.x : (int)blockIdx.x;
-  return m * (int)gridDim.x + pos;
+// The work items (largest first) are dealt to the G CTAs of a layer kernel in
+// rounds of G, alternating direction (round m: CTA b takes the item at
+// position b of the round if m is even, G - 1 - b if odd), so that no CTA
+// takes the largest item of every round.
+__host__ __device__ __forceinline__ int item_of(int m, int b, int G) { return m * G + ((m & 1) ? G - 1 - b : b); }
+
+__host__ __device__ __forceinline__ int items_of(int n_items, int b, int G) {
+  const int full = n_items / G;  // complete rounds
+  return full + (item_of(full, b, G) < n_items ? 1 : 0);
+}
+
+// CTA b's work item at step k of its processing order: those of rounds 0,
+// my_n-1, 1, my_n-2, ... (large, small, large, ...).
+__host__ __device__ __forceinline__ int cta_item(int k, int my_n, int b, int G) {
+  return item_of((k & 1) ? my_n - 1 - (k >> 1) : (k >> 1), b, G);
 }
 
 __device__ __forceinline__ int items_of_cta(const GroupWs& w) {
-  const int n_items = (int)ld_relaxed_u32(&w.ctl[kCtlItems]);
-  const int full = n_items / (int)gridDim.x;  // complete rounds
-  return full + (item_of_cta(full) < n_items ? 1 : 0);
+  return items_of((int)ld_relaxed_u32(&w.ctl[kCtlItems]), (int)blockIdx.x, (int)gridDim.x);
 }
 
-// Producer warp of the gather.  The CTA's work items are
-// items[item_of_cta(m)], m = 0 .. my_n-1, largest first; step k
-// takes them alternately from the front and the back (large, small, large,
-// ...), so the copies of small items proceed while the consumers work through
-// large ones.  Item records are read 32 at a time (one per lane) and each
-// item's token list one item ahead.  With `fs` (fused kernel) the producer
-// first copies the router phase's inputs (Wr; with staged hidden states also
-// the CTA's router tiles), then requests the row blocks of the first items
-// (one per slot) as their slots come free, and requests an item's gates only
-// when the router tiles of all of its tokens have flagged them stored (flags
-// read one item ahead with the token list).
+// Producer warp of the gather.  The CTA's work items are taken in cta_item
+// order, so the copies of small items proceed while the consumers work
+// through large ones.  Item records are read 32 at a time (one per lane) and
+// each item's token list one item ahead.  Per item: the row block's copies
+// and (grouped_gather_kernel) its tokens' gates into the item's slot, then
+// the token list.  With `ls` (CTA-local kernel, gates in shared memory) the
+// records come from the CTA's share, the row blocks of the first items go
+// out at once (slot W's once Wr is no longer needed there), and the warp
+// also writes the
+// NaN output rows of the bad-id tokens in its CTA's slice of the batch.
 template <int NP, bool kNf3>
 __device__ void ring_producer(const GArgs& p, const GroupWs& w, const GroupLayout& L, const Ring& r, int my_n,
-                              const FusedSync* fs) {
+                              const LocalSync* ls) {
   constexpr int C = kItemTokens;
   const int lane = threadIdx.x & 31;
   volatile int* abort = r.abort;
   const uint32_t row_bytes = (uint32_t)p.N * (uint32_t)p.D * 2u;
   const int NB = p.D >> 6;  // NF3 blocks per row
   const uint32_t code_bytes = (uint32_t)p.N * (uint32_t)NB * 24u, scale_bytes = (uint32_t)p.N * (uint32_t)NB * 2u;
-  const uint32_t W = (uint32_t)L.n_slots - 1u;  // Wr's slot (fused kernel)
-  // fused kernel: the small items first (they depend on few router tiles)
-  const int from_back = fs != nullptr ? 0 : 1;
   auto record = [&](int kk) {
-    const int m = ((kk & 1) == from_back) ? my_n - 1 - (kk >> 1) : (kk >> 1);
-    return kk < my_n ? w.items[item_of_cta(m)] : make_int4(0, 0, 0, 0);
+    if (kk >= my_n) return make_int4(0, 0, 0, 0);
+    return ls != nullptr ? ls->recs[kk] : w.items[cta_item(kk, my_n, (int)blockIdx.x, (int)gridDim.x)];
   };
   // the row block's copies into slot q, on its full barrier (lane 0)
   auto issue_rows = [&](uint32_t q, int row) {
@@ -654,90 +632,51 @@ __device__ void ring_producer(const GArgs& p, const GroupWs& w, const GroupLayou
   };
   // items 0 .. issued-1 went out in full
   int issued = 0;
-  // abandon the layer with items k .. last-1 holding row copies but no
-  // gates or token list: the flag first (consumers check it when a slot's
-  // phase completes), then their missing arrivals, so their phases complete
-  // when the copies land and the drain below waits for them
-  auto abandon = [&](int k, int last) {
-    *abort = 1;
-    __syncwarp();
-    if (lane == 0)
-      for (int kk = k; kk < last; ++kk) {
-        mbar_arrive(&r.full[ring_slot(r, L, kk)]);
-        mbar_arrive(&r.full[ring_slot(r, L, kk)]);
-      }
-    issued = last;
-  };
   // records of steps k0 + lane (my_item) and k0 + 32 + lane (nx_item)
   int k0 = 0;
   int4 my_item = record(lane);
   int4 nx_item = record(32 + lane);
   bool ok = true;
   int pre = 0;  // items whose row blocks went out ahead of the main loop
-  unsigned want = 0;
-  if (fs != nullptr) {
-    // the router phase's inputs: Wr into slot W, staged router tiles into
-    // slots 0 .. n_staged-1 (token row rr by lane rr)
-    if (lane == 0) {
-      const uint32_t wr_bytes = (uint32_t)p.N * (uint32_t)p.D * 2u;
-      mbar_expect_tx(fs->wr_full, wr_bytes);
-      bulk_g2s(r.slots + (size_t)W * L.slot_bytes, p.Wr, wr_bytes, fs->wr_full);
-    }
-    for (int j = 0; j < fs->n_staged; ++j) {
-      const int64_t t0 = ((int64_t)blockIdx.x + (int64_t)j * gridDim.x) * kTileMax;
-      const int rows = (int)(p.T - t0 < kTileMax ? p.T - t0 : kTileMax);
-      if (lane == 0) mbar_expect_tx(&fs->h_full[j], (uint32_t)rows * (uint32_t)p.D * 2u);
-      __syncwarp();
-      if (lane < rows)
-        bulk_g2s(r.slots + (size_t)j * L.slot_bytes + (size_t)lane * fs->h_pitch, p.h + (t0 + lane) * p.D,
-                 (uint32_t)p.D * 2u, &fs->h_full[j]);
-    }
-    // the row blocks of the first items, as their slots come free: W once
-    // the Wr fragments are in registers, a staged tile's slot once its MMAs
-    // are done, any other slot once Wr has landed (the router's inputs go
-    // first)
+  if (ls != nullptr) {
+    const uint32_t W = (uint32_t)L.n_slots - 1u;
     const int first = my_n < L.n_slots ? my_n : L.n_slots;  // n_slots <= 16 < 32: all in my_item
-    for (int k = 0; ok && k < first; ++k) {
+    for (int k = 0; k < first; ++k) {
       const int row = __shfl_sync(0xffffffffu, p.by_uid ? my_item.w : my_item.x, k);
       if (bad_row(row)) {
         ok = false;
         break;
       }
       const uint32_t q = ring_slot(r, L, k);
-      if (q == W)
-        ok = warp_wait(fs->wr_free, 0u, abort, p.err);
-      else if ((int)q < fs->n_staged)
-        ok = warp_wait(&fs->h_empty[q], 0u, abort, p.err);
-      else
-        ok = warp_wait(fs->wr_full, 0u, abort, p.err);
-      if (!ok) break;
+      if (q == W && !warp_wait(ls->wr_free, 0u, abort, p.err)) {
+        ok = false;
+        break;
+      }
       issue_rows(q, row);
       pre = k + 1;
     }
-    if (ok && my_n > 0) {
-      ok = warp_wait(fs->epoch, 0u, abort, p.err);
-      want = *fs->want_s;
+    if (!ok) {
+      // items 0 .. pre-1 hold row copies but no token list: their missing
+      // arrivals, so their phases complete when the copies land and the
+      // drain below waits for them (the consumers see the abort flag)
+      *abort = 1;
+      __syncwarp();
+      if (lane == 0)
+        for (int kk = 0; kk < pre; ++kk) mbar_arrive(&r.full[ring_slot(r, L, kk)]);
+      issued = pre;
     }
-    if (!ok) abandon(0, pre);
   }
-  // whether the router tile of this lane's token has stored its gates
-  auto tile_ready = [&](int tok) {
-    return tok < 0 || fs == nullptr || ld_acquire(&fs->tf.flag[tok / kTileMax]) == want;
-  };
   int next_tok = -1;
-  bool next_ready = true;
   if (my_n > 0 && ok) {
     const int pos = __shfl_sync(0xffffffffu, my_item.y, 0), n = __shfl_sync(0xffffffffu, my_item.z, 0);
     next_tok = lane < n ? w.list[pos + lane] : -1;
-    next_ready = tile_ready(next_tok);
   }
   for (int k = 0; ok && k < my_n; ++k) {
     const int row = __shfl_sync(0xffffffffu, p.by_uid ? my_item.w : my_item.x, k - k0);
     const int pos = __shfl_sync(0xffffffffu, my_item.y, k - k0);
     const int n = __shfl_sync(0xffffffffu, my_item.z, k - k0);
     const int tok = next_tok;
-    bool ready = next_ready;
-    if (k + 1 < my_n) {  // prefetch the next item's record batch, tokens and their flags
+    if (k + 1 < my_n) {  // prefetch the next item's record batch and tokens
       if (k + 1 - k0 == 32) {
         k0 = k + 1;
         my_item = nx_item;
@@ -746,7 +685,6 @@ __device__ void ring_producer(const GArgs& p, const GroupWs& w, const GroupLayou
       const int pos1 = __shfl_sync(0xffffffffu, my_item.y, k + 1 - k0);
       const int n1 = __shfl_sync(0xffffffffu, my_item.z, k + 1 - k0);
       next_tok = lane < n1 ? w.list[pos1 + lane] : -1;
-      next_ready = tile_ready(next_tok);
     }
     const uint32_t q = ring_slot(r, L, k);
     if (k >= pre) {
@@ -755,36 +693,8 @@ __device__ void ring_producer(const GArgs& p, const GroupWs& w, const GroupLayou
       if (!ok) break;
       issue_rows(q, row);
     }
-    if (fs != nullptr) {
-      // the item's gates exist once every token's router tile has flagged
-      // (bounded wait; a CTA that gives up abandons the layer)
-      if (!__all_sync(0xffffffffu, ready)) {
-        const uint64_t t0 = globaltimer();
-        int fail = 0;
-        while (!__all_sync(0xffffffffu, ready = tile_ready(tok))) {
-          if (lane == 0) {
-            if (*abort || ld_acquire(fs->tf.abort_word) != 0xFFFFFFFFu) {
-              fail = 1;
-            } else if (globaltimer() - t0 > kWaitLimitNs) {
-              atomicExch(fs->tf.abort_word, 1u);
-              atomicOr(p.err, kErrTimeout);
-              fail = 1;
-            }
-          }
-          if (__shfl_sync(0xffffffffu, fail, 0)) break;
-        }
-        if (__shfl_sync(0xffffffffu, fail, 0)) {
-          // this item's rows and those prefetched for the items after it are out
-          abandon(k, k + 1 > pre ? k + 1 : pre);
-          ok = false;
-          break;
-        }
-      }
-      __syncwarp();
-      if (lane == 0) fence_proxy_async_global();  // gates stored by other CTAs, read by a bulk copy
-    }
     uint8_t* slot = r.slots + (size_t)q * L.slot_bytes;
-    if (lane == 0) {
+    if (lane == 0 && ls == nullptr) {
       const uint32_t gate_bytes = (uint32_t)n * NP * 4u;
       mbar_expect_tx(&r.full[q], gate_bytes);
       bulk_g2s(slot + L.gates_off, w.gates + (int64_t)pos * NP, gate_bytes, &r.full[q]);
@@ -796,11 +706,19 @@ __device__ void ring_producer(const GArgs& p, const GroupWs& w, const GroupLayou
     if (lane == 0) mbar_arrive(&r.full[q]);
     issued = k + 1;
   }
-  if (lane == 0) {  // the last copies must have landed before the CTA exits
-    if (fs != nullptr) {
-      mbar_drain(fs->wr_full, 0u);
-      for (int j = 0; j < fs->n_staged; ++j) mbar_drain(&fs->h_full[j], 0u);
+  if (ls != nullptr) {
+    // tokens with a bad id are in no work item: NaN output rows for those of
+    // this CTA's slice of the batch
+    const int64_t t0 = (int64_t)blockIdx.x * p.T / gridDim.x, t1 = ((int64_t)blockIdx.x + 1) * p.T / gridDim.x;
+    for (int64_t t = t0 + lane; t < t1; t += 32) {
+      if (__ldg(w.tok_pos + t) >= 0) continue;
+      atomicOr(p.err, kErrIndex);
+      float* o = p.out + t * p.D;
+      for (int d = 0; d < p.D; d += 4) __stcs(reinterpret_cast<float4*>(o + d), make_float4(NAN, NAN, NAN, NAN));
     }
+  }
+  if (lane == 0) {  // the last copies must have landed before the CTA exits
+    if (ls != nullptr) mbar_drain(ls->wr_full, 0u);
     for (int kk = issued - 1; kk >= 0 && kk >= issued - L.n_slots; --kk)
       mbar_drain(&r.full[ring_slot(r, L, kk)], ring_parity(L, kk));
   }
@@ -809,8 +727,11 @@ __device__ void ring_producer(const GArgs& p, const GroupWs& w, const GroupLayou
 
 // Consumer warps of the gather.  unit = 4 consecutive elements of D; with
 // fewer units than consumer threads, Gt thread groups split the item's tokens.
+// Gates: from the item's slot, or (gl != nullptr) from the CTA's gate array,
+// the k-th item's at rows loff[k] ...
 template <int NT, bool kExactN, bool kNf3>
-__device__ void ring_consumers(const GArgs& p, const GroupLayout& L, const Ring& r, int my_n) {
+__device__ void ring_consumers(const GArgs& p, const GroupLayout& L, const Ring& r, int my_n,
+                               const float* gl = nullptr, const int* loff = nullptr) {
   constexpr int NP = 8 * NT;
   constexpr int C = kItemTokens;
   constexpr bool kPacked = !kNf3 && NP > 16;  // 32 experts: keep rows as bf16 pairs, convert per token
@@ -833,7 +754,7 @@ __device__ void ring_consumers(const GArgs& p, const GroupLayout& L, const Ring&
     if (active) {
       const int n = r.slot_n[q];
       const uint8_t* slot = r.slots + (size_t)q * L.slot_bytes;
-      const float* gs = reinterpret_cast<const float*>(slot + L.gates_off);
+      const float* gs = gl != nullptr ? gl + loff[k] * NP : reinterpret_cast<const float*>(slot + L.gates_off);
       for (int v = v0; v < units; v += vstep) {
         float xf[kPacked ? 1 : NP][4];
         uint2 xp[kPacked ? NP : 1];
@@ -921,23 +842,19 @@ __global__ void __launch_bounds__(kGroupThreads, 1) grouped_gather_kernel(const 
   __syncthreads();
 }
 
-// ---- fused layer kernel: router phase and gather in one launch ----
+// ---- CTA-local layer kernel: router and gather in one launch ----
 //
-// One CTA per SM.  The 8 consumer warps first compute the gates of 16-token
-// tiles (blockIdx.x, blockIdx.x + gridDim.x, ...) with mma.sync -- the same
-// k-step split, k-slot order, partial-sum order and softmax as the router
-// kernels, so the gates are bit-identical to theirs -- store them at the
-// tokens' list positions and flag each tile done.  Wr is brought into the
-// ring's last slot by one bulk copy, its fragments go to registers
-// (ldmatrix.trans) for the whole phase, and the slot returns to the ring.
-// Meanwhile the producer warp requests the row blocks of the CTA's first
-// items; it requests an item's gates once the tiles of all of the item's
-// tokens are flagged, so the gather starts while other CTAs are still
-// routing.  Then the consumers combine as in grouped_gather_kernel.  The
-// flag waits need every CTA resident: one CTA per SM, started when the
-// previous kernel lets it (all of that kernel's CTAs are running by then),
-// and each wait is bounded.  Batches large enough for the tensor-core router
-// kernel take that kernel and grouped_gather_kernel instead.
+// One CTA per SM, no waits on other CTAs.  The CTA's share of the grouping
+// (group_share_kernel) lists its work items in processing order and their
+// tokens.  The consumer warps compute those tokens' gates, two 16-token tiles
+// at a time -- A fragments loaded from h by token id, B fragments from Wr
+// (one bulk copy into the ring's last slot) by ldmatrix, mma.sync with the
+// router kernels' k-step split, k-slot order and partial-sum order, then
+// their softmax, so the gates are bit-identical to theirs -- into a gate array
+// in shared memory, and then combine as in grouped_gather_kernel, reading
+// each item's gates from that array.  Meanwhile the producer warp has
+// requested the row blocks of the first items (Wr's slot once the MMAs are
+// done).
 
 constexpr int kFusedKB = 16;  // k-steps per warp (D <= 2048)
 
@@ -988,56 +905,6 @@ __device__ __forceinline__ void wr_fragments_any(uint2 (&b)[NT], const uint16_t*
   }
 }
 
-// Softmax of one tile, its gates to the tokens' list positions (NaN output
-// rows for bad ids), then its flag.
-template <int NT>
-__device__ __forceinline__ void fused_tile_finish(const GArgs& p, const GroupWs& w, const Smem& s,
-                                                  const float (&acc)[NT][4], int64_t tile, int rows, unsigned* flag,
-                                                  unsigned want, int my_pos) {
-  constexpr int NP = 8 * NT;
-  const int64_t t0 = tile * kTileMax;
-  router_store_partials<NT>(s, acc);
-  // s.tok_id[r] = the list position of token t0 + r (thread r's my_pos)
-  router_softmax<true, NT, ConsumerSync, true>(s, rows, p.N, nullptr, t0, my_pos);
-  for (int i = threadIdx.x; i < rows * NP; i += kGroupCons * 32) {
-    const int r = i / NP, j = i - r * NP;
-    const int pos = s.tok_id[r];
-    if (pos >= 0) w.gates[(int64_t)pos * NP + j] = s.gates[i];
-  }
-  if ((int)threadIdx.x < rows && my_pos < 0) {  // a bad id: its thread writes the NaN output row
-    atomicOr(p.err, kErrIndex);
-    float* o = p.out + (t0 + threadIdx.x) * p.D;
-    for (int d = 0; d < p.D; d += 4) __stcs(reinterpret_cast<float4*>(o + d), make_float4(NAN, NAN, NAN, NAN));
-  }
-  // the flag is a release by thread 0 after the barrier: every consumer's
-  // gate stores precede it (the reader acquires the flag, then fences the
-  // async proxy before its bulk copy); s.gates and s.tok_id are rewritten
-  // only after the next tile's first barrier
-  ConsumerSync{}();
-  if (threadIdx.x == 0) st_release(&flag[tile], want);
-}
-
-// A fragments of a staged router tile (token rows at h_pitch bytes in
-// shared memory), in the same k-slot order as router_load_a: lane (g, c)
-// takes 8 bytes at d = 16 ks + 4c of rows g and g + 8 (zero past `rows`).
-// With h_pitch = 2 D + 32 the 32 lanes of one load hit every bank pair once.
-template <int KB>
-__device__ __forceinline__ void router_load_a_smem(RouterA<KB>& A, const uint8_t* tile_s, int h_pitch, int rows,
-                                                   int D) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
-  const bool ok0 = g < rows, ok1 = g + 8 < rows;
-  const uint8_t* r0 = tile_s + (size_t)g * h_pitch + 8 * c;
-  const uint8_t* r1 = tile_s + (size_t)(g + 8) * h_pitch + 8 * c;
-  const int ksteps = D >> 4;
-#pragma unroll
-  for (int i = 0; i < KB; ++i) {
-    const int ks = warp + i * kWarps;
-    const bool in = ks < ksteps;
-    A.a0[i] = (in && ok0) ? *reinterpret_cast<const uint2*>(r0 + ks * 32) : make_uint2(0u, 0u);
-    A.a1[i] = (in && ok1) ? *reinterpret_cast<const uint2*>(r1 + ks * 32) : make_uint2(0u, 0u);
-  }
-}
-
 // Waits of the consumer warps on a barrier of the router phase, with one
 // verdict for all of them (the tile loop holds barriers, so every warp must
 // take the same path): a warp whose wait failed says so before the barrier
@@ -1049,7 +916,7 @@ __device__ __forceinline__ bool consumers_wait(uint64_t* b, uint32_t parity, vol
   return *fail == 0;
 }
 
-// Router scratch of the staged path: two tiles finished together.
+// Router scratch of the local kernel: two tiles finished together.
 constexpr int kPairRows = 2 * kTileMax;
 
 template <int NP>
@@ -1106,83 +973,62 @@ __device__ __forceinline__ void pair_softmax(const PairScratch& ps, int rows, in
   }
 }
 
-// The gates of `rows` tokens (rows 0..15: tile ta; 16..: tile tb) to their
-// list positions (NaN output rows for bad ids), then the tiles' flags.
-// Thread r holds the list position of row r in my_pos.
-template <int NT>
-__device__ __forceinline__ void pair_finish(const GArgs& p, const GroupWs& w, const PairScratch& ps, int rows,
-                                            int64_t ta, int64_t tb, int my_pos, unsigned* flag, unsigned want) {
-  constexpr int NP = 8 * NT;
-  if (threadIdx.x < rows) ps.tok[threadIdx.x] = my_pos;  // (last read before the previous pair's final barrier)
-  ConsumerSync{}();
-  pair_softmax<NT>(ps, rows, p.N);
-  ConsumerSync{}();
-  for (int i = threadIdx.x; i < rows * NP; i += kGroupCons * 32) {
-    const int r = i / NP, j = i - r * NP;
-    const int pos = ps.tok[r];
-    if (pos >= 0) w.gates[(int64_t)pos * NP + j] = ps.gates[i];
-  }
-  if ((int)threadIdx.x < rows && my_pos < 0) {  // a bad id: its thread writes the NaN output row
-    atomicOr(p.err, kErrIndex);
-    const int r = threadIdx.x;
-    const int64_t t = (r < kTileMax ? ta * kTileMax + r : tb * kTileMax + r - kTileMax);
-    float* o = p.out + t * p.D;
-    for (int d = 0; d < p.D; d += 4) __stcs(reinterpret_cast<float4*>(o + d), make_float4(NAN, NAN, NAN, NAN));
-  }
-  // the flags are releases by thread 0 after the barrier: every consumer's
-  // gate stores precede them
-  ConsumerSync{}();
-  if (threadIdx.x == 0) {
-    st_release(&flag[ta], want);
-    if (rows > kTileMax) st_release(&flag[tb], want);
+// A fragments of a tile whose row rr is token tok[rr] (rr < rows; rows past
+// read as zero), in router_load_a's k-slot order.
+template <int KB>
+__device__ __forceinline__ void router_load_a_rows(RouterA<KB>& A, const uint16_t* __restrict__ h, const int* tok,
+                                                   int rows, int D, int kb) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+  const bool ok0 = g < rows, ok1 = g + 8 < rows;
+  const uint16_t* h0 = h + (int64_t)(ok0 ? __ldg(tok + g) : 0) * D + 4 * c;
+  const uint16_t* h1 = h + (int64_t)(ok1 ? __ldg(tok + g + 8) : 0) * D + 4 * c;
+  const int ksteps = D >> 4;
+#pragma unroll
+  for (int i = 0; i < KB; ++i) {
+    const int ks = kb + i * kWarps;
+    const bool in = ks < ksteps;
+    A.a0[i] = (in && ok0) ? __ldg(reinterpret_cast<const uint2*>(h0 + (ks << 4))) : make_uint2(0u, 0u);
+    A.a1[i] = (in && ok1) ? __ldg(reinterpret_cast<const uint2*>(h1 + (ks << 4))) : make_uint2(0u, 0u);
   }
 }
 
-// Router phase of the fused kernel (consumer warps).  Wr's fragments for
-// this warp's k-steps go to registers once (the Wr slot then returns to the
-// ring).  A fragments: with staged tiles (kStaged) from shared memory, each
-// tile's slot released after its MMAs; otherwise from global memory, a
-// tile's requested right after the previous tile's MMAs.  The tokens' list
-// positions are loaded a tile ahead.  A failed wait abandons the layer (the
-// remaining tiles are not flagged; the other CTAs' waits give up on the
-// abort word, and the error word is set).
-template <int NT, bool kExactN, bool kStaged>
-__device__ void fused_router_phase(const GArgs& p, const GroupWs& w, const Smem& s, const PairScratch& ps,
-                                   const Ring& r, const GroupLayout& L, const FusedSync& fs, unsigned want,
-                                   volatile int* fail) {
+// One bulk prefetch of `bytes` at p (16-byte aligned, a multiple of 16) into L2.
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// Consumer warps: the gates of the CTA's n_tok listed tokens (tok[i]) into
+// gl[n_tok][NP].  Every listed token's h row is first requested into L2 (one
+// bulk prefetch per row); the first tile's A fragments load while Wr
+// arrives; each warp then takes the B fragments of its k-steps into
+// registers and Wr's slot goes back to the ring.  The tiles' A fragments
+// load one tile at a time, the next right after the current tile's MMAs;
+// two tiles share one partial-sum exchange and softmax.  Returns false
+// (uniformly) if Wr never arrived.
+template <int NT, bool kExactN>
+__device__ bool local_router_phase(const GArgs& p, const PairScratch& ps, const uint16_t* wr_s, const LocalSync& ls,
+                                   const int* tok, int n_tok, float* gl, volatile int* abort, volatile int* fail) {
   constexpr int KB = kFusedKB;
+  constexpr int NP = 8 * NT;
   const int warp = threadIdx.x >> 5;
   const int ksteps = p.D >> 4;
-  const int64_t n_tiles = (p.T + kTileMax - 1) / kTileMax;
-  const int64_t G = gridDim.x;
-  volatile int* abort = r.abort;
-  const uint16_t* wr_s = reinterpret_cast<const uint16_t*>(r.slots + (size_t)(L.n_slots - 1) * L.slot_bytes);
-  auto rows_of = [&](int64_t tile) {
-    const int64_t t0 = tile * kTileMax;
-    return (int)(p.T - t0 < kTileMax ? p.T - t0 : kTileMax);
+  const int n_tiles = (n_tok + kTileMax - 1) / kTileMax;
+  auto rows_of = [&](int t) {
+    const int left = n_tok - t * kTileMax;
+    return left < 0 ? 0 : (left < kTileMax ? left : kTileMax);
   };
-  auto load_pos_row = [&](int64_t t, int rr) {  // the list position of token 16 t + rr
-    return (t < n_tiles && rr < rows_of(t)) ? __ldg(w.tok_pos + t * kTileMax + rr) : -1;
-  };
-  auto load_pos = [&](int64_t t) { return load_pos_row(t, (int)threadIdx.x); };
+  for (int i = threadIdx.x; i < n_tok; i += kGroupCons * 32)
+    prefetch_l2(p.h + (int64_t)__ldg(tok + i) * p.D, (uint32_t)p.D * 2u);
   RouterA<KB> A;
-  int64_t tile = blockIdx.x;
-  // staged: thread r < 32 holds the list position of row r of the pair
-  // (tiles tile, tile + G); otherwise thread r < 16 that of row r of the tile
-  auto load_pair_pos = [&](int64_t t) {
-    return kStaged && threadIdx.x >= kTileMax ? load_pos_row(t + G, threadIdx.x - kTileMax) : load_pos(t);
-  };
-  int my_pos = load_pair_pos(tile);
-  if (!kStaged && tile < n_tiles) router_load_a<KB>(A, p.h, tile * kTileMax, rows_of(tile), p.D, warp);
-  // B fragments of k-steps warp + 8i: {Wr[d][j] | Wr[d+1][j] << 16, Wr[d+2][j] | Wr[d+3][j] << 16},
-  // d = 16 ks + 4c, j = 8 nt + g (the router kernels' k-slot order)
-  bool ok = consumers_wait(fs.wr_full, 0u, abort, p.err, fail);
+  if (n_tiles > 0) router_load_a_rows<KB>(A, p.h, tok, rows_of(0), p.D, warp);
+  const bool ok = consumers_wait(ls.wr_full, 0u, abort, p.err, fail);
+  // B fragments of k-steps warp + 8i, in the router kernels' k-slot order
   uint2 bw[KB][NT];
 #pragma unroll
   for (int i = 0; i < KB; ++i) {
     const int ks = warp + i * kWarps;
     if (ok && ks < ksteps) {
-      if (kExactN && p.N == 8 * NT)
+      if (kExactN && p.N == NP)
         wr_fragments<NT>(bw[i], wr_s, ks);
       else
         wr_fragments_any<NT>(bw[i], wr_s, ks, p.N);
@@ -1192,46 +1038,9 @@ __device__ void fused_router_phase(const GArgs& p, const GroupWs& w, const Smem&
     }
   }
   ConsumerSync{}();
-  if (threadIdx.x == 0) mbar_arrive(fs.wr_free);  // the Wr slot goes back to the ring
-  if constexpr (kStaged) {
-    // the CTA's tiles two at a time: both tiles' MMAs, then one finish
-    for (int j = 0; ok && tile < n_tiles; tile += 2 * G, j += 2) {
-      const bool two = tile + G < n_tiles;
-      ok = consumers_wait(&fs.h_full[j], 0u, abort, p.err, fail);
-      if (ok && two) ok = consumers_wait(&fs.h_full[j + 1], 0u, abort, p.err, fail);
-      if (!ok) break;
-      float acc0[NT][4], acc1[NT][4];
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        float (&acc)[NT][4] = u == 0 ? acc0 : acc1;
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-        if (u == 1 && !two) continue;
-        router_load_a_smem<KB>(A, r.slots + (size_t)(j + u) * L.slot_bytes, fs.h_pitch, rows_of(tile + u * G), p.D);
-#pragma unroll
-        for (int i = 0; i < KB; ++i) {
-          if (warp + i * kWarps < ksteps) {
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-              mma_16816(acc[nt], A.a0[i].x, A.a1[i].x, A.a0[i].y, A.a1[i].y, bw[i][nt].x, bw[i][nt].y);
-          }
-        }
-      }
-      ConsumerSync{}();  // the tiles' slots go back to the ring
-      if (threadIdx.x == 0) {
-        mbar_arrive(&fs.h_empty[j]);
-        if (two) mbar_arrive(&fs.h_empty[j + 1]);
-      }
-      pair_store_partials<NT>(ps, acc0, 0);
-      if (two) pair_store_partials<NT>(ps, acc1, kTileMax);
-      const int rows = two ? kTileMax + rows_of(tile + G) : rows_of(tile);
-      const int pos = my_pos;
-      my_pos = load_pair_pos(tile + 2 * G);
-      pair_finish<NT>(p, w, ps, rows, tile, tile + G, pos, fs.tf.flag, want);
-    }
-  }
-  for (; !kStaged && ok && tile < n_tiles; tile += G) {
-    float acc[NT][4];
+  if (ok && threadIdx.x == 0) mbar_arrive(ls.wr_free);  // Wr's slot goes back to the ring
+  if (!ok) return false;
+  auto mma_tile = [&](float (&acc)[NT][4]) {
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
 #pragma unroll
@@ -1242,69 +1051,91 @@ __device__ void fused_router_phase(const GArgs& p, const GroupWs& w, const Smem&
           mma_16816(acc[nt], A.a0[i].x, A.a1[i].x, A.a0[i].y, A.a1[i].y, bw[i][nt].x, bw[i][nt].y);
       }
     }
-    const int pos = my_pos;
-    my_pos = load_pos(tile + G);
-    if (tile + G < n_tiles) router_load_a<KB>(A, p.h, (tile + G) * kTileMax, rows_of(tile + G), p.D, warp);
-    fused_tile_finish<NT>(p, w, s, acc, tile, rows_of(tile), fs.tf.flag, want, pos);
+  };
+  for (int t = 0; t < n_tiles; t += 2) {
+    const bool two = t + 1 < n_tiles;
+    float acc[NT][4];
+    mma_tile(acc);
+    if (t + 1 < n_tiles) router_load_a_rows<KB>(A, p.h, tok + (t + 1) * kTileMax, rows_of(t + 1), p.D, warp);
+    pair_store_partials<NT>(ps, acc, 0);
+    if (two) {
+      mma_tile(acc);
+      if (t + 2 < n_tiles) router_load_a_rows<KB>(A, p.h, tok + (t + 2) * kTileMax, rows_of(t + 2), p.D, warp);
+      pair_store_partials<NT>(ps, acc, kTileMax);
+    }
+    ConsumerSync{}();
+    PairScratch pg = ps;
+    pg.gates = gl + (size_t)t * kTileMax * NP;
+    pair_softmax<NT>(pg, rows_of(t) + rows_of(t + 1), p.N);
+    ConsumerSync{}();
   }
-  if (!ok && threadIdx.x == 0) {  // the producer stops too (it may wait for a staged tile's slot)
-    *abort = 1;
-    atomicExch(fs.tf.abort_word, 1u);
-  }
+  return true;
 }
 
-template <int NT, bool kExactN, bool kStaged>
-__global__ void __launch_bounds__(kGroupThreads, 1) grouped_fused_kernel(const GArgs p, const GroupWs w,
-                                                                         const GroupLayout L) {
+constexpr uint32_t kWrChunk = 4096;  // bytes per bulk copy of Wr
+
+template <int NT, bool kExactN>
+__global__ void __launch_bounds__(kGroupThreads, 1) grouped_local_kernel(const GArgs p, const GroupWs w,
+                                                                         const GroupLayout L, int scap) {
   constexpr int NP = 8 * NT;
   extern __shared__ __align__(128) uint8_t smem_raw[];
-  Ring r = carve_ring(smem_raw, L);
-  r.q0 = L.n_slots - 1;  // the first item goes into Wr's slot
-  // router scratch after the ring: partial sums, gates and list positions of
-  // a tile (or, staged, of a pair of tiles)
+  const Ring r = carve_ring(smem_raw, L);
   uint8_t* scratch = smem_raw + (ring_bytes(L.n_slots, L.slot_bytes) + 127) / 128 * 128;
-  const Smem s = carve<false, NP>(scratch, p.D);
-  const PairScratch ps{reinterpret_cast<float*>(scratch),
-                       reinterpret_cast<float*>(scratch + (size_t)kWarps * kPairRows * NP * 4),
-                       reinterpret_cast<int*>(scratch + (size_t)(kWarps + 1) * kPairRows * NP * 4)};
-  __shared__ unsigned want_s;
+  const PairScratch ps{reinterpret_cast<float*>(scratch), nullptr, nullptr};       // partial sums
+  float* gl = reinterpret_cast<float*>(scratch + (size_t)kWarps * kPairRows * NP * 4);  // [scap][NP] gates
+  int* loff = reinterpret_cast<int*>(gl + (size_t)scap * NP);                       // [scap + 1]
   __shared__ int skip_s, fail_s;
-  __shared__ __align__(8) uint64_t bars[3 + 2 * kMaxStagedTiles];
-  const int64_t n_tiles = (p.T + kTileMax - 1) / kTileMax;
-  const int my_tiles = n_tiles > blockIdx.x ? (int)((n_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x) : 0;
-  const FusedSync fs{&bars[0], &bars[1], &bars[2], &bars[3], &bars[3 + kMaxStagedTiles], &want_s,
-                     TileFlags{w.tile_flag, reinterpret_cast<unsigned long long*>(&w.ctl[kCtlLaunches]),
-                               &w.ctl[kCtlAbort]},
-                     kStaged ? my_tiles : 0, 2 * p.D + 32};
+  __shared__ __align__(8) uint64_t bars[2];
+  const int b = blockIdx.x, lane = threadIdx.x & 31;
+  const bool producer = (threadIdx.x >> 5) == kGroupProducer;
+  uint8_t* wr_slot = r.slots + (size_t)(L.n_slots - 1) * L.slot_bytes;
+  const int* tok = w.share_tok + (size_t)b * scap;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 3; ++i) mbar_init(&bars[i], 1);
-    for (int j = 0; j < kMaxStagedTiles; ++j) {
-      mbar_init(&fs.h_full[j], 1);
-      mbar_init(&fs.h_empty[j], 1);
-    }
-    ring_init(r, L);  // (its fence covers all of them)
+    for (int i = 0; i < 2; ++i) mbar_init(&bars[i], 1);
+    ring_init(r, L, 2);  // full: the row block's copies, the token list
   }
+  __syncthreads();
   pdl_trigger();
   pdl_wait();  // the grouping and every earlier kernel are complete
+  if (producer) {
+    // Wr first (the router phase waits for it), in chunks taken in a
+    // CTA-dependent order so that the CTAs' requests spread over L2
+    const uint32_t wr_bytes = (uint32_t)p.N * (uint32_t)p.D * 2u;
+    const uint32_t n_ch = (wr_bytes + kWrChunk - 1) / kWrChunk;  // <= 16 (N <= 16, D <= 2048)
+    if (lane == 0) mbar_expect_tx(&bars[0], wr_bytes);
+    __syncwarp();
+    if ((uint32_t)lane < n_ch) {
+      const uint32_t off = ((lane + (uint32_t)b) % n_ch) * kWrChunk;
+      bulk_g2s(wr_slot + off, reinterpret_cast<const uint8_t*>(p.Wr) + off,
+               wr_bytes - off < kWrChunk ? wr_bytes - off : kWrChunk, &bars[0]);
+    }
+  }
+  // the CTA's counts (all threads), the control words (thread 0)
+  const int2 sn = reinterpret_cast<const int2*>(w.share_n)[b];
   if (threadIdx.x == 0) {
-    skip_s = ld_relaxed_u32(fs.tf.abort_word) != 0xFFFFFFFFu;  // plan abandoned
+    const unsigned ab = ld_relaxed_u32(&w.ctl[kCtlAbort]), grid = ld_relaxed_u32(&w.ctl[kCtlShareGrid]);
+    // plan abandoned (error word set): skip; shares for another CTA count: error
+    skip_s = ab != 0xFFFFFFFFu ? 1 : (grid != gridDim.x || sn.x < 0 || sn.y < 0 || sn.x > scap || sn.y > scap) ? 2 : 0;
+    if (skip_s == 2) atomicOr(p.err, kErrGrouping);
     fail_s = 0;
   }
   __syncthreads();
-  if (skip_s) return;
-  const int my_n = items_of_cta(w);
-  if ((threadIdx.x >> 5) == kGroupProducer) {
-    ring_producer<NP, false>(p, w, L, r, my_n, &fs);
+  if (skip_s) {
+    if (producer && lane == 0) mbar_drain(&bars[0], 0u);
+    return;
+  }
+  const int my_n = sn.x, n_tok = sn.y;
+  const LocalSync ls{&bars[0], &bars[1], w.share_rec + (size_t)b * scap};
+  if (producer) {
+    ring_producer<NP, false>(p, w, L, r, my_n, &ls);
   } else {
-    unsigned want = 0;
-    if (threadIdx.x == 0) {  // this launch's flag value (see TileFlags)
-      const unsigned long long before = atomicAdd(fs.tf.arrivals, 1ull) + 1ull;
-      want = (unsigned)(before / gridDim.x) + 1u;
-      want_s = want;
-      mbar_arrive(fs.epoch);
-    }
-    fused_router_phase<NT, kExactN, kStaged>(p, w, s, ps, r, L, fs, want, &fail_s);
-    ring_consumers<NT, kExactN, false>(p, L, r, my_n);
+    // step offsets into shared memory (my_n <= scap < the consumer threads);
+    // the router phase's first barrier orders them before their readers
+    if ((int)threadIdx.x <= my_n) loff[threadIdx.x] = __ldg(w.share_off + (size_t)b * (scap + 1) + threadIdx.x);
+    const bool ok = local_router_phase<NT, kExactN>(p, ps, reinterpret_cast<const uint16_t*>(wr_slot), ls, tok, n_tok,
+                                                    gl, r.abort, &fail_s);
+    if (!ok && threadIdx.x == 0) *r.abort = 1;  // the producer stops too
+    ring_consumers<NT, kExactN, false>(p, L, r, ok ? my_n : 0, gl, loff);
   }
   __syncthreads();
 }
@@ -1331,40 +1162,33 @@ GroupLayout group_layout(int N, int D, bool nf3) {
 }
 
 
-// The fused layer kernel (bf16 table, N <= 16, D <= 2048: a warp's k-steps
-// fit the kFusedKB fragments held in registers).
-template <int NT, bool kExactN, bool kStaged>
-mole_status launch_fused_as(const GArgs& p, const GroupWs& w, const GroupLayout& L, size_t smem, int n_sm,
-                            cudaStream_t stream) {
-  auto kern = grouped_fused_kernel<NT, kExactN, kStaged>;
+// The CTA-local layer kernel (bf16 table, N <= 16, D <= 2048: a warp's
+// k-steps fit kFusedKB), one CTA per SM, on the grouping's shares (built for
+// this SM count when share_cap < kShareCapLimit).
+template <int NT, bool kExactN>
+mole_status launch_local(const GArgs& p, const GroupWs& w, cudaStream_t stream) {
+  constexpr int NP = 8 * NT;
+  static_assert(NT <= 2, "the router phase holds B fragments of at most 16 experts");
+  // (the h rows' L2 prefetches need 16-byte aligned rows)
+  if (p.D > 16 * kWarps * kFusedKB || !aligned16(p.Wr) || !aligned16(p.h) || p.D % 8 != 0)
+    return MOLE_ERR_UNSUPPORTED;
+  const GroupLayout L = group_layout<NT>(p.N, p.D, false);
+  if (L.n_slots < 2 || (int64_t)p.N * p.D * 2 > L.slot_bytes) return MOLE_ERR_UNSUPPORTED;
+  const int n_sm = num_sms();
+  if (n_sm <= 0) return MOLE_ERR_NO_DEVICE;
+  if (!shares_apply(p.T, n_sm)) return MOLE_ERR_UNSUPPORTED;
+  const int64_t scap = share_cap(p.T, n_sm);
+  static_assert(kShareCapLimit <= kGroupCons * 32, "a consumer thread per step offset");
+  const size_t smem = (ring_bytes(L.n_slots, L.slot_bytes) + 127) / 128 * 128 + (size_t)kWarps * kPairRows * NP * 4 +
+                      (size_t)scap * NP * 4 + (size_t)(scap + 1) * 4;
+  if (smem > 227 * 1024) return MOLE_ERR_UNSUPPORTED;
+  auto kern = grouped_local_kernel<NT, kExactN>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return MOLE_ERR_CUDA;
   int occ = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kGroupThreads, smem) != cudaSuccess || occ < 1)
     return MOLE_ERR_UNSUPPORTED;
-  // one CTA per SM: all resident once the previous kernel's CTAs have left
-  return cuda_status(launch_pdl(kern, (unsigned)n_sm, kGroupThreads, smem, stream, p, w, L));
-}
-
-template <int NT, bool kExactN>
-mole_status launch_fused(const GArgs& p, const GroupWs& w, cudaStream_t stream) {
-  constexpr int NP = 8 * NT;
-  static_assert(NT <= 2, "Wr fragments of 32 experts do not fit the registers");
-  if (p.D > 16 * kWarps * kFusedKB || !aligned16(p.Wr)) return MOLE_ERR_UNSUPPORTED;
-  const GroupLayout L = group_layout<NT>(p.N, p.D, false);
-  if (L.n_slots < 2 || (int64_t)p.N * p.D * 2 > L.slot_bytes) return MOLE_ERR_UNSUPPORTED;
-  const size_t ring = (ring_bytes(L.n_slots, L.slot_bytes) + 127) / 128 * 128;
-  const size_t smem = ring + smem_bytes_for<false, NP>(p.D), smem_staged = ring + pair_scratch_bytes<NP>();
-  if (smem > 227 * 1024) return MOLE_ERR_UNSUPPORTED;
-  const int n_sm = num_sms();
-  if (n_sm <= 0) return MOLE_ERR_NO_DEVICE;
-  // staged router tiles: every CTA's tiles fit the slots other than Wr's
-  const int64_t per_cta = ((p.T + kTileMax - 1) / kTileMax + n_sm - 1) / n_sm;
-  const bool staged = per_cta <= std::min<int64_t>(kMaxStagedTiles, L.n_slots - 1) &&
-                      (int64_t)kTileMax * (2 * p.D + 32) <= L.slot_bytes && aligned16(p.h) &&
-                      smem_staged <= 227 * 1024;
-  return staged ? launch_fused_as<NT, kExactN, true>(p, w, L, smem_staged, n_sm, stream)
-                : launch_fused_as<NT, kExactN, false>(p, w, L, smem, n_sm, stream);
+  return cuda_status(launch_pdl(kern, (unsigned)n_sm, kGroupThreads, smem, stream, p, w, L, (int)scap));
 }
 
 template <int NT, bool kExactN, bool kNf3>
@@ -1372,7 +1196,7 @@ mole_status launch_layer(const GArgs& p, const GroupWs& w, cudaStream_t stream) 
   constexpr int NP = 8 * NT;
   if constexpr (!kNf3 && NT <= 2) {
     if (!router_tc_supported(p.T, p.N, p.D, p.h, p.Wr)) {
-      const mole_status st = launch_fused<NT, kExactN>(p, w, stream);
+      const mole_status st = launch_local<NT, kExactN>(p, w, stream);
       if (st != MOLE_ERR_UNSUPPORTED) return st;
     }
   }
@@ -1422,6 +1246,69 @@ bool grouped_applies(int64_t T, int N, int D, bool nf3) {
   if (nf3 && (D % 64 != 0 || ((int64_t)N * (D / 64)) % 8 != 0)) return false;
   const GroupLayout L = group_layout<4>(N, D, nf3);  // the widest gate area
   return L.n_slots >= 2 && smem_bytes_for<true, 32>(D) <= 227 * 1024;
+}
+
+// ---- Shares: each layer-kernel CTA's work items and tokens (once per batch) ----
+// One warp per CTA b of a G-CTA layer kernel: b's item records in processing
+// order (cta_item), each step's token offset and the items' tokens in order,
+// so that the CTA reads all of them in one round of loads.  Runs after
+// group_plan_kernel; skipped if the plan was abandoned.
+constexpr int kShareWarps = 4;
+
+__global__ void __launch_bounds__(kShareWarps * 32) group_share_kernel(const GroupWs w, int G, int scap) {
+  __shared__ int soff[kShareWarps][kShareCapLimit + 1];
+  __shared__ int spos[kShareWarps][kShareCapLimit];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.x * kShareWarps + warp;
+  if (blockIdx.x == 0 && threadIdx.x == 0) w.ctl[kCtlShareGrid] = (unsigned)G;
+  if (b >= G || ld_relaxed_u32(&w.ctl[kCtlAbort]) != 0xFFFFFFFFu) return;
+  const int my_n = items_of((int)ld_relaxed_u32(&w.ctl[kCtlItems]), b, G);
+  int* so = soff[warp];
+  int* sp = spos[warp];
+  auto over = [&]() {  // beyond the capacity bound (not reached: see share_cap)
+    if (lane == 0) {
+      w.share_n[2 * b] = -1;
+      w.share_n[2 * b + 1] = -1;
+    }
+  };
+  if (my_n > scap) return over();
+  int run = 0;
+  for (int k0 = 0; k0 < my_n; k0 += 32) {
+    const int k = k0 + lane;
+    const int4 rec = k < my_n ? w.items[cta_item(k, my_n, b, G)] : make_int4(0, 0, 0, 0);
+    int inc = rec.z;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += v;
+    }
+    if (k < my_n) {
+      w.share_rec[(size_t)b * scap + k] = rec;
+      so[k + 1] = run + inc;
+      sp[k] = rec.y;
+    }
+    run += __shfl_sync(0xffffffffu, inc, 31);
+  }
+  if (lane == 0) so[0] = 0;
+  __syncwarp();
+  const int n_tok = run;
+  if (n_tok > scap) return over();
+  for (int k = lane; k <= my_n; k += 32) w.share_off[(size_t)b * (scap + 1) + k] = so[k];
+  for (int i = lane; i < n_tok; i += 32) {
+    int lo = 0, hi = my_n;  // the step k with so[k] <= i < so[k + 1]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (so[mid] <= i)
+        lo = mid;
+      else
+        hi = mid;
+    }
+    w.share_tok[(size_t)b * scap + i] = w.list[sp[lo] + (i - so[lo])];
+  }
+  if (lane == 0) {
+    w.share_n[2 * b] = my_n;
+    w.share_n[2 * b + 1] = n_tok;
+  }
 }
 
 // ---- Offloaded table: the batch's distinct row blocks into a staging buffer ----
@@ -1681,6 +1568,12 @@ mole_status token_groups_build(const int32_t* ids, int64_t T, int64_t V, int N, 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, group_plan_kernel, ids, T, V, w, err) != cudaSuccess) return MOLE_ERR_CUDA;
+  // the shares of a one-CTA-per-SM layer kernel on this device
+  if (shares_apply(T, n_sm)) {
+    group_share_kernel<<<(n_sm + kShareWarps - 1) / kShareWarps, kShareWarps * 32, 0, stream>>>(
+        w, n_sm, (int)share_cap(T, n_sm));
+    if (cudaGetLastError() != cudaSuccess) return MOLE_ERR_CUDA;
+  }
   return MOLE_OK;
 }
 

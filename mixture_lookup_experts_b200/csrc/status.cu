@@ -80,5 +80,6 @@ extern "C" mole_status mole_check(cudaStream_t stream, int timeout_ms) {
   if (cudaStreamSynchronize(stream) != cudaSuccess) return MOLE_ERR_CUDA;
   if (v & mole::kErrTimeout) return MOLE_ERR_TIMEOUT;
   if (v & mole::kErrIndex) return MOLE_ERR_INDEX;
+  if (v & mole::kErrGrouping) return MOLE_ERR_ARG;
   return MOLE_OK;
 }

@@ -15,8 +15,9 @@
 //   out[t] = sum_j g_j(h[t]) Y[u(t), j]                   (the combine kernels)
 // Backward of L with dL/dout = dout (all gradients accumulated, fp32):
 //   g, dg_j = <dout[t], Y[u(t), j]>, dz = g (dg - <g, dg>)
-//   dh[t] += dz[t] . Wr^T,  dWr += h^T dz                 (gate_grad_kernel, dwr_kernel)
-//   dY[u, j] = sum_{t: u(t) = u} g_j[t] dout[t]           (dy_kernel over the grouping's items)
+//   dh[t] += dz[t] . Wr^T,  dWr += h^T dz                 (gate_grad_kernel; dwr_kernel per
+//                                                          block of tokens, then dwr_reduce_kernel)
+//   dY[u, j] = sum_{t: u(t) = u} g_j[t] dout[t]           (dy_kernel, one CTA per distinct id)
 //   dpre_j = (dY_j . W2_j^T) * act'(pre_j)                (cuBLAS + act_grad_kernel)
 //   dW2_j += H_j^T dY_j,  dW1_j += Eu^T dpre_j,  dE[ids] += sum_j dpre_j . W1_j^T
 //                                                         (cuBLAS batched over the experts,
@@ -31,6 +32,7 @@ namespace mole {
 namespace {
 
 constexpr int kGradThreads = 256;
+constexpr int kDwrTokens = 256;  // tokens per block of dwr_kernel
 constexpr int64_t kCublasWorkspace = int64_t(32) << 20;
 
 // The caller's cache buffer (cap = min(T, V) row capacity).
@@ -45,6 +47,7 @@ struct TrainCache {
   uint16_t* dYb;  // [cap, N, D] bf16
   uint16_t* dP;   // [N, cap, Dr] bf16: dL/dpre (first dL/dH)
   float* dEu;     // [N, cap, D] fp32: each expert's share of dL/dEu
+  float* dWrp;    // [ceil(T / kDwrTokens), D, N] fp32: dWr per block of tokens
   void* blas_ws;  // cuBLAS workspace
   int* U;         // one device int
   size_t total;
@@ -68,6 +71,7 @@ size_t carve_cache(void* base, int64_t T, int64_t V, int N, int64_t D, int64_t D
   const size_t o_dyb = take(2 * (size_t)cap * N * D);
   const size_t o_dp = take(2 * (size_t)N * cap * Dr);
   const size_t o_deu = take(4 * (size_t)N * cap * D);
+  const size_t o_dwr = take(4 * (size_t)((T + kDwrTokens - 1) / kDwrTokens) * D * N);
   const size_t o_ws = take((size_t)kCublasWorkspace);
   const size_t o_u = take(16);
   if (c != nullptr && base != nullptr) {
@@ -82,6 +86,7 @@ size_t carve_cache(void* base, int64_t T, int64_t V, int N, int64_t D, int64_t D
     c->dYb = reinterpret_cast<uint16_t*>(b + o_dyb);
     c->dP = reinterpret_cast<uint16_t*>(b + o_dp);
     c->dEu = reinterpret_cast<float*>(b + o_deu);
+    c->dWrp = reinterpret_cast<float*>(b + o_dwr);
     c->blas_ws = b + o_ws;
     c->U = reinterpret_cast<int*>(b + o_u);
     c->total = off;
@@ -192,14 +197,12 @@ __global__ void __launch_bounds__(kGradThreads) gate_grad_kernel(const GroupWs w
   }
 }
 
-// dWr[d, j] += sum_t h[t, d] dz[t, j]: a thread per d of its block's 256,
-// over its block's range of tokens; one atomic add per (d, j) per block.
-constexpr int kDwrTokens = 256;
-
+// dWr over a block of kDwrTokens tokens: part[blockIdx.y][d][j] = sum over
+// the block's tokens t (in order) of h[t, d] dz[t, j]; a thread per d.
 template <int NP>
 __global__ void __launch_bounds__(kGradThreads) dwr_kernel(const GroupWs w, const uint16_t* __restrict__ h,
                                                            const float* __restrict__ dz, int64_t T, int N, int D,
-                                                           float* dWr) {
+                                                           float* part) {
   __shared__ float dzs[kDwrTokens][NP];
   const int d = blockIdx.x * kGradThreads + threadIdx.x;
   const int64_t t0 = (int64_t)blockIdx.y * kDwrTokens;
@@ -218,34 +221,85 @@ __global__ void __launch_bounds__(kGradThreads) dwr_kernel(const GroupWs w, cons
 #pragma unroll
     for (int j = 0; j < NP; ++j) acc[j] = fmaf(hv, dzs[r][j], acc[j]);
   }
+  float* o = part + ((int64_t)blockIdx.y * D + d) * N;
 #pragma unroll
   for (int j = 0; j < NP; ++j)
-    if (j < N) atomicAdd(dWr + (int64_t)d * N + j, acc[j]);
+    if (j < N) o[j] = acc[j];
 }
 
-// dY[u, j, :] += sum over the item's tokens of g[t, j] dout[t, :]: one CTA per
-// work item (up to 16 tokens of one id); items of the same id add atomically.
+// dWr[i] += sum over the token blocks, in order, of part[b][i] (i = d N + j).
+__global__ void dwr_reduce_kernel(const float* __restrict__ part, int n_blocks, int64_t n, float* dWr) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    float acc = 0.f;
+    for (int b = 0; b < n_blocks; ++b) acc += part[(int64_t)b * n + i];
+    dWr[i] += acc;
+  }
+}
+
+// dY[u, j, d] = sum over the tokens t of id u, in list order, of
+// g[t, j] dout[t, d].  Work unit = (work item, slice of kGradThreads
+// consecutive d); only units of an id's first work item do work, over all of
+// the id's tokens, so the sums do not depend on scheduling and a frequent id
+// spreads over D / kGradThreads CTAs.  A thread holds the N sums of its d;
+// tokens pass through shared memory kDyChunk at a time.  Every distinct id's
+// rows are written (no clearing needed).
+constexpr int kDyChunk = 64;
+
+template <int NP>
 __global__ void __launch_bounds__(kGradThreads) dy_kernel(const GroupWs w, const float* __restrict__ g,
                                                           const float* __restrict__ dout, int N, int D, float* dY) {
-  __shared__ int toks[kItemTokens];
-  __shared__ float gs[kItemTokens][32];
+  __shared__ int toks[kDyChunk];
+  __shared__ float gs[kDyChunk][NP];
+  __shared__ int cnt_s;
   const int n_items = (int)ld_relaxed_u32(&w.ctl[kCtlItems]);
-  for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+  const int n_slices = (D + kGradThreads - 1) / kGradThreads;
+  const int64_t n_units = (int64_t)n_items * n_slices;
+  for (int64_t unit = blockIdx.x; unit < n_units; unit += gridDim.x) {
+    const int it = (int)(unit / n_slices), sl = (int)(unit - (int64_t)it * n_slices);
     const int4 rec = w.items[it];  // {id, first list position, tokens, dense index}
+    // the id's first item starts its range of the list (uniform over the CTA)
+    if (rec.y > 0 && w.tok_uid[w.list[rec.y - 1]] == rec.w) continue;
+    __syncthreads();  // the previous unit's readers of cnt_s, toks and gs are done
+    if (threadIdx.x == 0) cnt_s = w.cnt[w.tok_slot[w.list[rec.y]]] + 1;
     __syncthreads();
-    if (threadIdx.x < rec.z) toks[threadIdx.x] = w.list[rec.y + threadIdx.x];
-    __syncthreads();
-    for (int i = threadIdx.x; i < rec.z * N; i += kGradThreads) {
-      const int k = i / N, j = i - k * N;
-      gs[k][j] = g[(int64_t)toks[k] * N + j];
+    const int c = cnt_s;
+    const int d = sl * kGradThreads + threadIdx.x;
+    float acc[NP];
+#pragma unroll
+    for (int j = 0; j < NP; ++j) acc[j] = 0.f;
+    for (int k0 = 0; k0 < c; k0 += kDyChunk) {
+      const int n = c - k0 < kDyChunk ? c - k0 : kDyChunk;
+      if (k0 > 0) __syncthreads();  // the previous chunk's readers are done
+      if (threadIdx.x < n) toks[threadIdx.x] = w.list[rec.y + k0 + threadIdx.x];
+      __syncthreads();
+      for (int i = threadIdx.x; i < n * NP; i += kGradThreads) {
+        const int k = i / NP, j = i - k * NP;
+        gs[k][j] = j < N ? g[(int64_t)toks[k] * N + j] : 0.f;
+      }
+      __syncthreads();
+      if (d < D) {
+        int k = 0;
+        for (; k + 4 <= n; k += 4) {  // four tokens' loads in flight
+          float x[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) x[q] = dout[(int64_t)toks[k + q] * D + d];
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+#pragma unroll
+            for (int j = 0; j < NP; ++j) acc[j] = fmaf(gs[k + q][j], x[q], acc[j]);
+        }
+        for (; k < n; ++k) {
+          const float x = dout[(int64_t)toks[k] * D + d];
+#pragma unroll
+          for (int j = 0; j < NP; ++j) acc[j] = fmaf(gs[k][j], x, acc[j]);
+        }
+      }
     }
-    __syncthreads();
-    float* dst = dY + (int64_t)rec.w * N * D;
-    for (int e = threadIdx.x; e < N * D; e += kGradThreads) {
-      const int j = e / D, d = e - j * D;
-      float acc = 0.f;
-      for (int k = 0; k < rec.z; ++k) acc = fmaf(gs[k][j], dout[(int64_t)toks[k] * D + d], acc);
-      atomicAdd(dst + e, acc);
+    if (d < D) {
+      float* dst = dY + (int64_t)rec.w * N * D + d;
+#pragma unroll
+      for (int j = 0; j < NP; ++j)
+        if (j < N) dst[(int64_t)j * D] = acc[j];
     }
   }
 }
@@ -366,18 +420,23 @@ mole_status train_backward(const void* groups, size_t gbytes, int64_t T, const v
   if (dWr != nullptr) {
     const dim3 gw((unsigned)((D + kGradThreads - 1) / kGradThreads), (unsigned)((T + kDwrTokens - 1) / kDwrTokens));
     if (N <= 8)
-      dwr_kernel<8><<<gw, kGradThreads, 0, stream>>>(w, h16, c.dz, T, N, (int)D, dWr);
+      dwr_kernel<8><<<gw, kGradThreads, 0, stream>>>(w, h16, c.dz, T, N, (int)D, c.dWrp);
     else if (N <= 16)
-      dwr_kernel<16><<<gw, kGradThreads, 0, stream>>>(w, h16, c.dz, T, N, (int)D, dWr);
+      dwr_kernel<16><<<gw, kGradThreads, 0, stream>>>(w, h16, c.dz, T, N, (int)D, c.dWrp);
     else
-      dwr_kernel<32><<<gw, kGradThreads, 0, stream>>>(w, h16, c.dz, T, N, (int)D, dWr);
+      dwr_kernel<32><<<gw, kGradThreads, 0, stream>>>(w, h16, c.dz, T, N, (int)D, c.dWrp);
+    dwr_reduce_kernel<<<grid_for(D * N, 256), 256, 0, stream>>>(c.dWrp, (int)gw.y, D * N, dWr);
     if (cudaGetLastError() != cudaSuccess) return MOLE_ERR_CUDA;
   }
   if (U == 0 || (dE == nullptr && dW1 == nullptr && dW2 == nullptr)) return MOLE_OK;
-  // dY by the grouping's items, then its bf16 copy for the GEMMs
+  // dY by distinct id, then its bf16 copy for the GEMMs
   const int64_t ny = (int64_t)U * N * D;
-  if (cudaMemsetAsync(c.dY, 0, ny * 4, stream) != cudaSuccess) return MOLE_ERR_CUDA;
-  dy_kernel<<<(unsigned)n_sm * 4, kGradThreads, 0, stream>>>(w, c.g, dout, N, (int)D, c.dY);
+  if (N <= 8)
+    dy_kernel<8><<<(unsigned)n_sm * 4, kGradThreads, 0, stream>>>(w, c.g, dout, N, (int)D, c.dY);
+  else if (N <= 16)
+    dy_kernel<16><<<(unsigned)n_sm * 4, kGradThreads, 0, stream>>>(w, c.g, dout, N, (int)D, c.dY);
+  else
+    dy_kernel<32><<<(unsigned)n_sm * 4, kGradThreads, 0, stream>>>(w, c.g, dout, N, (int)D, c.dY);
   to_bf16_kernel<<<grid_for(ny, 256), 256, 0, stream>>>(c.dY, c.dYb, ny);
   if (cudaGetLastError() != cudaSuccess) return MOLE_ERR_CUDA;
   cublasHandle_t hb = blas_handle();

@@ -43,6 +43,8 @@ def _both(mole, ids, h, Wr, lut):
     (128, 64, 32, 2048, "zipf"),       # 32 experts
     (64, 2048, 32, 1030, "uniform"),   # 128 KB row blocks: no ring fits, ungrouped kernels
     (777, 256, 16, 333, "zipf"),       # below the grouping threshold: ungrouped kernels
+    (20000, 128, 16, 14080, "zipf"),   # largest batch of the CTA-local kernel (16 experts)
+    (5000, 64, 8, 40000, "zipf"),      # too many tokens per SM for the CTA-local kernel
 ])
 def test_grouped_matches_oracle_and_ungrouped(mole, oracle_mod, V, D, N, T, kind):
     ids, h, Wr, lut = _layer(300 + D + N + T, V, D, N, T, kind)
