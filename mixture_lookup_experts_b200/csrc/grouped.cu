@@ -992,15 +992,8 @@ __device__ __forceinline__ void router_load_a_rows(RouterA<KB>& A, const uint16_
   }
 }
 
-// One bulk prefetch of `bytes` at p (16-byte aligned, a multiple of 16) into L2.
-__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
 // Consumer warps: the gates of the CTA's n_tok listed tokens (tok[i]) into
-// gl[n_tok][NP].  Every listed token's h row is first requested into L2 (one
-// bulk prefetch per row); the first tile's A fragments load while Wr
-// arrives; each warp then takes the B fragments of its k-steps into
+// gl[n_tok][NP].  The first tile's A fragments load while Wr arrives; each warp then takes the B fragments of its k-steps into
 // registers and Wr's slot goes back to the ring.  The tiles' A fragments
 // load one tile at a time, the next right after the current tile's MMAs;
 // two tiles share one partial-sum exchange and softmax.  Returns false
@@ -1017,8 +1010,6 @@ __device__ bool local_router_phase(const GArgs& p, const PairScratch& ps, const 
     const int left = n_tok - t * kTileMax;
     return left < 0 ? 0 : (left < kTileMax ? left : kTileMax);
   };
-  for (int i = threadIdx.x; i < n_tok; i += kGroupCons * 32)
-    prefetch_l2(p.h + (int64_t)__ldg(tok + i) * p.D, (uint32_t)p.D * 2u);
   RouterA<KB> A;
   if (n_tiles > 0) router_load_a_rows<KB>(A, p.h, tok, rows_of(0), p.D, warp);
   const bool ok = consumers_wait(ls.wr_full, 0u, abort, p.err, fail);
@@ -1169,9 +1160,7 @@ template <int NT, bool kExactN>
 mole_status launch_local(const GArgs& p, const GroupWs& w, cudaStream_t stream) {
   constexpr int NP = 8 * NT;
   static_assert(NT <= 2, "the router phase holds B fragments of at most 16 experts");
-  // (the h rows' L2 prefetches need 16-byte aligned rows)
-  if (p.D > 16 * kWarps * kFusedKB || !aligned16(p.Wr) || !aligned16(p.h) || p.D % 8 != 0)
-    return MOLE_ERR_UNSUPPORTED;
+  if (p.D > 16 * kWarps * kFusedKB || !aligned16(p.Wr)) return MOLE_ERR_UNSUPPORTED;
   const GroupLayout L = group_layout<NT>(p.N, p.D, false);
   if (L.n_slots < 2 || (int64_t)p.N * p.D * 2 > L.slot_bytes) return MOLE_ERR_UNSUPPORTED;
   const int n_sm = num_sms();
