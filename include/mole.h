@@ -149,15 +149,19 @@ mole_status mole_lookup_combine(const int32_t* ids, int64_t T, const void* h, co
  * contents are opaque; the grouping stays valid until the buffer is rebuilt.
  * Ids outside [0, V) are left out of every group and set the device error
  * word (MOLE_ERR_INDEX).  One cooperative kernel launch (all of its CTAs
- * resident at once).
+ * resident at once), then one plain launch that lists each SM's share of the
+ * work for the per-layer kernels; the grouping therefore belongs to the
+ * device it was built on (a layer call on a device with another SM count
+ * writes no output and mole_check reports MOLE_ERR_ARG).
  *
  * mole_lookup_combine_groups is mole_lookup_combine (same arguments, layouts,
  * results bit for bit, and error behaviour) for a batch whose grouping was
  * built from the same ids, T and N: each distinct id's row block is read once
- * and applied to all of that id's tokens.  The call also writes one layer's
- * gates into `groups`, so calls that share a groups buffer must not overlap
- * on the GPU.  The grouped kernels serve bf16 inputs with T >= 1024; other
- * calls run the mole_lookup_combine kernels (the grouping is then unused).
+ * and applied to all of that id's tokens.  The call may also write one
+ * layer's gates into `groups`, so calls that share a groups buffer must not
+ * overlap on the GPU.  The grouped kernels serve bf16 inputs with T >= 1024;
+ * other calls run the mole_lookup_combine kernels (the grouping is then
+ * unused).
  *
  * mole_lookup_combine_grouped builds the grouping in `workspace` and runs
  * mole_lookup_combine_groups, for a single layer;
