@@ -26,9 +26,10 @@
 //     their tokens (its share).
 //  Per layer, batches too small for the tensor-core router (fewer 128-token
 //  tiles than about 3/4 of the SMs):
-//  2. grouped_local_kernel (one CTA per SM, 9 warps): each CTA computes the
-//     gates of its own share's tokens (mma.sync router, gates kept in shared
-//     memory), then gathers and combines its work items as in 3.
+//  2. grouped_local_kernel (one CTA per SM, 9 warps; bf16 or NF3 table):
+//     each CTA computes the gates of its own share's tokens (mma.sync router,
+//     gates kept in shared memory), then gathers and combines its work items
+//     as in 3.
 //  Per layer, otherwise:
 //  2. the router: router_tc.cu's tcgen05 kernel for 16 experts, else
 //     router_group_kernel (persistent, 2 CTAs per SM, the mma.sync router of
@@ -548,14 +549,23 @@ __device__ __forceinline__ void ring_init(const Ring& r, const GroupLayout& L, i
 }
 
 // The CTA-local layer kernel's router input Wr arrives by bulk copies in the
-// ring's last slot W (wr_full) and goes back to the ring once every consumer
-// warp holds its B fragments in registers (wr_free).  The CTA's work item
-// records come from its share, in processing order.
+// ring's last slots wr_slot0 .. n_slots-1 (one slot of a bf16 table; the
+// smaller slots of an NF3 table take several) (wr_full) and goes back to the
+// ring once every consumer warp holds its B fragments in registers
+// (wr_free).  The CTA's work item records come from its share, in
+// processing order.
 struct LocalSync {
   uint64_t* wr_full;
   uint64_t* wr_free;
   const int4* recs;  // [my_n]
+  int wr_slot0;
 };
+
+// Ring slots that hold Wr in the CTA-local kernel: the last ones, as many as
+// its N * D bf16 values need.
+__host__ __device__ __forceinline__ int wr_slots(const GroupLayout& L, int N, int D) {
+  return (int)(((int64_t)N * D * 2 + L.slot_bytes - 1) / L.slot_bytes);
+}
 
 // Ring position of the CTA's k-th work item: slot k mod n_slots, in lap
 // k / n_slots.
@@ -594,7 +604,8 @@ __device__ __forceinline__ int items_of_cta(const GroupWs& w) {
 // and (grouped_gather_kernel) its tokens' gates into the item's slot, then
 // the token list.  With `ls` (CTA-local kernel, gates in shared memory) the
 // records come from the CTA's share, the row blocks of the first items go
-// out at once (slot W's once Wr is no longer needed there), and the warp
+// out at once (those of Wr's slots once Wr is no longer needed there), and
+// the warp
 // also writes the
 // NaN output rows of the bad-id tokens in its CTA's slice of the batch.
 template <int NP, bool kNf3>
@@ -639,7 +650,6 @@ __device__ void ring_producer(const GArgs& p, const GroupWs& w, const GroupLayou
   bool ok = true;
   int pre = 0;  // items whose row blocks went out ahead of the main loop
   if (ls != nullptr) {
-    const uint32_t W = (uint32_t)L.n_slots - 1u;
     const int first = my_n < L.n_slots ? my_n : L.n_slots;  // n_slots <= 16 < 32: all in my_item
     for (int k = 0; k < first; ++k) {
       const int row = __shfl_sync(0xffffffffu, p.by_uid ? my_item.w : my_item.x, k);
@@ -648,7 +658,7 @@ __device__ void ring_producer(const GArgs& p, const GroupWs& w, const GroupLayou
         break;
       }
       const uint32_t q = ring_slot(r, L, k);
-      if (q == W && !warp_wait(ls->wr_free, 0u, abort, p.err)) {
+      if ((int)q >= ls->wr_slot0 && !warp_wait(ls->wr_free, 0u, abort, p.err)) {
         ok = false;
         break;
       }
@@ -1065,7 +1075,7 @@ __device__ bool local_router_phase(const GArgs& p, const PairScratch& ps, const 
 
 constexpr uint32_t kWrChunk = 4096;  // bytes per bulk copy of Wr
 
-template <int NT, bool kExactN>
+template <int NT, bool kExactN, bool kNf3>
 __global__ void __launch_bounds__(kGroupThreads, 1) grouped_local_kernel(const GArgs p, const GroupWs w,
                                                                          const GroupLayout L, int scap) {
   constexpr int NP = 8 * NT;
@@ -1079,7 +1089,8 @@ __global__ void __launch_bounds__(kGroupThreads, 1) grouped_local_kernel(const G
   __shared__ __align__(8) uint64_t bars[2];
   const int b = blockIdx.x, lane = threadIdx.x & 31;
   const bool producer = (threadIdx.x >> 5) == kGroupProducer;
-  uint8_t* wr_slot = r.slots + (size_t)(L.n_slots - 1) * L.slot_bytes;
+  const int wr_slot0 = L.n_slots - wr_slots(L, p.N, p.D);
+  uint8_t* wr_slot = r.slots + (size_t)wr_slot0 * L.slot_bytes;
   const int* tok = w.share_tok + (size_t)b * scap;
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) mbar_init(&bars[i], 1);
@@ -1116,9 +1127,9 @@ __global__ void __launch_bounds__(kGroupThreads, 1) grouped_local_kernel(const G
     return;
   }
   const int my_n = sn.x, n_tok = sn.y;
-  const LocalSync ls{&bars[0], &bars[1], w.share_rec + (size_t)b * scap};
+  const LocalSync ls{&bars[0], &bars[1], w.share_rec + (size_t)b * scap, wr_slot0};
   if (producer) {
-    ring_producer<NP, false>(p, w, L, r, my_n, &ls);
+    ring_producer<NP, kNf3>(p, w, L, r, my_n, &ls);
   } else {
     // step offsets into shared memory (my_n <= scap < the consumer threads);
     // the router phase's first barrier orders them before their readers
@@ -1126,7 +1137,7 @@ __global__ void __launch_bounds__(kGroupThreads, 1) grouped_local_kernel(const G
     const bool ok = local_router_phase<NT, kExactN>(p, ps, reinterpret_cast<const uint16_t*>(wr_slot), ls, tok, n_tok,
                                                     gl, r.abort, &fail_s);
     if (!ok && threadIdx.x == 0) *r.abort = 1;  // the producer stops too
-    ring_consumers<NT, kExactN, false>(p, L, r, ok ? my_n : 0, gl, loff);
+    ring_consumers<NT, kExactN, kNf3>(p, L, r, ok ? my_n : 0, gl, loff);
   }
   __syncthreads();
 }
@@ -1153,16 +1164,16 @@ GroupLayout group_layout(int N, int D, bool nf3) {
 }
 
 
-// The CTA-local layer kernel (bf16 table, N <= 16, D <= 2048: a warp's
-// k-steps fit kFusedKB), one CTA per SM, on the grouping's shares (built for
-// this SM count when share_cap < kShareCapLimit).
-template <int NT, bool kExactN>
+// The CTA-local layer kernel (bf16 or NF3 table, N <= 16, D <= 2048: a
+// warp's k-steps fit kFusedKB), one CTA per SM, on the grouping's shares
+// (built for this SM count when share_cap < kShareCapLimit).
+template <int NT, bool kExactN, bool kNf3>
 mole_status launch_local(const GArgs& p, const GroupWs& w, cudaStream_t stream) {
   constexpr int NP = 8 * NT;
   static_assert(NT <= 2, "the router phase holds B fragments of at most 16 experts");
   if (p.D > 16 * kWarps * kFusedKB || !aligned16(p.Wr)) return MOLE_ERR_UNSUPPORTED;
-  const GroupLayout L = group_layout<NT>(p.N, p.D, false);
-  if (L.n_slots < 2 || (int64_t)p.N * p.D * 2 > L.slot_bytes) return MOLE_ERR_UNSUPPORTED;
+  const GroupLayout L = group_layout<NT>(p.N, p.D, kNf3);
+  if (L.n_slots < 2 || wr_slots(L, p.N, (int)p.D) >= L.n_slots) return MOLE_ERR_UNSUPPORTED;
   const int n_sm = num_sms();
   if (n_sm <= 0) return MOLE_ERR_NO_DEVICE;
   if (!shares_apply(p.T, n_sm)) return MOLE_ERR_UNSUPPORTED;
@@ -1171,7 +1182,7 @@ mole_status launch_local(const GArgs& p, const GroupWs& w, cudaStream_t stream) 
   const size_t smem = (ring_bytes(L.n_slots, L.slot_bytes) + 127) / 128 * 128 + (size_t)kWarps * kPairRows * NP * 4 +
                       (size_t)scap * NP * 4 + (size_t)(scap + 1) * 4;
   if (smem > 227 * 1024) return MOLE_ERR_UNSUPPORTED;
-  auto kern = grouped_local_kernel<NT, kExactN>;
+  auto kern = grouped_local_kernel<NT, kExactN, kNf3>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return MOLE_ERR_CUDA;
   int occ = 0;
@@ -1183,9 +1194,9 @@ mole_status launch_local(const GArgs& p, const GroupWs& w, cudaStream_t stream) 
 template <int NT, bool kExactN, bool kNf3>
 mole_status launch_layer(const GArgs& p, const GroupWs& w, cudaStream_t stream) {
   constexpr int NP = 8 * NT;
-  if constexpr (!kNf3 && NT <= 2) {
+  if constexpr (NT <= 2) {
     if (!router_tc_supported(p.T, p.N, p.D, p.h, p.Wr)) {
-      const mole_status st = launch_local<NT, kExactN>(p, w, stream);
+      const mole_status st = launch_local<NT, kExactN, kNf3>(p, w, stream);
       if (st != MOLE_ERR_UNSUPPORTED) return st;
     }
   }
