@@ -548,17 +548,28 @@ __device__ __forceinline__ void ring_init(const Ring& r, const GroupLayout& L, i
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
-// The CTA-local layer kernel's router input Wr arrives by bulk copies in the
-// ring's last slots wr_slot0 .. n_slots-1 (one slot of a bf16 table; the
+// The CTA-local layer kernel's router inputs.  Wr arrives by bulk copies in
+// the ring's last slots wr_slot0 .. n_slots-1 (one slot of a bf16 table; the
 // smaller slots of an NF3 table take several) (wr_full) and goes back to the
 // ring once every consumer warp holds its B fragments in registers
-// (wr_free).  The CTA's work item records come from its share, in
-// processing order.
+// (wr_free).  Where the slots before them can hold a 16-token tile of h rows
+// (pitch bytes apart), the router tiles stream through those staging slots
+// st_slot0 .. wr_slot0-1 one at a time, one bulk copy per row (h_full, one
+// phase per tile), each released once its MMAs are done (h_empty); after
+// the last tile they go back to the ring.  The CTA's work item records and
+// tokens come from its share, in processing order.
 struct LocalSync {
   uint64_t* wr_full;
   uint64_t* wr_free;
+  uint64_t* h_full;
+  uint64_t* h_empty;
   const int4* recs;  // [my_n]
+  const int* tok;    // [n_tok]
   int wr_slot0;
+  int st_slot0;      // == wr_slot0: no staging slots (A fragments from global memory)
+  int n_st;          // router tiles staged (all of them, or none)
+  int n_tok;
+  int pitch;
 };
 
 // Ring slots that hold Wr in the CTA-local kernel: the last ones, as many as
@@ -610,7 +621,7 @@ __device__ __forceinline__ int items_of_cta(const GroupWs& w) {
 // NaN output rows of the bad-id tokens in its CTA's slice of the batch.
 template <int NP, bool kNf3>
 __device__ void ring_producer(const GArgs& p, const GroupWs& w, const GroupLayout& L, const Ring& r, int my_n,
-                              const LocalSync* ls) {
+                              const LocalSync* ls, int tok0 = 0) {
   constexpr int C = kItemTokens;
   const int lane = threadIdx.x & 31;
   volatile int* abort = r.abort;
@@ -649,31 +660,71 @@ __device__ void ring_producer(const GArgs& p, const GroupWs& w, const GroupLayou
   int4 nx_item = record(32 + lane);
   bool ok = true;
   int pre = 0;  // items whose row blocks went out ahead of the main loop
+  int staged = 0;  // router tiles whose h rows went out
   if (ls != nullptr) {
-    const int first = my_n < L.n_slots ? my_n : L.n_slots;  // n_slots <= 16 < 32: all in my_item
-    for (int k = 0; k < first; ++k) {
-      const int row = __shfl_sync(0xffffffffu, p.by_uid ? my_item.w : my_item.x, k);
-      if (bad_row(row)) {
-        ok = false;
-        break;
+    // router tile t's h rows into the staging slots, lane r copying row r
+    // (its token id tk)
+    uint8_t* stage = r.slots + (size_t)ls->st_slot0 * L.slot_bytes;
+    const uint32_t h_row = (uint32_t)p.D * 2u;
+    auto stage_tile = [&](int t, int tk) {
+      const int rows = ls->n_tok - t * kTileMax < kTileMax ? ls->n_tok - t * kTileMax : kTileMax;
+      if (lane == 0) mbar_expect_tx(ls->h_full, (uint32_t)rows * h_row);
+      __syncwarp();
+      if (lane < rows) bulk_g2s(stage + (size_t)lane * ls->pitch, p.h + (int64_t)tk * p.D, h_row, ls->h_full);
+    };
+    // the remaining tiles, each once the previous one's MMAs are done
+    auto stage_rest = [&]() {
+      for (; staged < ls->n_st; ++staged) {
+        const int i = staged * kTileMax + lane;
+        const int tk = lane < kTileMax && i < ls->n_tok ? __ldg(ls->tok + i) : 0;
+        if (!warp_wait(ls->h_empty, (uint32_t)((staged - 1) & 1), abort, p.err)) return false;
+        stage_tile(staged, tk);
       }
-      const uint32_t q = ring_slot(r, L, k);
-      if ((int)q >= ls->wr_slot0 && !warp_wait(ls->wr_free, 0u, abort, p.err)) {
-        ok = false;
-        break;
-      }
-      issue_rows(q, row);
-      pre = k + 1;
+      return true;
+    };
+    if (ls->n_st > 0) {
+      stage_tile(0, tok0);
+      staged = 1;
     }
+    // the first lap (item k in slot k): the free slots at once, then Wr's
+    // slots once the B fragments are in registers, then the staging slots
+    // after the router's last tile
+    const int first = my_n < L.n_slots ? my_n : L.n_slots;  // n_slots <= 16 < 32: all in my_item
+    uint32_t sent = 0;  // lap-0 items whose row blocks went out
+    for (int pass = 0; ok && pass < 3; ++pass) {
+      for (int k = 0; k < first; ++k) {
+        const int q = (int)ring_slot(r, L, k);
+        const int kind = q >= ls->wr_slot0 ? 1 : (q >= ls->st_slot0 && ls->n_st > 0 ? 2 : 0);
+        if (kind != pass) continue;
+        const int row = __shfl_sync(0xffffffffu, p.by_uid ? my_item.w : my_item.x, k);
+        if (bad_row(row)) {
+          ok = false;
+          break;
+        }
+        if (kind == 1)
+          ok = warp_wait(ls->wr_free, 0u, abort, p.err);
+        else if (kind == 2)
+          ok = stage_rest() && warp_wait(ls->h_empty, (uint32_t)((ls->n_st - 1) & 1), abort, p.err);
+        if (!ok) break;
+        issue_rows((uint32_t)q, row);
+        sent |= 1u << k;
+      }
+    }
+    if (ok) ok = stage_rest();  // (fewer items than slots)
+    pre = first;
     if (!ok) {
-      // items 0 .. pre-1 hold row copies but no token list: their missing
-      // arrivals, so their phases complete when the copies land and the
-      // drain below waits for them (the consumers see the abort flag)
+      // the lap-0 items sent hold row copies but no token list: their
+      // missing arrivals, so their phases complete when the copies land,
+      // then wait for those (the consumers see the abort flag)
       *abort = 1;
       __syncwarp();
-      if (lane == 0)
-        for (int kk = 0; kk < pre; ++kk) mbar_arrive(&r.full[ring_slot(r, L, kk)]);
-      issued = pre;
+      if (lane == 0) {
+        for (int kk = 0; kk < first; ++kk)
+          if (sent >> kk & 1u) mbar_arrive(&r.full[ring_slot(r, L, kk)]);
+        for (int kk = 0; kk < first; ++kk)
+          if (sent >> kk & 1u) mbar_drain(&r.full[ring_slot(r, L, kk)], 0u);
+      }
+      issued = 0;
     }
   }
   int next_tok = -1;
@@ -728,7 +779,10 @@ __device__ void ring_producer(const GArgs& p, const GroupWs& w, const GroupLayou
     }
   }
   if (lane == 0) {  // the last copies must have landed before the CTA exits
-    if (ls != nullptr) mbar_drain(ls->wr_full, 0u);
+    if (ls != nullptr) {
+      mbar_drain(ls->wr_full, 0u);
+      if (staged > 0) mbar_drain(ls->h_full, (uint32_t)((staged - 1) & 1));
+    }
     for (int kk = issued - 1; kk >= 0 && kk >= issued - L.n_slots; --kk)
       mbar_drain(&r.full[ring_slot(r, L, kk)], ring_parity(L, kk));
   }
@@ -931,7 +985,7 @@ constexpr int kPairRows = 2 * kTileMax;
 
 template <int NP>
 __host__ __device__ constexpr size_t pair_scratch_bytes() {
-  return (size_t)kWarps * kPairRows * NP * 4 + (size_t)kPairRows * NP * 4 + (size_t)kPairRows * 4;
+  return (size_t)kWarps * kPairRows * NP * 4;  // the partial sums (the gates go elsewhere)
 }
 
 struct PairScratch {
@@ -1002,26 +1056,50 @@ __device__ __forceinline__ void router_load_a_rows(RouterA<KB>& A, const uint16_
   }
 }
 
+// A fragments of a staged router tile (row rr at stage + rr * pitch, rr <
+// rows; rows past read as zero), in router_load_a's k-slot order.  With
+// pitch = 2 D + 32 the 32 lanes of one load hit every bank pair once.
+template <int KB>
+__device__ __forceinline__ void router_load_a_smem(RouterA<KB>& A, const uint8_t* stage, int pitch, int rows, int D,
+                                                   int kb) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+  const bool ok0 = g < rows, ok1 = g + 8 < rows;
+  const uint8_t* r0 = stage + (size_t)g * pitch + 8 * c;
+  const uint8_t* r1 = stage + (size_t)(g + 8) * pitch + 8 * c;
+  const int ksteps = D >> 4;
+#pragma unroll
+  for (int i = 0; i < KB; ++i) {
+    const int ks = kb + i * kWarps;
+    const bool in = ks < ksteps;
+    A.a0[i] = (in && ok0) ? *reinterpret_cast<const uint2*>(r0 + ks * 32) : make_uint2(0u, 0u);
+    A.a1[i] = (in && ok1) ? *reinterpret_cast<const uint2*>(r1 + ks * 32) : make_uint2(0u, 0u);
+  }
+}
+
 // Consumer warps: the gates of the CTA's n_tok listed tokens (tok[i]) into
-// gl[n_tok][NP].  The first tile's A fragments load while Wr arrives; each warp then takes the B fragments of its k-steps into
-// registers and Wr's slot goes back to the ring.  The tiles' A fragments
-// load one tile at a time, the next right after the current tile's MMAs;
-// two tiles share one partial-sum exchange and softmax.  Returns false
-// (uniformly) if Wr never arrived.
+// gl[n_tok][NP].  Each warp takes the B fragments of its k-steps into
+// registers as soon as Wr lands and Wr's slots go back to the ring.  A
+// fragments: from the staging slots, tile by tile as the producer's bulk
+// copies land (each tile's slots released after its MMAs); without staging
+// slots, from h by token id, the next tile's right after the current tile's
+// MMAs.  Two tiles share one partial-sum exchange and softmax.  Returns
+// false (uniformly) if a copy never arrived.
 template <int NT, bool kExactN>
-__device__ bool local_router_phase(const GArgs& p, const PairScratch& ps, const uint16_t* wr_s, const LocalSync& ls,
-                                   const int* tok, int n_tok, float* gl, volatile int* abort, volatile int* fail) {
+__device__ bool local_router_phase(const GArgs& p, const PairScratch& ps, const uint16_t* wr_s, const uint8_t* stage,
+                                   const LocalSync& ls, const int* tok, int n_tok, float* gl, volatile int* abort,
+                                   volatile int* fail) {
   constexpr int KB = kFusedKB;
   constexpr int NP = 8 * NT;
   const int warp = threadIdx.x >> 5;
   const int ksteps = p.D >> 4;
   const int n_tiles = (n_tok + kTileMax - 1) / kTileMax;
+  const bool staged = ls.n_st > 0;
   auto rows_of = [&](int t) {
     const int left = n_tok - t * kTileMax;
     return left < 0 ? 0 : (left < kTileMax ? left : kTileMax);
   };
   RouterA<KB> A;
-  if (n_tiles > 0) router_load_a_rows<KB>(A, p.h, tok, rows_of(0), p.D, warp);
+  if (!staged && n_tiles > 0) router_load_a_rows<KB>(A, p.h, tok, rows_of(0), p.D, warp);
   const bool ok = consumers_wait(ls.wr_full, 0u, abort, p.err, fail);
   // B fragments of k-steps warp + 8i, in the router kernels' k-slot order
   uint2 bw[KB][NT];
@@ -1039,7 +1117,7 @@ __device__ bool local_router_phase(const GArgs& p, const PairScratch& ps, const 
     }
   }
   ConsumerSync{}();
-  if (ok && threadIdx.x == 0) mbar_arrive(ls.wr_free);  // Wr's slot goes back to the ring
+  if (ok && threadIdx.x == 0) mbar_arrive(ls.wr_free);  // Wr's slots go back to the ring
   if (!ok) return false;
   auto mma_tile = [&](float (&acc)[NT][4]) {
 #pragma unroll
@@ -1053,15 +1131,28 @@ __device__ bool local_router_phase(const GArgs& p, const PairScratch& ps, const 
       }
     }
   };
-  for (int t = 0; t < n_tiles; t += 2) {
-    const bool two = t + 1 < n_tiles;
-    float acc[NT][4];
-    mma_tile(acc);
-    if (t + 1 < n_tiles) router_load_a_rows<KB>(A, p.h, tok + (t + 1) * kTileMax, rows_of(t + 1), p.D, warp);
-    pair_store_partials<NT>(ps, acc, 0);
-    if (two) {
+  // tile t's MMAs into acc: a staged tile waits for its copies and releases
+  // the staging slots after its MMAs (every warp past them); otherwise the
+  // next tile's A fragments are requested right after
+  auto tile = [&](int t, float (&acc)[NT][4]) {
+    if (staged) {
+      if (!consumers_wait(ls.h_full, (uint32_t)(t & 1), abort, p.err, fail)) return false;
+      router_load_a_smem<KB>(A, stage, ls.pitch, rows_of(t), p.D, warp);
       mma_tile(acc);
-      if (t + 2 < n_tiles) router_load_a_rows<KB>(A, p.h, tok + (t + 2) * kTileMax, rows_of(t + 2), p.D, warp);
+      ConsumerSync{}();
+      if (threadIdx.x == 0) mbar_arrive(ls.h_empty);
+    } else {
+      mma_tile(acc);
+      if (t + 1 < n_tiles) router_load_a_rows<KB>(A, p.h, tok + (t + 1) * kTileMax, rows_of(t + 1), p.D, warp);
+    }
+    return true;
+  };
+  for (int t = 0; t < n_tiles; t += 2) {
+    float acc[NT][4];
+    if (!tile(t, acc)) return false;
+    pair_store_partials<NT>(ps, acc, 0);
+    if (t + 1 < n_tiles) {
+      if (!tile(t + 1, acc)) return false;
       pair_store_partials<NT>(ps, acc, kTileMax);
     }
     ConsumerSync{}();
@@ -1086,14 +1177,14 @@ __global__ void __launch_bounds__(kGroupThreads, 1) grouped_local_kernel(const G
   float* gl = reinterpret_cast<float*>(scratch + (size_t)kWarps * kPairRows * NP * 4);  // [scap][NP] gates
   int* loff = reinterpret_cast<int*>(gl + (size_t)scap * NP);                       // [scap + 1]
   __shared__ int skip_s, fail_s;
-  __shared__ __align__(8) uint64_t bars[2];
+  __shared__ __align__(8) uint64_t bars[4];
   const int b = blockIdx.x, lane = threadIdx.x & 31;
   const bool producer = (threadIdx.x >> 5) == kGroupProducer;
   const int wr_slot0 = L.n_slots - wr_slots(L, p.N, p.D);
   uint8_t* wr_slot = r.slots + (size_t)wr_slot0 * L.slot_bytes;
   const int* tok = w.share_tok + (size_t)b * scap;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&bars[i], 1);
     ring_init(r, L, 2);  // full: the row block's copies, the token list
   }
   __syncthreads();
@@ -1112,8 +1203,10 @@ __global__ void __launch_bounds__(kGroupThreads, 1) grouped_local_kernel(const G
                wr_bytes - off < kWrChunk ? wr_bytes - off : kWrChunk, &bars[0]);
     }
   }
-  // the CTA's counts (all threads), the control words (thread 0)
+  // the CTA's counts (all threads), the token ids of the first router tile
+  // (producer lanes 0-15; scap >= 32), the control words (thread 0)
   const int2 sn = reinterpret_cast<const int2*>(w.share_n)[b];
+  const int tok0 = producer && lane < kTileMax ? __ldg(tok + lane) : 0;
   if (threadIdx.x == 0) {
     const unsigned ab = ld_relaxed_u32(&w.ctl[kCtlAbort]), grid = ld_relaxed_u32(&w.ctl[kCtlShareGrid]);
     // plan abandoned (error word set): skip; shares for another CTA count: error
@@ -1127,15 +1220,22 @@ __global__ void __launch_bounds__(kGroupThreads, 1) grouped_local_kernel(const G
     return;
   }
   const int my_n = sn.x, n_tok = sn.y;
-  const LocalSync ls{&bars[0], &bars[1], w.share_rec + (size_t)b * scap, wr_slot0};
+  // staging slots for the router tiles: those before Wr's that hold 16 h
+  // rows, if at least one slot is left for row blocks
+  const int pitch = 2 * p.D + 32;
+  const int st_n = (int)(((int64_t)kTileMax * pitch + L.slot_bytes - 1) / L.slot_bytes);
+  const int st_slot0 = wr_slot0 - st_n >= 1 ? wr_slot0 - st_n : wr_slot0;
+  const LocalSync ls{&bars[0], &bars[1], &bars[2], &bars[3], w.share_rec + (size_t)b * scap, tok, wr_slot0, st_slot0,
+                     st_slot0 < wr_slot0 ? (n_tok + kTileMax - 1) / kTileMax : 0, n_tok, pitch};
   if (producer) {
-    ring_producer<NP, kNf3>(p, w, L, r, my_n, &ls);
+    ring_producer<NP, kNf3>(p, w, L, r, my_n, &ls, tok0);
   } else {
     // step offsets into shared memory (my_n <= scap < the consumer threads);
     // the router phase's first barrier orders them before their readers
     if ((int)threadIdx.x <= my_n) loff[threadIdx.x] = __ldg(w.share_off + (size_t)b * (scap + 1) + threadIdx.x);
-    const bool ok = local_router_phase<NT, kExactN>(p, ps, reinterpret_cast<const uint16_t*>(wr_slot), ls, tok, n_tok,
-                                                    gl, r.abort, &fail_s);
+    const bool ok = local_router_phase<NT, kExactN>(p, ps, reinterpret_cast<const uint16_t*>(wr_slot),
+                                                    r.slots + (size_t)st_slot0 * L.slot_bytes, ls, tok, n_tok, gl,
+                                                    r.abort, &fail_s);
     if (!ok && threadIdx.x == 0) *r.abort = 1;  // the producer stops too
     ring_consumers<NT, kExactN, kNf3>(p, L, r, ok ? my_n : 0, gl, loff);
   }
@@ -1171,7 +1271,9 @@ template <int NT, bool kExactN, bool kNf3>
 mole_status launch_local(const GArgs& p, const GroupWs& w, cudaStream_t stream) {
   constexpr int NP = 8 * NT;
   static_assert(NT <= 2, "the router phase holds B fragments of at most 16 experts");
-  if (p.D > 16 * kWarps * kFusedKB || !aligned16(p.Wr)) return MOLE_ERR_UNSUPPORTED;
+  // (the staged router tiles are bulk copies of h rows: 16-byte aligned rows)
+  if (p.D > 16 * kWarps * kFusedKB || !aligned16(p.Wr) || !aligned16(p.h) || p.D % 8 != 0)
+    return MOLE_ERR_UNSUPPORTED;
   const GroupLayout L = group_layout<NT>(p.N, p.D, kNf3);
   if (L.n_slots < 2 || wr_slots(L, p.N, (int)p.D) >= L.n_slots) return MOLE_ERR_UNSUPPORTED;
   const int n_sm = num_sms();
@@ -1179,7 +1281,7 @@ mole_status launch_local(const GArgs& p, const GroupWs& w, cudaStream_t stream) 
   if (!shares_apply(p.T, n_sm)) return MOLE_ERR_UNSUPPORTED;
   const int64_t scap = share_cap(p.T, n_sm);
   static_assert(kShareCapLimit <= kGroupCons * 32, "a consumer thread per step offset");
-  const size_t smem = (ring_bytes(L.n_slots, L.slot_bytes) + 127) / 128 * 128 + (size_t)kWarps * kPairRows * NP * 4 +
+  const size_t smem = (ring_bytes(L.n_slots, L.slot_bytes) + 127) / 128 * 128 + pair_scratch_bytes<NP>() +
                       (size_t)scap * NP * 4 + (size_t)(scap + 1) * 4;
   if (smem > 227 * 1024) return MOLE_ERR_UNSUPPORTED;
   auto kern = grouped_local_kernel<NT, kExactN, kNf3>;
