@@ -204,6 +204,25 @@ def kernel_source_hash() -> str:
     return h.hexdigest()
 
 
+def launches_per_step(T: int, N: int, layers: int, path: str) -> int:
+    """This library's kernel launches in one timed step.  Grouped path: the
+    grouping (plan kernel, plus the per-SM share kernel when a CTA's share
+    fits, 16 + T/SMs < 256 tokens), then per layer the tensor-core router and
+    the gather kernel where 128-token tiles fill 3/4 of the SMs (16 experts),
+    else the one CTA-local kernel; plain path: router + gather per layer.
+    Below 1024 tokens one combine kernel per layer."""
+    import torch
+    n_sm = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    if T < 1024:
+        return layers
+    if path != "grouped":
+        return 2 * layers
+    shares = (16 + -(-T // n_sm) + 15) // 16 * 16 < 256
+    tc_router = N == 16 and -(-T // 128) >= n_sm * 3 // 4
+    per_layer = 2 if (tc_router or not shares) else 1
+    return (2 if shares else 1) + per_layer * layers
+
+
 def profiled_traffic(path: str):
     """(bytes per launch, note) from the committed ncu summary if it was taken
     on the current kernel source; else (None, reason)."""
@@ -471,8 +490,7 @@ def main():
         "layer_tokens_per_s": value * L, "hbm_gbs": achieved_gbs,
         "roofline": roofline,
         "e2e": e2e,
-        # per layer: router kernel + gather kernel (T >= 1024); per step: the grouping kernel (grouped path)
-        "gpu_launches": K * L * (2 if T >= 1024 else 1) + (K if args.path == "grouped" else 0),
+        "gpu_launches": K * launches_per_step(T, N, L, args.path),
         "token_groups_build_us_per_step": max_prep_ms * 1e3 if args.path == "grouped" else None,
         "clocks": clocks.summary(),
     }
