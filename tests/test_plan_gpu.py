@@ -2,7 +2,6 @@
 sort + unique (MoLE page, 复杂度分析: a batch moves only its tokens' rows)."""
 import numpy as np
 import pytest
-import torch
 
 from helpers import dev
 from mixture_lookup_experts_b200 import inputs

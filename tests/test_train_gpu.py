@@ -18,7 +18,7 @@ import numpy as np
 import pytest
 import torch
 
-from helpers import dev, host_bits
+from helpers import dev
 from mixture_lookup_experts_b200 import inputs
 
 pytestmark = pytest.mark.gpu
