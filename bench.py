@@ -52,11 +52,8 @@ KERNEL_SOURCES = ["mixture_lookup_experts_b200/csrc/combine.cu", "mixture_lookup
 PROFILE_SUMMARY = {"grouped": "profiles/combine_grouped_bf16_1b_T16384_zipf.md",
                    "plain": "profiles/combine_bf16_1b_T16384_zipf.md"}
 KERNELS = {
-    "grouped": "mole_lookup_combine_groups = router_tc_kernel (tcgen05 router, TMA-streamed h, gates to the tokens' "
-               "list positions) + grouped_gather_kernel (one bulk copy per distinct row block, all of its tokens "
-               "combined from shared memory); duration = the call (the per-step grouping is timed apart)",
-    "plain": "mole_lookup_combine = router_tc_kernel (tcgen05 router, gates parked in the output rows) + "
-             "gather_kernel (bulk-copy ring of row blocks, consumer warps); duration = the call",
+    "grouped": "router_tc_kernel + grouped_gather_kernel (mole_lookup_combine_groups, per layer call)",
+    "plain": "router_tc_kernel + gather_kernel (mole_lookup_combine, per layer call)",
 }
 
 
@@ -117,15 +114,26 @@ def workload_config(T: int, kind: str, layers: int | None = None, path: str = "g
     layers = s.layers if layers is None else layers
     call = "mole_lookup_combine_groups" if path == "grouped" else "mole_lookup_combine"
     return {
-        "workload": f"1B-activated-shaped MoLE lookup path, {layers} layers x {call}"
-                    f"{' (one token grouping per step)' if path == 'grouped' else ''}, "
-                    f"prefill T={T}, {'Zipf(1.1)' if kind == 'zipf' else 'uniform'} ids shared by the layers",
+        "workload": f"1B-shaped MoLE lookup path: {layers} layers x {call}"
+                    f"{' (one grouping per step)' if path == 'grouped' else ''}, prefill T={T}, "
+                    f"{'Zipf(1.1)' if kind == 'zipf' else 'uniform'} ids",
         "V": s.V, "D": s.D, "N": s.N, "layers": layers, "tokens_per_step": T, "ids": kind,
-        "table_dtype": "bf16", "accumulate": "f32", "out_dtype": "f32",
-        "l2": "inputs larger than L2: each step reads 16 distinct 3.3 GB layer tables",
-        "data": "synthetic seeded N(0,0.02) tables; per step one id batch (shared by the layers) and per-layer "
-                "hidden states, rotating over a pool of 4",
+        "table_dtype": "bf16", "out_dtype": "f32",
+        "l2": "inputs larger than L2 (each step reads its layers' distinct 3.3 GB tables)",
+        "data": "seeded N(0,0.02) tables; ids and per-layer h rotate over a pool of 4 batches",
     }
+
+
+def compact(x, digits: int = 6):
+    """Floats rounded to `digits` significant digits, recursively (keeps the
+    headline line short)."""
+    if isinstance(x, float):
+        return float(f"{x:.{digits}g}")
+    if isinstance(x, dict):
+        return {k: compact(v, digits) for k, v in x.items()}
+    if isinstance(x, list):
+        return [compact(v, digits) for v in x]
+    return x
 
 
 # ---------------------------------------------------------------------------
@@ -475,48 +483,64 @@ def main():
     achieved_gbs = alg_bytes / (max_kern_ms / 1e3) / 1e9
     traffic, traffic_note = profiled_traffic(args.path)
     roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_peak, "unit": "GB/s",
-                "frac": achieved_gbs / hbm_peak, "traffic": traffic,
-                "kernel": KERNELS[args.path],
-                "algorithmic_bytes_per_launch": alg_bytes, "unique_rows_per_launch": U_avg,
-                "avg_launch_us": max_kern_ms * 1e3, "launch_timing": "per layer call = (step - grouping) / layers, "
-                "CUDA events per step on the launching stream", "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)",
-                "frac_of_8TBs": achieved_gbs / 8000.0, "traffic_source": traffic_note}
+                "frac": achieved_gbs / hbm_peak, "traffic": traffic, "kernel": KERNELS[args.path],
+                "bytes_per_launch": alg_bytes, "unique_rows": U_avg, "avg_launch_us": max_kern_ms * 1e3,
+                "peak_source": f"{peak_kind} hbm_gbs", "frac_of_8TBs": achieved_gbs / 8000.0,
+                "traffic_source": traffic_note}
 
-    line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
-        "ms_per_step": max_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic", "config": workload_config(T, args.ids, L, args.path),
-        "layer_tokens_per_s": value * L, "hbm_gbs": achieved_gbs,
-        "roofline": roofline,
-        "e2e": e2e,
-        "gpu_launches": K * launches_per_step(T, N, L, args.path),
-        "token_groups_build_us_per_step": max_prep_ms * 1e3 if args.path == "grouped" else None,
-        "clocks": clocks.summary(),
-    }
+    line = headline(value=value, world=world, K=K, W=W, max_ms=max_ms,
+                    cfg=workload_config(T, args.ids, L, args.path), roofline=roofline, e2e=e2e,
+                    launches=K * launches_per_step(T, N, L, args.path),
+                    prep_us=max_prep_ms * 1e3 if args.path == "grouped" else None, clocks=clocks.summary())
 
-    # ---- extras: other prefill cases, NF3 table, table build ----
+    # ---- extras, each printed as its own JSON line before the headline ----
+    def leg(name, fn):
+        res = fn()
+        if rank == 0:
+            print(json.dumps({"leg": name, name: res}), flush=True)
+
     if not args.no_extras:
-        line["cases"] = other_cases(mole, luts, routers, rng, g, dev, stream, W, T, args.ids, args.path, L)
-        line["nf3"] = nf3_leg(mole, luts, routers, id_pool, h_pool, uniq_counts, dev, stream, W, K, T, P, L)
+        leg("cases", lambda: other_cases(mole, luts, routers, rng, g, dev, stream, W, T, args.ids, args.path, L))
+        leg("nf3", lambda: nf3_leg(mole, luts, routers, id_pool, h_pool, uniq_counts, dev, stream, W, K, T, P, L))
         if not args.no_offload:
-            line["offload"] = offload_leg(mole, luts, routers, rng, g, dev, stream, W, L)
+            leg("offload", lambda: offload_leg(mole, luts, routers, rng, g, dev, stream, W, L))
         if not args.no_ffn:
-            line["ffn_block"] = ffn_leg(mole, luts, routers, rng, g, dev, stream, W, (bf16_peak, bf16_sust))
+            leg("ffn_block", lambda: ffn_leg(mole, luts, routers, rng, g, dev, stream, W, (bf16_peak, bf16_sust)))
         del luts
         torch.cuda.empty_cache()
         if not args.no_decode:
-            line["decode"] = decode_leg(mole, dev, stream)
+            leg("decode", lambda: decode_leg(mole, dev, stream))
         if not args.no_train:
-            line["train"] = train_leg(mole, rng, g, dev, stream, W, (bf16_peak, bf16_sust))
-        line["build"] = build_leg(mole, dev, stream, bf16_peak, bf16_sust, peak_kind)
+            leg("train", lambda: train_leg(mole, rng, g, dev, stream, W, (bf16_peak, bf16_sust)))
+        leg("build", lambda: build_leg(mole, dev, stream, bf16_peak, bf16_sust, peak_kind))
 
     if rank == 0 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(args)
+        line["cpu_baseline"] = compact(cpu_baseline(args))
     if rank == 0:
+        # the headline: one short line, printed last
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+HEADLINE_MAX_BYTES = 2048
+
+
+def headline(*, value, world, K, W, max_ms, cfg, roofline, e2e, launches, prep_us, clocks, cpu=None) -> dict:
+    """The headline JSON line (floats to 6 significant digits).  Printed
+    last and kept under HEADLINE_MAX_BYTES so that a reader keeping only
+    the tail of the output still holds all of it; the extra legs go on
+    lines of their own before it."""
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": max_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic", "config": cfg, "roofline": roofline, "e2e": e2e,
+        "gpu_launches": launches, "token_groups_build_us_per_step": prep_us, "clocks": clocks,
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    return compact(line)
 
 
 def e2e_leg(combine, id_pool, h_pool, routers, luts, out, dev, stream, world, W, K, T, L):
@@ -559,8 +583,7 @@ def e2e_leg(combine, id_pool, h_pool, routers, luts, out, dev, stream, world, W,
     (e_ms,) = max_over_ranks([e_start.elapsed_time(e_end)], dev)
     return {"value": whole_job_tokens_per_s(world, T, K_e2e, e_ms), "unit": UNIT,
             "h2d_bytes_per_step": L * T * D * 2 + T * 4, "d2h_bytes_per_step": L * T * D * 4,
-            "steps": K_e2e, "note": f"per step: the batch's ids + {L} hidden-state batches H2D from pinned memory, "
-                                    f"the token grouping and {L} combine calls through the C ABI, {L} outputs D2H"}
+            "steps": K_e2e, "note": f"per step: ids + {L} h H2D (pinned), {L} C-ABI calls, {L} outputs D2H"}
 
 
 def time_block(fn, n, stream):

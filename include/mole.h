@@ -92,23 +92,25 @@ mole_status mole_build_lut(const void* embed, const void* W1, const void* W2, in
 
 /*
  * mole_build_lut without caller-provided scratch, for callers that cannot
- * allocate device memory when they build a table: code running while a stream
- * is captured into a CUDA graph (an allocation there breaks the capture),
- * serving loops that allow no device allocation after start-up, and plugin
- * hosts that give plugins no allocator.  The MoLE page has no counterpart; it
- * is an interface convenience.
+ * allocate device memory when they build a table: serving loops that allow no
+ * device allocation after start-up (their memory footprint is fixed up
+ * front), and plugin hosts that own all device memory and give plugins no
+ * allocator.  The MoLE page has no counterpart; it is an interface
+ * convenience.
  *
  * Same arguments, layouts and results as mole_build_lut, minus the workspace:
  * the hidden activations of each group of experts live in a fixed 16 MiB array
  * in this library's device memory (held by every GPU that loads the library
  * until the process exits).  One expert's activations, V * Dr * (2 bytes for
  * bf16, 4 for fp32), must fit in it, else MOLE_ERR_WORKSPACE and nothing is
- * launched.  The first call on each device looks the array's device address
- * up (cudaGetSymbolAddress); make that first call before any stream capture.
- * Every call uses the same array: calls that overlap on the GPU (other
- * streams, other threads) race on it; the array needs no clearing between
- * calls (each expert's activations are written before they are read).  No
- * device memory is allocated or freed.
+ * launched; experts are built in groups of as many as fit.  The first call on
+ * each device looks the array's device address up (cudaGetSymbolAddress, with
+ * that device current), and looks it up again after the device's context has
+ * changed (a device reset); make that first call before any stream capture.
+ * Every call uses the same array, which keeps the last call's contents: calls
+ * that overlap on the GPU (other streams, other threads) race on it.  The
+ * array needs no clearing between calls (each expert's activations are
+ * written before they are read).  No device memory is allocated or freed.
  */
 mole_status mole_build_lut_noalloc(const void* embed, const void* W1, const void* W2, int64_t V,
                                    int64_t D, int32_t N, int64_t Dr, mole_act act, mole_dtype dt,
@@ -384,8 +386,9 @@ mole_status mole_gather_plan(const int32_t* ids, int64_t T, int64_t V, int32_t* 
                              int32_t* n_uniq, int32_t* slot, cudaStream_t stream);
 
 /*
- * Waits (polling, at most timeout_ms; < 0 = no limit) for `stream` to drain,
- * then reads and clears this device's error word.  Returns MOLE_OK,
+ * Waits (polling, at most timeout_ms >= 0 milliseconds) for `stream` to drain,
+ * then reads and clears this device's error word.  A negative timeout_ms is
+ * rejected with MOLE_ERR_ARG (no host wait is unbounded).  Returns MOLE_OK,
  * MOLE_ERR_INDEX (bad token id), MOLE_ERR_TIMEOUT (stream still busy, or a
  * device-side wait gave up), MOLE_ERR_ARG (a grouping was used on a device
  * with another SM count than the one it was built on; the layer's output was

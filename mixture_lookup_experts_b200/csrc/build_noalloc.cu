@@ -1,14 +1,15 @@
 // build_noalloc.cu -- table build for callers that cannot allocate device memory.
 //
 // mole_build_lut needs a scratch buffer for the expert hidden activations, and
-// the caller usually allocates it.  Some callers cannot: code that runs while a
-// stream is being captured into a CUDA graph (an allocation there breaks or
-// invalidates the capture), serving loops that forbid device allocations after
-// start-up so their memory use stays fixed, and plugin hosts that hand out all
-// device memory through their own pool and give plugins no allocator.  For
-// them, mole_build_lut_noalloc runs the same build kernels with the scratch
-// taken from a fixed array in this library's device memory (16 MiB; every GPU
-// that loads the library holds it until the process exits).
+// the caller usually allocates it.  Some callers cannot: serving loops that
+// forbid device allocations after start-up so that their memory use stays
+// fixed, and plugin hosts that hand out all device memory through their own
+// pool and give plugins no allocator.  For them, mole_build_lut_noalloc runs
+// the same build kernels with the scratch taken from a fixed array in this
+// library's device memory (16 MiB; every GPU that loads the library holds it
+// until the process exits).
+#include <cuda.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -19,25 +20,60 @@ constexpr size_t kScratchBytes = size_t(16) << 20;
 
 // The scratch array.  Host code must not pass its name to a kernel (on the
 // host it is only a stand-in symbol); scratch_device_ptr() resolves the device
-// address once per device.
+// address once per device (and context).
 static __device__ __align__(256) uint8_t g_build_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
-void* g_scratch_ptr[kMaxDevices];
+struct ScratchAddr {
+  unsigned long long ctx_id;  // the context the address belongs to
+  void* ptr;
+};
+ScratchAddr g_scratch[kMaxDevices];
 
-// Device address of g_build_scratch on the current device (set up on the
-// first call per device; nullptr if the lookup fails).
+typedef CUresult (*ctx_get_current_t)(CUcontext*);
+typedef CUresult (*ctx_get_id_t)(CUcontext, unsigned long long*);
+
+// Unique id of the current context (cuCtxGetId, fetched from the driver at
+// run time); 0 if it cannot be read.  A device reset or a new primary
+// context gets a new id, and with it the array a new device address.
+unsigned long long current_context_id() {
+  static ctx_get_current_t get_current = nullptr;
+  static ctx_get_id_t get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<ctx_get_current_t>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<ctx_get_id_t>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of g_build_scratch on the current device: looked up
+// (cudaGetSymbolAddress, with the device current) on the first call per
+// device, and again only when the device's context has changed since (after a
+// device reset the module is loaded anew and the array moves).  nullptr if the
+// lookup fails.
 void* scratch_device_ptr() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
   std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_build_scratch) != cudaSuccess) return nullptr;
-    g_scratch_ptr[dev] = p;
-  }
-  return g_scratch_ptr[dev];
+  ScratchAddr& s = g_scratch[dev];
+  if (s.ptr && s.ctx_id != 0 && s.ctx_id == current_context_id()) return s.ptr;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_build_scratch) != cudaSuccess || !p) return nullptr;
+  s = ScratchAddr{current_context_id(), p};  // the lookup has made the context current
+  return s.ptr;
 }
 
 }  // namespace

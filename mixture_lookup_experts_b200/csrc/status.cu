@@ -61,14 +61,14 @@ extern "C" const char* mole_status_str(mole_status s) {
 extern "C" int mole_version(void) { return 100; }
 
 extern "C" mole_status mole_check(cudaStream_t stream, int timeout_ms) {
+  if (timeout_ms < 0) return MOLE_ERR_ARG;  // every host wait has a limit
   using clock = std::chrono::steady_clock;
   const auto t0 = clock::now();
   for (;;) {
     cudaError_t e = cudaStreamQuery(stream);
     if (e == cudaSuccess) break;
     if (e != cudaErrorNotReady) return MOLE_ERR_CUDA;
-    if (timeout_ms >= 0 &&
-        std::chrono::duration_cast<std::chrono::milliseconds>(clock::now() - t0).count() > timeout_ms)
+    if (std::chrono::duration_cast<std::chrono::milliseconds>(clock::now() - t0).count() > timeout_ms)
       return MOLE_ERR_TIMEOUT;
     std::this_thread::sleep_for(std::chrono::microseconds(50));
   }

@@ -44,3 +44,20 @@ def mole():
     _build.build()
     from mixture_lookup_experts_b200 import mole as m
     return m
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Table-build diagnostics of the session (one line per comparison)."""
+    try:
+        from helpers import BUILD_DIAG
+    except ImportError:
+        return
+    if not BUILD_DIAG:
+        return
+    tr = terminalreporter
+    tr.write_sep("-", "table build vs oracle (bf16 ulps; floor 2^-8 rms(row))")
+    for d in BUILD_DIAG:
+        tr.write_line(f"{d['label'][:60]:60s} n={d['elements']:>9d} beyond-allow {d['max_ulps_beyond_allowance']:.2f} "
+                      f"unfloored-max {d['max_unfloored_ulps']:.3g} >2u-unfloored {d['pct_over_2_unfloored']:.4f}% "
+                      f">2u-floored-raw {d['pct_over_2_floored_before_allowance']:.4f}% "
+                      f"row-rel {d['max_row_rel_l2']:.2e}")

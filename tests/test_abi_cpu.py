@@ -70,6 +70,7 @@ def test_argument_checks_without_device(mole):
     assert lib.mole_build_lut(P, P, P, 10, 64, 2, 64, 0, 1, P, None, 0, None) == 4   # no workspace
     assert lib.mole_build_lut(P, P, P, 10, 64, 2, 64, 9, 1, P, P, 1 << 20, None) == 1  # bad act
     assert lib.mole_gather_plan(P, -3, 10, P, P, P, None) == 1
+    assert lib.mole_check(None, -1) == 1  # no unbounded host wait
 
 
 def test_valid_arguments_reach_the_device_check(mole):
