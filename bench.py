@@ -901,7 +901,8 @@ def train_leg(mole, rng, g, dev, stream, W, peaks):
     """One MoLE layer's training step at the 1B shape, T = 4096 Zipf tokens
     (§8(f) rank 4): the forward evaluates the routed experts on the batch's
     distinct ids only (tcgen05 build GEMMs), then the combine; the backward
-    (gate / router gradients, per-id dL/dY, cuBLAS GEMMs for the experts)."""
+    (gate / router gradients, per-id dL/dY, the four expert GEMMs on the same
+    tcgen05 kernels with transposed operand forms)."""
     import torch
     shape = inputs.SHAPES["1b"]
     V, D, N, Dr, T = shape.V, shape.D, shape.N, shape.Dr, 4096
@@ -942,7 +943,7 @@ def train_leg(mole, rng, g, dev, stream, W, peaks):
            "expert_flops_saved_vs_per_token": T / max(U[0], 1),
            "note": "forward: the table build restricted to the batch's distinct embedding rows (tcgen05) + the "
                    "grouped combine; the forward reads the distinct-id count back to the host (one sync); "
-                   "backward GEMMs in cuBLAS"}
+                   "backward expert GEMMs (dpre, dW2, dW1, dE) on tcgen05"}
     del E, W1, W2, cache, grads
     return res
 

@@ -67,7 +67,7 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
     objs = [os.path.join(OBJ, os.path.basename(s)[:-3] + ".o") for s in _sources()]
     if force or todo or _mtime(LIB) < max(_mtime(o) for o in objs):
         tmp = LIB + f".tmp{os.getpid()}"
-        cmd = [NVCC, *ARCH, "-shared", "-o", tmp, *objs, "-lcublas"]
+        cmd = [NVCC, *ARCH, "-shared", "-o", tmp, *objs]
         if verbose:
             print(" ".join(cmd), flush=True)
         subprocess.run(cmd, check=True)

@@ -7,6 +7,15 @@
 //   GEMM2  LUT[:, e, :]  = H[e] . W2[e]     H[e] [V, Dr] K-major, W2[e] [Dr, D] N-major
 // H is rounded to bf16 (the operand type of the second contraction).
 //
+// The same kernels serve the training backward, whose GEMMs take transposed
+// operands: A may also be MN-major (A[m, k] with m contiguous, loaded as
+// 64(M) x 64(K) boxes) and B K-major (B[k, n] with k contiguous, loaded as
+// 64(K) x 128(N) boxes); an operand's expert coordinate may also step its
+// innermost coordinate (a matrix of rows of N experts' blocks); the
+// contraction may run over several experts' K ranges (a sum over experts);
+// the epilogue may scale by the activation's derivative (bf16 out), or add
+// into an fp32 output, optionally through a row map.
+//
 // Kernel: persistent, one CTA per SM, 10 warps with fixed roles
 //   warp 0      TMA producer (one lane): A box 64(K) x 128(M), B four boxes
 //               64(N) x 64(K), all 128-byte swizzled, into a 4-stage ring;
@@ -45,14 +54,26 @@ constexpr int kEpiWarps = 8;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kSmemBytes = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES + 256 /*barriers*/;
 
-// Instruction descriptor, kind::f16: D fp32, A bf16 K-major, B bf16 N-major
-// (bit 16), N/8 at bits 17-22, M/16 at bits 24-28.
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
-                            ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+// Instruction descriptor, kind::f16: D fp32 (bits 4-5), A and B bf16 (bits
+// 7-9, 10-12), A MN-major (bit 15) or K-major, B MN-major (bit 16) or
+// K-major, N/8 at bits 17-22, M/16 at bits 24-28.
+template <bool kAmn, bool kBk, int kM>
+constexpr uint32_t idesc() {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (kAmn ? 1u << 15 : 0u) | (kBk ? 0u : 1u << 16) |
+         ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(kM >> 4) << 24);
+}
+constexpr int A_BOX = 64 * BK * 2;  // 8 KB: an MN-major A box, 64(M) x 64(K)
+constexpr int BK_BOX = BK * 128 * 2;  // 16 KB: a K-major B box, 64(K) x 128(N)
 
 struct Params {
   int M, N, K;            // per expert: C[M, N] = act(A[M, K] . B[K, N])
-  int a_batched;          // A has an expert coordinate (else shared by all experts)
+  // TMA coordinates of expert e's operand: (x + e * X_e0, y, e * X_e2), x
+  // the operand's innermost coordinate (A: a_e2 = 0 shares A by all experts)
+  int a_e0, a_e2, b_e0, b_e2;
+  // > 0: the contraction of output "expert" s runs over the K ranges of the
+  // k_experts experts s * k_experts .. s * k_experts + k_experts - 1 (a sum
+  // over experts), expert c's operands at coordinates as above with e = c
+  int k_experts;
   int act;
   uint16_t* C;            // bf16 output
   int64_t ldc;            // elements between rows of C
@@ -60,12 +81,19 @@ struct Params {
   int m_blocks, n_blocks;
   int64_t tiles;
   unsigned* err;
-  // fp32 output instead (one expert): Cf[m, n] = acc + add0[m, n] + add1[m, n]
-  // (either term may be absent), all three [M, N] row-major with stride ldc;
+  // fp32 output instead: Cf[e][r, n] = acc + add0[e][r, n] + add1[e][r, n]
+  // (either term may be absent), all three row-major with stride ldc and
+  // cf_estride elements between experts, r = c_rowmap[m] (or m if absent);
   // Cf may be add0 or add1 (each element is read, then written, by one thread)
   float* Cf;
   const float* add0;
   const float* add1;
+  int64_t cf_estride;
+  const int* c_rowmap;
+  // bf16 output scaled by the activation's derivative instead (training
+  // backward): C = bf16(acc * act'(grad_pre[e][m, n])), grad_pre fp32 with
+  // stride ldc and pre_estride elements between experts
+  const float* grad_pre;
   // NF3 table instead (second build GEMM): the bf16-rounded outputs of each
   // 64-column block quantised in registers; block (m, e, b) at
   // codes + (m * q_row + e * q_e + b) * 24 and scales + the same index
@@ -100,13 +128,24 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uin
   return d;
 }
 
-__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc_v,
+                                     uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
+      "l"(adesc), "l"(bdesc), "r"(idesc_v), "r"(accumulate)
       : "memory");
+}
+
+// Shared-memory descriptors of k-step k (16 elements of K) of a stage:
+// K-major operands advance 32 bytes inside the 128-byte swizzle atom (8-row
+// groups 1024 bytes apart); MN-major ones advance 16 rows of 128 bytes
+// (2048 bytes), their 64-element MN groups one box apart.
+template <bool kKMajor>
+__device__ __forceinline__ uint64_t operand_desc(uint32_t base, int k, uint32_t mn_group_bytes) {
+  if constexpr (kKMajor) return sw128_desc(base + 32 * k, 16, 1024);
+  else return sw128_desc(base + 2048 * k, mn_group_bytes, 1024);
 }
 
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
@@ -155,7 +194,8 @@ __device__ __forceinline__ void store_chunk_act(int act, const uint32_t (&r)[32]
   }
 }
 
-// The fp32 epilogue: 32 columns of one row, plus up to two fp32 terms.
+// The fp32 epilogue: 32 columns of one row, plus up to two fp32 terms, at
+// element offset `off` of Cf, add0 and add1.
 __device__ __forceinline__ void store_chunk_f32(const uint32_t (&r)[32], const Params& p, int64_t off) {
   float v[32];
 #pragma unroll
@@ -185,6 +225,38 @@ __device__ __forceinline__ void store_chunk_f32(const uint32_t (&r)[32], const P
   float4* o = reinterpret_cast<float4*>(p.Cf + off);
 #pragma unroll
   for (int q = 0; q < 8; ++q) o[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+}
+
+// The derivative epilogue: 32 columns of one row times act'(pre), rounded to
+// bf16, 16-byte stores.
+template <int ACT>
+__device__ __forceinline__ void store_chunk_grad(const uint32_t (&r)[32], const float* pre, uint16_t* dst_row) {
+  const float4* pv = reinterpret_cast<const float4*>(pre);
+  uint32_t packed[16];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const float4 u = pv[q];
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(__uint_as_float(r[4 * q]) * act_grad_t<ACT>(u.x),
+                                                    __uint_as_float(r[4 * q + 1]) * act_grad_t<ACT>(u.y));
+    const __nv_bfloat162 hi = __floats2bfloat162_rn(__uint_as_float(r[4 * q + 2]) * act_grad_t<ACT>(u.z),
+                                                    __uint_as_float(r[4 * q + 3]) * act_grad_t<ACT>(u.w));
+    packed[2 * q] = *reinterpret_cast<const uint32_t*>(&lo);
+    packed[2 * q + 1] = *reinterpret_cast<const uint32_t*>(&hi);
+  }
+  uint4* dst = reinterpret_cast<uint4*>(dst_row);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) dst[q] = make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+}
+
+__device__ __forceinline__ void store_chunk_grad_act(int act, const uint32_t (&r)[32], const float* pre,
+                                                     uint16_t* dst_row) {
+  switch (act) {
+    case MOLE_ACT_GELU_ERF: store_chunk_grad<MOLE_ACT_GELU_ERF>(r, pre, dst_row); break;
+    case MOLE_ACT_GELU_TANH: store_chunk_grad<MOLE_ACT_GELU_TANH>(r, pre, dst_row); break;
+    case MOLE_ACT_RELU: store_chunk_grad<MOLE_ACT_RELU>(r, pre, dst_row); break;
+    case MOLE_ACT_SILU: store_chunk_grad<MOLE_ACT_SILU>(r, pre, dst_row); break;
+    default: store_chunk_grad<MOLE_ACT_IDENTITY>(r, pre, dst_row); break;
+  }
 }
 
 // The NF3 epilogue: two 32-column chunks (one 64-element block) of one row,
@@ -230,7 +302,11 @@ __device__ __forceinline__ void epilogue_tile(const Params& p, uint32_t taddr, i
     tmem_ld32(taddr + chunk * 32, r);
     if (m < p.M) {
       if (p.Cf != nullptr) {
-        store_chunk_f32(r, p, (int64_t)m * p.ldc + col0);
+        const int64_t row = p.c_rowmap != nullptr ? (int64_t)p.c_rowmap[m] : (int64_t)m;
+        store_chunk_f32(r, p, (int64_t)e * p.cf_estride + row * p.ldc + col0);
+      } else if (p.grad_pre != nullptr) {
+        store_chunk_grad_act(p.act, r, p.grad_pre + (int64_t)e * p.pre_estride + (int64_t)m * p.ldc + col0,
+                             crow + col0);
       } else {
         if (p.pre != nullptr) {
           float4* dst = reinterpret_cast<float4*>(p.pre + (int64_t)e * p.pre_estride + (int64_t)m * p.ldc + col0);
@@ -253,6 +329,40 @@ __device__ __forceinline__ void decode_tile(const Params& p, int64_t tile, int& 
   nb = (int)(r - (int64_t)mb * p.n_blocks);
 }
 
+// Expert coordinate and k-block of step `kbt` of a tile of output expert e.
+__device__ __forceinline__ void k_step(const Params& p, int e, int kbt, int kblocks, int& ec, int& kb) {
+  if (p.k_experts > 0) {
+    const int q = kbt / kblocks;
+    ec = e * p.k_experts + q;
+    kb = kbt - q * kblocks;
+  } else {
+    ec = e;
+    kb = kbt;
+  }
+}
+
+// TMA loads of one stage (single CTA): A rows m0.., B columns n0.. (BN).
+template <bool kAmn, bool kBk>
+__device__ __forceinline__ void load_stage(uint8_t* sa, uint8_t* sb, const CUtensorMap* ma, const CUtensorMap* mb,
+                                           uint64_t* bar, const Params& p, int ec, int kb, int m0, int n0) {
+  const int k0 = kb * BK;
+  if constexpr (kAmn) {
+#pragma unroll
+    for (int q = 0; q < BM / 64; ++q) tma_load_3d(sa + q * A_BOX, ma, bar, m0 + q * 64 + ec * p.a_e0, k0, ec * p.a_e2);
+  } else {
+    tma_load_3d(sa, ma, bar, k0 + ec * p.a_e0, m0, ec * p.a_e2);
+  }
+  if constexpr (kBk) {
+#pragma unroll
+    for (int q = 0; q < BN / 128; ++q)
+      tma_load_3d(sb + q * BK_BOX, mb, bar, k0 + ec * p.b_e0, n0 + q * 128, ec * p.b_e2);
+  } else {
+#pragma unroll
+    for (int q = 0; q < BN / 64; ++q) tma_load_3d(sb + q * B_BOX, mb, bar, n0 + q * 64 + ec * p.b_e0, k0, ec * p.b_e2);
+  }
+}
+
+template <bool kAmn, bool kBk>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                    const Params p) {
@@ -293,6 +403,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int kblocks = (p.K + BK - 1) / BK;
+  const int ksteps = kblocks * (p.k_experts > 0 ? p.k_experts : 1);
+  constexpr uint32_t kId = idesc<kAmn, kBk, BM>();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -302,17 +414,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int64_t tile = blockIdx.x; ok && tile < p.tiles; tile += gridDim.x) {
         int e, mb, nb;
         decode_tile(p, tile, e, mb, nb);
-        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+        for (int kbt = 0; kbt < ksteps; ++kbt, ++it) {
           const uint32_t s = it % STAGES, ph = (it / STAGES) & 1u;
           if (!mbar_wait(&empty[s], ph ^ 1u, abort, p.err)) {
             ok = false;
             break;
           }
+          int ec, kb;
+          k_step(p, e, kbt, kblocks, ec, kb);
           mbar_expect_tx(&full[s], STAGE_BYTES);
-          tma_load_3d(sA + s * A_STAGE, &map_a, &full[s], kb * BK, mb * BM, p.a_batched ? e : 0);
-#pragma unroll
-          for (int q = 0; q < BN / 64; ++q)
-            tma_load_3d(sB + s * B_STAGE + q * B_BOX, &map_b, &full[s], nb * BN + q * 64, kb * BK, e);
+          load_stage<kAmn, kBk>(sA + s * A_STAGE, sB + s * B_STAGE, &map_a, &map_b, &full[s], p, ec, kb, mb * BM,
+                                nb * BN);
         }
       }
       // Drain: the last (up to STAGES) issued loads must have landed before exit.
@@ -330,7 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&tempty[acc], aph ^ 1u, abort, p.err)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
-        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+        for (int kbt = 0; kbt < ksteps; ++kbt, ++it) {
           const uint32_t s = it % STAGES, ph = (it / STAGES) & 1u;
           if (!mbar_wait(&full[s], ph, abort, p.err)) {
             ok = false;
@@ -339,12 +451,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + s * A_STAGE), b0 = smem_u32(sB + s * B_STAGE);
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
-            // A: K-major, advance 16 elements (32 B) inside the swizzle atom.
-            // B: N-major, advance 16 k-rows (2 atoms of 8 rows x 128 B).
-            umma(d_tmem, sw128_desc(a0 + 32 * k, 16, 1024), sw128_desc(b0 + 2048 * k, B_BOX, 1024),
-                 (kb | k) != 0);
-          }
+          for (int k = 0; k < BK / 16; ++k)
+            umma(d_tmem, operand_desc<!kAmn>(a0, k, A_BOX), operand_desc<kBk>(b0, k, B_BOX), kId, (kbt | k) != 0);
           issued = true;
           umma_commit(&empty[s]);
         }
@@ -405,8 +513,7 @@ constexpr int A_STAGE2 = BM * BK * 2;        // this CTA's 128 rows, 16 KB
 constexpr int B_STAGE2 = BK * (BN / 2) * 2;  // this CTA's 128 columns, 16 KB
 constexpr int STAGE2_BYTES = A_STAGE2 + B_STAGE2;
 constexpr int kSmemBytes2 = 1024 + STAGES2 * STAGE2_BYTES + 256;
-constexpr uint32_t kIdesc2 = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((uint32_t)(BN >> 3) << 17) |
-                             ((uint32_t)(2 * BM >> 4) << 24);
+
 
 __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
@@ -438,13 +545,37 @@ __device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* m
       : "memory");
 }
 
-__device__ __forceinline__ void umma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+__device__ __forceinline__ void umma_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc_v,
+                                          uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(kIdesc2), "r"(accumulate)
+      "l"(adesc), "l"(bdesc), "r"(idesc_v), "r"(accumulate)
       : "memory");
+}
+
+// TMA loads of one stage of one CTA of a pair: its 128 rows of A from m0,
+// its 128 columns of B from n0; completion on the even CTA's barrier.
+template <bool kAmn, bool kBk>
+__device__ __forceinline__ void load_stage_pair(uint8_t* sa, uint8_t* sb, const CUtensorMap* ma,
+                                                const CUtensorMap* mb, uint32_t bar, const Params& p, int ec, int kb,
+                                                int m0, int n0) {
+  const int k0 = kb * BK;
+  if constexpr (kAmn) {
+#pragma unroll
+    for (int q = 0; q < BM / 64; ++q)
+      tma_load_3d_pair(sa + q * A_BOX, ma, bar, m0 + q * 64 + ec * p.a_e0, k0, ec * p.a_e2);
+  } else {
+    tma_load_3d_pair(sa, ma, bar, k0 + ec * p.a_e0, m0, ec * p.a_e2);
+  }
+  if constexpr (kBk) {
+    tma_load_3d_pair(sb, mb, bar, k0 + ec * p.b_e0, n0, ec * p.b_e2);
+  } else {
+#pragma unroll
+    for (int q = 0; q < BN / 128; ++q)
+      tma_load_3d_pair(sb + q * B_BOX, mb, bar, n0 + q * 64 + ec * p.b_e0, k0, ec * p.b_e2);
+  }
 }
 
 // Arrive on the barrier at this offset in the CTAs of `mask` when all prior
@@ -463,6 +594,7 @@ __device__ __noinline__ void spin_ns(uint64_t ns) {
   }
 }
 
+template <bool kAmn, bool kBk>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                     const Params p) {
@@ -505,6 +637,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int kblocks = (p.K + BK - 1) / BK;
+  const int ksteps = kblocks * (p.k_experts > 0 ? p.k_experts : 1);
+  constexpr uint32_t kId = idesc<kAmn, kBk, 2 * BM>();
   const int64_t pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
   bool aborted = false;
 
@@ -516,20 +650,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       for (int64_t tile = pair; ok && tile < p.tiles; tile += n_pairs) {
         int e, mb, nb;
         decode_tile(p, tile, e, mb, nb);
-        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+        for (int kbt = 0; kbt < ksteps; ++kbt, ++it) {
           const uint32_t s = it % STAGES2, ph = (it / STAGES2) & 1u;
           if (!mbar_wait(&empty[s], ph ^ 1u, abort, p.err)) {
             ok = false;
             break;
           }
+          int ec, kb;
+          k_step(p, e, kbt, kblocks, ec, kb);
           if (leader) mbar_expect_tx(&full[s], 2 * STAGE2_BYTES);
           const uint32_t bar = mapa(smem_u32(&full[s]), 0);
-          tma_load_3d_pair(sA + s * A_STAGE2, &map_a, bar, kb * BK, mb * 2 * BM + (int)rank * BM,
-                           p.a_batched ? e : 0);
-#pragma unroll
-          for (int q = 0; q < BN / 128; ++q)
-            tma_load_3d_pair(sB + s * B_STAGE2 + q * B_BOX, &map_b, bar, nb * BN + (int)rank * (BN / 2) + q * 64,
-                             kb * BK, e);
+          load_stage_pair<kAmn, kBk>(sA + s * A_STAGE2, sB + s * B_STAGE2, &map_a, &map_b, bar, p, ec, kb,
+                                     mb * 2 * BM + (int)rank * BM, nb * BN + (int)rank * (BN / 2));
         }
       }
       if (leader) {
@@ -552,7 +684,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
-        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+        for (int kbt = 0; kbt < ksteps; ++kbt, ++it) {
           const uint32_t s = it % STAGES2, ph = (it / STAGES2) & 1u;
           if (!mbar_wait(&full[s], ph, abort, p.err)) {
             ok = false;
@@ -562,8 +694,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           const uint32_t a0 = smem_u32(sA + s * A_STAGE2), b0 = smem_u32(sB + s * B_STAGE2);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
-            umma_pair(d_tmem, sw128_desc(a0 + 32 * k, 16, 1024), sw128_desc(b0 + 2048 * k, B_BOX, 1024),
-                      (kb | k) != 0);
+            umma_pair(d_tmem, operand_desc<!kAmn>(a0, k, A_BOX), operand_desc<kBk>(b0, k, B_BOX), kId,
+                      (kbt | k) != 0);
           issued = true;
           umma_commit_pair(&empty[s], 0x3);
         }
@@ -641,15 +773,17 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+template <bool kAmn, bool kBk>
 mole_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, Params p, bool pair_tiles,
                         cudaStream_t stream) {
   static bool attr_set[64][2] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOLE_ERR_CUDA;
   if (!attr_set[dev][pair_tiles]) {
-    const cudaError_t e =
-        pair_tiles ? cudaFuncSetAttribute(gemm_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes2)
-                   : cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    const cudaError_t e = pair_tiles ? cudaFuncSetAttribute(gemm_tc2_kernel<kAmn, kBk>,
+                                                            cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes2)
+                                     : cudaFuncSetAttribute(gemm_tc_kernel<kAmn, kBk>,
+                                                            cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
     if (e != cudaSuccess) return MOLE_ERR_CUDA;
     attr_set[dev][pair_tiles] = true;
   }
@@ -657,12 +791,17 @@ mole_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, Params p, 
   if (n_sm <= 0) return MOLE_ERR_NO_DEVICE;
   if (pair_tiles) {
     const int64_t pairs = std::min<int64_t>(p.tiles, n_sm / 2);
-    gemm_tc2_kernel<<<(unsigned)(2 * pairs), kThreads, kSmemBytes2, stream>>>(ma, mb, p);
+    gemm_tc2_kernel<kAmn, kBk><<<(unsigned)(2 * pairs), kThreads, kSmemBytes2, stream>>>(ma, mb, p);
   } else {
     const int64_t grid = std::min<int64_t>(p.tiles, n_sm);
-    gemm_tc_kernel<<<(unsigned)grid, kThreads, kSmemBytes, stream>>>(ma, mb, p);
+    gemm_tc_kernel<kAmn, kBk><<<(unsigned)grid, kThreads, kSmemBytes, stream>>>(ma, mb, p);
   }
   return cuda_status(cudaGetLastError());
+}
+
+mole_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, Params p, bool pair_tiles,
+                        cudaStream_t stream) {
+  return launch_gemm<false, false>(ma, mb, p, pair_tiles, stream);
 }
 
 }  // namespace
@@ -701,7 +840,8 @@ mole_status shared_ffn_tc(const void* h, const void* W1s, const void* W2s, int64
   p1.M = (int)T;
   p1.N = (int)Ds;
   p1.K = (int)D;
-  p1.a_batched = 0;
+  p1.a_e2 = 0;
+  p1.b_e2 = 1;
   p1.act = act;
   p1.C = H;
   p1.ldc = Ds;
@@ -719,7 +859,8 @@ mole_status shared_ffn_tc(const void* h, const void* W1s, const void* W2s, int64
   p2.M = (int)T;
   p2.N = (int)D;
   p2.K = (int)Ds;
-  p2.a_batched = 1;
+  p2.a_e2 = 1;
+  p2.b_e2 = 1;
   p2.act = MOLE_ACT_IDENTITY;
   p2.ldc = D;
   p2.m_blocks = (int)((T + mtile - 1) / mtile);
@@ -765,7 +906,8 @@ mole_status train_experts_tc(const void* Eu, const void* W1, const void* W2, int
   p1.M = (int)M;
   p1.N = (int)Dr;
   p1.K = (int)D;
-  p1.a_batched = 0;
+  p1.a_e2 = 0;
+  p1.b_e2 = 1;
   p1.act = act;
   p1.C = H;
   p1.ldc = Dr;
@@ -784,7 +926,8 @@ mole_status train_experts_tc(const void* Eu, const void* W1, const void* W2, int
   p2.M = (int)M;
   p2.N = (int)D;
   p2.K = (int)Dr;
-  p2.a_batched = 1;
+  p2.a_e2 = 1;
+  p2.b_e2 = 1;
   p2.act = MOLE_ACT_IDENTITY;
   p2.C = Y;
   p2.ldc = (int64_t)N * D;
@@ -794,6 +937,146 @@ mole_status train_experts_tc(const void* Eu, const void* W1, const void* W2, int
   p2.tiles = (int64_t)N * p2.m_blocks * p2.n_blocks;
   p2.err = err;
   return launch_gemm(ma, mb, p2, pair_tiles, stream);
+}
+
+namespace {
+
+// dE[rowmap[u], :] += sum over the groups s, in order, of part[s][u, :]
+// (each distinct id once).
+__global__ void scatter_parts_kernel(const float* __restrict__ part, int64_t U, int64_t cap, int D, int S,
+                                     const int* __restrict__ rowmap, float* dE) {
+  const int64_t n = U * D;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t u = i / D, d = i - u * D;
+    float acc = 0.f;
+    for (int s = 0; s < S; ++s) acc += part[(int64_t)s * cap * D + i];
+    dE[(int64_t)rowmap[u] * D + d] += acc;
+  }
+}
+
+// Groups of experts for the dE contraction (a sum over all N experts' K):
+// S groups (S divides N) of N / S experts each, one output tile set per
+// group.  Fewer groups mean fewer partial sums to reduce but fewer tiles;
+// pick the S with the least modelled time: waves of tiles over the CTA
+// pairs, each wave as long as its tiles' K, plus a small cost per group.
+int choose_groups(int N, int64_t tiles_per_group, int64_t units) {
+  int best = 1;
+  double best_cost = 1e300;
+  for (int S = 1; S <= N; ++S) {
+    if (N % S != 0) continue;
+    const double waves = (double)((S * tiles_per_group + units - 1) / units);
+    const double cost = waves * (double)(N / S) + 0.1 * S;
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = S;
+    }
+  }
+  return best;
+}
+
+}  // namespace
+
+mole_status train_backward_tc(const uint16_t* dY, const uint16_t* H, const float* pre, const uint16_t* Eu,
+                              const void* W1, const void* W2, int64_t U, int64_t cap, int64_t D, int N, int64_t Dr,
+                              int act, uint16_t* dP, float* part, const int* rowmap, float* dW2, float* dW1,
+                              float* dE, cudaStream_t stream) {
+  if (U <= 0) return MOLE_OK;
+  if (U > (1LL << 31) - 1 || D % 64 != 0 || Dr % 64 != 0) return MOLE_ERR_UNSUPPORTED;
+  unsigned* err = error_word();
+  if (!err) return MOLE_ERR_CUDA;
+  const int n_sm = num_sms();
+  if (n_sm <= 0) return MOLE_ERR_NO_DEVICE;
+  const int64_t ND = (int64_t)N * D;
+  CUtensorMap ma, mb;
+  mole_status st;
+  auto base = [&](Params& q, int64_t M, int64_t Nc, int64_t K, int n_out) {
+    q.M = (int)M;
+    q.N = (int)Nc;
+    q.K = (int)K;
+    const int mtile = M >= 2 * BM ? 2 * BM : BM;
+    q.m_blocks = (int)((M + mtile - 1) / mtile);
+    q.n_blocks = (int)((Nc + BN - 1) / BN);
+    q.tiles = (int64_t)n_out * q.m_blocks * q.n_blocks;
+    q.err = err;
+    return M >= 2 * BM;  // CTA pairs once there are two 128-row blocks
+  };
+  if (dP != nullptr) {
+    // dP[e] = bf16((dY_e . W2[e]^T) * act'(pre[e])): A = dY_e K-major (the
+    // expert's block of each row), B = W2[e]^T K-major (W2[e] rows are k)
+    if (!make_map(&ma, dY, ND, U, 1, ND * 2, U * ND * 2, BM) ||
+        !make_map(&mb, W2, D, Dr, N, D * 2, Dr * D * 2, 128))
+      return MOLE_ERR_CUDA;
+    Params q{};
+    const bool pr = base(q, U, Dr, D, N);
+    q.a_e0 = (int)D;
+    q.b_e2 = 1;
+    q.act = act;
+    q.C = dP;
+    q.ldc = Dr;
+    q.c_estride = cap * Dr;
+    q.grad_pre = pre;
+    q.pre_estride = cap * Dr;
+    if ((st = launch_gemm<false, true>(ma, mb, q, pr, stream)) != MOLE_OK) return st;
+  }
+  if (dW2 != nullptr) {
+    // dW2[e] += H[e]^T . dY_e: A = H[e]^T MN-major (H[e] rows are k of the
+    // contraction), B = dY_e N-major
+    if (!make_map(&ma, H, Dr, U, N, Dr * 2, cap * Dr * 2, BK) || !make_map(&mb, dY, ND, U, 1, ND * 2, U * ND * 2, BK))
+      return MOLE_ERR_CUDA;
+    Params q{};
+    const bool pr = base(q, Dr, D, U, N);
+    q.a_e2 = 1;
+    q.b_e0 = (int)D;
+    q.Cf = dW2;
+    q.add0 = dW2;
+    q.ldc = D;
+    q.cf_estride = Dr * D;
+    if ((st = launch_gemm<true, false>(ma, mb, q, pr, stream)) != MOLE_OK) return st;
+  }
+  if (dW1 != nullptr) {
+    // dW1[e] += Eu^T . dP[e]: A = Eu^T MN-major, B = dP[e] N-major
+    if (!make_map(&ma, Eu, D, U, 1, D * 2, U * D * 2, BK) || !make_map(&mb, dP, Dr, U, N, Dr * 2, cap * Dr * 2, BK))
+      return MOLE_ERR_CUDA;
+    Params q{};
+    const bool pr = base(q, D, Dr, U, N);
+    q.b_e2 = 1;
+    q.Cf = dW1;
+    q.add0 = dW1;
+    q.ldc = Dr;
+    q.cf_estride = D * Dr;
+    if ((st = launch_gemm<true, false>(ma, mb, q, pr, stream)) != MOLE_OK) return st;
+  }
+  if (dE != nullptr) {
+    // sum_e dP[e] . W1[e]^T: A = dP[e] K-major, B = W1[e]^T K-major (W1[e]
+    // rows are d), the contraction over a group of experts' K ranges
+    if (!make_map(&ma, dP, Dr, U, N, Dr * 2, cap * Dr * 2, BM) ||
+        !make_map(&mb, W1, Dr, D, N, Dr * 2, D * Dr * 2, 128))
+      return MOLE_ERR_CUDA;
+    Params q{};
+    const bool pr = base(q, U, D, Dr, 1);
+    const int S = choose_groups(N, q.tiles, pr ? n_sm / 2 : n_sm);
+    q.tiles *= S;
+    q.a_e2 = 1;
+    q.b_e2 = 1;
+    q.k_experts = N / S;
+    q.ldc = D;
+    if (S == 1) {  // one group: straight into dE's rows
+      q.Cf = dE;
+      q.add0 = dE;
+      q.c_rowmap = rowmap;
+    } else {
+      q.Cf = part;
+      q.cf_estride = cap * D;
+    }
+    if ((st = launch_gemm<false, true>(ma, mb, q, pr, stream)) != MOLE_OK) return st;
+    if (S > 1) {
+      const int64_t n = U * D;
+      const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, (int64_t)n_sm * 16));
+      scatter_parts_kernel<<<grid, 256, 0, stream>>>(part, U, cap, (int)D, S, rowmap, dE);
+      if (cudaGetLastError() != cudaSuccess) return MOLE_ERR_CUDA;
+    }
+  }
+  return MOLE_OK;
 }
 
 mole_status build_tc_nf3(const void* E, const void* W1, const void* W2, int64_t V, int64_t D, int N, int64_t Dr,
@@ -829,7 +1112,8 @@ mole_status build_tc_any(const void* E, const void* W1, const void* W2, int64_t 
     p1.M = (int)V;
     p1.N = (int)Dr;
     p1.K = (int)D;
-    p1.a_batched = 0;
+    p1.a_e2 = 0;
+    p1.b_e2 = 1;
     p1.act = act;
     p1.C = H;
     p1.ldc = Dr;
@@ -847,7 +1131,8 @@ mole_status build_tc_any(const void* E, const void* W1, const void* W2, int64_t 
     p2.M = (int)V;
     p2.N = (int)D;
     p2.K = (int)Dr;
-    p2.a_batched = 1;
+    p2.a_e2 = 1;
+    p2.b_e2 = 1;
     p2.act = MOLE_ACT_IDENTITY;
     if (codes != nullptr) {
       const int64_t nb = D / 64;  // NF3 blocks per row

@@ -120,6 +120,36 @@ __device__ __forceinline__ float act_t(float x) {
   }
 }
 
+// Derivative of the expert activation at u, kind fixed at compile time (the
+// training backward's dL/dpre = dL/dH * act'(pre)).  GELU: Phi(u) + u phi(u),
+// Phi through the same Abramowitz & Stegun 7.1.26 erfc as the forward.
+template <int ACT>
+__device__ __forceinline__ float act_grad_t(float u) {
+  if constexpr (ACT == MOLE_ACT_GELU_ERF) {
+    const float x = fabsf(u) * 0.7071067811865476f;
+    const float t = __fdividef(1.0f, fmaf(0.3275911f, x, 1.0f));
+    float poly = fmaf(1.061405429f, t, -1.453152027f);
+    poly = fmaf(poly, t, 1.421413741f);
+    poly = fmaf(poly, t, -0.284496736f);
+    poly = fmaf(poly, t, 0.254829592f);
+    const float e = __expf(-x * x);                      // exp(-u^2 / 2)
+    const float half_erfc = 0.5f * (poly * t) * e;
+    const float Phi = u >= 0.f ? 1.0f - half_erfc : half_erfc;
+    return fmaf(u * 0.3989422804014327f, e, Phi);       // + u phi(u), phi(u) = e / sqrt(2 pi)
+  } else if constexpr (ACT == MOLE_ACT_GELU_TANH) {
+    const float c = 0.7978845608028654f;
+    const float th = tanhf(c * fmaf(0.044715f * u, u * u, u));
+    return 0.5f * (1.f + th) + 0.5f * u * (1.f - th * th) * c * fmaf(3.f * 0.044715f, u * u, 1.f);
+  } else if constexpr (ACT == MOLE_ACT_RELU) {
+    return u > 0.f ? 1.f : 0.f;
+  } else if constexpr (ACT == MOLE_ACT_SILU) {
+    const float sg = __fdividef(1.f, 1.f + __expf(-u));
+    return sg * fmaf(u, 1.f - sg, 1.f);
+  } else {
+    return 1.f;
+  }
+}
+
 // Expert FFN activation (reading of the page's "GELU FFN": exact GELU x*Phi(x)).
 __device__ __forceinline__ float apply_act(int act, float x) {
   switch (act) {
@@ -148,6 +178,18 @@ mole_status build_tc(const void* E, const void* W1, const void* W2, int64_t V, i
 // The routed experts of a training step on the rows of Eu (build_tc.cu).
 mole_status train_experts_tc(const void* Eu, const void* W1, const void* W2, int64_t M, int64_t ld_rows, int64_t D,
                              int N, int64_t Dr, int act, uint16_t* H, float* pre, uint16_t* Y, cudaStream_t stream);
+// The four expert GEMMs of a training step's backward (build_tc.cu), on the
+// U distinct ids' rows (matrices of `cap` rows per expert, the first U used):
+//   dP[e]  = bf16((dY[:, e, :] . W2[e]^T) * act'(pre[e]))       dY [cap, N, D] bf16
+//   dW2[e] += H[e]^T . dY[:, e, :]                              H, pre, dP [N, cap, Dr]
+//   dW1[e] += Eu^T . dP[e]                                      Eu [cap, D] bf16
+//   dE[rowmap[u]] += sum_e dP[e][u] . W1[e]^T                   part [N, cap, D] fp32 scratch
+// Each is one tcgen05 GEMM launch (the last plus a reduction over groups of
+// experts when the sum is split); any of dW2, dW1, dE may be null.
+mole_status train_backward_tc(const uint16_t* dY, const uint16_t* H, const float* pre, const uint16_t* Eu,
+                              const void* W1, const void* W2, int64_t U, int64_t cap, int64_t D, int N, int64_t Dr,
+                              int act, uint16_t* dP, float* part, const int* rowmap, float* dW2, float* dW1,
+                              float* dE, cudaStream_t stream);
 // The build with the NF3 quantiser in the second GEMM's epilogue (no bf16 table).
 mole_status build_tc_nf3(const void* E, const void* W1, const void* W2, int64_t V, int64_t D, int N, int64_t Dr,
                          int act, uint8_t* codes, uint16_t* scales, void* ws, size_t ws_bytes, cudaStream_t stream);

@@ -18,14 +18,13 @@
 //   dh[t] += dz[t] . Wr^T,  dWr += h^T dz                 (gate_grad_kernel; dwr_kernel per
 //                                                          block of tokens, then dwr_reduce_kernel)
 //   dY[u, j] = sum_{t: u(t) = u} g_j[t] dout[t]           (dy_kernel, one CTA per distinct id)
-//   dpre_j = (dY_j . W2_j^T) * act'(pre_j)                (cuBLAS + act_grad_kernel)
-//   dW2_j += H_j^T dY_j,  dW1_j += Eu^T dpre_j,  dE[ids] += sum_j dpre_j . W1_j^T
-//                                                         (cuBLAS batched over the experts,
-//                                                          scatter_rows_kernel sums the experts)
-// The backward GEMMs are plain transposed bf16 GEMMs with fp32 accumulation
-// and run in cuBLAS; their bf16 operands dY and dpre are rounded from fp32.
-#include <cublas_v2.h>
-
+//   dpre_j = (dY_j . W2_j^T) * act'(pre_j)                (tcgen05 GEMM, derivative in its epilogue)
+//   dW2_j += H_j^T dY_j,  dW1_j += Eu^T dpre_j             (tcgen05 GEMMs batched over the experts,
+//                                                          fp32 gradients added in the epilogue)
+//   dE[ids] += sum_j dpre_j . W1_j^T                      (tcgen05 GEMM whose contraction runs over
+//                                                          the experts, rows scattered by id)
+// The backward GEMMs are the table build's kernels with transposed operand
+// forms (build_tc.cu); their bf16 operands dY and dpre are rounded from fp32.
 #include "groups.cuh"
 
 namespace mole {
@@ -33,7 +32,6 @@ namespace {
 
 constexpr int kGradThreads = 256;
 constexpr int kDwrTokens = 256;  // tokens per block of dwr_kernel
-constexpr int64_t kCublasWorkspace = int64_t(32) << 20;
 
 // The caller's cache buffer (cap = min(T, V) row capacity).
 struct TrainCache {
@@ -43,12 +41,10 @@ struct TrainCache {
   float* pre;     // [N, cap, Dr] fp32
   float* g;       // [T, N] gates
   float* dz;      // [T, N] logit gradients
-  float* dY;      // [cap, N, D] fp32
-  uint16_t* dYb;  // [cap, N, D] bf16
-  uint16_t* dP;   // [N, cap, Dr] bf16: dL/dpre (first dL/dH)
-  float* dEu;     // [N, cap, D] fp32: each expert's share of dL/dEu
+  uint16_t* dYb;  // [cap, N, D] bf16: dL/dY by distinct id
+  uint16_t* dP;   // [N, cap, Dr] bf16: dL/dpre
+  float* dEu;     // [N, cap, D] fp32: partial sums of dL/dEu over groups of experts
   float* dWrp;    // [ceil(T / kDwrTokens), D, N] fp32: dWr per block of tokens
-  void* blas_ws;  // cuBLAS workspace
   int* U;         // one device int
   size_t total;
 };
@@ -67,12 +63,10 @@ size_t carve_cache(void* base, int64_t T, int64_t V, int N, int64_t D, int64_t D
   const size_t o_pre = take(4 * (size_t)N * cap * Dr);
   const size_t o_g = take(4 * (size_t)T * N);
   const size_t o_dz = take(4 * (size_t)T * N);
-  const size_t o_dy = take(4 * (size_t)cap * N * D);
   const size_t o_dyb = take(2 * (size_t)cap * N * D);
   const size_t o_dp = take(2 * (size_t)N * cap * Dr);
   const size_t o_deu = take(4 * (size_t)N * cap * D);
   const size_t o_dwr = take(4 * (size_t)((T + kDwrTokens - 1) / kDwrTokens) * D * N);
-  const size_t o_ws = take((size_t)kCublasWorkspace);
   const size_t o_u = take(16);
   if (c != nullptr && base != nullptr) {
     uint8_t* b = static_cast<uint8_t*>(base);
@@ -82,12 +76,10 @@ size_t carve_cache(void* base, int64_t T, int64_t V, int N, int64_t D, int64_t D
     c->pre = reinterpret_cast<float*>(b + o_pre);
     c->g = reinterpret_cast<float*>(b + o_g);
     c->dz = reinterpret_cast<float*>(b + o_dz);
-    c->dY = reinterpret_cast<float*>(b + o_dy);
     c->dYb = reinterpret_cast<uint16_t*>(b + o_dyb);
     c->dP = reinterpret_cast<uint16_t*>(b + o_dp);
     c->dEu = reinterpret_cast<float*>(b + o_deu);
     c->dWrp = reinterpret_cast<float*>(b + o_dwr);
-    c->blas_ws = b + o_ws;
     c->U = reinterpret_cast<int*>(b + o_u);
     c->total = off;
   }
@@ -95,31 +87,6 @@ size_t carve_cache(void* base, int64_t T, int64_t V, int N, int64_t D, int64_t D
 }
 
 __device__ __forceinline__ float ld_bf16(const uint16_t* p) { return __uint_as_float((uint32_t)*p << 16); }
-
-// Derivative of the expert activation at the pre-activation u.
-__device__ __forceinline__ float act_grad(int act, float u) {
-  switch (act) {
-    case MOLE_ACT_GELU_ERF: {  // Phi(u) + u phi(u)
-      const float Phi = 0.5f * erfcf(-u * 0.70710678118654752f);
-      const float phi = 0.39894228040143268f * expf(-0.5f * u * u);
-      return Phi + u * phi;
-    }
-    case MOLE_ACT_GELU_TANH: {  // d/du 0.5 u (1 + tanh(c (u + 0.044715 u^3)))
-      const float c = 0.79788456080286536f;
-      const float k = c * (u + 0.044715f * u * u * u);
-      const float th = tanhf(k);
-      return 0.5f * (1.f + th) + 0.5f * u * (1.f - th * th) * c * (1.f + 3.f * 0.044715f * u * u);
-    }
-    case MOLE_ACT_RELU:
-      return u > 0.f ? 1.f : 0.f;
-    case MOLE_ACT_SILU: {
-      const float s = 1.f / (1.f + expf(-u));
-      return s * (1.f + u * (1.f - s));
-    }
-    default:
-      return 1.f;
-  }
-}
 
 // One warp per token: the gates (router logits h[t] . Wr in fp32, softmax),
 // dg_j = <dout[t], Y[u(t), j]>, dz = g (dg - <g, dg>), and dh[t] += dz . Wr^T.
@@ -237,7 +204,7 @@ __global__ void dwr_reduce_kernel(const float* __restrict__ part, int n_blocks, 
 }
 
 // dY[u, j, d] = sum over the tokens t of id u, in list order, of
-// g[t, j] dout[t, d].  Work unit = (work item, slice of kGradThreads
+// g[t, j] dout[t, d], rounded to bf16 (the operand of the backward GEMMs).  Work unit = (work item, slice of kGradThreads
 // consecutive d); only units of an id's first work item do work, over all of
 // the id's tokens, so the sums do not depend on scheduling and a frequent id
 // spreads over D / kGradThreads CTAs.  A thread holds the N sums of its d;
@@ -247,7 +214,7 @@ constexpr int kDyChunk = 64;
 
 template <int NP>
 __global__ void __launch_bounds__(kGradThreads) dy_kernel(const GroupWs w, const float* __restrict__ g,
-                                                          const float* __restrict__ dout, int N, int D, float* dY) {
+                                                          const float* __restrict__ dout, int N, int D, uint16_t* dY) {
   __shared__ int toks[kDyChunk];
   __shared__ float gs[kDyChunk][NP];
   __shared__ int cnt_s;
@@ -296,70 +263,17 @@ __global__ void __launch_bounds__(kGradThreads) dy_kernel(const GroupWs w, const
       }
     }
     if (d < D) {
-      float* dst = dY + (int64_t)rec.w * N * D + d;
+      uint16_t* dst = dY + (int64_t)rec.w * N * D + d;
 #pragma unroll
       for (int j = 0; j < NP; ++j)
-        if (j < N) dst[(int64_t)j * D] = acc[j];
+        if (j < N) dst[(int64_t)j * D] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[j]));
     }
-  }
-}
-
-__global__ void to_bf16_kernel(const float* __restrict__ x, uint16_t* __restrict__ y, int64_t n) {
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
-    y[i] = __bfloat16_as_ushort(__float2bfloat16_rn(x[i]));
-}
-
-// dP = bf16(dH * act'(pre)) over the first U rows of each expert's [cap, Dr] block.
-__global__ void act_grad_kernel(uint16_t* dP, const float* __restrict__ pre, int64_t U, int64_t cap, int64_t Dr,
-                                int N, int act) {
-  const int64_t per = U * Dr, n = per * N;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t j = i / per, r = i - j * per;
-    const int64_t k = j * cap * Dr + r;
-    const float dh = ld_bf16(dP + k);
-    dP[k] = __bfloat16_as_ushort(__float2bfloat16_rn(dh * act_grad(act, pre[k])));
-  }
-}
-
-// dE[id(u), :] += sum_j dEu[j, u, :] (each distinct id once; experts summed
-// in order).
-__global__ void scatter_rows_kernel(const GroupWs w, const float* __restrict__ dEu, int64_t U, int64_t cap, int D,
-                                    int N, float* dE) {
-  const int64_t n = U * D;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t u = i / D, d = i - u * D;
-    float acc = 0.f;
-    for (int j = 0; j < N; ++j) acc += dEu[(int64_t)j * cap * D + i];
-    dE[(int64_t)w.uid_id[u] * D + d] += acc;
   }
 }
 
 unsigned grid_for(int64_t n, int per_block) {
   const int n_sm = num_sms();
   return (unsigned)std::max<int64_t>(1, std::min<int64_t>((n + per_block - 1) / per_block, (int64_t)n_sm * 16));
-}
-
-// ---- cuBLAS: one handle per device, bound to the caller's stream and to a
-// workspace in the cache at each call ----
-cublasHandle_t blas_handle() {
-  static cublasHandle_t handles[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (handles[dev] == nullptr && cublasCreate(&handles[dev]) != CUBLAS_STATUS_SUCCESS) handles[dev] = nullptr;
-  return handles[dev];
-}
-
-// Row-major C[M, N] (ldc, stride sC) = alpha op(A)[M, K] op(B)[K, N] + beta C,
-// `batch` times: A, B bf16 (row-major, lda / ldb, strides sA / sB); C fp32 or
-// bf16.  (cuBLAS is column-major: it computes C^T = op(B)^T op(A)^T.)
-bool rm_gemm(cublasHandle_t hb, bool ta, bool tb, int64_t M, int64_t N, int64_t K, const void* A, int64_t lda,
-             int64_t sA, const void* B, int64_t ldb, int64_t sB, float beta, void* C, bool c_f32, int64_t ldc, int64_t sC,
-             int batch) {
-  const float alpha = 1.f;
-  return cublasGemmStridedBatchedEx(hb, tb ? CUBLAS_OP_T : CUBLAS_OP_N, ta ? CUBLAS_OP_T : CUBLAS_OP_N, (int)N,
-                                    (int)M, (int)K, &alpha, B, CUDA_R_16BF, (int)ldb, sB, A, CUDA_R_16BF, (int)lda,
-                                    sA, &beta, C, c_f32 ? CUDA_R_32F : CUDA_R_16BF, (int)ldc, sC, batch,
-                                    CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT) == CUBLAS_STATUS_SUCCESS;
 }
 
 }  // namespace
@@ -429,41 +343,17 @@ mole_status train_backward(const void* groups, size_t gbytes, int64_t T, const v
     if (cudaGetLastError() != cudaSuccess) return MOLE_ERR_CUDA;
   }
   if (U == 0 || (dE == nullptr && dW1 == nullptr && dW2 == nullptr)) return MOLE_OK;
-  // dY by distinct id, then its bf16 copy for the GEMMs
-  const int64_t ny = (int64_t)U * N * D;
+  // dY by distinct id (bf16), then the expert GEMMs
   if (N <= 8)
-    dy_kernel<8><<<(unsigned)n_sm * 4, kGradThreads, 0, stream>>>(w, c.g, dout, N, (int)D, c.dY);
+    dy_kernel<8><<<(unsigned)n_sm * 4, kGradThreads, 0, stream>>>(w, c.g, dout, N, (int)D, c.dYb);
   else if (N <= 16)
-    dy_kernel<16><<<(unsigned)n_sm * 4, kGradThreads, 0, stream>>>(w, c.g, dout, N, (int)D, c.dY);
+    dy_kernel<16><<<(unsigned)n_sm * 4, kGradThreads, 0, stream>>>(w, c.g, dout, N, (int)D, c.dYb);
   else
-    dy_kernel<32><<<(unsigned)n_sm * 4, kGradThreads, 0, stream>>>(w, c.g, dout, N, (int)D, c.dY);
-  to_bf16_kernel<<<grid_for(ny, 256), 256, 0, stream>>>(c.dY, c.dYb, ny);
+    dy_kernel<32><<<(unsigned)n_sm * 4, kGradThreads, 0, stream>>>(w, c.g, dout, N, (int)D, c.dYb);
   if (cudaGetLastError() != cudaSuccess) return MOLE_ERR_CUDA;
-  cublasHandle_t hb = blas_handle();
-  if (hb == nullptr || cublasSetStream(hb, stream) != CUBLAS_STATUS_SUCCESS ||
-      cublasSetWorkspace(hb, c.blas_ws, (size_t)kCublasWorkspace) != CUBLAS_STATUS_SUCCESS)
-    return MOLE_ERR_CUDA;
-  // dH_j = dY_j . W2_j^T -> dP (bf16), then dP = dH * act'(pre)
-  if (!rm_gemm(hb, false, true, U, Dr, D, c.dYb, (int64_t)N * D, D, W2, D, Dr * D, 0.f, c.dP, false, Dr, cap * Dr, N))
-    return MOLE_ERR_CUDA;
-  act_grad_kernel<<<grid_for((int64_t)N * U * Dr, 256), 256, 0, stream>>>(c.dP, c.pre, U, cap, Dr, N, act);
-  if (cudaGetLastError() != cudaSuccess) return MOLE_ERR_CUDA;
-  // dW2_j += H_j^T dY_j
-  if (dW2 != nullptr &&
-      !rm_gemm(hb, true, false, Dr, D, U, c.H, Dr, cap * Dr, c.dYb, (int64_t)N * D, D, 1.f, dW2, true, D, Dr * D, N))
-    return MOLE_ERR_CUDA;
-  // dW1_j += Eu^T dP_j
-  if (dW1 != nullptr &&
-      !rm_gemm(hb, true, false, D, Dr, U, c.Eu, D, 0, c.dP, Dr, cap * Dr, 1.f, dW1, true, Dr, D * Dr, N))
-    return MOLE_ERR_CUDA;
-  // dEu_j = dP_j . W1_j^T for all experts in one batched GEMM, then
-  // dE[ids] += sum_j dEu_j
-  if (dE != nullptr) {
-    if (!rm_gemm(hb, false, true, U, D, Dr, c.dP, Dr, cap * Dr, W1, Dr, D * Dr, 0.f, c.dEu, true, D, cap * D, N))
-      return MOLE_ERR_CUDA;
-    scatter_rows_kernel<<<grid_for((int64_t)U * D, 256), 256, 0, stream>>>(w, c.dEu, U, cap, (int)D, N, dE);
-    if (cudaGetLastError() != cudaSuccess) return MOLE_ERR_CUDA;
-  }
+  const bool need_dp = dW1 != nullptr || dE != nullptr;
+  return train_backward_tc(c.dYb, c.H, c.pre, c.Eu, W1, W2, U, cap, D, N, Dr, act, need_dp ? c.dP : nullptr, c.dEu,
+                           w.uid_id, dW2, dW1, dE, stream);
   return MOLE_OK;
 }
 

@@ -227,7 +227,8 @@ def _act64_grad(name, u):
     return np.ones_like(u)
 
 
-def train_step(ids, h, Wr, E, W1, W2, act_name: str = "gelu", dout=None, round_h: bool = True):
+def train_step(ids, h, Wr, E, W1, W2, act_name: str = "gelu", dout=None, round_h: bool = True,
+               round_ops: bool = False):
     """One MoLE layer in training, forward and backward, in fp64 (numpy).
 
     MoLE page, 训练阶段: the routed experts take the token's embedding row,
@@ -238,6 +239,14 @@ def train_step(ids, h, Wr, E, W1, W2, act_name: str = "gelu", dout=None, round_h
     rounding as identity).  Returns (out, grads) where grads holds the
     gradients of L = sum(out * dout): dh, dWr, dE, dW1, dW2 (all fp64).
     Every id must lie in [0, V).
+
+    A routed expert's output depends on the token id alone, so the experts
+    are evaluated once per distinct id and the per-token terms summed by id
+    (equal to the per-token definition; a pin checks that on tiny inputs).
+    round_ops (with round_h) adds the bf16 precision points of a bf16 device
+    step: the expert outputs held as a bf16 table row, dL/dY (summed over a
+    distinct id's tokens) and dL/dpre, each the bf16 operand of a backward
+    contraction, rounded to bf16 (ties to even) where the device rounds them.
     """
     ids = np.asarray(ids, dtype=np.int64)
     hf, Wrf, Ef, W1f, W2f = (_bits_f64(x) for x in (h, Wr, E, W1, W2))
@@ -249,6 +258,8 @@ def train_step(ids, h, Wr, E, W1, W2, act_name: str = "gelu", dout=None, round_h
     if round_h:
         a = round_bf16_array(a)
     Y = np.einsum("jur,jrd->ujd", a, W2f)              # [U, N, D]
+    if round_ops:
+        Y = round_bf16_array(Y)
     z = hf @ Wrf
     z = z - z.max(axis=1, keepdims=True)
     g = np.exp(z)
@@ -261,8 +272,12 @@ def train_step(ids, h, Wr, E, W1, W2, act_name: str = "gelu", dout=None, round_h
         dz = g * (dg - (g * dg).sum(axis=1, keepdims=True))
         dY = np.zeros_like(Y)
         np.add.at(dY, inv, g[:, :, None] * do[:, None, :])
+        if round_ops:
+            dY = round_bf16_array(dY)
         dA = np.einsum("ujd,jrd->jur", dY, W2f)
         dpre = dA * _act64_grad(act_name, pre)
+        if round_ops:
+            dpre = round_bf16_array(dpre)
         dE = np.zeros_like(Ef)
         dE[uniq] = np.einsum("jur,jdr->ud", dpre, W1f)
         grads = {"dh": dz @ Wrf.T, "dWr": hf.T @ dz, "dE": dE,

@@ -49,12 +49,16 @@ def mole():
 def pytest_terminal_summary(terminalreporter):
     """Table-build diagnostics of the session (one line per comparison)."""
     try:
-        from helpers import BUILD_DIAG
+        from helpers import BUILD_DIAG, ERR_DIAG
     except ImportError:
         return
+    tr = terminalreporter
+    if ERR_DIAG:
+        tr.write_sep("-", "measured errors against the oracle")
+        for label, v in ERR_DIAG:
+            tr.write_line(f"{label[:100]:100s} {v:.3e}")
     if not BUILD_DIAG:
         return
-    tr = terminalreporter
     tr.write_sep("-", "table build vs oracle (bf16 ulps; floor 2^-8 rms(row))")
     for d in BUILD_DIAG:
         tr.write_line(f"{d['label'][:60]:60s} n={d['elements']:>9d} beyond-allow {d['max_ulps_beyond_allowance']:.2f} "

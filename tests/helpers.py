@@ -21,6 +21,8 @@ BUILD_ROW_RTOL = 2.0 ** -8
 # diagnostics of every build comparison made in this session (printed in the
 # terminal summary): see assert_build_close
 BUILD_DIAG: list = []
+# other measured errors of the session (label, value), printed likewise
+ERR_DIAG: list = []
 
 
 def dev(a: np.ndarray, device="cuda") -> torch.Tensor:

@@ -509,6 +509,60 @@ def test_train_step_gradients_match_finite_differences(oracle_mod, act):
             assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, fd, an)
 
 
+def test_train_step_equals_the_per_token_definition(oracle_mod):
+    """Brute force on tiny inputs: every token evaluates every expert on its
+    own embedding row (no grouping by id), its output and its share of every
+    gradient accumulated token by token; the oracle's evaluation once per
+    distinct id must give the same numbers (ids repeat here)."""
+    from scipy.special import erf
+    ids, h, Wr, E, W1, W2, dout = _train_inputs(82, T=9, V=4)
+    assert len(np.unique(ids)) < len(ids)
+    out_o, g_o = oracle_mod.train_step(ids, h, Wr, E, W1, W2, "gelu", dout, round_h=False)
+    T, D = h.shape
+    N, _, Dr = W1.shape
+    gelu = lambda u: 0.5 * u * (1.0 + erf(u / np.sqrt(2.0)))
+    dgelu = lambda u: 0.5 * (1.0 + erf(u / np.sqrt(2.0))) + u * np.exp(-0.5 * u * u) / np.sqrt(2.0 * np.pi)
+    out = np.zeros((T, D))
+    dh, dWr, dE = np.zeros_like(h), np.zeros_like(Wr), np.zeros_like(E)
+    dW1, dW2 = np.zeros_like(W1), np.zeros_like(W2)
+    for t in range(T):
+        x = E[ids[t]]
+        z = h[t] @ Wr
+        gt = np.exp(z - z.max())
+        gt /= gt.sum()
+        ys = []
+        for j in range(N):
+            u = x @ W1[j]
+            y = gelu(u) @ W2[j]
+            ys.append(y)
+            out[t] += gt[j] * y
+            dy = gt[j] * dout[t]                       # dL/dy of this token's expert j
+            du = (W2[j] @ dy) * dgelu(u)
+            dW2[j] += np.outer(gelu(u), dy)
+            dW1[j] += np.outer(x, du)
+            dE[ids[t]] += W1[j] @ du
+        dg = np.array([dout[t] @ y for y in ys])
+        dz = gt * (dg - gt @ dg)
+        dh[t] = Wr @ dz
+        dWr += np.outer(h[t], dz)
+    np.testing.assert_allclose(out_o, out, rtol=1e-12, atol=1e-13)
+    for name, ref in (("dh", dh), ("dWr", dWr), ("dE", dE), ("dW1", dW1), ("dW2", dW2)):
+        np.testing.assert_allclose(g_o[name], ref, rtol=1e-11, atol=1e-12, err_msg=name)
+
+
+def test_train_step_precision_points(oracle_mod):
+    """round_ops rounds the expert rows, dL/dY and dL/dpre to bf16: each of
+    those arrays then holds only bf16 values, and the gradients move from the
+    unrounded ones by no more than the bf16 rounding level."""
+    ids, h, Wr, E, W1, W2, dout = _train_inputs(83, T=11, V=5, D=8, N=3, Dr=16)
+    _, g0 = oracle_mod.train_step(ids, h, Wr, E, W1, W2, "gelu", dout)
+    out1, g1 = oracle_mod.train_step(ids, h, Wr, E, W1, W2, "gelu", dout, round_ops=True)
+    for name in g0:
+        rel = np.linalg.norm(g1[name] - g0[name]) / np.linalg.norm(g0[name])
+        assert 0 < rel < 2 ** -6, (name, rel)
+    assert np.isfinite(out1).all()
+
+
 def test_train_forward_is_build_plus_combine(oracle_mod):
     # the training forward equals the inference path: the table built by the
     # oracle (experts on every embedding row) and the oracle combine

@@ -7,24 +7,32 @@ the router on the previous layer's output.
 Forward: equal to the inference path (mole_build_lut, then
 mole_lookup_combine on the same ids) -- the same kernels on the same rows; the
 expert GEMM may take its single-CTA or CTA-pair form depending on the row
-count, so the comparison allows fp32 rounding (2e-6 relative) -- and that path
-is itself checked against the oracle.  Backward: per gradient tensor ||gpu - ref||_2 / ||ref||_2 within
-GRAD_RTOL (the backward GEMMs take bf16 operands -- dL/dY, dL/dpre, the bf16
-expert rows and hidden activations -- each rounded with relative error up to
-2^-9) or within ROUTER_RTOL for dh and dWr (fp32 arithmetic on bf16 expert
-rows, whose rounding the oracle does not do).
+count, so the comparison allows fp32 rounding (2e-6 relative) -- and per
+token within FWD_RTOL of the oracle's output on its bf16-rounded expert rows
+(an expert row element that fp32 and fp64 round to neighbouring bf16 values
+moves a token's output by about 2^-8 / sqrt(D) relative).
+Backward: the oracle rounds where the device rounds (hidden activation,
+expert rows, dL/dY and dL/dpre: the bf16 operands of the backward GEMMs), so
+what remains is fp32 accumulation and the rare bf16 rounding of a value that
+fp32 and fp64 put on different sides of a rounding boundary (one bf16 ulp of
+that element).  Per gradient tensor ||gpu - ref||_2 / ||ref||_2 within
+GRAD_RTOL (expert gradients) or ROUTER_RTOL (dh, dWr: fp32 arithmetic on the
+same bf16 rows).
 """
 import numpy as np
 import pytest
 import torch
 
-from helpers import dev
+import os
+
+from helpers import ERR_DIAG, dev
 from mixture_lookup_experts_b200 import inputs
 
 pytestmark = pytest.mark.gpu
 
-GRAD_RTOL = 2e-2
-ROUTER_RTOL = 1e-2
+GRAD_RTOL = 1e-3
+ROUTER_RTOL = 5e-4
+FWD_RTOL = 4e-3
 
 
 def _layer(seed, T, V, D, N, Dr, kind="zipf"):
@@ -71,14 +79,19 @@ def test_train_step_matches_inference_and_oracle(mole, oracle_mod, T, V, D, N, D
     ref_out = mole.mole_lookup_combine(dids, dh_, dWr_, lut)
     assert mole.mole_check() == 0
     torch.testing.assert_close(out, ref_out, rtol=2e-6, atol=1e-8)
-    # backward against the oracle
+    # backward (and forward) against the oracle at the device's precision points
     g = _grads(mole, dids, groups, dh_, dWr_, dE_, dW1_, dW2_, dev(dout), cache, U, act)
     assert mole.mole_check() == 0
-    _, ref = oracle_mod.train_step(ids, h, Wr, E, W1, W2, act, dout)
+    ref_o, ref = oracle_mod.train_step(ids, h, Wr, E, W1, W2, act, dout, round_ops=True)
+    here = os.environ.get("PYTEST_CURRENT_TEST", "").split("::")[-1]
+    fwd = float((np.linalg.norm(out.cpu().numpy() - ref_o, axis=1) / np.linalg.norm(ref_o, axis=1)).max())
+    ERR_DIAG.append((f"{here} out (max token rel L2)", fwd))
+    assert fwd <= FWD_RTOL
     for name, tol in [("dh", ROUTER_RTOL), ("dWr", ROUTER_RTOL), ("dE", GRAD_RTOL), ("dW1", GRAD_RTOL),
                       ("dW2", GRAD_RTOL)]:
         got = g[name].cpu().numpy()
         assert np.isfinite(got).all(), name
+        ERR_DIAG.append((f"{here} {name} (rel L2)", _rel(got, ref[name])))
         assert _rel(got, ref[name]) <= tol, (name, _rel(got, ref[name]))
     # dE touches only the batch's rows
     untouched = np.setdiff1d(np.arange(V), ids)
@@ -122,7 +135,7 @@ def test_train_bad_ids(mole, oracle_mod):
     g = _grads(mole, dids, groups, dh_, dWr_, dE_, dW1_, dW2_, dev(dout), cache, U, "gelu")
     assert mole.mole_check() == 0
     # the oracle on the good tokens only (a bad token contributes nothing)
-    _, ref = oracle_mod.train_step(ids[~bad], h[~bad], Wr, E, W1, W2, "gelu", dout[~bad])
+    _, ref = oracle_mod.train_step(ids[~bad], h[~bad], Wr, E, W1, W2, "gelu", dout[~bad], round_ops=True)
     assert not g["dh"][torch.from_numpy(np.flatnonzero(bad)).cuda()].any()
     assert _rel(g["dh"].cpu().numpy()[~bad], ref["dh"]) <= ROUTER_RTOL
     for name in ("dE", "dW1", "dW2"):
