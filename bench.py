@@ -948,16 +948,30 @@ def train_leg(mole, rng, g, dev, stream, W, peaks):
     return res
 
 
-def graph_pass_us(passes, stream, dev, replays=60):
+def graph_pass_us(passes, stream, dev, replays=60, flush=None):
     """Median device time (us) of one replay of a CUDA graph captured from
     each of `passes` (one graph per pooled batch, replayed in rotation), and
-    the same passes run eagerly (host-launched) for comparison.  Returns
-    (graph_us or None, eager_us, note)."""
+    the same passes run eagerly (host-launched) for comparison.  With
+    `flush` (a device buffer larger than L2) the buffer is rewritten before
+    every timed pass, outside its events, so each pass starts with a cold L2.
+    Returns (graph_us or None, eager_us, note)."""
     import torch
     P = len(passes)
+
+    def timed(run, n):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        for i in range(n):
+            if flush is not None:
+                flush.fill_(i & 0xff)
+            ev[i][0].record(stream)
+            run(i)
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        return statistics.median(a.elapsed_time(b) for a, b in ev) * 1e3
+
     for p in range(P):
         passes[p]()
-    eager = time_block(lambda i: passes[i % P](), 4 * P, stream) / (4 * P) * 1e3
+    eager = timed(lambda i: passes[i % P](), 4 * P)
     try:
         graphs = []
         side = torch.cuda.Stream(device=dev)
@@ -973,15 +987,10 @@ def graph_pass_us(passes, stream, dev, replays=60):
         return None, eager, f"graph capture failed: {type(e).__name__}: {str(e)[:120]}"
     for i in range(3 * P):
         graphs[i % P].replay()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(replays)]
-    for i in range(replays):
-        ev[i][0].record(stream)
-        graphs[i % P].replay()
-        ev[i][1].record(stream)
-    torch.cuda.synchronize()
-    us = statistics.median(a.elapsed_time(b) for a, b in ev) * 1e3
+    us = timed(lambda i: graphs[i % P].replay(), replays)
     del graphs
-    return us, eager, "median of CUDA-graph replays (one graph per pooled batch, rotated)"
+    return us, eager, ("median of CUDA-graph replays (one graph per pooled batch, rotated)"
+                       + ("; L2 flushed before each pass" if flush is not None else ""))
 
 
 def decode_leg(mole, dev, stream):
@@ -990,11 +999,15 @@ def decode_leg(mole, dev, stream):
     the combine of every layer (own table, router, hidden states; the batch's
     ids shared), captured as a CUDA graph per pooled batch (4 batches,
     rotated, so consecutive replays read other ids), timed as the median of
-    60 replays; the eager (host-launched) pass is reported beside it."""
+    60 replays, the L2 flushed before every pass (a 256 MB write outside the
+    pass's events: each pass starts cold, as after a step's other work); the
+    eager (host-launched) pass is reported beside it, and the same passes
+    preceded by mole_prefetch_rows of every layer's rows."""
     import torch
     hbm_peak = measured_peaks()[0]
     res = {}
     P = 4
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # 2x the L2: every pass starts cold
     sweeps = [("160m", (1, 8, 64), False), ("410m", (1, 2, 4, 8, 16, 32, 64, 128, 256), False),
               ("1b_nf3", (1, 8, 64, 256, 1024, 4096, 16384), True)]
     for name, Ts, nf3 in sweeps:
@@ -1011,6 +1024,7 @@ def decode_leg(mole, dev, stream):
             else:
                 tables.append(lut)
         routers = [(torch.randn((D, N), generator=g, device=dev) * 0.02).to(torch.bfloat16) for _ in range(L)]
+        zero_id = torch.zeros(1, dtype=torch.int32, device=dev)
         rng = np.random.default_rng(shape.seed)
         for T in Ts:
             ids = [torch.from_numpy(inputs.draw_ids(rng, T, V, "zipf")).to(dev) for _ in range(P)]
@@ -1019,9 +1033,23 @@ def decode_leg(mole, dev, stream):
             outs = [torch.empty((T, D), dtype=torch.float32, device=dev) for _ in range(L)]
             groups = [mole.mole_token_groups_build(x, V, N, stream=stream) for x in ids] if T >= 1024 else None
 
-            def make_pass(p):
+            def prefetch_layers(p, lays):
+                mole.mole_prefetch_rows(zero_id, [routers[x].view(1, -1) for x in lays])
+                if nf3:
+                    mole.mole_prefetch_rows(ids[p], [tables[x][0] for x in lays])
+                    mole.mole_prefetch_rows(ids[p], [tables[x][1] for x in lays])
+                else:
+                    mole.mole_prefetch_rows(ids[p], [tables[x] for x in lays])
+
+            def make_pass(p, prefetch=None):
                 def run():
+                    if prefetch == "all":  # every layer's rows and router for this step, asked of L2 up front
+                        prefetch_layers(p, range(L))
+                    elif prefetch == "ahead":
+                        prefetch_layers(p, [0])
                     for lay in range(L):
+                        if prefetch == "ahead" and lay + 1 < L:  # the next layer's, while this one runs
+                            prefetch_layers(p, [lay + 1])
                         if nf3 and groups is not None:
                             mole.mole_lookup_combine_nf3_groups(ids[p], groups[p], hs[p][lay], routers[lay],
                                                                 *tables[lay], out=outs[lay])
@@ -1032,7 +1060,10 @@ def decode_leg(mole, dev, stream):
                             mole.mole_lookup_combine(ids[p], hs[p][lay], routers[lay], tables[lay], out=outs[lay])
                 return run
 
-            graph_us, eager_us, note = graph_pass_us([make_pass(p) for p in range(P)], stream, dev)
+            graph_us, eager_us, note = graph_pass_us([make_pass(p) for p in range(P)], stream, dev, flush=flush)
+            pf_us, pf_eager_us, _ = graph_pass_us([make_pass(p, "all") for p in range(P)], stream, dev, flush=flush)
+            pa_us, pa_eager_us, _ = graph_pass_us([make_pass(p, "ahead") for p in range(P)], stream, dev,
+                                                  flush=flush)
             st = mole.mole_check(stream)
             if st != 0:
                 raise RuntimeError(f"device status {st} in the {name} T={T} sweep")
@@ -1043,6 +1074,10 @@ def decode_leg(mole, dev, stream):
                 "tokens_per_s": T / (pass_us / 1e6), "layer_tokens_per_s": T * L / (pass_us / 1e6),
                 "unique_rows": U, "achieved_gbs": b / (pass_us / L / 1e6) / 1e9,
                 "frac_of_measured_hbm": b / (pass_us / L / 1e6) / 1e9 / hbm_peak, "layers": L,
+                "prefetch_all_us_per_layer_call": (pf_us if pf_us is not None else pf_eager_us) / L,
+                "prefetch_ahead_us_per_layer_call": (pa_us if pa_us is not None else pa_eager_us) / L,
+                "prefetch_note": "mole_prefetch_rows of the rows (and router) of every layer at the pass start "
+                                 "(all), or of layer l+1 before layer l's combine (ahead)",
                 "call": ("mole_lookup_combine_nf3_groups (grouping built once per batch, outside the pass)"
                          if nf3 and groups is not None else
                          "mole_lookup_combine_nf3" if nf3 else "mole_lookup_combine"),

@@ -386,6 +386,31 @@ mole_status mole_gather_plan(const int32_t* ids, int64_t T, int64_t V, int32_t* 
                              int32_t* n_uniq, int32_t* slot, cudaStream_t stream);
 
 /*
+ * ---- Cross-layer row prefetch (MoLE page, 推理阶段 + 复杂度分析) ----
+ *
+ * Every MoLE layer indexes its own table with the step's input token ids, so
+ * all layers' rows are known before the first layer runs.  For each of the
+ * n_tables tables and each token t with 0 <= ids[t] < V, asks the GPU's L2
+ * cache to fetch row ids[t] of that table (row_bytes bytes at
+ * tables[l] + ids[t] * row_bytes): bulk L2 prefetches, issued from many SMs,
+ * that move no data into the SMs and that nothing waits for.  Later calls
+ * that read those rows (the layers' combines, in this stream or another)
+ * then hit L2 while the rows stay resident (126 MB of L2: prefetch no more
+ * than fits).  Results of every call are unchanged; this is a hint.
+ *
+ *   ids    : [T] int32 device; ids outside [0, V) are skipped (the combine
+ *            that reads them reports them)
+ *   tables : HOST array of n_tables (<= 64) device pointers, 16-byte aligned;
+ *            an NF3 table is two tables (codes, row_bytes = N * D / 64 * 24;
+ *            scales, row_bytes = N * D / 64 * 2)
+ *   row_bytes : bytes of one row, a multiple of 16 (bf16 table: N * D * 2)
+ * MOLE_ERR_ALIGN for unaligned tables or row_bytes, MOLE_ERR_UNSUPPORTED for
+ * more than 64 tables.  T == 0 or n_tables == 0 is a no-op.
+ */
+mole_status mole_prefetch_rows(const int32_t* ids, int64_t T, const void* const* tables, int32_t n_tables,
+                               int64_t V, int64_t row_bytes, cudaStream_t stream);
+
+/*
  * Waits (polling, at most timeout_ms >= 0 milliseconds) for `stream` to drain,
  * then reads and clears this device's error word.  A negative timeout_ms is
  * rejected with MOLE_ERR_ARG (no host wait is unbounded).  Returns MOLE_OK,

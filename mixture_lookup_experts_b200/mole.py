@@ -62,6 +62,7 @@ SIGNATURES = {
     "mole_nf3_levels": ([_P], None),
     "mole_nf3_midpoints": ([_P], None),
     "mole_gather_plan": ([_P, _I64, _I64, _P, _P, _P, _P], _I),
+    "mole_prefetch_rows": ([_P, _I64, _P, _I32, _I64, _I64, _P], _I),
     "mole_check": ([_P, _I], _I),
 }
 for _name, (_args, _res) in SIGNATURES.items():
@@ -445,6 +446,24 @@ def mole_gather_plan(ids: torch.Tensor, V: int, stream=None):
         "mole_gather_plan")
     k = int(n.item())
     return uniq[:k], slot[:T]
+
+
+def mole_prefetch_rows(ids: torch.Tensor, tables, stream=None) -> None:
+    """L2 prefetch of the rows of `tables` (device tensors of V rows each:
+    bf16 [V, N, D] tables, NF3 code [V, N, D/64, 24] and scale [V, N, D/64]
+    arrays) that the step's `ids` address (see mole.h)."""
+    _contig(ids, *tables)
+    tables = list(tables)
+    if not tables:
+        return
+    V = tables[0].shape[0]
+    row_bytes = tables[0].numel() // V * tables[0].element_size()
+    for t in tables:
+        if t.shape[0] != V or t.numel() // V * t.element_size() != row_bytes:
+            raise ValueError("mole_prefetch_rows: tables of one call share V and the row size")
+    arr = (ctypes.c_void_p * len(tables))(*[t.data_ptr() for t in tables])
+    _ok(lib.mole_prefetch_rows(_ptr(ids), ids.numel(), arr, len(tables), V, row_bytes, _stream(stream)),
+        "mole_prefetch_rows")
 
 
 def mole_check(stream=None, timeout_ms: int = 10000) -> int:

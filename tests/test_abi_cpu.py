@@ -71,6 +71,14 @@ def test_argument_checks_without_device(mole):
     assert lib.mole_build_lut(P, P, P, 10, 64, 2, 64, 9, 1, P, P, 1 << 20, None) == 1  # bad act
     assert lib.mole_gather_plan(P, -3, 10, P, P, P, None) == 1
     assert lib.mole_check(None, -1) == 1  # no unbounded host wait
+    tabs = (ctypes.c_void_p * 2)(P, P + 4096)
+    assert lib.mole_prefetch_rows(P, 4, tabs, 2, 10, 24, None) == 2      # row bytes not a multiple of 16
+    assert lib.mole_prefetch_rows(P, 4, tabs, 65, 10, 32, None) == 3     # more than 64 tables
+    assert lib.mole_prefetch_rows(P, -1, tabs, 2, 10, 32, None) == 1     # negative T
+    assert lib.mole_prefetch_rows(P, 4, None, 2, 10, 32, None) == 1      # no table list
+    bad = (ctypes.c_void_p * 1)(P + 8)
+    assert lib.mole_prefetch_rows(P, 4, bad, 1, 10, 32, None) == 2       # unaligned table
+    assert lib.mole_prefetch_rows(P, 0, tabs, 2, 10, 32, None) == 0      # T == 0: no-op
 
 
 def test_valid_arguments_reach_the_device_check(mole):
