@@ -546,7 +546,11 @@ def headline(*, value, world, K, W, max_ms, cfg, roofline, e2e, launches, prep_u
 def e2e_leg(combine, id_pool, h_pool, routers, luts, out, dev, stream, world, W, K, T, L):
     """The same metric through the C ABI with host buffers: per step the ids
     and the L hidden-state batches are copied host -> device from pinned
-    memory, the L combine calls run, and the L outputs are copied back."""
+    memory, the L combine calls run, and the L outputs are copied back.  The
+    copies run on their own streams, double-buffered on the device: layer
+    l+1's h goes in while layer l combines and layer l-1's output comes back
+    (the host link carries both directions at once), every copy and call
+    ordered by events."""
     import torch
     import torch.distributed as dist
     D = out.shape[1]
@@ -556,16 +560,43 @@ def e2e_leg(combine, id_pool, h_pool, routers, luts, out, dev, stream, world, W,
     for s in range(min(2, L)):
         h_host[s].copy_(h_pool[0][s])
     ids_host.copy_(id_pool[0][0].cpu())
-    h_stage = torch.empty((T, D), dtype=torch.bfloat16, device=dev)
+    h_stage = [torch.empty((T, D), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    o_stage = [out, torch.empty_like(out)]
     ids_stage = torch.empty((T,), dtype=torch.int32, device=dev)
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    n_ev = 4
+    ev_h = [torch.cuda.Event() for _ in range(n_ev)]   # h of call g is on the device
+    ev_c = [torch.cuda.Event() for _ in range(n_ev)]   # call g is done (its h buffer is free)
+    ev_o = [torch.cuda.Event() for _ in range(n_ev)]   # call g's output is back (its buffer is free)
+    ev_ids = torch.cuda.Event()
+    g = [0]  # calls issued so far (events of call g at g % n_ev)
 
     def e2e_step():
-        ids_stage.copy_(ids_host, non_blocking=True)
+        s_in.wait_stream(stream)  # the previous step's grouping has read ids_stage
+        with torch.cuda.stream(s_in):
+            ids_stage.copy_(ids_host, non_blocking=True)
+            ev_ids.record(s_in)
+        stream.wait_event(ev_ids)
         combine.prepare(ids_stage, stream)
         for layer in range(L):
-            h_stage.copy_(h_host[layer % 2], non_blocking=True)
-            combine(ids_stage, h_stage, routers[layer], luts[layer], out, stream)
-            out_host.copy_(out, non_blocking=True)
+            c = g[0]
+            b = c % 2
+            with torch.cuda.stream(s_in):
+                if c >= 2:
+                    s_in.wait_event(ev_c[(c - 2) % n_ev])
+                h_stage[b].copy_(h_host[layer % 2], non_blocking=True)
+                ev_h[c % n_ev].record(s_in)
+            stream.wait_event(ev_h[c % n_ev])
+            if c >= 2:
+                stream.wait_event(ev_o[(c - 2) % n_ev])
+            combine(ids_stage, h_stage[b], routers[layer], luts[layer], o_stage[b], stream)
+            ev_c[c % n_ev].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_c[c % n_ev])
+                out_host.copy_(o_stage[b], non_blocking=True)
+                ev_o[c % n_ev].record(s_out)
+            g[0] += 1
+        stream.wait_event(ev_o[(g[0] - 1) % n_ev])  # the step ends when its last output is back
 
     for _ in range(min(W, 3)):
         e2e_step()
@@ -583,7 +614,8 @@ def e2e_leg(combine, id_pool, h_pool, routers, luts, out, dev, stream, world, W,
     (e_ms,) = max_over_ranks([e_start.elapsed_time(e_end)], dev)
     return {"value": whole_job_tokens_per_s(world, T, K_e2e, e_ms), "unit": UNIT,
             "h2d_bytes_per_step": L * T * D * 2 + T * 4, "d2h_bytes_per_step": L * T * D * 4,
-            "steps": K_e2e, "note": f"per step: ids + {L} h H2D (pinned), {L} C-ABI calls, {L} outputs D2H"}
+            "steps": K_e2e, "note": f"per step: ids + {L} h H2D (pinned), {L} C-ABI calls, {L} outputs D2H; "
+                                    f"copies overlapped with the calls on two copy streams"}
 
 
 def time_block(fn, n, stream):

@@ -695,31 +695,51 @@ void nf3_tables(uint16_t levels[8], float mid[7]) {
 }
 
 // ---- NF3 quantiser ---------------------------------------------------------
-// One thread per 64-element block of one (v, j) row, all in IEEE fp32:
-// amax -> fp16 scale (saturating, ties to even) -> correctly rounded x / s ->
-// number of midpoints below -> 3-bit code at bits [3e, 3e+3) of the block.
-__global__ void __launch_bounds__(256) nf3_quantize_kernel(const uint16_t* __restrict__ lut,
-                                                           int64_t n_blocks, uint8_t* __restrict__ codes,
-                                                           uint16_t* __restrict__ scales) {
+// One thread per 64-element block of one (v, j) row, the quantiser of
+// nf3.cuh in two passes over the block's 128 bytes (the second from L1) so
+// that no thread holds the whole block in registers and 4 CTAs fit per SM:
+// amax -> fp16 scale (saturating, ties to even); then per element the number
+// of midpoints below the correctly rounded x / s, found by comparing x with
+// the block's 7 thresholds on the bf16 grid -> 3-bit code at bits [3e, 3e+3).
+__global__ void __launch_bounds__(256, 4) nf3_quantize_kernel(const uint16_t* __restrict__ lut,
+                                                              int64_t n_blocks, uint8_t* __restrict__ codes,
+                                                              uint16_t* __restrict__ scales) {
   const int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (blk >= n_blocks) return;
   const uint4* src = reinterpret_cast<const uint4*>(lut + blk * 64);
-  uint32_t xw[32];
+  float amax = 0.f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const uint4 v = __ldg(src + i);
-    xw[4 * i + 0] = v.x;
-    xw[4 * i + 1] = v.y;
-    xw[4 * i + 2] = v.z;
-    xw[4 * i + 3] = v.w;
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(w[q])), fabsf(bf16_hi(w[q]))));
   }
-  uint32_t packed[6];
-  const uint16_t s16 = nf3_quantize_block(xw, packed);
+  const __half s16 = nf3_scale(amax);
+  const float sc = __half2float(s16);
+  uint32_t packed[6] = {0u, 0u, 0u, 0u, 0u, 0u};
+  if (sc == 0.f) {
+#pragma unroll
+    for (int e = 0; e < 64; ++e) nf3_put(packed, e, (uint32_t)kNf3ZeroCode);
+  } else {
+    float t[7];
+    nf3_thresholds(sc, t);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint4 v = __ldg(src + i);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        nf3_put(packed, 8 * i + 2 * q, nf3_code(bf16_lo(w[q]), t));
+        nf3_put(packed, 8 * i + 2 * q + 1, nf3_code(bf16_hi(w[q]), t));
+      }
+    }
+  }
   uint2* dst = reinterpret_cast<uint2*>(codes + blk * 24);
   dst[0] = make_uint2(packed[0], packed[1]);
   dst[1] = make_uint2(packed[2], packed[3]);
   dst[2] = make_uint2(packed[4], packed[5]);
-  scales[blk] = s16;
+  scales[blk] = __half_as_ushort(s16);
 }
 
 mole_status nf3_quantize_launch(const void* lut, int64_t V, int N, int64_t D, uint8_t* codes,

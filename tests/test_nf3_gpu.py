@@ -40,6 +40,39 @@ def test_quantize_bit_exact(mole, oracle_mod, V, N, D):
     np.testing.assert_array_equal(host_bits(scales), ref_scales)
 
 
+def _boundary_blocks(oracle_mod, n_blocks, seed):
+    """Blocks whose elements sit on both sides of the decision boundaries:
+    element 0 is the block's absmax A (a bf16 value inside the fp16 range, so
+    the scale is A itself), the others the bf16 values nearest to m_k * A for
+    each midpoint m_k -- the two neighbours and one more on each side -- so
+    x / s lands within a few fp32 ulps of a midpoint, where a quantiser that
+    does not compare exactly as the division rule would pick the other code."""
+    rng = np.random.default_rng(seed)
+    mids = oracle_mod.nf3_midpoints().astype(np.float64)
+    blocks = np.zeros((n_blocks, 64), dtype=np.float32)
+    for b in range(n_blocks):
+        A = np.float32(inputs.bf16_bits_to_f32(inputs.f32_to_bf16_bits(
+            np.array([rng.choice([1.0, -1.0]) * np.exp(rng.uniform(np.log(1e-4), np.log(6e4)))], np.float32)))[0])
+        vals = [A]
+        for m in mids:
+            target = np.float32(m * abs(A))
+            u = int(inputs.f32_to_bf16_bits(np.array([target], np.float32))[0])
+            for du in (-2, -1, 0, 1, 2):  # bf16 neighbours by bit pattern (same sign)
+                bits = np.array([(u + du) & 0xffff], np.uint16)
+                vals.append(float(inputs.bf16_bits_to_f32(bits)[0]))
+        vals = [v for v in vals if abs(v) <= abs(A)]
+        blocks[b, :len(vals[:64])] = vals[:64]
+    return inputs.f32_to_bf16_bits(blocks)
+
+
+def test_quantize_bit_exact_at_the_decision_boundaries(mole, oracle_mod):
+    lut = _boundary_blocks(oracle_mod, 4096, 11).reshape(64, 16, 4 * 64)
+    codes, scales = mole.mole_quantize_lut_nf3(dev(lut))
+    ref_codes, ref_scales = oracle_mod.quantize_nf3(lut)
+    np.testing.assert_array_equal(host_bits(scales), ref_scales)
+    np.testing.assert_array_equal(codes.cpu().numpy(), ref_codes)
+
+
 @pytest.mark.parametrize("V,N,D,T,dtype", [
     (300, 16, 2048, 300, "bf16"), (100, 16, 128, 77, "bf16"), (50, 5, 64, 19, "bf16"),
     (64, 24, 256, 40, "bf16"), (80, 8, 192, 33, "f32"),
