@@ -372,13 +372,20 @@ __device__ __forceinline__ float bf16_hi_held(uint32_t x) {
 constexpr int kGroupThreads = (kGroupCons + 1) * 32;
 constexpr int kGroupProducer = kGroupCons;
 
-// out[t, 4v .. 4v+3] for one token from the N rows of the unit (x, fp32 or
-// packed bf16 pairs) and the token's gates g (NP floats in shared memory).
+// Packed fp32 FMA (two lanes per instruction, each rounded as fmaf): the
+// gate g times an element pair, plus the pair's running sums.
+__device__ __forceinline__ float2 ffma2(float g, float2 x, float2 acc) {
+  return __ffma2_rn(make_float2(g, g), x, acc);
+}
+
+// out[t, 4v .. 4v+3] for one token from the N rows of the unit (x, fp32
+// pairs or packed bf16 pairs) and the token's gates g (NP floats in shared
+// memory).  Per element the FMAs run over j = 0..N-1 in order.
 template <int NP, bool kExactN, bool kPacked>
-__device__ __forceinline__ float4 combine_unit(const float (&xf)[kPacked ? 1 : NP][4], const uint2 (&xp)[kPacked ? NP : 1],
+__device__ __forceinline__ float4 combine_unit(const float2 (&xf)[kPacked ? 1 : NP][2], const uint2 (&xp)[kPacked ? NP : 1],
                                                const float* g, int N) {
   const float4* g4 = reinterpret_cast<const float4*>(g);
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
 #pragma unroll
   for (int jq = 0; jq < NP / 4; ++jq) {
     const float4 gv = g4[jq];
@@ -387,36 +394,27 @@ __device__ __forceinline__ float4 combine_unit(const float (&xf)[kPacked ? 1 : N
     for (int e = 0; e < 4; ++e) {
       const int j = 4 * jq + e;
       if (kExactN || j < N) {
-        float x0, x1, x2, x3;
         if (kPacked) {
           const uint2 r = xp[kPacked ? j : 0];
-          x0 = bf16_lo(r.x);
-          x1 = bf16_hi(r.x);
-          x2 = bf16_lo(r.y);
-          x3 = bf16_hi(r.y);
+          a01 = ffma2(gg[e], make_float2(bf16_lo(r.x), bf16_hi(r.x)), a01);
+          a23 = ffma2(gg[e], make_float2(bf16_lo(r.y), bf16_hi(r.y)), a23);
         } else {
-          x0 = xf[kPacked ? 0 : j][0];
-          x1 = xf[kPacked ? 0 : j][1];
-          x2 = xf[kPacked ? 0 : j][2];
-          x3 = xf[kPacked ? 0 : j][3];
+          a01 = ffma2(gg[e], xf[kPacked ? 0 : j][0], a01);
+          a23 = ffma2(gg[e], xf[kPacked ? 0 : j][1], a23);
         }
-        a0 = fmaf(gg[e], x0, a0);
-        a1 = fmaf(gg[e], x1, a1);
-        a2 = fmaf(gg[e], x2, a2);
-        a3 = fmaf(gg[e], x3, a3);
       }
     }
   }
-  return make_float4(a0, a1, a2, a3);
+  return make_float4(a01.x, a01.y, a23.x, a23.y);
 }
 
 // out for 4 tokens at once (gates at g + k * gstride floats, k = 0..3):
-// 16 independent FMA chains over the N rows held in fp32.
+// 16 independent FMA chains (8 packed pairs) over the N rows held in fp32.
 template <int NP, bool kExactN>
-__device__ __forceinline__ void combine_quad(const float (&xf)[NP][4], const float* g, int gstride, int N,
-                                             float (&o)[4][4]) {
+__device__ __forceinline__ void combine_quad(const float2 (&xf)[NP][2], const float* g, int gstride, int N,
+                                             float2 (&o)[4][2]) {
 #pragma unroll
-  for (int k = 0; k < 4; ++k) o[k][0] = o[k][1] = o[k][2] = o[k][3] = 0.f;
+  for (int k = 0; k < 4; ++k) o[k][0] = o[k][1] = make_float2(0.f, 0.f);
 #pragma unroll
   for (int jq = 0; jq < NP / 4; ++jq) {
     float4 gv[4];
@@ -429,10 +427,8 @@ __device__ __forceinline__ void combine_quad(const float (&xf)[NP][4], const flo
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const float gk = e == 0 ? gv[k].x : e == 1 ? gv[k].y : e == 2 ? gv[k].z : gv[k].w;
-          o[k][0] = fmaf(gk, xf[j][0], o[k][0]);
-          o[k][1] = fmaf(gk, xf[j][1], o[k][1]);
-          o[k][2] = fmaf(gk, xf[j][2], o[k][2]);
-          o[k][3] = fmaf(gk, xf[j][3], o[k][3]);
+          o[k][0] = ffma2(gk, xf[j][0], o[k][0]);
+          o[k][1] = ffma2(gk, xf[j][1], o[k][1]);
         }
       }
     }
@@ -443,10 +439,10 @@ __device__ __forceinline__ void combine_quad(const float (&xf)[NP][4], const flo
 // block scale; per token the gate and the scale are multiplied first and the
 // product scales the levels, as the ungrouped kernels do.
 template <int NP, bool kExactN>
-__device__ __forceinline__ void combine_quad_nf3(const float (&xf)[NP][4], const float (&sc)[NP], const float* g,
-                                                 int gstride, int N, float (&o)[4][4]) {
+__device__ __forceinline__ void combine_quad_nf3(const float2 (&xf)[NP][2], const float (&sc)[NP], const float* g,
+                                                 int gstride, int N, float2 (&o)[4][2]) {
 #pragma unroll
-  for (int k = 0; k < 4; ++k) o[k][0] = o[k][1] = o[k][2] = o[k][3] = 0.f;
+  for (int k = 0; k < 4; ++k) o[k][0] = o[k][1] = make_float2(0.f, 0.f);
 #pragma unroll
   for (int jq = 0; jq < NP / 4; ++jq) {
     float4 gv[4];
@@ -459,10 +455,8 @@ __device__ __forceinline__ void combine_quad_nf3(const float (&xf)[NP][4], const
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const float a = (e == 0 ? gv[k].x : e == 1 ? gv[k].y : e == 2 ? gv[k].z : gv[k].w) * sc[j];
-          o[k][0] = fmaf(a, xf[j][0], o[k][0]);
-          o[k][1] = fmaf(a, xf[j][1], o[k][1]);
-          o[k][2] = fmaf(a, xf[j][2], o[k][2]);
-          o[k][3] = fmaf(a, xf[j][3], o[k][3]);
+          o[k][0] = ffma2(a, xf[j][0], o[k][0]);
+          o[k][1] = ffma2(a, xf[j][1], o[k][1]);
         }
       }
     }
@@ -470,20 +464,18 @@ __device__ __forceinline__ void combine_quad_nf3(const float (&xf)[NP][4], const
 }
 
 template <int NP, bool kExactN>
-__device__ __forceinline__ float4 combine_unit_nf3(const float (&xf)[NP][4], const float (&sc)[NP], const float* g,
+__device__ __forceinline__ float4 combine_unit_nf3(const float2 (&xf)[NP][2], const float (&sc)[NP], const float* g,
                                                    int N) {
-  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
 #pragma unroll
   for (int j = 0; j < NP; ++j) {
     if (kExactN || j < N) {
       const float a = g[j] * sc[j];
-      a0 = fmaf(a, xf[j][0], a0);
-      a1 = fmaf(a, xf[j][1], a1);
-      a2 = fmaf(a, xf[j][2], a2);
-      a3 = fmaf(a, xf[j][3], a3);
+      a01 = ffma2(a, xf[j][0], a01);
+      a23 = ffma2(a, xf[j][1], a23);
     }
   }
-  return make_float4(a0, a1, a2, a3);
+  return make_float4(a01.x, a01.y, a23.x, a23.y);
 }
 
 __device__ __forceinline__ float held(float x) {
@@ -820,7 +812,7 @@ __device__ void ring_consumers(const GArgs& p, const GroupLayout& L, const Ring&
       const uint8_t* slot = r.slots + (size_t)q * L.slot_bytes;
       const float* gs = gl != nullptr ? gl + loff[k] * NP : reinterpret_cast<const float*>(slot + L.gates_off);
       for (int v = v0; v < units; v += vstep) {
-        float xf[kPacked ? 1 : NP][4];
+        float2 xf[kPacked ? 1 : NP][2];
         uint2 xp[kPacked ? NP : 1];
         float sc[NP];
         if constexpr (kNf3) {
@@ -837,10 +829,8 @@ __device__ void ring_consumers(const GArgs& p, const GroupLayout& L, const Ring&
               nf3_levels4(x, f);
               sc[j] = held(__half2float(__ushort_as_half(ss[j * NB + b])));
             }
-            xf[j][0] = held(f[0]);
-            xf[j][1] = held(f[1]);
-            xf[j][2] = held(f[2]);
-            xf[j][3] = held(f[3]);
+            xf[j][0] = make_float2(held(f[0]), held(f[1]));
+            xf[j][1] = make_float2(held(f[2]), held(f[3]));
           }
         } else {
 #pragma unroll
@@ -850,10 +840,8 @@ __device__ void ring_consumers(const GArgs& p, const GroupLayout& L, const Ring&
             if (kPacked) {
               xp[kPacked ? j : 0] = rw;
             } else {
-              xf[kPacked ? 0 : j][0] = bf16_lo_held(rw.x);
-              xf[kPacked ? 0 : j][1] = bf16_hi_held(rw.x);
-              xf[kPacked ? 0 : j][2] = bf16_lo_held(rw.y);
-              xf[kPacked ? 0 : j][3] = bf16_hi_held(rw.y);
+              xf[kPacked ? 0 : j][0] = make_float2(bf16_lo_held(rw.x), bf16_hi_held(rw.x));
+              xf[kPacked ? 0 : j][1] = make_float2(bf16_lo_held(rw.y), bf16_hi_held(rw.y));
             }
           }
         }
@@ -861,7 +849,7 @@ __device__ void ring_consumers(const GArgs& p, const GroupLayout& L, const Ring&
         if constexpr (!kPacked) {
           // four tokens at a time (16 independent FMA chains)
           for (; i + 3 * Gt < n; i += 4 * Gt) {
-            float o[4][4];
+            float2 o[4][2];
             if constexpr (kNf3)
               combine_quad_nf3<NP, kExactN>(xf, sc, gs + i * NP, Gt * NP, p.N, o);
             else
@@ -869,7 +857,7 @@ __device__ void ring_consumers(const GArgs& p, const GroupLayout& L, const Ring&
 #pragma unroll
             for (int k2 = 0; k2 < 4; ++k2)
               __stcs(reinterpret_cast<float4*>(p.out + (int64_t)r.slot_tok[q * C + i + k2 * Gt] * p.D + 4 * v),
-                     make_float4(o[k2][0], o[k2][1], o[k2][2], o[k2][3]));
+                     make_float4(o[k2][0].x, o[k2][0].y, o[k2][1].x, o[k2][1].y));
           }
         }
         for (; i < n; i += Gt) {
