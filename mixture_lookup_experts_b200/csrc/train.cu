@@ -88,15 +88,38 @@ size_t carve_cache(void* base, int64_t T, int64_t V, int N, int64_t D, int64_t D
 
 __device__ __forceinline__ float ld_bf16(const uint16_t* p) { return __uint_as_float((uint32_t)*p << 16); }
 
+// Wr staged in shared memory as [D][NP] bf16 (experts past N zero), with 16
+// bytes of padding after every 8 rows: a lane reads the 8 rows of its 8
+// consecutive d, lanes 8 rows apart, so the padding spreads them over the banks.
+__host__ __device__ __forceinline__ int wr_row(int d, int NP) { return d * NP + (d >> 3) * 8; }
+__host__ __device__ __forceinline__ size_t wr_stage_bytes(int D, int NP) { return (size_t)(D * NP + (D >> 3) * 8) * 2; }
+
+__device__ __forceinline__ void unpack8(const uint4 v, float (&f)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
 // One warp per token: the gates (router logits h[t] . Wr in fp32, softmax),
 // dg_j = <dout[t], Y[u(t), j]>, dz = g (dg - <g, dg>), and dh[t] += dz . Wr^T.
-// Tokens with a bad id (dense index -1) get no gradient.
+// Lane l takes d = 8l + 256i (16-byte loads of h, dout and the expert rows;
+// Wr from the CTA's staged copy), then the partial sums are reduced across
+// the warp.  Tokens with a bad id (dense index -1) get no gradient.
 template <int NP>
 __global__ void __launch_bounds__(kGradThreads) gate_grad_kernel(const GroupWs w, const uint16_t* __restrict__ h,
                                                                  const uint16_t* __restrict__ Wr,
                                                                  const uint16_t* __restrict__ Y,
                                                                  const float* __restrict__ dout, int64_t T, int N,
                                                                  int D, float* g_out, float* dz_out, float* dh) {
+  extern __shared__ __align__(16) uint16_t wr_s[];
+  for (int i = threadIdx.x; i < D * NP; i += kGradThreads) {
+    const int d = i / NP, j = i - d * NP;
+    wr_s[wr_row(d, NP) + j] = j < N ? Wr[(int64_t)d * N + j] : (uint16_t)0;
+  }
+  __syncthreads();
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (kGradThreads / 32);
   for (int64_t t = (int64_t)blockIdx.x * (kGradThreads / 32) + (threadIdx.x >> 5); t < T; t += warps) {
@@ -108,14 +131,33 @@ __global__ void __launch_bounds__(kGradThreads) gate_grad_kernel(const GroupWs w
     const uint16_t* hr = h + t * D;
     const float* dr = dout + t * D;
     const uint16_t* yr = Y + (int64_t)u * N * D;
-    for (int d = lane; d < D; d += 32) {
-      const float hv = ld_bf16(hr + d), dv = dr[d];
+    for (int d0 = 8 * lane; d0 < D; d0 += 256) {
+      float hf[8], of[8];
+      unpack8(*reinterpret_cast<const uint4*>(hr + d0), hf);
+      const float4 o0 = *reinterpret_cast<const float4*>(dr + d0);
+      const float4 o1 = *reinterpret_cast<const float4*>(dr + d0 + 4);
+      of[0] = o0.x; of[1] = o0.y; of[2] = o0.z; of[3] = o0.w;
+      of[4] = o1.x; of[5] = o1.y; of[6] = o1.z; of[7] = o1.w;
 #pragma unroll
-      for (int j = 0; j < NP; ++j)
-        if (j < N) {
-          z[j] = fmaf(hv, ld_bf16(Wr + (int64_t)d * N + j), z[j]);
-          dg[j] = fmaf(dv, ld_bf16(yr + (int64_t)j * D + d), dg[j]);
+      for (int e = 0; e < 8; ++e) {
+        const uint4* wr = reinterpret_cast<const uint4*>(wr_s + wr_row(d0 + e, NP));
+#pragma unroll
+        for (int q = 0; q < NP / 8; ++q) {
+          float wf[8];
+          unpack8(wr[q], wf);
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) z[8 * q + jj] = fmaf(hf[e], wf[jj], z[8 * q + jj]);
         }
+      }
+#pragma unroll
+      for (int j = 0; j < NP; ++j) {
+        if (j < N) {
+          float yf[8];
+          unpack8(*reinterpret_cast<const uint4*>(yr + (int64_t)j * D + d0), yf);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) dg[j] = fmaf(of[e], yf[e], dg[j]);
+        }
+      }
     }
 #pragma unroll
     for (int j = 0; j < NP; ++j)
@@ -153,12 +195,26 @@ __global__ void __launch_bounds__(kGradThreads) gate_grad_kernel(const GroupWs w
     }
     if (dh != nullptr) {
       float* o = dh + t * D;
-      for (int d = lane; d < D; d += 32) {
-        float acc = 0.f;
+      for (int d0 = 8 * lane; d0 < D; d0 += 256) {
+        float acc[8];
 #pragma unroll
-        for (int j = 0; j < NP; ++j)
-          if (j < N) acc = fmaf(dz[j], ld_bf16(Wr + (int64_t)d * N + j), acc);
-        o[d] += acc;
+        for (int e = 0; e < 8; ++e) {
+          const uint4* wr = reinterpret_cast<const uint4*>(wr_s + wr_row(d0 + e, NP));
+          acc[e] = 0.f;
+#pragma unroll
+          for (int q = 0; q < NP / 8; ++q) {
+            float wf[8];
+            unpack8(wr[q], wf);
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) acc[e] = fmaf(dz[8 * q + jj], wf[jj], acc[e]);
+          }
+        }
+        float4* o4 = reinterpret_cast<float4*>(o + d0);
+        float4 a = o4[0], c = o4[1];
+        a.x += acc[0]; a.y += acc[1]; a.z += acc[2]; a.w += acc[3];
+        c.x += acc[4]; c.y += acc[5]; c.z += acc[6]; c.w += acc[7];
+        o4[0] = a;
+        o4[1] = c;
       }
     }
   }
@@ -322,15 +378,21 @@ mole_status train_backward(const void* groups, size_t gbytes, int64_t T, const v
   const uint16_t* wr16 = static_cast<const uint16_t*>(Wr);
   const int n_sm = num_sms();
   if (n_sm <= 0) return MOLE_ERR_NO_DEVICE;
-  // gates, logit gradients, dh
-  const unsigned gg = (unsigned)std::min<int64_t>((T + 7) / 8, (int64_t)n_sm * 8);
-  if (N <= 8)
-    gate_grad_kernel<8><<<gg, kGradThreads, 0, stream>>>(w, h16, wr16, c.Y, dout, T, N, (int)D, c.g, c.dz, dh);
-  else if (N <= 16)
-    gate_grad_kernel<16><<<gg, kGradThreads, 0, stream>>>(w, h16, wr16, c.Y, dout, T, N, (int)D, c.g, c.dz, dh);
-  else
-    gate_grad_kernel<32><<<gg, kGradThreads, 0, stream>>>(w, h16, wr16, c.Y, dout, T, N, (int)D, c.g, c.dz, dh);
-  if (cudaGetLastError() != cudaSuccess) return MOLE_ERR_CUDA;
+  // gates, logit gradients, dh (Wr staged per CTA: a few CTAs per SM)
+  {
+    const int NP = N <= 8 ? 8 : N <= 16 ? 16 : 32;
+    const size_t smem = wr_stage_bytes((int)D, NP);
+    auto kern = N <= 8 ? gate_grad_kernel<8> : N <= 16 ? gate_grad_kernel<16> : gate_grad_kernel<32>;
+    if (smem > 227 * 1024) return MOLE_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      return MOLE_ERR_CUDA;
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kGradThreads, smem) != cudaSuccess || occ < 1)
+      return MOLE_ERR_UNSUPPORTED;
+    const unsigned gg = (unsigned)std::min<int64_t>((T + 7) / 8, (int64_t)n_sm * occ);
+    kern<<<gg, kGradThreads, smem, stream>>>(w, h16, wr16, c.Y, dout, T, N, (int)D, c.g, c.dz, dh);
+    if (cudaGetLastError() != cudaSuccess) return MOLE_ERR_CUDA;
+  }
   if (dWr != nullptr) {
     const dim3 gw((unsigned)((D + kGradThreads - 1) / kGradThreads), (unsigned)((T + kDwrTokens - 1) / kDwrTokens));
     if (N <= 8)
