@@ -209,6 +209,62 @@ __device__ __forceinline__ void combine_tile_nf3(const Smem& s, const UnitMap& u
   }
 }
 
+// The same with units of 8 elements (one 24-bit code group of one 64-element
+// block per expert row): per element the same FMAs in the same order, so the
+// output is bit-identical; four times as many units per token, for tiles
+// whose 32-element units would leave most of the CTA's threads idle.
+template <int NT, bool kExactN>
+__device__ __forceinline__ void combine_tile_nf3_fine(const Smem& s, const UnitMap& um,
+                                                      const uint8_t* __restrict__ codes,
+                                                      const uint16_t* __restrict__ scales, int64_t V, int N,
+                                                      int D, int64_t t0, int rows, float* __restrict__ out,
+                                                      unsigned* err) {
+  constexpr int NP = 8 * NT;
+  const int NB = D >> 6;  // 64-element blocks per row
+  const int QB = D >> 3;  // 8-element units per row
+  for (int r = um.r0; r < rows; r += um.rstep) {
+    const int id = s.tok_id[r];
+    float g[NP];
+    load_gates(s.gates + r * NP, g, NP);
+    for (int u = um.v0; u < QB; u += um.vstep) {
+      float* o = out + (t0 + r) * (int64_t)D + u * 8;
+      if (id < 0 || (int64_t)id >= V) {
+        if (u == 0) atomicOr(err, kErrIndex);
+        store_nan(o, 8);
+        continue;
+      }
+      const int b = u >> 3, bit = 24 * (u & 7), wi = bit >> 5, sh = bit & 31;
+      const int64_t blk0 = (int64_t)id * N * NB + b;  // block of expert 0
+      float acc[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+      uint32_t x[NP];
+      float sc[NP];
+#pragma unroll
+      for (int j = 0; j < NP; ++j) {  // every load first, then the arithmetic
+        const int jj = kExactN ? j : min(j, N - 1);
+        const int64_t blk = blk0 + (int64_t)jj * NB;
+        const uint32_t* cw = reinterpret_cast<const uint32_t*>(codes + blk * 24);
+        const uint32_t lo = __ldg(cw + wi), hi = wi < 5 ? __ldg(cw + wi + 1) : 0u;
+        x[j] = __funnelshift_r(lo, hi, sh) & 0xffffffu;
+        sc[j] = __half2float(__ushort_as_half(__ldg(scales + blk)));
+      }
+#pragma unroll
+      for (int j = 0; j < NP; ++j) {
+        if (kExactN || j < N) {
+          const float a = g[j] * sc[j];
+          uint32_t sl, shi;
+          nf3_selectors(x[j], sl, shi);
+          nf3_fma4(sl, a, acc + 0);
+          nf3_fma4(shi, a, acc + 4);
+        }
+      }
+      __stcs(reinterpret_cast<float4*>(o), make_float4(acc[0], acc[1], acc[2], acc[3]));
+      __stcs(reinterpret_cast<float4*>(o + 4), make_float4(acc[4], acc[5], acc[6], acc[7]));
+    }
+  }
+}
+
 struct CombineArgs {
   const int32_t* ids;
   int64_t T;
@@ -523,7 +579,10 @@ __global__ void __launch_bounds__(kThreads, 2) combine_kernel(const CombineArgs 
     stage_wrt<NP, kThreads, false>(s.wrt, static_cast<const uint16_t*>(p.Wr), p.N, p.D);
     __syncthreads();
   }
-  const int per_tok = kTable == kTableBf16 ? (p.D >> 3) : kTable == kTableF32 ? (p.D >> 2) : (p.D >> 5);
+  const int per_tok = kTable == kTableBf16 ? (p.D >> 3)
+                      : kTable == kTableF32 ? (p.D >> 2)
+                      : kTable == kTableNf3Fine ? (p.D >> 3)
+                                                : (p.D >> 5);
   const UnitMap um(per_tok);
   for (int64_t tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x) {
     const int64_t t0 = tile * p.TT;
@@ -535,6 +594,9 @@ __global__ void __launch_bounds__(kThreads, 2) combine_kernel(const CombineArgs 
     else if (kTable == kTableF32)
       combine_tile_f32<NT, kExactN>(s, um, static_cast<const float*>(p.table), p.V, p.N, p.D, t0, rows,
                                     p.out, p.err);
+    else if (kTable == kTableNf3Fine)
+      combine_tile_nf3_fine<NT, kExactN>(s, um, static_cast<const uint8_t*>(p.table), p.scales, p.V, p.N, p.D,
+                                         t0, rows, p.out, p.err);
     else
       combine_tile_nf3<NT, kExactN>(s, um, static_cast<const uint8_t*>(p.table), p.scales, p.V, p.N, p.D,
                                     t0, rows, p.out, p.err);
@@ -679,6 +741,9 @@ mole_status combine_dispatch(const int32_t* ids, int64_t T, const void* h, const
     if (!bf16_inputs) return launch_combine<false, kTableNf3>(p, stream);
     const mole_status st = launch_staged<kTableNf3>(p, stream);
     if (st != MOLE_ERR_UNSUPPORTED) return st;
+    // 8-element units where 32-element ones would leave threads idle
+    const int n_sm = num_sms();
+    if (n_sm > 0 && T * (int64_t)(D >> 5) < (int64_t)n_sm * kThreads) return launch_combine<true, kTableNf3Fine>(p, stream);
     return launch_combine<true, kTableNf3>(p, stream);
   }
   if (table_kind == kTableBf16) {

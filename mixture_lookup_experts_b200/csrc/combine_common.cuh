@@ -16,7 +16,9 @@ constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kTileMax = 16;  // rows of the m16n8k16 router MMA
 
-enum TableKind { kTableBf16 = 0, kTableF32 = 1, kTableNf3 = 2 };
+// kTableNf3Fine: the NF3 table with 8-element units instead of 32 (four
+// times the threads per token, for batches too small to fill the CTA).
+enum TableKind { kTableBf16 = 0, kTableF32 = 1, kTableNf3 = 2, kTableNf3Fine = 3 };
 
 
 // Byte planes of the fp16 levels, for prmt lookups: plane[k] holds byte k of
