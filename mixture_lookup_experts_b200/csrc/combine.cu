@@ -765,7 +765,8 @@ void nf3_tables(uint16_t levels[8], float mid[7]) {
 // that no thread holds the whole block in registers and 4 CTAs fit per SM:
 // amax -> fp16 scale (saturating, ties to even); then per element the number
 // of midpoints below the correctly rounded x / s, found by comparing x with
-// the block's 7 thresholds on the bf16 grid -> 3-bit code at bits [3e, 3e+3).
+// the block's 7 thresholds on the bf16 grid (packed compares of bf16 pairs)
+// -> 3-bit code at bits [3e, 3e+3).
 __global__ void __launch_bounds__(256, 4) nf3_quantize_kernel(const uint16_t* __restrict__ lut,
                                                               int64_t n_blocks, uint8_t* __restrict__ codes,
                                                               uint16_t* __restrict__ scales) {
@@ -789,14 +790,17 @@ __global__ void __launch_bounds__(256, 4) nf3_quantize_kernel(const uint16_t* __
   } else {
     float t[7];
     nf3_thresholds(sc, t);
+    __nv_bfloat162 t2[7];
+    nf3_threshold_pairs(t, t2);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const uint4 v = __ldg(src + i);
       const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        nf3_put(packed, 8 * i + 2 * q, nf3_code(bf16_lo(w[q]), t));
-        nf3_put(packed, 8 * i + 2 * q + 1, nf3_code(bf16_hi(w[q]), t));
+        const uint32_t c = nf3_code_pair(w[q], t2);
+        nf3_put(packed, 8 * i + 2 * q, c & 0xffffu);
+        nf3_put(packed, 8 * i + 2 * q + 1, c >> 16);
       }
     }
   }

@@ -4,6 +4,7 @@
 // epilogue (build_tc.cu), so both produce the same codes bit for bit.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
 #include "common.cuh"
@@ -40,6 +41,26 @@ __device__ __forceinline__ void nf3_thresholds(float sc, float (&t)[7]) {
     if ((u >> 31) != 0u && (u & 0xffffu) != 0u) r += 0x10000u;  // negative: away from zero is down
     t[k] = __uint_as_float(r);
   }
+}
+
+// The codes of both elements of a bf16 pair word xw (element 2i in the low
+// half) against the thresholds, as bf16 pairs (t_k, t_k): seven packed
+// compares (1.0 where x > t_k) added to 128.0 in bf16 -- 128 + c is exact
+// for c <= 7 (the bf16 unit in [128, 256) is 1), and its low three bits are
+// c.  Both x and the thresholds are bf16 values, so each compare is the
+// exact comparison of nf3_code.  Returns lo | hi << 16.
+__device__ __forceinline__ uint32_t nf3_code_pair(uint32_t xw, const __nv_bfloat162 (&t2)[7]) {
+  const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162*>(&xw);
+  __nv_bfloat162 c = __floats2bfloat162_rn(128.f, 128.f);
+#pragma unroll
+  for (int k = 0; k < 7; ++k) c = __hadd2(c, __hgt2(x, t2[k]));
+  return *reinterpret_cast<const uint32_t*>(&c) & 0x00070007u;
+}
+
+// The thresholds as bf16 pairs (each t_k is a bf16 value, so exactly).
+__device__ __forceinline__ void nf3_threshold_pairs(const float (&t)[7], __nv_bfloat162 (&t2)[7]) {
+#pragma unroll
+  for (int k = 0; k < 7; ++k) t2[k] = __floats2bfloat162_rn(t[k], t[k]);
 }
 
 // Code of one element x against the block's thresholds t (scale > 0).
@@ -80,8 +101,14 @@ __device__ __forceinline__ uint16_t nf3_quantize_block(const uint32_t (&xw)[32],
   }
   float t[7];
   nf3_thresholds(sc, t);
+  __nv_bfloat162 t2[7];
+  nf3_threshold_pairs(t, t2);
 #pragma unroll
-  for (int e = 0; e < 64; ++e) nf3_put(packed, e, nf3_code((e & 1) ? bf16_hi(xw[e >> 1]) : bf16_lo(xw[e >> 1]), t));
+  for (int i = 0; i < 32; ++i) {
+    const uint32_t c = nf3_code_pair(xw[i], t2);
+    nf3_put(packed, 2 * i, c & 0xffffu);
+    nf3_put(packed, 2 * i + 1, c >> 16);
+  }
   return __half_as_ushort(s16);
 }
 
