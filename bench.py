@@ -52,8 +52,8 @@ KERNEL_SOURCES = ["mixture_lookup_experts_b200/csrc/combine.cu", "mixture_lookup
 PROFILE_SUMMARY = {"grouped": "profiles/combine_grouped_bf16_1b_T16384_zipf.md",
                    "plain": "profiles/combine_bf16_1b_T16384_zipf.md"}
 KERNELS = {
-    "grouped": "router_tc_kernel + grouped_gather_kernel (mole_lookup_combine_groups, per layer call)",
-    "plain": "router_tc_kernel + gather_kernel (mole_lookup_combine, per layer call)",
+    "grouped": "grouped_stream_kernel (mole_lookup_combine_groups, one launch per layer call)",
+    "plain": "router_gates_kernel + gather_kernel (mole_lookup_combine, per layer call)",
 }
 
 
@@ -212,12 +212,12 @@ def kernel_source_hash() -> str:
 
 
 def launches_per_step(T: int, N: int, layers: int, path: str) -> int:
-    """This library's kernel launches in one timed step.  Grouped path: the
-    grouping (plan kernel, plus the per-SM share kernel when a CTA's share
-    fits, 16 + T/SMs < 256 tokens), then per layer the tensor-core router and
-    the gather kernel where 128-token tiles fill 3/4 of the SMs (16 experts),
-    else the one CTA-local kernel; plain path: router + gather per layer.
-    Below 1024 tokens one combine kernel per layer."""
+    """This library's kernel launches in one timed step (bf16 table).  Grouped
+    path: the grouping (plan kernel, plus the per-SM share kernel when a CTA's
+    share fits, 16 + T/SMs < 256 tokens), then per layer one kernel (the
+    interleaved or the CTA-local kernel) where the shares exist, else router +
+    gather; plain path: router + gather per layer.  Below 1024 tokens one
+    combine kernel per layer."""
     import torch
     n_sm = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
     if T < 1024:
@@ -225,8 +225,7 @@ def launches_per_step(T: int, N: int, layers: int, path: str) -> int:
     if path != "grouped":
         return 2 * layers
     shares = (16 + -(-T // n_sm) + 15) // 16 * 16 < 256
-    tc_router = N == 16 and -(-T // 128) >= n_sm * 3 // 4
-    per_layer = 2 if (tc_router or not shares) else 1
+    per_layer = 1 if shares else 2
     return (2 if shares else 1) + per_layer * layers
 
 

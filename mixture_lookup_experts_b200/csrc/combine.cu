@@ -675,7 +675,9 @@ mole_status launch_two_kernel(CombineArgs p, cudaStream_t stream) {
   int occ = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, rkern, kThreads, rsmem) != cudaSuccess || occ < 1)
     return MOLE_ERR_UNSUPPORTED;
-  if (router_tc_supported(p.T, p.N, p.D, p.h, p.Wr)) {
+  // the tensor-core router for NF3 tables only: the bf16 paths (this one,
+  // the grouped kernels) all take the mma.sync router arithmetic
+  if (kTable != kTableBf16 && router_tc_supported(p.T, p.N, p.D, p.h, p.Wr)) {
     const mole_status st = router_tc_launch(p.h, p.Wr, p.T, p.D, false, p.out, nullptr, nullptr, stream);
     if (st != MOLE_OK) return st;
   } else if (launch_pdl(rkern, (unsigned)std::min<int64_t>(p.n_tiles, (int64_t)occ * n_sm), kThreads, rsmem, stream,

@@ -24,17 +24,24 @@
 //     Then group_share_kernel (once per batch) lists, for each CTA of a
 //     one-CTA-per-SM layer kernel, its work items in processing order and
 //     their tokens (its share).
-//  Per layer, batches too small for the tensor-core router (fewer 128-token
-//  tiles than about 3/4 of the SMs):
-//  2. grouped_local_kernel (one CTA per SM, 9 warps; bf16 or NF3 table):
-//     each CTA computes the gates of its own share's tokens (mma.sync router,
-//     gates kept in shared memory), then gathers and combines its work items
-//     as in 3.
-//  Per layer, otherwise:
-//  2. the router: router_tc.cu's tcgen05 kernel for 16 experts, else
-//     router_group_kernel (persistent, 2 CTAs per SM, the mma.sync router of
-//     combine_common.cuh); each token's gates go to its list position, so an
-//     item's gates are contiguous.
+//  Per layer, bf16 table, batches of at least about 3/4 of a 128-token tile
+//  per SM (the prefill sizes):
+//  2. grouped_stream_kernel (one CTA per SM, 9 warps): the CTA's share
+//     streams through one ring of shared-memory slots as two kinds of
+//     entries -- a router tile (16 of its tokens' h rows) placed just ahead
+//     of the first work item that needs it, and each work item's row block --
+//     so h and the row blocks come from memory together; the consumer warps
+//     turn a tile into gates (mma.sync router, gates kept in shared memory)
+//     and combine an item as in 3.
+//  Per layer, smaller batches (bf16 or NF3 table):
+//  2. grouped_local_kernel (one CTA per SM, 9 warps): each CTA computes the
+//     gates of its own share's tokens first, then gathers and combines its
+//     work items as in 3.
+//  Per layer, NF3 table at the prefill sizes (or where neither applies):
+//  2. the router: router_tc.cu's tcgen05 kernel for an NF3 table with 16
+//     experts, else router_group_kernel (persistent, 2 CTAs per SM, the
+//     mma.sync router of combine_common.cuh); each token's gates go to its
+//     list position, so an item's gates are contiguous.
 //  3. grouped_gather_kernel (one CTA per SM, 9 warps): a producer warp
 //     copies each work item's row block and its tokens' gates (two
 //     cp.async.bulk) into a ring of shared-memory slots; 8 consumer warps
@@ -785,90 +792,109 @@ __device__ void ring_producer(const GArgs& p, const GroupWs& w, const GroupLayou
 // fewer units than consumer threads, Gt thread groups split the item's tokens.
 // Gates: from the item's slot, or (gl != nullptr) from the CTA's gate array,
 // the k-th item's at rows loff[k] ...
+// A consumer thread's share of an item: units v0, v0 + vstep, ... of D / 4,
+// tokens grp, grp + Gt, ... of the item.
+struct UnitSplit {
+  int units, Gt, grp, v0, vstep;
+  bool active;
+  __device__ __forceinline__ explicit UnitSplit(int D) {
+    constexpr int kCT = kGroupCons * 32;
+    const int lt = threadIdx.x;
+    units = D >> 2;
+    Gt = units >= kCT ? 1 : kCT / units;
+    grp = units >= kCT ? 0 : lt / units;
+    v0 = units >= kCT ? lt : lt - grp * units;
+    vstep = units >= kCT ? kCT : units;
+    active = grp < Gt;
+  }
+};
+
+// One work item from its slot: the n tokens tok[0..n-1] with gates gs[i *
+// NP ..] (this thread's units and tokens).
+template <int NT, bool kExactN, bool kNf3>
+__device__ __forceinline__ void combine_item(const GArgs& p, const GroupLayout& L, const UnitSplit& us,
+                                             const uint8_t* slot, const float* gs, const int* tok, int n) {
+  constexpr int NP = 8 * NT;
+  constexpr bool kPacked = !kNf3 && NP > 16;  // 32 experts: keep rows as bf16 pairs, convert per token
+  static_assert(!kNf3 || NP <= 16, "the NF3 consumer holds 16 rows");
+  const int NB = p.D >> 6;
+  const int units = us.units, Gt = us.Gt, grp = us.grp, v0 = us.v0, vstep = us.vstep;
+  for (int v = v0; v < units; v += vstep) {
+    float2 xf[kPacked ? 1 : NP][2];
+    uint2 xp[kPacked ? NP : 1];
+    float sc[NP];
+    if constexpr (kNf3) {
+      // 4 codes at bits [12u, 12u + 12) of the row's block v / 16
+      const int b = v >> 4, bit = 12 * (v & 15), wi = bit >> 5, sh = bit & 31;
+      const uint16_t* ss = reinterpret_cast<const uint16_t*>(slot + L.scales_off);
+#pragma unroll
+      for (int j = 0; j < NP; ++j) {
+        float f[4] = {0.f, 0.f, 0.f, 0.f};
+        sc[j] = 0.f;
+        if (kExactN || j < p.N) {
+          const uint32_t* cw = reinterpret_cast<const uint32_t*>(slot + (size_t)(j * NB + b) * 24);
+          const uint32_t x = __funnelshift_r(cw[wi], wi < 5 ? cw[wi + 1] : 0u, sh) & 0xfffu;
+          nf3_levels4(x, f);
+          sc[j] = held(__half2float(__ushort_as_half(ss[j * NB + b])));
+        }
+        xf[j][0] = make_float2(held(f[0]), held(f[1]));
+        xf[j][1] = make_float2(held(f[2]), held(f[3]));
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < NP; ++j) {
+        uint2 rw = make_uint2(0u, 0u);
+        if (kExactN || j < p.N) rw = *reinterpret_cast<const uint2*>(slot + ((size_t)j * p.D + 4 * v) * 2);
+        if (kPacked) {
+          xp[kPacked ? j : 0] = rw;
+        } else {
+          xf[kPacked ? 0 : j][0] = make_float2(bf16_lo_held(rw.x), bf16_hi_held(rw.x));
+          xf[kPacked ? 0 : j][1] = make_float2(bf16_lo_held(rw.y), bf16_hi_held(rw.y));
+        }
+      }
+    }
+    int i = grp;
+    if constexpr (!kPacked) {
+      // four tokens at a time (16 independent FMA chains)
+      for (; i + 3 * Gt < n; i += 4 * Gt) {
+        float2 o[4][2];
+        if constexpr (kNf3)
+          combine_quad_nf3<NP, kExactN>(xf, sc, gs + i * NP, Gt * NP, p.N, o);
+        else
+          combine_quad<NP, kExactN>(xf, gs + i * NP, Gt * NP, p.N, o);
+#pragma unroll
+        for (int k2 = 0; k2 < 4; ++k2)
+          __stcs(reinterpret_cast<float4*>(p.out + (int64_t)tok[i + k2 * Gt] * p.D + 4 * v),
+                 make_float4(o[k2][0].x, o[k2][0].y, o[k2][1].x, o[k2][1].y));
+      }
+    }
+    for (; i < n; i += Gt) {
+      float4 o0;
+      if constexpr (kNf3)
+        o0 = combine_unit_nf3<NP, kExactN>(xf, sc, gs + i * NP, p.N);
+      else
+        o0 = combine_unit<NP, kExactN, kPacked>(xf, xp, gs + i * NP, p.N);
+      __stcs(reinterpret_cast<float4*>(p.out + (int64_t)tok[i] * p.D + 4 * v), o0);
+    }
+  }
+}
+
 template <int NT, bool kExactN, bool kNf3>
 __device__ void ring_consumers(const GArgs& p, const GroupLayout& L, const Ring& r, int my_n,
                                const float* gl = nullptr, const int* loff = nullptr) {
   constexpr int NP = 8 * NT;
   constexpr int C = kItemTokens;
-  constexpr bool kPacked = !kNf3 && NP > 16;  // 32 experts: keep rows as bf16 pairs, convert per token
-  static_assert(!kNf3 || NP <= 16, "the NF3 consumer holds 16 rows");
   const int lane = threadIdx.x & 31;
   volatile int* abort = r.abort;
-  const int NB = p.D >> 6;
-  const int lt = threadIdx.x;
-  const int units = p.D >> 2;
-  constexpr int kCT = kGroupCons * 32;
-  const int Gt = units >= kCT ? 1 : kCT / units;
-  const int grp = units >= kCT ? 0 : lt / units;
-  const int v0 = units >= kCT ? lt : lt - grp * units;
-  const int vstep = units >= kCT ? kCT : units;
-  const bool active = grp < Gt;
+  const UnitSplit us(p.D);
   for (int k = 0; k < my_n; ++k) {
     const uint32_t q = ring_slot(r, L, k);
     if (!warp_wait(&r.full[q], ring_parity(L, k), abort, p.err)) break;
     if (*abort) break;  // a phase completed without its item (the producer gave up)
-    if (active) {
-      const int n = r.slot_n[q];
+    if (us.active) {
       const uint8_t* slot = r.slots + (size_t)q * L.slot_bytes;
       const float* gs = gl != nullptr ? gl + loff[k] * NP : reinterpret_cast<const float*>(slot + L.gates_off);
-      for (int v = v0; v < units; v += vstep) {
-        float2 xf[kPacked ? 1 : NP][2];
-        uint2 xp[kPacked ? NP : 1];
-        float sc[NP];
-        if constexpr (kNf3) {
-          // 4 codes at bits [12u, 12u + 12) of the row's block v / 16
-          const int b = v >> 4, bit = 12 * (v & 15), wi = bit >> 5, sh = bit & 31;
-          const uint16_t* ss = reinterpret_cast<const uint16_t*>(slot + L.scales_off);
-#pragma unroll
-          for (int j = 0; j < NP; ++j) {
-            float f[4] = {0.f, 0.f, 0.f, 0.f};
-            sc[j] = 0.f;
-            if (kExactN || j < p.N) {
-              const uint32_t* cw = reinterpret_cast<const uint32_t*>(slot + (size_t)(j * NB + b) * 24);
-              const uint32_t x = __funnelshift_r(cw[wi], wi < 5 ? cw[wi + 1] : 0u, sh) & 0xfffu;
-              nf3_levels4(x, f);
-              sc[j] = held(__half2float(__ushort_as_half(ss[j * NB + b])));
-            }
-            xf[j][0] = make_float2(held(f[0]), held(f[1]));
-            xf[j][1] = make_float2(held(f[2]), held(f[3]));
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < NP; ++j) {
-            uint2 rw = make_uint2(0u, 0u);
-            if (kExactN || j < p.N) rw = *reinterpret_cast<const uint2*>(slot + ((size_t)j * p.D + 4 * v) * 2);
-            if (kPacked) {
-              xp[kPacked ? j : 0] = rw;
-            } else {
-              xf[kPacked ? 0 : j][0] = make_float2(bf16_lo_held(rw.x), bf16_hi_held(rw.x));
-              xf[kPacked ? 0 : j][1] = make_float2(bf16_lo_held(rw.y), bf16_hi_held(rw.y));
-            }
-          }
-        }
-        int i = grp;
-        if constexpr (!kPacked) {
-          // four tokens at a time (16 independent FMA chains)
-          for (; i + 3 * Gt < n; i += 4 * Gt) {
-            float2 o[4][2];
-            if constexpr (kNf3)
-              combine_quad_nf3<NP, kExactN>(xf, sc, gs + i * NP, Gt * NP, p.N, o);
-            else
-              combine_quad<NP, kExactN>(xf, gs + i * NP, Gt * NP, p.N, o);
-#pragma unroll
-            for (int k2 = 0; k2 < 4; ++k2)
-              __stcs(reinterpret_cast<float4*>(p.out + (int64_t)r.slot_tok[q * C + i + k2 * Gt] * p.D + 4 * v),
-                     make_float4(o[k2][0].x, o[k2][0].y, o[k2][1].x, o[k2][1].y));
-          }
-        }
-        for (; i < n; i += Gt) {
-          float4 o0;
-          if constexpr (kNf3)
-            o0 = combine_unit_nf3<NP, kExactN>(xf, sc, gs + i * NP, p.N);
-          else
-            o0 = combine_unit<NP, kExactN, kPacked>(xf, xp, gs + i * NP, p.N);
-          __stcs(reinterpret_cast<float4*>(p.out + (int64_t)r.slot_tok[q * C + i] * p.D + 4 * v), o0);
-        }
-      }
+      combine_item<NT, kExactN, kNf3>(p, L, us, slot, gs, r.slot_tok + q * C, r.slot_n[q]);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&r.empty[q]);
@@ -1230,6 +1256,254 @@ __global__ void __launch_bounds__(kGroupThreads, 1) grouped_local_kernel(const G
   __syncthreads();
 }
 
+// ---- Interleaved layer kernel: router tiles and work items in one ring ----
+//
+// One CTA per SM on the grouping's shares, like the CTA-local kernel, but its
+// ring carries two kinds of entries in one order: a router tile (the h rows
+// of 16 consecutive tokens of the share, one bulk copy per row, pitch bytes
+// apart) and a work item (the id's row block).  A tile goes in just before
+// the first item with a token in it, so h and the row blocks stream from
+// memory together and an item's gates are computed right before it is
+// combined, instead of in a router pass over the whole share first.  Wr
+// arrives once, in the ring's last slot, and stays in registers as each
+// consumer warp's B fragments; the slot then joins the ring.  The gates
+// (same mma.sync k-step split, k-slot order, partial-sum order and softmax as
+// the router kernels) go to a gate array in shared memory; the combine is
+// that of grouped_gather_kernel.
+
+struct StreamSync {
+  uint64_t* wr_full;  // Wr's copies landed
+  uint64_t* wr_free;  // every consumer warp holds its B fragments
+  const int4* recs;   // the CTA's item records (global memory), processing order
+  const int* loff;    // [my_n + 1] token offset of each item in the share (shared memory)
+  const int* tok;     // [n_tok] the share's tokens (shared memory)
+  int my_n, n_tok, n_tiles, pitch, wr_slot;
+};
+
+// Whether the next ring entry, with t tiles and k items before it, is tile
+// t: while a tile holds a token of item k (or of an earlier one).  Once all
+// items are placed, all tiles are (the last item ends at n_tok).
+__device__ __forceinline__ bool stream_tile_next(const StreamSync& ss, int t, int k) {
+  return t < ss.n_tiles && t * kTileMax < ss.loff[k + 1];
+}
+
+// Producer warp of the interleaved kernel: entry e into slot e mod n_slots
+// once its previous entry is consumed (in the first lap at once, Wr's slot
+// once the B fragments are in registers); a tile's rows by its lanes, an
+// item's row block by lane 0.  Item records are read 32 at a time.
+template <int NP>
+__device__ void stream_producer(const GArgs& p, const GroupWs& w, const GroupLayout& L, const Ring& r,
+                                const StreamSync& ss) {
+  const int lane = threadIdx.x & 31;
+  volatile int* abort = r.abort;
+  const uint32_t row_bytes = (uint32_t)p.N * (uint32_t)p.D * 2u, h_row = (uint32_t)p.D * 2u;
+  const int n_entries = ss.n_tiles + ss.my_n;
+  const int4 none = make_int4(0, 0, 0, 0);
+  int t = 0, k = 0, k0 = 0, issued = 0;
+  int4 rec = lane < ss.my_n ? ss.recs[lane] : none;
+  for (int e = 0; e < n_entries; ++e) {
+    const uint32_t q = ring_slot(r, L, e);
+    bool ok = true;
+    if (e >= L.n_slots)
+      ok = warp_wait(&r.empty[q], ring_parity(L, e) ^ 1u, abort, p.err);
+    else if ((int)q == ss.wr_slot)
+      ok = warp_wait(ss.wr_free, 0u, abort, p.err);
+    if (!ok) break;
+    uint8_t* slot = r.slots + (size_t)q * L.slot_bytes;
+    if (stream_tile_next(ss, t, k)) {
+      const int rows = ss.n_tok - t * kTileMax < kTileMax ? ss.n_tok - t * kTileMax : kTileMax;
+      if (lane == 0) mbar_expect_tx(&r.full[q], (uint32_t)rows * h_row);
+      __syncwarp();
+      if (lane < rows)
+        bulk_g2s(slot + (size_t)lane * ss.pitch, p.h + (int64_t)ss.tok[t * kTileMax + lane] * p.D, h_row, &r.full[q]);
+      ++t;
+    } else {
+      if (k - k0 == 32) {
+        k0 = k;
+        rec = k0 + lane < ss.my_n ? ss.recs[k0 + lane] : none;
+      }
+      const int row = __shfl_sync(0xffffffffu, p.by_uid ? rec.w : rec.x, k - k0);
+      if (p.by_uid && (int64_t)row >= p.rows) {  // staging buffer smaller than the batch's distinct ids
+        if (lane == 0) atomicOr(p.err, kErrIndex);
+        *abort = 1;
+        break;
+      }
+      if (lane == 0) {
+        mbar_expect_tx(&r.full[q], row_bytes);
+        bulk_g2s(slot, p.table + (int64_t)row * p.N * p.D, row_bytes, &r.full[q]);
+      }
+      ++k;
+    }
+    issued = e + 1;
+  }
+  // tokens with a bad id are in no work item: NaN output rows for those of
+  // this CTA's slice of the batch
+  const int64_t t0 = (int64_t)blockIdx.x * p.T / gridDim.x, t1 = ((int64_t)blockIdx.x + 1) * p.T / gridDim.x;
+  for (int64_t tt = t0 + lane; tt < t1; tt += 32) {
+    if (__ldg(w.tok_pos + tt) >= 0) continue;
+    atomicOr(p.err, kErrIndex);
+    float* o = p.out + tt * p.D;
+    for (int d = 0; d < p.D; d += 4) __stcs(reinterpret_cast<float4*>(o + d), make_float4(NAN, NAN, NAN, NAN));
+  }
+  if (lane == 0) {  // the last copies must have landed before the CTA exits
+    mbar_drain(ss.wr_full, 0u);
+    for (int e = issued - 1; e >= 0 && e >= issued - L.n_slots; --e)
+      mbar_drain(&r.full[ring_slot(r, L, e)], ring_parity(L, e));
+  }
+  __syncwarp();
+}
+
+// Consumer warps of the interleaved kernel.  A tile: A fragments from the
+// slot (then the slot is released), MMAs against the held B fragments,
+// partial sums exchanged, softmax into the gate array -- every consumer
+// warp takes part, so tile waits give one verdict for all.  An item: the
+// combine of ring_consumers with the gates from the gate array.  A warp whose
+// item wait failed skips the remaining items but still meets the other warps
+// at the next tile, where all of them stop.
+template <int NT, bool kExactN>
+__device__ void stream_consumers(const GArgs& p, const GroupLayout& L, const Ring& r, const StreamSync& ss,
+                                 const PairScratch& ps, float* gl, const uint16_t* wr_s, volatile int* fail) {
+  constexpr int KB = kFusedKB;
+  constexpr int NP = 8 * NT;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ksteps = p.D >> 4;
+  volatile int* abort = r.abort;
+  const bool ok = consumers_wait(ss.wr_full, 0u, abort, p.err, fail);
+  // B fragments of k-steps warp + 8i, in the router kernels' k-slot order
+  uint2 bw[KB][NT];
+#pragma unroll
+  for (int i = 0; i < KB; ++i) {
+    const int ks = warp + i * kWarps;
+    if (ok && ks < ksteps) {
+      if (kExactN && p.N == NP)
+        wr_fragments<NT>(bw[i], wr_s, ks);
+      else
+        wr_fragments_any<NT>(bw[i], wr_s, ks, p.N);
+    } else {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) bw[i][nt] = make_uint2(0u, 0u);
+    }
+  }
+  ConsumerSync{}();
+  if (ok && threadIdx.x == 0) mbar_arrive(ss.wr_free);  // Wr's slot goes back to the ring
+  if (!ok) return;
+  const UnitSplit us(p.D);
+  const int n_entries = ss.n_tiles + ss.my_n;
+  int t = 0, k = 0;
+  bool dead = false;
+  for (int e = 0; e < n_entries; ++e) {
+    const uint32_t q = ring_slot(r, L, e), par = ring_parity(L, e);
+    const uint8_t* slot = r.slots + (size_t)q * L.slot_bytes;
+    if (stream_tile_next(ss, t, k)) {
+      if (!consumers_wait(&r.full[q], par, abort, p.err, fail)) return;
+      const int rows = ss.n_tok - t * kTileMax < kTileMax ? ss.n_tok - t * kTileMax : kTileMax;
+      RouterA<KB> A;
+      router_load_a_smem<KB>(A, slot, ss.pitch, rows, p.D, warp);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&r.empty[q]);
+      float acc[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll
+      for (int i = 0; i < KB; ++i) {
+        if (warp + i * kWarps < ksteps) {
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+            mma_16816(acc[nt], A.a0[i].x, A.a1[i].x, A.a0[i].y, A.a1[i].y, bw[i][nt].x, bw[i][nt].y);
+        }
+      }
+      pair_store_partials<NT>(ps, acc, 0);
+      ConsumerSync{}();
+      PairScratch pg = ps;
+      pg.gates = gl + (size_t)t * kTileMax * NP;
+      pair_softmax<NT>(pg, rows, p.N);
+      ConsumerSync{}();
+      ++t;
+    } else {
+      if (!dead) {
+        dead = !warp_wait(&r.full[q], par, abort, p.err);
+        if (!dead && us.active) {
+          const int o = ss.loff[k];
+          combine_item<NT, kExactN, false>(p, L, us, slot, gl + (size_t)o * NP, ss.tok + o, ss.loff[k + 1] - o);
+        }
+        __syncwarp();
+        if (lane == 0) {
+          if (dead)
+            *fail = 1;
+          else
+            mbar_arrive(&r.empty[q]);
+        }
+      }
+      ++k;
+    }
+  }
+}
+
+template <int NT, bool kExactN>
+__global__ void __launch_bounds__(kGroupThreads, 1) grouped_stream_kernel(const GArgs p, const GroupWs w,
+                                                                          const GroupLayout L, int scap, int pitch) {
+  constexpr int NP = 8 * NT;
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  const Ring r = carve_ring(smem_raw, L);
+  uint8_t* scratch = smem_raw + (ring_bytes(L.n_slots, L.slot_bytes) + 127) / 128 * 128;
+  const PairScratch ps{reinterpret_cast<float*>(scratch), nullptr, nullptr};  // partial sums
+  float* gl = reinterpret_cast<float*>(scratch + pair_scratch_bytes<NP>());    // [scap][NP] gates
+  int* loff = reinterpret_cast<int*>(gl + (size_t)scap * NP);                   // [scap + 1]
+  int* tok_s = loff + scap + 1;                                                 // [scap]
+  __shared__ int skip_s, fail_s;
+  __shared__ __align__(8) uint64_t bars[2];
+  const int b = blockIdx.x, lane = threadIdx.x & 31;
+  const bool producer = (threadIdx.x >> 5) == kGroupProducer;
+  const int wr_slot = L.n_slots - 1;
+  uint8_t* wr_p = r.slots + (size_t)wr_slot * L.slot_bytes;
+  if (threadIdx.x == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    ring_init(r, L, 1);  // full: one arrival, with the entry's copy bytes
+  }
+  __syncthreads();
+  pdl_trigger();
+  pdl_wait();  // the grouping and every earlier kernel are complete
+  if (producer) {
+    // Wr (one slot), in chunks taken in a CTA-dependent order so that the
+    // CTAs' requests spread over L2
+    const uint32_t wr_bytes = (uint32_t)p.N * (uint32_t)p.D * 2u;
+    const uint32_t n_ch = (wr_bytes + kWrChunk - 1) / kWrChunk;  // <= 16 (N <= 16, D <= 2048)
+    if (lane == 0) mbar_expect_tx(&bars[0], wr_bytes);
+    __syncwarp();
+    if ((uint32_t)lane < n_ch) {
+      const uint32_t off = ((lane + (uint32_t)b) % n_ch) * kWrChunk;
+      bulk_g2s(wr_p + off, reinterpret_cast<const uint8_t*>(p.Wr) + off,
+               wr_bytes - off < kWrChunk ? wr_bytes - off : kWrChunk, &bars[0]);
+    }
+  }
+  const int2 sn = reinterpret_cast<const int2*>(w.share_n)[b];
+  if (threadIdx.x == 0) {
+    const unsigned ab = ld_relaxed_u32(&w.ctl[kCtlAbort]), grid = ld_relaxed_u32(&w.ctl[kCtlShareGrid]);
+    // plan abandoned (error word set): skip; shares for another CTA count: error
+    skip_s = ab != 0xFFFFFFFFu ? 1 : (grid != gridDim.x || sn.x < 0 || sn.y < 0 || sn.x > scap || sn.y > scap) ? 2 : 0;
+    if (skip_s == 2) atomicOr(p.err, kErrGrouping);
+    fail_s = 0;
+  }
+  __syncthreads();
+  if (skip_s) {
+    if (producer && lane == 0) mbar_drain(&bars[0], 0u);
+    return;
+  }
+  const int my_n = sn.x, n_tok = sn.y;
+  // the share's item offsets and tokens into shared memory
+  for (int i = threadIdx.x; i <= my_n; i += kGroupThreads) loff[i] = __ldg(w.share_off + (size_t)b * (scap + 1) + i);
+  for (int i = threadIdx.x; i < n_tok; i += kGroupThreads) tok_s[i] = __ldg(w.share_tok + (size_t)b * scap + i);
+  __syncthreads();
+  const StreamSync ss{&bars[0], &bars[1], w.share_rec + (size_t)b * scap, loff, tok_s, my_n, n_tok,
+                      (n_tok + kTileMax - 1) / kTileMax, pitch, wr_slot};
+  if (producer)
+    stream_producer<NP>(p, w, L, r, ss);
+  else
+    stream_consumers<NT, kExactN>(p, L, r, ss, ps, gl, reinterpret_cast<const uint16_t*>(wr_p), &fail_s);
+  __syncthreads();
+}
+
 // Ring slot of a work item: the id's row block (bf16 table: N rows of D;
 // NF3 table: N x D/64 24-byte code blocks, then the fp16 scales at
 // scales_off), then the gates of up to kItemTokens tokens at gates_off.
@@ -1281,11 +1555,63 @@ mole_status launch_local(const GArgs& p, const GroupWs& w, cudaStream_t stream) 
   return cuda_status(launch_pdl(kern, (unsigned)n_sm, kGroupThreads, smem, stream, p, w, L, (int)scap));
 }
 
+// The interleaved layer kernel (bf16 table, N <= 16, D <= 2048), one CTA
+// per SM, on the grouping's shares.  Slots hold a row block or a 16-row
+// router tile, whichever is larger; at least three of them.
+template <int NT, bool kExactN>
+mole_status launch_stream(const GArgs& p, const GroupWs& w, cudaStream_t stream) {
+  constexpr int NP = 8 * NT;
+  if (p.D > 16 * kWarps * kFusedKB || !aligned16(p.Wr) || !aligned16(p.h) || p.D % 8 != 0)
+    return MOLE_ERR_UNSUPPORTED;
+  const int n_sm = num_sms();
+  if (n_sm <= 0) return MOLE_ERR_NO_DEVICE;
+  if (!shares_apply(p.T, n_sm)) return MOLE_ERR_UNSUPPORTED;
+  const int64_t scap = share_cap(p.T, n_sm);
+  const int pitch = 2 * p.D + 32;
+  GroupLayout L{};
+  const int64_t need = std::max<int64_t>((int64_t)p.N * p.D * 2, (int64_t)kTileMax * pitch);
+  L.slot_bytes = (int)((need + 127) / 128 * 128);
+  L.gates_off = L.slot_bytes;
+  const size_t fixed = pair_scratch_bytes<NP>() + (size_t)scap * NP * 4 + (size_t)(2 * scap + 1) * 4;
+  constexpr size_t kMax = 227 * 1024 - 256;  // (the static barriers and flags)
+  int n = 16;
+  while (n >= 3 && (ring_bytes(n, L.slot_bytes) + 127) / 128 * 128 + fixed > kMax) --n;
+  if (n < 3) return MOLE_ERR_UNSUPPORTED;
+  L.n_slots = n;
+  const size_t smem = (ring_bytes(n, L.slot_bytes) + 127) / 128 * 128 + fixed;
+  auto kern = grouped_stream_kernel<NT, kExactN>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return MOLE_ERR_CUDA;
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kGroupThreads, smem) != cudaSuccess || occ < 1)
+    return MOLE_ERR_UNSUPPORTED;
+  return cuda_status(launch_pdl(kern, (unsigned)n_sm, kGroupThreads, smem, stream, p, w, L, (int)scap, pitch));
+}
+
+// Batches from about 3/4 of a 128-token tile per SM up take the interleaved
+// kernel; below that the CTA-local kernel's router pass over its share is
+// short (at 4096 tokens on 148 SMs, two tiles) and it is as fast.
+bool stream_preferred(int64_t T) {
+  const int n_sm = num_sms();
+  return n_sm > 0 && (T + 127) / 128 >= (int64_t)n_sm * 3 / 4;
+}
+
+// Kernel choice per layer call.  bf16 table: the interleaved kernel (large
+// batches) or the CTA-local kernel, else the mma.sync router kernel + gather
+// -- every bf16 path computes its gates with the mma.sync router arithmetic,
+// so grouped and ungrouped calls agree bit for bit.  NF3 table: the
+// CTA-local kernel below the tensor-core router's size, else that router
+// (as the ungrouped NF3 call) + gather.
 template <int NT, bool kExactN, bool kNf3>
 mole_status launch_layer(const GArgs& p, const GroupWs& w, cudaStream_t stream) {
   constexpr int NP = 8 * NT;
+  const bool tc_router = kNf3 && router_tc_supported(p.T, p.N, p.D, p.h, p.Wr);
   if constexpr (NT <= 2) {
-    if (!router_tc_supported(p.T, p.N, p.D, p.h, p.Wr)) {
+    if (!kNf3 && stream_preferred(p.T)) {
+      const mole_status st = launch_stream<NT, kExactN>(p, w, stream);
+      if (st != MOLE_ERR_UNSUPPORTED) return st;
+    }
+    if (!tc_router) {
       const mole_status st = launch_local<NT, kExactN, kNf3>(p, w, stream);
       if (st != MOLE_ERR_UNSUPPORTED) return st;
     }
@@ -1306,7 +1632,7 @@ mole_status launch_layer(const GArgs& p, const GroupWs& w, cudaStream_t stream) 
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, rkern, kThreads, rsmem) != cudaSuccess || occ < 1)
     return MOLE_ERR_UNSUPPORTED;
   const int64_t n_tiles = (p.T + kTileMax - 1) / kTileMax;
-  if (router_tc_supported(p.T, p.N, p.D, p.h, p.Wr)) {
+  if (tc_router) {
     const mole_status st = router_tc_launch(p.h, p.Wr, p.T, p.D, true, p.out, w.tok_pos, w.gates, stream);
     if (st != MOLE_OK) return st;
   } else if (launch_pdl(rkern, (unsigned)std::min<int64_t>(n_tiles, (int64_t)occ * n_sm), kThreads, rsmem, stream,

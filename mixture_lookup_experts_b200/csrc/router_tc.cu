@@ -1,10 +1,11 @@
 // router_tc.cu -- the router of a prefill batch on the tcgen05 tensor cores
 // (MoLE page, 训练阶段: the gates are a softmax over all routed experts of the
-// hidden state times the router weight).
+// hidden state times the router weight), taken by the NF3-table calls; the
+// bf16-table calls route with the mma.sync router arithmetic throughout.
 //
 // z[T, 16] = h[T, D] . Wr[D, 16] is a skinny GEMM bound by reading h (2D bytes
 // per token).  One CTA per SM, persistent over 128-token tiles:
-//   warp 0     TMA producer (one lane): the h box 64(d) x 128(tokens) with
+//   warp 0     TMA producer (one lane): the h box 64(d) x rows(tokens) with
 //              128-byte swizzle and the Wr box 16(j) x 64(d) with 32-byte
 //              swizzle -- Wr is read in its own [D, N] layout as the N-major
 //              B operand -- into an 8-stage ring of 18 KB;
@@ -30,13 +31,16 @@
 namespace mole {
 namespace {
 
-constexpr int RM = 128, RK = 64, RN = 16, RSTAGES = 8;
-constexpr int RA_STAGE = RM * RK * 2;  // 16 KB of h
-constexpr int RB_STAGE = RK * RN * 2;  // 2 KB of Wr
+constexpr int RM = 128, RK = 64, RN = 16, RSTAGES = 8, RBOX = 1;
+constexpr int RKS = RK * RBOX;              // hidden dims per stage
+constexpr int RA_BOX = RM * RK * 2;          // one 16 KB h box (64 dims x 128 tokens)
+constexpr int RA_STAGE = RA_BOX * RBOX;
+constexpr int RB_STAGE = RKS * RN * 2;       // Wr rows of the stage
 constexpr int kRThreads = 6 * 32;
 constexpr int kREpiWarps = 4;
 constexpr int kRSmem = 1024 /*alignment slack*/ + RSTAGES * (RA_STAGE + RB_STAGE) + 256 /*barriers*/;
 constexpr uint32_t kRTmemCols = 32;  // two 16-column accumulators
+constexpr bool kRotateK = true;
 
 // Instruction descriptor, kind::f16: D fp32 (bit 4), A bf16 (bits 7-9) K-major,
 // B bf16 (bits 10-12) N-major (bit 16), N/8 at bits 17-22, M/16 at bits 24-28.
@@ -48,6 +52,7 @@ enum RouterSink { kSinkOutRows = 0, kSinkGrouped = 1 };
 struct RtArgs {
   int64_t T;
   int D;
+  int rows;  // tokens per tile (<= RM; the MMA still runs M = RM, extra lanes are dropped)
   int64_t tiles;
   float* out;           // [T, D]
   const int* tok_pos;   // grouped: list position of each token (-1: bad id)
@@ -150,23 +155,29 @@ __global__ void __launch_bounds__(kRThreads, 1)
   pdl_trigger();
   pdl_wait();
   const uint32_t tmem_base = *tmem_slot;
-  const int kblocks = (p.D + RK - 1) / RK;
+  const int kblocks = (p.D + RKS - 1) / RKS;
 
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer ----------------
       uint32_t it = 0;
       bool ok = true;
+      const uint32_t box_bytes = (uint32_t)p.rows * RK * 2;
       for (int64_t tile = blockIdx.x; ok && tile < p.tiles; tile += gridDim.x) {
-        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+        const int k0 = kRotateK ? (int)(tile % kblocks) : 0;
+        for (int i = 0; i < kblocks; ++i, ++it) {
+          const int kb = k0 + i < kblocks ? k0 + i : k0 + i - kblocks;
           const uint32_t s = it % RSTAGES, ph = (it / RSTAGES) & 1u;
           if (!mbar_wait(&empty[s], ph ^ 1u, abort, p.err)) {
             ok = false;
             break;
           }
-          mbar_expect_tx(&full[s], RA_STAGE + RB_STAGE);
-          rt_tma_load_3d(sA + s * RA_STAGE, &map_h, &full[s], kb * RK, (int)(tile * RM), 0);
-          rt_tma_load_3d(sB + s * RB_STAGE, &map_w, &full[s], 0, kb * RK, 0);
+          const int nbox = min(RBOX, (p.D - kb * RKS + RK - 1) / RK);
+          mbar_expect_tx(&full[s], (uint32_t)nbox * box_bytes + RB_STAGE);
+          for (int b = 0; b < nbox; ++b)
+            rt_tma_load_3d(sA + s * RA_STAGE + b * RA_BOX, &map_h, &full[s], kb * RKS + b * RK, (int)(tile * p.rows),
+                           0);
+          rt_tma_load_3d(sB + s * RB_STAGE, &map_w, &full[s], 0, kb * RKS, 0);
         }
       }
       const uint32_t first = it > (uint32_t)RSTAGES ? it - RSTAGES : 0u;
@@ -183,7 +194,9 @@ __global__ void __launch_bounds__(kRThreads, 1)
         if (!mbar_wait(&tempty[acc], aph ^ 1u, abort, p.err)) break;
         rt_fence_after();
         const uint32_t d_tmem = tmem_base + acc * RN;
-        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+        const int k0 = kRotateK ? (int)(tile % kblocks) : 0;
+        for (int i = 0; i < kblocks; ++i, ++it) {
+          const int kb = k0 + i < kblocks ? k0 + i : k0 + i - kblocks;
           const uint32_t s = it % RSTAGES, ph = (it / RSTAGES) & 1u;
           if (!mbar_wait(&full[s], ph, abort, p.err)) {
             ok = false;
@@ -191,11 +204,15 @@ __global__ void __launch_bounds__(kRThreads, 1)
           }
           rt_fence_after();
           const uint32_t a0 = smem_u32(sA + s * RA_STAGE), b0 = smem_u32(sB + s * RB_STAGE);
+          const int nk = min(RKS, p.D - kb * RKS) / 16;
 #pragma unroll
-          for (int k = 0; k < RK / 16; ++k) {
-            // A (h): K-major, 128-byte rows; advance 16 elements (32 B) inside the swizzle atom.
+          for (int k = 0; k < RKS / 16; ++k) {
+            if (k >= nk) break;
+            // A (h): K-major, 128-byte rows; advance 16 elements (32 B) inside the swizzle atom,
+            // and a whole 16 KB box every 64 elements.
             // B (Wr): N-major, 32-byte rows of 16 experts; 8-row atoms of 256 B; advance 16 rows (512 B).
-            rt_umma(d_tmem, rt_desc(a0 + 32 * k, 16, 1024, 2), rt_desc(b0 + 512 * k, 0, 256, 6), (kb | k) != 0);
+            rt_umma(d_tmem, rt_desc(a0 + (k >> 2) * RA_BOX + 32 * (k & 3), 16, 1024, 2),
+                    rt_desc(b0 + 512 * k, 0, 256, 6), (i | k) != 0);
           }
           issued = true;
           rt_commit(&empty[s]);
@@ -224,8 +241,9 @@ __global__ void __launch_bounds__(kRThreads, 1)
       rt_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty[acc]);
-      const int64_t t = tile * RM + quad * 32 + lane;
-      if (t >= p.T) continue;
+      const int r = quad * 32 + lane;
+      const int64_t t = tile * p.rows + r;
+      if (r >= p.rows || t >= p.T) continue;
       float m = z[0];
 #pragma unroll
       for (int j = 1; j < 16; ++j) m = fmaxf(m, z[j]);
@@ -289,6 +307,16 @@ bool rt_map(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Tokens per tile: as many rounds of RM-token tiles as the batch needs over
+// the SMs, then the rows evened out over them (a multiple of 16), so that the
+// last round does not leave SMs idle -- 16384 tokens on 148 SMs take 147
+// tiles of 112 rows rather than 128 tiles of 128.
+int router_tile_rows(int64_t T, int n_sm) {
+  const int64_t rounds = (T + (int64_t)n_sm * RM - 1) / ((int64_t)n_sm * RM);
+  const int64_t per = (T + (int64_t)n_sm * rounds - 1) / ((int64_t)n_sm * rounds);
+  return (int)std::min<int64_t>(RM, (per + 15) / 16 * 16);
+}
+
 }  // namespace
 
 bool router_tc_supported(int64_t T, int N, int64_t D, const void* h, const void* Wr) {
@@ -308,8 +336,11 @@ bool router_tc_supported(int64_t T, int N, int64_t D, const void* h, const void*
 mole_status router_tc_launch(const void* h, const void* Wr, int64_t T, int64_t D, bool grouped, float* out,
                              const int* tok_pos, float* gates, cudaStream_t stream) {
   CUtensorMap mh, mw;
-  if (!rt_map(&mh, h, (uint64_t)D, (uint64_t)T, (uint64_t)D * 2, RK, RM, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !rt_map(&mw, Wr, RN, (uint64_t)D, RN * 2, RN, RK, CU_TENSOR_MAP_SWIZZLE_32B))
+  const int n_sm = num_sms();
+  if (n_sm <= 0) return MOLE_ERR_NO_DEVICE;
+  const int rows = router_tile_rows(T, n_sm);
+  if (!rt_map(&mh, h, (uint64_t)D, (uint64_t)T, (uint64_t)D * 2, RK, (uint32_t)rows, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !rt_map(&mw, Wr, RN, (uint64_t)D, RN * 2, RN, RKS, CU_TENSOR_MAP_SWIZZLE_32B))
     return MOLE_ERR_CUDA;
   static bool attr_set[64][2] = {};
   int dev = 0;
@@ -320,12 +351,11 @@ mole_status router_tc_launch(const void* h, const void* Wr, int64_t T, int64_t D
       return MOLE_ERR_CUDA;
     attr_set[dev][grouped] = true;
   }
-  const int n_sm = num_sms();
-  if (n_sm <= 0) return MOLE_ERR_NO_DEVICE;
   RtArgs p{};
   p.T = T;
   p.D = (int)D;
-  p.tiles = (T + RM - 1) / RM;
+  p.rows = rows;
+  p.tiles = (T + rows - 1) / rows;
   p.out = out;
   p.tok_pos = tok_pos;
   p.gates = gates;

@@ -44,6 +44,11 @@ def _both(mole, ids, h, Wr, lut):
     (64, 2048, 32, 1030, "uniform"),   # 128 KB row blocks: no ring fits, ungrouped kernels
     (777, 256, 16, 333, "zipf"),       # below the grouping threshold: ungrouped kernels
     (20000, 128, 16, 14080, "zipf"),   # largest batch of the CTA-local kernel (16 experts)
+    (20000, 128, 16, 14208, "zipf"),   # smallest batch of the interleaved kernel (148 SMs)
+    (60000, 128, 16, 15000, "uniform"),  # interleaved: ~100 single-token items per CTA
+    (700, 256, 12, 16000, "zipf"),     # interleaved, padded expert count
+    (3000, 64, 8, 20011, "uniform"),   # interleaved, 8 experts, ragged last tile
+    (400, 64, 32, 15000, "zipf"),      # 32 experts at a prefill size: router + gather kernels
     (5000, 64, 8, 40000, "zipf"),      # too many tokens per SM for the CTA-local kernel
 ])
 def test_grouped_matches_oracle_and_ungrouped(mole, oracle_mod, V, D, N, T, kind):
@@ -56,9 +61,11 @@ def test_grouped_matches_oracle_and_ungrouped(mole, oracle_mod, V, D, N, T, kind
     np.testing.assert_array_equal(got, plain)
 
 
-def test_grouped_single_hot_id(mole, oracle_mod):
-    """All 5000 tokens share one id: 313 work items of that id."""
-    V, D, N, T = 100, 256, 16, 5000
+@pytest.mark.parametrize("T", [5000, 16000])
+def test_grouped_single_hot_id(mole, oracle_mod, T):
+    """All tokens share one id: 313 (1000) work items of that id; at 16000
+    tokens each item of the interleaved kernel has a router tile of its own."""
+    V, D, N = 100, 256, 16
     ids, h, Wr, lut = _layer(41, V, D, N, T)
     ids[:] = 7
     got, st, plain, _ = _both(mole, ids, h, Wr, lut)
@@ -174,7 +181,7 @@ def test_token_groups_serve_every_layer(mole, oracle_mod):
 
 def test_token_groups_bad_ids_and_small_batches(mole, oracle_mod):
     V, D, N = 300, 128, 16
-    for T in (1500, 200):  # grouped kernels; below their threshold the plain ones
+    for T in (1500, 200, 15000):  # grouped kernels (CTA-local, interleaved); below their threshold the plain ones
         ids, h, Wr, lut = _layer(62 + T, V, D, N, T, "zipf")
         ids[[1, T - 1]] = [V + 5, -2]
         groups = mole.mole_token_groups_build(dev(ids), V, N)
