@@ -152,6 +152,8 @@ def test_nf3_full_size_sampled(mole, oracle_mod, T, kind):
     (100, 13, 512, 1200, "zipf"),   # padded expert count (13 * 8 blocks = 104, a multiple of 8)
     (100, 5, 128, 1200, "zipf"),    # N * D/64 not a multiple of 8: ungrouped kernels
     (64, 16, 256, 300, "zipf"),     # below the grouping threshold: ungrouped kernels
+    (3000, 16, 128, 15000, "zipf"),  # a prefill size: tensor-core router + grouped gather
+    (2000, 8, 128, 40000, "zipf"),   # too many tokens per SM for the shares: mma.sync router + grouped gather
 ])
 def test_combine_nf3_groups_matches_oracle_and_ungrouped(mole, oracle_mod, V, N, D, T, kind):
     rng = np.random.default_rng(T + D + N)
