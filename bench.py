@@ -213,21 +213,23 @@ def kernel_source_hash() -> str:
     return h.hexdigest()
 
 
-def launches_per_step(T: int, N: int, layers: int, path: str) -> int:
+def launches_per_step(T: int, N: int, layers: int, path: str, n_sm: int | None = None) -> int:
     """This library's kernel launches in one timed step (bf16 table).  Grouped
     path: the grouping (plan kernel, plus the per-SM share kernel when a CTA's
     share fits, 16 + T/SMs < 256 tokens), then per layer one kernel (the
-    interleaved or the CTA-local kernel) where the shares exist, else router +
-    gather; plain path: router + gather per layer.  Below 1024 tokens one
-    combine kernel per layer."""
-    import torch
-    n_sm = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+    interleaved or the CTA-local kernel, N <= 16) where the shares exist, else
+    router + gather; plain path: router + gather per layer.  Below 1024 tokens
+    one combine kernel per layer.  n_sm: the device's SM count (queried when
+    not given)."""
+    if n_sm is None:
+        import torch
+        n_sm = torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
     if T < 1024:
         return layers
     if path != "grouped":
         return 2 * layers
     shares = (16 + -(-T // n_sm) + 15) // 16 * 16 < 256
-    per_layer = 1 if shares else 2
+    per_layer = 1 if (shares and N <= 16) else 2
     return (2 if shares else 1) + per_layer * layers
 
 

@@ -45,3 +45,15 @@ def test_compact_rounds_floats_only():
     assert bench.compact({"a": [1.23456789, 7], "b": "x", "c": None, "d": True}) == \
         {"a": [1.23457, 7], "b": "x", "c": None, "d": True}
     assert bench.compact(1234567890.5) == pytest.approx(1234570000.0)
+
+
+def test_launch_count_of_the_headline_step():
+    """The headline step on 148 SMs: the grouping (plan + shares) and one
+    interleaved-kernel launch per layer; past the shares' size, router +
+    gather per layer; the plain path two per layer; decode sizes one."""
+    assert bench.launches_per_step(16384, 16, 16, "grouped", n_sm=148) == 2 + 16
+    assert bench.launches_per_step(4096, 16, 16, "grouped", n_sm=148) == 2 + 16
+    assert bench.launches_per_step(40000, 16, 16, "grouped", n_sm=148) == 1 + 2 * 16
+    assert bench.launches_per_step(16384, 32, 16, "grouped", n_sm=148) == 2 + 2 * 16
+    assert bench.launches_per_step(16384, 16, 16, "plain", n_sm=148) == 32
+    assert bench.launches_per_step(64, 16, 12, "grouped", n_sm=148) == 12
